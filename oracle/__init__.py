@@ -1,0 +1,185 @@
+"""CPU oracle for MoE token dispatch and combine -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the C-ABI library in
+``combine_topk_ids_scan_b200``) never touches it, and the two share no code.
+
+The arithmetic lives in ``oracle.c`` (plain single-threaded C, built with gcc
+without fast-math or FP contraction).  This module only builds that file and
+marshals numpy arrays to it.  Page citations for every function are in
+``oracle.h`` / ``oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_HDR = os.path.join(_HERE, "oracle.h")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+STATUS_ID_RANGE = 1
+STATUS_DUP_ID = 2
+STATUS_CAPACITY = 4
+FLAG_CHECK_DUPLICATES = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, -O2, IEEE)."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
+    if not force and os.path.exists(_LIB_PATH) and os.path.getmtime(_LIB_PATH) >= newest:
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math",
+           "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        i32, i64, u32, f32, vp = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
+                                  ctypes.c_float, ctypes.c_void_p)
+        L.orc_layout.restype = u32
+        L.orc_layout.argtypes = [i32, i32, i32, i32, i64, i32, u32, i32,
+                                 vp, vp, vp, vp, vp, vp, vp]
+        L.orc_permute_bf16.argtypes = [i64, i32, vp, vp, vp]
+        L.orc_permute_fp8.argtypes = [i64, i32, vp, vp, vp, vp]
+        L.orc_permute_nvfp4.argtypes = [i64, i32, vp, vp, f32, vp, vp]
+        L.orc_combine.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp]
+        for n in ("orc_bf16_from_f32_n", "orc_e4m3_from_f32_n", "orc_e2m1_from_f32_n"):
+            getattr(L, n).argtypes = [vp, vp, i64]
+        L.orc_e4m3_to_f32.restype = f32
+        L.orc_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+        L.orc_e2m1_to_f32.restype = f32
+        L.orc_e2m1_to_f32.argtypes = [ctypes.c_uint8]
+        L.orc_bf16_to_f32.restype = f32
+        L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- formats
+def bf16_from_f32(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib().orc_bf16_from_f32_n(_p(x), _p(out), x.size)
+    return out
+
+
+def e4m3_from_f32(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    lib().orc_e4m3_from_f32_n(_p(x), _p(out), x.size)
+    return out
+
+
+def e2m1_from_f32(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    lib().orc_e2m1_from_f32_n(_p(x), _p(out), x.size)
+    return out
+
+
+def e4m3_to_f32(code: int) -> float:
+    return lib().orc_e4m3_to_f32(code)
+
+
+def e2m1_to_f32(code: int) -> float:
+    return lib().orc_e2m1_to_f32(code)
+
+
+# ---------------------------------------------------------------- layout
+class Layout:
+    """Outputs of the dispatch layout for one problem."""
+
+    def __init__(self, status, expert_counts, expert_offsets, meta, row_src,
+                 pair_slot, drop_mask):
+        self.status = status
+        self.expert_counts = expert_counts
+        self.expert_offsets = expert_offsets
+        self.meta = meta
+        self.row_src = row_src
+        self.pair_slot = pair_slot
+        self.drop_mask = drop_mask
+
+
+def layout(ids: np.ndarray, num_experts: int, num_segments: int, hidden: int,
+           recv_capacity: int = 0, expert_capacity: int = 0,
+           flags: int = 0) -> Layout:
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    N, k = ids.shape
+    E, S = num_experts, num_segments
+    rows = E * expert_capacity if expert_capacity > 0 else recv_capacity
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    meta = np.empty((4, S), np.uint32)
+    row_src = np.empty(rows, np.int32)
+    pair_slot = np.empty((N, k), np.int32)
+    drop = np.empty((N, k), np.uint8)
+    st = lib().orc_layout(N, k, E, S, recv_capacity, expert_capacity, flags, hidden,
+                          _p(ids), _p(counts), _p(offsets), _p(meta), _p(row_src),
+                          _p(pair_slot), _p(drop))
+    return Layout(int(st), counts, offsets, meta, row_src, pair_slot, drop)
+
+
+# ---------------------------------------------------------------- permute
+def permute_bf16(hidden_bits: np.ndarray, row_src: np.ndarray) -> np.ndarray:
+    """hidden_bits: uint16 [N,H] bf16 bit patterns; returns uint16 [rows,H]."""
+    hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
+    row_src = np.ascontiguousarray(row_src, dtype=np.int32)
+    H = hidden_bits.shape[1]
+    out = np.empty((row_src.size, H), np.uint16)
+    lib().orc_permute_bf16(row_src.size, H, _p(hidden_bits), _p(row_src), _p(out))
+    return out
+
+
+def permute_fp8(hidden_bits: np.ndarray, row_src: np.ndarray):
+    hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
+    row_src = np.ascontiguousarray(row_src, dtype=np.int32)
+    H = hidden_bits.shape[1]
+    q = np.empty((row_src.size, H), np.uint8)
+    sc = np.empty((row_src.size, H // 128), np.float32)
+    lib().orc_permute_fp8(row_src.size, H, _p(hidden_bits), _p(row_src), _p(q), _p(sc))
+    return q, sc
+
+
+def permute_nvfp4(hidden_bits: np.ndarray, row_src: np.ndarray, global_scale: float):
+    hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
+    row_src = np.ascontiguousarray(row_src, dtype=np.int32)
+    H = hidden_bits.shape[1]
+    q = np.empty((row_src.size, H // 2), np.uint8)
+    sc = np.empty((row_src.size, H // 16), np.uint8)
+    lib().orc_permute_nvfp4(row_src.size, H, _p(hidden_bits), _p(row_src),
+                            float(np.float32(global_scale)), _p(q), _p(sc))
+    return q, sc
+
+
+# ---------------------------------------------------------------- combine
+def combine(expert_out_bits: np.ndarray, gates: np.ndarray,
+            pair_slot: np.ndarray) -> np.ndarray:
+    """expert_out_bits: uint16 [rows,H] bf16; gates f32 [N,k]; returns uint16 [N,H]."""
+    expert_out_bits = np.ascontiguousarray(expert_out_bits, dtype=np.uint16)
+    gates = np.ascontiguousarray(gates, dtype=np.float32)
+    pair_slot = np.ascontiguousarray(pair_slot, dtype=np.int32)
+    N, k = pair_slot.shape
+    rows, H = expert_out_bits.shape
+    y = np.empty((N, H), np.uint16)
+    lib().orc_combine(N, k, H, rows, _p(expert_out_bits), _p(gates), _p(pair_slot), _p(y))
+    return y

@@ -1,0 +1,389 @@
+/*
+ * oracle.c -- CPU oracle for MoE dispatch layout, permute (bf16 / block FP8
+ * / NVFP4) and combine.  TEST INFRASTRUCTURE ONLY: see oracle.h for who may
+ * call it and for the sources each part follows.
+ *
+ * Written as the plain definitions: one sequential pass over the pairs in
+ * ascending (token, k) order, one output row at a time, one block at a
+ * time.  No tiling, no reordering, no shared tables with the GPU path.
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math (IEEE binary32 with
+ * round-to-nearest-even; fused multiply-add only where fmaf is written).
+ */
+#include "oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ */
+/* Number formats                                                      */
+/* ------------------------------------------------------------------ */
+
+static uint32_t f32_bits(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  return u;
+}
+
+static float f32_from_bits(uint32_t u) {
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* bfloat16 keeps the sign, the 8 exponent bits and the top 7 fraction bits
+ * of binary32.  Rounding to nearest, ties to even, on the dropped 16 bits:
+ * add 0x7FFF plus the lowest kept bit, then truncate.  A carry out of the
+ * fraction increments the exponent, which is the correct rounding (and
+ * yields infinity past the largest finite value).  NaN stays a quiet NaN. */
+uint16_t orc_bf16_from_f32(float f) {
+  uint32_t u = f32_bits(f);
+  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu) != 0)
+    return (uint16_t)((u >> 16) | 0x0040u);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+float orc_bf16_to_f32(uint16_t b) { return f32_from_bits((uint32_t)b << 16); }
+
+/* Round a non-negative double that holds an exact value to the nearest
+ * integer, ties to even (rint under the default rounding mode). */
+static double rne_int(double v) { return rint(v); }
+
+/* OCP 8-bit FP, E4M3 ("fn": no infinities; S.1111.111 is NaN).
+ * Exponent bias 7.  Normal: (1 + m/8) * 2^(e-7), e in 1..15, with
+ * (e,m) = (15,7) reserved for NaN, so the largest finite value is
+ * 1.75 * 2^8 = 448.  Subnormal (e = 0): m/8 * 2^-6 = m * 2^-9.
+ * Conversion: round to nearest, ties to even code; magnitudes beyond 448
+ * saturate to 448 (the satfinite rule).  Sign is kept, also for zero. */
+uint8_t orc_e4m3_from_f32(float f) {
+  uint8_t sign = signbit(f) ? 0x80 : 0x00;
+  if (isnan(f)) return (uint8_t)(sign | 0x7F);
+  double a = fabs((double)f);
+  if (a > 448.0) return (uint8_t)(sign | 0x7E);
+  uint32_t code;
+  if (a < ldexp(1.0, -6)) {
+    /* subnormal range: integer multiples of 2^-9; 8 * 2^-9 is the
+     * smallest normal and gets code 8 = (e=1, m=0) automatically */
+    code = (uint32_t)rne_int(a * 512.0);
+  } else {
+    int e2;
+    double fr = frexp(a, &e2); /* a = fr * 2^e2, fr in [0.5, 1) */
+    int e = e2 - 1;            /* a = (2*fr) * 2^e, 2*fr in [1, 2) */
+    double m = rne_int((2.0 * fr - 1.0) * 8.0);
+    if (m >= 8.0) {
+      m = 0.0;
+      e += 1;
+    }
+    code = (uint32_t)(((e + 7) << 3) | (int)m);
+    if (code > 0x7E) code = 0x7E;
+  }
+  return (uint8_t)(sign | code);
+}
+
+float orc_e4m3_to_f32(uint8_t c) {
+  int s = (c >> 7) & 1, e = (c >> 3) & 15, m = c & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m, -9);
+  else
+    v = ldexp(1.0 + m / 8.0, e - 7);
+  return (float)(s ? -v : v);
+}
+
+/* OCP MX E2M1: exponent bias 1.  Normal: (1 + m/2) * 2^(e-1), e in 1..3;
+ * subnormal (e = 0): m * 0.5.  Values {0, .5, 1, 1.5, 2, 3, 4, 6}; no inf
+ * or NaN.  Round to nearest, ties to even code; saturate beyond 6. */
+uint8_t orc_e2m1_from_f32(float f) {
+  uint8_t sign = signbit(f) ? 0x8 : 0x0;
+  if (isnan(f)) return (uint8_t)(sign | 0x7);
+  double a = fabs((double)f);
+  if (a > 6.0) return (uint8_t)(sign | 0x7);
+  uint32_t code;
+  if (a < 1.0) {
+    code = (uint32_t)rne_int(a * 2.0); /* 0, 1 (=0.5) or 2 (=1.0) */
+  } else {
+    int e2;
+    double fr = frexp(a, &e2);
+    int e = e2 - 1;
+    double m = rne_int((2.0 * fr - 1.0) * 2.0);
+    if (m >= 2.0) {
+      m = 0.0;
+      e += 1;
+    }
+    code = (uint32_t)(((e + 1) << 1) | (int)m);
+    if (code > 0x7) code = 0x7;
+  }
+  return (uint8_t)(sign | code);
+}
+
+float orc_e2m1_to_f32(uint8_t c) {
+  int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+  double v = (e == 0) ? 0.5 * m : ldexp(1.0 + m / 2.0, e - 1);
+  return (float)(s ? -v : v);
+}
+
+void orc_bf16_from_f32_n(const float *in, uint16_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_from_f32(in[i]);
+}
+void orc_e4m3_from_f32_n(const float *in, uint8_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_from_f32(in[i]);
+}
+void orc_e2m1_from_f32_n(const float *in, uint8_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m1_from_f32(in[i]);
+}
+
+/* ------------------------------------------------------------------ */
+/* Dispatch layout                                                     */
+/* ------------------------------------------------------------------ */
+
+/* Counting sort of the routed pairs by expert, stable in pair order.
+ *
+ * A pair p = t*k + j routes token t to expert ids[p].  Id -1 means the
+ * pair is masked out (NeMo token_dispatcher, _indices_to_multihot and
+ * _HybridEPMetadataProcessor.forward: invalid slots contain -1); any other
+ * id outside [0, E) is reported and treated as masked.
+ *
+ * Packed (dropless) mode, NKI permute_a2av: rows are packed expert-major
+ * (hence destination-segment-major, since segment s holds experts
+ * [s*L, (s+1)*L)); expert e's rows start at the exclusive cumulative sum of
+ * the counts; within an expert, rows follow ascending pair index.  Rows
+ * [total, C) are padding.  A pair whose row would be >= C gets no row
+ * (status CAPACITY); the counts stay the true counts.
+ *
+ * Capacity mode, DeepSpeed capacity dispatch ([e, c, m] buffer) with the
+ * capacity of NeMo's moe_expert_capacity_factor: the r-th pair routed to
+ * expert e (in ascending pair order) takes row e*Ce + r when r < Ce and is
+ * dropped otherwise.
+ *
+ * send_counts / send_displs / recv_counts / recv_displs (NKI [4, EP]
+ * uint32 metadata, in elements): per destination segment the kept rows
+ * times H, and their exclusive cumulative sum (packed) or the static
+ * segment start s*L*Ce*H (capacity).  On one device the receive rows equal
+ * the send rows. */
+uint32_t orc_layout(int32_t N, int32_t k, int32_t E, int32_t S, int64_t C,
+                    int32_t Ce, uint32_t flags, int32_t H,
+                    const int32_t *ids, int32_t *expert_counts,
+                    int32_t *expert_offsets, uint32_t *meta, int32_t *row_src,
+                    int32_t *pair_slot, uint8_t *drop_mask) {
+  uint32_t status = 0;
+  const int64_t P = (int64_t)N * k;
+  const int capacity_mode = Ce > 0;
+  const int64_t rows = capacity_mode ? (int64_t)E * Ce : C;
+  const int32_t L = E / S;
+
+  int64_t *cnt = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+  int64_t *seen = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+  int64_t *off = (int64_t *)calloc((size_t)E + 1, sizeof(int64_t));
+
+  /* 1. count the routed pairs per expert (tokens per expert, NeMo
+   *    get_number_of_tokens_per_expert) */
+  for (int64_t p = 0; p < P; ++p) {
+    int32_t e = ids[p];
+    if (e == -1) continue;
+    if (e < 0 || e >= E) {
+      status |= ORC_STATUS_ID_RANGE;
+      continue;
+    }
+    cnt[e] += 1;
+  }
+
+  /* optional: a token naming one expert twice (NKI recv_capacity note:
+   * duplicates invalidate the dropless bound) */
+  if (flags & ORC_FLAG_CHECK_DUPLICATES) {
+    for (int32_t t = 0; t < N; ++t)
+      for (int32_t a = 0; a < k; ++a)
+        for (int32_t b = a + 1; b < k; ++b) {
+          int32_t ea = ids[(int64_t)t * k + a], eb = ids[(int64_t)t * k + b];
+          if (ea >= 0 && ea < E && ea == eb) status |= ORC_STATUS_DUP_ID;
+        }
+  }
+
+  /* 2. expert start rows: exclusive cumulative sum (packed) or e*Ce */
+  for (int32_t e = 0; e < E; ++e)
+    off[e + 1] = off[e] + (capacity_mode ? (int64_t)Ce : cnt[e]);
+  for (int32_t e = 0; e <= E; ++e) expert_offsets[e] = (int32_t)off[e];
+  for (int32_t e = 0; e < E; ++e)
+    expert_counts[e] = (int32_t)(capacity_mode && cnt[e] > Ce ? Ce : cnt[e]);
+
+  /* 3. every row starts as padding (source -1) */
+  for (int64_t r = 0; r < rows; ++r) row_src[r] = -1;
+
+  /* 4. place the pairs in ascending pair order */
+  for (int64_t p = 0; p < P; ++p) {
+    int32_t e = ids[p];
+    int32_t slot = -1;
+    int dropped = 0;
+    if (e >= 0 && e < E) {
+      int64_t r = seen[e]++;
+      int64_t row;
+      if (capacity_mode) {
+        row = (r < Ce) ? (int64_t)e * Ce + r : -1;
+      } else {
+        row = off[e] + r;
+        if (row >= C) {
+          row = -1;
+          status |= ORC_STATUS_CAPACITY;
+        }
+      }
+      if (row >= 0) {
+        slot = (int32_t)row;
+        row_src[row] = (int32_t)(p / k);
+      } else {
+        dropped = 1;
+      }
+    }
+    pair_slot[p] = slot;
+    if (drop_mask) drop_mask[p] = (uint8_t)dropped;
+  }
+
+  /* 5. [4, S] uint32 metadata in elements (rows * H) */
+  int64_t disp = 0;
+  for (int32_t s = 0; s < S; ++s) {
+    int64_t seg_rows = 0;
+    for (int32_t e = s * L; e < (s + 1) * L; ++e) seg_rows += expert_counts[e];
+    uint32_t count_el = (uint32_t)(seg_rows * H);
+    uint32_t displ_el =
+        capacity_mode ? (uint32_t)((int64_t)s * L * Ce * H) : (uint32_t)disp;
+    meta[0 * S + s] = count_el;
+    meta[1 * S + s] = displ_el;
+    meta[2 * S + s] = count_el;
+    meta[3 * S + s] = displ_el;
+    disp += seg_rows * H;
+  }
+
+  free(cnt);
+  free(seen);
+  free(off);
+  return status;
+}
+
+/* ------------------------------------------------------------------ */
+/* Permute                                                             */
+/* ------------------------------------------------------------------ */
+
+/* NKI permute_a2av return value: [C, H] rows, packed, followed by
+ * deterministic zero padding.  Mojo ep_comm BF16TokenFormat: the full row
+ * in bfloat16.  Row r is hidden row row_src[r]; a padding row is zeros. */
+void orc_permute_bf16(int64_t rows, int32_t H, const uint16_t *hidden,
+                      const int32_t *row_src, uint16_t *out) {
+  for (int64_t r = 0; r < rows; ++r) {
+    uint16_t *dst = out + r * H;
+    int32_t t = row_src[r];
+    if (t < 0) {
+      for (int32_t h = 0; h < H; ++h) dst[h] = 0;
+    } else {
+      const uint16_t *src = hidden + (int64_t)t * H;
+      for (int32_t h = 0; h < H; ++h) dst[h] = src[h];
+    }
+  }
+}
+
+/* Mojo ep_comm BlockwiseFP8TokenFormat: FP8 with block-wise scales.  Each
+ * 1x128 block of a row gets one fp32 scale = amax / 448 (the decode
+ * multiplier: x ~ q * scale); every element is x / scale rounded to E4M3
+ * (nearest even, saturating).  A block whose amax is 0 gets scale 0 and
+ * zero codes.  Padding rows: zero codes and zero scales. */
+void orc_permute_fp8(int64_t rows, int32_t H, const uint16_t *hidden,
+                     const int32_t *row_src, uint8_t *q, float *scales) {
+  const int32_t nb = H / 128;
+  for (int64_t r = 0; r < rows; ++r) {
+    int32_t t = row_src[r];
+    for (int32_t b = 0; b < nb; ++b) {
+      uint8_t *qd = q + r * H + (int64_t)b * 128;
+      float *sd = scales + r * nb + b;
+      if (t < 0) {
+        memset(qd, 0, 128);
+        *sd = 0.0f;
+        continue;
+      }
+      const uint16_t *src = hidden + (int64_t)t * H + (int64_t)b * 128;
+      float amax = 0.0f;
+      for (int32_t i = 0; i < 128; ++i) {
+        float a = fabsf(orc_bf16_to_f32(src[i]));
+        if (a > amax) amax = a;
+      }
+      if (amax == 0.0f) {
+        memset(qd, 0, 128);
+        *sd = 0.0f;
+        continue;
+      }
+      float sc = amax / 448.0f;
+      *sd = sc;
+      for (int32_t i = 0; i < 128; ++i)
+        qd[i] = orc_e4m3_from_f32(orc_bf16_to_f32(src[i]) / sc);
+    }
+  }
+}
+
+/* Mojo ep_comm NVBlockScaledTokenFormat and the
+ * ep.dispatch_async.block.scaled.nv op (global input scales supplied by the
+ * caller): E2M1 codes, one E4M3 scale per 16 elements, one fp32 global
+ * scale gs per tensor.  Per block: amax; block scale code
+ * sq = e4m3((amax / 6) / gs); decode scale d = float(sq) * gs; each
+ * element is x / d rounded to E2M1 (nearest even, saturating), or 0 when
+ * d == 0.  Two codes per byte, element 2m in the low nibble of byte m.
+ * Scales are stored row-major [rows, H/16].  Padding rows are all zero. */
+void orc_permute_nvfp4(int64_t rows, int32_t H, const uint16_t *hidden,
+                       const int32_t *row_src, float global_scale,
+                       uint8_t *q, uint8_t *scales) {
+  const int32_t nb = H / 16;
+  for (int64_t r = 0; r < rows; ++r) {
+    int32_t t = row_src[r];
+    for (int32_t b = 0; b < nb; ++b) {
+      uint8_t *qd = q + r * (H / 2) + (int64_t)b * 8;
+      uint8_t *sd = scales + r * nb + b;
+      if (t < 0) {
+        memset(qd, 0, 8);
+        *sd = 0;
+        continue;
+      }
+      const uint16_t *src = hidden + (int64_t)t * H + (int64_t)b * 16;
+      float amax = 0.0f;
+      for (int32_t i = 0; i < 16; ++i) {
+        float a = fabsf(orc_bf16_to_f32(src[i]));
+        if (a > amax) amax = a;
+      }
+      uint8_t sq = orc_e4m3_from_f32((amax / 6.0f) / global_scale);
+      float d = orc_e4m3_to_f32(sq) * global_scale;
+      *sd = sq;
+      for (int32_t m = 0; m < 8; ++m) {
+        uint8_t lo = 0, hi = 0;
+        if (d > 0.0f) {
+          lo = orc_e2m1_from_f32(orc_bf16_to_f32(src[2 * m]) / d);
+          hi = orc_e2m1_from_f32(orc_bf16_to_f32(src[2 * m + 1]) / d);
+        }
+        qd[m] = (uint8_t)(lo | (hi << 4));
+      }
+    }
+  }
+}
+
+/* ------------------------------------------------------------------ */
+/* Combine                                                             */
+/* ------------------------------------------------------------------ */
+
+/* DeepSpeed combine: gather each token's expert results back and weight
+ * them by the gate values.  NeMo moe_router_dtype = 'fp32': weights and
+ * the weighted average in fp32.  Mojo ep_comm router_weights_wrapper_type:
+ * one fp32 weight per (token, k).  For token t the accumulator starts at
+ * +0 and takes acc = fma(w[t,j], x[slot(t,j)], acc) for j = 0..k-1 in
+ * order, skipping a pair without a row (masked, dropped, or a slot outside
+ * [0, rows)); the result is rounded once to bfloat16. */
+void orc_combine(int32_t N, int32_t k, int32_t H, int64_t rows,
+                 const uint16_t *expert_out, const float *gates,
+                 const int32_t *pair_slot, uint16_t *y) {
+  for (int32_t t = 0; t < N; ++t) {
+    for (int32_t h = 0; h < H; ++h) {
+      float acc = 0.0f;
+      for (int32_t j = 0; j < k; ++j) {
+        int32_t s = pair_slot[(int64_t)t * k + j];
+        if (s < 0 || s >= rows) continue;
+        float x = orc_bf16_to_f32(expert_out[(int64_t)s * H + h]);
+        acc = fmaf(gates[(int64_t)t * k + j], x, acc);
+      }
+      y[(int64_t)t * H + h] = orc_bf16_from_f32(acc);
+    }
+  }
+}

@@ -1,0 +1,98 @@
+/*
+ * oracle.h -- plain, slow, single-threaded CPU oracle for MoE token
+ * dispatch (layout + permute, bf16 / block FP8 / NVFP4 payloads) and
+ * combine.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load or call this code.  It shares no
+ * source, header, table or helper with the CUDA library; the two agree
+ * only because both follow the same definitions.
+ *
+ * Sources the functions follow (cited by page title and section):
+ *   [NKI]  AWS Neuron NKI "Permute A2AV Kernel API Reference", permute_a2av
+ *          parameters (packed_source_indices, send_counts, recv_capacity)
+ *          and return values ([C,H] packed rows + deterministic zero
+ *          padding; [4,EP] uint32 counts/displacements in elements).
+ *   [NEMO] NeMo AutoModel token_dispatcher API: _indices_to_multihot
+ *          ("-1 means masked out"), get_number_of_tokens_per_expert,
+ *          TokenDispatcherConfig.moe_expert_capacity_factor and
+ *          moe_router_dtype (fp32 routing weights and weighted averaging).
+ *   [DS]   DeepSpeed v0.19.4 function list: the combine docstring (gather
+ *          each token's expert results and weight them by the gates) and
+ *          the capacity dispatch docstring ([e, c, m] expert-slot buffer).
+ *   [EPC]  Mojo MAX ep_comm module: BF16TokenFormat,
+ *          BlockwiseFP8TokenFormat, NVBlockScaledTokenFormat,
+ *          router_weights_wrapper_type (fp32 gate per (token, k)).
+ *   [EPD]  Mojo MAX Struct_ep_dispatch_async_block_scaled_nv: NVFP4
+ *          payload with a global input scale supplied by the caller.
+ * Format definitions written out from the public specifications:
+ *   IEEE 754 binary32; bfloat16 = top half of binary32 rounded to nearest
+ *   even; OCP 8-bit floating point (E4M3, "fn" variant: no infinities,
+ *   max 448); OCP Microscaling v1.0 (E2M1: max 6, no inf/NaN).
+ *
+ * Parity status: every function here is pinned by tests/test_oracle_*.py
+ * to something other than itself (library sorts, torch casts, brute-force
+ * nearest-value search over the format tables, closed forms, invariants
+ * the pages state).  The block-scale conventions of the FP8 and NVFP4
+ * quantisers (divide by the stored scale; scale = amax/448; NVFP4 block
+ * scale = e4m3((amax/6)/global_scale)) are readings of the pages, which
+ * print no worked example; the arithmetic under those readings is pinned.
+ */
+#ifndef MOE_ORACLE_H
+#define MOE_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status bits reported by orc_layout (same meaning as the library's). */
+#define ORC_STATUS_ID_RANGE 1u  /* an id outside [-1, E)                  */
+#define ORC_STATUS_DUP_ID 2u    /* a token names one expert twice          */
+#define ORC_STATUS_CAPACITY 4u  /* packed mode: more routed rows than C    */
+#define ORC_FLAG_CHECK_DUPLICATES 1u
+
+/* ---- number formats -------------------------------------------------- */
+uint16_t orc_bf16_from_f32(float f);
+float orc_bf16_to_f32(uint16_t b);
+uint8_t orc_e4m3_from_f32(float f); /* RNE, saturate to +-448 */
+float orc_e4m3_to_f32(uint8_t c);
+uint8_t orc_e2m1_from_f32(float f); /* RNE, saturate to +-6, 4-bit code */
+float orc_e2m1_to_f32(uint8_t c);
+
+void orc_bf16_from_f32_n(const float *in, uint16_t *out, int64_t n);
+void orc_e4m3_from_f32_n(const float *in, uint8_t *out, int64_t n);
+void orc_e2m1_from_f32_n(const float *in, uint8_t *out, int64_t n);
+
+/* ---- dispatch layout --------------------------------------------------
+ * ids[N*k] int32 (row-major [N,k]); E experts in S contiguous segments of
+ * L = E/S experts.  expert_capacity Ce == 0 selects packed (dropless) mode
+ * with C = recv_capacity rows; Ce > 0 selects the capacity layout [E,Ce].
+ * Outputs: expert_counts[E], expert_offsets[E+1], meta[4*S] (row-major
+ * [4,S]), row_src[rows] (rows = C, or E*Ce), pair_slot[N*k], drop_mask[N*k]
+ * (may be NULL).  Returns status bits.                                   */
+uint32_t orc_layout(int32_t N, int32_t k, int32_t E, int32_t S, int64_t C,
+                    int32_t Ce, uint32_t flags, int32_t H,
+                    const int32_t *ids, int32_t *expert_counts,
+                    int32_t *expert_offsets, uint32_t *meta, int32_t *row_src,
+                    int32_t *pair_slot, uint8_t *drop_mask);
+
+/* ---- permute: out row r = hidden row row_src[r], or zeros ------------- */
+void orc_permute_bf16(int64_t rows, int32_t H, const uint16_t *hidden,
+                      const int32_t *row_src, uint16_t *out);
+void orc_permute_fp8(int64_t rows, int32_t H, const uint16_t *hidden,
+                     const int32_t *row_src, uint8_t *q, float *scales);
+void orc_permute_nvfp4(int64_t rows, int32_t H, const uint16_t *hidden,
+                       const int32_t *row_src, float global_scale,
+                       uint8_t *q, uint8_t *scales);
+
+/* ---- combine ---------------------------------------------------------- */
+void orc_combine(int32_t N, int32_t k, int32_t H, int64_t rows,
+                 const uint16_t *expert_out, const float *gates,
+                 const int32_t *pair_slot, uint16_t *y);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
