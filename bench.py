@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the single-GPU MoE dispatch + combine hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N
+
+One step = one pass of the whole hot path over one batch:
+    dispatch layout (count + look-back scan, emit)  ->  permute bf16  ->
+    permute + block FP8  ->  permute + NVFP4  ->  combine (bf16 out)
+on the metric workload N=8192 tokens, H=7168, E=256 experts, top_k=8,
+S=8 segments, recv_capacity = N*top_k (seeded synthetic inputs, uniform
+distinct routing, 1% outlier rows, expert outputs ~N(0,1)).
+
+Each rank runs its own batch (replicas; weak scaling, no data-path
+collective); the timed region is bracketed by a barrier and device
+synchronisation, every step is timed with CUDA events on the launching stream,
+and the max over ranks is reported.  L2 is flushed (a write of twice its
+size) before every step, outside the events.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine tokens/s and HBM GB/s (% of peak) at N=8192 H=7168 E=256 k=8"
+WORKLOAD = "fp8_metric"
+FALLBACK_HBM_GBS = 6650.0
+
+# dram bytes per launch from one ncu capture, keyed by kernel, valid only
+# while the kernel source is unchanged (sha256 of the .cu file at capture)
+NCU_TRAFFIC: dict[str, dict] = {}
+
+
+def _kernel_src_sha(name: str) -> str:
+    path = os.path.join(ROOT, "combine_topk_ids_scan_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ bytes
+def algorithmic_bytes(w, total_rows: int) -> dict:
+    """Compulsory HBM bytes per step phase (each input read once, each output
+    written once) for workload w whose layout routed `total_rows` rows."""
+    N, H, k, P, rows, E, S = w.N, w.H, w.k, w.P, w.rows, w.E, w.S
+    maps_read = 4 * P + 4 * rows          # pair_slot + row_src read by a permute
+    return {
+        "layout": 4 * P + 4 * P + 4 * rows + P + 8 * E + 4 + 16 * S,
+        "permute_bf16": 2 * N * H + maps_read + 2 * rows * H,
+        "permute_fp8": 2 * N * H + maps_read + rows * H + 4 * rows * (H // 128),
+        "permute_nvfp4": 2 * N * H + maps_read + rows * H // 2 + rows * (H // 16) + 4,
+        "combine": 2 * total_rows * H + 4 * P + 4 * P + 2 * N * H,
+    }
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.lines: list[str] = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            if self.uuid and self.uuid not in f[0]:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ dist
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ------------------------------------------------------------------ oracle
+def oracle_tokens_per_s(w, n_tokens: int, start: int = 0) -> tuple[float, float]:
+    """Time the CPU oracle (as it stands, single thread) on the sub-batch of
+    tokens [start, start+n): layout, the three permutes and the combine.
+    Returns (tokens/s, seconds)."""
+    import oracle
+    oracle.build()
+    n = min(n_tokens, w.N)
+    idx = (np.arange(n) + start) % w.N
+    ids = np.ascontiguousarray(w.ids[idx])
+    hidden = np.ascontiguousarray(w.hidden[idx])
+    gates = np.ascontiguousarray(w.gates[idx])
+    C = n * w.k
+    X = np.ascontiguousarray(w.expert_out[:C]) if w.expert_out is not None else None
+    t0 = time.perf_counter()
+    lay = oracle.layout(ids, w.E, w.S, w.H, recv_capacity=C)
+    oracle.permute_bf16(hidden, lay.row_src)
+    oracle.permute_fp8(hidden, lay.row_src)
+    oracle.permute_nvfp4(hidden, lay.row_src, w.global_scale)
+    if X is not None:
+        oracle.combine(X, gates, lay.pair_slot)
+    dt = time.perf_counter() - t0
+    return n / dt, dt
+
+
+def run_reference(args, rank: int, world: int) -> int:
+    """Reference arm: the CPU oracle timed on bounded samples of the workload."""
+    if rank != 0:
+        return 0
+    from combine_topk_ids_scan_b200.inputs import make_workload
+    w = make_workload(WORKLOAD)
+    # ~1.8 ms of oracle work per token; keep the whole run near a minute
+    per_step = max(8, min(2048, int(60.0 / max(1, args.steps + args.warmup) / 1.8e-3)))
+    for i in range(args.warmup):
+        oracle_tokens_per_s(w, per_step, start=i * per_step)
+    times = []
+    for i in range(args.steps):
+        _, dt = oracle_tokens_per_s(w, per_step, start=(args.warmup + i) * per_step)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = per_step / (ms / 1e3)
+    sample = (f"{per_step} consecutive tokens of the {WORKLOAD} batch per step "
+              f"(own layout with recv_capacity = {per_step}*k)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w) -> dict:
+    return {"workload": f"{w.name}: N={w.N} H={w.H} E={w.E} top_k={w.k} S={w.S} "
+                        f"recv_capacity={w.recv_capacity}",
+            "N": w.N, "H": w.H, "E": w.E, "top_k": w.k, "segments": w.S,
+            "recv_capacity": w.recv_capacity,
+            "step": "layout + permute(bf16) + permute(fp8 1x128) + permute(nvfp4) + combine",
+            "l2": "flushed before every step (write of 2x L2 size), outside the timed events",
+            "parallelism": "replicas (independent token batches per GPU)"}
+
+
+# ------------------------------------------------------------------ ours
+def run_ours(args, rank: int, world: int, local: int) -> int:
+    import torch
+    import torch.distributed as dist
+
+    from combine_topk_ids_scan_b200 import binding as B
+    from combine_topk_ids_scan_b200.inputs import make_workload
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    B.load()
+    w = make_workload(WORKLOAD, seed=None if rank == 0 else 1002 + 7919 * rank)
+    prob = B.Problem(num_tokens=w.N, hidden=w.H, num_experts=w.E, top_k=w.k,
+                     num_segments=w.S, recv_capacity=w.recv_capacity,
+                     expert_capacity=w.expert_capacity)
+    buf = B.Buffers(prob, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # host inputs (pinned) and their device copies
+    h_ids = torch.from_numpy(w.ids).pin_memory()
+    h_hidden = torch.from_numpy(w.hidden.view(np.int16)).pin_memory()
+    h_gates = torch.from_numpy(w.gates).pin_memory()
+    h_x = torch.from_numpy(w.expert_out.view(np.int16)).pin_memory()
+    h_gs = torch.tensor([w.global_scale], dtype=torch.float32).pin_memory()
+    d_ids = h_ids.to(dev)
+    d_hidden = h_hidden.to(dev).view(torch.bfloat16)
+    d_gates = h_gates.to(dev)
+    d_x = h_x.to(dev).view(torch.bfloat16)
+    d_gs = h_gs.to(dev)
+    d_y = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
+    h_y = torch.empty((w.N, w.H), dtype=torch.int16).pin_memory()
+    h_status = torch.empty(1 + w.E, dtype=torch.int32).pin_memory()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        B.layout(prob, d_ids, buf)
+        if ev is not None:
+            ev[1].record(stream)
+        B.moe_permute(prob, d_hidden, buf.row_src, buf.pair_slot, buf.out)
+        if ev is not None:
+            ev[2].record(stream)
+        B.moe_permute_quant_fp8(prob, d_hidden, buf.row_src, buf.pair_slot, buf.out_fp8,
+                                buf.scales_fp8)
+        if ev is not None:
+            ev[3].record(stream)
+        B.moe_permute_quant_nvfp4(prob, d_hidden, buf.row_src, buf.pair_slot, d_gs,
+                                  buf.out_fp4, buf.scales_fp4)
+        if ev is not None:
+            ev[4].record(stream)
+        B.moe_combine(prob, d_x, d_gates, buf.pair_slot, d_y)
+        if ev is not None:
+            ev[5].record(stream)
+
+    launches_per_step = (2 if w.P > 0 else 1) + 4
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    st = int(buf.status.cpu().numpy().view(np.uint32)[0])
+    total_rows = int(buf.expert_counts.sum().item())
+
+    # ---- device-resident timed region
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    phases = ["layout", "permute_bf16", "permute_fp8", "permute_nvfp4", "combine"]
+    per = {p: [] for p in phases}
+    step_ms = []
+    for e in evs:
+        for i, p in enumerate(phases):
+            per[p].append(e[i].elapsed_time(e[i + 1]))
+        step_ms.append(e[0].elapsed_time(e[5]))
+    ms = sum(step_ms) / len(step_ms)
+    phase_ms = {p: sum(v) / len(v) for p, v in per.items()}
+
+    # ---- end to end through the public API from pinned host memory
+    e2e_steps = max(3, min(args.steps, 20))
+    h2d = (h_ids.numel() * 4 + h_hidden.numel() * 2 + h_gates.numel() * 4 + h_x.numel() * 2 + 4)
+    d2h = h_y.numel() * 2 + 4 * (1 + w.E)
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e_start.record(stream)
+    for _ in range(e2e_steps):
+        d_ids.copy_(h_ids, non_blocking=True)
+        d_hidden.view(torch.int16).copy_(h_hidden, non_blocking=True)
+        d_gates.copy_(h_gates, non_blocking=True)
+        d_x.view(torch.int16).copy_(h_x, non_blocking=True)
+        d_gs.copy_(h_gs, non_blocking=True)
+        step()
+        h_y.copy_(d_y.view(torch.int16), non_blocking=True)
+        h_status[:1].copy_(buf.status, non_blocking=True)
+        h_status[1:].copy_(buf.expert_counts, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end) / e2e_steps
+
+    # ---- max over ranks
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms] + [phase_ms[p] for p in phases], device=dev,
+                         dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+        phase_ms = {p: float(t[2 + i]) for i, p in enumerate(phases)}
+
+    if rank == 0:
+        nbytes = algorithmic_bytes(w, total_rows)
+        step_bytes = sum(nbytes.values())
+        peak, peak_kind = _peaks()
+        dom = max(("permute_bf16", "permute_fp8", "permute_nvfp4", "combine"),
+                  key=lambda p: phase_ms[p])
+        achieved = nbytes[dom] / (phase_ms[dom] * 1e-3) / 1e9
+        src = {"permute_bf16": "permute.cu", "permute_fp8": "permute.cu",
+               "permute_nvfp4": "permute.cu", "combine": "combine.cu"}[dom]
+        tr = NCU_TRAFFIC.get(dom)
+        traffic = tr["bytes_per_launch"] if tr and tr.get("src_sha") == _kernel_src_sha(src) \
+            else None
+        value = world * w.N / (ms * 1e-3)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp32", "data": "synthetic", "config": workload_config(w),
+            "hbm_gbs": step_bytes / (ms * 1e-3) / 1e9,
+            "hbm_frac_of_peak": step_bytes / (ms * 1e-3) / 1e9 / peak,
+            "phases_us": {p: round(1e3 * v, 2) for p, v in phase_ms.items()},
+            "phases_gbs": {p: round(nbytes[p] / (phase_ms[p] * 1e-3) / 1e9, 1)
+                           for p in phases},
+            "dispatch_bf16_plus_combine_tokens_per_s":
+                world * w.N / ((phase_ms["layout"] + phase_ms["permute_bf16"]
+                                + phase_ms["combine"]) * 1e-3),
+            "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
+                         "peak_source": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_bytes": nbytes[dom]},
+            "e2e": {"value": world * w.N / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks, "layout_status": st,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            n_cpu = args.cpu_tokens
+            tps, dt = oracle_tokens_per_s(w, n_cpu)
+            line["cpu_baseline"] = {
+                "value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "sample": f"first {n_cpu} tokens of the batch, own layout with "
+                          f"recv_capacity = {n_cpu}*k; {dt:.1f} s single-threaded"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main() -> int:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-tokens", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

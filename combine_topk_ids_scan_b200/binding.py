@@ -1,0 +1,220 @@
+"""Thin ctypes binding of libmoedc.so (declared in include/moe_dc.h).
+
+Each function has the name of the C entry point it calls and only marshals
+arguments: torch tensors become device pointers, the current torch CUDA
+stream becomes the launch stream.  Every step of the computation runs in the
+library's CUDA kernels; there is no fallback of any kind -- if the library
+cannot be loaded, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoedc.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED_SHAPE = 2
+MOE_ERR_CUDA = 3
+
+MOE_STATUS_ID_RANGE = 1
+MOE_STATUS_DUP_ID = 2
+MOE_STATUS_CAPACITY = 4
+MOE_STATUS_TIMEOUT = 8
+
+MOE_FLAG_CHECK_DUPLICATES = 1
+MOE_FLAG_TEST_STALL_SCAN = 0x80000000
+
+MOE_MAX_EXPERTS = 2048
+MOE_MAX_TOPK = 16
+
+# every symbol include/moe_dc.h declares
+EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout", "moe_permute",
+            "moe_permute_quant_fp8", "moe_permute_quant_nvfp4", "moe_combine",
+            "moe_status_string", "moe_version")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {status_string(code)} (moe_status {code})")
+        self.code = code
+
+
+class moe_problem(ctypes.Structure):
+    _fields_ = [("num_tokens", ctypes.c_int32), ("hidden", ctypes.c_int32),
+                ("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("num_segments", ctypes.c_int32), ("expert_capacity", ctypes.c_int32),
+                ("recv_capacity", ctypes.c_int64), ("flags", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32)]
+
+
+@dataclass
+class Problem:
+    """Sizes of one dispatch / combine problem (see moe_problem in moe_dc.h)."""
+    num_tokens: int
+    hidden: int
+    num_experts: int
+    top_k: int
+    num_segments: int = 1
+    recv_capacity: int = 0
+    expert_capacity: int = 0
+    flags: int = 0
+
+    def c(self) -> moe_problem:
+        return moe_problem(self.num_tokens, self.hidden, self.num_experts, self.top_k,
+                           self.num_segments, self.expert_capacity, self.recv_capacity,
+                           self.flags & 0xFFFFFFFF, 0)
+
+
+_lib = None
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load libmoedc.so (once).  Raises if it is missing: there is no
+    fallback path."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"libmoedc.so not found at {path}; build it with "
+                           "`python -m combine_topk_ids_scan_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, P = ctypes.c_void_p, ctypes.POINTER(moe_problem)
+    L.moe_output_rows.restype = ctypes.c_int64
+    L.moe_output_rows.argtypes = [P]
+    L.moe_workspace_bytes.restype = ctypes.c_size_t
+    L.moe_workspace_bytes.argtypes = [P]
+    L.moe_dispatch_layout.restype = ctypes.c_int
+    L.moe_dispatch_layout.argtypes = [P] + [vp] * 10
+    L.moe_permute.restype = ctypes.c_int
+    L.moe_permute.argtypes = [P] + [vp] * 5
+    L.moe_permute_quant_fp8.restype = ctypes.c_int
+    L.moe_permute_quant_fp8.argtypes = [P] + [vp] * 6
+    L.moe_permute_quant_nvfp4.restype = ctypes.c_int
+    L.moe_permute_quant_nvfp4.argtypes = [P] + [vp] * 7
+    L.moe_combine.restype = ctypes.c_int
+    L.moe_combine.argtypes = [P] + [vp] * 5
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_status_string.argtypes = [ctypes.c_int]
+    L.moe_version.restype = ctypes.c_char_p
+    L.moe_version.argtypes = []
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return load().moe_status_string(code).decode()
+
+
+def version() -> str:
+    return load().moe_version().decode()
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: torch.cuda.Stream | None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(code: int, where: str) -> None:
+    if code != MOE_OK:
+        raise MoeError(code, where)
+
+
+def moe_output_rows(prob: Problem) -> int:
+    return int(load().moe_output_rows(ctypes.byref(prob.c())))
+
+
+def moe_workspace_bytes(prob: Problem) -> int:
+    return int(load().moe_workspace_bytes(ctypes.byref(prob.c())))
+
+
+def moe_dispatch_layout(prob: Problem, topk_ids, expert_counts, expert_offsets, meta, row_src,
+                        pair_slot, drop_mask, status, workspace, stream=None) -> None:
+    c = prob.c()
+    _check(load().moe_dispatch_layout(ctypes.byref(c), _ptr(topk_ids), _ptr(expert_counts),
+                                      _ptr(expert_offsets), _ptr(meta), _ptr(row_src),
+                                      _ptr(pair_slot), _ptr(drop_mask), _ptr(status),
+                                      _ptr(workspace), _stream(stream)),
+           "moe_dispatch_layout")
+
+
+def moe_permute(prob: Problem, hidden_states, row_src, pair_slot, out, stream=None) -> None:
+    c = prob.c()
+    _check(load().moe_permute(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
+                              _ptr(pair_slot), _ptr(out), _stream(stream)), "moe_permute")
+
+
+def moe_permute_quant_fp8(prob: Problem, hidden_states, row_src, pair_slot, out_e4m3, scales,
+                          stream=None) -> None:
+    c = prob.c()
+    _check(load().moe_permute_quant_fp8(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
+                                        _ptr(pair_slot), _ptr(out_e4m3), _ptr(scales),
+                                        _stream(stream)), "moe_permute_quant_fp8")
+
+
+def moe_permute_quant_nvfp4(prob: Problem, hidden_states, row_src, pair_slot, global_scale,
+                            out_e2m1, scales_e4m3, stream=None) -> None:
+    c = prob.c()
+    _check(load().moe_permute_quant_nvfp4(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
+                                          _ptr(pair_slot), _ptr(global_scale), _ptr(out_e2m1),
+                                          _ptr(scales_e4m3), _stream(stream)),
+           "moe_permute_quant_nvfp4")
+
+
+def moe_combine(prob: Problem, expert_out, gates, pair_slot, out, stream=None) -> None:
+    c = prob.c()
+    _check(load().moe_combine(ctypes.byref(c), _ptr(expert_out), _ptr(gates), _ptr(pair_slot),
+                              _ptr(out), _stream(stream)), "moe_combine")
+
+
+# ----------------------------------------------------------------- buffers
+class Buffers:
+    """Device buffers for one problem (allocated by torch; the library itself
+    allocates nothing).  Convenience for callers and tests."""
+
+    def __init__(self, prob: Problem, device="cuda", quant: bool = True):
+        N, H, E, k, S = (prob.num_tokens, prob.hidden, prob.num_experts, prob.top_k,
+                         prob.num_segments)
+        rows = moe_output_rows(prob)
+        if rows < 0:
+            raise MoeError(MOE_ERR_INVALID_ARG, "Buffers")
+        i32, u8 = torch.int32, torch.uint8
+        self.rows = rows
+        self.expert_counts = torch.empty(E, dtype=i32, device=device)
+        self.expert_offsets = torch.empty(E + 1, dtype=i32, device=device)
+        self.meta = torch.empty((4, S), dtype=torch.int32, device=device)  # uint32 bits
+        self.row_src = torch.empty(max(rows, 1), dtype=i32, device=device)
+        self.pair_slot = torch.empty((max(N, 1), k), dtype=i32, device=device)
+        self.drop_mask = torch.empty((max(N, 1), k), dtype=u8, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.workspace = torch.zeros(max(moe_workspace_bytes(prob), 16), dtype=u8, device=device)
+        self.out = torch.empty((max(rows, 1), H), dtype=torch.bfloat16, device=device)
+        if quant:
+            self.out_fp8 = torch.empty((max(rows, 1), H), dtype=u8, device=device)
+            self.scales_fp8 = torch.empty((max(rows, 1), max(H // 128, 1)), dtype=torch.float32,
+                                          device=device)
+            self.out_fp4 = torch.empty((max(rows, 1), H // 2), dtype=u8, device=device)
+            self.scales_fp4 = torch.empty((max(rows, 1), max(H // 16, 1)), dtype=u8,
+                                          device=device)
+
+
+def layout(prob: Problem, topk_ids: torch.Tensor, buf: Buffers, stream=None) -> None:
+    moe_dispatch_layout(prob, topk_ids, buf.expert_counts, buf.expert_offsets, buf.meta,
+                        buf.row_src, buf.pair_slot, buf.drop_mask, buf.status, buf.workspace,
+                        stream)

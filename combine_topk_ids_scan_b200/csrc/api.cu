@@ -1,0 +1,187 @@
+// api.cu -- the extern "C" entry points of libmoedc.so declared in
+// include/moe_dc.h: host-side validation of the problem and the pointers,
+// then kernel launches on the caller's stream.  Nothing here allocates or
+// synchronises.
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <vector>
+
+#include "internal.h"
+#include "moe_dc.h"
+
+namespace moe {
+
+int device_sm_count() {
+  static std::mutex mu;
+  static std::vector<int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace moe
+
+namespace {
+
+constexpr int64_t kU32Max = 4294967295ll;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Validates the problem and fills the derived sizes.
+moe_status make_shape(const moe_problem *p, moe::Shape *s) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (p->num_tokens < 0 || p->hidden <= 0 || p->num_experts <= 0 || p->top_k <= 0 ||
+      p->num_segments <= 0 || p->expert_capacity < 0 || p->recv_capacity < 0 ||
+      p->reserved != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (p->num_experts > MOE_MAX_EXPERTS || p->top_k > MOE_MAX_TOPK ||
+      p->num_experts % p->num_segments != 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  s->N = p->num_tokens;
+  s->H = p->hidden;
+  s->E = p->num_experts;
+  s->k = p->top_k;
+  s->S = p->num_segments;
+  s->Ce = p->expert_capacity;
+  s->C = p->expert_capacity > 0 ? 0 : p->recv_capacity;
+  s->rows = p->expert_capacity > 0 ? (int64_t)p->num_experts * p->expert_capacity
+                                   : p->recv_capacity;
+  s->P = (int64_t)p->num_tokens * p->top_k;
+  s->flags = p->flags;
+  // slots are int32; the [4, S] table counts elements in uint32
+  if (s->rows > 2147483647ll || s->P > 2147483647ll) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s->rows * s->H > kU32Max || s->P * s->H > kU32Max) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int64_t moe_output_rows(const moe_problem *problem) {
+  moe::Shape s;
+  if (make_shape(problem, &s) != MOE_OK) return -1;
+  return s.rows;
+}
+
+size_t moe_workspace_bytes(const moe_problem *problem) {
+  moe::Shape s;
+  if (make_shape(problem, &s) != MOE_OK) return 0;
+  return moe::layout_workspace_bytes(s);
+}
+
+moe_status moe_dispatch_layout(const moe_problem *problem, const int32_t *topk_ids,
+                               int32_t *expert_counts, int32_t *expert_offsets,
+                               uint32_t *meta, int32_t *row_src, int32_t *pair_slot,
+                               uint8_t *drop_mask, uint32_t *status, void *workspace,
+                               moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (!expert_counts || !expert_offsets || !meta || !status || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (s.P > 0 && (!topk_ids || !pair_slot)) return MOE_ERR_INVALID_ARG;
+  if (s.rows > 0 && !row_src) return MOE_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16) || !aligned(topk_ids, 4) || !aligned(pair_slot, 4) ||
+      !aligned(row_src, 4) || !aligned(status, 4))
+    return MOE_ERR_INVALID_ARG;
+  moe::LayoutWorkspace ws = moe::layout_workspace_view(s, workspace);
+  return from_cuda(moe::launch_layout(s, topk_ids, expert_counts, expert_offsets, meta, row_src,
+                                      pair_slot, drop_mask, status, ws,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute(const moe_problem *problem, const void *hidden_states,
+                       const int32_t *row_src, const int32_t *pair_slot, void *out,
+                       moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.rows == 0) return MOE_OK;
+  if (!row_src || !out || (s.P > 0 && (!hidden_states || !pair_slot)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(hidden_states, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_permute_bf16(s, hidden_states, row_src, pair_slot, out,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute_quant_fp8(const moe_problem *problem, const void *hidden_states,
+                                 const int32_t *row_src, const int32_t *pair_slot,
+                                 uint8_t *out_e4m3, float *scales, moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.rows == 0) return MOE_OK;
+  if (!row_src || !out_e4m3 || !scales || (s.P > 0 && (!hidden_states || !pair_slot)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(hidden_states, 16) || !aligned(out_e4m3, 16) || !aligned(scales, 4))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_permute_fp8(s, hidden_states, row_src, pair_slot, out_e4m3,
+                                           scales, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute_quant_nvfp4(const moe_problem *problem, const void *hidden_states,
+                                   const int32_t *row_src, const int32_t *pair_slot,
+                                   const float *global_scale, uint8_t *out_e2m1,
+                                   uint8_t *scales_e4m3, moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 32 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.rows == 0) return MOE_OK;
+  if (!row_src || !out_e2m1 || !scales_e4m3 || !global_scale ||
+      (s.P > 0 && (!hidden_states || !pair_slot)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(hidden_states, 16) || !aligned(out_e2m1, 16) || !aligned(scales_e4m3, 2) ||
+      !aligned(global_scale, 4))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_permute_nvfp4(s, hidden_states, row_src, pair_slot, global_scale,
+                                             out_e2m1, scales_e4m3,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_combine(const moe_problem *problem, const void *expert_out, const float *gates,
+                       const int32_t *pair_slot, void *out, moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.N == 0) return MOE_OK;
+  if (!out || !gates || !pair_slot || (s.rows > 0 && !expert_out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(expert_out, 16) || !aligned(out, 16) || !aligned(gates, 4))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_combine(s, expert_out, gates, pair_slot, out,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char *moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK:
+      return "ok";
+    case MOE_ERR_INVALID_ARG:
+      return "invalid argument (null or misaligned pointer, negative size, reserved field)";
+    case MOE_ERR_UNSUPPORTED_SHAPE:
+      return "unsupported shape (size outside the library's limits)";
+    case MOE_ERR_CUDA:
+      return "CUDA error while launching";
+    default:
+      return "unknown status";
+  }
+}
+
+const char *moe_version(void) { return "moedc 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

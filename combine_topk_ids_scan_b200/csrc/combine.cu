@@ -1,0 +1,129 @@
+// combine.cu -- gather each token's k expert-output rows back and sum them
+// weighted by the token's gates: fp32 fused multiply-adds in fixed j order,
+// one round-to-nearest-even to bf16 at the end.
+//
+// Definitions: DeepSpeed combine docstring (gather each token's expert results
+// back and weight them by the gate values); NeMo AutoModel TokenDispatcher
+// config moe_router_dtype = 'fp32' (routing weights and the weighted average
+// in fp32); Mojo MAX ep_comm router_weights_wrapper_type (an fp32 weight per
+// (token, k)).
+//
+// One warp per token (persistent grid).  Lane j < k fetches the pair's row
+// and gate, shuffles broadcast them; per step each lane loads one 16-byte
+// vector (8 bf16) from every live row -- U steps at once, so up to k*U
+// independent 16-byte loads per lane are in flight -- and writes one 16-byte
+// vector of the result.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr uint32_t kFull = 0xFFFFFFFFu;
+
+template <int KMAX, int U>
+__global__ void __launch_bounds__(kThreads)
+    combine_kernel(const uint4 *__restrict__ x, const float *__restrict__ gates,
+                   const int32_t *__restrict__ pair_slot, uint4 *__restrict__ out, int32_t N,
+                   int32_t k, int64_t rows, int32_t vecs) {
+  const int lane = threadIdx.x % kWarp;
+  const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) / kWarp;
+
+  for (int64_t t = gw; t < N; t += nw) {
+    int32_t my_slot = -1;
+    float my_w = 0.0f;
+    if (lane < k) {
+      const int32_t s = __ldg(pair_slot + t * k + lane);
+      if (s >= 0 && s < rows) {
+        my_slot = s;
+        my_w = __ldg(gates + t * k + lane);
+      }
+    }
+    int64_t row[KMAX];
+    float w[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      const int32_t s = __shfl_sync(kFull, my_slot, j);
+      row[j] = s;
+      w[j] = __shfl_sync(kFull, my_w, j);
+    }
+    uint4 *dst = out + t * vecs;
+    for (int v0 = 0; v0 < vecs; v0 += kWarp * U) {
+      uint4 in[KMAX][U];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * kWarp + lane;
+          in[j][u] = (row[j] >= 0 && v < vecs) ? ld_stream_v4(x + row[j] * vecs + v)
+                                                : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int v = v0 + u * kWarp + lane;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          if (row[j] < 0) continue;
+          const uint32_t e[4] = {in[j][u].x, in[j][u].y, in[j][u].z, in[j][u].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] = fmaf(w[j], bf16lo(e[i]), acc[2 * i]);
+            acc[2 * i + 1] = fmaf(w[j], bf16hi(e[i]), acc[2 * i + 1]);
+          }
+        }
+        if (v < vecs)
+          st_v4(dst + v, make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                    pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7])));
+      }
+    }
+  }
+}
+
+template <typename Kernel>
+int grid_for(Kernel kernel, int64_t N) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const int64_t need = std::max<int64_t>(1, (N + kThreads / kWarp - 1) / (kThreads / kWarp));
+  return (int)std::min<int64_t>(need, (int64_t)per_sm * device_sm_count());
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const Shape &s, const void *expert_out, const float *gates,
+                           const int32_t *pair_slot, void *out, cudaStream_t stream) {
+  if (s.N == 0) return cudaSuccess;
+  const uint4 *x = static_cast<const uint4 *>(expert_out);
+  uint4 *o = static_cast<uint4 *>(out);
+  const int32_t vecs = s.H / 8;
+  if (s.k <= 2) {
+    auto kernel = combine_kernel<2, 4>;
+    kernel<<<grid_for(kernel, s.N), kThreads, 0, stream>>>(x, gates, pair_slot, o, s.N, s.k,
+                                                            s.rows, vecs);
+  } else if (s.k <= 4) {
+    auto kernel = combine_kernel<4, 2>;
+    kernel<<<grid_for(kernel, s.N), kThreads, 0, stream>>>(x, gates, pair_slot, o, s.N, s.k,
+                                                            s.rows, vecs);
+  } else if (s.k <= 8) {
+    auto kernel = combine_kernel<8, 2>;
+    kernel<<<grid_for(kernel, s.N), kThreads, 0, stream>>>(x, gates, pair_slot, o, s.N, s.k,
+                                                            s.rows, vecs);
+  } else {
+    auto kernel = combine_kernel<16, 1>;
+    kernel<<<grid_for(kernel, s.N), kThreads, 0, stream>>>(x, gates, pair_slot, o, s.N, s.k,
+                                                            s.rows, vecs);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

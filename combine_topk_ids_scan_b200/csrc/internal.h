@@ -1,0 +1,55 @@
+// internal.h -- host-side interface between the C-ABI layer and the kernel
+// launchers of libmoedc.  Not installed; the public interface is moe_dc.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_dc.h"
+
+namespace moe {
+
+// Problem sizes after host validation.
+struct Shape {
+  int32_t N, H, E, k, S, Ce;
+  int64_t C;     // packed recv_capacity (0 in capacity mode)
+  int64_t rows;  // rows of the dispatch output
+  int64_t P;     // N * k pairs
+  uint32_t flags;
+};
+
+// Layout workspace: control words, per-expert totals, scan tile states.
+struct LayoutWorkspace {
+  uint32_t *ctrl;    // [0] tile ticket, [1] emit blocks done, [2] status bits
+  int32_t *totals;   // [E] routed pairs per expert (written by the last tile)
+  uint64_t *tiles;   // [T * E] scan tile states (flag << 32 | value)
+  int32_t num_tiles; // T
+};
+
+int32_t layout_num_tiles(int64_t P);
+size_t layout_workspace_bytes(const Shape &s);
+LayoutWorkspace layout_workspace_view(const Shape &s, void *workspace);
+
+cudaError_t launch_layout(const Shape &s, const int32_t *ids, int32_t *expert_counts,
+                          int32_t *expert_offsets, uint32_t *meta, int32_t *row_src,
+                          int32_t *pair_slot, uint8_t *drop_mask, uint32_t *status,
+                          const LayoutWorkspace &ws, cudaStream_t stream);
+
+cudaError_t launch_permute_bf16(const Shape &s, const void *hidden, const int32_t *row_src,
+                                const int32_t *pair_slot, void *out, cudaStream_t stream);
+
+cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t *row_src,
+                               const int32_t *pair_slot, uint8_t *q, float *scales,
+                               cudaStream_t stream);
+
+cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32_t *row_src,
+                                 const int32_t *pair_slot, const float *global_scale,
+                                 uint8_t *q, uint8_t *scales, cudaStream_t stream);
+
+cudaError_t launch_combine(const Shape &s, const void *expert_out, const float *gates,
+                           const int32_t *pair_slot, void *out, cudaStream_t stream);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace moe

@@ -1,0 +1,228 @@
+/*
+ * moe_dc.h -- C ABI of libmoedc.so: the single-GPU core of Mixture-of-Experts
+ * token dispatch and combine on NVIDIA B200 (sm_100a).
+ *
+ * Five calls follow one another on one CUDA stream:
+ *
+ *   moe_dispatch_layout      topk_ids [N,k] -> per-expert counts and start
+ *                            rows, the [4,S] counts/displacements table, the
+ *                            source-row map row_src and the per-pair rows
+ *                            pair_slot
+ *   moe_permute              hidden_states [N,H] bf16 -> [rows,H] bf16,
+ *                            expert-major, zero padding rows
+ *   moe_permute_quant_fp8    same rows, E4M3 codes + one fp32 scale per 1x128
+ *   moe_permute_quant_nvfp4  same rows, E2M1 codes (2 per byte) + one E4M3
+ *                            scale per 16 elements + caller's global scale
+ *   moe_combine              expert outputs [rows,H] bf16 + gates [N,k] fp32
+ *                            -> [N,H] bf16, fp32 weighted sum in fixed k order
+ *
+ * Notation: N tokens, H hidden size, E experts, k = top_k choices per token,
+ * S destination segments of L = E/S consecutive experts, P = N*k pairs; pair
+ * p = t*k + j routes token t to expert topk_ids[p].  rows = recv_capacity in
+ * packed mode, E*expert_capacity in capacity mode (moe_output_rows()).
+ *
+ * Conventions for every call:
+ *   - Pointers named *_ids, *_states, out*, scales*, gates, pair_slot,
+ *     row_src, expert_*, meta, status and workspace are DEVICE pointers
+ *     owned by the caller; the library allocates no memory.  moe_problem is
+ *     a HOST pointer, read during the call only.
+ *   - bf16 data is passed as void* to 16-byte-aligned buffers of IEEE
+ *     bfloat16 (the layout of __nv_bfloat16), row-major with no padding.
+ *   - Every call only enqueues kernels on `stream` (a cudaStream_t) and
+ *     returns; nothing synchronises with the host.
+ *   - A moe_status return reports argument errors found on the host before
+ *     anything is launched (nothing is launched then) and launch errors
+ *     (MOE_ERR_CUDA).  Data-dependent conditions found on the device are
+ *     reported in the `status` word of moe_dispatch_layout (MOE_STATUS_*).
+ *   - Results are deterministic: identical for identical inputs, whatever
+ *     the grid size or scheduling.
+ */
+#ifndef MOE_DC_H
+#define MOE_DC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported entry points keep default visibility even when the library is
+ * built with hidden visibility. */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers (same type). */
+typedef struct CUstream_st *moe_stream_t;
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,       /* null pointer, negative size, misaligned */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2, /* a size outside the supported limits     */
+  MOE_ERR_CUDA = 3               /* a CUDA launch or runtime error          */
+} moe_status;
+
+/* Bits of the device status word written by moe_dispatch_layout. */
+enum {
+  MOE_STATUS_ID_RANGE = 1u, /* an id outside [-1, E): treated as masked     */
+  MOE_STATUS_DUP_ID = 2u,   /* a token names one expert twice (checked only
+                               with MOE_FLAG_CHECK_DUPLICATES)             */
+  MOE_STATUS_CAPACITY = 4u, /* packed mode: more routed pairs than
+                               recv_capacity; the excess pairs get no row  */
+  MOE_STATUS_TIMEOUT = 8u   /* a bounded wait of the scan gave up (about one
+                               second); counts and rows are then invalid   */
+};
+
+/* Problem flags. */
+enum {
+  MOE_FLAG_CHECK_DUPLICATES = 1u,
+  /* Test hook: the first scan tile never publishes its counts, so every
+   * later tile's bounded wait runs out and MOE_STATUS_TIMEOUT is reported.
+   * Results are invalid; used only to test the timeout path. */
+  MOE_FLAG_TEST_STALL_SCAN = 0x80000000u
+};
+
+/* Supported limits (MOE_ERR_UNSUPPORTED_SHAPE beyond them). */
+#define MOE_MAX_EXPERTS 2048
+#define MOE_MAX_TOPK 16
+
+typedef struct moe_problem {
+  int32_t num_tokens;      /* N >= 0                                       */
+  int32_t hidden;          /* H > 0; H % 8 == 0 (bf16 permute, combine),
+                              H % 128 == 0 (FP8), H % 32 == 0 (NVFP4)      */
+  int32_t num_experts;     /* E, 1..MOE_MAX_EXPERTS                        */
+  int32_t top_k;           /* k, 1..MOE_MAX_TOPK                           */
+  int32_t num_segments;    /* S >= 1 with E % S == 0                       */
+  int32_t expert_capacity; /* Ce: 0 = packed dropless layout with
+                              recv_capacity rows; > 0 = capacity layout
+                              [E, Ce] rows, overflow dropped               */
+  int64_t recv_capacity;   /* C rows of the packed layout (ignored when
+                              Ce > 0)                                      */
+  uint32_t flags;          /* MOE_FLAG_*                                   */
+  uint32_t reserved;       /* must be 0                                    */
+} moe_problem;
+
+/* Rows of the dispatch output: recv_capacity, or E * expert_capacity.
+ * Returns -1 for an invalid problem. */
+MOE_API int64_t moe_output_rows(const moe_problem *problem);
+
+/* Bytes of device workspace moe_dispatch_layout needs for this problem
+ * (control counters, per-expert totals, scan tile states).  The workspace
+ * must be zero-filled once before its first use (e.g. cudaMemset); every
+ * completed layout call returns its counters and tile states to zero (the
+ * totals are scratch that each call overwrites), so a workspace sized for
+ * the largest problem can serve any later call on the same stream.  Calls
+ * sharing one workspace must not overlap on the GPU.  Returns 0 for an
+ * invalid problem. */
+MOE_API size_t moe_workspace_bytes(const moe_problem *problem);
+
+/* Dispatch layout: a stable counting sort of the pairs by expert.
+ *
+ * Defines (NKI "Permute A2AV Kernel API Reference", permute_a2av):
+ * packed_source_indices (here row_src) lists source tokens in
+ * destination-major order; send_counts / displacements form a [4, EP]
+ * uint32 table "all measured in elements"; recv_capacity is the static row
+ * count of the packed buffer, padded with zeros.  Id -1 means masked (NeMo
+ * AutoModel token_dispatcher, _indices_to_multihot).  Tokens per expert:
+ * NeMo get_number_of_tokens_per_expert.  Capacity layout: DeepSpeed capacity
+ * dispatch ([e, c, m] expert-slot buffer) with NeMo's expert capacity.
+ *
+ * Inputs:
+ *   topk_ids       int32 [N, k] row-major.  Entries in [0, E) route a pair,
+ *                  -1 masks it; anything else sets MOE_STATUS_ID_RANGE and
+ *                  is treated as masked.
+ * Outputs (all fully overwritten):
+ *   expert_counts  int32 [E]: routed pairs per expert (packed: the true
+ *                  count, even past recv_capacity; capacity: min(count, Ce)).
+ *   expert_offsets int32 [E+1]: first row of each expert (packed: exclusive
+ *                  cumulative sum of expert_counts, [E] = total; capacity:
+ *                  e*Ce).
+ *   meta           uint32 [4, S] row-major, in elements (rows * H): row 0
+ *                  send counts per segment, row 1 send displacements
+ *                  (packed: exclusive cumulative sum of row 0; capacity:
+ *                  s*L*Ce*H), rows 2-3 the receive counts / displacements,
+ *                  equal to rows 0-1 on one GPU.
+ *   row_src        int32 [rows]: source token of each row, -1 for padding.
+ *                  Within an expert rows follow ascending pair index t*k+j.
+ *   pair_slot      int32 [N, k]: row of each pair, -1 when the pair is
+ *                  masked, out of range, dropped (capacity mode) or beyond
+ *                  recv_capacity (packed mode).
+ *   drop_mask      uint8 [N, k] or NULL: 1 for a pair with a valid id that
+ *                  got no row, else 0.
+ *   status         uint32 device word, overwritten with this call's
+ *                  MOE_STATUS_* bits when the call's kernels complete.
+ *   workspace      moe_workspace_bytes() bytes, see there.
+ * Host checks: sizes within limits, E % S == 0, rows*H and N*k*H fit in
+ * uint32 (the metadata is uint32 elements), required pointers non-null. */
+MOE_API moe_status moe_dispatch_layout(const moe_problem *problem, const int32_t *topk_ids,
+                               int32_t *expert_counts, int32_t *expert_offsets,
+                               uint32_t *meta, int32_t *row_src, int32_t *pair_slot,
+                               uint8_t *drop_mask, uint32_t *status, void *workspace,
+                               moe_stream_t stream);
+
+/* Permute, bf16 payload: out[r, :] = hidden_states[row_src[r], :], or zeros
+ * when row_src[r] == -1.  NKI permute_a2av return value ([C, H] packed rows
+ * followed by deterministic zero padding); Mojo MAX ep_comm BF16TokenFormat.
+ *   hidden_states  bf16 [N, H], 16-byte aligned
+ *   row_src        int32 [rows] and pair_slot int32 [N, k] from the layout
+ *   out            bf16 [rows, H], 16-byte aligned, fully overwritten
+ * Requires H % 8 == 0.  Each token row is read from HBM once and written to
+ * its k rows; pair_slot entries outside [0, rows) are skipped. */
+MOE_API moe_status moe_permute(const moe_problem *problem, const void *hidden_states,
+                       const int32_t *row_src, const int32_t *pair_slot, void *out,
+                       moe_stream_t stream);
+
+/* Permute with block FP8 quantisation (Mojo MAX ep_comm
+ * BlockwiseFP8TokenFormat).  For each output row and each 1x128 block:
+ * amax = max |x|; scale = amax / 448 (fp32, round to nearest); code =
+ * E4M3(x / scale) rounded to nearest even with saturation to +-448; a block
+ * with amax == 0 gets scale 0 and codes 0.  Padding rows: codes 0, scales 0.
+ *   out_e4m3  uint8 [rows, H] (16-byte aligned), scales fp32 [rows, H/128]
+ * Requires H % 128 == 0. */
+MOE_API moe_status moe_permute_quant_fp8(const moe_problem *problem, const void *hidden_states,
+                                 const int32_t *row_src, const int32_t *pair_slot,
+                                 uint8_t *out_e4m3, float *scales, moe_stream_t stream);
+
+/* Permute with NVFP4 quantisation (Mojo MAX ep_comm NVBlockScaledTokenFormat
+ * and Struct_ep_dispatch_async_block_scaled_nv: the global input scale is an
+ * input).  global_scale is a device fp32 scalar gs (the decode global scale,
+ * positive and finite).  Per 16-element block: amax; scale code sq =
+ * E4M3((amax / 6) / gs); d = float(sq) * gs; code_i = E2M1(x_i / d) rounded
+ * to nearest even with saturation to +-6, or 0 when d == 0.  Element 2m is
+ * the low nibble of byte m.  Padding rows are all zero.
+ *   out_e2m1     uint8 [rows, H/2] (16-byte aligned)
+ *   scales_e4m3  uint8 [rows, H/16] (2-byte aligned), linear row-major
+ * Requires H % 32 == 0. */
+MOE_API moe_status moe_permute_quant_nvfp4(const moe_problem *problem, const void *hidden_states,
+                                   const int32_t *row_src, const int32_t *pair_slot,
+                                   const float *global_scale, uint8_t *out_e2m1,
+                                   uint8_t *scales_e4m3, moe_stream_t stream);
+
+/* Combine (DeepSpeed: gather each token's expert results back and weight
+ * them by the gate values; NeMo moe_router_dtype 'fp32'; Mojo MAX ep_comm
+ * router_weights_wrapper_type: one fp32 weight per (token, k)).
+ *   expert_out  bf16 [rows, H], 16-byte aligned
+ *   gates       fp32 [N, k]
+ *   pair_slot   int32 [N, k] from the layout
+ *   out         bf16 [N, H], 16-byte aligned, fully overwritten
+ * out[t,:] = bf16_rne(acc) with acc = +0 then acc = fmaf(gates[t,j],
+ * expert_out[pair_slot[t,j],:], acc) for j = 0..k-1 in order, skipping
+ * pairs whose slot is outside [0, rows).  No renormalisation after drops.
+ * Requires H % 8 == 0. */
+MOE_API moe_status moe_combine(const moe_problem *problem, const void *expert_out,
+                       const float *gates, const int32_t *pair_slot, void *out,
+                       moe_stream_t stream);
+
+/* Static description of a moe_status value. */
+MOE_API const char *moe_status_string(moe_status status);
+
+/* Library version string. */
+MOE_API const char *moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_DC_H */

@@ -1,0 +1,109 @@
+"""CPU-side checks of the C ABI: the library builds for sm_100a, loads,
+exports every entry point include/moe_dc.h declares, and its host-side logic
+(sizes, workspace, argument validation) behaves -- without launching anything."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from combine_topk_ids_scan_b200 import binding as B
+from combine_topk_ids_scan_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return B.load()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(moe_\w+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = declared_functions()
+    assert declared == set(B.EXPORTED)
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (moe_\w+)", out))
+    assert declared <= exported, declared - exported
+    # nothing else leaks out under the moe_ prefix
+    assert exported == declared
+
+
+def test_built_for_sm100a(lib):
+    out = subprocess.run(["cuobjdump", "--list-elf", B.LIB_PATH], capture_output=True,
+                         text=True)
+    if out.returncode == 0:
+        assert "sm_100a" in out.stdout
+
+
+def test_host_only_entry_points(lib):
+    assert B.version().startswith("moedc")
+    assert "invalid" in B.status_string(B.MOE_ERR_INVALID_ARG)
+    p = B.Problem(num_tokens=8192, hidden=7168, num_experts=256, top_k=8, num_segments=8,
+                  recv_capacity=65536)
+    assert B.moe_output_rows(p) == 65536
+    # control (256 B) + totals (1 KiB) + 16 tiles x 256 experts x 8 B
+    assert B.moe_workspace_bytes(p) == 256 + 1024 + 16 * 256 * 8
+    p.expert_capacity = 5
+    assert B.moe_output_rows(p) == 1280
+    p.num_segments = 3
+    assert B.moe_output_rows(p) == -1 and B.moe_workspace_bytes(p) == 0
+
+
+def _call(lib, fn, prob, nptr):
+    c = prob.c()
+    return getattr(lib, fn)(ctypes.byref(c), *([None] * nptr))
+
+
+@pytest.mark.parametrize("mutate,code", [
+    (dict(num_segments=3), B.MOE_ERR_UNSUPPORTED_SHAPE),        # E % S != 0
+    (dict(num_experts=4096, num_segments=1), B.MOE_ERR_UNSUPPORTED_SHAPE),
+    (dict(top_k=17), B.MOE_ERR_UNSUPPORTED_SHAPE),
+    (dict(num_tokens=-1), B.MOE_ERR_INVALID_ARG),
+    (dict(hidden=0), B.MOE_ERR_INVALID_ARG),
+    (dict(recv_capacity=1 << 40), B.MOE_ERR_UNSUPPORTED_SHAPE),  # int32 rows
+    (dict(hidden=1 << 20, recv_capacity=1 << 13), B.MOE_ERR_UNSUPPORTED_SHAPE),  # uint32 meta
+    ({}, B.MOE_ERR_INVALID_ARG),                                  # null pointers
+])
+def test_layout_validation(lib, mutate, code):
+    p = B.Problem(num_tokens=100, hidden=64, num_experts=8, top_k=2, num_segments=2,
+                  recv_capacity=200)
+    for k, v in mutate.items():
+        setattr(p, k, v)
+    assert _call(lib, "moe_dispatch_layout", p, 10) == code
+
+
+def test_payload_shape_rules(lib):
+    p = B.Problem(num_tokens=10, hidden=100, num_experts=8, top_k=2, num_segments=2,
+                  recv_capacity=20)
+    assert _call(lib, "moe_permute", p, 5) == B.MOE_ERR_UNSUPPORTED_SHAPE       # H % 8
+    assert _call(lib, "moe_combine", p, 5) == B.MOE_ERR_UNSUPPORTED_SHAPE
+    p.hidden = 96
+    assert _call(lib, "moe_permute_quant_fp8", p, 6) == B.MOE_ERR_UNSUPPORTED_SHAPE  # H % 128
+    p.hidden = 80
+    assert _call(lib, "moe_permute_quant_nvfp4", p, 7) == B.MOE_ERR_UNSUPPORTED_SHAPE  # H % 32
+    p.hidden = 128
+    for fn, n in (("moe_permute", 5), ("moe_permute_quant_fp8", 6),
+                  ("moe_permute_quant_nvfp4", 7), ("moe_combine", 5)):
+        assert _call(lib, fn, p, n) == B.MOE_ERR_INVALID_ARG, fn      # null pointers
+    assert lib.moe_permute(None, *([None] * 5)) == B.MOE_ERR_INVALID_ARG
+    bad = B.moe_problem(10, 128, 8, 2, 2, 0, 20, 0, 7)                   # reserved != 0
+    assert lib.moe_combine(ctypes.byref(bad), *([None] * 5)) == B.MOE_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(B, "_lib", None)
+    with pytest.raises(RuntimeError, match="not found"):
+        B.load(str(tmp_path / "nope.so"))

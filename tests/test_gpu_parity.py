@@ -1,0 +1,259 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Integer, index and byte outputs must match bit for bit; the combine is
+computed with the same fp32 fused multiply-adds in the same order, so it must
+match bit for bit as well (which is inside the 1-bf16-ulp contract; the
+contract bound itself is checked separately against a float64 sum).
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from combine_topk_ids_scan_b200 import binding as B
+from combine_topk_ids_scan_b200.inputs import Workload, make_workload, normal_bf16, softmax_gates
+from gpu_util import GpuRun, bf16_np, problem_of, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from combine_topk_ids_scan_b200 import build
+    build.build()
+    B.load()
+
+
+def custom(N, H, E, k, S, C=None, Ce=0, ids=None, seed=0, p_mask=0.0, p_bad=0.0,
+           distinct=True, with_out=True):
+    ss = np.random.SeedSequence(seed)
+    s_ids, s_g, s_h, s_o = ss.spawn(4)
+    rng = np.random.Generator(np.random.PCG64(s_ids))
+    if ids is None:
+        if distinct and k <= E:
+            ids = np.argsort(rng.random((N, E)), axis=1)[:, :k].astype(np.int32)
+        else:
+            ids = rng.integers(0, E, size=(N, k)).astype(np.int32)
+        m = rng.random((N, k))
+        ids[m < p_mask] = -1
+        bad = rng.random((N, k)) < p_bad
+        ids[bad] = rng.choice([-7, E, E + 3, -2], size=int(bad.sum()))
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    if C is None:
+        C = N * k
+    rows = E * Ce if Ce > 0 else C
+    hidden = normal_bf16(s_h, N, H) if N > 0 else np.zeros((0, H), np.uint16)
+    hv = (hidden.astype(np.uint32) << 16).view(np.float32)
+    amax = float(np.abs(hv).max()) if hv.size else 0.0
+    gs = float(np.float32(amax) / np.float32(2688.0)) if amax > 0 else 1.0
+    gates = softmax_gates(np.random.Generator(np.random.PCG64(s_g)), N, k)
+    X = normal_bf16(s_o, rows, H) if with_out else None
+    return Workload(name="custom", N=N, H=H, E=E, k=k, S=S,
+                    recv_capacity=0 if Ce > 0 else C, expert_capacity=Ce, ids=ids,
+                    gates=gates, hidden=hidden, expert_out=X, global_scale=gs, seed=seed)
+
+
+def oracle_layout(orc, w, flags=0):
+    return orc.layout(w.ids, w.E, w.S, w.H, recv_capacity=w.recv_capacity,
+                      expert_capacity=w.expert_capacity, flags=flags)
+
+
+def assert_layout(run, ref):
+    assert run.status == ref.status, (hex(run.status), hex(ref.status))
+    for key in ("expert_counts", "expert_offsets", "meta", "row_src", "pair_slot", "drop_mask"):
+        got, want = getattr(run, key), getattr(ref, key)
+        assert np.array_equal(np.asarray(got).reshape(-1).astype(np.int64),
+                              np.asarray(want).reshape(-1).astype(np.int64)), key
+
+
+def assert_all_outputs(orc, w, run, ref, rows_sample=None, tokens_sample=None):
+    """Compare payloads and combine; full, or on sampled rows / tokens."""
+    row_src = ref.row_src
+    idx = np.arange(row_src.size) if rows_sample is None else rows_sample
+    want = orc.permute_bf16(w.hidden, row_src[idx])
+    assert np.array_equal(run.out[idx], want), "bf16 permute"
+    if run.has_fp8:
+        q, s = orc.permute_fp8(w.hidden, row_src[idx])
+        assert np.array_equal(run.q8[idx], q), "fp8 codes"
+        assert np.array_equal(run.s8[idx].view(np.uint32), s.view(np.uint32)), "fp8 scales"
+    if run.has_fp4:
+        q, s = orc.permute_nvfp4(w.hidden, row_src[idx], w.global_scale)
+        assert np.array_equal(run.q4[idx], q), "nvfp4 codes"
+        assert np.array_equal(run.s4[idx], s), "nvfp4 scales"
+    if run.y is not None:
+        tok = np.arange(w.N) if tokens_sample is None else tokens_sample
+        y = orc.combine(w.expert_out, w.gates[tok], ref.pair_slot[tok])
+        assert np.array_equal(run.y[tok], y), "combine"
+
+
+# ------------------------------------------------------------ the workloads
+@pytest.mark.parametrize("cfg", ["tiny", "mid_zipf", "decode_capacity"])
+def test_workload_full_parity(orc, cfg):
+    w = make_workload(cfg)
+    run = GpuRun(w)
+    ref = oracle_layout(orc, w)
+    assert_layout(run, ref)
+    assert_all_outputs(orc, w, run, ref)
+
+
+@pytest.mark.parametrize("cfg", ["fp8_metric", "nvfp4_hot", "balanced_static"])
+def test_full_size_workload_sampled_parity(orc, cfg):
+    """Full sizes, the launch configuration the benchmark times; layout and
+    bf16 rows compared in full, quantised rows and combined tokens sampled."""
+    w = make_workload(cfg)
+    run = GpuRun(w)
+    ref = oracle_layout(orc, w)
+    assert_layout(run, ref)
+    assert np.array_equal(run.out, orc.permute_bf16(w.hidden, ref.row_src)), "bf16 permute"
+    rng = np.random.default_rng(11)
+    rows = np.unique(np.concatenate([rng.choice(ref.row_src.size, 3000, replace=False),
+                                     [0, ref.row_src.size - 1]]))
+    toks = np.unique(np.concatenate([rng.choice(w.N, 1500, replace=False), [0, w.N - 1]]))
+    assert_all_outputs(orc, w, run, ref, rows_sample=rows, tokens_sample=toks)
+
+
+def test_identity_expert_round_trip_gpu(orc):
+    w = make_workload("tiny")
+    run = GpuRun(w, quant=False, combine=False)
+    prob = problem_of(w)
+    gates = torch.from_numpy(w.gates).cuda()
+    y = torch.empty((w.N, w.H), dtype=torch.bfloat16, device="cuda")
+    B.moe_combine(prob, run.buf.out, gates, run.buf.pair_slot, y)
+    assert np.array_equal(bf16_np(y), w.hidden)
+
+
+def test_combine_within_contract_of_exact_sum(orc):
+    """The spec contract: <= 1 bf16 ulp of the exact weighted sum (plus
+    the fp32 accumulation error bound)."""
+    w = make_workload("mid_zipf", n_tokens=512)
+    run = GpuRun(w, quant=False)
+    xf = (w.expert_out.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    exact = np.zeros((w.N, w.H))
+    mag = np.zeros((w.N, w.H))
+    for j in range(w.k):
+        s = run.pair_slot[:, j]
+        term = w.gates[:, j:j + 1].astype(np.float64) * xf[s]
+        exact += term
+        mag += np.abs(term)
+    got = (run.y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact), 2.0**-126))) - 7)
+    assert np.all(np.abs(got - exact) <= ulp + w.k * 2.0**-23 * mag)
+
+
+# ------------------------------------------------------------ edge cases
+EDGE = {
+    "ragged_masked_badids": dict(N=3001, H=384, E=40, k=3, S=5, p_mask=0.1, p_bad=0.02),
+    "packed_overflow": dict(N=700, H=256, E=16, k=4, S=4, C=1900),
+    "padding_large": dict(N=300, H=128, E=8, k=2, S=2, C=1500, p_mask=0.3),
+    "all_masked": dict(N=64, H=128, E=4, k=2, S=1, C=40, p_mask=1.1),
+    "k1": dict(N=5000, H=96, E=7, k=1, S=7),
+    "k16": dict(N=1300, H=256, E=64, k=16, S=16),
+    "E1": dict(N=999, H=64, E=1, k=1, S=1),
+    "E2048_S2048": dict(N=2048, H=32, E=2048, k=8, S=2048),
+    "duplicates": dict(N=1000, H=128, E=6, k=4, S=3, distinct=False),
+    "capacity_drops": dict(N=900, H=256, E=32, k=4, S=8, Ce=3),
+    "capacity_masked": dict(N=333, H=160, E=12, k=3, S=4, Ce=40, p_mask=0.2, p_bad=0.01),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_edge_case_parity(orc, name):
+    spec = dict(EDGE[name])
+    w = custom(seed=zlib.crc32(name.encode()) % 1000, **spec)
+    flags = B.MOE_FLAG_CHECK_DUPLICATES
+    run = GpuRun(w, flags=flags)
+    ref = oracle_layout(orc, w, flags=orc.FLAG_CHECK_DUPLICATES)
+    assert_layout(run, ref)
+    assert_all_outputs(orc, w, run, ref)
+
+
+def test_empty_problem(orc):
+    w = custom(N=0, H=128, E=8, k=2, S=2, C=16)
+    run = GpuRun(w)
+    ref = oracle_layout(orc, w)
+    assert_layout(run, ref)
+    assert np.all(run.out == 0) and np.all(run.q8 == 0) and np.all(run.s4 == 0)
+
+
+def test_many_tiles_multi_wave_scan(orc):
+    """4M pairs = 1024 scan tiles, more than one wave of CTAs: the look-back
+    chain crosses waves."""
+    N, k, E = 262144, 16, 64
+    rng = np.random.default_rng(5)
+    ids = rng.integers(0, E, size=(N, k)).astype(np.int32)
+    w = custom(N=N, H=8, E=E, k=k, S=4, ids=ids, with_out=False)
+    run = GpuRun(w, quant=False, combine=False)
+    ref = oracle_layout(orc, w)
+    assert_layout(run, ref)
+
+
+def test_workspace_reuse_across_problems(orc):
+    """The layout leaves its workspace zeroed, so one buffer serves a
+    sequence of different problems."""
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    for i, spec in enumerate([dict(N=5000, H=64, E=32, k=4, S=4),
+                              dict(N=700, H=64, E=256, k=8, S=8),
+                              dict(N=9000, H=64, E=5, k=2, S=5, p_mask=0.2)]):
+        w = custom(seed=100 + i, with_out=False, **spec)
+        prob = problem_of(w)
+        assert B.moe_workspace_bytes(prob) <= ws.numel()
+        buf = B.Buffers(prob, quant=False)
+        buf.workspace = ws
+        for _ in range(2):
+            B.layout(prob, torch.from_numpy(w.ids).cuda(), buf)
+            torch.cuda.synchronize()
+            ref = oracle_layout(orc, w)
+            assert np.array_equal(buf.pair_slot.cpu().numpy()[:w.N], ref.pair_slot)
+            assert np.array_equal(buf.row_src.cpu().numpy()[:buf.rows], ref.row_src)
+        # control words and scan tile states are back at zero (the per-expert
+        # totals in between are scratch that is always overwritten)
+        tiles_at = 256 + (w.E * 4 + 255) // 256 * 256
+        assert int(ws[:256].count_nonzero()) == 0
+        assert int(ws[tiles_at:].count_nonzero()) == 0
+
+
+def test_scan_wait_times_out_with_status(orc):
+    """The test hook withholds the first tile's counts: every later tile's
+    bounded wait runs out (about a second), the kernels finish, the status
+    word reports MOE_STATUS_TIMEOUT and the device stays usable."""
+    w = custom(N=3000, H=64, E=16, k=4, S=4, with_out=False)   # 12000 pairs, 3 tiles
+    run = GpuRun(w, flags=B.MOE_FLAG_TEST_STALL_SCAN, quant=False, combine=False)
+    assert run.status & B.MOE_STATUS_TIMEOUT
+    # the context is intact and the workspace was cleaned: a normal call works
+    run = GpuRun(w, quant=False, combine=False)
+    ref = oracle_layout(orc, w)
+    assert_layout(run, ref)
+
+
+def test_deterministic_repeat(orc):
+    w = make_workload("mid_zipf")
+    a = GpuRun(w)
+    b = GpuRun(w)
+    for key in ("pair_slot", "row_src", "out", "q8", "s8", "q4", "s4", "y"):
+        assert np.array_equal(getattr(a, key), getattr(b, key)), key
+
+
+# ------------------------------------------------------------ host checks
+def test_host_argument_errors():
+    prob = B.Problem(num_tokens=16, hidden=100, num_experts=8, top_k=2, num_segments=2,
+                     recv_capacity=32)
+    x = torch.zeros((16, 100), dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros((32, 100), dtype=torch.bfloat16, device="cuda")
+    rs = torch.zeros(32, dtype=torch.int32, device="cuda")
+    ps = torch.zeros((16, 2), dtype=torch.int32, device="cuda")
+    with pytest.raises(B.MoeError) as e:
+        B.moe_permute(prob, x, rs, ps, out)          # H % 8 != 0
+    assert e.value.code == B.MOE_ERR_UNSUPPORTED_SHAPE
+    prob.hidden = 96
+    x2 = torch.zeros(16 * 96 + 8, dtype=torch.bfloat16, device="cuda")[1:].view(-1)[:16 * 96]
+    with pytest.raises(B.MoeError) as e:
+        B.moe_permute(prob, x2, rs, ps, out)         # misaligned hidden
+    assert e.value.code == B.MOE_ERR_INVALID_ARG
+    prob.num_segments = 3                            # E % S != 0
+    buf_ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    with pytest.raises(B.MoeError) as e:
+        B.moe_dispatch_layout(prob, ps, rs, rs, rs, rs, ps, None, rs, buf_ws)
+    assert e.value.code == B.MOE_ERR_UNSUPPORTED_SHAPE
