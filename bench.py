@@ -14,8 +14,9 @@ distinct routing, 1% outlier rows, expert outputs ~N(0,1)).
 Each rank runs its own batch (replicas; weak scaling, no data-path
 collective); the timed region is bracketed by a barrier and device
 synchronisation, every step is timed with CUDA events on the launching stream,
-and the max over ranks is reported.  L2 is flushed (a write of twice its
-size) before every step, outside the events.  Rank 0 prints one JSON line.
+and the max over ranks is reported.  L2 is flushed before every step (a write
+of a buffer twice its size, then a read of another such buffer so the dirty
+lines are retired there), outside the events.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -142,6 +143,24 @@ def dist_env():
     return rank, world, local
 
 
+def seed_for_rank(rank: int) -> int | None:
+    """Rank 0 runs the canonical seeded batch; every other rank draws its own
+    independent batch of the same shape (weak scaling over replicas)."""
+    return None if rank == 0 else 1002 + 7919 * rank
+
+
+def max_over_ranks(values, device, world: int):
+    """Element-wise max of a list of floats over all ranks (a timing
+    reduction only; the data path has no collective)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 # ------------------------------------------------------------------ oracle
 def oracle_tokens_per_s(w, n_tokens: int, start: int = 0) -> tuple[float, float]:
     """Time the CPU oracle (as it stands, single thread) on the sub-batch of
@@ -205,7 +224,8 @@ def workload_config(w) -> dict:
             "N": w.N, "H": w.H, "E": w.E, "top_k": w.k, "segments": w.S,
             "recv_capacity": w.recv_capacity,
             "step": "layout + permute(bf16) + permute(fp8 1x128) + permute(nvfp4) + combine",
-            "l2": "flushed before every step (write of 2x L2 size), outside the timed events",
+            "l2": "flushed before every step (write of a 2x-L2 buffer, then a read of another "
+                  "2x-L2 buffer to retire the dirty lines), outside the timed events",
             "parallelism": "replicas (independent token batches per GPU)"}
 
 
@@ -229,7 +249,7 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
             dist.barrier()
 
     B.load()
-    w = make_workload(WORKLOAD, seed=None if rank == 0 else 1002 + 7919 * rank)
+    w = make_workload(WORKLOAD, seed=seed_for_rank(rank))
     prob = B.Problem(num_tokens=w.N, hidden=w.H, num_experts=w.E, top_k=w.k,
                      num_segments=w.S, recv_capacity=w.recv_capacity,
                      expert_capacity=w.expert_capacity)
@@ -251,7 +271,15 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
     h_y = torch.empty((w.N, w.H), dtype=torch.int16).pin_memory()
     h_status = torch.empty(1 + w.E, dtype=torch.int32).pin_memory()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8,
+                          device=dev)
+    flush_r = torch.zeros(max(2 * l2, 256 << 20) // 4, dtype=torch.int32, device=dev)
+
+    def flush_l2():
+        # write a buffer twice the L2 size, then read another one so the
+        # dirty lines are written back here, outside the timed events
+        flush_w.zero_()
+        flush_r.max()
 
     def step(ev=None):
         if ev is not None:
@@ -276,7 +304,7 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
 
     launches_per_step = (2 if w.P > 0 else 1) + 4
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         step()
     torch.cuda.synchronize(dev)
     st = int(buf.status.cpu().numpy().view(np.uint32)[0])
@@ -296,7 +324,7 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
     barrier()
     torch.cuda.synchronize(dev)
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2()
         step(evs[i])
     torch.cuda.synchronize(dev)
     barrier()
@@ -336,12 +364,9 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
     e2e_ms = e_start.elapsed_time(e_end) / e2e_steps
 
     # ---- max over ranks
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms] + [phase_ms[p] for p in phases], device=dev,
-                         dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
-        phase_ms = {p: float(t[2 + i]) for i, p in enumerate(phases)}
+    t = max_over_ranks([ms, e2e_ms] + [phase_ms[p] for p in phases], dev, world)
+    ms, e2e_ms = t[0], t[1]
+    phase_ms = {p: t[2 + i] for i, p in enumerate(phases)}
 
     if rank == 0:
         nbytes = algorithmic_bytes(w, total_rows)

@@ -28,6 +28,7 @@ MOE_STATUS_CAPACITY = 4
 MOE_STATUS_TIMEOUT = 8
 
 MOE_FLAG_CHECK_DUPLICATES = 1
+MOE_FLAG_LAYOUT_TWO_PASS = 2
 MOE_FLAG_TEST_STALL_SCAN = 0x80000000
 
 MOE_MAX_EXPERTS = 2048

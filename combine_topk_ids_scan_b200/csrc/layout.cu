@@ -1,32 +1,40 @@
-// layout.cu -- dispatch layout: stable counting sort of (token, k) pairs by
-// expert, in two kernels.
+// layout.cu -- dispatch layout: a stable counting sort of the (token, k)
+// pairs by expert.
 //
-//  count_scan  One CTA per tile of 4096 consecutive pairs, tiles taken in
-//              launch order from an atomic ticket.  Each warp owns 256
-//              consecutive pairs and walks them in 8 rounds of 32; in a round,
-//              lanes naming the same expert find each other with
-//              __match_any_sync, take their rank from the popcount of lower
-//              peers, and the highest peer bumps the warp's private
-//              shared-memory histogram (so the histogram needs no atomics and
-//              ranks are in pair order).  A scan over the 16 warp histograms
-//              gives each warp its per-expert base inside the tile.  Tiles
-//              then chain their per-expert counts with a single-pass
-//              decoupled look-back (one 64-bit word per (tile, expert): flag
-//              in the high half, count in the low half), giving each tile its
-//              exclusive per-expert prefix.  The result per pair is its rank
-//              among all earlier pairs of the same expert -- stable by
-//              (token, k) by construction.  The last tile stores the totals.
-//  emit        Exclusive scan of the per-expert totals (every CTA, in shared
-//              memory), then per pair: row = expert start + rank (packed), or
-//              e*Ce + rank with rank >= Ce dropped (capacity); writes
-//              pair_slot, row_src, drop_mask, padding rows, counts, offsets,
-//              the [4,S] table, and returns the workspace to zero.
+// Scan tiles.  The pairs are cut into tiles of 4096 consecutive pairs; a CTA
+// takes the next tile from an atomic ticket, so tiles start in order.  Each of
+// its 16 warps owns 256 consecutive pairs and walks them in 8 rounds of 32.
+// In a round the warp aggregates its lanes per expert in shared memory: each
+// lane ORs its bit into the warp's mask word for its expert, reads the mask
+// back (its peers), takes its rank from the popcount of lower peers, and the
+// highest peer adds the group's size to the warp's private histogram and
+// clears the mask (ranks are in pair order; measured on B200 about 4x cheaper
+// per round than __match_any_sync and 2x cheaper than one ballot per id bit).  A scan over the 16 warp histograms gives every
+// warp its per-expert base inside the tile, and the tiles chain their
+// per-expert counts with a single-pass decoupled look-back (one 64-bit word
+// per (tile, expert): flag in the high half, count in the low half; a window
+// of predecessors is read per poll), which gives each tile its exclusive
+// per-expert prefix.  A pair's rank among all earlier pairs of its expert is
+// then prefix + warp base + in-warp rank: stable by (token, k) by
+// construction, and independent of scheduling.
+//
+// Each tile stores its pairs' ranks in pair_slot, and the last tile the
+// per-expert totals.  The emit step then scans the totals into expert start
+// rows (in shared memory, per CTA) and turns ranks into rows: pair_slot,
+// row_src, drop_mask, padding rows, counts and the [4,S] table; the last CTA
+// to finish returns the workspace to zero and publishes the status word.
+// One-launch path: a cooperative grid of up to one CTA per SM; the first T
+// CTAs scan the T tiles, then every CTA waits (bounded) until all tiles are
+// done and runs the emit step over its share of the pairs, so the scattered
+// row_src stores are spread over all SMs.  Two-kernel path (any size): a scan
+// kernel of T CTAs, then an emit kernel.
 //
 // Layout definitions: NKI "Permute A2AV Kernel API Reference" (permute_a2av
 // packed_source_indices, send_counts, recv_capacity, [4, EP] metadata in
 // elements); DeepSpeed capacity dispatch ([e, c, m] buffer); NeMo AutoModel
 // token_dispatcher (-1 ids are masked; tokens per expert).
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "internal.h"
@@ -36,76 +44,128 @@ namespace moe {
 namespace {
 
 constexpr int kScanThreads = 512;
-constexpr int kScanWarps = kScanThreads / kWarp;  // 16
-constexpr int kScanRounds = 8;                     // pairs per lane
+constexpr int kScanWarps = kScanThreads / kWarp;        // 16
+constexpr int kScanRounds = 8;                          // pairs per lane
 constexpr int kTilePairs = kScanThreads * kScanRounds;  // 4096
 constexpr int kWarpPairs = kWarp * kScanRounds;         // 256
 constexpr uint64_t kFlagAggregate = 1ull;
 constexpr uint64_t kFlagInclusive = 2ull;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bounded look-back wait: 1 s
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // every bounded wait: 1 s
+constexpr int kLookWindow = 8;                    // predecessor tiles per poll
+constexpr int kFusedMaxTiles = 128;               // last CTA clears <= 128*E words
 
 constexpr int kEmitThreads = 256;
 
+// control words at the start of the workspace
+enum { kCtrlTicket = 0, kCtrlDone = 1, kCtrlStatus = 2, kCtrlTilesDone = 3 };
+
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// dynamic shared memory of a scan CTA: per-warp counts (u16), per-warp lane
+// masks (u32), tile prefix (u32)
 __host__ __device__ inline size_t scan_smem_bytes(int E) {
-  return align_up((size_t)kScanWarps * E * sizeof(uint16_t), 16) + (size_t)E * sizeof(uint32_t);
+  return align_up((size_t)kScanWarps * E * sizeof(uint16_t), 16) +
+         (size_t)kScanWarps * E * sizeof(uint32_t) + align_up((size_t)E * sizeof(uint32_t), 16);
 }
 
-__global__ void __launch_bounds__(kScanThreads)
-    layout_count_scan_kernel(const int32_t *__restrict__ ids, int64_t P, int32_t E,
-                             int32_t num_tiles, uint32_t flags, uint32_t *ctrl,
-                             int32_t *__restrict__ totals, uint64_t *tiles,
-                             int32_t *__restrict__ pair_rank) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint16_t *wcnt = reinterpret_cast<uint16_t *>(smem);  // [warps][E]
-  uint32_t *tile_prefix =
-      reinterpret_cast<uint32_t *>(smem + align_up((size_t)kScanWarps * E * 2, 16));  // [E]
-  __shared__ int s_tile;
-  __shared__ uint32_t s_status;
+struct ScanSmem {
+  uint16_t *wcnt;        // [warps][E] counts, then warp bases
+  uint32_t *wmask;       // [warps][E] lane masks of the current round
+  uint32_t *tile_prefix; // [E] tile aggregate, then tile exclusive prefix
+};
 
-  const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
-  if (tid == 0) {
-    s_tile = (int)atomicAdd(&ctrl[0], 1u);
-    s_status = 0;
+__device__ __forceinline__ ScanSmem scan_smem(uint8_t *smem, int32_t E) {
+  ScanSmem m;
+  m.wcnt = reinterpret_cast<uint16_t *>(smem);
+  m.wmask = reinterpret_cast<uint32_t *>(smem + align_up((size_t)kScanWarps * E * 2, 16));
+  m.tile_prefix = m.wmask + (size_t)kScanWarps * E;
+  return m;
+}
+
+// Bounded wait helper: true while the deadline (set on first call) has not
+// passed.
+__device__ __forceinline__ bool keep_waiting(uint64_t &deadline) {
+  const uint64_t now = globaltimer_ns();
+  if (deadline == 0) {
+    deadline = now + kWaitLimitNs;
+    return true;
   }
-  for (int i = tid; i < kScanWarps * E; i += kScanThreads) wcnt[i] = 0;
+  return now <= deadline;
+}
+
+// Per-CTA state of one scan tile.  pk[r] packs the lane's r-th pair: expert
+// id in the low 16 bits (0xFFFF: no expert), rank inside the warp's 256 pairs
+// in the high 16 bits.
+struct TileScan {
+  int tile;
+  uint32_t pk[kScanRounds];
+  int64_t base;  // first pair of this warp
+  __device__ __forceinline__ int32_t expert(int r) const {
+    const uint32_t e = pk[r] & 0xFFFFu;
+    return e == 0xFFFFu ? -1 : (int32_t)e;
+  }
+  __device__ __forceinline__ uint32_t rank(int r) const { return pk[r] >> 16; }
+};
+
+// Phases 1-3 of a tile: in-warp ranks, warp bases (left in wcnt), tile
+// exclusive prefix per expert (left in tile_prefix); the last tile also
+// stores the per-expert totals.  Returns false when the ticket is past the
+// last tile (a workspace that was not zero-filled).
+__device__ bool scan_tile(TileScan &ts, const int32_t *__restrict__ ids, int64_t P, int32_t E,
+                          int32_t num_tiles, uint32_t flags, uint32_t *ctrl, uint64_t *tiles,
+                          int32_t *totals, const ScanSmem &sm, int *s_tile, uint32_t *s_status) {
+  const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
+  uint16_t *wcnt = sm.wcnt;
+  uint32_t *tile_prefix = sm.tile_prefix;
+  if (tid == 0) {
+    *s_tile = (int)atomicAdd(&ctrl[kCtrlTicket], 1u);
+    *s_status = 0;
+  }
   __syncthreads();
-  const int tile = s_tile;
-  // a ticket past the last tile only happens with a workspace that was not
-  // zero-filled before first use: do nothing (the other tiles' bounded waits
-  // then report MOE_STATUS_TIMEOUT)
-  if (tile >= num_tiles) return;
+  if (*s_tile >= num_tiles) return false;
+  for (int i = tid; i < kScanWarps * E; i += kScanThreads) {
+    wcnt[i] = 0;
+    sm.wmask[i] = 0;
+  }
+  __syncthreads();
+  ts.tile = *s_tile;
 
   // ---- 1. per-warp stable ranks and histograms
-  const int64_t base = (int64_t)tile * kTilePairs + (int64_t)warp * kWarpPairs;
+  ts.base = (int64_t)ts.tile * kTilePairs + (int64_t)warp * kWarpPairs;
   int32_t ex[kScanRounds];
 #pragma unroll
   for (int r = 0; r < kScanRounds; ++r) {
-    const int64_t p = base + r * kWarp + lane;
+    const int64_t p = ts.base + r * kWarp + lane;
     ex[r] = p < P ? __ldg(ids + p) : -1;
   }
-  uint16_t rank[kScanRounds];
   bool bad_id = false;
   uint16_t *my_cnt = wcnt + (size_t)warp * E;
+  uint32_t *my_mask = sm.wmask + (size_t)warp * E;
 #pragma unroll
   for (int r = 0; r < kScanRounds; ++r) {
     const int32_t e = ex[r];
     const bool valid = (uint32_t)e < (uint32_t)E;
     bad_id |= (!valid && e != -1);
-    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, valid ? (uint32_t)e : 0xFFFFFFFFu);
-    uint32_t before = 0;
-    if (valid) before = my_cnt[e];
+    if (valid) atomicOr(&my_mask[e], 1u << lane);
     __syncwarp();
-    rank[r] = 0;
+    uint32_t peers = 0, before = 0;
     if (valid) {
-      rank[r] = (uint16_t)(before + __popc(peers & lanemask_lt()));
-      if (lane == 31 - __clz(peers)) my_cnt[e] = (uint16_t)(before + __popc(peers));
+      peers = my_mask[e];
+      before = my_cnt[e];
     }
     __syncwarp();
-    ex[r] = valid ? e : -1;
+    uint32_t rank = 0;
+    if (valid) {
+      rank = before + __popc(peers & lanemask_lt());
+      if (lane == 31 - __clz(peers)) {
+        my_cnt[e] = (uint16_t)(before + __popc(peers));
+        my_mask[e] = 0;
+      }
+    }
+    __syncwarp();
+    ts.pk[r] = (rank << 16) | (valid ? (uint32_t)e : 0xFFFFu);
   }
-  if (__any_sync(0xFFFFFFFFu, bad_id) && lane == 0) atomicOr(&s_status, MOE_STATUS_ID_RANGE);
+  if (__any_sync(0xFFFFFFFFu, bad_id) && lane == 0) atomicOr(s_status, MOE_STATUS_ID_RANGE);
   __syncthreads();
 
   // ---- 2. per expert: exclusive scan over the warps, tile aggregate
@@ -121,6 +181,7 @@ __global__ void __launch_bounds__(kScanThreads)
   }
 
   // ---- 3. decoupled look-back across tiles, one chain per expert
+  const int tile = ts.tile;
   const bool withhold = (flags & MOE_FLAG_TEST_STALL_SCAN) && tile == 0;
   bool timed_out = false;
   uint64_t deadline = 0;
@@ -131,57 +192,90 @@ __global__ void __launch_bounds__(kScanThreads)
       if (!withhold) st_relaxed_gpu_u64(&tiles[e], (kFlagInclusive << 32) | agg);
     } else {
       st_relaxed_gpu_u64(&tiles[(size_t)tile * E + e], (kFlagAggregate << 32) | agg);
+      // Read a window of predecessors per poll (independent loads: one L2
+      // round trip), add aggregates in order until an inclusive prefix ends
+      // the chain or an unpublished tile makes us poll again.
       int look = tile - 1;
       while (look >= 0) {
-        const uint64_t v = ld_relaxed_gpu_u64(&tiles[(size_t)look * E + e]);
-        const uint64_t f = v >> 32;
-        if (f == 0) {
-          // predecessor has not published yet: it holds an earlier ticket, so
-          // it is running; wait for it, but never longer than the limit
-          const uint64_t now = globaltimer_ns();
-          if (deadline == 0) {
-            deadline = now + kWaitLimitNs;
-          } else if (now > deadline) {
+        uint64_t v[kLookWindow];
+#pragma unroll
+        for (int i = 0; i < kLookWindow; ++i)
+          v[i] = look - i >= 0 ? ld_relaxed_gpu_u64(&tiles[(size_t)(look - i) * E + e])
+                               : (kFlagInclusive << 32);
+        bool stop = false, done = false;
+        int advanced = 0;
+#pragma unroll
+        for (int i = 0; i < kLookWindow; ++i) {
+          if (!stop) {
+            const uint64_t f = v[i] >> 32;
+            if (f == 0) {
+              stop = true;
+            } else {
+              excl += (uint32_t)v[i];
+              ++advanced;
+              if (f == kFlagInclusive) stop = done = true;
+            }
+          }
+        }
+        if (done) break;
+        look -= advanced;
+        if (advanced < kLookWindow) {
+          // tile `look` has not published: it holds an earlier ticket, so it
+          // is running; wait for it, but never longer than the limit
+          if (!keep_waiting(deadline)) {
             timed_out = true;
             break;
           }
-          __nanosleep(64);
-          continue;
+          __nanosleep(32);
         }
-        excl += (uint32_t)v;
-        if (f == kFlagInclusive) break;
-        --look;
       }
       st_relaxed_gpu_u64(&tiles[(size_t)tile * E + e], (kFlagInclusive << 32) | (excl + agg));
     }
     tile_prefix[e] = excl;
     if (tile == num_tiles - 1) totals[e] = (int32_t)(excl + agg);
   }
-  if (timed_out) atomicOr(&s_status, MOE_STATUS_TIMEOUT);
+  if (timed_out) atomicOr(s_status, MOE_STATUS_TIMEOUT);
   __syncthreads();
-
-  // ---- 4. rank of each pair among all earlier pairs of its expert
-#pragma unroll
-  for (int r = 0; r < kScanRounds; ++r) {
-    const int64_t p = base + r * kWarp + lane;
-    if (p < P) {
-      const int32_t e = ex[r];
-      pair_rank[p] = e >= 0 ? (int32_t)(tile_prefix[e] + my_cnt[e] + rank[r]) : -1;
-    }
-  }
-  if (tid == 0 && s_status) atomicOr(&ctrl[2], s_status);
+  return true;
 }
 
-// Block-wide exclusive scan of n <= 8 * kEmitThreads values in place.
-__device__ void block_exclusive_scan(int32_t *v, int n, int32_t *total_out) {
-  __shared__ int32_t warp_sums[kEmitThreads / kWarp];
-  constexpr int kPer = 8;
+// Rank of the lane's r-th pair among all earlier pairs of its expert.
+__device__ __forceinline__ int32_t pair_rank_of(const TileScan &ts, int r, const uint16_t *wcnt,
+                                                const uint32_t *tile_prefix, int32_t E) {
+  const int warp = threadIdx.x / kWarp;
+  const int32_t e = ts.expert(r);
+  return (int32_t)(tile_prefix[e] + wcnt[(size_t)warp * E + e] + ts.rank(r));
+}
+
+// Row of a pair from its expert and rank; -1 with `dropped` set when it gets
+// none.  Sets MOE_STATUS_CAPACITY bits for packed overflow.
+__device__ __forceinline__ int32_t row_of(int32_t e, int32_t r, const int32_t *s_off, int64_t C,
+                                          int32_t Ce, bool capacity, uint8_t &dropped,
+                                          uint32_t &bits) {
+  dropped = 0;
+  if (capacity) {
+    if (r >= 0 && r < Ce) return e * Ce + r;
+    dropped = 1;
+    return -1;
+  }
+  const int64_t row = (int64_t)s_off[e] + r;
+  if (r >= 0 && row >= 0 && row < C) return (int32_t)row;
+  dropped = 1;
+  bits |= MOE_STATUS_CAPACITY;
+  return -1;
+}
+
+// Block-wide exclusive scan of n <= PER * THREADS values in place; returns
+// the total.  Called by all threads of the block.
+template <int THREADS, int PER>
+__device__ int32_t block_exclusive_scan(int32_t *v, int n) {
+  __shared__ int32_t warp_sums[THREADS / kWarp];
   const int tid = threadIdx.x, lane = tid % kWarp, warp = tid / kWarp;
-  int32_t local[kPer];
+  int32_t local[PER];
   int32_t sum = 0;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int idx = tid * kPer + i;
+  for (int i = 0; i < PER; ++i) {
+    const int idx = tid * PER + i;
     local[i] = idx < n ? v[idx] : 0;
     sum += local[i];
   }
@@ -194,110 +288,64 @@ __device__ void block_exclusive_scan(int32_t *v, int n, int32_t *total_out) {
   if (lane == kWarp - 1) warp_sums[warp] = incl;
   __syncthreads();
   int32_t warp_base = 0, total = 0;
-  for (int w = 0; w < kEmitThreads / kWarp; ++w) {
+#pragma unroll
+  for (int w = 0; w < THREADS / kWarp; ++w) {
     if (w < warp) warp_base += warp_sums[w];
     total += warp_sums[w];
   }
   int32_t run = warp_base + incl - sum;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int idx = tid * kPer + i;
+  for (int i = 0; i < PER; ++i) {
+    const int idx = tid * PER + i;
     if (idx < n) v[idx] = run;
     run += local[i];
   }
-  *total_out = total;
   __syncthreads();
+  return total;
 }
 
-__global__ void __launch_bounds__(kEmitThreads)
-    layout_emit_kernel(const int32_t *__restrict__ ids, int32_t N, int32_t k, int32_t E,
-                       int32_t S, int64_t C, int32_t Ce, int32_t H, uint32_t flags,
-                       int32_t num_tiles, uint32_t *ctrl, const int32_t *__restrict__ totals,
-                       uint64_t *tiles, int32_t *__restrict__ expert_counts,
-                       int32_t *__restrict__ expert_offsets, uint32_t *__restrict__ meta,
-                       int32_t *__restrict__ row_src, int32_t *__restrict__ pair_slot,
-                       uint8_t *__restrict__ drop_mask, uint32_t *status_out) {
-  extern __shared__ __align__(16) int32_t s_emit[];
-  int32_t *s_off = s_emit;           // [E + 1] first row per expert
-  int32_t *s_kept = s_emit + E + 1;  // [E] rows kept per expert
-  __shared__ uint32_t s_status;
-  const int tid = threadIdx.x;
+// Expert start rows s_off[E+1] and kept rows s_kept[E] from the totals.
+template <int THREADS>
+__device__ void expert_offsets_from_totals(const int32_t *totals, bool have_totals, int32_t E,
+                                           int32_t Ce, int32_t *s_off, int32_t *s_kept) {
   const bool capacity = Ce > 0;
-  const int64_t P = (int64_t)N * k;
-  const int64_t rows = capacity ? (int64_t)E * Ce : C;
-  if (tid == 0) s_status = 0;
-
-  for (int e = tid; e < E; e += kEmitThreads) {
-    const int32_t t = num_tiles > 0 ? totals[e] : 0;
+  for (int e = threadIdx.x; e < E; e += THREADS) {
+    const int32_t t = have_totals ? __ldcg(totals + e) : 0;
     s_kept[e] = capacity ? min(t, Ce) : t;
     s_off[e] = capacity ? e * Ce : t;
   }
   __syncthreads();
-  int32_t total = 0;
   if (!capacity) {
-    block_exclusive_scan(s_off, E, &total);
-    if (tid == 0) s_off[E] = total;
-  } else if (tid == 0) {
+    const int32_t total = block_exclusive_scan<THREADS, (MOE_MAX_EXPERTS + THREADS - 1) / THREADS>(
+        s_off, E);
+    if (threadIdx.x == 0) s_off[E] = total;
+  } else if (threadIdx.x == 0) {
     s_off[E] = E * Ce;
   }
   __syncthreads();
+}
 
-  const int64_t gtid = (int64_t)blockIdx.x * kEmitThreads + tid;
-  const int64_t gstride = (int64_t)gridDim.x * kEmitThreads;
-  uint32_t bits = 0;
-
-  // ---- per pair: rank -> row
-  for (int64_t p = gtid; p < P; p += gstride) {
-    const int32_t e = __ldg(ids + p);
-    int32_t slot = -1;
-    uint8_t dropped = 0;
-    if ((uint32_t)e < (uint32_t)E) {
-      const int32_t r = pair_slot[p];
-      if (capacity) {
-        if (r >= 0 && r < Ce) slot = e * Ce + r;
-        else dropped = 1;
-      } else {
-        const int64_t row = (int64_t)s_off[e] + r;
-        if (r >= 0 && row >= 0 && row < C) {
-          slot = (int32_t)row;
-        } else {
-          dropped = 1;
-          bits |= MOE_STATUS_CAPACITY;
-        }
-      }
-    }
-    pair_slot[p] = slot;
-    if (drop_mask) drop_mask[p] = dropped;
-    if (slot >= 0) row_src[slot] = (int32_t)(p / k);
-  }
-
-  // ---- optional duplicate check, per token
-  if (flags & MOE_FLAG_CHECK_DUPLICATES) {
-    for (int64_t t = gtid; t < N; t += gstride) {
-      const int32_t *row = ids + t * k;
-      for (int a = 0; a < k; ++a) {
-        const int32_t ea = __ldg(row + a);
-        if ((uint32_t)ea >= (uint32_t)E) continue;
-        for (int b = a + 1; b < k; ++b)
-          if (__ldg(row + b) == ea) bits |= MOE_STATUS_DUP_ID;
-      }
-    }
-  }
-
-  // ---- padding rows
-  for (int64_t r = gtid; r < rows; r += gstride) {
+// Padding rows of [r0, rows) in steps of `stride`, counts/offsets/meta when
+// `write_meta`, duplicate check for tokens [t0, t1) in steps of `tstride`.
+template <int THREADS>
+__device__ void emit_common(int64_t r0, int64_t stride, int64_t rows, int32_t E, int32_t S,
+                            int32_t Ce, int32_t H, const int32_t *s_off, const int32_t *s_kept,
+                            int32_t *__restrict__ row_src, bool write_meta,
+                            int32_t *__restrict__ expert_counts,
+                            int32_t *__restrict__ expert_offsets, uint32_t *__restrict__ meta) {
+  const bool capacity = Ce > 0;
+  for (int64_t r = r0; r < rows; r += stride) {
     bool pad;
     if (capacity) pad = (int32_t)(r % Ce) >= s_kept[r / Ce];
     else pad = r >= (int64_t)s_off[E];
     if (pad) row_src[r] = -1;
   }
-
-  // ---- counts, offsets, [4, S] metadata (block 0)
-  if (blockIdx.x == 0) {
-    for (int e = tid; e < E; e += kEmitThreads) expert_counts[e] = s_kept[e];
-    for (int e = tid; e <= E; e += kEmitThreads) expert_offsets[e] = s_off[e];
+  if (write_meta) {
+    const int tid = threadIdx.x;
+    for (int e = tid; e < E; e += THREADS) expert_counts[e] = s_kept[e];
+    for (int e = tid; e <= E; e += THREADS) expert_offsets[e] = s_off[e];
     const int32_t L = E / S;
-    for (int s = tid; s < S; s += kEmitThreads) {
+    for (int s = tid; s < S; s += THREADS) {
       int64_t seg_rows = 0;
       for (int e = s * L; e < (s + 1) * L; ++e) seg_rows += s_kept[e];
       const uint32_t count_el = (uint32_t)(seg_rows * H);
@@ -308,26 +356,196 @@ __global__ void __launch_bounds__(kEmitThreads)
       meta[2 * S + s] = count_el;
       meta[3 * S + s] = displ_el;
     }
-    if (tid == 0) ctrl[0] = 0;  // the scan kernel has finished: reset its ticket
   }
+}
 
-  // ---- return the scan tile states to zero for the next call
-  const int64_t n_states = (int64_t)num_tiles * E;
-  for (int64_t i = gtid; i < n_states; i += gstride) tiles[i] = 0;
-
-  // ---- status: the last block to finish publishes this call's bits
-  if (bits) atomicOr(&s_status, bits);
-  __syncthreads();
-  if (tid == 0) {
-    if (s_status) atomicOr(&ctrl[2], s_status);
-    __threadfence();
-    const uint32_t done = atomicAdd(&ctrl[1], 1u);
-    if (done == gridDim.x - 1) {
-      __threadfence();
-      *status_out = atomicExch(&ctrl[2], 0u);
-      atomicExch(&ctrl[1], 0u);
+__device__ uint32_t duplicate_bits(const int32_t *__restrict__ ids, int64_t t0, int64_t t1,
+                                   int64_t tstride, int32_t k, int32_t E) {
+  uint32_t bits = 0;
+  for (int64_t t = t0; t < t1; t += tstride) {
+    const int32_t *row = ids + t * k;
+    for (int a = 0; a < k; ++a) {
+      const int32_t ea = __ldg(row + a);
+      if ((uint32_t)ea >= (uint32_t)E) continue;
+      for (int b = a + 1; b < k; ++b)
+        if (__ldg(row + b) == ea) bits |= MOE_STATUS_DUP_ID;
     }
   }
+  return bits;
+}
+
+// The last block to arrive publishes the status word and returns the
+// workspace (tile states, totals, control words) to zero.  Called by all
+// threads of every block, last thing in the kernel.
+template <int THREADS>
+__device__ void finish_and_clean(uint32_t bits, uint32_t *s_status, uint32_t *ctrl,
+                                 int32_t *totals, uint64_t *tiles, int64_t n_states, int32_t E,
+                                 uint32_t *status_out, uint32_t n_blocks) {
+  __shared__ bool s_last;
+  if (bits) atomicOr(s_status, bits);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (*s_status) atomicOr(&ctrl[kCtrlStatus], *s_status);
+    __threadfence();
+    s_last = atomicAdd(&ctrl[kCtrlDone], 1u) == n_blocks - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int64_t i = threadIdx.x; i < n_states; i += THREADS) tiles[i] = 0;
+  for (int e = threadIdx.x; e < E; e += THREADS) totals[e] = 0;
+  if (threadIdx.x == 0) {
+    *status_out = atomicExch(&ctrl[kCtrlStatus], 0u);
+    ctrl[kCtrlTicket] = 0;
+    ctrl[kCtrlTilesDone] = 0;
+    atomicExch(&ctrl[kCtrlDone], 0u);
+  }
+}
+
+// ------------------------------------------------------------ kernels
+struct LayoutArgs {
+  const int32_t *ids;
+  int64_t P;
+  int32_t N, k, E, S, Ce, H;
+  int64_t C, rows;
+  uint32_t flags;
+  int32_t num_tiles;
+  uint32_t *ctrl;
+  int32_t *totals;
+  uint64_t *tiles;
+  int32_t *expert_counts, *expert_offsets;
+  uint32_t *meta;
+  int32_t *row_src, *pair_slot;
+  uint8_t *drop_mask;
+  uint32_t *status_out;
+};
+
+// Scan step of one CTA: if it draws a tile, rank the tile's pairs and store
+// the ranks in pair_slot (the last tile also stores the totals).
+template <bool COUNT_DONE>
+__device__ void scan_step(const LayoutArgs &a, uint8_t *smem, uint32_t *s_status) {
+  __shared__ int s_tile;
+  const ScanSmem sm = scan_smem(smem, a.E);
+  TileScan ts;
+  if (!scan_tile(ts, a.ids, a.P, a.E, a.num_tiles, a.flags, a.ctrl, a.tiles, a.totals, sm,
+                 &s_tile, s_status))
+    return;
+  const int lane = threadIdx.x % kWarp;
+#pragma unroll
+  for (int r = 0; r < kScanRounds; ++r) {
+    const int64_t p = ts.base + r * kWarp + lane;
+    if (p < a.P)
+      a.pair_slot[p] = ts.expert(r) >= 0 ? pair_rank_of(ts, r, sm.wcnt, sm.tile_prefix, a.E) : -1;
+  }
+  if (COUNT_DONE) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      atomicAdd(&a.ctrl[kCtrlTilesDone], 1u);
+    }
+  }
+}
+
+// Emit step: ranks -> rows for the pairs [gtid, P) in steps of gstride, the
+// padding rows, counts / offsets / meta (block 0), the duplicate check, then
+// the last block cleans up.  n_states: tile states the last block clears.
+template <int THREADS>
+__device__ void emit_step(const LayoutArgs &a, int64_t gtid, int64_t gstride,
+                          uint32_t *s_status, int64_t n_states) {
+  __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
+  __shared__ int32_t s_kept[MOE_MAX_EXPERTS];
+  expert_offsets_from_totals<THREADS>(a.totals, a.num_tiles > 0, a.E, a.Ce, s_off, s_kept);
+  const bool capacity = a.Ce > 0;
+  uint32_t bits = 0;
+  for (int64_t p = gtid; p < a.P; p += gstride) {
+    const int32_t e = __ldg(a.ids + p);
+    int32_t slot = -1;
+    uint8_t dropped = 0;
+    if ((uint32_t)e < (uint32_t)a.E)
+      slot = row_of(e, __ldcg(a.pair_slot + p), s_off, a.C, a.Ce, capacity, dropped, bits);
+    a.pair_slot[p] = slot;
+    if (a.drop_mask) a.drop_mask[p] = dropped;
+    if (slot >= 0) a.row_src[slot] = (int32_t)p / a.k;
+  }
+  emit_common<THREADS>(gtid, gstride, a.rows, a.E, a.S, a.Ce, a.H, s_off, s_kept, a.row_src,
+                       blockIdx.x == 0, a.expert_counts, a.expert_offsets, a.meta);
+  if (a.flags & MOE_FLAG_CHECK_DUPLICATES)
+    bits |= duplicate_bits(a.ids, gtid, a.N, gstride, a.k, a.E);
+  finish_and_clean<THREADS>(bits, s_status, a.ctrl, a.totals, a.tiles, n_states, a.E,
+                            a.status_out, (uint32_t)gridDim.x);
+}
+
+// One cooperative launch: scan (first T CTAs), grid-wide wait, emit (all).
+__global__ void __launch_bounds__(kScanThreads, 1) layout_fused_kernel(LayoutArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ uint32_t s_status;
+  if (threadIdx.x == 0) s_status = 0;
+  __syncthreads();
+  scan_step<true>(a, smem, &s_status);
+  // wait (bounded) until every tile has stored its ranks and the totals
+  if (threadIdx.x == 0) {
+    uint64_t deadline = 0;
+    while (ld_acquire_gpu_u32(&a.ctrl[kCtrlTilesDone]) < (uint32_t)a.num_tiles) {
+      if (!keep_waiting(deadline)) {
+        atomicOr(&s_status, MOE_STATUS_TIMEOUT);
+        break;
+      }
+      __nanosleep(20);
+    }
+  }
+  __syncthreads();
+  const int64_t gtid = (int64_t)blockIdx.x * kScanThreads + threadIdx.x;
+  const int64_t gstride = (int64_t)gridDim.x * kScanThreads;
+  // every look-back has finished: the tile states can be cleared by everyone
+  for (int64_t i = gtid; i < (int64_t)a.num_tiles * a.E; i += gstride) a.tiles[i] = 0;
+  emit_step<kScanThreads>(a, gtid, gstride, &s_status, 0);
+}
+
+__global__ void __launch_bounds__(kScanThreads, 1) layout_count_scan_kernel(LayoutArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ uint32_t s_status;
+  scan_step<false>(a, smem, &s_status);
+  __syncthreads();
+  if (threadIdx.x == 0 && s_status) atomicOr(&a.ctrl[kCtrlStatus], s_status);
+}
+
+__global__ void __launch_bounds__(kEmitThreads) layout_emit_kernel(LayoutArgs a) {
+  __shared__ uint32_t s_status;
+  if (threadIdx.x == 0) s_status = 0;
+  const int64_t gtid = (int64_t)blockIdx.x * kEmitThreads + threadIdx.x;
+  const int64_t gstride = (int64_t)gridDim.x * kEmitThreads;
+  // the scan kernel has finished: its tile states can be cleared by everyone
+  for (int64_t i = gtid; i < (int64_t)a.num_tiles * a.E; i += gstride) a.tiles[i] = 0;
+  emit_step<kEmitThreads>(a, gtid, gstride, &s_status, 0);
+}
+
+constexpr int kMaxDevices = 64;
+
+// Opt the scan kernels in to more than 48 KB of dynamic shared memory, once
+// per device.
+cudaError_t opt_in_smem() {
+  static std::atomic<bool> done[kMaxDevices];
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < kMaxDevices && done[dev].load()) return cudaSuccess;
+  const int bytes = (int)scan_smem_bytes(MOE_MAX_EXPERTS);
+  err = cudaFuncSetAttribute(layout_count_scan_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(layout_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               bytes);
+  if (err == cudaSuccess && dev < kMaxDevices) done[dev].store(true);
+  return err;
+}
+
+// Largest grid of the fused kernel that is guaranteed co-resident.
+int fused_capacity(size_t smem) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel, kScanThreads,
+                                                    smem) != cudaSuccess)
+    return 0;
+  return per_sm * device_sm_count();
 }
 
 }  // namespace
@@ -353,28 +571,61 @@ cudaError_t launch_layout(const Shape &s, const int32_t *ids, int32_t *expert_co
                           int32_t *expert_offsets, uint32_t *meta, int32_t *row_src,
                           int32_t *pair_slot, uint8_t *drop_mask, uint32_t *status,
                           const LayoutWorkspace &ws, cudaStream_t stream) {
-  if (ws.num_tiles > 0) {
-    const size_t smem = scan_smem_bytes(s.E);
-    if (smem > 48 * 1024) {
-      cudaError_t err = cudaFuncSetAttribute(layout_count_scan_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-      if (err != cudaSuccess) return err;
+  LayoutArgs a;
+  a.ids = ids;
+  a.P = s.P;
+  a.N = s.N;
+  a.k = s.k;
+  a.E = s.E;
+  a.S = s.S;
+  a.Ce = s.Ce;
+  a.H = s.H;
+  a.C = s.C;
+  a.rows = s.rows;
+  a.flags = s.flags;
+  a.num_tiles = ws.num_tiles;
+  a.ctrl = ws.ctrl;
+  a.totals = ws.totals;
+  a.tiles = ws.tiles;
+  a.expert_counts = expert_counts;
+  a.expert_offsets = expert_offsets;
+  a.meta = meta;
+  a.row_src = row_src;
+  a.pair_slot = pair_slot;
+  a.drop_mask = drop_mask;
+  a.status_out = status;
+
+  const size_t smem = scan_smem_bytes(s.E);
+  if (ws.num_tiles > 0 && smem > 32 * 1024) {
+    cudaError_t err = opt_in_smem();
+    if (err != cudaSuccess) return err;
+  }
+
+  if (ws.num_tiles > 0 && ws.num_tiles <= kFusedMaxTiles &&
+      !(s.flags & MOE_FLAG_LAYOUT_TWO_PASS)) {
+    // one CTA per tile at least, one thread per pair or row at most, all
+    // co-resident (the grid-wide wait needs every CTA running)
+    const int capacity = fused_capacity(smem);
+    const int64_t work = std::max<int64_t>(s.P, s.rows);
+    const int64_t want = std::max<int64_t>(ws.num_tiles, (work + kScanThreads - 1) / kScanThreads);
+    const int grid = (int)std::min<int64_t>(want, capacity);
+    if (grid >= ws.num_tiles) {
+      void *args[] = {&a};
+      return cudaLaunchCooperativeKernel((const void *)layout_fused_kernel, dim3(grid),
+                                         dim3(kScanThreads), args, smem, stream);
     }
-    layout_count_scan_kernel<<<ws.num_tiles, kScanThreads, smem, stream>>>(
-        ids, s.P, s.E, ws.num_tiles, s.flags, ws.ctrl, ws.totals, ws.tiles, pair_slot);
+  }
+  if (ws.num_tiles > 0) {
+    layout_count_scan_kernel<<<ws.num_tiles, kScanThreads, smem, stream>>>(a);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
   const int64_t work = std::max<int64_t>(std::max<int64_t>(s.P, s.rows),
                                          (int64_t)ws.num_tiles * s.E);
-  const int64_t max_blocks = (int64_t)device_sm_count() * 4;
+  const int64_t max_blocks = (int64_t)device_sm_count() * 8;
   const int blocks = (int)std::max<int64_t>(
-      1, std::min<int64_t>(max_blocks, (work + kEmitThreads * 4 - 1) / (kEmitThreads * 4)));
-  const size_t smem = (size_t)(2 * s.E + 1) * sizeof(int32_t);
-  layout_emit_kernel<<<blocks, kEmitThreads, smem, stream>>>(
-      ids, s.N, s.k, s.E, s.S, s.C, s.Ce, s.H, s.flags, ws.num_tiles, ws.ctrl, ws.totals,
-      ws.tiles, expert_counts, expert_offsets, meta, row_src, pair_slot, drop_mask, status);
+      1, std::min<int64_t>(max_blocks, (work + kEmitThreads - 1) / kEmitThreads));
+  layout_emit_kernel<<<blocks, kEmitThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

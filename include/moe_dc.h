@@ -79,6 +79,10 @@ enum {
 /* Problem flags. */
 enum {
   MOE_FLAG_CHECK_DUPLICATES = 1u,
+  /* Run the layout as two kernels (scan, then emit) even where the one-launch
+   * cooperative kernel applies.  Results are identical; for testing and
+   * tuning. */
+  MOE_FLAG_LAYOUT_TWO_PASS = 2u,
   /* Test hook: the first scan tile never publishes its counts, so every
    * later tile's bounded wait runs out and MOE_STATUS_TIMEOUT is reported.
    * Results are invalid; used only to test the timeout path. */
@@ -112,8 +116,7 @@ MOE_API int64_t moe_output_rows(const moe_problem *problem);
 /* Bytes of device workspace moe_dispatch_layout needs for this problem
  * (control counters, per-expert totals, scan tile states).  The workspace
  * must be zero-filled once before its first use (e.g. cudaMemset); every
- * completed layout call returns its counters and tile states to zero (the
- * totals are scratch that each call overwrites), so a workspace sized for
+ * completed layout call returns all of it to zero, so a workspace sized for
  * the largest problem can serve any later call on the same stream.  Calls
  * sharing one workspace must not overlap on the GPU.  Returns 0 for an
  * invalid problem. */

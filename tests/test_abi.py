@@ -54,7 +54,7 @@ def test_host_only_entry_points(lib):
     p = B.Problem(num_tokens=8192, hidden=7168, num_experts=256, top_k=8, num_segments=8,
                   recv_capacity=65536)
     assert B.moe_output_rows(p) == 65536
-    # control (256 B) + totals (1 KiB) + 16 tiles x 256 experts x 8 B
+    # control (256 B) + totals (1 KiB) + 16 scan tiles x 256 experts x 8 B
     assert B.moe_workspace_bytes(p) == 256 + 1024 + 16 * 256 * 8
     p.expert_capacity = 5
     assert B.moe_output_rows(p) == 1280
