@@ -35,9 +35,11 @@ MOE_MAX_EXPERTS = 2048
 MOE_MAX_TOPK = 16
 
 # every symbol include/moe_dc.h declares
-EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout", "moe_permute",
-            "moe_permute_quant_fp8", "moe_permute_quant_nvfp4", "moe_combine",
-            "moe_status_string", "moe_version")
+EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout",
+            "moe_dispatch_layout_noalloc", "moe_permute", "moe_permute_quant_fp8",
+            "moe_permute_quant_nvfp4", "moe_combine", "moe_status_string", "moe_version")
+
+MOE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
 class MoeError(RuntimeError):
@@ -93,6 +95,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     L.moe_workspace_bytes.argtypes = [P]
     L.moe_dispatch_layout.restype = ctypes.c_int
     L.moe_dispatch_layout.argtypes = [P] + [vp] * 10
+    L.moe_dispatch_layout_noalloc.restype = ctypes.c_int
+    L.moe_dispatch_layout_noalloc.argtypes = [P] + [vp] * 9
     L.moe_permute.restype = ctypes.c_int
     L.moe_permute.argtypes = [P] + [vp] * 5
     L.moe_permute_quant_fp8.restype = ctypes.c_int
@@ -153,6 +157,18 @@ def moe_dispatch_layout(prob: Problem, topk_ids, expert_counts, expert_offsets, 
                                       _ptr(pair_slot), _ptr(drop_mask), _ptr(status),
                                       _ptr(workspace), _stream(stream)),
            "moe_dispatch_layout")
+
+
+def moe_dispatch_layout_noalloc(prob: Problem, topk_ids, expert_counts, expert_offsets, meta,
+                                row_src, pair_slot, drop_mask, status, stream=None) -> None:
+    """The layout without a caller workspace (for callers that cannot
+    allocate); see moe_dispatch_layout_noalloc in moe_dc.h for its limits."""
+    c = prob.c()
+    _check(load().moe_dispatch_layout_noalloc(ctypes.byref(c), _ptr(topk_ids),
+                                              _ptr(expert_counts), _ptr(expert_offsets),
+                                              _ptr(meta), _ptr(row_src), _ptr(pair_slot),
+                                              _ptr(drop_mask), _ptr(status), _stream(stream)),
+           "moe_dispatch_layout_noalloc")
 
 
 def moe_permute(prob: Problem, hidden_states, row_src, pair_slot, out, stream=None) -> None:

@@ -166,6 +166,38 @@ MOE_API moe_status moe_dispatch_layout(const moe_problem *problem, const int32_t
                                uint8_t *drop_mask, uint32_t *status, void *workspace,
                                moe_stream_t stream);
 
+/* Size of the static scratch of moe_dispatch_layout_noalloc (1 MiB). */
+#define MOE_NOALLOC_SCRATCH_BYTES 1048576
+
+/* moe_dispatch_layout for callers that cannot allocate device memory.  The
+ * pages have no counterpart: this entry point exists for callers that may not
+ * call cudaMalloc or any allocating routine -- for example code whose device
+ * memory is wholly owned by a framework's caching allocator or a fixed
+ * up-front memory plan, or plugin code with no handle to an allocator -- and
+ * so cannot provide the workspace buffer.
+ *
+ * Same arguments, outputs, checks and results as moe_dispatch_layout, minus
+ * `workspace`: the scratch is a static device array of
+ * MOE_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits.  Nothing is allocated or freed.
+ *   - A problem whose moe_workspace_bytes() exceeds MOE_NOALLOC_SCRATCH_BYTES
+ *     is rejected with MOE_ERR_UNSUPPORTED_SHAPE before anything is launched
+ *     (at E = 256 that is above about 2 million pairs); use
+ *     moe_dispatch_layout with a workspace for such problems.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (it must be the current device); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array and finds what the previous call left
+ *     in it; each call zero-fills the part it uses on its own stream before
+ *     launching.  Calls that overlap on the GPU (other streams, other host
+ *     threads) race on the array: serialise them. */
+MOE_API moe_status moe_dispatch_layout_noalloc(const moe_problem *problem,
+                                               const int32_t *topk_ids, int32_t *expert_counts,
+                                               int32_t *expert_offsets, uint32_t *meta,
+                                               int32_t *row_src, int32_t *pair_slot,
+                                               uint8_t *drop_mask, uint32_t *status,
+                                               moe_stream_t stream);
+
 /* Permute, bf16 payload: out[r, :] = hidden_states[row_src[r], :], or zeros
  * when row_src[r] == -1.  NKI permute_a2av return value ([C, H] packed rows
  * followed by deterministic zero padding); Mojo MAX ep_comm BF16TokenFormat.
