@@ -40,9 +40,15 @@ METRIC = "dispatch+combine tokens/s and HBM GB/s (% of peak) at N=8192 H=7168 E=
 WORKLOAD = "fp8_metric"
 FALLBACK_HBM_GBS = 6650.0
 
-# dram bytes per launch from one ncu capture, keyed by kernel, valid only
-# while the kernel source is unchanged (sha256 of the .cu file at capture)
-NCU_TRAFFIC: dict[str, dict] = {}
+# dram bytes (read + write) per launch from one ncu --set full capture on the
+# metric workload (summaries under profiles/), keyed by kernel; valid only
+# while the kernel's source file is unchanged (sha256 prefix at capture time)
+NCU_TRAFFIC: dict[str, dict] = {
+    "permute_bf16": {"bytes_per_launch": 117978624 + 881600512, "src_sha": "7f0bbb0aa172d04b"},
+    "permute_fp8": {"bytes_per_launch": 118048512 + 428314624, "src_sha": "7f0bbb0aa172d04b"},
+    "permute_nvfp4": {"bytes_per_launch": 118004736 + 207263488, "src_sha": "7f0bbb0aa172d04b"},
+    "combine": {"bytes_per_launch": 940062720 + 67858688, "src_sha": "e2707ccbc781905c"},
+}
 
 
 def _kernel_src_sha(name: str) -> str:
