@@ -5,11 +5,12 @@
 // Movement is token-major ("push"): each token's row is read from HBM once
 // with 16-byte streaming loads and stored (or its quantised form) to each of
 // its k destination rows with 16-byte stores, so the quantisation is computed
-// once per token, not once per copy.  The unit of work is one 1024-element
-// chunk of one token (2 KB of bf16): one warp takes one unit and exits.  Short
-// warps over a grid of many blocks keep the write stream denser than
-// long-lived persistent warps do (measured on B200: 175 us vs 195 us for the
-// bf16 permute at N=8192, H=7168, k=8).  Warps past the token units each
+// once per token, not once per copy.  The unit of work is one chunk of one
+// token (512 elements for bf16, 1024 for the quantisers): one warp takes one
+// unit and exits.  Short warps over a grid of many blocks keep the write
+// stream denser than long-lived persistent warps do (measured on B200 for the
+// bf16 permute at N=8192, H=7168, k=8: 195 us persistent, 170 us with
+// 1024-element units, 166 us with 512).  Warps past the token units each
 // check 32 rows of row_src and zero-fill the rows whose source is -1.
 //
 #include <algorithm>
@@ -37,7 +38,8 @@ __device__ __forceinline__ uint32_t load_token_slots(const int32_t *__restrict__
   return __ballot_sync(kFull, my_slot >= 0);
 }
 
-constexpr int kChunk = 1024;  // elements of one token per unit of work
+constexpr int kChunk = 1024;     // elements of one token per unit (quantisers)
+constexpr int kBf16Chunk = 512;  // elements of one token per unit (bf16)
 
 // Zero-fill every row r in [32*c, 32*c + 32) whose source is -1; `row_vecs`
 // 16-byte vectors per row of `out`, `srow` 2-byte words per row of `scales`.
@@ -62,12 +64,12 @@ __device__ __forceinline__ void zero_padding_rows(int64_t c, int lane,
 }
 
 // ------------------------------------------------------------------- bf16
-// Unit = (token, 1024 elements): each lane loads 4 vectors of 8 bf16.
+// Unit = (token, 512 elements): each lane loads 2 vectors of 8 bf16.
 __global__ void __launch_bounds__(kThreads)
     permute_bf16_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                         const int32_t *__restrict__ pair_slot, uint4 *__restrict__ out,
                         int32_t N, int32_t k, int64_t rows, int32_t vecs, int32_t chunks) {
-  constexpr int U = kChunk / 8 / kWarp;  // 4
+  constexpr int U = kBf16Chunk / 8 / kWarp;  // 2
   const int lane = threadIdx.x % kWarp;
   const int64_t w = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
@@ -76,7 +78,7 @@ __global__ void __launch_bounds__(kThreads)
     return;
   }
   const int64_t t = w / chunks;
-  const int v0 = (int)(w % chunks) * (kChunk / 8);
+  const int v0 = (int)(w % chunks) * (kBf16Chunk / 8);
   int32_t my_slot;
   uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
   const uint4 *src = hidden + t * vecs;
@@ -272,14 +274,14 @@ inline int64_t unit_blocks(const Shape &s, int32_t chunks) {
   return (warps + kThreads / kWarp - 1) / (kThreads / kWarp);
 }
 
-inline int32_t chunks_of(int32_t H) { return (H + kChunk - 1) / kChunk; }
+inline int32_t chunks_of(int32_t H, int32_t chunk = kChunk) { return (H + chunk - 1) / chunk; }
 
 }  // namespace
 
 cudaError_t launch_permute_bf16(const Shape &s, const void *hidden, const int32_t *row_src,
                                 const int32_t *pair_slot, void *out, cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
-  const int32_t chunks = chunks_of(s.H);
+  const int32_t chunks = chunks_of(s.H, kBf16Chunk);
   permute_bf16_kernel<<<(unsigned)unit_blocks(s, chunks), kThreads, 0, stream>>>(
       static_cast<const uint4 *>(hidden), row_src, pair_slot, static_cast<uint4 *>(out), s.N,
       s.k, s.rows, s.H / 8, chunks);

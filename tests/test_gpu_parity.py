@@ -311,3 +311,75 @@ def test_cuda_graph_capture_and_replay(orc):
         q, sc = orc.permute_nvfp4(w.hidden, ref.row_src, w.global_scale)
         assert np.array_equal(buf.scales_fp4.cpu().numpy(), sc)
         assert np.array_equal(bf16_np(y), orc.combine(w.expert_out, w.gates, ref.pair_slot))
+
+
+# ------------------------------------------------------------ rounding edges
+def _bits(x):
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).view(
+        torch.int16).numpy().view(np.uint16)
+
+
+def _one_token_per_row(orc, rows_f32, gs=1.0):
+    """Each row of rows_f32 is one token routed to one expert (k = 1), so the
+    dispatch output is the rows in order; returns (workload, run, layout)."""
+    N, H = rows_f32.shape
+    ids = np.zeros((N, 1), np.int32)
+    w = Workload(name="edge", N=N, H=H, E=1, k=1, S=1, recv_capacity=N, expert_capacity=0,
+                 ids=ids, gates=np.ones((N, 1), np.float32), hidden=_bits(rows_f32),
+                 expert_out=None, global_scale=float(np.float32(gs)), seed=0)
+    run = GpuRun(w, combine=False)
+    ref = oracle_layout(orc, w)
+    assert_layout(run, ref)
+    return w, run, ref
+
+
+def test_fp8_rounding_ties_and_edges(orc):
+    """Quotients exactly on E4M3 midpoints (ties to even), on codes, in the
+    subnormal range, at the saturation edge and signed zeros: the block scale
+    is a power of two, so x / scale is exact."""
+    mids = np.array([8.5, 9.5, 17, 19, 36, 40, 104, 232, 240, 1.0625, 1.1875,
+                     0.0029296875, 0.0048828125, 0.0068359375, 0.0009765625], np.float32)
+    codes = np.array([16, 18, 448, 0.015625, 0.001953125, 2.0, 3.5], np.float32)
+    rng = np.random.default_rng(3)
+    rows = []
+    for k in range(-6, 6):
+        for sign in (1, -1):
+            blk = np.zeros(128, np.float32)
+            blk[0] = 448.0                                   # amax -> scale 2^k
+            vals = np.concatenate([mids, -mids, codes, [-0.0, 0.0]])
+            blk[1:1 + vals.size] = vals
+            blk[1 + vals.size:] = rng.standard_normal(127 - vals.size) * 50
+            rows.append(sign * blk * np.float32(2.0 ** k))
+    x = np.stack(rows).reshape(-1, 256)
+    w, run, ref = _one_token_per_row(orc, x)
+    q, s = orc.permute_fp8(w.hidden, ref.row_src)
+    assert np.array_equal(run.q8, q)
+    assert np.array_equal(run.s8.view(np.uint32), s.view(np.uint32))
+
+
+@pytest.mark.parametrize("gs", [1.0, 1.0 + 2.0 ** -23, 1.0 - 2.0 ** -24, 1.0 + 2.0 ** -22,
+                                0.3333333432674408, 2.0 ** -7])
+def test_nvfp4_rounding_ties_and_near_ties(orc, gs):
+    """Blocks whose amax makes the decode scale d = float(e4m3 scale) * gs
+    equal to gs (amax = 6 * gs-ish), with elements on E2M1 midpoints: with gs
+    a power of two the quotients are exact ties; with gs one ulp off 1 they
+    are one or two ulps off the midpoints, where a reciprocal product and the
+    division can round differently."""
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1.0, 1.5, 2, 3, 4, 6,
+                     0.125], np.float32)
+    rows = []
+    rng = np.random.default_rng(int(gs * 1000) % 97)
+    scale_of = np.float32(6.0) * np.float32(gs) if gs < 0.9 else np.float32(6.0)
+    for sign in (1, -1):
+        for r in range(8):
+            blk = np.zeros(32, np.float32)
+            blk[0] = scale_of
+            blk[1:1 + mids.size] = mids * (np.float32(gs) if gs < 0.9 else 1)
+            blk[16] = scale_of
+            blk[17:] = rng.uniform(-6, 6, 15) * (np.float32(gs) if gs < 0.9 else 1)
+            rows.append(sign * blk)
+    x = np.stack(rows)
+    w, run, ref = _one_token_per_row(orc, x, gs=gs)
+    q, s = orc.permute_nvfp4(w.hidden, ref.row_src, w.global_scale)
+    assert np.array_equal(run.s4, s)
+    assert np.array_equal(run.q4, q)
