@@ -44,9 +44,9 @@ FALLBACK_HBM_GBS = 6650.0
 # metric workload (summaries under profiles/), keyed by kernel; valid only
 # while the kernel's source file is unchanged (sha256 prefix at capture time)
 NCU_TRAFFIC: dict[str, dict] = {
-    "permute_bf16": {"bytes_per_launch": 117978624 + 881600512, "src_sha": "7f0bbb0aa172d04b"},
-    "permute_fp8": {"bytes_per_launch": 118048512 + 428314624, "src_sha": "7f0bbb0aa172d04b"},
-    "permute_nvfp4": {"bytes_per_launch": 118004736 + 207263488, "src_sha": "7f0bbb0aa172d04b"},
+    "permute_bf16": {"bytes_per_launch": 117994240 + 881679104, "src_sha": "5f3b2a0f2b412c22"},
+    "permute_fp8": {"bytes_per_launch": 118048768 + 426491648, "src_sha": "5f3b2a0f2b412c22"},
+    "permute_nvfp4": {"bytes_per_launch": 117995520 + 205992960, "src_sha": "5f3b2a0f2b412c22"},
     "combine": {"bytes_per_launch": 940062720 + 67858688, "src_sha": "e2707ccbc781905c"},
 }
 
