@@ -57,8 +57,9 @@ def lib():
         i32, i64, u32, f32, vp = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
                                   ctypes.c_float, ctypes.c_void_p)
         L.orc_layout.restype = u32
-        L.orc_layout.argtypes = [i32, i32, i32, i32, i64, i32, u32, i32,
+        L.orc_layout.argtypes = [i32, i32, i32, i32, i64, i32, i32, u32, i32,
                                  vp, vp, vp, vp, vp, vp, vp]
+        L.orc_swizzle_scales.argtypes = [i64, i32, vp, vp]
         L.orc_permute_bf16.argtypes = [i64, i32, vp, vp, vp]
         L.orc_permute_fp8.argtypes = [i64, i32, vp, vp, vp, vp]
         L.orc_permute_nvfp4.argtypes = [i64, i32, vp, vp, f32, vp, vp]
@@ -122,7 +123,7 @@ class Layout:
 
 def layout(ids: np.ndarray, num_experts: int, num_segments: int, hidden: int,
            recv_capacity: int = 0, expert_capacity: int = 0,
-           flags: int = 0) -> Layout:
+           flags: int = 0, expert_pad_multiple: int = 0) -> Layout:
     ids = np.ascontiguousarray(ids, dtype=np.int32)
     N, k = ids.shape
     E, S = num_experts, num_segments
@@ -133,7 +134,8 @@ def layout(ids: np.ndarray, num_experts: int, num_segments: int, hidden: int,
     row_src = np.empty(rows, np.int32)
     pair_slot = np.empty((N, k), np.int32)
     drop = np.empty((N, k), np.uint8)
-    st = lib().orc_layout(N, k, E, S, recv_capacity, expert_capacity, flags, hidden,
+    st = lib().orc_layout(N, k, E, S, recv_capacity, expert_capacity, expert_pad_multiple,
+                          flags, hidden,
                           _p(ids), _p(counts), _p(offsets), _p(meta), _p(row_src),
                           _p(pair_slot), _p(drop))
     return Layout(int(st), counts, offsets, meta, row_src, pair_slot, drop)
@@ -169,6 +171,15 @@ def permute_nvfp4(hidden_bits: np.ndarray, row_src: np.ndarray, global_scale: fl
     lib().orc_permute_nvfp4(row_src.size, H, _p(hidden_bits), _p(row_src),
                             float(np.float32(global_scale)), _p(q), _p(sc))
     return q, sc
+
+
+def swizzle_scales(linear: np.ndarray) -> np.ndarray:
+    """[rows, nsf] uint8 scales -> the 128x4 atom layout (flat uint8)."""
+    linear = np.ascontiguousarray(linear, dtype=np.uint8)
+    rows, nsf = linear.shape
+    out = np.empty(((rows + 127) // 128 * 128) * ((nsf + 3) // 4 * 4), np.uint8)
+    lib().orc_swizzle_scales(rows, nsf, _p(linear), _p(out))
+    return out
 
 
 # ---------------------------------------------------------------- combine

@@ -157,13 +157,19 @@ void orc_e2m1_from_f32_n(const float *in, uint8_t *out, int64_t n) {
  * expert e (in ascending pair order) takes row e*Ce + r when r < Ce and is
  * dropped otherwise.
  *
+ * Per-expert padding (NeMo moe_router_expert_pad_multiple, packed mode):
+ * expert e's block of rows is its count rounded up to a multiple of pad, so
+ * every expert starts at a multiple of pad; the rows past the count are
+ * padding like the rows past the total.
+ *
  * send_counts / send_displs / recv_counts / recv_displs (NKI [4, EP]
- * uint32 metadata, in elements): per destination segment the kept rows
- * times H, and their exclusive cumulative sum (packed) or the static
- * segment start s*L*Ce*H (capacity).  On one device the receive rows equal
- * the send rows. */
+ * uint32 metadata, in elements): per destination segment its rows times H
+ * -- the expert blocks, per-expert padding included, in packed mode; the
+ * kept rows in capacity mode -- and where they start: the exclusive
+ * cumulative sum (packed) or the static segment start s*L*Ce*H (capacity).
+ * On one device the receive rows equal the send rows. */
 uint32_t orc_layout(int32_t N, int32_t k, int32_t E, int32_t S, int64_t C,
-                    int32_t Ce, uint32_t flags, int32_t H,
+                    int32_t Ce, int32_t pad, uint32_t flags, int32_t H,
                     const int32_t *ids, int32_t *expert_counts,
                     int32_t *expert_offsets, uint32_t *meta, int32_t *row_src,
                     int32_t *pair_slot, uint8_t *drop_mask) {
@@ -200,9 +206,13 @@ uint32_t orc_layout(int32_t N, int32_t k, int32_t E, int32_t S, int64_t C,
         }
   }
 
-  /* 2. expert start rows: exclusive cumulative sum (packed) or e*Ce */
-  for (int32_t e = 0; e < E; ++e)
-    off[e + 1] = off[e] + (capacity_mode ? (int64_t)Ce : cnt[e]);
+  /* 2. expert start rows: exclusive cumulative sum of the (padded) counts
+   *    (packed) or e*Ce */
+  for (int32_t e = 0; e < E; ++e) {
+    int64_t block = cnt[e];
+    if (!capacity_mode && pad > 1) block = (cnt[e] + pad - 1) / pad * pad;
+    off[e + 1] = off[e] + (capacity_mode ? (int64_t)Ce : block);
+  }
   for (int32_t e = 0; e <= E; ++e) expert_offsets[e] = (int32_t)off[e];
   for (int32_t e = 0; e < E; ++e)
     expert_counts[e] = (int32_t)(capacity_mode && cnt[e] > Ce ? Ce : cnt[e]);
@@ -238,19 +248,24 @@ uint32_t orc_layout(int32_t N, int32_t k, int32_t E, int32_t S, int64_t C,
     if (drop_mask) drop_mask[p] = (uint8_t)dropped;
   }
 
-  /* 5. [4, S] uint32 metadata in elements (rows * H) */
-  int64_t disp = 0;
+  /* 5. [4, S] uint32 metadata in elements (rows * H): per segment its rows
+   *    (the kept rows in capacity mode; the expert blocks, padding included,
+   *    in packed mode) and where they start */
   for (int32_t s = 0; s < S; ++s) {
-    int64_t seg_rows = 0;
-    for (int32_t e = s * L; e < (s + 1) * L; ++e) seg_rows += expert_counts[e];
+    int64_t seg_rows = 0, start;
+    if (capacity_mode) {
+      for (int32_t e = s * L; e < (s + 1) * L; ++e) seg_rows += expert_counts[e];
+      start = (int64_t)s * L * Ce;
+    } else {
+      seg_rows = off[(s + 1) * L] - off[s * L];
+      start = off[s * L];
+    }
     uint32_t count_el = (uint32_t)(seg_rows * H);
-    uint32_t displ_el =
-        capacity_mode ? (uint32_t)((int64_t)s * L * Ce * H) : (uint32_t)disp;
+    uint32_t displ_el = (uint32_t)(start * H);
     meta[0 * S + s] = count_el;
     meta[1 * S + s] = displ_el;
     meta[2 * S + s] = count_el;
     meta[3 * S + s] = displ_el;
-    disp += seg_rows * H;
   }
 
   free(cnt);
@@ -358,6 +373,24 @@ void orc_permute_nvfp4(int64_t rows, int32_t H, const uint16_t *hidden,
       }
     }
   }
+}
+
+/* Scale-factor atom layout: see oracle.h. */
+void orc_swizzle_scales(int64_t rows, int32_t nsf, const uint8_t *linear,
+                        uint8_t *out) {
+  const int32_t atom_rows = 32 * 4;            /* SF_ATOM_M[0] * 4 row groups */
+  const int32_t atom_cols = 4;                 /* SF_ATOM_M[1]                */
+  const int32_t row_stride = atom_cols * 4;    /* SF_ROW_STRIDE_LOCAL = 16    */
+  const int32_t atom_bytes = 32 * row_stride;  /* SF_ATOM_ELEMS_LOCAL = 512   */
+  const int64_t row_tiles = (rows + atom_rows - 1) / atom_rows;
+  const int64_t col_tiles = (nsf + atom_cols - 1) / atom_cols;
+  memset(out, 0, (size_t)(row_tiles * col_tiles * atom_bytes));
+  for (int64_t m = 0; m < rows; ++m)
+    for (int32_t c = 0; c < nsf; ++c) {
+      int64_t atom = (m / atom_rows) * col_tiles + c / atom_cols;
+      int64_t inner = (m % 32) * row_stride + ((m / 32) % 4) * 4 + c % atom_cols;
+      out[atom * atom_bytes + inner] = linear[m * nsf + c];
+    }
 }
 
 /* ------------------------------------------------------------------ */

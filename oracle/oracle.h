@@ -69,14 +69,28 @@ void orc_e2m1_from_f32_n(const float *in, uint8_t *out, int64_t n);
  * ids[N*k] int32 (row-major [N,k]); E experts in S contiguous segments of
  * L = E/S experts.  expert_capacity Ce == 0 selects packed (dropless) mode
  * with C = recv_capacity rows; Ce > 0 selects the capacity layout [E,Ce].
+ * pad > 1 (packed mode only) starts every expert's rows at a multiple of pad
+ * (NeMo TokenDispatcherConfig.moe_router_expert_pad_multiple).
  * Outputs: expert_counts[E], expert_offsets[E+1], meta[4*S] (row-major
  * [4,S]), row_src[rows] (rows = C, or E*Ce), pair_slot[N*k], drop_mask[N*k]
  * (may be NULL).  Returns status bits.                                   */
 uint32_t orc_layout(int32_t N, int32_t k, int32_t E, int32_t S, int64_t C,
-                    int32_t Ce, uint32_t flags, int32_t H,
+                    int32_t Ce, int32_t pad, uint32_t flags, int32_t H,
                     const int32_t *ids, int32_t *expert_counts,
                     int32_t *expert_offsets, uint32_t *meta, int32_t *row_src,
                     int32_t *pair_slot, uint8_t *drop_mask);
+
+/* ---- block-scale atom layout ------------------------------------------
+ * Mojo MAX ep_comm: SF_ROW_STRIDE_LOCAL = SF_ATOM_M[1] * 4 and
+ * SF_ATOM_ELEMS_LOCAL = SF_ATOM_M[0] * SF_ROW_STRIDE_LOCAL, with SF_ATOM_M
+ * read as (32, 4): an atom holds the scales of 128 rows x 4 scale columns in
+ * 512 bytes.  Scale (m, c) of a [rows, nsf] matrix goes to atom
+ * (m / 128, c / 4) -- atoms row-tile-major, ceil(nsf / 4) per row tile --
+ * at byte (m % 32) * 16 + ((m / 32) % 4) * 4 + c % 4 of the atom.
+ * out has ceil(rows/128)*128 * ceil(nsf/4)*4 bytes; bytes no scale maps to
+ * are zero.                                                              */
+void orc_swizzle_scales(int64_t rows, int32_t nsf, const uint8_t *linear,
+                        uint8_t *out);
 
 /* ---- permute: out row r = hidden row row_src[r], or zeros ------------- */
 void orc_permute_bf16(int64_t rows, int32_t H, const uint16_t *hidden,

@@ -18,7 +18,7 @@ from combine_topk_ids_scan_b200.inputs import make_workload
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
-def numpy_layout(ids, E, S, H, C=0, Ce=0):
+def numpy_layout(ids, E, S, H, C=0, Ce=0, pad=0):
     """Second formulation of the layout through numpy's stable sort."""
     N, k = ids.shape
     flat = ids.reshape(-1).astype(np.int64)
@@ -40,17 +40,22 @@ def numpy_layout(ids, E, S, H, C=0, Ce=0):
         offsets = np.arange(E + 1) * Ce
     else:
         rows = C
+        block = cnt if pad <= 1 else -(-cnt // pad) * pad     # counts rounded up
+        start = np.concatenate([[0], np.cumsum(block)])
         pos = np.full(flat.size, -1, np.int64)
-        pos[order] = np.arange(order.size)
+        pos[valid] = start[flat[valid]] + rank[valid]
         keep = valid & (pos < C)
         slot[keep] = pos[keep]
         drop[valid & ~keep] = 1
         counts = cnt
-        offsets = first
+        offsets = start
     row_src = np.full(rows, -1, np.int64)
     row_src[slot[slot >= 0]] = np.nonzero(slot >= 0)[0] // k
     L = E // S
-    seg_rows = counts.reshape(S, L).sum(axis=1)
+    if Ce > 0:
+        seg_rows = counts.reshape(S, L).sum(axis=1)
+    else:
+        seg_rows = (offsets[1:] - offsets[:-1]).reshape(S, L).sum(axis=1)
     m0 = seg_rows * H
     m1 = (np.arange(S) * L * Ce * H) if Ce > 0 else np.concatenate([[0], np.cumsum(m0)[:-1]])
     meta = np.stack([m0, m1, m0, m1]).astype(np.uint32)
@@ -84,6 +89,11 @@ def test_hand_worked_example(orc):
                 "drop_mask"):
         assert np.array_equal(getattr(lay, key).reshape(-1).astype(np.int64),
                               fx["capacity." + key]), key
+    lay = orc.layout(ids, 4, 2, 10, recv_capacity=16, expert_pad_multiple=4)
+    assert lay.status == 0
+    for key in ("expert_counts", "expert_offsets", "pair_slot", "row_src", "meta"):
+        assert np.array_equal(getattr(lay, key).reshape(-1).astype(np.int64),
+                              fx["pad4." + key]), key
 
 
 @pytest.mark.parametrize("N,k,E,S", [(1, 1, 2, 1), (2, 2, 2, 2), (3, 2, 3, 1), (2, 3, 2, 1)])
@@ -104,6 +114,9 @@ def test_brute_force_all_id_matrices(orc, N, k, E, S):
             lay = orc.layout(ids, E, S, H, expert_capacity=Ce)
             check_equal(lay, numpy_layout(ids, E, S, H, Ce=Ce))
             assert lay.status == 0
+        for pad, C in ((2, N * k * 2), (3, N * k + 2)):
+            lay = orc.layout(ids, E, S, H, recv_capacity=C, expert_pad_multiple=pad)
+            check_equal(lay, numpy_layout(ids, E, S, H, C=C, pad=pad))
 
 
 def test_id_range_and_duplicates_status(orc):
@@ -193,3 +206,27 @@ def test_capacity_mode_decode_workload(orc):
         assert np.all(s[5:] == -1)
     m = lay.meta.astype(np.int64)
     assert np.array_equal(m[1], np.arange(w.S) * (w.E // w.S) * 5 * w.H)
+
+
+@pytest.mark.parametrize("pad", [1, 4, 16, 128])
+def test_expert_padding_invariants(orc, pad):
+    """Every expert block starts at a multiple of pad and holds the expert's
+    rows first, then padding; nothing else changes."""
+    w = make_workload("mid_zipf", n_tokens=1024, with_expert_out=False, with_hidden=False)
+    C = w.N * w.k + w.E * pad
+    lay = orc.layout(w.ids, w.E, w.S, w.H, recv_capacity=C, expert_pad_multiple=pad)
+    assert lay.status == 0
+    check_equal(lay, numpy_layout(w.ids, w.E, w.S, w.H, C=C, pad=pad))
+    off = lay.expert_offsets.astype(np.int64)
+    assert np.all(off % max(pad, 1) == 0)
+    for e in range(w.E):
+        n = lay.expert_counts[e]
+        blk = lay.row_src[off[e]:off[e + 1]]
+        assert np.all(blk[:n] >= 0) and np.all(blk[n:] == -1)
+        assert off[e + 1] - off[e] == -(-n // max(pad, 1)) * max(pad, 1)
+    base = orc.layout(w.ids, w.E, w.S, w.H, recv_capacity=C)
+    # the source order inside each expert is the unpadded one
+    for e in range(w.E):
+        n = lay.expert_counts[e]
+        assert np.array_equal(lay.row_src[off[e]:off[e] + n],
+                              base.row_src[base.expert_offsets[e]:base.expert_offsets[e] + n])
