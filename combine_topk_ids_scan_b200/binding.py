@@ -29,6 +29,7 @@ MOE_STATUS_TIMEOUT = 8
 
 MOE_FLAG_CHECK_DUPLICATES = 1
 MOE_FLAG_LAYOUT_TWO_PASS = 2
+MOE_FLAG_NVFP4_SWIZZLED_SCALES = 4
 MOE_FLAG_TEST_STALL_SCAN = 0x80000000
 
 MOE_MAX_EXPERTS = 2048
@@ -53,7 +54,7 @@ class moe_problem(ctypes.Structure):
                 ("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("num_segments", ctypes.c_int32), ("expert_capacity", ctypes.c_int32),
                 ("recv_capacity", ctypes.c_int64), ("flags", ctypes.c_uint32),
-                ("reserved", ctypes.c_uint32)]
+                ("expert_pad_multiple", ctypes.c_int32)]
 
 
 @dataclass
@@ -67,11 +68,12 @@ class Problem:
     recv_capacity: int = 0
     expert_capacity: int = 0
     flags: int = 0
+    expert_pad_multiple: int = 0
 
     def c(self) -> moe_problem:
         return moe_problem(self.num_tokens, self.hidden, self.num_experts, self.top_k,
                            self.num_segments, self.expert_capacity, self.recv_capacity,
-                           self.flags & 0xFFFFFFFF, 0)
+                           self.flags & 0xFFFFFFFF, self.expert_pad_multiple)
 
 
 _lib = None
@@ -200,6 +202,11 @@ def moe_combine(prob: Problem, expert_out, gates, pair_slot, out, stream=None) -
                               _ptr(out), _stream(stream)), "moe_combine")
 
 
+def nvfp4_swizzled_scale_bytes(rows: int, hidden: int) -> int:
+    """Bytes of NVFP4 scales in the 128x4 atom layout (see moe_dc.h)."""
+    return max(1, -(-rows // 128) * 128 * (-(-hidden // 64) * 4))
+
+
 # ----------------------------------------------------------------- buffers
 class Buffers:
     """Device buffers for one problem (allocated by torch; the library itself
@@ -227,8 +234,12 @@ class Buffers:
             self.scales_fp8 = torch.empty((max(rows, 1), max(H // 128, 1)), dtype=torch.float32,
                                           device=device)
             self.out_fp4 = torch.empty((max(rows, 1), H // 2), dtype=u8, device=device)
-            self.scales_fp4 = torch.empty((max(rows, 1), max(H // 16, 1)), dtype=u8,
-                                          device=device)
+            if prob.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES:
+                self.scales_fp4 = torch.empty(nvfp4_swizzled_scale_bytes(rows, H), dtype=u8,
+                                              device=device)
+            else:
+                self.scales_fp4 = torch.empty((max(rows, 1), max(H // 16, 1)), dtype=u8,
+                                              device=device)
 
 
 def layout(prob: Problem, topk_ids: torch.Tensor, buf: Buffers, stream=None) -> None:

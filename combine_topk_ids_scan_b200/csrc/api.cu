@@ -41,7 +41,7 @@ moe_status make_shape(const moe_problem *p, moe::Shape *s) {
   if (!p) return MOE_ERR_INVALID_ARG;
   if (p->num_tokens < 0 || p->hidden <= 0 || p->num_experts <= 0 || p->top_k <= 0 ||
       p->num_segments <= 0 || p->expert_capacity < 0 || p->recv_capacity < 0 ||
-      p->reserved != 0)
+      p->expert_pad_multiple < 0 || (p->expert_pad_multiple > 1 && p->expert_capacity > 0))
     return MOE_ERR_INVALID_ARG;
   if (p->num_experts > MOE_MAX_EXPERTS || p->top_k > MOE_MAX_TOPK ||
       p->num_experts % p->num_segments != 0)
@@ -57,9 +57,12 @@ moe_status make_shape(const moe_problem *p, moe::Shape *s) {
                                    : p->recv_capacity;
   s->P = (int64_t)p->num_tokens * p->top_k;
   s->flags = p->flags;
-  // slots are int32; the [4, S] table counts elements in uint32
-  if (s->rows > 2147483647ll || s->P > 2147483647ll) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (s->rows * s->H > kU32Max || s->P * s->H > kU32Max) return MOE_ERR_UNSUPPORTED_SHAPE;
+  s->pad = p->expert_pad_multiple > 1 ? p->expert_pad_multiple : 1;
+  // slots are int32; the [4, S] table counts elements in uint32; padded
+  // expert blocks add at most E * (pad - 1) rows
+  const int64_t padded = s->P + (int64_t)s->E * (s->pad - 1);
+  if (s->rows > 2147483647ll || padded > 2147483647ll) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s->rows * s->H > kU32Max || padded * s->H > kU32Max) return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
 
@@ -145,8 +148,9 @@ moe_status moe_permute_quant_nvfp4(const moe_problem *problem, const void *hidde
   if (!row_src || !out_e2m1 || !scales_e4m3 || !global_scale ||
       (s.P > 0 && (!hidden_states || !pair_slot)))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned(hidden_states, 16) || !aligned(out_e2m1, 16) || !aligned(scales_e4m3, 2) ||
-      !aligned(global_scale, 4))
+  const uintptr_t scale_align = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) ? 4 : 2;
+  if (!aligned(hidden_states, 16) || !aligned(out_e2m1, 16) ||
+      !aligned(scales_e4m3, scale_align) || !aligned(global_scale, 4))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_permute_nvfp4(s, hidden_states, row_src, pair_slot, global_scale,
                                              out_e2m1, scales_e4m3,
@@ -172,7 +176,7 @@ const char *moe_status_string(moe_status status) {
     case MOE_OK:
       return "ok";
     case MOE_ERR_INVALID_ARG:
-      return "invalid argument (null or misaligned pointer, negative size, reserved field)";
+      return "invalid argument (null or misaligned pointer, negative size, bad field)";
     case MOE_ERR_UNSUPPORTED_SHAPE:
       return "unsupported shape (size outside the library's limits)";
     case MOE_ERR_CUDA:

@@ -16,6 +16,7 @@ struct Shape {
   int64_t rows;  // rows of the dispatch output
   int64_t P;     // N * k pairs
   uint32_t flags;
+  int32_t pad;   // per-expert row multiple (1 = none)
 };
 
 // Layout workspace: control words, per-expert totals, scan tile states.

@@ -304,15 +304,17 @@ __device__ int32_t block_exclusive_scan(int32_t *v, int n) {
   return total;
 }
 
-// Expert start rows s_off[E+1] and kept rows s_kept[E] from the totals.
+// Expert start rows s_off[E+1] and kept rows s_kept[E] from the totals
+// (packed mode: each expert's block is its count rounded up to `pad`).
 template <int THREADS>
 __device__ void expert_offsets_from_totals(const int32_t *totals, bool have_totals, int32_t E,
-                                           int32_t Ce, int32_t *s_off, int32_t *s_kept) {
+                                           int32_t Ce, int32_t pad, int32_t *s_off,
+                                           int32_t *s_kept) {
   const bool capacity = Ce > 0;
   for (int e = threadIdx.x; e < E; e += THREADS) {
     const int32_t t = have_totals ? __ldcg(totals + e) : 0;
     s_kept[e] = capacity ? min(t, Ce) : t;
-    s_off[e] = capacity ? e * Ce : t;
+    s_off[e] = capacity ? e * Ce : (pad > 1 ? (t + pad - 1) / pad * pad : t);
   }
   __syncthreads();
   if (!capacity) {
@@ -325,19 +327,33 @@ __device__ void expert_offsets_from_totals(const int32_t *totals, bool have_tota
   __syncthreads();
 }
 
-// Padding rows of [r0, rows) in steps of `stride`, counts/offsets/meta when
-// `write_meta`, duplicate check for tokens [t0, t1) in steps of `tstride`.
+// Padding rows of [r0, rows) in steps of `stride` and counts/offsets/meta
+// when `write_meta`.
 template <int THREADS>
 __device__ void emit_common(int64_t r0, int64_t stride, int64_t rows, int32_t E, int32_t S,
-                            int32_t Ce, int32_t H, const int32_t *s_off, const int32_t *s_kept,
-                            int32_t *__restrict__ row_src, bool write_meta,
-                            int32_t *__restrict__ expert_counts,
+                            int32_t Ce, int32_t pad_multiple, int32_t H, const int32_t *s_off,
+                            const int32_t *s_kept, int32_t *__restrict__ row_src,
+                            bool write_meta, int32_t *__restrict__ expert_counts,
                             int32_t *__restrict__ expert_offsets, uint32_t *__restrict__ meta) {
   const bool capacity = Ce > 0;
   for (int64_t r = r0; r < rows; r += stride) {
     bool pad;
-    if (capacity) pad = (int32_t)(r % Ce) >= s_kept[r / Ce];
-    else pad = r >= (int64_t)s_off[E];
+    if (capacity) {
+      pad = (int32_t)(r % Ce) >= s_kept[r / Ce];
+    } else if (r >= (int64_t)s_off[E]) {
+      pad = true;
+    } else if (pad_multiple > 1) {
+      // the expert whose block holds r: last e with s_off[e] <= r
+      int lo = 0, hi = E - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if ((int64_t)s_off[mid] <= r) lo = mid;
+        else hi = mid - 1;
+      }
+      pad = r - s_off[lo] >= s_kept[lo];
+    } else {
+      pad = false;
+    }
     if (pad) row_src[r] = -1;
   }
   if (write_meta) {
@@ -347,7 +363,11 @@ __device__ void emit_common(int64_t r0, int64_t stride, int64_t rows, int32_t E,
     const int32_t L = E / S;
     for (int s = tid; s < S; s += THREADS) {
       int64_t seg_rows = 0;
-      for (int e = s * L; e < (s + 1) * L; ++e) seg_rows += s_kept[e];
+      if (capacity) {
+        for (int e = s * L; e < (s + 1) * L; ++e) seg_rows += s_kept[e];
+      } else {
+        seg_rows = (int64_t)s_off[(s + 1) * L] - s_off[s * L];  // blocks incl. padding
+      }
       const uint32_t count_el = (uint32_t)(seg_rows * H);
       const uint32_t displ_el = capacity ? (uint32_t)((int64_t)s * L * Ce * H)
                                          : (uint32_t)((int64_t)s_off[s * L] * H);
@@ -406,7 +426,7 @@ __device__ void finish_and_clean(uint32_t bits, uint32_t *s_status, uint32_t *ct
 struct LayoutArgs {
   const int32_t *ids;
   int64_t P;
-  int32_t N, k, E, S, Ce, H;
+  int32_t N, k, E, S, Ce, H, pad;
   int64_t C, rows;
   uint32_t flags;
   int32_t num_tiles;
@@ -454,7 +474,8 @@ __device__ void emit_step(const LayoutArgs &a, int64_t gtid, int64_t gstride,
                           uint32_t *s_status, int64_t n_states) {
   __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_kept[MOE_MAX_EXPERTS];
-  expert_offsets_from_totals<THREADS>(a.totals, a.num_tiles > 0, a.E, a.Ce, s_off, s_kept);
+  expert_offsets_from_totals<THREADS>(a.totals, a.num_tiles > 0, a.E, a.Ce, a.pad, s_off,
+                                      s_kept);
   const bool capacity = a.Ce > 0;
   uint32_t bits = 0;
   for (int64_t p = gtid; p < a.P; p += gstride) {
@@ -467,8 +488,8 @@ __device__ void emit_step(const LayoutArgs &a, int64_t gtid, int64_t gstride,
     if (a.drop_mask) a.drop_mask[p] = dropped;
     if (slot >= 0) a.row_src[slot] = (int32_t)p / a.k;
   }
-  emit_common<THREADS>(gtid, gstride, a.rows, a.E, a.S, a.Ce, a.H, s_off, s_kept, a.row_src,
-                       blockIdx.x == 0, a.expert_counts, a.expert_offsets, a.meta);
+  emit_common<THREADS>(gtid, gstride, a.rows, a.E, a.S, a.Ce, a.pad, a.H, s_off, s_kept,
+                       a.row_src, blockIdx.x == 0, a.expert_counts, a.expert_offsets, a.meta);
   if (a.flags & MOE_FLAG_CHECK_DUPLICATES)
     bits |= duplicate_bits(a.ids, gtid, a.N, gstride, a.k, a.E);
   finish_and_clean<THREADS>(bits, s_status, a.ctrl, a.totals, a.tiles, n_states, a.E,
@@ -580,6 +601,7 @@ cudaError_t launch_layout(const Shape &s, const int32_t *ids, int32_t *expert_co
   a.S = s.S;
   a.Ce = s.Ce;
   a.H = s.H;
+  a.pad = s.pad;
   a.C = s.C;
   a.rows = s.rows;
   a.flags = s.flags;

@@ -215,20 +215,62 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float *f, float gs, uint32
   return sq;
 }
 
+// Block-scale atom layout (Mojo MAX ep_comm SF_ATOM_M = (32, 4),
+// SF_ROW_STRIDE_LOCAL = 16, SF_ATOM_ELEMS_LOCAL = 512): byte of scale (m, c)
+// when a 128-row tile spans `col_tiles` atoms.
+__device__ __forceinline__ int64_t sf_atom_offset(int64_t m, int32_t c, int32_t col_tiles) {
+  return ((m >> 7) * col_tiles + (c >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (c & 3);
+}
+
+// Swizzled-scale padding for the 32 rows [32*c, 32*c + 32) of the padded row
+// range: rows without a source (padding rows of the output and the rows that
+// only complete the last 128-row tile) get zero scales (and zero codes when
+// they are output rows); every output row gets zeros in the scale columns
+// that only complete its last group of 4.
+__device__ __forceinline__ void zero_swizzled_padding(int64_t c, int lane,
+                                                      const int32_t *__restrict__ row_src,
+                                                      int64_t rows, int64_t rows_padded,
+                                                      uint4 *q, int32_t q_vecs, uint8_t *scales,
+                                                      int32_t nsf) {
+  const int32_t groups = (nsf + 3) / 4;
+  const int64_t r = c * kWarp + lane;
+  const bool in_range = r < rows_padded;
+  const bool no_src = in_range && (r >= rows || __ldg(row_src + r) < 0);
+  uint32_t m = __ballot_sync(kFull, no_src);
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+  while (m) {
+    const int j = __ffs(m) - 1;
+    m &= m - 1;
+    const int64_t row = c * kWarp + j;
+    if (row < rows) {
+      uint4 *dst = q + row * q_vecs;
+      for (int v = lane; v < q_vecs; v += kWarp) st_v4(dst + v, zero);
+    }
+    for (int g = lane; g < groups; g += kWarp)
+      *reinterpret_cast<uint32_t *>(scales + sf_atom_offset(row, 4 * g, groups)) = 0u;
+  }
+  if ((nsf & 3) != 0 && in_range && !no_src)  // nsf is even: two columns complete the group
+    *reinterpret_cast<uint16_t *>(scales + sf_atom_offset(r, nsf, groups)) = 0;
+}
+
 __global__ void __launch_bounds__(kThreads)
     permute_nvfp4_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                          const int32_t *__restrict__ pair_slot,
                          const float *__restrict__ global_scale, uint8_t *__restrict__ q,
                          uint8_t *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
-                         int32_t H, int32_t chunks) {
+                         int32_t H, int32_t chunks, bool swizzled) {
   const int lane = threadIdx.x % kWarp;
   const int64_t w = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
   const int32_t vecs = H / 8;
   const int32_t qrow = H / 2, srow = H / 16;
   if (w >= units) {
-    zero_padding_rows(w - units, lane, row_src, rows, reinterpret_cast<uint4 *>(q), qrow / 16,
-                      reinterpret_cast<uint16_t *>(scales), srow / 2);
+    if (swizzled)
+      zero_swizzled_padding(w - units, lane, row_src, rows, (rows + 127) / 128 * 128,
+                            reinterpret_cast<uint4 *>(q), qrow / 16, scales, srow);
+    else
+      zero_padding_rows(w - units, lane, row_src, rows, reinterpret_cast<uint4 *>(q),
+                        qrow / 16, reinterpret_cast<uint16_t *>(scales), srow / 2);
     return;
   }
   const int64_t t = w / chunks;
@@ -262,15 +304,19 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t s = __shfl_sync(kFull, my_slot, j);
     if (active) {
       st_v4(reinterpret_cast<uint4 *>(q + s * qrow + col / 2), codes);
-      *reinterpret_cast<uint16_t *>(scales + s * srow + col / 16) = sq;
+      const int64_t so = swizzled ? sf_atom_offset(s, col / 16, (srow + 3) / 4)
+                                  : s * srow + col / 16;
+      *reinterpret_cast<uint16_t *>(scales + so) = sq;
     }
   }
 }
 
-// One warp per unit: token units first, then one warp per 32 rows for the
-// padding check.
-inline int64_t unit_blocks(const Shape &s, int32_t chunks) {
-  const int64_t warps = (int64_t)s.N * chunks + (s.rows + kWarp - 1) / kWarp;
+// One warp per unit: token units first, then one warp per 32 rows (of
+// `check_rows`, the output rows or, for swizzled scales, the rows rounded up
+// to the 128-row tile) for the padding check.
+inline int64_t unit_blocks(const Shape &s, int32_t chunks, int64_t check_rows = -1) {
+  if (check_rows < 0) check_rows = s.rows;
+  const int64_t warps = (int64_t)s.N * chunks + (check_rows + kWarp - 1) / kWarp;
   return (warps + kThreads / kWarp - 1) / (kThreads / kWarp);
 }
 
@@ -304,9 +350,11 @@ cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32
                                  uint8_t *q, uint8_t *scales, cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
   const int32_t chunks = chunks_of(s.H);
-  permute_nvfp4_kernel<<<(unsigned)unit_blocks(s, chunks), kThreads, 0, stream>>>(
+  const bool swizzled = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) != 0;
+  const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
+  permute_nvfp4_kernel<<<(unsigned)unit_blocks(s, chunks, check_rows), kThreads, 0, stream>>>(
       static_cast<const uint4 *>(hidden), row_src, pair_slot, global_scale, q, scales, s.N, s.k,
-      s.rows, s.H, chunks);
+      s.rows, s.H, chunks, swizzled);
   return cudaGetLastError();
 }
 

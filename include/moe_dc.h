@@ -83,6 +83,10 @@ enum {
    * cooperative kernel applies.  Results are identical; for testing and
    * tuning. */
   MOE_FLAG_LAYOUT_TWO_PASS = 2u,
+  /* moe_permute_quant_nvfp4 writes the E4M3 scales in the block-scale atom
+   * layout of NVIDIA block-scaled tensor-core operands instead of row-major
+   * (see moe_permute_quant_nvfp4). */
+  MOE_FLAG_NVFP4_SWIZZLED_SCALES = 4u,
   /* Test hook: the first scan tile never publishes its counts, so every
    * later tile's bounded wait runs out and MOE_STATUS_TIMEOUT is reported.
    * Results are invalid; used only to test the timeout path. */
@@ -106,7 +110,12 @@ typedef struct moe_problem {
   int64_t recv_capacity;   /* C rows of the packed layout (ignored when
                               Ce > 0)                                      */
   uint32_t flags;          /* MOE_FLAG_*                                   */
-  uint32_t reserved;       /* must be 0                                    */
+  int32_t expert_pad_multiple; /* packed mode: 0 or 1 = experts packed back
+                              to back; m > 1 = every expert's block of rows
+                              is its count rounded up to a multiple of m
+                              (NeMo moe_router_expert_pad_multiple), so each
+                              expert starts at a multiple of m; must be 0
+                              in capacity mode                             */
 } moe_problem;
 
 /* Rows of the dispatch output: recv_capacity, or E * expert_capacity.
@@ -141,15 +150,19 @@ MOE_API size_t moe_workspace_bytes(const moe_problem *problem);
  *   expert_counts  int32 [E]: routed pairs per expert (packed: the true
  *                  count, even past recv_capacity; capacity: min(count, Ce)).
  *   expert_offsets int32 [E+1]: first row of each expert (packed: exclusive
- *                  cumulative sum of expert_counts, [E] = total; capacity:
- *                  e*Ce).
+ *                  cumulative sum of expert_counts, each rounded up to
+ *                  expert_pad_multiple when that is > 1, [E] = total;
+ *                  capacity: e*Ce).
  *   meta           uint32 [4, S] row-major, in elements (rows * H): row 0
- *                  send counts per segment, row 1 send displacements
- *                  (packed: exclusive cumulative sum of row 0; capacity:
- *                  s*L*Ce*H), rows 2-3 the receive counts / displacements,
- *                  equal to rows 0-1 on one GPU.
- *   row_src        int32 [rows]: source token of each row, -1 for padding.
- *                  Within an expert rows follow ascending pair index t*k+j.
+ *                  send counts per segment (packed: the segment's expert
+ *                  blocks, padding included; capacity: kept rows), row 1
+ *                  send displacements (packed: exclusive cumulative sum of
+ *                  row 0; capacity: s*L*Ce*H), rows 2-3 the receive counts /
+ *                  displacements, equal to rows 0-1 on one GPU.
+ *   row_src        int32 [rows]: source token of each row, -1 for padding
+ *                  (rows past the total and, with expert_pad_multiple > 1,
+ *                  the tail of each expert's block).  Within an expert rows
+ *                  follow ascending pair index t*k+j.
  *   pair_slot      int32 [N, k]: row of each pair, -1 when the pair is
  *                  masked, out of range, dropped (capacity mode) or beyond
  *                  recv_capacity (packed mode).
@@ -158,8 +171,9 @@ MOE_API size_t moe_workspace_bytes(const moe_problem *problem);
  *   status         uint32 device word, overwritten with this call's
  *                  MOE_STATUS_* bits when the call's kernels complete.
  *   workspace      moe_workspace_bytes() bytes, see there.
- * Host checks: sizes within limits, E % S == 0, rows*H and N*k*H fit in
- * uint32 (the metadata is uint32 elements), required pointers non-null. */
+ * Host checks: sizes within limits, E % S == 0, rows*H and (N*k +
+ * E*(expert_pad_multiple-1))*H fit in uint32 (the metadata is uint32
+ * elements), required pointers non-null. */
 MOE_API moe_status moe_dispatch_layout(const moe_problem *problem, const int32_t *topk_ids,
                                int32_t *expert_counts, int32_t *expert_offsets,
                                uint32_t *meta, int32_t *row_src, int32_t *pair_slot,
@@ -229,7 +243,16 @@ MOE_API moe_status moe_permute_quant_fp8(const moe_problem *problem, const void 
  * to nearest even with saturation to +-6, or 0 when d == 0.  Element 2m is
  * the low nibble of byte m.  Padding rows are all zero.
  *   out_e2m1     uint8 [rows, H/2] (16-byte aligned)
- *   scales_e4m3  uint8 [rows, H/16] (2-byte aligned), linear row-major
+ *   scales_e4m3  uint8 [rows, H/16] (2-byte aligned), linear row-major; or,
+ *                with MOE_FLAG_NVFP4_SWIZZLED_SCALES, the block-scale atom
+ *                layout (Mojo MAX ep_comm SF_ATOM_M, SF_ROW_STRIDE_LOCAL,
+ *                SF_ATOM_ELEMS_LOCAL, with SF_ATOM_M = (32, 4)): atoms of
+ *                128 rows x 4 scale columns in 512 bytes, atoms row-tile
+ *                major, ceil(H/64) atoms per 128-row tile; scale (m, c) at
+ *                byte ((m/128)*ceil(H/64) + c/4)*512 + (m%32)*16 +
+ *                ((m/32)%4)*4 + c%4.  The buffer then holds
+ *                ceil(rows/128)*128 * ceil(H/64)*4 bytes (4-byte aligned),
+ *                every one of them written (zero where no scale maps).
  * Requires H % 32 == 0. */
 MOE_API moe_status moe_permute_quant_nvfp4(const moe_problem *problem, const void *hidden_states,
                                    const int32_t *row_src, const int32_t *pair_slot,

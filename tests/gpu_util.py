@@ -16,10 +16,11 @@ def bf16_np(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def problem_of(w, flags: int = 0) -> B.Problem:
+def problem_of(w, flags: int = 0, pad: int = 0) -> B.Problem:
     return B.Problem(num_tokens=w.N, hidden=w.H, num_experts=w.E, top_k=w.k,
                      num_segments=w.S, recv_capacity=w.recv_capacity,
-                     expert_capacity=w.expert_capacity, flags=flags)
+                     expert_capacity=w.expert_capacity, flags=flags,
+                     expert_pad_multiple=pad)
 
 
 class GpuRun:
@@ -27,8 +28,8 @@ class GpuRun:
     where the shape allows them, combine)."""
 
     def __init__(self, w, flags: int = 0, quant: bool = True, combine: bool = True,
-                 expert_out: np.ndarray | None = None):
-        prob = problem_of(w, flags)
+                 expert_out: np.ndarray | None = None, pad: int = 0):
+        prob = problem_of(w, flags, pad)
         self.prob = prob
         buf = B.Buffers(prob)
         self.buf = buf
@@ -70,6 +71,9 @@ class GpuRun:
             self.s8 = buf.scales_fp8.cpu().numpy()[:rows]
         if self.has_fp4:
             self.q4 = buf.out_fp4.cpu().numpy()[:rows]
-            self.s4 = buf.scales_fp4.cpu().numpy()[:rows]
+            if flags & B.MOE_FLAG_NVFP4_SWIZZLED_SCALES:
+                self.s4 = buf.scales_fp4.cpu().numpy().reshape(-1)   # atom layout, flat
+            else:
+                self.s4 = buf.scales_fp4.cpu().numpy()[:rows]
         if combine and w.N > 0:
             self.y = bf16_np(self.y_dev)

@@ -99,7 +99,9 @@ def test_payload_shape_rules(lib):
                   ("moe_permute_quant_nvfp4", 7), ("moe_combine", 5)):
         assert _call(lib, fn, p, n) == B.MOE_ERR_INVALID_ARG, fn      # null pointers
     assert lib.moe_permute(None, *([None] * 5)) == B.MOE_ERR_INVALID_ARG
-    bad = B.moe_problem(10, 128, 8, 2, 2, 0, 20, 0, 7)                   # reserved != 0
+    bad = B.moe_problem(10, 128, 8, 2, 2, 0, 20, 0, -3)                  # negative pad
+    assert lib.moe_combine(ctypes.byref(bad), *([None] * 5)) == B.MOE_ERR_INVALID_ARG
+    bad = B.moe_problem(10, 128, 8, 2, 2, 4, 0, 0, 8)                    # pad with Ce
     assert lib.moe_combine(ctypes.byref(bad), *([None] * 5)) == B.MOE_ERR_INVALID_ARG
 
 

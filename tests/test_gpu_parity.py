@@ -56,9 +56,10 @@ def custom(N, H, E, k, S, C=None, Ce=0, ids=None, seed=0, p_mask=0.0, p_bad=0.0,
                     gates=gates, hidden=hidden, expert_out=X, global_scale=gs, seed=seed)
 
 
-def oracle_layout(orc, w, flags=0):
+def oracle_layout(orc, w, flags=0, pad=0):
     return orc.layout(w.ids, w.E, w.S, w.H, recv_capacity=w.recv_capacity,
-                      expert_capacity=w.expert_capacity, flags=flags)
+                      expert_capacity=w.expert_capacity, flags=flags,
+                      expert_pad_multiple=pad)
 
 
 def assert_layout(run, ref):
@@ -383,3 +384,50 @@ def test_nvfp4_rounding_ties_and_near_ties(orc, gs):
     q, s = orc.permute_nvfp4(w.hidden, ref.row_src, w.global_scale)
     assert np.array_equal(run.s4, s)
     assert np.array_equal(run.q4, q)
+
+
+# ------------------------------------------------------------ expert padding
+PAD_EDGE = {
+    "pad4_masked": (dict(N=1000, H=256, E=16, k=4, S=4, C=1000 * 4 + 16 * 3, p_mask=0.1), 4),
+    "pad128": (dict(N=2048, H=512, E=64, k=8, S=8, C=2048 * 8 + 64 * 127), 128),
+    "pad16_overflow": (dict(N=500, H=128, E=8, k=2, S=2, C=900), 16),
+    "pad3_badids": (dict(N=3001, H=96, E=40, k=3, S=5, C=3001 * 3 + 80, p_bad=0.02), 3),
+}
+
+
+@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
+@pytest.mark.parametrize("name", sorted(PAD_EDGE))
+def test_expert_padding_parity(orc, name, two_pass):
+    spec, pad = PAD_EDGE[name]
+    w = custom(seed=zlib.crc32(name.encode()) % 1000, **spec)
+    flags = B.MOE_FLAG_CHECK_DUPLICATES | (B.MOE_FLAG_LAYOUT_TWO_PASS if two_pass else 0)
+    run = GpuRun(w, flags=flags, pad=pad)
+    ref = oracle_layout(orc, w, flags=orc.FLAG_CHECK_DUPLICATES, pad=pad)
+    assert_layout(run, ref)
+    assert np.all(ref.expert_offsets % pad == 0)
+    assert_all_outputs(orc, w, run, ref)
+
+
+# ------------------------------------------------------------ scale atom layout
+@pytest.mark.parametrize("spec", [
+    dict(N=700, H=96, E=8, k=3, S=2, p_mask=0.2),          # 6 scale columns: column padding
+    dict(N=300, H=256, E=4, k=2, S=1, C=1000, p_mask=0.1),  # rows not a multiple of 128
+    dict(N=64, H=7168, E=256, k=8, S=8),
+], ids=["H96", "rows1000", "H7168"])
+def test_nvfp4_swizzled_scales(orc, spec):
+    w = custom(seed=5, **spec)
+    run = GpuRun(w, flags=B.MOE_FLAG_NVFP4_SWIZZLED_SCALES, combine=False)
+    ref = oracle_layout(orc, w)
+    assert_layout(run, ref)
+    q, s_lin = orc.permute_nvfp4(w.hidden, ref.row_src, w.global_scale)
+    assert np.array_equal(run.q4, q)
+    assert np.array_equal(run.s4, orc.swizzle_scales(s_lin))
+
+
+def test_nvfp4_swizzled_scales_workload(orc):
+    w = make_workload("mid_zipf")
+    run = GpuRun(w, flags=B.MOE_FLAG_NVFP4_SWIZZLED_SCALES, combine=False)
+    ref = oracle_layout(orc, w)
+    q, s_lin = orc.permute_nvfp4(w.hidden, ref.row_src, w.global_scale)
+    assert np.array_equal(run.q4, q)
+    assert np.array_equal(run.s4, orc.swizzle_scales(s_lin))
