@@ -64,6 +64,8 @@ def lib():
         L.orc_permute_fp8.argtypes = [i64, i32, vp, vp, vp, vp]
         L.orc_permute_nvfp4.argtypes = [i64, i32, vp, vp, f32, vp, vp]
         L.orc_combine.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp]
+        L.orc_permute_backward.argtypes = [i32, i32, i32, i64, vp, vp, vp]
+        L.orc_combine_backward.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp, vp, vp]
         for n in ("orc_bf16_from_f32_n", "orc_e4m3_from_f32_n", "orc_e2m1_from_f32_n"):
             getattr(L, n).argtypes = [vp, vp, i64]
         L.orc_e4m3_to_f32.restype = f32
@@ -194,3 +196,31 @@ def combine(expert_out_bits: np.ndarray, gates: np.ndarray,
     y = np.empty((N, H), np.uint16)
     lib().orc_combine(N, k, H, rows, _p(expert_out_bits), _p(gates), _p(pair_slot), _p(y))
     return y
+
+
+# ---------------------------------------------------------------- backward
+def permute_backward(grad_out_bits: np.ndarray, pair_slot: np.ndarray) -> np.ndarray:
+    """grad_out: uint16 [rows,H] bf16; returns grad_hidden uint16 [N,H]."""
+    grad_out_bits = np.ascontiguousarray(grad_out_bits, dtype=np.uint16)
+    pair_slot = np.ascontiguousarray(pair_slot, dtype=np.int32)
+    N, k = pair_slot.shape
+    rows, H = grad_out_bits.shape
+    gh = np.empty((N, H), np.uint16)
+    lib().orc_permute_backward(N, k, H, rows, _p(grad_out_bits), _p(pair_slot), _p(gh))
+    return gh
+
+
+def combine_backward(grad_y_bits: np.ndarray, expert_out_bits: np.ndarray, gates: np.ndarray,
+                     pair_slot: np.ndarray):
+    """Returns (grad_expert_out uint16 [rows,H], grad_gates float32 [N,k])."""
+    grad_y_bits = np.ascontiguousarray(grad_y_bits, dtype=np.uint16)
+    expert_out_bits = np.ascontiguousarray(expert_out_bits, dtype=np.uint16)
+    gates = np.ascontiguousarray(gates, dtype=np.float32)
+    pair_slot = np.ascontiguousarray(pair_slot, dtype=np.int32)
+    N, k = pair_slot.shape
+    rows, H = expert_out_bits.shape
+    gx = np.empty((rows, H), np.uint16)
+    gw = np.empty((N, k), np.float32)
+    lib().orc_combine_backward(N, k, H, rows, _p(grad_y_bits), _p(expert_out_bits), _p(gates),
+                               _p(pair_slot), _p(gx), _p(gw))
+    return gx, gw

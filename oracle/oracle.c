@@ -420,3 +420,51 @@ void orc_combine(int32_t N, int32_t k, int32_t H, int64_t rows,
     }
   }
 }
+
+/* ------------------------------------------------------------------ */
+/* Backward                                                            */
+/* ------------------------------------------------------------------ */
+
+/* The dispatch copies token t's row to the rows of its pairs, so the
+ * token's gradient is the sum of those rows' gradients (fp32, j in order,
+ * one rounding to bfloat16). */
+void orc_permute_backward(int32_t N, int32_t k, int32_t H, int64_t rows,
+                          const uint16_t *grad_out, const int32_t *pair_slot,
+                          uint16_t *grad_hidden) {
+  for (int32_t t = 0; t < N; ++t)
+    for (int32_t h = 0; h < H; ++h) {
+      float acc = 0.0f;
+      for (int32_t j = 0; j < k; ++j) {
+        int32_t s = pair_slot[(int64_t)t * k + j];
+        if (s < 0 || s >= rows) continue;
+        acc = acc + orc_bf16_to_f32(grad_out[(int64_t)s * H + h]);
+      }
+      grad_hidden[(int64_t)t * H + h] = orc_bf16_from_f32(acc);
+    }
+}
+
+/* y[t] = sum_j w[t,j] * x[slot(t,j)] (DeepSpeed combine), so
+ * d y / d x[slot(t,j)] = w[t,j] and d y / d w[t,j] = x[slot(t,j)]. */
+void orc_combine_backward(int32_t N, int32_t k, int32_t H, int64_t rows,
+                          const uint16_t *grad_y, const uint16_t *expert_out,
+                          const float *gates, const int32_t *pair_slot,
+                          uint16_t *grad_expert_out, float *grad_gates) {
+  for (int64_t i = 0; i < rows * H; ++i) grad_expert_out[i] = 0;
+  for (int32_t t = 0; t < N; ++t)
+    for (int32_t j = 0; j < k; ++j) {
+      int64_t p = (int64_t)t * k + j;
+      int32_t s = pair_slot[p];
+      if (s < 0 || s >= rows) {
+        grad_gates[p] = 0.0f;
+        continue;
+      }
+      double dot = 0.0;
+      for (int32_t h = 0; h < H; ++h) {
+        float g = orc_bf16_to_f32(grad_y[(int64_t)t * H + h]);
+        float x = orc_bf16_to_f32(expert_out[(int64_t)s * H + h]);
+        grad_expert_out[(int64_t)s * H + h] = orc_bf16_from_f32(gates[p] * g);
+        dot += (double)g * (double)x;
+      }
+      grad_gates[p] = (float)dot;
+    }
+}

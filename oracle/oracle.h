@@ -106,6 +106,23 @@ void orc_combine(int32_t N, int32_t k, int32_t H, int64_t rows,
                  const uint16_t *expert_out, const float *gates,
                  const int32_t *pair_slot, uint16_t *y);
 
+/* ---- backward -----------------------------------------------------------
+ * The gradients of the two data movements (training, NeMo token_dispatcher
+ * top-k probabilities [T, K] whose gradient flows back through combine):
+ *   permute backward: grad_hidden[t] = bf16(sum over j of grad_out[slot(t,j)])
+ *     in fp32, j in order, pairs without a row skipped;
+ *   combine backward: grad_expert_out[slot(t,j)] = bf16(w[t,j] * grad_y[t])
+ *     (fp32 product), rows no pair owns are zero; grad_gates[t,j] =
+ *     sum over h of grad_y[t,h] * expert_out[slot(t,j),h], evaluated in
+ *     float64 and rounded once to fp32 (0 for a pair without a row).      */
+void orc_permute_backward(int32_t N, int32_t k, int32_t H, int64_t rows,
+                          const uint16_t *grad_out, const int32_t *pair_slot,
+                          uint16_t *grad_hidden);
+void orc_combine_backward(int32_t N, int32_t k, int32_t H, int64_t rows,
+                          const uint16_t *grad_y, const uint16_t *expert_out,
+                          const float *gates, const int32_t *pair_slot,
+                          uint16_t *grad_expert_out, float *grad_gates);
+
 #ifdef __cplusplus
 }
 #endif
