@@ -308,7 +308,10 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
         if ev is not None:
             ev[5].record(stream)
 
-    launches_per_step = (2 if w.P > 0 else 1) + 4
+    # the layout is one cooperative launch up to 128 scan tiles of 4096 pairs,
+    # else a scan and an emit launch; then three permutes and the combine
+    tiles = (w.P + 4095) // 4096
+    launches_per_step = (1 if tiles <= 128 else 2) + 4
     for _ in range(args.warmup):
         flush_l2()
         step()
@@ -344,6 +347,98 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
         step_ms.append(e[0].elapsed_time(e[5]))
     ms = sum(step_ms) / len(step_ms)
     phase_ms = {p: sum(v) / len(v) for p, v in per.items()}
+
+    # ---- grouped-GEMM-ready dispatch (NEXT row f1): experts padded to 128
+    # rows, NVFP4 scales in the 128x4 atom layout; recv_capacity covers the
+    # worst case N*k + E*127 and every one of its rows is written
+    f1 = None
+    if args.next_rows:
+        pad = 128
+        prob_p = B.Problem(num_tokens=w.N, hidden=w.H, num_experts=w.E, top_k=w.k,
+                           num_segments=w.S, recv_capacity=w.N * w.k + w.E * (pad - 1),
+                           flags=B.MOE_FLAG_NVFP4_SWIZZLED_SCALES, expert_pad_multiple=pad)
+        buf_p = B.Buffers(prob_p, device=dev)
+        f1_steps = max(10, args.steps // 10)
+
+        def f1_step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            B.layout(prob_p, d_ids, buf_p)
+            if ev is not None:
+                ev[1].record(stream)
+            B.moe_permute_quant_nvfp4(prob_p, d_hidden, buf_p.row_src, buf_p.pair_slot, d_gs,
+                                      buf_p.out_fp4, buf_p.scales_fp4)
+            if ev is not None:
+                ev[2].record(stream)
+
+        for _ in range(3):
+            flush_l2()
+            f1_step()
+        f1_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                 for _ in range(f1_steps)]
+        torch.cuda.synchronize(dev)
+        for i in range(f1_steps):
+            flush_l2()
+            f1_step(f1_ev[i])
+        torch.cuda.synchronize(dev)
+        lay_us = 1e3 * sum(e[0].elapsed_time(e[1]) for e in f1_ev) / f1_steps
+        nv_us = 1e3 * sum(e[1].elapsed_time(e[2]) for e in f1_ev) / f1_steps
+        rows_p = buf_p.rows
+        nv_bytes = (2 * w.N * w.H + 4 * w.P + 4 * rows_p + rows_p * w.H // 2
+                    + B.nvfp4_swizzled_scale_bytes(rows_p, w.H) + 4)
+        padded_total = int(buf_p.expert_offsets[-1].item())
+        f1 = {"expert_pad_multiple": pad, "recv_capacity": rows_p,
+              "padded_rows_routed": padded_total, "steps": f1_steps,
+              "layout_us": round(lay_us, 2), "permute_nvfp4_swizzled_us": round(nv_us, 2),
+              "permute_nvfp4_swizzled_gbs": round(nv_bytes / (nv_us * 1e-6) / 1e9, 1),
+              "tokens_per_s": w.N / ((lay_us + nv_us) * 1e-6)}
+        del buf_p
+
+    # ---- backward (NEXT row f4): dispatch backward (gather-sum of the rows'
+    # gradients) and combine backward (scaled scatter + gate gradients)
+    f4 = None
+    if args.next_rows:
+        d_grows = d_x                      # a [C, H] bf16 gradient of the dispatch output
+        d_gtok = d_hidden                  # an [N, H] bf16 gradient of the combine output
+        d_gh = torch.empty_like(d_hidden)
+        d_gx = torch.empty_like(d_x)
+        d_gw = torch.empty_like(d_gates)
+        f4_steps = max(10, args.steps // 10)
+
+        def f4_step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            B.moe_permute_backward(prob, d_grows, buf.pair_slot, d_gh)
+            if ev is not None:
+                ev[1].record(stream)
+            B.moe_combine_backward(prob, d_gtok, d_x, d_gates, buf.pair_slot, buf.row_src, d_gx,
+                                   d_gw)
+            if ev is not None:
+                ev[2].record(stream)
+
+        for _ in range(3):
+            flush_l2()
+            f4_step()
+        f4_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                 for _ in range(f4_steps)]
+        torch.cuda.synchronize(dev)
+        for i in range(f4_steps):
+            flush_l2()
+            f4_step(f4_ev[i])
+        torch.cuda.synchronize(dev)
+        pb_us = 1e3 * sum(e[0].elapsed_time(e[1]) for e in f4_ev) / f4_steps
+        cb_us = 1e3 * sum(e[1].elapsed_time(e[2]) for e in f4_ev) / f4_steps
+        rows = buf.rows
+        pb_bytes = 2 * total_rows * w.H + 4 * w.P + 2 * w.N * w.H
+        cb_bytes = (2 * w.N * w.H + 2 * 2 * total_rows * w.H + 2 * (rows - total_rows) * w.H
+                    + 4 * w.P * 3 + 4 * rows)
+        f4 = {"steps": f4_steps,
+              "permute_backward_us": round(pb_us, 2),
+              "permute_backward_gbs": round(pb_bytes / (pb_us * 1e-6) / 1e9, 1),
+              "combine_backward_us": round(cb_us, 2),
+              "combine_backward_gbs": round(cb_bytes / (cb_us * 1e-6) / 1e9, 1),
+              "tokens_per_s": w.N / ((pb_us + cb_us) * 1e-6)}
+        del d_gh, d_gx, d_gw
 
     # ---- end to end through the public API from pinned host memory
     # Every step: H2D of the step's inputs (ids, hidden rows, gates, global
@@ -456,6 +551,8 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
                             "combined rows, status and counts; copies of neighbouring steps "
                             "overlap on separate streams"},
             "gpu_launches": launches_per_step * args.steps,
+            "next_rows": ({"f1_grouped_gemm_ready_nvfp4": f1, "f4_backward": f4}
+                          if f1 or f4 else None),
             "clocks": clocks, "layout_status": st,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -479,6 +576,8 @@ def main() -> int:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-tokens", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", dest="next_rows", action="store_false",
+                    help="skip the extra measurement of the grouped-GEMM-ready dispatch")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

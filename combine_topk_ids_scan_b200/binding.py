@@ -38,7 +38,8 @@ MOE_MAX_TOPK = 16
 # every symbol include/moe_dc.h declares
 EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout",
             "moe_dispatch_layout_noalloc", "moe_permute", "moe_permute_quant_fp8",
-            "moe_permute_quant_nvfp4", "moe_combine", "moe_status_string", "moe_version")
+            "moe_permute_quant_nvfp4", "moe_combine", "moe_permute_backward",
+            "moe_combine_backward", "moe_status_string", "moe_version")
 
 MOE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
@@ -107,6 +108,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
     L.moe_permute_quant_nvfp4.argtypes = [P] + [vp] * 7
     L.moe_combine.restype = ctypes.c_int
     L.moe_combine.argtypes = [P] + [vp] * 5
+    L.moe_permute_backward.restype = ctypes.c_int
+    L.moe_permute_backward.argtypes = [P] + [vp] * 4
+    L.moe_combine_backward.restype = ctypes.c_int
+    L.moe_combine_backward.argtypes = [P] + [vp] * 8
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_status_string.argtypes = [ctypes.c_int]
     L.moe_version.restype = ctypes.c_char_p
@@ -205,6 +210,22 @@ def moe_combine(prob: Problem, expert_out, gates, pair_slot, out, stream=None) -
 def nvfp4_swizzled_scale_bytes(rows: int, hidden: int) -> int:
     """Bytes of NVFP4 scales in the 128x4 atom layout (see moe_dc.h)."""
     return max(1, -(-rows // 128) * 128 * (-(-hidden // 64) * 4))
+
+
+def moe_permute_backward(prob: Problem, grad_out, pair_slot, grad_hidden, stream=None) -> None:
+    c = prob.c()
+    _check(load().moe_permute_backward(ctypes.byref(c), _ptr(grad_out), _ptr(pair_slot),
+                                       _ptr(grad_hidden), _stream(stream)),
+           "moe_permute_backward")
+
+
+def moe_combine_backward(prob: Problem, grad_y, expert_out, gates, pair_slot, row_src,
+                         grad_expert_out, grad_gates, stream=None) -> None:
+    c = prob.c()
+    _check(load().moe_combine_backward(ctypes.byref(c), _ptr(grad_y), _ptr(expert_out),
+                                       _ptr(gates), _ptr(pair_slot), _ptr(row_src),
+                                       _ptr(grad_expert_out), _ptr(grad_gates),
+                                       _stream(stream)), "moe_combine_backward")
 
 
 # ----------------------------------------------------------------- buffers

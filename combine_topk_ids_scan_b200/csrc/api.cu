@@ -171,6 +171,40 @@ moe_status moe_combine(const moe_problem *problem, const void *expert_out, const
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_permute_backward(const moe_problem *problem, const void *grad_out,
+                                const int32_t *pair_slot, void *grad_hidden,
+                                moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.N == 0) return MOE_OK;
+  if (!grad_hidden || !pair_slot || (s.rows > 0 && !grad_out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(grad_out, 16) || !aligned(grad_hidden, 16)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_combine(s, grad_out, nullptr, pair_slot, grad_hidden,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_combine_backward(const moe_problem *problem, const void *grad_y,
+                                const void *expert_out, const float *gates,
+                                const int32_t *pair_slot, const int32_t *row_src,
+                                void *grad_expert_out, float *grad_gates, moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.N == 0 && s.rows == 0) return MOE_OK;
+  if ((s.N > 0 && (!grad_y || !gates || !pair_slot || !grad_gates)) ||
+      (s.rows > 0 && (!expert_out || !row_src || !grad_expert_out)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(grad_y, 16) || !aligned(expert_out, 16) || !aligned(grad_expert_out, 16) ||
+      !aligned(gates, 4) || !aligned(grad_gates, 4))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_combine_backward(s, grad_y, expert_out, gates, pair_slot, row_src,
+                                                grad_expert_out, grad_gates,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char *moe_status_string(moe_status status) {
   switch (status) {
     case MOE_OK:

@@ -41,7 +41,9 @@ __global__ void __launch_bounds__(kThreads)
       const int32_t s = __ldg(pair_slot + t * k + lane);
       if (s >= 0 && s < rows) {
         my_slot = s;
-        my_w = __ldg(gates + t * k + lane);
+        // no gates: unit weights (the dispatch backward); fmaf(1, x, acc)
+        // is exactly acc + x
+        my_w = gates ? __ldg(gates + t * k + lane) : 1.0f;
       }
     }
     int64_t row[KMAX];
@@ -87,6 +89,97 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// Combine backward.  y[t] = sum_j w[t,j] x[slot(t,j)], so the expert rows get
+// grad_x[slot(t,j)] = bf16(w[t,j] * grad_y[t]) and the gates get
+// grad_w[t,j] = <grad_y[t], x[slot(t,j)]>.  One warp per token: per step a
+// lane loads one 16-byte vector of grad_y and of each live row, writes the
+// scaled gradient vector to each row and accumulates the dot products in
+// fp32 (elements in order, then the vectors in order); the lanes' partial
+// dots are summed by an xor-shuffle tree.  Rows no pair owns (row_src -1)
+// are zero-filled by a second phase, 32 rows per warp.
+template <int KMAX>
+__global__ void __launch_bounds__(kThreads)
+    combine_backward_kernel(const uint4 *__restrict__ grad_y, const uint4 *__restrict__ x,
+                            const float *__restrict__ gates,
+                            const int32_t *__restrict__ pair_slot,
+                            const int32_t *__restrict__ row_src, uint4 *__restrict__ grad_x,
+                            float *__restrict__ grad_gates, int32_t N, int32_t k, int64_t rows,
+                            int32_t vecs) {
+  const int lane = threadIdx.x % kWarp;
+  const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) / kWarp;
+
+  for (int64_t t = gw; t < N; t += nw) {
+    int32_t my_slot = -1;
+    float my_w = 0.0f;
+    if (lane < k) {
+      const int32_t s = __ldg(pair_slot + t * k + lane);
+      if (s >= 0 && s < rows) {
+        my_slot = s;
+        my_w = __ldg(gates + t * k + lane);
+      }
+    }
+    int64_t row[KMAX];
+    float w[KMAX], dot[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      row[j] = __shfl_sync(kFull, my_slot, j);
+      w[j] = __shfl_sync(kFull, my_w, j);
+      dot[j] = 0.0f;
+    }
+    const uint4 *gy = grad_y + t * vecs;
+    for (int v = lane; v < vecs; v += kWarp) {
+      const uint4 g4 = ld_stream_v4(gy + v);
+      uint4 in[KMAX];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        in[j] = row[j] >= 0 ? ld_stream_v4(x + row[j] * vecs + v) : make_uint4(0, 0, 0, 0);
+      const uint32_t ge[4] = {g4.x, g4.y, g4.z, g4.w};
+      float g[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        g[2 * i] = bf16lo(ge[i]);
+        g[2 * i + 1] = bf16hi(ge[i]);
+      }
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (row[j] < 0) continue;
+        const uint32_t xe[4] = {in[j].x, in[j].y, in[j].z, in[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          dot[j] = fmaf(g[2 * i], bf16lo(xe[i]), dot[j]);
+          dot[j] = fmaf(g[2 * i + 1], bf16hi(xe[i]), dot[j]);
+        }
+        st_v4(grad_x + row[j] * vecs + v,
+              make_uint4(pack_bf16x2(w[j] * g[0], w[j] * g[1]),
+                         pack_bf16x2(w[j] * g[2], w[j] * g[3]),
+                         pack_bf16x2(w[j] * g[4], w[j] * g[5]),
+                         pack_bf16x2(w[j] * g[6], w[j] * g[7])));
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      float d = dot[j];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(kFull, d, o);
+      if (lane == j && j < k) grad_gates[t * k + j] = row[j] >= 0 ? d : 0.0f;
+    }
+  }
+
+  // rows no pair owns carry no gradient
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+  for (int64_t c = gw; c * kWarp < rows; c += nw) {
+    const int64_t r = c * kWarp + lane;
+    uint32_t m = __ballot_sync(kFull, r < rows && __ldg(row_src + r) < 0);
+    while (m) {
+      const int j = __ffs(m) - 1;
+      m &= m - 1;
+      uint4 *dst = grad_x + (c * kWarp + j) * vecs;
+      for (int v = lane; v < vecs; v += kWarp) st_v4(dst + v, zero);
+    }
+  }
+}
+
 template <typename Kernel>
 int grid_for(Kernel kernel, int64_t N) {
   int per_sm = 0;
@@ -99,6 +192,32 @@ int grid_for(Kernel kernel, int64_t N) {
 }
 
 }  // namespace
+
+cudaError_t launch_combine_backward(const Shape &s, const void *grad_y, const void *expert_out,
+                                    const float *gates, const int32_t *pair_slot,
+                                    const int32_t *row_src, void *grad_expert_out,
+                                    float *grad_gates, cudaStream_t stream) {
+  const uint4 *gy = static_cast<const uint4 *>(grad_y);
+  const uint4 *x = static_cast<const uint4 *>(expert_out);
+  uint4 *gx = static_cast<uint4 *>(grad_expert_out);
+  const int32_t vecs = s.H / 8;
+  const int64_t work = std::max<int64_t>((int64_t)s.N, (s.rows + kWarp - 1) / kWarp);
+  if (work == 0) return cudaSuccess;
+  if (s.k <= 4) {
+    auto kernel = combine_backward_kernel<4>;
+    kernel<<<grid_for(kernel, work), kThreads, 0, stream>>>(gy, x, gates, pair_slot, row_src, gx,
+                                                            grad_gates, s.N, s.k, s.rows, vecs);
+  } else if (s.k <= 8) {
+    auto kernel = combine_backward_kernel<8>;
+    kernel<<<grid_for(kernel, work), kThreads, 0, stream>>>(gy, x, gates, pair_slot, row_src, gx,
+                                                            grad_gates, s.N, s.k, s.rows, vecs);
+  } else {
+    auto kernel = combine_backward_kernel<16>;
+    kernel<<<grid_for(kernel, work), kThreads, 0, stream>>>(gy, x, gates, pair_slot, row_src, gx,
+                                                            grad_gates, s.N, s.k, s.rows, vecs);
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const Shape &s, const void *expert_out, const float *gates,
                            const int32_t *pair_slot, void *out, cudaStream_t stream) {

@@ -47,8 +47,14 @@ cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32
                                  const int32_t *pair_slot, const float *global_scale,
                                  uint8_t *q, uint8_t *scales, cudaStream_t stream);
 
+// gates == nullptr: unit weights (the dispatch backward)
 cudaError_t launch_combine(const Shape &s, const void *expert_out, const float *gates,
                            const int32_t *pair_slot, void *out, cudaStream_t stream);
+
+cudaError_t launch_combine_backward(const Shape &s, const void *grad_y, const void *expert_out,
+                                    const float *gates, const int32_t *pair_slot,
+                                    const int32_t *row_src, void *grad_expert_out,
+                                    float *grad_gates, cudaStream_t stream);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

@@ -10,9 +10,14 @@
 // unit and exits.  Short warps over a grid of many blocks keep the write
 // stream denser than long-lived persistent warps do (measured on B200 for the
 // bf16 permute at N=8192, H=7168, k=8: 195 us persistent, 170 us with
-// 1024-element units, 166 us with 512).  Warps past the token units each
-// check 32 rows of row_src and zero-fill the rows whose source is -1.
+// 1024-element units, 166 us with 512).
 //
+// Padding rows (row_src -1) are zero-filled by padding warps placed first in
+// the grid: warp g checks the 32 rows [32g, 32g+32) and zero-fills those
+// without a source.  Scheduled first, they cost little when there is no
+// padding, and a long run of padding rows is written while the token units
+// run instead of as a tail (measured on B200, bf16 with 32K padding rows of
+// 98K: 240 us vs 336 us with the padding warps last).
 #include <algorithm>
 
 #include "common.cuh"
@@ -24,6 +29,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
+constexpr int kChunk = 1024;     // elements of one token per unit (quantisers)
+constexpr int kBf16Chunk = 512;  // elements of one token per unit (bf16)
 
 // Lane j < k holds pair (t, j)'s row, or -1 when the pair has no row in
 // [0, rows).  Returns the ballot of lanes holding a row.
@@ -38,27 +45,31 @@ __device__ __forceinline__ uint32_t load_token_slots(const int32_t *__restrict__
   return __ballot_sync(kFull, my_slot >= 0);
 }
 
-constexpr int kChunk = 1024;     // elements of one token per unit (quantisers)
-constexpr int kBf16Chunk = 512;  // elements of one token per unit (bf16)
+// Ballot of the rows of [32g, 32g+32) without a source: row_src -1, or at or
+// past `rows` but below `check_rows`.
+__device__ __forceinline__ uint32_t padding_mask(int64_t g, int lane,
+                                                 const int32_t *__restrict__ row_src,
+                                                 int64_t rows, int64_t check_rows) {
+  const int64_t r = g * kWarp + lane;
+  return __ballot_sync(kFull, r < check_rows && (r >= rows || __ldg(row_src + r) < 0));
+}
 
-// Zero-fill every row r in [32*c, 32*c + 32) whose source is -1; `row_vecs`
-// 16-byte vectors per row of `out`, `srow` 2-byte words per row of `scales`.
-__device__ __forceinline__ void zero_padding_rows(int64_t c, int lane,
-                                                  const int32_t *__restrict__ row_src,
-                                                  int64_t rows, uint4 *out, int32_t row_vecs,
-                                                  uint16_t *scales, int32_t scale_words) {
-  const int64_t r = c * kWarp + lane;
-  uint32_t m = __ballot_sync(kFull, r < rows && __ldg(row_src + r) < 0);
+// Zero 16-byte vectors [v0, v1) of each row in `m` (rows 32g + bit) and,
+// when scales is not null, 2-byte words [s0, s1) of its scale row.
+__device__ __forceinline__ void zero_rows(uint32_t m, int64_t g, int lane, uint4 *out,
+                                          int32_t row_vecs, int32_t v0, int32_t v1,
+                                          uint16_t *scales, int32_t scale_words, int32_t s0,
+                                          int32_t s1) {
   const uint4 zero = make_uint4(0, 0, 0, 0);
   while (m) {
     const int j = __ffs(m) - 1;
     m &= m - 1;
-    const int64_t row = c * kWarp + j;
+    const int64_t row = g * kWarp + j;
     uint4 *dst = out + row * row_vecs;
-    for (int v = lane; v < row_vecs; v += kWarp) st_v4(dst + v, zero);
+    for (int v = v0 + lane; v < v1; v += kWarp) st_v4(dst + v, zero);
     if (scales) {
       uint16_t *sd = scales + row * scale_words;
-      for (int v = lane; v < scale_words; v += kWarp) sd[v] = 0;
+      for (int v = s0 + lane; v < s1; v += kWarp) sd[v] = 0;
     }
   }
 }
@@ -71,33 +82,39 @@ __global__ void __launch_bounds__(kThreads)
                         int32_t N, int32_t k, int64_t rows, int32_t vecs, int32_t chunks) {
   constexpr int U = kBf16Chunk / 8 / kWarp;  // 2
   const int lane = threadIdx.x % kWarp;
-  const int64_t w = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
+  const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
-  if (w >= units) {
-    zero_padding_rows(w - units, lane, row_src, rows, out, vecs, nullptr, 0);
+  const int64_t pad_units = (rows + kWarp - 1) / kWarp;
+  if (w0 < pad_units) {
+    if (const uint32_t m = padding_mask(w0, lane, row_src, rows, rows))
+      zero_rows(m, w0, lane, out, vecs, 0, vecs, nullptr, 0, 0, 0);
     return;
   }
-  const int64_t t = w / chunks;
-  const int v0 = (int)(w % chunks) * (kBf16Chunk / 8);
-  int32_t my_slot;
-  uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
-  const uint4 *src = hidden + t * vecs;
-  uint4 x[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int v = v0 + u * kWarp + lane;
-    if (v < vecs) x[u] = ld_stream_v4(src + v);
-  }
-  while (live) {
-    const int j = __ffs(live) - 1;
-    live &= live - 1;
-    uint4 *dst = out + (int64_t)__shfl_sync(kFull, my_slot, j) * vecs;
+  const int64_t w = w0 - pad_units;
+  if (w < units) {
+    const int64_t t = w / chunks;
+    const int v0 = (int)(w % chunks) * (kBf16Chunk / 8);
+    int32_t my_slot;
+    uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+    const uint4 *src = hidden + t * vecs;
+    uint4 x[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int v = v0 + u * kWarp + lane;
-      if (v < vecs) st_v4(dst + v, x[u]);
+      if (v < vecs) x[u] = ld_stream_v4(src + v);
+    }
+    while (live) {
+      const int j = __ffs(live) - 1;
+      live &= live - 1;
+      uint4 *dst = out + (int64_t)__shfl_sync(kFull, my_slot, j) * vecs;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int v = v0 + u * kWarp + lane;
+        if (v < vecs) st_v4(dst + v, x[u]);
+      }
     }
   }
+
 }
 
 // ------------------------------------------------------------------- FP8
@@ -112,77 +129,84 @@ __global__ void __launch_bounds__(kThreads)
                        int32_t H, int32_t chunks) {
   constexpr int U = kChunk / 512;  // 2
   const int lane = threadIdx.x % kWarp;
-  const int64_t w = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
+  const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
+  const int64_t pad_units = (rows + kWarp - 1) / kWarp;
   const int32_t vecs = H / 8;
   const int32_t nb = H / 128;
-  if (w >= units) {
-    const int64_t c = w - units;
-    // codes: H bytes per row; scales: nb floats = 2*nb 2-byte words
-    zero_padding_rows(c, lane, row_src, rows, reinterpret_cast<uint4 *>(q), H / 16,
-                      reinterpret_cast<uint16_t *>(scales), 2 * nb);
+  if (w0 < pad_units) {
+    if (const uint32_t m = padding_mask(w0, lane, row_src, rows, rows))
+      zero_rows(m, w0, lane, reinterpret_cast<uint4 *>(q), H / 16, 0, H / 16,
+                reinterpret_cast<uint16_t *>(scales), 2 * nb, 0, 2 * nb);
     return;
   }
-  const int64_t t = w / chunks;
-  const int c0 = (int)(w % chunks) * kChunk;
-  int32_t my_slot;
-  uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
-  const uint4 *src = hidden + t * vecs;
-  uint4 a[U], b[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int col = c0 + u * 512 + lane * 16;
-    if (col < H) {
-      a[u] = ld_stream_v4(src + col / 8);
-      b[u] = ld_stream_v4(src + col / 8 + 1);
-    } else {
-      a[u] = b[u] = make_uint4(0, 0, 0, 0);
-    }
-  }
-  uint4 codes[U];
-  float scale[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const uint32_t wd[8] = {a[u].x, a[u].y, a[u].z, a[u].w, b[u].x, b[u].y, b[u].z, b[u].w};
-    float f[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      f[2 * i] = bf16lo(wd[i]);
-      f[2 * i + 1] = bf16hi(wd[i]);
-    }
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
-    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
-    uint32_t cw[4] = {0, 0, 0, 0};
-    float sc = 0.0f;
-    if (amax > 0.0f) {
-      sc = amax / 448.0f;  // IEEE round-to-nearest division
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = cvt_e4m3x2(f[4 * i] / sc, f[4 * i + 1] / sc);
-        const uint32_t hi = cvt_e4m3x2(f[4 * i + 2] / sc, f[4 * i + 3] / sc);
-        cw[i] = lo | (hi << 16);
-      }
-    }
-    codes[u] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-    scale[u] = sc;
-  }
-  while (live) {
-    const int j = __ffs(live) - 1;
-    live &= live - 1;
-    const int64_t s = __shfl_sync(kFull, my_slot, j);
+  const int64_t w = w0 - pad_units;
+
+  if (w < units) {
+    const int64_t t = w / chunks;
+    const int c0 = (int)(w % chunks) * kChunk;
+    int32_t my_slot;
+    uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+    const uint4 *src = hidden + t * vecs;
+    uint4 a[U], b[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int col = c0 + u * 512 + lane * 16;
       if (col < H) {
-        st_v4(reinterpret_cast<uint4 *>(q + s * H + col), codes[u]);
-        if ((lane & 7) == 0) scales[s * nb + col / 128] = scale[u];
+        a[u] = ld_stream_v4(src + col / 8);
+        b[u] = ld_stream_v4(src + col / 8 + 1);
+      } else {
+        a[u] = b[u] = make_uint4(0, 0, 0, 0);
+      }
+    }
+    uint4 codes[U];
+    float scale[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t wd[8] = {a[u].x, a[u].y, a[u].z, a[u].w, b[u].x, b[u].y, b[u].z, b[u].w};
+      float f[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        f[2 * i] = bf16lo(wd[i]);
+        f[2 * i + 1] = bf16hi(wd[i]);
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
+      uint32_t cw[4] = {0, 0, 0, 0};
+      float sc = 0.0f;
+      if (amax > 0.0f) {
+        sc = amax / 448.0f;  // IEEE round-to-nearest division
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t lo = cvt_e4m3x2(f[4 * i] / sc, f[4 * i + 1] / sc);
+          const uint32_t hi = cvt_e4m3x2(f[4 * i + 2] / sc, f[4 * i + 3] / sc);
+          cw[i] = lo | (hi << 16);
+        }
+      }
+      codes[u] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      scale[u] = sc;
+    }
+    while (live) {
+      const int j = __ffs(live) - 1;
+      live &= live - 1;
+      const int64_t s = __shfl_sync(kFull, my_slot, j);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int col = c0 + u * 512 + lane * 16;
+        if (col < H) {
+          st_v4(reinterpret_cast<uint4 *>(q + s * H + col), codes[u]);
+          if ((lane & 7) == 0) scales[s * nb + col / 128] = scale[u];
+        }
       }
     }
   }
+
+  // codes: H bytes per row, 64 vectors per chunk; scales: nb floats per row
+  // = 2*nb 2-byte words, 16 words (8 scales) per chunk
 }
 
 // ------------------------------------------------------------------- NVFP4
@@ -222,37 +246,6 @@ __device__ __forceinline__ int64_t sf_atom_offset(int64_t m, int32_t c, int32_t 
   return ((m >> 7) * col_tiles + (c >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (c & 3);
 }
 
-// Swizzled-scale padding for the 32 rows [32*c, 32*c + 32) of the padded row
-// range: rows without a source (padding rows of the output and the rows that
-// only complete the last 128-row tile) get zero scales (and zero codes when
-// they are output rows); every output row gets zeros in the scale columns
-// that only complete its last group of 4.
-__device__ __forceinline__ void zero_swizzled_padding(int64_t c, int lane,
-                                                      const int32_t *__restrict__ row_src,
-                                                      int64_t rows, int64_t rows_padded,
-                                                      uint4 *q, int32_t q_vecs, uint8_t *scales,
-                                                      int32_t nsf) {
-  const int32_t groups = (nsf + 3) / 4;
-  const int64_t r = c * kWarp + lane;
-  const bool in_range = r < rows_padded;
-  const bool no_src = in_range && (r >= rows || __ldg(row_src + r) < 0);
-  uint32_t m = __ballot_sync(kFull, no_src);
-  const uint4 zero = make_uint4(0, 0, 0, 0);
-  while (m) {
-    const int j = __ffs(m) - 1;
-    m &= m - 1;
-    const int64_t row = c * kWarp + j;
-    if (row < rows) {
-      uint4 *dst = q + row * q_vecs;
-      for (int v = lane; v < q_vecs; v += kWarp) st_v4(dst + v, zero);
-    }
-    for (int g = lane; g < groups; g += kWarp)
-      *reinterpret_cast<uint32_t *>(scales + sf_atom_offset(row, 4 * g, groups)) = 0u;
-  }
-  if ((nsf & 3) != 0 && in_range && !no_src)  // nsf is even: two columns complete the group
-    *reinterpret_cast<uint16_t *>(scales + sf_atom_offset(r, nsf, groups)) = 0;
-}
-
 __global__ void __launch_bounds__(kThreads)
     permute_nvfp4_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                          const int32_t *__restrict__ pair_slot,
@@ -260,67 +253,95 @@ __global__ void __launch_bounds__(kThreads)
                          uint8_t *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
                          int32_t H, int32_t chunks, bool swizzled) {
   const int lane = threadIdx.x % kWarp;
-  const int64_t w = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
+  const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
+  // swizzled scales: the rows that only complete the last 128-row tile are
+  // padding for the scales too
+  const int64_t check_rows = swizzled ? (rows + 127) / 128 * 128 : rows;
+  const int64_t pad_units = (check_rows + kWarp - 1) / kWarp;
   const int32_t vecs = H / 8;
   const int32_t qrow = H / 2, srow = H / 16;
-  if (w >= units) {
-    if (swizzled)
-      zero_swizzled_padding(w - units, lane, row_src, rows, (rows + 127) / 128 * 128,
-                            reinterpret_cast<uint4 *>(q), qrow / 16, scales, srow);
-    else
-      zero_padding_rows(w - units, lane, row_src, rows, reinterpret_cast<uint4 *>(q),
-                        qrow / 16, reinterpret_cast<uint16_t *>(scales), srow / 2);
+  const int32_t groups = (srow + 3) / 4;  // 4-scale groups per row (atom layout)
+  if (w0 < pad_units) {
+    // codes: H/2 bytes per row; scales: linear H/16 bytes per row, or the
+    // row's `groups` 4-byte groups in the atom layout
+    const uint32_t m = padding_mask(w0, lane, row_src, rows, check_rows);
+    if (m && !swizzled) {
+      zero_rows(m, w0, lane, reinterpret_cast<uint4 *>(q), qrow / 16, 0, qrow / 16,
+                reinterpret_cast<uint16_t *>(scales), srow / 2, 0, srow / 2);
+    } else if (m) {
+      uint32_t mm = m;
+      const uint4 zero = make_uint4(0, 0, 0, 0);
+      while (mm) {
+        const int j = __ffs(mm) - 1;
+        mm &= mm - 1;
+        const int64_t row = w0 * kWarp + j;
+        if (row < rows) {
+          uint4 *dst = reinterpret_cast<uint4 *>(q) + row * (qrow / 16);
+          for (int v = lane; v < qrow / 16; v += kWarp) st_v4(dst + v, zero);
+        }
+        for (int gg = lane; gg < groups; gg += kWarp)
+          *reinterpret_cast<uint32_t *>(scales + sf_atom_offset(row, 4 * gg, groups)) = 0u;
+      }
+    }
     return;
   }
-  const int64_t t = w / chunks;
-  const int col = (int)(w % chunks) * kChunk + lane * 32;
-  const bool active = col < H;
-  int32_t my_slot;
-  uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
-  const float gs = __ldg(global_scale);
-  const uint4 *src = hidden + t * vecs;
-  uint4 x[4];
+  const int64_t w = w0 - pad_units;
+
+  if (w < units) {
+    const int64_t t = w / chunks;
+    const int col = (int)(w % chunks) * kChunk + lane * 32;
+    const bool active = col < H;
+    int32_t my_slot;
+    uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+    const float gs = __ldg(global_scale);
+    const uint4 *src = hidden + t * vecs;
+    uint4 x[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    x[i] = active ? ld_stream_v4(src + col / 8 + i) : make_uint4(0, 0, 0, 0);
-  float f[32];
+    for (int i = 0; i < 4; ++i)
+      x[i] = active ? ld_stream_v4(src + col / 8 + i) : make_uint4(0, 0, 0, 0);
+    float f[32];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t wd[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t wd[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      f[8 * i + 2 * e] = bf16lo(wd[e]);
-      f[8 * i + 2 * e + 1] = bf16hi(wd[e]);
+      for (int e = 0; e < 4; ++e) {
+        f[8 * i + 2 * e] = bf16lo(wd[e]);
+        f[8 * i + 2 * e + 1] = bf16hi(wd[e]);
+      }
     }
-  }
-  uint4 codes;
-  const uint32_t sq0 = nvfp4_block(f, gs, codes.x, codes.y);
-  const uint32_t sq1 = nvfp4_block(f + 16, gs, codes.z, codes.w);
-  const uint16_t sq = (uint16_t)(sq0 | (sq1 << 8));
-  while (live) {
-    const int j = __ffs(live) - 1;
-    live &= live - 1;
-    const int64_t s = __shfl_sync(kFull, my_slot, j);
-    if (active) {
-      st_v4(reinterpret_cast<uint4 *>(q + s * qrow + col / 2), codes);
-      const int64_t so = swizzled ? sf_atom_offset(s, col / 16, (srow + 3) / 4)
-                                  : s * srow + col / 16;
-      *reinterpret_cast<uint16_t *>(scales + so) = sq;
+    uint4 codes;
+    const uint32_t sq0 = nvfp4_block(f, gs, codes.x, codes.y);
+    const uint32_t sq1 = nvfp4_block(f + 16, gs, codes.z, codes.w);
+    const uint32_t sq = sq0 | (sq1 << 8);
+    // atom layout: an even lane holds scale columns 4g, 4g+1 and its odd
+    // neighbour 4g+2, 4g+3 -- one 4-byte store per pair of lanes (an
+    // inactive neighbour contributes zeros: the column padding of a partial
+    // last group)
+    const uint32_t quad = sq | (__shfl_down_sync(kFull, active ? sq : 0u, 1) << 16);
+    while (live) {
+      const int j = __ffs(live) - 1;
+      live &= live - 1;
+      const int64_t s = __shfl_sync(kFull, my_slot, j);
+      if (active) {
+        st_v4(reinterpret_cast<uint4 *>(q + s * qrow + col / 2), codes);
+        if (!swizzled)
+          *reinterpret_cast<uint16_t *>(scales + s * srow + col / 16) = (uint16_t)sq;
+        else if ((lane & 1) == 0)
+          *reinterpret_cast<uint32_t *>(scales + sf_atom_offset(s, col / 16, groups)) = quad;
+      }
     }
   }
 }
 
-// One warp per unit: token units first, then one warp per 32 rows (of
-// `check_rows`, the output rows or, for swizzled scales, the rows rounded up
-// to the 128-row tile) for the padding check.
-inline int64_t unit_blocks(const Shape &s, int32_t chunks, int64_t check_rows = -1) {
-  if (check_rows < 0) check_rows = s.rows;
-  const int64_t warps = (int64_t)s.N * chunks + (check_rows + kWarp - 1) / kWarp;
-  return (warps + kThreads / kWarp - 1) / (kThreads / kWarp);
+// One warp per unit: ceil(check_rows / 32) padding warps, then N * chunks
+// token units.
+inline int64_t unit_blocks(const Shape &s, int32_t chunks, int64_t check_rows) {
+  const int64_t warps = (check_rows + kWarp - 1) / kWarp + (int64_t)s.N * chunks;
+  return std::max<int64_t>(1, (warps + kThreads / kWarp - 1) / (kThreads / kWarp));
 }
 
-inline int32_t chunks_of(int32_t H, int32_t chunk = kChunk) { return (H + chunk - 1) / chunk; }
+inline int32_t chunks_of(int32_t H, int32_t chunk) { return (H + chunk - 1) / chunk; }
 
 }  // namespace
 
@@ -328,7 +349,7 @@ cudaError_t launch_permute_bf16(const Shape &s, const void *hidden, const int32_
                                 const int32_t *pair_slot, void *out, cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
   const int32_t chunks = chunks_of(s.H, kBf16Chunk);
-  permute_bf16_kernel<<<(unsigned)unit_blocks(s, chunks), kThreads, 0, stream>>>(
+  permute_bf16_kernel<<<(unsigned)unit_blocks(s, chunks, s.rows), kThreads, 0, stream>>>(
       static_cast<const uint4 *>(hidden), row_src, pair_slot, static_cast<uint4 *>(out), s.N,
       s.k, s.rows, s.H / 8, chunks);
   return cudaGetLastError();
@@ -338,8 +359,8 @@ cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t
                                const int32_t *pair_slot, uint8_t *q, float *scales,
                                cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
-  const int32_t chunks = chunks_of(s.H);
-  permute_fp8_kernel<<<(unsigned)unit_blocks(s, chunks), kThreads, 0, stream>>>(
+  const int32_t chunks = chunks_of(s.H, kChunk);
+  permute_fp8_kernel<<<(unsigned)unit_blocks(s, chunks, s.rows), kThreads, 0, stream>>>(
       static_cast<const uint4 *>(hidden), row_src, pair_slot, q, scales, s.N, s.k, s.rows, s.H,
       chunks);
   return cudaGetLastError();
@@ -349,7 +370,7 @@ cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32
                                  const int32_t *pair_slot, const float *global_scale,
                                  uint8_t *q, uint8_t *scales, cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
-  const int32_t chunks = chunks_of(s.H);
+  const int32_t chunks = chunks_of(s.H, kChunk);
   const bool swizzled = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) != 0;
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
   permute_nvfp4_kernel<<<(unsigned)unit_blocks(s, chunks, check_rows), kThreads, 0, stream>>>(

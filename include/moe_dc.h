@@ -274,6 +274,44 @@ MOE_API moe_status moe_combine(const moe_problem *problem, const void *expert_ou
                        const float *gates, const int32_t *pair_slot, void *out,
                        moe_stream_t stream);
 
+/* ---- backward (training) -------------------------------------------------
+ * The gradients of the data movements above, for training with top-k
+ * probabilities whose gradient flows back through the combine (NeMo
+ * AutoModel token_dispatcher: token_probs [tokens, top_k] and the router
+ * gradient layout).  Same problem, maps and conventions as the forward. */
+
+/* Dispatch backward: the dispatch copies token t's row to the rows of its
+ * pairs, so grad_hidden[t,:] = bf16_rne(sum over j of grad_out[slot(t,j),:])
+ * in fp32 with j in order, pairs whose slot is outside [0, rows) skipped.
+ *   grad_out     bf16 [rows, H], 16-byte aligned
+ *   pair_slot    int32 [N, k] from the layout
+ *   grad_hidden  bf16 [N, H], 16-byte aligned, fully overwritten
+ * Requires H % 8 == 0. */
+MOE_API moe_status moe_permute_backward(const moe_problem *problem, const void *grad_out,
+                                        const int32_t *pair_slot, void *grad_hidden,
+                                        moe_stream_t stream);
+
+/* Combine backward: y[t] = sum_j w[t,j] * x[slot(t,j)] (DeepSpeed combine),
+ * so for every pair with a row
+ *   grad_expert_out[slot(t,j),:] = bf16_rne(w[t,j] * grad_y[t,:])  (fp32 product)
+ *   grad_gates[t,j] = <grad_y[t,:], expert_out[slot(t,j),:]>         (fp32)
+ * grad_gates is 0 for a pair without a row, and rows whose row_src is -1
+ * get zeros.  The dot product is accumulated in fp32 in a fixed order
+ * (deterministic): each of 32 lanes sums its elements in order, then a
+ * butterfly over the lanes; it is within 2^-24 * (H/32 + 8) * sum|g*x| of
+ * the exact value.
+ *   grad_y           bf16 [N, H], 16-byte aligned
+ *   expert_out       bf16 [rows, H], 16-byte aligned (the forward input)
+ *   gates            fp32 [N, k];  pair_slot int32 [N, k];  row_src int32 [rows]
+ *   grad_expert_out  bf16 [rows, H], 16-byte aligned, fully overwritten
+ *   grad_gates       fp32 [N, k], fully overwritten
+ * Requires H % 8 == 0. */
+MOE_API moe_status moe_combine_backward(const moe_problem *problem, const void *grad_y,
+                                        const void *expert_out, const float *gates,
+                                        const int32_t *pair_slot, const int32_t *row_src,
+                                        void *grad_expert_out, float *grad_gates,
+                                        moe_stream_t stream);
+
 /* Static description of a moe_status value. */
 MOE_API const char *moe_status_string(moe_status status);
 

@@ -431,3 +431,43 @@ def test_nvfp4_swizzled_scales_workload(orc):
     q, s_lin = orc.permute_nvfp4(w.hidden, ref.row_src, w.global_scale)
     assert np.array_equal(run.q4, q)
     assert np.array_equal(run.s4, orc.swizzle_scales(s_lin))
+
+
+# ------------------------------------------------------------ backward
+@pytest.mark.parametrize("cfg,n", [("tiny", None), ("mid_zipf", 1024), ("decode_capacity", None),
+                                   ("fp8_metric", 1024)])
+def test_backward_parity(orc, cfg, n):
+    w = make_workload(cfg, n_tokens=n)
+    run = GpuRun(w, quant=False, combine=False)
+    ref = oracle_layout(orc, w)
+    assert_layout(run, ref)
+    prob = run.prob
+    rows = run.buf.rows
+    rng = np.random.default_rng(23)
+    g_rows = _bits(rng.standard_normal((rows, w.H)))
+    g_tok = _bits(rng.standard_normal((w.N, w.H)))
+    # dispatch backward: bit-exact (fp32 adds in j order, one bf16 rounding)
+    gh = torch.empty((w.N, w.H), dtype=torch.bfloat16, device="cuda")
+    B.moe_permute_backward(prob, to_dev_bf16(g_rows), run.buf.pair_slot, gh)
+    # combine backward: bit-exact expert-row gradients, gate gradients within
+    # the fp32 accumulation bound of the exact dot products
+    gx = torch.empty((rows, w.H), dtype=torch.bfloat16, device="cuda")
+    gw = torch.empty((w.N, w.k), dtype=torch.float32, device="cuda")
+    X = w.expert_out
+    B.moe_combine_backward(prob, to_dev_bf16(g_tok), to_dev_bf16(X),
+                           torch.from_numpy(w.gates).cuda(), run.buf.pair_slot, run.buf.row_src,
+                           gx, gw)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_np(gh), orc.permute_backward(g_rows, ref.pair_slot))
+    ogx, ogw = orc.combine_backward(g_tok, X, w.gates, ref.pair_slot)
+    assert np.array_equal(bf16_np(gx), ogx)
+    gw_gpu = gw.cpu().numpy()
+    f = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    mag = np.zeros_like(ogw, dtype=np.float64)
+    for j in range(w.k):
+        s = ref.pair_slot[:, j]
+        ok = s >= 0
+        mag[:, j] = np.where(ok, np.sum(np.abs(f(g_tok) * f(X[np.maximum(s, 0)])), axis=1), 0)
+    bound = 2.0 ** -24 * (w.H / 32 + 8) * mag + 2.0 ** -23 * np.abs(ogw)
+    assert np.all(np.abs(gw_gpu.astype(np.float64) - ogw) <= bound)
+    assert np.all(gw_gpu[ref.pair_slot < 0] == 0)
