@@ -65,6 +65,14 @@ def lib():
         L.orc_permute_nvfp4.argtypes = [i64, i32, vp, vp, f32, vp, vp]
         L.orc_combine.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp]
         L.orc_permute_backward.argtypes = [i32, i32, i32, i64, vp, vp, vp]
+        L.orc_exp.restype = f32
+        L.orc_exp.argtypes = [f32]
+        L.orc_silu.restype = f32
+        L.orc_silu.argtypes = [f32]
+        L.orc_exp_n.argtypes = [vp, vp, i64]
+        L.orc_e8m0_from_exponent.restype = ctypes.c_uint8
+        L.orc_e8m0_from_exponent.argtypes = [i32]
+        L.orc_swiglu_quant.argtypes = [i64, i32, vp, ctypes.c_int, vp, ctypes.c_int, f32, vp, vp]
         L.orc_combine_backward.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp, vp, vp]
         for n in ("orc_bf16_from_f32_n", "orc_e4m3_from_f32_n", "orc_e2m1_from_f32_n"):
             getattr(L, n).argtypes = [vp, vp, i64]
@@ -224,3 +232,28 @@ def combine_backward(grad_y_bits: np.ndarray, expert_out_bits: np.ndarray, gates
     lib().orc_combine_backward(N, k, H, rows, _p(grad_y_bits), _p(expert_out_bits), _p(gates),
                                _p(pair_slot), _p(gx), _p(gw))
     return gx, gw
+
+
+# ---------------------------------------------------------------- SwiGLU
+FMT_NVFP4, FMT_MXFP8, FMT_MXFP4 = 0, 1, 2
+
+
+def exp_f32(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty_like(x)
+    lib().orc_exp_n(_p(x), _p(out), x.size)
+    return out
+
+
+def swiglu_quant(gate_up_bits: np.ndarray, row_src: np.ndarray, fmt: int,
+                 interleaved: bool = False, global_scale: float = 1.0):
+    """gate_up: uint16 [rows, 2I] bf16 bits; returns (codes, scales) uint8."""
+    gate_up_bits = np.ascontiguousarray(gate_up_bits, dtype=np.uint16)
+    row_src = np.ascontiguousarray(row_src, dtype=np.int32)
+    rows, two_i = gate_up_bits.shape
+    I = two_i // 2
+    codes = np.empty((rows, I if fmt == FMT_MXFP8 else I // 2), np.uint8)
+    scales = np.empty((rows, I // 16 if fmt == FMT_NVFP4 else I // 32), np.uint8)
+    lib().orc_swiglu_quant(rows, I, _p(gate_up_bits), int(interleaved), _p(row_src), fmt,
+                           float(np.float32(global_scale)), _p(codes), _p(scales))
+    return codes, scales

@@ -468,3 +468,130 @@ void orc_combine_backward(int32_t N, int32_t k, int32_t H, int64_t rows,
       grad_gates[p] = (float)dot;
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* SwiGLU + requantisation                                             */
+/* ------------------------------------------------------------------ */
+
+/* 2^n as a float for n in [-126, 127]. */
+static float pow2i(int n) { return f32_from_bits((uint32_t)(n + 127) << 23); }
+
+float orc_exp(float x) {
+  const float log2e = 1.44269504f;          /* RN(log2 e)                      */
+  const float ln2_hi = 0.693145751953125f;  /* ln 2 to 16 significant bits     */
+  const float ln2_lo = 1.42860682e-06f;     /* RN(ln 2 - ln2_hi)               */
+  if (isnan(x)) return x;
+  if (x > 88.75f) return INFINITY;
+  if (x < -104.0f) return 0.0f;
+  const float n = rintf(x * log2e);
+  float r = fmaf(-n, ln2_hi, x);
+  r = fmaf(-n, ln2_lo, r);
+  /* e^r = sum r^i / i!, i = 0..7, Horner */
+  float p = 1.98412698e-04f;                /* 1/7! */
+  p = fmaf(p, r, 1.38888889e-03f);          /* 1/6! */
+  p = fmaf(p, r, 8.33333333e-03f);          /* 1/5! */
+  p = fmaf(p, r, 4.16666667e-02f);          /* 1/4! */
+  p = fmaf(p, r, 1.66666667e-01f);          /* 1/3! */
+  p = fmaf(p, r, 0.5f);                     /* 1/2! */
+  p = fmaf(p, r, 1.0f);
+  p = fmaf(p, r, 1.0f);
+  const int ni = (int)n;
+  if (ni > 127) return (p * pow2i(127)) * pow2i(ni - 127);
+  if (ni < -126) return (p * pow2i(ni + 64)) * pow2i(-64);
+  return p * pow2i(ni);
+}
+
+void orc_exp_n(const float *in, float *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_exp(in[i]);
+}
+
+float orc_silu(float g) { return g / (1.0f + orc_exp(-g)); }
+
+uint8_t orc_e8m0_from_exponent(int32_t e) {
+  int32_t c = e + 127;
+  if (c < 0) c = 0;
+  if (c > 254) c = 254;
+  return (uint8_t)c;
+}
+
+/* floor(log2 a) of a finite a > 0 (subnormals included) */
+static int32_t floor_log2(float a) {
+  int e;
+  frexpf(a, &e); /* a = f * 2^e, f in [0.5, 1) */
+  return e - 1;
+}
+
+void orc_swiglu_quant(int64_t rows, int32_t I, const uint16_t *gate_up,
+                      int interleaved, const int32_t *row_src, int format,
+                      float global_scale, uint8_t *codes, uint8_t *scales) {
+  const int64_t code_row = format == 1 ? I : I / 2;
+  const int64_t scale_row = format == 0 ? I / 16 : I / 32;
+  float *y = (float *)malloc(sizeof(float) * (size_t)I);
+  for (int64_t r = 0; r < rows; ++r) {
+    uint8_t *cd = codes + r * code_row;
+    uint8_t *sd = scales + r * scale_row;
+    if (row_src[r] < 0) {
+      memset(cd, 0, (size_t)code_row);
+      memset(sd, 0, (size_t)scale_row);
+      continue;
+    }
+    const uint16_t *in = gate_up + r * 2 * (int64_t)I;
+    for (int32_t i = 0; i < I; ++i) {
+      float g = orc_bf16_to_f32(interleaved ? in[2 * i] : in[i]);
+      float u = orc_bf16_to_f32(interleaved ? in[2 * i + 1] : in[I + i]);
+      y[i] = orc_silu(g) * u;
+    }
+    if (format == 0) {
+      /* NVFP4, exactly the dispatch's rule on the fp32 values */
+      for (int32_t b = 0; b < I / 16; ++b) {
+        float amax = 0.0f;
+        for (int32_t i = 0; i < 16; ++i) {
+          float a = fabsf(y[16 * b + i]);
+          if (a > amax) amax = a;
+        }
+        uint8_t sq = orc_e4m3_from_f32((amax / 6.0f) / global_scale);
+        float d = orc_e4m3_to_f32(sq) * global_scale;
+        sd[b] = sq;
+        for (int32_t m = 0; m < 8; ++m) {
+          uint8_t lo = 0, hi = 0;
+          if (d > 0.0f) {
+            lo = orc_e2m1_from_f32(y[16 * b + 2 * m] / d);
+            hi = orc_e2m1_from_f32(y[16 * b + 2 * m + 1] / d);
+          }
+          cd[8 * b + m] = (uint8_t)(lo | (hi << 4));
+        }
+      }
+    } else {
+      const int32_t emax = format == 1 ? 8 : 2;
+      for (int32_t b = 0; b < I / 32; ++b) {
+        float amax = 0.0f;
+        for (int32_t i = 0; i < 32; ++i) {
+          float a = fabsf(y[32 * b + i]);
+          if (a > amax) amax = a;
+        }
+        if (amax == 0.0f) {
+          sd[b] = 0;
+          if (format == 1) memset(cd + 32 * b, 0, 32);
+          else memset(cd + 16 * b, 0, 16);
+          continue;
+        }
+        const uint8_t sc = orc_e8m0_from_exponent(floor_log2(amax) - emax);
+        sd[b] = sc;
+        const int32_t X = (int32_t)sc - 127;
+        for (int32_t i = 0; i < 32; ++i) {
+          /* y * 2^-X: X in [-127, 127] */
+          float v = -X >= -126 ? y[32 * b + i] * pow2i(-X)
+                               : (y[32 * b + i] * pow2i(-X - 64)) * pow2i(64);
+          if (format == 1) {
+            cd[32 * b + i] = orc_e4m3_from_f32(v);
+          } else if (i % 2 == 0) {
+            cd[16 * b + i / 2] = orc_e2m1_from_f32(v);
+          } else {
+            cd[16 * b + i / 2] |= (uint8_t)(orc_e2m1_from_f32(v) << 4);
+          }
+        }
+      }
+    }
+  }
+  free(y);
+}

@@ -106,6 +106,35 @@ void orc_combine(int32_t N, int32_t k, int32_t H, int64_t rows,
                  const uint16_t *expert_out, const float *gates,
                  const int32_t *pair_slot, uint16_t *y);
 
+/* ---- SwiGLU + requantisation (Mojo MAX ep_comm fused_silu_*_kernel and
+ * MXTokenFormat) -----------------------------------------------------------
+ * e^x: Cody-Waite range reduction (n = rint(x * log2 e), r = x - n*ln2 with
+ * ln2 split in two constants) and the degree-7 Taylor polynomial of e^r in
+ * Horner form with fmaf, then scaling by 2^n; one fixed fp32 operation
+ * sequence, written from the mathematics (Cody & Waite, Software Manual for
+ * the Elementary Functions, 1980).  x < -104 gives 0, x > 88.75 gives inf.
+ * silu(g) = g / (1 + e^-g);  swiglu(g, u) = silu(g) * u  (fp32, no fused
+ * multiply-add except inside e^x).
+ * E8M0 (OCP MX v1.0 shared scale): code c means 2^(c-127), 255 is NaN.     */
+float orc_exp(float x);
+float orc_silu(float g);
+uint8_t orc_e8m0_from_exponent(int32_t e); /* 2^e -> code, clamped to [0,254] */
+void orc_exp_n(const float *in, float *out, int64_t n);
+
+/* rows x I SwiGLU of bf16 gate/up rows (split: columns [0,I) gate and
+ * [I,2I) up; interleaved: gate at even, up at odd columns), quantised:
+ *   format 0 NVFP4: E2M1 codes [rows, I/2], E4M3 scales [rows, I/16] as in
+ *            the dispatch (global scale gs)
+ *   format 1 MXFP8: E4M3 codes [rows, I], E8M0 scales [rows, I/32]
+ *   format 2 MXFP4: E2M1 codes [rows, I/2], E8M0 scales [rows, I/32]
+ * MX block of 32: X = floor(log2(amax)) - emax (8 for E4M3, 2 for E2M1),
+ * scale code E8M0(X), element code = E(y * 2^-X) rounded to nearest even with
+ * saturation; an all-zero block gets scale code 0 and codes 0.  Rows whose
+ * row_src is -1 (no routed token) are all-zero bytes and are not read.     */
+void orc_swiglu_quant(int64_t rows, int32_t I, const uint16_t *gate_up,
+                      int interleaved, const int32_t *row_src, int format,
+                      float global_scale, uint8_t *codes, uint8_t *scales);
+
 /* ---- backward -----------------------------------------------------------
  * The gradients of the two data movements (training, NeMo token_dispatcher
  * top-k probabilities [T, K] whose gradient flows back through combine):
