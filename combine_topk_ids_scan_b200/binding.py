@@ -39,7 +39,10 @@ MOE_MAX_TOPK = 16
 EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout",
             "moe_dispatch_layout_noalloc", "moe_permute", "moe_permute_quant_fp8",
             "moe_permute_quant_nvfp4", "moe_combine", "moe_permute_backward",
-            "moe_combine_backward", "moe_status_string", "moe_version")
+            "moe_combine_backward", "moe_swiglu_quant", "moe_status_string", "moe_version")
+
+MOE_QUANT_NVFP4, MOE_QUANT_MXFP8, MOE_QUANT_MXFP4 = 0, 1, 2
+MOE_GATE_UP_SPLIT, MOE_GATE_UP_INTERLEAVED = 0, 1
 
 MOE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
@@ -112,6 +115,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     L.moe_permute_backward.argtypes = [P] + [vp] * 4
     L.moe_combine_backward.restype = ctypes.c_int
     L.moe_combine_backward.argtypes = [P] + [vp] * 8
+    L.moe_swiglu_quant.restype = ctypes.c_int
+    L.moe_swiglu_quant.argtypes = [P, ctypes.c_int32, ctypes.c_uint32, ctypes.c_uint32] + \
+        [vp] * 6
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_status_string.argtypes = [ctypes.c_int]
     L.moe_version.restype = ctypes.c_char_p
@@ -226,6 +232,24 @@ def moe_combine_backward(prob: Problem, grad_y, expert_out, gates, pair_slot, ro
                                        _ptr(gates), _ptr(pair_slot), _ptr(row_src),
                                        _ptr(grad_expert_out), _ptr(grad_gates),
                                        _stream(stream)), "moe_combine_backward")
+
+
+def moe_swiglu_quant(prob: Problem, intermediate: int, fmt: int, gate_up_layout: int, gate_up,
+                     row_src, global_scale, codes, scales, stream=None) -> None:
+    c = prob.c()
+    _check(load().moe_swiglu_quant(ctypes.byref(c), intermediate, fmt, gate_up_layout,
+                                   _ptr(gate_up), _ptr(row_src), _ptr(global_scale), _ptr(codes),
+                                   _ptr(scales), _stream(stream)), "moe_swiglu_quant")
+
+
+def swiglu_buffers(rows: int, intermediate: int, fmt: int, device="cuda"):
+    """(codes, scales) uint8 device buffers for moe_swiglu_quant."""
+    I = intermediate
+    codes = torch.empty((max(rows, 1), I if fmt == MOE_QUANT_MXFP8 else I // 2),
+                        dtype=torch.uint8, device=device)
+    scales = torch.empty((max(rows, 1), I // 16 if fmt == MOE_QUANT_NVFP4 else I // 32),
+                         dtype=torch.uint8, device=device)
+    return codes, scales
 
 
 # ----------------------------------------------------------------- buffers

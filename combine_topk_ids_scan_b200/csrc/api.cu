@@ -205,6 +205,31 @@ moe_status moe_combine_backward(const moe_problem *problem, const void *grad_y,
                                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_swiglu_quant(const moe_problem *problem, int32_t intermediate, uint32_t format,
+                            uint32_t gate_up_layout, const void *gate_up,
+                            const int32_t *row_src, const float *global_scale,
+                            uint8_t *codes, uint8_t *scales, moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (intermediate <= 0 || format > MOE_QUANT_MXFP4 || gate_up_layout > MOE_GATE_UP_INTERLEAVED)
+    return MOE_ERR_INVALID_ARG;
+  if (intermediate % 32 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const int64_t I = intermediate;
+  if (s.rows * 2 * I > 2147483647ll * 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.rows == 0) return MOE_OK;
+  if (!gate_up || !row_src || !codes || !scales || (format == MOE_QUANT_NVFP4 && !global_scale))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(gate_up, 16) || !aligned(codes, 16) ||
+      !aligned(scales, format == MOE_QUANT_NVFP4 ? 2 : 1) ||
+      (global_scale && !aligned(global_scale, 4)))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_swiglu_quant(s, intermediate, format,
+                                            gate_up_layout == MOE_GATE_UP_INTERLEAVED, gate_up,
+                                            row_src, global_scale, codes, scales,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char *moe_status_string(moe_status status) {
   switch (status) {
     case MOE_OK:

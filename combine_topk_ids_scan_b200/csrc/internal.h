@@ -56,6 +56,11 @@ cudaError_t launch_combine_backward(const Shape &s, const void *grad_y, const vo
                                     const int32_t *row_src, void *grad_expert_out,
                                     float *grad_gates, cudaStream_t stream);
 
+cudaError_t launch_swiglu_quant(const Shape &s, int32_t I, uint32_t format, bool interleaved,
+                                const void *gate_up, const int32_t *row_src,
+                                const float *global_scale, uint8_t *codes, uint8_t *scales,
+                                cudaStream_t stream);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 

@@ -274,6 +274,42 @@ MOE_API moe_status moe_combine(const moe_problem *problem, const void *expert_ou
                        const float *gates, const int32_t *pair_slot, void *out,
                        moe_stream_t stream);
 
+/* ---- fused SwiGLU + requantisation -----------------------------------------
+ * The step after the experts' gate/up projection (Mojo MAX ep_comm:
+ * fused_silu_kernel, fused_silu_mx_kernel, fused_silu_nvfp4_kernel,
+ * fused_silu_mxfp8_interleaved_kernel, MXTokenFormat).  The host does not know
+ * how many rows each expert received, so the kernel takes the layout's
+ * row_src: a row without a routed token (-1) is written as zero bytes and its
+ * input is not read.  For the other rows, per column i < I:
+ *   y = silu(g) * u,  silu(g) = g / (1 + e^-g)   in fp32
+ * where e^x is one fixed fp32 sequence (Cody-Waite reduction with ln 2 split
+ * as 0.693145751953125 + 1.42860682e-06, n = rint(x * 1.44269504), the
+ * Taylor polynomial of degree 7 in Horner form with fmaf, scaling by 2^n;
+ * x < -104 gives 0, x > 88.75 gives inf), and y is quantised:
+ *   MOE_QUANT_NVFP4  codes E2M1 [rows, I/2], scales E4M3 [rows, I/16]: the
+ *                    rule of moe_permute_quant_nvfp4 (global_scale needed)
+ *   MOE_QUANT_MXFP8  codes E4M3 [rows, I], scales E8M0 [rows, I/32]
+ *   MOE_QUANT_MXFP4  codes E2M1 [rows, I/2] (element 2m low nibble), scales
+ *                    E8M0 [rows, I/32]
+ * MX (OCP Microscaling v1.0): per block of 32, X = floor(log2(amax)) - emax
+ * (emax 8 for E4M3, 2 for E2M1), scale code clamp(X + 127, 0, 254), code =
+ * E(y * 2^-X) rounded to nearest even, saturating; an all-zero block gets
+ * scale code 0 and codes 0.
+ *   gate_up  bf16 [rows, 2*I], 16-byte aligned: MOE_GATE_UP_SPLIT = columns
+ *            [0, I) gate and [I, 2I) up; MOE_GATE_UP_INTERLEAVED = gate at
+ *            even and up at odd columns
+ *   row_src  int32 [rows] from the layout
+ *   codes    16-byte aligned; scales 2-byte aligned (NVFP4); both fully
+ *            overwritten
+ * Requires I % 32 == 0. */
+enum { MOE_QUANT_NVFP4 = 0, MOE_QUANT_MXFP8 = 1, MOE_QUANT_MXFP4 = 2 };
+enum { MOE_GATE_UP_SPLIT = 0, MOE_GATE_UP_INTERLEAVED = 1 };
+MOE_API moe_status moe_swiglu_quant(const moe_problem *problem, int32_t intermediate,
+                                    uint32_t format, uint32_t gate_up_layout,
+                                    const void *gate_up, const int32_t *row_src,
+                                    const float *global_scale, uint8_t *codes,
+                                    uint8_t *scales, moe_stream_t stream);
+
 /* ---- backward (training) -------------------------------------------------
  * The gradients of the data movements above, for training with top-k
  * probabilities whose gradient flows back through the combine (NeMo

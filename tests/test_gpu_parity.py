@@ -471,3 +471,57 @@ def test_backward_parity(orc, cfg, n):
     bound = 2.0 ** -24 * (w.H / 32 + 8) * mag + 2.0 ** -23 * np.abs(ogw)
     assert np.all(np.abs(gw_gpu.astype(np.float64) - ogw) <= bound)
     assert np.all(gw_gpu[ref.pair_slot < 0] == 0)
+
+
+# ------------------------------------------------------------ SwiGLU + requant
+@pytest.mark.parametrize("fmt", [0, 1, 2], ids=["nvfp4", "mxfp8", "mxfp4"])
+@pytest.mark.parametrize("interleaved", [False, True], ids=["split", "interleaved"])
+@pytest.mark.parametrize("I", [2048, 96 * 32 + 32])
+def test_swiglu_quant_parity(orc, fmt, interleaved, I):
+    w = make_workload("mid_zipf", n_tokens=256, with_expert_out=False)
+    C = w.N * w.k + 100                       # some rows without a token
+    w = Workload(**{**w.__dict__, "recv_capacity": C})
+    run = GpuRun(w, quant=False, combine=False)
+    ref = oracle_layout(orc, w)
+    assert_layout(run, ref)
+    rng = np.random.default_rng(31 + I + fmt)
+    gu = _bits(rng.standard_normal((C, 2 * I)) * np.float32(2.5))
+    gu[3, :8] = _bits(np.array([0, -0.0, 30, -30, 90, -90, 1e-3, -1e-3], np.float32))
+    codes, scales = B.swiglu_buffers(C, I, fmt)
+    gs = torch.tensor([0.01], dtype=torch.float32, device="cuda")
+    B.moe_swiglu_quant(run.prob, I, fmt, int(interleaved), to_dev_bf16(gu), run.buf.row_src,
+                       gs, codes, scales)
+    torch.cuda.synchronize()
+    want_c, want_s = orc.swiglu_quant(gu, ref.row_src, fmt, interleaved=interleaved,
+                                      global_scale=0.01)
+    assert np.array_equal(codes.cpu().numpy(), want_c)
+    assert np.array_equal(scales.cpu().numpy(), want_s)
+
+
+def test_swiglu_exp_matches_oracle_bitwise(orc):
+    """The kernel's e^x sequence is the oracle's: silu(g) * 1 over a dense
+    sweep of bf16 gate values, MXFP8-coded with a power-of-two block scale,
+    so any difference in e^x at the codes' resolution shows."""
+    I = 1024
+    g = np.arange(-(1 << 15), 1 << 15, dtype=np.int64).astype(np.uint16)  # every bf16 pattern
+    g = g[((g >> 7) & 0xFF) != 0xFF]                                    # drop inf / NaN
+    rows = len(g) // I
+    g = g[:rows * I].reshape(rows, I)
+    u = np.full((rows, I), 0x3F80, np.uint16)                           # 1.0
+    gu = np.ascontiguousarray(np.concatenate([g, u], axis=1))
+    ids = np.zeros((rows, 1), np.int32)
+    ww = Workload(name="sweep", N=rows, H=64, E=1, k=1, S=1, recv_capacity=rows,
+                  expert_capacity=0, ids=ids, gates=np.ones((rows, 1), np.float32),
+                  hidden=np.zeros((rows, 64), np.uint16), expert_out=None, global_scale=1.0,
+                  seed=0)
+    run = GpuRun(ww, quant=False, combine=False)
+    for fmt in (0, 1):
+        codes, scales = B.swiglu_buffers(rows, I, fmt)
+        gs = torch.tensor([1.0], dtype=torch.float32, device="cuda")
+        B.moe_swiglu_quant(run.prob, I, fmt, 0, to_dev_bf16(gu), run.buf.row_src, gs, codes,
+                           scales)
+        torch.cuda.synchronize()
+        want_c, want_s = orc.swiglu_quant(gu, np.arange(rows, dtype=np.int32), fmt,
+                                          global_scale=1.0)
+        assert np.array_equal(codes.cpu().numpy(), want_c)
+        assert np.array_equal(scales.cpu().numpy(), want_s)
