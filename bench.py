@@ -440,6 +440,39 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
               "tokens_per_s": w.N / ((pb_us + cb_us) * 1e-6)}
         del d_gh, d_gx, d_gw
 
+    # ---- fused SwiGLU + requantisation (NEXT row f3): the synthetic expert
+    # outputs [C, H] read as gate|up rows of intermediate size I = H / 2
+    f3 = None
+    if args.next_rows:
+        I = w.H // 2
+        f3 = {"intermediate": I, "gate_up": "split", "rows": buf.rows}
+        for fmt, name in ((B.MOE_QUANT_MXFP8, "mxfp8"), (B.MOE_QUANT_NVFP4, "nvfp4"),
+                          (B.MOE_QUANT_MXFP4, "mxfp4")):
+            codes, scales = B.swiglu_buffers(buf.rows, I, fmt, device=dev)
+            n_steps = max(10, args.steps // 20)
+
+            def f3_call():
+                B.moe_swiglu_quant(prob, I, fmt, B.MOE_GATE_UP_SPLIT, d_x, buf.row_src, d_gs,
+                                   codes, scales)
+
+            for _ in range(3):
+                flush_l2()
+                f3_call()
+            evp = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                   for _ in range(n_steps)]
+            torch.cuda.synchronize(dev)
+            for i in range(n_steps):
+                flush_l2()
+                evp[i][0].record(stream)
+                f3_call()
+                evp[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            us = 1e3 * sum(e[0].elapsed_time(e[1]) for e in evp) / n_steps
+            nbytes = (2 * 2 * I * total_rows + 4 * buf.rows + codes.numel() + scales.numel())
+            f3[name + "_us"] = round(us, 2)
+            f3[name + "_gbs"] = round(nbytes / (us * 1e-6) / 1e9, 1)
+            del codes, scales
+
     # ---- end to end through the public API from pinned host memory
     # Every step: H2D of the step's inputs (ids, hidden rows, gates, global
     # scale), the whole path with identity experts (the combine reads the bf16
@@ -551,8 +584,8 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
                             "combined rows, status and counts; copies of neighbouring steps "
                             "overlap on separate streams"},
             "gpu_launches": launches_per_step * args.steps,
-            "next_rows": ({"f1_grouped_gemm_ready_nvfp4": f1, "f4_backward": f4}
-                          if f1 or f4 else None),
+            "next_rows": ({"f1_grouped_gemm_ready_nvfp4": f1, "f3_swiglu_requant": f3,
+                           "f4_backward": f4} if f1 or f3 or f4 else None),
             "clocks": clocks, "layout_status": st,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -10,15 +10,26 @@
 // is not read.
 //
 // e^x is one fixed fp32 operation sequence (Cody-Waite range reduction, the
-// degree-7 Taylor polynomial in Horner form with fmaf, scaling by 2^n;
-// Cody & Waite, Software Manual for the Elementary Functions, 1980), not the
-// library expf, so that the quantised codes are a reproducible function of
-// the inputs.  Products and sums outside it use __fmul_rn / __fadd_rn so the
-// compiler cannot contract them.
+// degree-7 Taylor polynomial in Horner form with fused multiply-adds, scaling
+// by 2^n; Cody & Waite, Software Manual for the Elementary Functions, 1980),
+// not the library expf, so that the quantised codes are a reproducible
+// function of the inputs.  The kernel evaluates it two columns at a time with
+// the packed fp32x2 operations of sm_100 (__fmul2_rn, __fadd2_rn, __ffma2_rn):
+// each half of a packed operation rounds exactly as the scalar operation, so
+// the result is that of the scalar sequence bit for bit.
 //
-// One warp per unit (row, 1024 columns of the intermediate size I); a lane
-// owns 32 consecutive columns: eight 16-byte loads of gate/up, one MX block
-// or two NVFP4 blocks.
+// silu(g) depends on the 16-bit gate value alone, so each CTA first
+// evaluates it once for every bf16 g with 2^-25 <= |g| < 128 (32 binades of
+// 128 significands per sign, 8192 fp32 values = 32 KB of shared memory) and
+// afterwards reads it from that table.  A lane whose 32 gate values include
+// one outside the table (zero, tiny, huge, inf, NaN) evaluates the same
+// sequence directly, so the table changes no result, only the work.
+//
+// Persistent grid: the row-major list of (row, 32-column group) pairs is
+// dealt out lane by lane, consecutive lanes taking consecutive groups, so
+// no lane idles when I is not a multiple of 1024.  A lane owns 32
+// consecutive columns: eight 16-byte loads of gate/up, one MX block or two
+// NVFP4 blocks.
 #include <algorithm>
 
 #include "common.cuh"
@@ -29,35 +40,147 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr uint32_t kFull = 0xFFFFFFFFu;
-constexpr int kUnitCols = 1024;
+constexpr int kGroupCols = 32;  // columns of one lane
+
+// silu table: slot (b mod 4096) + 4096 * sign for the bf16 patterns b whose
+// magnitude bits lie in [0x3300, 0x4300), i.e. 2^-25 <= |g| < 2^7.  Those are
+// 4096 consecutive values, so b mod 4096 is one-to-one on them.
+constexpr uint32_t kTabFirst = 0x3300u;
+constexpr int kTabHalf = 4096;
+constexpr int kTabSize = 2 * kTabHalf;
 
 __device__ __forceinline__ float pow2i(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
 
-__device__ __forceinline__ float fixed_exp(float x) {
-  if (x != x) return x;
-  if (x > 88.75f) return __uint_as_float(0x7F800000u);
-  if (x < -104.0f) return 0.0f;
-  const float n = rintf(__fmul_rn(x, 1.44269504f));
-  float r = fmaf(-n, 0.693145751953125f, x);
-  r = fmaf(-n, 1.42860682e-06f, r);
-  float p = 1.98412698e-04f;
-  p = fmaf(p, r, 1.38888889e-03f);
-  p = fmaf(p, r, 8.33333333e-03f);
-  p = fmaf(p, r, 4.16666667e-02f);
-  p = fmaf(p, r, 1.66666667e-01f);
-  p = fmaf(p, r, 0.5f);
-  p = fmaf(p, r, 1.0f);
-  p = fmaf(p, r, 1.0f);
-  const int ni = (int)n;
-  if (ni > 127) return __fmul_rn(__fmul_rn(p, pow2i(127)), pow2i(ni - 127));
-  if (ni < -126) return __fmul_rn(__fmul_rn(p, pow2i(ni + 64)), pow2i(-64));
-  return __fmul_rn(p, pow2i(ni));
+// max / min that return NaN when either operand is NaN
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float min_nan(float a, float b) {
+  float r;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
 }
 
-__device__ __forceinline__ float swiglu(float g, float u) {
-  const float silu = __fdiv_rn(g, __fadd_rn(1.0f, fixed_exp(-g)));
-  return __fmul_rn(silu, u);
+__device__ __forceinline__ float2 splat(float v) { return make_float2(v, v); }
+
+// e^x of both halves.
+//  * Range: the sequence gives +inf at x = 88.75 (2^128 overflows) and +0 at
+//    x = -104 (below half the smallest subnormal), so clamping x to
+//    [-104, 88.75] is exactly "x > 88.75 -> inf, x < -104 -> 0"; NaN passes
+//    through the clamp and the arithmetic.
+//  * n = rint(x log2 e) by the 1.5 * 2^23 shifter: for |t| < 2^22, t + 1.5 * 2^23
+//    rounds t to the nearest integer, ties to even (the sum's unit is 1), the
+//    subtraction is exact, and the integer n sits in the sum's low bits.
+//  * 2^n as two normal factors 2^floor(n/2) * 2^ceil(n/2): for n in
+//    [-150, 128] p * 2^floor(n/2) is exact, so the product rounds once, to
+//    RN(p * 2^n), whichever way the scalar sequence splits the scaling.
+__device__ __forceinline__ float2 fixed_exp2(float2 x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  x.x = min_nan(max_nan(x.x, -104.0f), 88.75f);
+  x.y = min_nan(max_nan(x.y, -104.0f), 88.75f);
+  const float2 sh = __fadd2_rn(__fmul2_rn(x, splat(1.44269504f)), splat(kShift));
+  const float2 n = __fadd2_rn(sh, splat(-kShift));
+  float2 r = __ffma2_rn(n, splat(-0.693145751953125f), x);  // ln 2, high 16 bits
+  r = __ffma2_rn(n, splat(-1.42860682e-06f), r);             // ln 2, the rest
+  float2 p = splat(1.98412698e-04f);                         // 1/7!
+  p = __ffma2_rn(p, r, splat(1.38888889e-03f));
+  p = __ffma2_rn(p, r, splat(8.33333333e-03f));
+  p = __ffma2_rn(p, r, splat(4.16666667e-02f));
+  p = __ffma2_rn(p, r, splat(1.66666667e-01f));
+  p = __ffma2_rn(p, r, splat(0.5f));
+  p = __ffma2_rn(p, r, splat(1.0f));
+  p = __ffma2_rn(p, r, splat(1.0f));
+  const int n0 = __float_as_int(sh.x) - 0x4B400000, n1 = __float_as_int(sh.y) - 0x4B400000;
+  p = __fmul2_rn(p, make_float2(pow2i(n0 >> 1), pow2i(n1 >> 1)));               // 2^floor(n/2)
+  return __fmul2_rn(p, make_float2(pow2i((n0 + 1) >> 1), pow2i((n1 + 1) >> 1)));  // 2^ceil(n/2)
+}
+
+// silu(g) = g / (1 + e^-g) of both halves; IEEE division.
+__device__ __forceinline__ float2 silu2(float2 g) {
+  const float2 d = __fadd2_rn(splat(1.0f), fixed_exp2(make_float2(-g.x, -g.y)));
+  return make_float2(__fdiv_rn(g.x, d.x), __fdiv_rn(g.y, d.y));
+}
+
+// The gate value of table slot i.
+__device__ __forceinline__ float tab_gate(int i) {
+  const uint32_t mag = kTabFirst + (((uint32_t)i - kTabFirst) & 0xFFFu);
+  return __uint_as_float((((uint32_t)(i >> 12) << 15) | mag) << 16);
+}
+
+// Byte offsets into the table of the low and high bf16 of a 32-bit word:
+// 4 * ((b & 0xFFF) | (sign << 12)) for each half b.
+__device__ __forceinline__ void table_offsets(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  const uint32_t m = ((w << 2) & 0x3FFC3FFCu) | ((w >> 1) & 0x40004000u);
+  lo = m & 0x7FFCu;
+  hi = m >> 16;
+}
+__device__ __forceinline__ float table_at(const float *tab, uint32_t off) {
+  return *reinterpret_cast<const float *>(reinterpret_cast<const char *>(tab) + off);
+}
+
+// max(a, |b|, |c|) in one three-input maximum
+__device__ __forceinline__ float max_abs3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+  return r;
+}
+
+// Eight floats -> eight E2M1 codes (nearest even, saturating to +-6), the
+// first in bits 0-3.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t3, %8, %7;\n\t"
+      "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+      : "=r"(r)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+  return r;
+}
+
+// Four floats -> four E4M3 codes (nearest even, saturating to +-448), the
+// first in bits 0-7.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float2 a, float2 b) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t0, t1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 t0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 t1, %4, %3;\n\t"
+      "mov.b32 %0, {t0, t1};\n\t}"
+      : "=r"(r)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+// Bits 12..15 and 28..31 of the result are zero iff both bf16 of w are in
+// the table: for a magnitude in [0x3300, 0x4300), magnitude + 0x4D00 lies in
+// [0x8000, 0x9000) (and never carries into the other half, being at most
+// 0xCCFF), so flipping bit 15 leaves it below 0x1000.
+__device__ __forceinline__ uint32_t table_check(uint32_t w) {
+  return ((w & 0x7FFF7FFFu) + 0x4D004D00u) ^ 0x80008000u;
+}
+constexpr uint32_t kTableCheckBits = 0xF000F000u;
+
+// RN(a / d) of both halves for the E2M1 code, from rd = RN(1/d), by two
+// steps of Markstein's correction q + (a - d q) * rd (P. Markstein,
+// Computation of elementary functions on the IBM RISC System/6000 processor,
+// IBM J. Res. Dev. 34(1), 1990: if rd is within half an ulp of 1/d and q
+// within one ulp of a/d, the corrected q rounds correctly).  q0 = RN(a rd) is
+// within two ulps, the first step brings it within one, the second rounds
+// correctly.  Preconditions, checked by the caller: d in [2^-100, 2^124],
+// which keeps the remainders exact for every quotient >= 2^-3 (a smaller one
+// encodes to +-0 whatever its last bits), and |a / d| <= 12.01, which keeps
+// them finite (a block scale that did not saturate is at least half of
+// amax / 6).  A zero quotient takes the sign of a, as IEEE division does.
+__device__ __forceinline__ float2 e2m1_quotient2(float2 a, float d, float rd) {
+  const float2 nd = splat(-d), r2 = splat(rd);
+  float2 q = __fmul2_rn(a, r2);
+  q = __ffma2_rn(__ffma2_rn(nd, q, a), r2, q);
+  q = __ffma2_rn(__ffma2_rn(nd, q, a), r2, q);
+  return make_float2(copysignf(q.x, a.x), copysignf(q.y, a.y));
 }
 
 // floor(log2(a)) of a finite a > 0, subnormals included.
@@ -68,28 +191,17 @@ __device__ __forceinline__ int floor_log2(float a) {
   return (31 - __clz((int)(b & 0x7FFFFFu))) - 149;
 }
 
-// y * 2^-X for X in [-127, 127], as two exact scalings when 2^-X alone is not
-// a normal float.
-__device__ __forceinline__ float scale_down(float y, int X) {
-  return -X >= -126 ? __fmul_rn(y, pow2i(-X)) : __fmul_rn(__fmul_rn(y, pow2i(-X - 64)), pow2i(64));
-}
-
+// One lane's 32 columns [c, c + 32) of row r.
 template <int FORMAT, bool INTERLEAVED>
-__global__ void __launch_bounds__(kThreads)
-    swiglu_quant_kernel(const uint4 *__restrict__ gate_up, const int32_t *__restrict__ row_src,
-                        const float *__restrict__ global_scale, uint8_t *__restrict__ codes,
-                        uint8_t *__restrict__ scales, int64_t rows, int32_t I, int32_t chunks) {
-  const int lane = threadIdx.x % kWarp;
-  const int64_t w = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
-  if (w >= rows * chunks) return;
-  const int64_t r = w / chunks;
-  const int c = (int)(w % chunks) * kUnitCols + lane * 32;
-  const bool active = c < I;
+__device__ __forceinline__ void swiglu_group(const float *tab, const uint4 *__restrict__ gate_up,
+                                             const int32_t *__restrict__ row_src, float gs,
+                                             uint8_t *__restrict__ codes,
+                                             uint8_t *__restrict__ scales, int64_t r, int32_t c,
+                                             int32_t I) {
   const int64_t code_row = FORMAT == 1 ? I : I / 2;
   const int64_t scale_row = FORMAT == 0 ? I / 16 : I / 32;
   uint8_t *cd = codes + r * code_row + (FORMAT == 1 ? c : c / 2);
   uint8_t *sd = scales + r * scale_row + (FORMAT == 0 ? c / 16 : c / 32);
-  if (!active) return;
 
   if (__ldg(row_src + r) < 0) {  // no routed token: zero bytes, input not read
     const uint4 zero = make_uint4(0, 0, 0, 0);
@@ -101,8 +213,7 @@ __global__ void __launch_bounds__(kThreads)
   }
 
   // ---- 32 gate and 32 up values
-  const int64_t row_vecs = (int64_t)I / 4;  // 2I bf16 = I/4 vectors of 8
-  const uint4 *in = gate_up + r * row_vecs;
+  const uint4 *in = gate_up + r * ((int64_t)I / 4);  // 2I bf16 = I/4 vectors of 8
   uint4 gv[4], uv[4];
   if (INTERLEAVED) {
     uint4 iv[8];
@@ -124,42 +235,66 @@ __global__ void __launch_bounds__(kThreads)
       uv[i] = ld_stream_v4(in + I / 8 + c / 8 + i);
     }
   }
-  float y[32];
+
+  // ---- y = silu(g) * u, two columns at a time: y[j] = columns 2j, 2j+1
+  uint32_t check = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    check |= table_check(gv[i].x) | table_check(gv[i].y) | table_check(gv[i].z) |
+             table_check(gv[i].w);
+  float2 y[16];
+  if ((check & kTableCheckBits) == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t g4[4] = {gv[i].x, gv[i].y, gv[i].z, gv[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t lo, hi;
+        table_offsets(g4[e], lo, hi);
+        y[4 * i + e] = make_float2(table_at(tab, lo), table_at(tab, hi));
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t g4[4] = {gv[i].x, gv[i].y, gv[i].z, gv[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) y[4 * i + e] = silu2(make_float2(bf16lo(g4[e]), bf16hi(g4[e])));
+    }
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t g4[4] = {gv[i].x, gv[i].y, gv[i].z, gv[i].w};
     const uint32_t u4[4] = {uv[i].x, uv[i].y, uv[i].z, uv[i].w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      y[8 * i + 2 * e] = swiglu(bf16lo(g4[e]), bf16lo(u4[e]));
-      y[8 * i + 2 * e + 1] = swiglu(bf16hi(g4[e]), bf16hi(u4[e]));
-    }
+    for (int e = 0; e < 4; ++e)
+      y[4 * i + e] = __fmul2_rn(y[4 * i + e], make_float2(bf16lo(u4[e]), bf16hi(u4[e])));
   }
 
   if (FORMAT == 0) {
     // ---- NVFP4: the dispatch's rule on the fp32 values, two blocks of 16
-    const float gs = __ldg(global_scale);
     uint32_t cw[4] = {0, 0, 0, 0};
     uint32_t sq2 = 0;
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(y[16 * b + i]));
+      for (int j = 0; j < 8; ++j) amax = max_abs3(amax, y[8 * b + j].x, y[8 * b + j].y);
       const uint32_t sq = cvt_e4m3x2(__fdiv_rn(__fdiv_rn(amax, 6.0f), gs), 0.0f) & 0xFFu;
       const float d = __fmul_rn(e4m3_to_float(sq), gs);
       sq2 |= sq << (8 * b);
       if (d > 0.0f) {
+        float2 q[8];
+        if (sq < 0x7Eu && d >= 0x1p-100f && d <= 0x1p124f) {  // 0x7E: saturated at 448
+          const float rd = __frcp_rn(d);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t word = 0;
+          for (int j = 0; j < 8; ++j) q[j] = e2m1_quotient2(y[8 * b + j], d, rd);
+        } else {
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const int i = 16 * b + 8 * h + 2 * m;
-            word |= cvt_e2m1x2(__fdiv_rn(y[i], d), __fdiv_rn(y[i + 1], d)) << (8 * m);
-          }
-          cw[2 * b + h] = word;
+          for (int j = 0; j < 8; ++j)
+            q[j] = make_float2(__fdiv_rn(y[8 * b + j].x, d), __fdiv_rn(y[8 * b + j].y, d));
         }
+        cw[2 * b] = cvt_e2m1x8(q[0], q[1], q[2], q[3]);
+        cw[2 * b + 1] = cvt_e2m1x8(q[4], q[5], q[6], q[7]);
       }
     }
     st_v4(reinterpret_cast<uint4 *>(cd), make_uint4(cw[0], cw[1], cw[2], cw[3]));
@@ -169,31 +304,23 @@ __global__ void __launch_bounds__(kThreads)
     constexpr int kEmax = FORMAT == 1 ? 8 : 2;
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(y[i]));
+    for (int j = 0; j < 16; ++j) amax = max_abs3(amax, y[j].x, y[j].y);
     uint32_t sc = 0;
     uint32_t cw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (amax > 0.0f) {
       sc = (uint32_t)min(254, max(0, floor_log2(amax) - kEmax + 127));
-      const int X = (int)sc - 127;
+      // X = sc - 127 lies in [-127, 127 - kEmax], so 2^-X is a normal float
+      // and y * 2^-X is one rounding
+      const float2 s2 = splat(pow2i(127 - (int)sc));
       if (FORMAT == 1) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t lo = cvt_e4m3x2(scale_down(y[4 * i], X), scale_down(y[4 * i + 1], X));
-          const uint32_t hi =
-              cvt_e4m3x2(scale_down(y[4 * i + 2], X), scale_down(y[4 * i + 3], X));
-          cw[i] = lo | (hi << 16);
-        }
+        for (int i = 0; i < 8; ++i)
+          cw[i] = cvt_e4m3x4(__fmul2_rn(y[2 * i], s2), __fmul2_rn(y[2 * i + 1], s2));
       } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t word = 0;
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const int e = 8 * i + 2 * m;
-            word |= cvt_e2m1x2(scale_down(y[e], X), scale_down(y[e + 1], X)) << (8 * m);
-          }
-          cw[i] = word;
-        }
+        for (int i = 0; i < 4; ++i)
+          cw[i] = cvt_e2m1x8(__fmul2_rn(y[4 * i], s2), __fmul2_rn(y[4 * i + 1], s2),
+                             __fmul2_rn(y[4 * i + 2], s2), __fmul2_rn(y[4 * i + 3], s2));
       }
     }
     st_v4(reinterpret_cast<uint4 *>(cd), make_uint4(cw[0], cw[1], cw[2], cw[3]));
@@ -203,14 +330,62 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// Persistent: thread t of the grid takes groups t, t + stride, ... of the
+// rows * G groups (G = I / 32 per row); (row, group) advance by
+// (step_rows, step_cols) = divmod(stride, G).
+template <int FORMAT, bool INTERLEAVED>
+__global__ void __launch_bounds__(kThreads, 3)
+    swiglu_quant_kernel(const uint4 *__restrict__ gate_up, const int32_t *__restrict__ row_src,
+                        const float *__restrict__ global_scale, uint8_t *__restrict__ codes,
+                        uint8_t *__restrict__ scales, int64_t groups, int32_t I, int32_t G,
+                        int64_t step_rows, int32_t step_cols) {
+  __shared__ float tab[kTabSize];
+  for (int i = 2 * threadIdx.x; i < kTabSize; i += 2 * kThreads) {
+    const float2 v = silu2(make_float2(tab_gate(i), tab_gate(i + 1)));
+    tab[i] = v.x;
+    tab[i + 1] = v.y;
+  }
+  __syncthreads();
+
+  const float gs = FORMAT == 0 ? __ldg(global_scale) : 0.0f;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t t = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  int64_t row = t / G;
+  int32_t cg = (int32_t)(t - row * G);
+  for (; t < groups; t += stride) {
+    swiglu_group<FORMAT, INTERLEAVED>(tab, gate_up, row_src, gs, codes, scales, row,
+                                      cg * kGroupCols, I);
+    row += step_rows;
+    cg += step_cols;
+    if (cg >= G) {
+      cg -= G;
+      ++row;
+    }
+  }
+}
+
 template <int FORMAT, bool INTERLEAVED>
 cudaError_t launch(const uint4 *in, const int32_t *row_src, const float *gs, uint8_t *codes,
                    uint8_t *scales, int64_t rows, int32_t I, cudaStream_t stream) {
-  const int32_t chunks = (I + kUnitCols - 1) / kUnitCols;
-  const int64_t warps = rows * chunks;
-  const int64_t blocks = std::max<int64_t>(1, (warps + kThreads / kWarp - 1) / (kThreads / kWarp));
-  swiglu_quant_kernel<FORMAT, INTERLEAVED><<<(unsigned)blocks, kThreads, 0, stream>>>(
-      in, row_src, gs, codes, scales, rows, I, chunks);
+  auto kernel = swiglu_quant_kernel<FORMAT, INTERLEAVED>;
+  static int per_sm[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // resident CTAs per SM, by device
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  int &cap = per_sm[dev & 7];
+  if (cap == 0) {
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cap, kernel, kThreads, 0);
+    if (err != cudaSuccess) return err;
+    cap = std::max(cap, 1);
+  }
+  const int32_t G = I / kGroupCols;
+  const int64_t groups = rows * G;
+  const int64_t want = (groups + kThreads - 1) / kThreads;
+  const int64_t blocks = std::max<int64_t>(
+      1, std::min<int64_t>(want, (int64_t)cap * device_sm_count()));
+  const int64_t stride = blocks * kThreads;
+  kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(in, row_src, gs, codes, scales, groups, I, G,
+                                                    stride / G, (int32_t)(stride % G));
   return cudaGetLastError();
 }
 

@@ -525,3 +525,40 @@ def test_swiglu_exp_matches_oracle_bitwise(orc):
                                           global_scale=1.0)
         assert np.array_equal(codes.cpu().numpy(), want_c)
         assert np.array_equal(scales.cpu().numpy(), want_s)
+
+
+@pytest.mark.parametrize("gscale", [1e-33, 2e-6, 0.37, 3e4, 1e36])
+def test_swiglu_quant_wide_range(orc, gscale):
+    """Gate/up values drawn from every finite bf16 bit pattern (all binades,
+    subnormals, signed zeros) and global scales from tiny to huge: NVFP4
+    blocks then take every path of the quotient (the corrected reciprocal,
+    the division fallback for a tiny or huge block scale, the clamp of
+    quotients above 8), and MX blocks every E8M0 clamp."""
+    I = 1024
+    rows = 96
+    rng = np.random.default_rng(int(gscale * 1e3) % 1000 + 7)
+    gu = rng.integers(0, 1 << 16, size=(rows, 2 * I), dtype=np.uint32).astype(np.uint16)
+    # exponent fields above 189 (|x| >= 2^63, inf, NaN) folded down, so that
+    # gate * up stays finite
+    ex = (gu >> 7) & 0xFF
+    gu = (gu & 0x807F) | (np.where(ex > 189, ex - 66, ex) << 7).astype(np.uint16)
+    # some rows of one narrow binade so that a block's amax sits near its values
+    gu[::7, :] = (gu[::7, :] & 0x807F) | 0x3F00
+    # a row near the top of the fp32 range: block scales above 2^124
+    gu[5, :] = 0x5F7F
+    ids = np.zeros((rows, 1), np.int32)
+    ww = Workload(name="wide", N=rows, H=64, E=1, k=1, S=1, recv_capacity=rows,
+                  expert_capacity=0, ids=ids, gates=np.ones((rows, 1), np.float32),
+                  hidden=np.zeros((rows, 64), np.uint16), expert_out=None, global_scale=1.0,
+                  seed=0)
+    run = GpuRun(ww, quant=False, combine=False)
+    for fmt in (0, 1, 2):
+        codes, scales = B.swiglu_buffers(rows, I, fmt)
+        gs = torch.tensor([gscale], dtype=torch.float32, device="cuda")
+        B.moe_swiglu_quant(run.prob, I, fmt, 0, to_dev_bf16(gu), run.buf.row_src, gs, codes,
+                           scales)
+        torch.cuda.synchronize()
+        want_c, want_s = orc.swiglu_quant(gu, np.arange(rows, dtype=np.int32), fmt,
+                                          global_scale=float(np.float32(gscale)))
+        assert np.array_equal(scales.cpu().numpy(), want_s), fmt
+        assert np.array_equal(codes.cpu().numpy(), want_c), fmt
