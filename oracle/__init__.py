@@ -63,6 +63,8 @@ def lib():
         L.orc_permute_bf16.argtypes = [i64, i32, vp, vp, vp]
         L.orc_permute_fp8.argtypes = [i64, i32, vp, vp, vp, vp]
         L.orc_permute_nvfp4.argtypes = [i64, i32, vp, vp, f32, vp, vp]
+        L.orc_permute_mxfp4.argtypes = [i64, i32, vp, vp, vp, vp]
+        L.orc_pack_fp6.argtypes = [vp, i64, vp]
         L.orc_combine.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp]
         L.orc_permute_backward.argtypes = [i32, i32, i32, i64, vp, vp, vp]
         L.orc_exp.restype = f32
@@ -74,8 +76,12 @@ def lib():
         L.orc_e8m0_from_exponent.argtypes = [i32]
         L.orc_swiglu_quant.argtypes = [i64, i32, vp, ctypes.c_int, vp, ctypes.c_int, f32, vp, vp]
         L.orc_combine_backward.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp, vp, vp]
-        for n in ("orc_bf16_from_f32_n", "orc_e4m3_from_f32_n", "orc_e2m1_from_f32_n"):
+        for n in ("orc_bf16_from_f32_n", "orc_e4m3_from_f32_n", "orc_e2m1_from_f32_n",
+                  "orc_e2m3_from_f32_n", "orc_e3m2_from_f32_n"):
             getattr(L, n).argtypes = [vp, vp, i64]
+        for n in ("orc_e2m3_to_f32", "orc_e3m2_to_f32"):
+            getattr(L, n).restype = f32
+            getattr(L, n).argtypes = [ctypes.c_uint8]
         L.orc_e4m3_to_f32.restype = f32
         L.orc_e4m3_to_f32.argtypes = [ctypes.c_uint8]
         L.orc_e2m1_to_f32.restype = f32
@@ -105,6 +111,35 @@ def e2m1_from_f32(x: np.ndarray) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float32)
     out = np.empty(x.shape, dtype=np.uint8)
     lib().orc_e2m1_from_f32_n(_p(x), _p(out), x.size)
+    return out
+
+
+def e2m3_from_f32(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint8)
+    lib().orc_e2m3_from_f32_n(_p(x), _p(out), x.size)
+    return out
+
+
+def e3m2_from_f32(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint8)
+    lib().orc_e3m2_from_f32_n(_p(x), _p(out), x.size)
+    return out
+
+
+def e2m3_to_f32(code: int) -> float:
+    return float(lib().orc_e2m3_to_f32(code))
+
+
+def e3m2_to_f32(code: int) -> float:
+    return float(lib().orc_e3m2_to_f32(code))
+
+
+def pack_fp6(codes: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8).reshape(-1)
+    out = np.empty(codes.size * 3 // 4, np.uint8)
+    lib().orc_pack_fp6(_p(codes), codes.size, _p(out))
     return out
 
 
@@ -183,6 +218,16 @@ def permute_nvfp4(hidden_bits: np.ndarray, row_src: np.ndarray, global_scale: fl
     return q, sc
 
 
+def permute_mxfp4(hidden_bits: np.ndarray, row_src: np.ndarray):
+    hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
+    row_src = np.ascontiguousarray(row_src, dtype=np.int32)
+    H = hidden_bits.shape[1]
+    q = np.empty((row_src.size, H // 2), np.uint8)
+    sc = np.empty((row_src.size, H // 32), np.uint8)
+    lib().orc_permute_mxfp4(row_src.size, H, _p(hidden_bits), _p(row_src), _p(q), _p(sc))
+    return q, sc
+
+
 def swizzle_scales(linear: np.ndarray) -> np.ndarray:
     """[rows, nsf] uint8 scales -> the 128x4 atom layout (flat uint8)."""
     linear = np.ascontiguousarray(linear, dtype=np.uint8)
@@ -235,7 +280,18 @@ def combine_backward(grad_y_bits: np.ndarray, expert_out_bits: np.ndarray, gates
 
 
 # ---------------------------------------------------------------- SwiGLU
-FMT_NVFP4, FMT_MXFP8, FMT_MXFP4 = 0, 1, 2
+FMT_NVFP4, FMT_MXFP8, FMT_MXFP4, FMT_BF16, FMT_MXFP6_E2M3, FMT_MXFP6_E3M2 = 0, 1, 2, 3, 4, 5
+
+
+def swiglu_code_bytes(I: int, fmt: int) -> int:
+    """Bytes of one row of swiglu_quant codes."""
+    return {FMT_NVFP4: I // 2, FMT_MXFP8: I, FMT_MXFP4: I // 2, FMT_BF16: 2 * I,
+            FMT_MXFP6_E2M3: 3 * I // 4, FMT_MXFP6_E3M2: 3 * I // 4}[fmt]
+
+
+def swiglu_scale_bytes(I: int, fmt: int) -> int:
+    """Bytes of one row of swiglu_quant scales (0 for bf16)."""
+    return I // 16 if fmt == FMT_NVFP4 else 0 if fmt == FMT_BF16 else I // 32
 
 
 def exp_f32(x: np.ndarray) -> np.ndarray:
@@ -252,8 +308,8 @@ def swiglu_quant(gate_up_bits: np.ndarray, row_src: np.ndarray, fmt: int,
     row_src = np.ascontiguousarray(row_src, dtype=np.int32)
     rows, two_i = gate_up_bits.shape
     I = two_i // 2
-    codes = np.empty((rows, I if fmt == FMT_MXFP8 else I // 2), np.uint8)
-    scales = np.empty((rows, I // 16 if fmt == FMT_NVFP4 else I // 32), np.uint8)
+    codes = np.empty((rows, swiglu_code_bytes(I, fmt)), np.uint8)
+    scales = np.empty((rows, swiglu_scale_bytes(I, fmt)), np.uint8)
     lib().orc_swiglu_quant(rows, I, _p(gate_up_bits), int(interleaved), _p(row_src), fmt,
                            float(np.float32(global_scale)), _p(codes), _p(scales))
     return codes, scales

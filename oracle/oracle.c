@@ -124,6 +124,65 @@ float orc_e2m1_to_f32(uint8_t c) {
   return (float)(s ? -v : v);
 }
 
+/* OCP MX v1.0 FP6 element formats, no infinities or NaN:
+ *   E2M3: exponent bias 1; normal (1 + m/8) * 2^(e-1), e in 1..3; subnormal
+ *         m/8; largest 7.5.
+ *   E3M2: exponent bias 3; normal (1 + m/4) * 2^(e-3), e in 1..7; subnormal
+ *         m/16; largest 28.
+ * Code layout: sign in bit 5, then the exponent, then the mantissa.        */
+static double fp6_magnitude(int code, int ebits) {
+  const int mbits = 5 - ebits, bias = ebits == 2 ? 1 : 3;
+  const int e = code >> mbits, m = code & ((1 << mbits) - 1);
+  if (e == 0) return ldexp((double)m, 1 - bias - mbits);
+  return ldexp(1.0 + (double)m / (double)(1 << mbits), e - bias);
+}
+
+/* Round to the nearest of the 32 magnitudes (searched one by one), ties to
+ * the even code, anything above the largest to the largest (saturation);
+ * the sign is kept, NaN maps to the signed largest value. */
+static uint8_t fp6_from_f32(float f, int ebits) {
+  const uint8_t sign = signbit(f) ? 0x20 : 0x00;
+  if (isnan(f)) return (uint8_t)(sign | 0x1F);
+  const double a = fabs((double)f);
+  if (a >= fp6_magnitude(31, ebits)) return (uint8_t)(sign | 31); /* saturate */
+  int best = 0;
+  for (int c = 1; c < 32; ++c) {
+    const double dc = fabs(a - fp6_magnitude(c, ebits));
+    const double db = fabs(a - fp6_magnitude(best, ebits));
+    if (dc < db || (dc == db && (c & 1) == 0)) best = c;
+  }
+  return (uint8_t)(sign | best);
+}
+
+uint8_t orc_e2m3_from_f32(float f) { return fp6_from_f32(f, 2); }
+uint8_t orc_e3m2_from_f32(float f) { return fp6_from_f32(f, 3); }
+float orc_e2m3_to_f32(uint8_t c) {
+  const double v = fp6_magnitude(c & 0x1F, 2);
+  return (float)((c & 0x20) ? -v : v);
+}
+float orc_e3m2_to_f32(uint8_t c) {
+  const double v = fp6_magnitude(c & 0x1F, 3);
+  return (float)((c & 0x20) ? -v : v);
+}
+void orc_e2m3_from_f32_n(const float *in, uint8_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m3_from_f32(in[i]);
+}
+void orc_e3m2_from_f32_n(const float *in, uint8_t *out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e3m2_from_f32(in[i]);
+}
+
+/* Four 6-bit codes in three bytes: code i at bits [6i, 6i + 6) of the
+ * little-endian 24-bit group. */
+void orc_pack_fp6(const uint8_t *codes, int64_t n, uint8_t *out) {
+  for (int64_t g = 0; g < n / 4; ++g) {
+    uint32_t w = 0;
+    for (int i = 0; i < 4; ++i) w |= (uint32_t)(codes[4 * g + i] & 0x3F) << (6 * i);
+    out[3 * g] = (uint8_t)(w & 0xFF);
+    out[3 * g + 1] = (uint8_t)((w >> 8) & 0xFF);
+    out[3 * g + 2] = (uint8_t)((w >> 16) & 0xFF);
+  }
+}
+
 void orc_bf16_from_f32_n(const float *in, uint16_t *out, int64_t n) {
   for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_from_f32(in[i]);
 }
@@ -375,6 +434,60 @@ void orc_permute_nvfp4(int64_t rows, int32_t H, const uint16_t *hidden,
   }
 }
 
+/* E8M0 code of the OCP MX shared scale of a block with largest magnitude
+ * amax > 0 (finite): X = floor(log2(amax)) - emax_elem, code = X + 127
+ * clamped to [0, 254]. */
+static uint8_t mx_scale_code(float amax, int32_t emax) {
+  int e;
+  frexpf(amax, &e); /* amax = f * 2^e, f in [0.5, 1) */
+  int32_t c = (e - 1) - emax + 127;
+  if (c < 0) c = 0;
+  if (c > 254) c = 254;
+  return (uint8_t)c;
+}
+
+/* y * 2^(127 - code): the MX scaling of an element (one rounding). */
+static float mx_scale_down(float y, uint8_t code) {
+  const int32_t X = (int32_t)code - 127;
+  return -X >= -126 ? y * f32_from_bits((uint32_t)(-X + 127) << 23)
+                    : (y * f32_from_bits((uint32_t)(-X - 64 + 127) << 23)) *
+                          f32_from_bits((uint32_t)(64 + 127) << 23);
+}
+
+/* Mojo MAX ep_comm MXTokenFormat (MX FP4 token format): OCP MX v1.0 MXFP4,
+ * blocks of 32 along H, E2M1 codes two per byte (element 2m in the low
+ * nibble of byte m), one E8M0 scale per block: X = floor(log2(amax)) - 2,
+ * code = E2M1 of x * 2^-X (nearest even, saturating); an all-zero block
+ * has scale code 0 and codes 0.  Scales row-major [rows, H/32].  Padding
+ * rows are all zero. */
+void orc_permute_mxfp4(int64_t rows, int32_t H, const uint16_t *hidden,
+                       const int32_t *row_src, uint8_t *q, uint8_t *scales) {
+  const int32_t nb = H / 32;
+  for (int64_t r = 0; r < rows; ++r) {
+    int32_t t = row_src[r];
+    for (int32_t b = 0; b < nb; ++b) {
+      uint8_t *qd = q + r * (H / 2) + (int64_t)b * 16;
+      uint8_t *sd = scales + r * nb + b;
+      memset(qd, 0, 16);
+      *sd = 0;
+      if (t < 0) continue;
+      const uint16_t *src = hidden + (int64_t)t * H + (int64_t)b * 32;
+      float amax = 0.0f;
+      for (int32_t i = 0; i < 32; ++i) {
+        float a = fabsf(orc_bf16_to_f32(src[i]));
+        if (a > amax) amax = a;
+      }
+      if (amax == 0.0f) continue;
+      const uint8_t sc = mx_scale_code(amax, 2);
+      *sd = sc;
+      for (int32_t i = 0; i < 32; ++i) {
+        const uint8_t c = orc_e2m1_from_f32(mx_scale_down(orc_bf16_to_f32(src[i]), sc));
+        qd[i / 2] |= (uint8_t)(i % 2 ? c << 4 : c);
+      }
+    }
+  }
+}
+
 /* Scale-factor atom layout: see oracle.h. */
 void orc_swizzle_scales(int64_t rows, int32_t nsf, const uint8_t *linear,
                         uint8_t *out) {
@@ -524,15 +637,18 @@ static int32_t floor_log2(float a) {
 void orc_swiglu_quant(int64_t rows, int32_t I, const uint16_t *gate_up,
                       int interleaved, const int32_t *row_src, int format,
                       float global_scale, uint8_t *codes, uint8_t *scales) {
-  const int64_t code_row = format == 1 ? I : I / 2;
-  const int64_t scale_row = format == 0 ? I / 16 : I / 32;
+  const int64_t code_row = format == 0 || format == 2 ? I / 2
+                           : format == 1               ? I
+                           : format == 3               ? 2 * (int64_t)I
+                                                       : 3 * (int64_t)I / 4;
+  const int64_t scale_row = format == 0 ? I / 16 : format == 3 ? 0 : I / 32;
   float *y = (float *)malloc(sizeof(float) * (size_t)I);
   for (int64_t r = 0; r < rows; ++r) {
     uint8_t *cd = codes + r * code_row;
     uint8_t *sd = scales + r * scale_row;
     if (row_src[r] < 0) {
       memset(cd, 0, (size_t)code_row);
-      memset(sd, 0, (size_t)scale_row);
+      if (scale_row) memset(sd, 0, (size_t)scale_row);
       continue;
     }
     const uint16_t *in = gate_up + r * 2 * (int64_t)I;
@@ -541,7 +657,37 @@ void orc_swiglu_quant(int64_t rows, int32_t I, const uint16_t *gate_up,
       float u = orc_bf16_to_f32(interleaved ? in[2 * i + 1] : in[I + i]);
       y[i] = orc_silu(g) * u;
     }
-    if (format == 0) {
+    if (format == 3) {
+      /* bf16, rounded to nearest even, little-endian */
+      for (int32_t i = 0; i < I; ++i) {
+        const uint16_t b = orc_bf16_from_f32(y[i]);
+        cd[2 * i] = (uint8_t)(b & 0xFF);
+        cd[2 * i + 1] = (uint8_t)(b >> 8);
+      }
+    } else if (format == 4 || format == 5) {
+      /* MXFP6: E2M3 (emax 2) or E3M2 (emax 4) codes, E8M0 scale per 32,
+       * 24 bytes of packed codes per block */
+      const int32_t emax = format == 4 ? 2 : 4;
+      uint8_t c6[32];
+      for (int32_t b = 0; b < I / 32; ++b) {
+        float amax = 0.0f;
+        for (int32_t i = 0; i < 32; ++i) {
+          float a = fabsf(y[32 * b + i]);
+          if (a > amax) amax = a;
+        }
+        uint8_t sc = 0;
+        memset(c6, 0, sizeof c6);
+        if (amax > 0.0f) {
+          sc = mx_scale_code(amax, emax);
+          for (int32_t i = 0; i < 32; ++i) {
+            const float v = mx_scale_down(y[32 * b + i], sc);
+            c6[i] = format == 4 ? orc_e2m3_from_f32(v) : orc_e3m2_from_f32(v);
+          }
+        }
+        sd[b] = sc;
+        orc_pack_fp6(c6, 32, cd + 24 * b);
+      }
+    } else if (format == 0) {
       /* NVFP4, exactly the dispatch's rule on the fp32 values */
       for (int32_t b = 0; b < I / 16; ++b) {
         float amax = 0.0f;

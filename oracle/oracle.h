@@ -64,6 +64,17 @@ float orc_e2m1_to_f32(uint8_t c);
 void orc_bf16_from_f32_n(const float *in, uint16_t *out, int64_t n);
 void orc_e4m3_from_f32_n(const float *in, uint8_t *out, int64_t n);
 void orc_e2m1_from_f32_n(const float *in, uint8_t *out, int64_t n);
+/* OCP MX v1.0 FP6: E2M3 (max 7.5) and E3M2 (max 28), 6-bit codes with the
+ * sign in bit 5; RNE, saturating, by nearest-value search over the codes. */
+uint8_t orc_e2m3_from_f32(float f);
+uint8_t orc_e3m2_from_f32(float f);
+float orc_e2m3_to_f32(uint8_t c);
+float orc_e3m2_to_f32(uint8_t c);
+void orc_e2m3_from_f32_n(const float *in, uint8_t *out, int64_t n);
+void orc_e3m2_from_f32_n(const float *in, uint8_t *out, int64_t n);
+/* n (a multiple of 4) 6-bit codes -> 3n/4 bytes: code i at bits [6i, 6i+6)
+ * of each little-endian 24-bit group of four. */
+void orc_pack_fp6(const uint8_t *codes, int64_t n, uint8_t *out);
 
 /* ---- dispatch layout --------------------------------------------------
  * ids[N*k] int32 (row-major [N,k]); E experts in S contiguous segments of
@@ -100,6 +111,11 @@ void orc_permute_fp8(int64_t rows, int32_t H, const uint16_t *hidden,
 void orc_permute_nvfp4(int64_t rows, int32_t H, const uint16_t *hidden,
                        const int32_t *row_src, float global_scale,
                        uint8_t *q, uint8_t *scales);
+/* MX token format (OCP MXFP4): E2M1 codes [rows, H/2], E8M0 scales
+ * [rows, H/32]; X = floor(log2(amax)) - 2 per block of 32, codes of
+ * x * 2^-X; an all-zero block has scale code 0. */
+void orc_permute_mxfp4(int64_t rows, int32_t H, const uint16_t *hidden,
+                       const int32_t *row_src, uint8_t *q, uint8_t *scales);
 
 /* ---- combine ---------------------------------------------------------- */
 void orc_combine(int32_t N, int32_t k, int32_t H, int64_t rows,
@@ -127,7 +143,11 @@ void orc_exp_n(const float *in, float *out, int64_t n);
  *            the dispatch (global scale gs)
  *   format 1 MXFP8: E4M3 codes [rows, I], E8M0 scales [rows, I/32]
  *   format 2 MXFP4: E2M1 codes [rows, I/2], E8M0 scales [rows, I/32]
- * MX block of 32: X = floor(log2(amax)) - emax (8 for E4M3, 2 for E2M1),
+ *   format 3 BF16:  bf16 [rows, I] (2I bytes a row, little-endian), no scales
+ *   format 4 MXFP6 E2M3: packed 6-bit codes [rows, 3I/4], E8M0 [rows, I/32]
+ *   format 5 MXFP6 E3M2: packed 6-bit codes [rows, 3I/4], E8M0 [rows, I/32]
+ * MX block of 32: X = floor(log2(amax)) - emax (8 for E4M3, 2 for E2M1 and
+ * E2M3, 4 for E3M2),
  * scale code E8M0(X), element code = E(y * 2^-X) rounded to nearest even with
  * saturation; an all-zero block gets scale code 0 and codes 0.  Rows whose
  * row_src is -1 (no routed token) are all-zero bytes and are not read.     */
