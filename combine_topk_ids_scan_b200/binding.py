@@ -38,10 +38,12 @@ MOE_MAX_TOPK = 16
 # every symbol include/moe_dc.h declares
 EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout",
             "moe_dispatch_layout_noalloc", "moe_permute", "moe_permute_quant_fp8",
-            "moe_permute_quant_nvfp4", "moe_combine", "moe_permute_backward",
+            "moe_permute_quant_nvfp4", "moe_permute_quant_mxfp4", "moe_combine",
+            "moe_permute_backward",
             "moe_combine_backward", "moe_swiglu_quant", "moe_status_string", "moe_version")
 
-MOE_QUANT_NVFP4, MOE_QUANT_MXFP8, MOE_QUANT_MXFP4 = 0, 1, 2
+(MOE_QUANT_NVFP4, MOE_QUANT_MXFP8, MOE_QUANT_MXFP4, MOE_QUANT_BF16, MOE_QUANT_MXFP6_E2M3,
+ MOE_QUANT_MXFP6_E3M2) = 0, 1, 2, 3, 4, 5
 MOE_GATE_UP_SPLIT, MOE_GATE_UP_INTERLEAVED = 0, 1
 
 MOE_NOALLOC_SCRATCH_BYTES = 1 << 20
@@ -109,6 +111,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     L.moe_permute_quant_fp8.argtypes = [P] + [vp] * 6
     L.moe_permute_quant_nvfp4.restype = ctypes.c_int
     L.moe_permute_quant_nvfp4.argtypes = [P] + [vp] * 7
+    L.moe_permute_quant_mxfp4.restype = ctypes.c_int
+    L.moe_permute_quant_mxfp4.argtypes = [P] + [vp] * 6
     L.moe_combine.restype = ctypes.c_int
     L.moe_combine.argtypes = [P] + [vp] * 5
     L.moe_permute_backward.restype = ctypes.c_int
@@ -207,15 +211,25 @@ def moe_permute_quant_nvfp4(prob: Problem, hidden_states, row_src, pair_slot, gl
            "moe_permute_quant_nvfp4")
 
 
+def moe_permute_quant_mxfp4(prob: Problem, hidden_states, row_src, pair_slot, out_e2m1,
+                            scales_e8m0, stream=None) -> None:
+    c = prob.c()
+    _check(load().moe_permute_quant_mxfp4(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
+                                          _ptr(pair_slot), _ptr(out_e2m1), _ptr(scales_e8m0),
+                                          _stream(stream)),
+           "moe_permute_quant_mxfp4")
+
+
 def moe_combine(prob: Problem, expert_out, gates, pair_slot, out, stream=None) -> None:
     c = prob.c()
     _check(load().moe_combine(ctypes.byref(c), _ptr(expert_out), _ptr(gates), _ptr(pair_slot),
                               _ptr(out), _stream(stream)), "moe_combine")
 
 
-def nvfp4_swizzled_scale_bytes(rows: int, hidden: int) -> int:
-    """Bytes of NVFP4 scales in the 128x4 atom layout (see moe_dc.h)."""
-    return max(1, -(-rows // 128) * 128 * (-(-hidden // 64) * 4))
+def nvfp4_swizzled_scale_bytes(rows: int, hidden: int, block: int = 16) -> int:
+    """Bytes of FP4 block scales (block 16: NVFP4, 32: MXFP4) in the 128x4
+    atom layout (see moe_dc.h)."""
+    return max(1, -(-rows // 128) * 128 * (-(-(hidden // block) // 4) * 4))
 
 
 def moe_permute_backward(prob: Problem, grad_out, pair_slot, grad_hidden, stream=None) -> None:
@@ -245,10 +259,12 @@ def moe_swiglu_quant(prob: Problem, intermediate: int, fmt: int, gate_up_layout:
 def swiglu_buffers(rows: int, intermediate: int, fmt: int, device="cuda"):
     """(codes, scales) uint8 device buffers for moe_swiglu_quant."""
     I = intermediate
-    codes = torch.empty((max(rows, 1), I if fmt == MOE_QUANT_MXFP8 else I // 2),
-                        dtype=torch.uint8, device=device)
-    scales = torch.empty((max(rows, 1), I // 16 if fmt == MOE_QUANT_NVFP4 else I // 32),
-                         dtype=torch.uint8, device=device)
+    code_bytes = {MOE_QUANT_NVFP4: I // 2, MOE_QUANT_MXFP8: I, MOE_QUANT_MXFP4: I // 2,
+                  MOE_QUANT_BF16: 2 * I, MOE_QUANT_MXFP6_E2M3: 3 * I // 4,
+                  MOE_QUANT_MXFP6_E3M2: 3 * I // 4}[fmt]
+    scale_bytes = I // 16 if fmt == MOE_QUANT_NVFP4 else 0 if fmt == MOE_QUANT_BF16 else I // 32
+    codes = torch.empty((max(rows, 1), code_bytes), dtype=torch.uint8, device=device)
+    scales = torch.empty((max(rows, 1), max(scale_bytes, 1)), dtype=torch.uint8, device=device)
     return codes, scales
 
 
@@ -282,9 +298,14 @@ class Buffers:
             if prob.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES:
                 self.scales_fp4 = torch.empty(nvfp4_swizzled_scale_bytes(rows, H), dtype=u8,
                                               device=device)
+                self.scales_mx4 = torch.empty(nvfp4_swizzled_scale_bytes(rows, H, 32),
+                                              dtype=u8, device=device)
             else:
                 self.scales_fp4 = torch.empty((max(rows, 1), max(H // 16, 1)), dtype=u8,
                                               device=device)
+                self.scales_mx4 = torch.empty((max(rows, 1), max(H // 32, 1)), dtype=u8,
+                                              device=device)
+            self.out_mx4 = torch.empty((max(rows, 1), H // 2), dtype=u8, device=device)
 
 
 def layout(prob: Problem, topk_ids: torch.Tensor, buf: Buffers, stream=None) -> None:

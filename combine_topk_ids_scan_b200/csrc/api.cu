@@ -157,6 +157,24 @@ moe_status moe_permute_quant_nvfp4(const moe_problem *problem, const void *hidde
                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_permute_quant_mxfp4(const moe_problem *problem, const void *hidden_states,
+                                   const int32_t *row_src, const int32_t *pair_slot,
+                                   uint8_t *out_e2m1, uint8_t *scales_e8m0, moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 32 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.rows == 0) return MOE_OK;
+  if (!row_src || !out_e2m1 || !scales_e8m0 || (s.P > 0 && (!hidden_states || !pair_slot)))
+    return MOE_ERR_INVALID_ARG;
+  const uintptr_t scale_align = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) ? 4 : 1;
+  if (!aligned(hidden_states, 16) || !aligned(out_e2m1, 16) || !aligned(scales_e8m0, scale_align))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_permute_mxfp4(s, hidden_states, row_src, pair_slot, out_e2m1,
+                                             scales_e8m0,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_combine(const moe_problem *problem, const void *expert_out, const float *gates,
                        const int32_t *pair_slot, void *out, moe_stream_t stream) {
   moe::Shape s;
@@ -212,16 +230,20 @@ moe_status moe_swiglu_quant(const moe_problem *problem, int32_t intermediate, ui
   moe::Shape s;
   moe_status st = make_shape(problem, &s);
   if (st != MOE_OK) return st;
-  if (intermediate <= 0 || format > MOE_QUANT_MXFP4 || gate_up_layout > MOE_GATE_UP_INTERLEAVED)
+  if (intermediate <= 0 || format > MOE_QUANT_MXFP6_E3M2 ||
+      gate_up_layout > MOE_GATE_UP_INTERLEAVED)
     return MOE_ERR_INVALID_ARG;
   if (intermediate % 32 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   const int64_t I = intermediate;
   if (s.rows * 2 * I > 2147483647ll * 8) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (s.rows == 0) return MOE_OK;
-  if (!gate_up || !row_src || !codes || !scales || (format == MOE_QUANT_NVFP4 && !global_scale))
+  const bool has_scales = format != MOE_QUANT_BF16;
+  if (!gate_up || !row_src || !codes || (has_scales && !scales) ||
+      (format == MOE_QUANT_NVFP4 && !global_scale))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned(gate_up, 16) || !aligned(codes, 16) ||
-      !aligned(scales, format == MOE_QUANT_NVFP4 ? 2 : 1) ||
+  const bool fp6 = format == MOE_QUANT_MXFP6_E2M3 || format == MOE_QUANT_MXFP6_E3M2;
+  if (!aligned(gate_up, 16) || !aligned(codes, fp6 ? 8 : 16) ||
+      (has_scales && !aligned(scales, format == MOE_QUANT_NVFP4 ? 2 : 1)) ||
       (global_scale && !aligned(global_scale, 4)))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_swiglu_quant(s, intermediate, format,

@@ -90,6 +90,25 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
   return r;
 }
 
+// floor(log2(a)) of a finite a > 0, subnormals included.
+__device__ __forceinline__ int floor_log2(float a) {
+  const uint32_t b = __float_as_uint(a);
+  const int e = (int)((b >> 23) & 0xFFu);
+  if (e != 0) return e - 127;
+  return (31 - __clz((int)(b & 0x7FFFFFu))) - 149;
+}
+
+// 2^n as a float for n in [-126, 127].
+__device__ __forceinline__ float pow2i(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
+
+// E8M0 code of the OCP MX shared scale of a block with largest magnitude
+// amax > 0 (finite): X = floor(log2(amax)) - emax, code clamp(X + 127, 0, 254).
+// For every emax >= 2 used here, 2^(127 - code) is a normal float, so the
+// element scaling y * 2^-X is a single multiply.
+__device__ __forceinline__ uint32_t mx_scale_code(float amax, int emax) {
+  return (uint32_t)min(254, max(0, floor_log2(amax) - emax + 127));
+}
+
 // One E4M3 code -> float (exact): through the f16x2 conversion.
 __device__ __forceinline__ float e4m3_to_float(uint32_t code) {
   uint32_t h2;

@@ -47,6 +47,10 @@ cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32
                                  const int32_t *pair_slot, const float *global_scale,
                                  uint8_t *q, uint8_t *scales, cudaStream_t stream);
 
+cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32_t *row_src,
+                                 const int32_t *pair_slot, uint8_t *q, uint8_t *scales,
+                                 cudaStream_t stream);
+
 // gates == nullptr: unit weights (the dispatch backward)
 cudaError_t launch_combine(const Shape &s, const void *expert_out, const float *gates,
                            const int32_t *pair_slot, void *out, cudaStream_t stream);

@@ -239,6 +239,32 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float *f, float gs, uint32
   return sq;
 }
 
+// MX token format (OCP MXFP4): one block of 32 -> 16 bytes of E2M1 codes and
+// the E8M0 scale code; an all-zero block is scale 0, codes 0.
+__device__ __forceinline__ uint32_t mxfp4_block(const float *f, uint4 &codes) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  uint32_t c[4] = {0, 0, 0, 0};
+  uint32_t sc = 0;
+  if (amax > 0.0f) {
+    sc = mx_scale_code(amax, 2);
+    const float m = pow2i(127 - (int)sc);  // 2^-X, a normal float
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = 8 * h + 2 * j;
+        word |= cvt_e2m1x2(__fmul_rn(f[i], m), __fmul_rn(f[i + 1], m)) << (8 * j);
+      }
+      c[h] = word;
+    }
+  }
+  codes = make_uint4(c[0], c[1], c[2], c[3]);
+  return sc;
+}
+
 // Block-scale atom layout (Mojo MAX ep_comm SF_ATOM_M = (32, 4),
 // SF_ROW_STRIDE_LOCAL = 16, SF_ATOM_ELEMS_LOCAL = 512): byte of scale (m, c)
 // when a 128-row tile spans `col_tiles` atoms.
@@ -246,12 +272,15 @@ __device__ __forceinline__ int64_t sf_atom_offset(int64_t m, int32_t c, int32_t 
   return ((m >> 7) * col_tiles + (c >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (c & 3);
 }
 
+// MX == false: NVFP4 (two 16-element blocks per lane, E4M3 scales);
+// MX == true: MXFP4 (one 32-element block per lane, E8M0 scales).
+template <bool MX>
 __global__ void __launch_bounds__(kThreads)
-    permute_nvfp4_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
-                         const int32_t *__restrict__ pair_slot,
-                         const float *__restrict__ global_scale, uint8_t *__restrict__ q,
-                         uint8_t *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
-                         int32_t H, int32_t chunks, bool swizzled) {
+    permute_fp4_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
+                       const int32_t *__restrict__ pair_slot,
+                       const float *__restrict__ global_scale, uint8_t *__restrict__ q,
+                       uint8_t *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
+                       int32_t H, int32_t chunks, bool swizzled) {
   const int lane = threadIdx.x % kWarp;
   const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
@@ -260,13 +289,24 @@ __global__ void __launch_bounds__(kThreads)
   const int64_t check_rows = swizzled ? (rows + 127) / 128 * 128 : rows;
   const int64_t pad_units = (check_rows + kWarp - 1) / kWarp;
   const int32_t vecs = H / 8;
-  const int32_t qrow = H / 2, srow = H / 16;
+  const int32_t qrow = H / 2, srow = MX ? H / 32 : H / 16;
   const int32_t groups = (srow + 3) / 4;  // 4-scale groups per row (atom layout)
   if (w0 < pad_units) {
-    // codes: H/2 bytes per row; scales: linear H/16 bytes per row, or the
+    // codes: H/2 bytes per row; scales: linear srow bytes per row, or the
     // row's `groups` 4-byte groups in the atom layout
     const uint32_t m = padding_mask(w0, lane, row_src, rows, check_rows);
-    if (m && !swizzled) {
+    if (m && !swizzled && MX) {
+      uint32_t mm = m;
+      const uint4 zero = make_uint4(0, 0, 0, 0);
+      while (mm) {
+        const int j = __ffs(mm) - 1;
+        mm &= mm - 1;
+        const int64_t row = w0 * kWarp + j;
+        uint4 *dst = reinterpret_cast<uint4 *>(q) + row * (qrow / 16);
+        for (int v = lane; v < qrow / 16; v += kWarp) st_v4(dst + v, zero);
+        for (int v = lane; v < srow; v += kWarp) scales[row * srow + v] = 0;
+      }
+    } else if (m && !swizzled) {
       zero_rows(m, w0, lane, reinterpret_cast<uint4 *>(q), qrow / 16, 0, qrow / 16,
                 reinterpret_cast<uint16_t *>(scales), srow / 2, 0, srow / 2);
     } else if (m) {
@@ -294,7 +334,7 @@ __global__ void __launch_bounds__(kThreads)
     const bool active = col < H;
     int32_t my_slot;
     uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
-    const float gs = __ldg(global_scale);
+    const float gs = MX ? 0.0f : __ldg(global_scale);
     const uint4 *src = hidden + t * vecs;
     uint4 x[4];
 #pragma unroll
@@ -311,24 +351,38 @@ __global__ void __launch_bounds__(kThreads)
       }
     }
     uint4 codes;
-    const uint32_t sq0 = nvfp4_block(f, gs, codes.x, codes.y);
-    const uint32_t sq1 = nvfp4_block(f + 16, gs, codes.z, codes.w);
-    const uint32_t sq = sq0 | (sq1 << 8);
-    // atom layout: an even lane holds scale columns 4g, 4g+1 and its odd
-    // neighbour 4g+2, 4g+3 -- one 4-byte store per pair of lanes (an
-    // inactive neighbour contributes zeros: the column padding of a partial
-    // last group)
-    const uint32_t quad = sq | (__shfl_down_sync(kFull, active ? sq : 0u, 1) << 16);
+    uint32_t sq, quad;
+    if (MX) {
+      sq = mxfp4_block(f, codes);
+      // atom layout: lanes 4g..4g+3 hold scale columns 4g..4g+3 -- one
+      // 4-byte store per four lanes (inactive lanes contribute zeros: the
+      // column padding of a partial last group)
+      const uint32_t a = active ? sq : 0u;
+      quad = a | (__shfl_down_sync(kFull, a, 1) << 8) | (__shfl_down_sync(kFull, a, 2) << 16) |
+             (__shfl_down_sync(kFull, a, 3) << 24);
+    } else {
+      const uint32_t sq0 = nvfp4_block(f, gs, codes.x, codes.y);
+      const uint32_t sq1 = nvfp4_block(f + 16, gs, codes.z, codes.w);
+      sq = sq0 | (sq1 << 8);
+      // atom layout: an even lane holds scale columns 4g, 4g+1 and its odd
+      // neighbour 4g+2, 4g+3 -- one 4-byte store per pair of lanes (an
+      // inactive neighbour contributes zeros: the column padding of a
+      // partial last group)
+      quad = sq | (__shfl_down_sync(kFull, active ? sq : 0u, 1) << 16);
+    }
+    const int sc_col = MX ? col / 32 : col / 16;
     while (live) {
       const int j = __ffs(live) - 1;
       live &= live - 1;
       const int64_t s = __shfl_sync(kFull, my_slot, j);
       if (active) {
         st_v4(reinterpret_cast<uint4 *>(q + s * qrow + col / 2), codes);
-        if (!swizzled)
-          *reinterpret_cast<uint16_t *>(scales + s * srow + col / 16) = (uint16_t)sq;
-        else if ((lane & 1) == 0)
-          *reinterpret_cast<uint32_t *>(scales + sf_atom_offset(s, col / 16, groups)) = quad;
+        if (!swizzled) {
+          if (MX) scales[s * srow + sc_col] = (uint8_t)sq;
+          else *reinterpret_cast<uint16_t *>(scales + s * srow + sc_col) = (uint16_t)sq;
+        } else if ((lane & (MX ? 3 : 1)) == 0) {
+          *reinterpret_cast<uint32_t *>(scales + sf_atom_offset(s, sc_col, groups)) = quad;
+        }
       }
     }
   }
@@ -373,9 +427,24 @@ cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32
   const int32_t chunks = chunks_of(s.H, kChunk);
   const bool swizzled = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) != 0;
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
-  permute_nvfp4_kernel<<<(unsigned)unit_blocks(s, chunks, check_rows), kThreads, 0, stream>>>(
-      static_cast<const uint4 *>(hidden), row_src, pair_slot, global_scale, q, scales, s.N, s.k,
-      s.rows, s.H, chunks, swizzled);
+  permute_fp4_kernel<false>
+      <<<(unsigned)unit_blocks(s, chunks, check_rows), kThreads, 0, stream>>>(
+          static_cast<const uint4 *>(hidden), row_src, pair_slot, global_scale, q, scales, s.N,
+          s.k, s.rows, s.H, chunks, swizzled);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32_t *row_src,
+                                 const int32_t *pair_slot, uint8_t *q, uint8_t *scales,
+                                 cudaStream_t stream) {
+  if (s.rows == 0) return cudaSuccess;
+  const int32_t chunks = chunks_of(s.H, kChunk);
+  const bool swizzled = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) != 0;
+  const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
+  permute_fp4_kernel<true>
+      <<<(unsigned)unit_blocks(s, chunks, check_rows), kThreads, 0, stream>>>(
+          static_cast<const uint4 *>(hidden), row_src, pair_slot, nullptr, q, scales, s.N, s.k,
+          s.rows, s.H, chunks, swizzled);
   return cudaGetLastError();
 }
 

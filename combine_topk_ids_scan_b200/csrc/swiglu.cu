@@ -49,7 +49,6 @@ constexpr uint32_t kTabFirst = 0x3300u;
 constexpr int kTabHalf = 4096;
 constexpr int kTabSize = 2 * kTabHalf;
 
-__device__ __forceinline__ float pow2i(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
 
 // max / min that return NaN when either operand is NaN
 __device__ __forceinline__ float max_nan(float a, float b) {
@@ -155,6 +154,35 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4(float2 a, float2 b) {
   return r;
 }
 
+// Eight floats -> eight OCP MX FP6 codes (E2M3 or E3M2, nearest even,
+// saturating), packed at bits [6i, 6i + 6) of a 48-bit little-endian value
+// returned as (low 32 bits, high 16 bits).  The conversion leaves each 6-bit
+// code in the low bits of its byte.
+template <bool E2M3>
+__device__ __forceinline__ void cvt_fp6x8(const float2 *v, uint32_t &lo32, uint32_t &hi16) {
+  uint32_t p[4];  // p[i] = code(2i) | code(2i + 1) << 8
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (E2M3)
+      asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e2m3x2.f32 t, %2, %1;\n\t"
+          "cvt.u32.u16 %0, t;\n\t}"
+          : "=r"(p[i])
+          : "f"(v[i].x), "f"(v[i].y));
+    else
+      asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e3m2x2.f32 t, %2, %1;\n\t"
+          "cvt.u32.u16 %0, t;\n\t}"
+          : "=r"(p[i])
+          : "f"(v[i].x), "f"(v[i].y));
+  }
+  // two codes a | b << 8 -> a | b << 6 (12 bits)
+  uint32_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) q[i] = p[i] - 192u * (p[i] >> 8);
+  const uint32_t g0 = q[0] | (q[1] << 12), g1 = q[2] | (q[3] << 12);  // 24 bits each
+  lo32 = g0 | (g1 << 24);
+  hi16 = g1 >> 8;
+}
+
 // Bits 12..15 and 28..31 of the result are zero iff both bf16 of w are in
 // the table: for a magnitude in [0x3300, 0x4300), magnitude + 0x4D00 lies in
 // [0x8000, 0x9000) (and never carries into the other half, being at most
@@ -183,13 +211,6 @@ __device__ __forceinline__ float2 e2m1_quotient2(float2 a, float d, float rd) {
   return make_float2(copysignf(q.x, a.x), copysignf(q.y, a.y));
 }
 
-// floor(log2(a)) of a finite a > 0, subnormals included.
-__device__ __forceinline__ int floor_log2(float a) {
-  const uint32_t b = __float_as_uint(a);
-  const int e = (int)((b >> 23) & 0xFFu);
-  if (e != 0) return e - 127;
-  return (31 - __clz((int)(b & 0x7FFFFFu))) - 149;
-}
 
 // One lane's 32 columns [c, c + 32) of row r.
 template <int FORMAT, bool INTERLEAVED>
@@ -198,17 +219,24 @@ __device__ __forceinline__ void swiglu_group(const float *tab, const uint4 *__re
                                              uint8_t *__restrict__ codes,
                                              uint8_t *__restrict__ scales, int64_t r, int32_t c,
                                              int32_t I) {
-  const int64_t code_row = FORMAT == 1 ? I : I / 2;
+  // bytes of codes per column group of 32 and per row
+  constexpr int kCodeBytes = FORMAT == 1 ? 32 : FORMAT == 3 ? 64 : FORMAT >= 4 ? 24 : 16;
+  const int64_t code_row = (int64_t)I / 32 * kCodeBytes;
   const int64_t scale_row = FORMAT == 0 ? I / 16 : I / 32;
-  uint8_t *cd = codes + r * code_row + (FORMAT == 1 ? c : c / 2);
+  uint8_t *cd = codes + r * code_row + (int64_t)(c / 32) * kCodeBytes;
   uint8_t *sd = scales + r * scale_row + (FORMAT == 0 ? c / 16 : c / 32);
 
   if (__ldg(row_src + r) < 0) {  // no routed token: zero bytes, input not read
-    const uint4 zero = make_uint4(0, 0, 0, 0);
-    st_v4(reinterpret_cast<uint4 *>(cd), zero);
-    if (FORMAT == 1) st_v4(reinterpret_cast<uint4 *>(cd) + 1, zero);
+    if (kCodeBytes == 24) {
+      uint2 *d2 = reinterpret_cast<uint2 *>(cd);
+#pragma unroll
+      for (int i = 0; i < 3; ++i) d2[i] = make_uint2(0, 0);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kCodeBytes / 16; ++i) st_v4(reinterpret_cast<uint4 *>(cd) + i, make_uint4(0, 0, 0, 0));
+    }
     if (FORMAT == 0) *reinterpret_cast<uint16_t *>(sd) = 0;
-    else *sd = 0;
+    else if (FORMAT != 3) *sd = 0;
     return;
   }
 
@@ -270,7 +298,47 @@ __device__ __forceinline__ void swiglu_group(const float *tab, const uint4 *__re
       y[4 * i + e] = __fmul2_rn(y[4 * i + e], make_float2(bf16lo(u4[e]), bf16hi(u4[e])));
   }
 
-  if (FORMAT == 0) {
+  if (FORMAT == 3) {
+    // ---- bf16, rounded to nearest even
+    uint32_t w[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(y[j].x, y[j].y);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      st_v4(reinterpret_cast<uint4 *>(cd) + i,
+            make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+  } else if (FORMAT >= 4) {
+    // ---- MXFP6 (E2M3 emax 2, E3M2 emax 4): one block of 32, 24 bytes
+    constexpr int kEmax = FORMAT == 4 ? 2 : 4;
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) amax = max_abs3(amax, y[j].x, y[j].y);
+    uint32_t sc = 0;
+    uint32_t cw[6] = {0, 0, 0, 0, 0, 0};
+    if (amax > 0.0f) {
+      sc = mx_scale_code(amax, kEmax);
+      const float2 s2 = splat(pow2i(127 - (int)sc));
+      float2 v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = __fmul2_rn(y[j], s2);
+      // 48 bits per 8 codes: words (lo, hi16) of four groups -> six words
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) cvt_fp6x8<FORMAT == 4>(v + 4 * g, lo[g], hi[g]);
+      // group g occupies bits [48g, 48g + 48) of the 192-bit run
+      cw[0] = lo[0];
+      cw[1] = hi[0] | (lo[1] << 16);
+      cw[2] = (lo[1] >> 16) | (hi[1] << 16);
+      cw[3] = lo[2];
+      cw[4] = hi[2] | (lo[3] << 16);
+      cw[5] = (lo[3] >> 16) | (hi[3] << 16);
+    }
+    uint2 *d2 = reinterpret_cast<uint2 *>(cd);
+    d2[0] = make_uint2(cw[0], cw[1]);
+    d2[1] = make_uint2(cw[2], cw[3]);
+    d2[2] = make_uint2(cw[4], cw[5]);
+    *sd = (uint8_t)sc;
+  } else if (FORMAT == 0) {
     // ---- NVFP4: the dispatch's rule on the fp32 values, two blocks of 16
     uint32_t cw[4] = {0, 0, 0, 0};
     uint32_t sq2 = 0;
@@ -308,7 +376,7 @@ __device__ __forceinline__ void swiglu_group(const float *tab, const uint4 *__re
     uint32_t sc = 0;
     uint32_t cw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (amax > 0.0f) {
-      sc = (uint32_t)min(254, max(0, floor_log2(amax) - kEmax + 127));
+      sc = mx_scale_code(amax, kEmax);
       // X = sc - 127 lies in [-127, 127 - kEmax], so 2^-X is a normal float
       // and y * 2^-X is one rounding
       const float2 s2 = splat(pow2i(127 - (int)sc));
@@ -397,14 +465,22 @@ cudaError_t launch_swiglu_quant(const Shape &s, int32_t I, uint32_t format, bool
                                 cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
   const uint4 *in = static_cast<const uint4 *>(gate_up);
+#define MOE_SWIGLU_CASE(F)                                                                 \
+  case 2 * F:                                                                              \
+    return launch<F, false>(in, row_src, global_scale, codes, scales, s.rows, I, stream);   \
+  case 2 * F + 1:                                                                          \
+    return launch<F, true>(in, row_src, global_scale, codes, scales, s.rows, I, stream);
   switch (format * 2 + (interleaved ? 1 : 0)) {
-    case 0: return launch<0, false>(in, row_src, global_scale, codes, scales, s.rows, I, stream);
-    case 1: return launch<0, true>(in, row_src, global_scale, codes, scales, s.rows, I, stream);
-    case 2: return launch<1, false>(in, row_src, global_scale, codes, scales, s.rows, I, stream);
-    case 3: return launch<1, true>(in, row_src, global_scale, codes, scales, s.rows, I, stream);
-    case 4: return launch<2, false>(in, row_src, global_scale, codes, scales, s.rows, I, stream);
-    default: return launch<2, true>(in, row_src, global_scale, codes, scales, s.rows, I, stream);
+    MOE_SWIGLU_CASE(0)
+    MOE_SWIGLU_CASE(1)
+    MOE_SWIGLU_CASE(2)
+    MOE_SWIGLU_CASE(3)
+    MOE_SWIGLU_CASE(4)
+    MOE_SWIGLU_CASE(5)
+    default:
+      return cudaErrorInvalidValue;
   }
+#undef MOE_SWIGLU_CASE
 }
 
 }  // namespace moe

@@ -259,6 +259,24 @@ MOE_API moe_status moe_permute_quant_nvfp4(const moe_problem *problem, const voi
                                    const float *global_scale, uint8_t *out_e2m1,
                                    uint8_t *scales_e4m3, moe_stream_t stream);
 
+/* MX token format (Mojo MAX ep_comm MXTokenFormat: MX FP4 quantisation of
+ * the dispatched tokens; OCP Microscaling v1.0 MXFP4).  Same rows as
+ * moe_permute; per block of 32 elements along H:
+ *   X = floor(log2(amax)) - 2,  scale code = clamp(X + 127, 0, 254) (E8M0),
+ *   code_i = E2M1_rne_satfinite(x_i * 2^-X);
+ * an all-zero block has scale code 0 and codes 0.
+ *   out_e2m1     uint8 [rows, H/2], element 2m in the low nibble of byte m,
+ *                16-byte aligned, fully overwritten (padding rows 0)
+ *   scales_e8m0  uint8 [rows, H/32] row-major, or, with
+ *                MOE_FLAG_NVFP4_SWIZZLED_SCALES, the block-scale atom layout
+ *                of moe_permute_quant_nvfp4 with H/32 scale columns
+ *                (4-byte aligned then); fully overwritten
+ * Requires H % 32 == 0. */
+MOE_API moe_status moe_permute_quant_mxfp4(const moe_problem *problem, const void *hidden_states,
+                                   const int32_t *row_src, const int32_t *pair_slot,
+                                   uint8_t *out_e2m1, uint8_t *scales_e8m0,
+                                   moe_stream_t stream);
+
 /* Combine (DeepSpeed: gather each token's expert results back and weight
  * them by the gate values; NeMo moe_router_dtype 'fp32'; Mojo MAX ep_comm
  * router_weights_wrapper_type: one fp32 weight per (token, k)).
@@ -277,7 +295,8 @@ MOE_API moe_status moe_combine(const moe_problem *problem, const void *expert_ou
 /* ---- fused SwiGLU + requantisation -----------------------------------------
  * The step after the experts' gate/up projection (Mojo MAX ep_comm:
  * fused_silu_kernel, fused_silu_mx_kernel, fused_silu_nvfp4_kernel,
- * fused_silu_mxfp8_interleaved_kernel, MXTokenFormat).  The host does not know
+ * fused_silu_nvfp4_interleaved_kernel, fused_silu_mxfp8_interleaved_kernel,
+ * fused_silu_mxfp6_kernel).  The host does not know
  * how many rows each expert received, so the kernel takes the layout's
  * row_src: a row without a routed token (-1) is written as zero bytes and its
  * input is not read.  For the other rows, per column i < I:
@@ -291,18 +310,33 @@ MOE_API moe_status moe_combine(const moe_problem *problem, const void *expert_ou
  *   MOE_QUANT_MXFP8  codes E4M3 [rows, I], scales E8M0 [rows, I/32]
  *   MOE_QUANT_MXFP4  codes E2M1 [rows, I/2] (element 2m low nibble), scales
  *                    E8M0 [rows, I/32]
+ *   MOE_QUANT_BF16   y rounded to bf16 (nearest even) [rows, I]; no scales
+ *                    (scales may be NULL)
+ *   MOE_QUANT_MXFP6_E2M3, MOE_QUANT_MXFP6_E3M2
+ *                    OCP MX FP6 codes (6 bits: sign, exponent, mantissa;
+ *                    E2M3 max 7.5, E3M2 max 28) packed densely [rows, 3I/4]:
+ *                    code i of a row at bits [6i, 6i+6) of the row's
+ *                    little-endian bit stream (4 codes in 3 bytes); scales
+ *                    E8M0 [rows, I/32]
  * MX (OCP Microscaling v1.0): per block of 32, X = floor(log2(amax)) - emax
- * (emax 8 for E4M3, 2 for E2M1), scale code clamp(X + 127, 0, 254), code =
- * E(y * 2^-X) rounded to nearest even, saturating; an all-zero block gets
- * scale code 0 and codes 0.
+ * (emax 8 for E4M3, 2 for E2M1 and E2M3, 4 for E3M2), scale code
+ * clamp(X + 127, 0, 254), code = E(y * 2^-X) rounded to nearest even,
+ * saturating; an all-zero block gets scale code 0 and codes 0.
  *   gate_up  bf16 [rows, 2*I], 16-byte aligned: MOE_GATE_UP_SPLIT = columns
  *            [0, I) gate and [I, 2I) up; MOE_GATE_UP_INTERLEAVED = gate at
  *            even and up at odd columns
  *   row_src  int32 [rows] from the layout
- *   codes    16-byte aligned; scales 2-byte aligned (NVFP4); both fully
- *            overwritten
+ *   codes    16-byte aligned (8 for MXFP6); scales 2-byte aligned (NVFP4);
+ *            both fully overwritten
  * Requires I % 32 == 0. */
-enum { MOE_QUANT_NVFP4 = 0, MOE_QUANT_MXFP8 = 1, MOE_QUANT_MXFP4 = 2 };
+enum {
+  MOE_QUANT_NVFP4 = 0,
+  MOE_QUANT_MXFP8 = 1,
+  MOE_QUANT_MXFP4 = 2,
+  MOE_QUANT_BF16 = 3,
+  MOE_QUANT_MXFP6_E2M3 = 4,
+  MOE_QUANT_MXFP6_E3M2 = 5
+};
 enum { MOE_GATE_UP_SPLIT = 0, MOE_GATE_UP_INTERLEAVED = 1 };
 MOE_API moe_status moe_swiglu_quant(const moe_problem *problem, int32_t intermediate,
                                     uint32_t format, uint32_t gate_up_layout,

@@ -47,6 +47,8 @@ class GpuRun:
             gs = torch.tensor([w.global_scale], dtype=torch.float32, device="cuda")
             B.moe_permute_quant_nvfp4(prob, hidden, buf.row_src, buf.pair_slot, gs,
                                       buf.out_fp4, buf.scales_fp4)
+            B.moe_permute_quant_mxfp4(prob, hidden, buf.row_src, buf.pair_slot, buf.out_mx4,
+                                      buf.scales_mx4)
         self.y = None
         if combine and w.N > 0:
             X = expert_out if expert_out is not None else w.expert_out
@@ -71,9 +73,12 @@ class GpuRun:
             self.s8 = buf.scales_fp8.cpu().numpy()[:rows]
         if self.has_fp4:
             self.q4 = buf.out_fp4.cpu().numpy()[:rows]
+            self.qmx = buf.out_mx4.cpu().numpy()[:rows]
             if flags & B.MOE_FLAG_NVFP4_SWIZZLED_SCALES:
                 self.s4 = buf.scales_fp4.cpu().numpy().reshape(-1)   # atom layout, flat
+                self.smx = buf.scales_mx4.cpu().numpy().reshape(-1)
             else:
                 self.s4 = buf.scales_fp4.cpu().numpy()[:rows]
+                self.smx = buf.scales_mx4.cpu().numpy()[:rows]
         if combine and w.N > 0:
             self.y = bf16_np(self.y_dev)

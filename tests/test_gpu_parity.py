@@ -84,6 +84,9 @@ def assert_all_outputs(orc, w, run, ref, rows_sample=None, tokens_sample=None):
         q, s = orc.permute_nvfp4(w.hidden, row_src[idx], w.global_scale)
         assert np.array_equal(run.q4[idx], q), "nvfp4 codes"
         assert np.array_equal(run.s4[idx], s), "nvfp4 scales"
+        q, s = orc.permute_mxfp4(w.hidden, row_src[idx])
+        assert np.array_equal(run.qmx[idx], q), "mxfp4 codes"
+        assert np.array_equal(run.smx[idx], s), "mxfp4 scales"
     if run.y is not None:
         tok = np.arange(w.N) if tokens_sample is None else tokens_sample
         y = orc.combine(w.expert_out, w.gates[tok], ref.pair_slot[tok])
@@ -422,6 +425,9 @@ def test_nvfp4_swizzled_scales(orc, spec):
     q, s_lin = orc.permute_nvfp4(w.hidden, ref.row_src, w.global_scale)
     assert np.array_equal(run.q4, q)
     assert np.array_equal(run.s4, orc.swizzle_scales(s_lin))
+    q, s_lin = orc.permute_mxfp4(w.hidden, ref.row_src)
+    assert np.array_equal(run.qmx, q)
+    assert np.array_equal(run.smx, orc.swizzle_scales(s_lin))
 
 
 def test_nvfp4_swizzled_scales_workload(orc):
@@ -474,7 +480,8 @@ def test_backward_parity(orc, cfg, n):
 
 
 # ------------------------------------------------------------ SwiGLU + requant
-@pytest.mark.parametrize("fmt", [0, 1, 2], ids=["nvfp4", "mxfp8", "mxfp4"])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 3, 4, 5],
+                         ids=["nvfp4", "mxfp8", "mxfp4", "bf16", "mxfp6e2m3", "mxfp6e3m2"])
 @pytest.mark.parametrize("interleaved", [False, True], ids=["split", "interleaved"])
 @pytest.mark.parametrize("I", [2048, 96 * 32 + 32])
 def test_swiglu_quant_parity(orc, fmt, interleaved, I):
@@ -495,7 +502,8 @@ def test_swiglu_quant_parity(orc, fmt, interleaved, I):
     want_c, want_s = orc.swiglu_quant(gu, ref.row_src, fmt, interleaved=interleaved,
                                       global_scale=0.01)
     assert np.array_equal(codes.cpu().numpy(), want_c)
-    assert np.array_equal(scales.cpu().numpy(), want_s)
+    if fmt != B.MOE_QUANT_BF16:                # bf16 output has no scales
+        assert np.array_equal(scales.cpu().numpy(), want_s)
 
 
 def test_swiglu_exp_matches_oracle_bitwise(orc):
@@ -552,7 +560,7 @@ def test_swiglu_quant_wide_range(orc, gscale):
                   hidden=np.zeros((rows, 64), np.uint16), expert_out=None, global_scale=1.0,
                   seed=0)
     run = GpuRun(ww, quant=False, combine=False)
-    for fmt in (0, 1, 2):
+    for fmt in (0, 1, 2, 3, 4, 5):
         codes, scales = B.swiglu_buffers(rows, I, fmt)
         gs = torch.tensor([gscale], dtype=torch.float32, device="cuda")
         B.moe_swiglu_quant(run.prob, I, fmt, 0, to_dev_bf16(gu), run.buf.row_src, gs, codes,
@@ -560,5 +568,6 @@ def test_swiglu_quant_wide_range(orc, gscale):
         torch.cuda.synchronize()
         want_c, want_s = orc.swiglu_quant(gu, np.arange(rows, dtype=np.int32), fmt,
                                           global_scale=float(np.float32(gscale)))
-        assert np.array_equal(scales.cpu().numpy(), want_s), fmt
+        if fmt != B.MOE_QUANT_BF16:
+            assert np.array_equal(scales.cpu().numpy(), want_s), fmt
         assert np.array_equal(codes.cpu().numpy(), want_c), fmt
