@@ -348,6 +348,26 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
     ms = sum(step_ms) / len(step_ms)
     phase_ms = {p: sum(v) / len(v) for p, v in per.items()}
 
+    def time_phases(calls, n_steps):
+        """Average device time (us) of each call in `calls`, run in order as
+        one step; L2 flushed before every step, 3 untimed warm-up steps."""
+        for _ in range(3):
+            flush_l2()
+            for c in calls:
+                c()
+        evp = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+               for _ in range(n_steps)]
+        torch.cuda.synchronize(dev)
+        for i in range(n_steps):
+            flush_l2()
+            evp[i][0].record(stream)
+            for j, c in enumerate(calls):
+                c()
+                evp[i][j + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        return [1e3 * sum(e[j].elapsed_time(e[j + 1]) for e in evp) / n_steps
+                for j in range(len(calls))]
+
     # ---- grouped-GEMM-ready dispatch (NEXT row f1): experts padded to 128
     # rows, NVFP4 scales in the 128x4 atom layout; recv_capacity covers the
     # worst case N*k + E*127 and every one of its rows is written
@@ -359,30 +379,11 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
                            flags=B.MOE_FLAG_NVFP4_SWIZZLED_SCALES, expert_pad_multiple=pad)
         buf_p = B.Buffers(prob_p, device=dev)
         f1_steps = max(10, args.steps // 10)
-
-        def f1_step(ev=None):
-            if ev is not None:
-                ev[0].record(stream)
-            B.layout(prob_p, d_ids, buf_p)
-            if ev is not None:
-                ev[1].record(stream)
-            B.moe_permute_quant_nvfp4(prob_p, d_hidden, buf_p.row_src, buf_p.pair_slot, d_gs,
-                                      buf_p.out_fp4, buf_p.scales_fp4)
-            if ev is not None:
-                ev[2].record(stream)
-
-        for _ in range(3):
-            flush_l2()
-            f1_step()
-        f1_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
-                 for _ in range(f1_steps)]
-        torch.cuda.synchronize(dev)
-        for i in range(f1_steps):
-            flush_l2()
-            f1_step(f1_ev[i])
-        torch.cuda.synchronize(dev)
-        lay_us = 1e3 * sum(e[0].elapsed_time(e[1]) for e in f1_ev) / f1_steps
-        nv_us = 1e3 * sum(e[1].elapsed_time(e[2]) for e in f1_ev) / f1_steps
+        lay_us, nv_us = time_phases(
+            [lambda: B.layout(prob_p, d_ids, buf_p),
+             lambda: B.moe_permute_quant_nvfp4(prob_p, d_hidden, buf_p.row_src, buf_p.pair_slot,
+                                               d_gs, buf_p.out_fp4, buf_p.scales_fp4)],
+            f1_steps)
         rows_p = buf_p.rows
         nv_bytes = (2 * w.N * w.H + 4 * w.P + 4 * rows_p + rows_p * w.H // 2
                     + B.nvfp4_swizzled_scale_bytes(rows_p, w.H) + 4)
@@ -404,30 +405,11 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
         d_gx = torch.empty_like(d_x)
         d_gw = torch.empty_like(d_gates)
         f4_steps = max(10, args.steps // 10)
-
-        def f4_step(ev=None):
-            if ev is not None:
-                ev[0].record(stream)
-            B.moe_permute_backward(prob, d_grows, buf.pair_slot, d_gh)
-            if ev is not None:
-                ev[1].record(stream)
-            B.moe_combine_backward(prob, d_gtok, d_x, d_gates, buf.pair_slot, buf.row_src, d_gx,
-                                   d_gw)
-            if ev is not None:
-                ev[2].record(stream)
-
-        for _ in range(3):
-            flush_l2()
-            f4_step()
-        f4_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
-                 for _ in range(f4_steps)]
-        torch.cuda.synchronize(dev)
-        for i in range(f4_steps):
-            flush_l2()
-            f4_step(f4_ev[i])
-        torch.cuda.synchronize(dev)
-        pb_us = 1e3 * sum(e[0].elapsed_time(e[1]) for e in f4_ev) / f4_steps
-        cb_us = 1e3 * sum(e[1].elapsed_time(e[2]) for e in f4_ev) / f4_steps
+        pb_us, cb_us = time_phases(
+            [lambda: B.moe_permute_backward(prob, d_grows, buf.pair_slot, d_gh),
+             lambda: B.moe_combine_backward(prob, d_gtok, d_x, d_gates, buf.pair_slot,
+                                            buf.row_src, d_gx, d_gw)],
+            f4_steps)
         rows = buf.rows
         pb_bytes = 2 * total_rows * w.H + 4 * w.P + 2 * w.N * w.H
         cb_bytes = (2 * w.N * w.H + 2 * 2 * total_rows * w.H + 2 * (rows - total_rows) * w.H
@@ -440,37 +422,30 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
               "tokens_per_s": w.N / ((pb_us + cb_us) * 1e-6)}
         del d_gh, d_gx, d_gw
 
-    # ---- fused SwiGLU + requantisation (NEXT row f3): the synthetic expert
-    # outputs [C, H] read as gate|up rows of intermediate size I = H / 2
+    # ---- MX token format and fused SwiGLU + requantisation (NEXT row f3):
+    # the MXFP4 dispatch of the same tokens, and the synthetic expert outputs
+    # [C, H] read as gate|up rows of intermediate size I = H / 2
     f3 = None
     if args.next_rows:
+        n3 = max(10, args.steps // 20)
+        (mx_us,) = time_phases([lambda: B.moe_permute_quant_mxfp4(
+            prob, d_hidden, buf.row_src, buf.pair_slot, buf.out_mx4, buf.scales_mx4)], n3)
+        mx_bytes = (2 * w.N * w.H + 4 * w.P + 4 * buf.rows + buf.rows * w.H // 2
+                    + buf.rows * w.H // 32)
         I = w.H // 2
-        f3 = {"intermediate": I, "gate_up": "split", "rows": buf.rows}
+        f3 = {"permute_mxfp4_us": round(mx_us, 2),
+              "permute_mxfp4_gbs": round(mx_bytes / (mx_us * 1e-6) / 1e9, 1),
+              "swiglu": {"intermediate": I, "gate_up": "split", "rows": buf.rows}}
         for fmt, name in ((B.MOE_QUANT_MXFP8, "mxfp8"), (B.MOE_QUANT_NVFP4, "nvfp4"),
-                          (B.MOE_QUANT_MXFP4, "mxfp4")):
+                          (B.MOE_QUANT_MXFP4, "mxfp4"), (B.MOE_QUANT_MXFP6_E2M3, "mxfp6_e2m3"),
+                          (B.MOE_QUANT_BF16, "bf16")):
             codes, scales = B.swiglu_buffers(buf.rows, I, fmt, device=dev)
-            n_steps = max(10, args.steps // 20)
-
-            def f3_call():
-                B.moe_swiglu_quant(prob, I, fmt, B.MOE_GATE_UP_SPLIT, d_x, buf.row_src, d_gs,
-                                   codes, scales)
-
-            for _ in range(3):
-                flush_l2()
-                f3_call()
-            evp = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
-                   for _ in range(n_steps)]
-            torch.cuda.synchronize(dev)
-            for i in range(n_steps):
-                flush_l2()
-                evp[i][0].record(stream)
-                f3_call()
-                evp[i][1].record(stream)
-            torch.cuda.synchronize(dev)
-            us = 1e3 * sum(e[0].elapsed_time(e[1]) for e in evp) / n_steps
-            nbytes = (2 * 2 * I * total_rows + 4 * buf.rows + codes.numel() + scales.numel())
-            f3[name + "_us"] = round(us, 2)
-            f3[name + "_gbs"] = round(nbytes / (us * 1e-6) / 1e9, 1)
+            (us,) = time_phases([lambda: B.moe_swiglu_quant(
+                prob, I, fmt, B.MOE_GATE_UP_SPLIT, d_x, buf.row_src, d_gs, codes, scales)], n3)
+            nbytes = (2 * 2 * I * total_rows + 4 * buf.rows + codes.numel()
+                      + (scales.numel() if fmt != B.MOE_QUANT_BF16 else 0))
+            f3["swiglu"][name + "_us"] = round(us, 2)
+            f3["swiglu"][name + "_gbs"] = round(nbytes / (us * 1e-6) / 1e9, 1)
             del codes, scales
 
     # ---- end to end through the public API from pinned host memory
@@ -584,7 +559,7 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
                             "combined rows, status and counts; copies of neighbouring steps "
                             "overlap on separate streams"},
             "gpu_launches": launches_per_step * args.steps,
-            "next_rows": ({"f1_grouped_gemm_ready_nvfp4": f1, "f3_swiglu_requant": f3,
+            "next_rows": ({"f1_grouped_gemm_ready_nvfp4": f1, "f3_mx_and_swiglu_requant": f3,
                            "f4_backward": f4} if f1 or f3 or f4 else None),
             "clocks": clocks, "layout_status": st,
         }

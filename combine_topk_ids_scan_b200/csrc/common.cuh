@@ -109,6 +109,28 @@ __device__ __forceinline__ uint32_t mx_scale_code(float amax, int emax) {
   return (uint32_t)min(254, max(0, floor_log2(amax) - emax + 127));
 }
 
+// RN(a / d) of both halves from rd = RN(1/d), by two steps of Markstein's
+// correction q + (a - d q) * rd (P. Markstein, Computation of elementary
+// functions on the IBM RISC System/6000 processor, IBM J. Res. Dev. 34(1),
+// 1990: if rd is within half an ulp of 1/d and q within one ulp of a/d, the
+// corrected q rounds correctly).  q0 = RN(a rd) is within two ulps of a/d,
+// the first step brings it within one, the second rounds correctly.  The
+// caller guarantees d in [2^-90, 2^124] (kQuotientMinDivisor,
+// kQuotientMaxDivisor) and |a / d| <= 2^24.  Then every remainder is exact
+// (no underflow) for quotients >= 2^-13 and the result is RN(a / d); a
+// smaller quotient comes out below 2^-12 in magnitude with the sign of a,
+// which every 8- and 4-bit code here rounds to the same signed zero.  A zero
+// quotient takes the sign of a, as IEEE division does.
+constexpr float kQuotientMinDivisor = 0x1p-90f;
+constexpr float kQuotientMaxDivisor = 0x1p124f;
+__device__ __forceinline__ float2 rn_quotient2(float2 a, float d, float rd) {
+  const float2 nd = make_float2(-d, -d), r2 = make_float2(rd, rd);
+  float2 q = __fmul2_rn(a, r2);
+  q = __ffma2_rn(__ffma2_rn(nd, q, a), r2, q);
+  q = __ffma2_rn(__ffma2_rn(nd, q, a), r2, q);
+  return make_float2(copysignf(q.x, a.x), copysignf(q.y, a.y));
+}
+
 // One E4M3 code -> float (exact): through the f16x2 conversion.
 __device__ __forceinline__ float e4m3_to_float(uint32_t code) {
   uint32_t h2;

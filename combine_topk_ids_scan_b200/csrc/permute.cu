@@ -180,10 +180,19 @@ __global__ void __launch_bounds__(kThreads)
       float sc = 0.0f;
       if (amax > 0.0f) {
         sc = amax / 448.0f;  // IEEE round-to-nearest division
+        float2 qt[8];        // x / sc, |x / sc| <= 448
+        if (sc >= kQuotientMinDivisor && sc <= kQuotientMaxDivisor) {
+          const float rs = __frcp_rn(sc);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) qt[i] = rn_quotient2(make_float2(f[2 * i], f[2 * i + 1]), sc, rs);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) qt[i] = make_float2(f[2 * i] / sc, f[2 * i + 1] / sc);
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const uint32_t lo = cvt_e4m3x2(f[4 * i] / sc, f[4 * i + 1] / sc);
-          const uint32_t hi = cvt_e4m3x2(f[4 * i + 2] / sc, f[4 * i + 3] / sc);
+          const uint32_t lo = cvt_e4m3x2(qt[2 * i].x, qt[2 * i].y);
+          const uint32_t hi = cvt_e4m3x2(qt[2 * i + 1].x, qt[2 * i + 1].y);
           cw[i] = lo | (hi << 16);
         }
       }
@@ -223,14 +232,22 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float *f, float gs, uint32
   const float d = e4m3_to_float(sq) * gs;
   uint32_t c[2] = {0, 0};
   if (d > 0.0f) {
+    float2 qt[8];  // x / d
+    // |x / d| <= 12.01 unless the block scale saturated at 448 (0x7E): an
+    // unsaturated E4M3 scale is at least half of amax / 6
+    if (sq < 0x7Eu && d >= kQuotientMinDivisor && d <= kQuotientMaxDivisor) {
+      const float rd = __frcp_rn(d);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qt[i] = rn_quotient2(make_float2(f[2 * i], f[2 * i + 1]), d, rd);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qt[i] = make_float2(f[2 * i] / d, f[2 * i + 1] / d);
+    }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t word = 0;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int i = 8 * h + 2 * m;
-        word |= cvt_e2m1x2(f[i] / d, f[i + 1] / d) << (8 * m);
-      }
+      for (int m = 0; m < 4; ++m) word |= cvt_e2m1x2(qt[4 * h + m].x, qt[4 * h + m].y) << (8 * m);
       c[h] = word;
     }
   }

@@ -192,24 +192,6 @@ __device__ __forceinline__ uint32_t table_check(uint32_t w) {
 }
 constexpr uint32_t kTableCheckBits = 0xF000F000u;
 
-// RN(a / d) of both halves for the E2M1 code, from rd = RN(1/d), by two
-// steps of Markstein's correction q + (a - d q) * rd (P. Markstein,
-// Computation of elementary functions on the IBM RISC System/6000 processor,
-// IBM J. Res. Dev. 34(1), 1990: if rd is within half an ulp of 1/d and q
-// within one ulp of a/d, the corrected q rounds correctly).  q0 = RN(a rd) is
-// within two ulps, the first step brings it within one, the second rounds
-// correctly.  Preconditions, checked by the caller: d in [2^-100, 2^124],
-// which keeps the remainders exact for every quotient >= 2^-3 (a smaller one
-// encodes to +-0 whatever its last bits), and |a / d| <= 12.01, which keeps
-// them finite (a block scale that did not saturate is at least half of
-// amax / 6).  A zero quotient takes the sign of a, as IEEE division does.
-__device__ __forceinline__ float2 e2m1_quotient2(float2 a, float d, float rd) {
-  const float2 nd = splat(-d), r2 = splat(rd);
-  float2 q = __fmul2_rn(a, r2);
-  q = __ffma2_rn(__ffma2_rn(nd, q, a), r2, q);
-  q = __ffma2_rn(__ffma2_rn(nd, q, a), r2, q);
-  return make_float2(copysignf(q.x, a.x), copysignf(q.y, a.y));
-}
 
 
 // One lane's 32 columns [c, c + 32) of row r.
@@ -352,10 +334,12 @@ __device__ __forceinline__ void swiglu_group(const float *tab, const uint4 *__re
       sq2 |= sq << (8 * b);
       if (d > 0.0f) {
         float2 q[8];
-        if (sq < 0x7Eu && d >= 0x1p-100f && d <= 0x1p124f) {  // 0x7E: saturated at 448
+        // |y / d| <= 12.01 unless the block scale saturated at 448 (0x7E): an
+        // unsaturated E4M3 scale is at least half of amax / 6
+        if (sq < 0x7Eu && d >= kQuotientMinDivisor && d <= kQuotientMaxDivisor) {
           const float rd = __frcp_rn(d);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) q[j] = e2m1_quotient2(y[8 * b + j], d, rd);
+          for (int j = 0; j < 8; ++j) q[j] = rn_quotient2(y[8 * b + j], d, rd);
         } else {
 #pragma unroll
           for (int j = 0; j < 8; ++j)
