@@ -44,8 +44,8 @@ FALLBACK_HBM_GBS = 6650.0
 # metric workload (summaries under profiles/), keyed by kernel; valid only
 # while the kernel's source file is unchanged (sha256 prefix at capture time)
 NCU_TRAFFIC: dict[str, dict] = {
-    "permute_bf16": {"bytes_per_launch": 117994240 + 881679104, "src_sha": "5f3b2a0f2b412c22"},
-    "permute_fp8": {"bytes_per_launch": 118048768 + 426491648, "src_sha": "5f3b2a0f2b412c22"},
+    "permute_bf16": {"bytes_per_launch": 117978624 + 881097984, "src_sha": "5be478fbcd4e6021"},
+    "permute_fp8": {"bytes_per_launch": 118063104 + 426921984, "src_sha": "5be478fbcd4e6021"},
     "permute_nvfp4": {"bytes_per_launch": 117995520 + 205992960, "src_sha": "5f3b2a0f2b412c22"},
     "combine": {"bytes_per_launch": 940062720 + 67858688, "src_sha": "e2707ccbc781905c"},
 }

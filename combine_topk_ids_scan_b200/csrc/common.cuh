@@ -109,6 +109,41 @@ __device__ __forceinline__ uint32_t mx_scale_code(float amax, int emax) {
   return (uint32_t)min(254, max(0, floor_log2(amax) - emax + 127));
 }
 
+// max(a, |b|, |c|) in one three-input maximum
+__device__ __forceinline__ float max_abs3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+  return r;
+}
+
+// Eight floats -> eight E2M1 codes (nearest even, saturating to +-6), the
+// first in bits 0-3.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t3, %8, %7;\n\t"
+      "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+      : "=r"(r)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+  return r;
+}
+
+// Four floats -> four E4M3 codes (nearest even, saturating to +-448), the
+// first in bits 0-7.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float2 a, float2 b) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t0, t1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 t0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 t1, %4, %3;\n\t"
+      "mov.b32 %0, {t0, t1};\n\t}"
+      : "=r"(r)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
 // RN(a / d) of both halves from rd = RN(1/d), by two steps of Markstein's
 // correction q + (a - d q) * rd (P. Markstein, Computation of elementary
 // functions on the IBM RISC System/6000 processor, IBM J. Res. Dev. 34(1),

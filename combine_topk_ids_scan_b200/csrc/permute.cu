@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kThreads)
       }
       float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      for (int i = 0; i < 8; ++i) amax = max_abs3(amax, f[2 * i], f[2 * i + 1]);
       amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
       amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
@@ -190,11 +190,7 @@ __global__ void __launch_bounds__(kThreads)
           for (int i = 0; i < 8; ++i) qt[i] = make_float2(f[2 * i] / sc, f[2 * i + 1] / sc);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t lo = cvt_e4m3x2(qt[2 * i].x, qt[2 * i].y);
-          const uint32_t hi = cvt_e4m3x2(qt[2 * i + 1].x, qt[2 * i + 1].y);
-          cw[i] = lo | (hi << 16);
-        }
+        for (int i = 0; i < 4; ++i) cw[i] = cvt_e4m3x4(qt[2 * i], qt[2 * i + 1]);
       }
       codes[u] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
       scale[u] = sc;
@@ -226,7 +222,7 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float *f, float gs, uint32
                                                 uint32_t &codes_hi) {
   float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  for (int i = 0; i < 8; ++i) amax = max_abs3(amax, f[2 * i], f[2 * i + 1]);
   const float sf = (amax / 6.0f) / gs;
   const uint32_t sq = cvt_e4m3x2(sf, 0.0f) & 0xFFu;
   const float d = e4m3_to_float(sq) * gs;
@@ -243,13 +239,8 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float *f, float gs, uint32
 #pragma unroll
       for (int i = 0; i < 8; ++i) qt[i] = make_float2(f[2 * i] / d, f[2 * i + 1] / d);
     }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int m = 0; m < 4; ++m) word |= cvt_e2m1x2(qt[4 * h + m].x, qt[4 * h + m].y) << (8 * m);
-      c[h] = word;
-    }
+    c[0] = cvt_e2m1x8(qt[0], qt[1], qt[2], qt[3]);
+    c[1] = cvt_e2m1x8(qt[4], qt[5], qt[6], qt[7]);
   }
   codes_lo = c[0];
   codes_hi = c[1];
@@ -261,22 +252,17 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float *f, float gs, uint32
 __device__ __forceinline__ uint32_t mxfp4_block(const float *f, uint4 &codes) {
   float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  for (int i = 0; i < 16; ++i) amax = max_abs3(amax, f[2 * i], f[2 * i + 1]);
   uint32_t c[4] = {0, 0, 0, 0};
   uint32_t sc = 0;
   if (amax > 0.0f) {
     sc = mx_scale_code(amax, 2);
     const float m = pow2i(127 - (int)sc);  // 2^-X, a normal float
+    float2 v[16];
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      uint32_t word = 0;
+    for (int i = 0; i < 16; ++i) v[i] = __fmul2_rn(make_float2(f[2 * i], f[2 * i + 1]), make_float2(m, m));
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int i = 8 * h + 2 * j;
-        word |= cvt_e2m1x2(__fmul_rn(f[i], m), __fmul_rn(f[i + 1], m)) << (8 * j);
-      }
-      c[h] = word;
-    }
+    for (int h = 0; h < 4; ++h) c[h] = cvt_e2m1x8(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
   }
   codes = make_uint4(c[0], c[1], c[2], c[3]);
   return sc;

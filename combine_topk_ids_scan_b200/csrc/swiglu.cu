@@ -119,41 +119,6 @@ __device__ __forceinline__ float table_at(const float *tab, uint32_t off) {
   return *reinterpret_cast<const float *>(reinterpret_cast<const char *>(tab) + off);
 }
 
-// max(a, |b|, |c|) in one three-input maximum
-__device__ __forceinline__ float max_abs3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
-  return r;
-}
-
-// Eight floats -> eight E2M1 codes (nearest even, saturating to +-6), the
-// first in bits 0-3.
-__device__ __forceinline__ uint32_t cvt_e2m1x8(float2 a, float2 b, float2 c, float2 d) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t3, %8, %7;\n\t"
-      "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
-      : "=r"(r)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
-  return r;
-}
-
-// Four floats -> four E4M3 codes (nearest even, saturating to +-448), the
-// first in bits 0-7.
-__device__ __forceinline__ uint32_t cvt_e4m3x4(float2 a, float2 b) {
-  uint32_t r;
-  asm("{\n\t.reg .b16 t0, t1;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 t0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 t1, %4, %3;\n\t"
-      "mov.b32 %0, {t0, t1};\n\t}"
-      : "=r"(r)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return r;
-}
-
 // Eight floats -> eight OCP MX FP6 codes (E2M3 or E3M2, nearest even,
 // saturating), packed at bits [6i, 6i + 6) of a 48-bit little-endian value
 // returned as (low 32 bits, high 16 bits).  The conversion leaves each 6-bit
