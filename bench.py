@@ -46,8 +46,8 @@ FALLBACK_HBM_GBS = 6650.0
 NCU_TRAFFIC: dict[str, dict] = {
     "permute_bf16": {"bytes_per_launch": 117978624 + 881097984, "src_sha": "5be478fbcd4e6021"},
     "permute_fp8": {"bytes_per_launch": 118063104 + 426921984, "src_sha": "5be478fbcd4e6021"},
-    "permute_nvfp4": {"bytes_per_launch": 117995520 + 205992960, "src_sha": "5f3b2a0f2b412c22"},
-    "combine": {"bytes_per_launch": 940062720 + 67858688, "src_sha": "e2707ccbc781905c"},
+    "permute_nvfp4": {"bytes_per_launch": 118008832 + 207333888, "src_sha": "5be478fbcd4e6021"},
+    "combine": {"bytes_per_launch": 940089088 + 69039616, "src_sha": "3409373de95ae4e3"},
 }
 
 
