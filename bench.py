@@ -287,26 +287,27 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
         flush_w.zero_()
         flush_r.max()
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+    def step(ev=None, phase_events=False):
+        """One step; ev[0] / ev[5] bracket it, ev[1..4] (only with
+        phase_events) separate its kernels.  An event between two kernels
+        ends the programmatic overlap of the second with the first, so the
+        timed steps record only the bracketing pair."""
+        def mark(i):
+            if ev is not None and (phase_events or i in (0, 5)):
+                ev[i].record(stream)
+        mark(0)
         B.layout(prob, d_ids, buf)
-        if ev is not None:
-            ev[1].record(stream)
+        mark(1)
         B.moe_permute(prob, d_hidden, buf.row_src, buf.pair_slot, buf.out)
-        if ev is not None:
-            ev[2].record(stream)
+        mark(2)
         B.moe_permute_quant_fp8(prob, d_hidden, buf.row_src, buf.pair_slot, buf.out_fp8,
                                 buf.scales_fp8)
-        if ev is not None:
-            ev[3].record(stream)
+        mark(3)
         B.moe_permute_quant_nvfp4(prob, d_hidden, buf.row_src, buf.pair_slot, d_gs,
                                   buf.out_fp4, buf.scales_fp4)
-        if ev is not None:
-            ev[4].record(stream)
+        mark(4)
         B.moe_combine(prob, d_x, d_gates, buf.pair_slot, d_y)
-        if ev is not None:
-            ev[5].record(stream)
+        mark(5)
 
     # the layout is one cooperative launch up to 128 scan tiles of 4096 pairs,
     # else a scan and an emit launch; then three permutes and the combine
@@ -338,15 +339,24 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
     torch.cuda.synchronize(dev)
     barrier()
     clocks = sampler.stop() if sampler else None
+    step_ms = [e[0].elapsed_time(e[5]) for e in evs]
+    ms = sum(step_ms) / len(step_ms)
+
+    # ---- per-kernel breakdown: further steps with an event between kernels
     phases = ["layout", "permute_bf16", "permute_fp8", "permute_nvfp4", "combine"]
+    n_phase = max(10, min(args.steps, 300))
+    pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_phase)]
+    torch.cuda.synchronize(dev)
+    for i in range(n_phase):
+        flush_l2()
+        step(pevs[i], phase_events=True)
+    torch.cuda.synchronize(dev)
     per = {p: [] for p in phases}
-    step_ms = []
-    for e in evs:
+    for e in pevs:
         for i, p in enumerate(phases):
             per[p].append(e[i].elapsed_time(e[i + 1]))
-        step_ms.append(e[0].elapsed_time(e[5]))
-    ms = sum(step_ms) / len(step_ms)
     phase_ms = {p: sum(v) / len(v) for p, v in per.items()}
+    phase_step_ms = sum(e[0].elapsed_time(e[5]) for e in pevs) / n_phase
 
     def time_phases(calls, n_steps):
         """Average device time (us) of each call in `calls`, run in order as
@@ -542,6 +552,9 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
             "hbm_gbs": step_bytes / (ms * 1e-3) / 1e9,
             "hbm_frac_of_peak": step_bytes / (ms * 1e-3) / 1e9 / peak,
             "phases_us": {p: round(1e3 * v, 2) for p, v in phase_ms.items()},
+            "phases_timing": (f"{n_phase} further steps with an event between kernels (an event "
+                              f"ends the programmatic overlap of consecutive kernels); their "
+                              f"mean step {phase_step_ms:.4f} ms"),
             "phases_gbs": {p: round(nbytes[p] / (phase_ms[p] * 1e-3) / 1e9, 1)
                            for p in phases},
             "dispatch_bf16_plus_combine_tokens_per_s":

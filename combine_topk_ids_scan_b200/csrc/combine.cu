@@ -30,6 +30,8 @@ __global__ void __launch_bounds__(kThreads)
     combine_kernel(const uint4 *__restrict__ x, const float *__restrict__ gates,
                    const int32_t *__restrict__ pair_slot, uint4 *__restrict__ out, int32_t N,
                    int32_t k, int64_t rows, int32_t vecs) {
+  allow_dependents();
+  grid_dependency_wait();
   const int lane = threadIdx.x % kWarp;
   const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t nw = ((int64_t)gridDim.x * kThreads) / kWarp;
@@ -105,6 +107,8 @@ __global__ void __launch_bounds__(kThreads)
                             const int32_t *__restrict__ row_src, uint4 *__restrict__ grad_x,
                             float *__restrict__ grad_gates, int32_t N, int32_t k, int64_t rows,
                             int32_t vecs) {
+  allow_dependents();
+  grid_dependency_wait();
   const int lane = threadIdx.x % kWarp;
   const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t nw = ((int64_t)gridDim.x * kThreads) / kWarp;
@@ -180,15 +184,40 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// Grid of a persistent kernel: resident CTAs per SM (queried once per
+// kernel and device into `cache`, which the caller keeps per kernel) x SMs,
+// or fewer when there is less work.
 template <typename Kernel>
-int grid_for(Kernel kernel, int64_t N) {
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) !=
-          cudaSuccess ||
-      per_sm < 1)
+int grid_for(Kernel kernel, int64_t N, int (&cache)[8]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  int &per_sm = cache[dev & 7];
+  if (per_sm == 0 &&
+      (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) !=
+           cudaSuccess ||
+       per_sm < 1))
     per_sm = 1;
   const int64_t need = std::max<int64_t>(1, (N + kThreads / kWarp - 1) / (kThreads / kWarp));
   return (int)std::min<int64_t>(need, (int64_t)per_sm * device_sm_count());
+}
+
+template <int KMAX>
+cudaError_t launch_backward(const Shape &s, const uint4 *gy, const uint4 *x, const float *gates,
+                            const int32_t *pair_slot, const int32_t *row_src, uint4 *gx,
+                            float *grad_gates, int64_t work, cudaStream_t stream) {
+  static int cache[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  auto kernel = combine_backward_kernel<KMAX>;
+  return launch_pdl(kernel, dim3(grid_for(kernel, work, cache)), dim3(kThreads), 0, stream, gy, x,
+                    gates, pair_slot, row_src, gx, grad_gates, s.N, s.k, s.rows, s.H / 8);
+}
+
+template <int KMAX, int U>
+cudaError_t launch_forward(const Shape &s, const uint4 *x, const float *gates,
+                           const int32_t *pair_slot, uint4 *o, cudaStream_t stream) {
+  static int cache[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  auto kernel = combine_kernel<KMAX, U>;
+  return launch_pdl(kernel, dim3(grid_for(kernel, s.N, cache)), dim3(kThreads), 0, stream, x, gates,
+                    pair_slot, o, s.N, s.k, s.rows, s.H / 8);
 }
 
 }  // namespace
@@ -200,23 +229,13 @@ cudaError_t launch_combine_backward(const Shape &s, const void *grad_y, const vo
   const uint4 *gy = static_cast<const uint4 *>(grad_y);
   const uint4 *x = static_cast<const uint4 *>(expert_out);
   uint4 *gx = static_cast<uint4 *>(grad_expert_out);
-  const int32_t vecs = s.H / 8;
   const int64_t work = std::max<int64_t>((int64_t)s.N, (s.rows + kWarp - 1) / kWarp);
   if (work == 0) return cudaSuccess;
-  if (s.k <= 4) {
-    auto kernel = combine_backward_kernel<4>;
-    kernel<<<grid_for(kernel, work), kThreads, 0, stream>>>(gy, x, gates, pair_slot, row_src, gx,
-                                                            grad_gates, s.N, s.k, s.rows, vecs);
-  } else if (s.k <= 8) {
-    auto kernel = combine_backward_kernel<8>;
-    kernel<<<grid_for(kernel, work), kThreads, 0, stream>>>(gy, x, gates, pair_slot, row_src, gx,
-                                                            grad_gates, s.N, s.k, s.rows, vecs);
-  } else {
-    auto kernel = combine_backward_kernel<16>;
-    kernel<<<grid_for(kernel, work), kThreads, 0, stream>>>(gy, x, gates, pair_slot, row_src, gx,
-                                                            grad_gates, s.N, s.k, s.rows, vecs);
-  }
-  return cudaGetLastError();
+  if (s.k <= 4)
+    return launch_backward<4>(s, gy, x, gates, pair_slot, row_src, gx, grad_gates, work, stream);
+  if (s.k <= 8)
+    return launch_backward<8>(s, gy, x, gates, pair_slot, row_src, gx, grad_gates, work, stream);
+  return launch_backward<16>(s, gy, x, gates, pair_slot, row_src, gx, grad_gates, work, stream);
 }
 
 cudaError_t launch_combine(const Shape &s, const void *expert_out, const float *gates,
@@ -224,25 +243,10 @@ cudaError_t launch_combine(const Shape &s, const void *expert_out, const float *
   if (s.N == 0) return cudaSuccess;
   const uint4 *x = static_cast<const uint4 *>(expert_out);
   uint4 *o = static_cast<uint4 *>(out);
-  const int32_t vecs = s.H / 8;
-  if (s.k <= 2) {
-    auto kernel = combine_kernel<2, 4>;
-    kernel<<<grid_for(kernel, s.N), kThreads, 0, stream>>>(x, gates, pair_slot, o, s.N, s.k,
-                                                            s.rows, vecs);
-  } else if (s.k <= 4) {
-    auto kernel = combine_kernel<4, 2>;
-    kernel<<<grid_for(kernel, s.N), kThreads, 0, stream>>>(x, gates, pair_slot, o, s.N, s.k,
-                                                            s.rows, vecs);
-  } else if (s.k <= 8) {
-    auto kernel = combine_kernel<8, 2>;
-    kernel<<<grid_for(kernel, s.N), kThreads, 0, stream>>>(x, gates, pair_slot, o, s.N, s.k,
-                                                            s.rows, vecs);
-  } else {
-    auto kernel = combine_kernel<16, 1>;
-    kernel<<<grid_for(kernel, s.N), kThreads, 0, stream>>>(x, gates, pair_slot, o, s.N, s.k,
-                                                            s.rows, vecs);
-  }
-  return cudaGetLastError();
+  if (s.k <= 2) return launch_forward<2, 4>(s, x, gates, pair_slot, o, stream);
+  if (s.k <= 4) return launch_forward<4, 2>(s, x, gates, pair_slot, o, stream);
+  if (s.k <= 8) return launch_forward<8, 2>(s, x, gates, pair_slot, o, stream);
+  return launch_forward<16, 1>(s, x, gates, pair_slot, o, stream);
 }
 
 }  // namespace moe

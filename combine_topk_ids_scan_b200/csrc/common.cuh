@@ -10,6 +10,22 @@ namespace moe {
 
 constexpr int kWarp = 32;
 
+// Programmatic dependent launch (sm_90 and later).  The library's kernels
+// after the first of a step are launched with programmatic stream
+// serialisation allowed (launch_pdl in internal.h), so their CTAs may be
+// scheduled while the previous kernel on the stream drains its last wave.
+// Each kernel executes grid_dependency_wait() before its first global
+// memory access: it returns once the previous kernel has completed and its
+// writes are visible, so stream order is kept for every load and store.
+// allow_dependents() lets the next kernel be scheduled once every CTA of
+// this one has started.  Both are no-ops for a kernel launched normally.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- memory
 // Streaming 16-byte load that bypasses L1 (data is read once).
 __device__ __forceinline__ uint4 ld_stream_v4(const uint4 *p) {

@@ -498,6 +498,7 @@ __device__ void emit_step(const LayoutArgs &a, int64_t gtid, int64_t gstride,
 
 // One cooperative launch: scan (first T CTAs), grid-wide wait, emit (all).
 __global__ void __launch_bounds__(kScanThreads, 1) layout_fused_kernel(LayoutArgs a) {
+  allow_dependents();  // the next kernel may be scheduled; it waits for this grid
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ uint32_t s_status;
   if (threadIdx.x == 0) s_status = 0;
@@ -523,6 +524,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) layout_fused_kernel(LayoutArg
 }
 
 __global__ void __launch_bounds__(kScanThreads, 1) layout_count_scan_kernel(LayoutArgs a) {
+  allow_dependents();
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ uint32_t s_status;
   scan_step<false>(a, smem, &s_status);
@@ -531,6 +533,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) layout_count_scan_kernel(Layo
 }
 
 __global__ void __launch_bounds__(kEmitThreads) layout_emit_kernel(LayoutArgs a) {
+  allow_dependents();
+  grid_dependency_wait();
   __shared__ uint32_t s_status;
   if (threadIdx.x == 0) s_status = 0;
   const int64_t gtid = (int64_t)blockIdx.x * kEmitThreads + threadIdx.x;
@@ -647,8 +651,7 @@ cudaError_t launch_layout(const Shape &s, const int32_t *ids, int32_t *expert_co
   const int64_t max_blocks = (int64_t)device_sm_count() * 8;
   const int blocks = (int)std::max<int64_t>(
       1, std::min<int64_t>(max_blocks, (work + kEmitThreads - 1) / kEmitThreads));
-  layout_emit_kernel<<<blocks, kEmitThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(layout_emit_kernel, dim3(blocks), dim3(kEmitThreads), 0, stream, a);
 }
 
 }  // namespace moe

@@ -80,6 +80,8 @@ __global__ void __launch_bounds__(kThreads)
     permute_bf16_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                         const int32_t *__restrict__ pair_slot, uint4 *__restrict__ out,
                         int32_t N, int32_t k, int64_t rows, int32_t vecs, int32_t chunks) {
+  allow_dependents();
+  grid_dependency_wait();
   constexpr int U = kBf16Chunk / 8 / kWarp;  // 2
   const int lane = threadIdx.x % kWarp;
   const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
@@ -127,6 +129,8 @@ __global__ void __launch_bounds__(kThreads)
                        const int32_t *__restrict__ pair_slot, uint8_t *__restrict__ q,
                        float *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
                        int32_t H, int32_t chunks) {
+  allow_dependents();
+  grid_dependency_wait();
   constexpr int U = kChunk / 512;  // 2
   const int lane = threadIdx.x % kWarp;
   const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
@@ -284,6 +288,8 @@ __global__ void __launch_bounds__(kThreads)
                        const float *__restrict__ global_scale, uint8_t *__restrict__ q,
                        uint8_t *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
                        int32_t H, int32_t chunks, bool swizzled) {
+  allow_dependents();
+  grid_dependency_wait();
   const int lane = threadIdx.x % kWarp;
   const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
@@ -406,10 +412,9 @@ cudaError_t launch_permute_bf16(const Shape &s, const void *hidden, const int32_
                                 const int32_t *pair_slot, void *out, cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
   const int32_t chunks = chunks_of(s.H, kBf16Chunk);
-  permute_bf16_kernel<<<(unsigned)unit_blocks(s, chunks, s.rows), kThreads, 0, stream>>>(
-      static_cast<const uint4 *>(hidden), row_src, pair_slot, static_cast<uint4 *>(out), s.N,
-      s.k, s.rows, s.H / 8, chunks);
-  return cudaGetLastError();
+  return launch_pdl(permute_bf16_kernel, dim3((unsigned)unit_blocks(s, chunks, s.rows)),
+                    dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src,
+                    pair_slot, static_cast<uint4 *>(out), s.N, s.k, s.rows, s.H / 8, chunks);
 }
 
 cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t *row_src,
@@ -417,10 +422,9 @@ cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t
                                cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
   const int32_t chunks = chunks_of(s.H, kChunk);
-  permute_fp8_kernel<<<(unsigned)unit_blocks(s, chunks, s.rows), kThreads, 0, stream>>>(
-      static_cast<const uint4 *>(hidden), row_src, pair_slot, q, scales, s.N, s.k, s.rows, s.H,
-      chunks);
-  return cudaGetLastError();
+  return launch_pdl(permute_fp8_kernel, dim3((unsigned)unit_blocks(s, chunks, s.rows)),
+                    dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src,
+                    pair_slot, q, scales, s.N, s.k, s.rows, s.H, chunks);
 }
 
 cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32_t *row_src,
@@ -430,11 +434,9 @@ cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32
   const int32_t chunks = chunks_of(s.H, kChunk);
   const bool swizzled = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) != 0;
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
-  permute_fp4_kernel<false>
-      <<<(unsigned)unit_blocks(s, chunks, check_rows), kThreads, 0, stream>>>(
-          static_cast<const uint4 *>(hidden), row_src, pair_slot, global_scale, q, scales, s.N,
-          s.k, s.rows, s.H, chunks, swizzled);
-  return cudaGetLastError();
+  return launch_pdl(permute_fp4_kernel<false>, dim3((unsigned)unit_blocks(s, chunks, check_rows)),
+                    dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src,
+                    pair_slot, global_scale, q, scales, s.N, s.k, s.rows, s.H, chunks, swizzled);
 }
 
 cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32_t *row_src,
@@ -444,11 +446,10 @@ cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32
   const int32_t chunks = chunks_of(s.H, kChunk);
   const bool swizzled = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) != 0;
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
-  permute_fp4_kernel<true>
-      <<<(unsigned)unit_blocks(s, chunks, check_rows), kThreads, 0, stream>>>(
-          static_cast<const uint4 *>(hidden), row_src, pair_slot, nullptr, q, scales, s.N, s.k,
-          s.rows, s.H, chunks, swizzled);
-  return cudaGetLastError();
+  return launch_pdl(permute_fp4_kernel<true>, dim3((unsigned)unit_blocks(s, chunks, check_rows)),
+                    dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src,
+                    pair_slot, static_cast<const float *>(nullptr), q, scales, s.N, s.k, s.rows,
+                    s.H, chunks, swizzled);
 }
 
 }  // namespace moe

@@ -356,13 +356,17 @@ __global__ void __launch_bounds__(kThreads, 3)
                         const float *__restrict__ global_scale, uint8_t *__restrict__ codes,
                         uint8_t *__restrict__ scales, int64_t groups, int32_t I, int32_t G,
                         int64_t step_rows, int32_t step_cols) {
+  allow_dependents();
   __shared__ float tab[kTabSize];
+  // the table needs no global memory: it is built while the previous kernel
+  // on the stream may still be running
   for (int i = 2 * threadIdx.x; i < kTabSize; i += 2 * kThreads) {
     const float2 v = silu2(make_float2(tab_gate(i), tab_gate(i + 1)));
     tab[i] = v.x;
     tab[i + 1] = v.y;
   }
   __syncthreads();
+  grid_dependency_wait();
 
   const float gs = FORMAT == 0 ? __ldg(global_scale) : 0.0f;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
@@ -401,9 +405,8 @@ cudaError_t launch(const uint4 *in, const int32_t *row_src, const float *gs, uin
   const int64_t blocks = std::max<int64_t>(
       1, std::min<int64_t>(want, (int64_t)cap * device_sm_count()));
   const int64_t stride = blocks * kThreads;
-  kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(in, row_src, gs, codes, scales, groups, I, G,
-                                                    stride / G, (int32_t)(stride % G));
-  return cudaGetLastError();
+  return launch_pdl(kernel, dim3((unsigned)blocks), dim3(kThreads), 0, stream, in, row_src, gs,
+                    codes, scales, groups, I, G, stride / G, (int32_t)(stride % G));
 }
 
 }  // namespace
