@@ -27,6 +27,19 @@ __device__ __forceinline__ void allow_dependents() {
 }
 
 // ---------------------------------------------------------------- memory
+// 4-byte store whose L2 line is kept in preference to others (evict_last):
+// the block-scale atom layout scatters 4-byte groups of different tokens
+// into the same 32-byte sectors, and keeping those lines resident until
+// they are complete saves partial-sector write-backs (measured on B200,
+// NVFP4 dispatch with 128-padded experts: 158 -> 129 us).
+__device__ __forceinline__ void st_u32_evict_last(void *p, uint32_t v) {
+  asm volatile(
+      "{\n\t.reg .b64 pol;\n\tcreatepolicy.fractional.L2::evict_last.b64 pol, 1.0;\n\t"
+      "st.global.L2::cache_hint.b32 [%0], %1, pol;\n\t}" ::"l"(p),
+      "r"(v)
+      : "memory");
+}
+
 // Streaming 16-byte load that bypasses L1 (data is read once).
 __device__ __forceinline__ uint4 ld_stream_v4(const uint4 *p) {
   uint4 v;

@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kThreads)
           for (int v = lane; v < qrow / 16; v += kWarp) st_v4(dst + v, zero);
         }
         for (int gg = lane; gg < groups; gg += kWarp)
-          *reinterpret_cast<uint32_t *>(scales + sf_atom_offset(row, 4 * gg, groups)) = 0u;
+          st_u32_evict_last(scales + sf_atom_offset(row, 4 * gg, groups), 0u);
       }
     }
     return;
@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(kThreads)
           if (MX) scales[s * srow + sc_col] = (uint8_t)sq;
           else *reinterpret_cast<uint16_t *>(scales + s * srow + sc_col) = (uint16_t)sq;
         } else if ((lane & (MX ? 3 : 1)) == 0) {
-          *reinterpret_cast<uint32_t *>(scales + sf_atom_offset(s, sc_col, groups)) = quad;
+          st_u32_evict_last(scales + sf_atom_offset(s, sc_col, groups), quad);
         }
       }
     }
