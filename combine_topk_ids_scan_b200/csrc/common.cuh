@@ -109,16 +109,6 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
-// Two floats -> two E2M1 codes (nearest even, saturating to +-6); `lo` in
-// bits 0-3, `hi` in bits 4-7.
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
-      : "=r"(r)
-      : "f"(hi), "f"(lo));
-  return r;
-}
-
 // floor(log2(a)) of a finite a > 0, subnormals included.
 __device__ __forceinline__ int floor_log2(float a) {
   const uint32_t b = __float_as_uint(a);
