@@ -281,13 +281,18 @@ __device__ __forceinline__ int64_t sf_atom_offset(int64_t m, int32_t c, int32_t 
 
 // MX == false: NVFP4 (two 16-element blocks per lane, E4M3 scales);
 // MX == true: MXFP4 (one 32-element block per lane, E8M0 scales).
-template <bool MX>
-__global__ void __launch_bounds__(kThreads)
+// SWIZZLED: scales in the block-scale atom layout.  The linear-scale kernels
+// are held to 5 resident CTAs per SM (48 registers; measured on B200 at the
+// metric shape: NVFP4 74 -> 70 us, MXFP4 61.4 -> 60.0 us), the atom-layout
+// kernels to 4 (with 5 they were slower).
+template <bool MX, bool SWIZZLED>
+__global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
     permute_fp4_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                        const int32_t *__restrict__ pair_slot,
                        const float *__restrict__ global_scale, uint8_t *__restrict__ q,
                        uint8_t *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
-                       int32_t H, int32_t chunks, bool swizzled) {
+                       int32_t H, int32_t chunks) {
+  constexpr bool swizzled = SWIZZLED;
   allow_dependents();
   grid_dependency_wait();
   const int lane = threadIdx.x % kWarp;
@@ -434,9 +439,10 @@ cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32
   const int32_t chunks = chunks_of(s.H, kChunk);
   const bool swizzled = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) != 0;
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
-  return launch_pdl(permute_fp4_kernel<false>, dim3((unsigned)unit_blocks(s, chunks, check_rows)),
-                    dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src,
-                    pair_slot, global_scale, q, scales, s.N, s.k, s.rows, s.H, chunks, swizzled);
+  return launch_pdl(swizzled ? permute_fp4_kernel<false, true> : permute_fp4_kernel<false, false>,
+                    dim3((unsigned)unit_blocks(s, chunks, check_rows)), dim3(kThreads), 0, stream,
+                    static_cast<const uint4 *>(hidden), row_src, pair_slot, global_scale, q,
+                    scales, s.N, s.k, s.rows, s.H, chunks);
 }
 
 cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32_t *row_src,
@@ -446,10 +452,11 @@ cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32
   const int32_t chunks = chunks_of(s.H, kChunk);
   const bool swizzled = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) != 0;
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
-  return launch_pdl(permute_fp4_kernel<true>, dim3((unsigned)unit_blocks(s, chunks, check_rows)),
-                    dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src,
-                    pair_slot, static_cast<const float *>(nullptr), q, scales, s.N, s.k, s.rows,
-                    s.H, chunks, swizzled);
+  return launch_pdl(swizzled ? permute_fp4_kernel<true, true> : permute_fp4_kernel<true, false>,
+                    dim3((unsigned)unit_blocks(s, chunks, check_rows)), dim3(kThreads), 0, stream,
+                    static_cast<const uint4 *>(hidden), row_src, pair_slot,
+                    static_cast<const float *>(nullptr), q, scales, s.N, s.k, s.rows, s.H,
+                    chunks);
 }
 
 }  // namespace moe
