@@ -1,13 +1,15 @@
 // swiglu.cu -- fused SwiGLU + requantisation of the experts' gate/up rows
 // (Mojo MAX ep_comm: fused_silu_kernel, fused_silu_mx_kernel,
-// fused_silu_nvfp4_kernel, fused_silu_mxfp8_interleaved_kernel; MXTokenFormat).
+// fused_silu_nvfp4_kernel, fused_silu_nvfp4_interleaved_kernel,
+// fused_silu_mxfp8_interleaved_kernel, fused_silu_mxfp6_kernel).
 //
 // For every dispatch row r with a routed token (row_src[r] >= 0 -- the
 // layout's answer to how many rows were received, read on the device),
-// y = silu(gate) * up in fp32 and y is quantised to NVFP4 (E2M1 + E4M3 per 16
-// + global scale, as the dispatch does), MXFP8 (E4M3 + E8M0 per 32) or MXFP4
-// (E2M1 + E8M0 per 32).  Rows without a token are zero bytes and their input
-// is not read.
+// y = silu(gate) * up in fp32 and y is written as bf16 or quantised to NVFP4
+// (E2M1 + E4M3 per 16 + global scale, as the dispatch does), MXFP8 (E4M3 +
+// E8M0 per 32), MXFP4 (E2M1 + E8M0 per 32) or MXFP6 (E2M3 or E3M2 + E8M0 per
+// 32, 6-bit codes packed four to three bytes).  Rows without a token are
+// zero bytes and their input is not read.
 //
 // e^x is one fixed fp32 operation sequence (Cody-Waite range reduction, the
 // degree-7 Taylor polynomial in Horner form with fused multiply-adds, scaling
