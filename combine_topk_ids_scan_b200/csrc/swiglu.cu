@@ -349,6 +349,152 @@ __device__ __forceinline__ void swiglu_group(const float *tab, const uint4 *__re
   }
 }
 
+// ---- split layout: coalesced warp units
+// A warp takes a unit of 512 columns of one row; lane l holds the 8 columns
+// [c0 + 256 s + 8 l, +8) for s = 0, 1, so every 16-byte load and every code
+// store of the warp covers one contiguous run (measured on B200: the
+// lane-contiguous groups above, 64 bytes apart per lane, kept the L1TEX data
+// path at 91% of its peak).  A 32-column MX block spans 4 lanes: its
+// maximum is a two-step xor-shuffle reduction.  Used for MXFP8, MXFP4 and
+// bf16 (measured on B200, rows = 65,536, I = 3584, N(0,1) inputs: 238 -> 231,
+// 217 -> 209, 298 -> 209 us); for NVFP4 and MXFP6 the per-block scale work,
+// repeated by every lane of a block, made it slower than the lane-contiguous
+// kernel, which they keep.
+constexpr int kUnitCols = 512;
+
+template <int FORMAT>
+__device__ __forceinline__ void swiglu_unit_split(const float *tab, const uint4 *__restrict__ gate_up,
+                                                  bool live, uint8_t *__restrict__ codes,
+                                                  uint8_t *__restrict__ scales, int64_t r,
+                                                  int32_t c0, int32_t I, int lane) {
+  static_assert(FORMAT == 1 || FORMAT == 2 || FORMAT == 3, "MXFP8, MXFP4 or bf16");
+  constexpr uint32_t kFull = 0xFFFFFFFFu;
+  // code bytes per 8 columns
+  constexpr int kCode8 = FORMAT == 1 ? 8 : FORMAT == 3 ? 16 : 4;
+  const int64_t code_row = (int64_t)I / 8 * kCode8;
+  const int64_t scale_row = I / 32;
+  const uint4 *in = gate_up + r * ((int64_t)I / 4);  // 2I bf16 = I/4 vectors of 8
+
+  int c[2];
+  bool act[2];
+  uint4 gv[2], uv[2];
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    c[s] = c0 + s * (kUnitCols / 2) + 8 * lane;
+    act[s] = c[s] < I;
+    gv[s] = uv[s] = make_uint4(0, 0, 0, 0);
+    if (live && act[s]) {
+      gv[s] = ld_stream_v4(in + c[s] / 8);
+      uv[s] = ld_stream_v4(in + I / 8 + c[s] / 8);
+    }
+  }
+
+  // ---- y = silu(g) * u: y[4 s + e] = columns c[s] + 2e, +1
+  float2 y[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) y[j] = make_float2(0.0f, 0.0f);
+  if (live) {
+    uint32_t check = 0;
+#pragma unroll
+    for (int s = 0; s < 2; ++s)
+      if (act[s])
+        check |= table_check(gv[s].x) | table_check(gv[s].y) | table_check(gv[s].z) |
+                 table_check(gv[s].w);
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const uint32_t g4[4] = {gv[s].x, gv[s].y, gv[s].z, gv[s].w};
+      const uint32_t u4[4] = {uv[s].x, uv[s].y, uv[s].z, uv[s].w};
+      if ((check & kTableCheckBits) == 0) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint32_t lo, hi;
+          table_offsets(g4[e], lo, hi);
+          y[4 * s + e] = make_float2(table_at(tab, lo), table_at(tab, hi));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) y[4 * s + e] = silu2(make_float2(bf16lo(g4[e]), bf16hi(g4[e])));
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        y[4 * s + e] = __fmul2_rn(y[4 * s + e], make_float2(bf16lo(u4[e]), bf16hi(u4[e])));
+    }
+  }
+
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    const float2 *v = y + 4 * s;
+    uint8_t *cd = codes + r * code_row + (int64_t)(c[s] / 8) * kCode8;
+    float amax = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) amax = max_abs3(amax, v[e].x, v[e].y);
+    if (FORMAT == 3) {
+      // ---- bf16, rounded to nearest even
+      if (act[s])
+        st_v4(reinterpret_cast<uint4 *>(cd),
+              make_uint4(pack_bf16x2(v[0].x, v[0].y), pack_bf16x2(v[1].x, v[1].y),
+                         pack_bf16x2(v[2].x, v[2].y), pack_bf16x2(v[3].x, v[3].y)));
+    } else {
+      // ---- MX: 32-column blocks over lane quads, E8M0 scale 2^X
+      constexpr int kEmax = FORMAT == 1 ? 8 : 2;
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+      // an all-zero block is scale 0 and codes 0 (also for -0 elements)
+      const bool nz = amax > 0.0f;
+      const uint32_t sc = nz ? mx_scale_code(amax, kEmax) : 0u;
+      const float2 s2 = splat(pow2i(127 - (int)sc));
+      float2 w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) w[e] = __fmul2_rn(v[e], s2);
+      if (FORMAT == 1) {
+        if (act[s])
+          *reinterpret_cast<uint2 *>(cd) = nz ? make_uint2(cvt_e4m3x4(w[0], w[1]),
+                                                           cvt_e4m3x4(w[2], w[3]))
+                                              : make_uint2(0u, 0u);
+      } else {
+        if (act[s])
+          *reinterpret_cast<uint32_t *>(cd) = nz ? cvt_e2m1x8(w[0], w[1], w[2], w[3]) : 0u;
+      }
+      if (act[s] && (lane & 3) == 0) scales[r * scale_row + c[s] / 32] = (uint8_t)sc;
+    }
+  }
+}
+
+// Persistent over warp units: warp w takes units w, w + warps, ... of the
+// rows * U units (U = ceil(I / 512) per row); (row, unit) advance by
+// (step_rows, step_cols) = divmod(warps, U).  The row_src test is per warp.
+template <int FORMAT>
+__global__ void __launch_bounds__(kThreads, 3)
+    swiglu_split_kernel(const uint4 *__restrict__ gate_up, const int32_t *__restrict__ row_src,
+                        uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int64_t units,
+                        int32_t I, int32_t U, int64_t step_rows, int32_t step_cols) {
+  allow_dependents();
+  __shared__ float tab[kTabSize];
+  for (int i = 2 * threadIdx.x; i < kTabSize; i += 2 * kThreads) {
+    const float2 v = silu2(make_float2(tab_gate(i), tab_gate(i + 1)));
+    tab[i] = v.x;
+    tab[i + 1] = v.y;
+  }
+  __syncthreads();
+  grid_dependency_wait();
+
+  const int lane = threadIdx.x % kWarp;
+  const int64_t warps = (int64_t)gridDim.x * (kThreads / kWarp);
+  int64_t w = (int64_t)blockIdx.x * (kThreads / kWarp) + threadIdx.x / kWarp;
+  int64_t row = w / U;
+  int32_t cu = (int32_t)(w - row * U);
+  for (; w < units; w += warps) {
+    const bool live = __ldg(row_src + row) >= 0;  // no routed token: zero bytes
+    swiglu_unit_split<FORMAT>(tab, gate_up, live, codes, scales, row, cu * kUnitCols, I, lane);
+    row += step_rows;
+    cu += step_cols;
+    if (cu >= U) {
+      cu -= U;
+      ++row;
+    }
+  }
+}
+
 // Persistent: thread t of the grid takes groups t, t + stride, ... of the
 // rows * G groups (G = I / 32 per row); (row, group) advance by
 // (step_rows, step_cols) = divmod(stride, G).
@@ -387,9 +533,37 @@ __global__ void __launch_bounds__(kThreads, 3)
   }
 }
 
+template <int FORMAT>
+cudaError_t launch_split(const uint4 *in, const int32_t *row_src, uint8_t *codes,
+                         uint8_t *scales, int64_t rows, int32_t I, cudaStream_t stream) {
+  auto kernel = swiglu_split_kernel<FORMAT>;
+  static int per_sm[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // resident CTAs per SM, by device
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  int &cap = per_sm[dev & 7];
+  if (cap == 0) {
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cap, kernel, kThreads, 0);
+    if (err != cudaSuccess) return err;
+    cap = std::max(cap, 1);
+  }
+  const int32_t U = (I + kUnitCols - 1) / kUnitCols;
+  const int64_t units = rows * U;
+  const int64_t per_block = kThreads / kWarp;
+  const int64_t want = (units + per_block - 1) / per_block;
+  const int64_t blocks = std::max<int64_t>(
+      1, std::min<int64_t>(want, (int64_t)cap * device_sm_count()));
+  const int64_t warps = blocks * per_block;
+  return launch_pdl(kernel, dim3((unsigned)blocks), dim3(kThreads), 0, stream, in, row_src,
+                    codes, scales, units, I, U, warps / U, (int32_t)(warps % U));
+}
+
 template <int FORMAT, bool INTERLEAVED>
 cudaError_t launch(const uint4 *in, const int32_t *row_src, const float *gs, uint8_t *codes,
                    uint8_t *scales, int64_t rows, int32_t I, cudaStream_t stream) {
+  if (!INTERLEAVED && (FORMAT == 1 || FORMAT == 2 || FORMAT == 3))
+    return launch_split<(FORMAT == 1 || FORMAT == 2) ? FORMAT : 3>(in, row_src, codes, scales,
+                                                                  rows, I, stream);
   auto kernel = swiglu_quant_kernel<FORMAT, INTERLEAVED>;
   static int per_sm[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // resident CTAs per SM, by device
   int dev = 0;

@@ -494,6 +494,9 @@ def test_swiglu_quant_parity(orc, fmt, interleaved, I):
     rng = np.random.default_rng(31 + I + fmt)
     gu = _bits(rng.standard_normal((C, 2 * I)) * np.float32(2.5))
     gu[3, :8] = _bits(np.array([0, -0.0, 30, -30, 90, -90, 1e-3, -1e-3], np.float32))
+    gu[5, :I] = 0x8000                        # gate -0: a row of -0 outputs (all-zero blocks)
+    gu[5, I:] = 0x3F80
+    gu[6, :64] = 0                            # two zero blocks at the start of a row
     codes, scales = B.swiglu_buffers(C, I, fmt)
     gs = torch.tensor([0.01], dtype=torch.float32, device="cuda")
     B.moe_swiglu_quant(run.prob, I, fmt, int(interleaved), to_dev_bf16(gu), run.buf.row_src,
