@@ -105,6 +105,33 @@ def test_payload_shape_rules(lib):
     assert lib.moe_combine(ctypes.byref(bad), *([None] * 5)) == B.MOE_ERR_INVALID_ARG
 
 
+def test_next_row_argument_rules(lib):
+    """MX dispatch, SwiGLU and backward entry points reject bad shapes and
+    arguments on the host, before anything is launched."""
+    p = B.Problem(num_tokens=10, hidden=80, num_experts=8, top_k=2, num_segments=2,
+                  recv_capacity=20)
+    assert _call(lib, "moe_permute_quant_mxfp4", p, 6) == B.MOE_ERR_UNSUPPORTED_SHAPE  # H % 32
+    p.hidden = 128
+    assert _call(lib, "moe_permute_quant_mxfp4", p, 6) == B.MOE_ERR_INVALID_ARG        # nulls
+    assert _call(lib, "moe_permute_backward", p, 4) == B.MOE_ERR_INVALID_ARG
+    assert _call(lib, "moe_combine_backward", p, 8) == B.MOE_ERR_INVALID_ARG
+    c = p.c()
+    sw = lib.moe_swiglu_quant
+    vp = [None] * 6
+    assert sw(ctypes.byref(c), 96, 6, 0, *vp) == B.MOE_ERR_INVALID_ARG          # format
+    assert sw(ctypes.byref(c), 96, 1, 2, *vp) == B.MOE_ERR_INVALID_ARG          # gate/up layout
+    assert sw(ctypes.byref(c), 0, 1, 0, *vp) == B.MOE_ERR_INVALID_ARG           # I <= 0
+    assert sw(ctypes.byref(c), 100, 1, 0, *vp) == B.MOE_ERR_UNSUPPORTED_SHAPE   # I % 32
+    for fmt in range(6):
+        assert sw(ctypes.byref(c), 96, fmt, 0, *vp) == B.MOE_ERR_INVALID_ARG    # null pointers
+    # misaligned codes (MXFP6 needs 8 bytes, the others 16): reported, nothing launched
+    buf = ctypes.create_string_buffer(4096)
+    base = (ctypes.addressof(buf) + 255) // 256 * 256
+    ptrs = [base, base + 256, base + 512, base + 1024 + 8, base + 2048]  # gate_up, row_src, gs, codes, scales
+    assert sw(ctypes.byref(c), 96, 1, 0, ptrs[0], ptrs[1], ptrs[2], ptrs[3], ptrs[4],
+              None) == B.MOE_ERR_INVALID_ARG
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(B, "_lib", None)
     with pytest.raises(RuntimeError, match="not found"):
