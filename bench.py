@@ -47,7 +47,7 @@ NCU_TRAFFIC: dict[str, dict] = {
     "permute_bf16": {"bytes_per_launch": 117978624 + 881097984, "src_sha": "5be478fbcd4e6021"},
     "permute_fp8": {"bytes_per_launch": 118063104 + 426921984, "src_sha": "5be478fbcd4e6021"},
     "permute_nvfp4": {"bytes_per_launch": 118008832 + 207333888, "src_sha": "5be478fbcd4e6021"},
-    "combine": {"bytes_per_launch": 940089088 + 69039616, "src_sha": "3409373de95ae4e3"},
+    "combine": {"bytes_per_launch": 940064768 + 68223488, "src_sha": "3f9751dcacae9354"},
 }
 
 
