@@ -184,19 +184,11 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-// Grid of a persistent kernel: resident CTAs per SM (queried once per
-// kernel and device into `cache`, which the caller keeps per kernel) x SMs,
-// or fewer when there is less work.
+// Grid of a persistent kernel: resident CTAs per SM x SMs, or fewer when
+// there is less work.
 template <typename Kernel>
-int grid_for(Kernel kernel, int64_t N, int (&cache)[8]) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-  int &per_sm = cache[dev & 7];
-  if (per_sm == 0 &&
-      (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) !=
-           cudaSuccess ||
-       per_sm < 1))
-    per_sm = 1;
+int grid_for(Kernel kernel, int64_t N, OccupancyCache &cache) {
+  const int per_sm = resident_ctas(cache, reinterpret_cast<const void *>(kernel), kThreads, 0);
   const int64_t need = std::max<int64_t>(1, (N + kThreads / kWarp - 1) / (kThreads / kWarp));
   return (int)std::min<int64_t>(need, (int64_t)per_sm * device_sm_count());
 }
@@ -205,7 +197,7 @@ template <int KMAX>
 cudaError_t launch_backward(const Shape &s, const uint4 *gy, const uint4 *x, const float *gates,
                             const int32_t *pair_slot, const int32_t *row_src, uint4 *gx,
                             float *grad_gates, int64_t work, cudaStream_t stream) {
-  static int cache[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  static OccupancyCache cache;
   auto kernel = combine_backward_kernel<KMAX>;
   return launch_pdl(kernel, dim3(grid_for(kernel, work, cache)), dim3(kThreads), 0, stream, gy, x,
                     gates, pair_slot, row_src, gx, grad_gates, s.N, s.k, s.rows, s.H / 8);
@@ -214,7 +206,7 @@ cudaError_t launch_backward(const Shape &s, const uint4 *gy, const uint4 *x, con
 template <int KMAX, int U>
 cudaError_t launch_forward(const Shape &s, const uint4 *x, const float *gates,
                            const int32_t *pair_slot, uint4 *o, cudaStream_t stream) {
-  static int cache[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  static OccupancyCache cache;
   auto kernel = combine_kernel<KMAX, U>;
   return launch_pdl(kernel, dim3(grid_for(kernel, s.N, cache)), dim3(kThreads), 0, stream, x, gates,
                     pair_slot, o, s.N, s.k, s.rows, s.H / 8);

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "moe_dc.h"
 
 namespace moe {
@@ -67,6 +69,28 @@ cudaError_t launch_swiglu_quant(const Shape &s, int32_t I, uint32_t format, bool
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
+
+// Resident CTAs per SM of one kernel configuration, queried once per device
+// (devices 0..kMaxDevices-1; others are queried on every call).  Each launch
+// site keeps its own cache (one per kernel instantiation).
+constexpr int kMaxDevices = 64;
+struct OccupancyCache {
+  std::atomic<int> per_sm[kMaxDevices] = {};
+};
+inline int resident_ctas(OccupancyCache &cache, const void *kernel, int threads, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int v = cache.per_sm[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess ||
+      n < 1)
+    n = 1;
+  if (dev >= 0 && dev < kMaxDevices) cache.per_sm[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
 
 // kernel<<<grid, block, smem, stream>>>(args...) with programmatic dependent
 // launch allowed (see grid_dependency_wait in common.cuh).

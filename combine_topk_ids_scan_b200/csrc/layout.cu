@@ -544,8 +544,6 @@ __global__ void __launch_bounds__(kEmitThreads) layout_emit_kernel(LayoutArgs a)
   emit_step<kEmitThreads>(a, gtid, gstride, &s_status, 0);
 }
 
-constexpr int kMaxDevices = 64;
-
 // Opt the scan kernels in to more than 48 KB of dynamic shared memory, once
 // per device.
 cudaError_t opt_in_smem() {

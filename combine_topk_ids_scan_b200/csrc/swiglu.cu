@@ -539,16 +539,8 @@ template <int FORMAT>
 cudaError_t launch_split(const uint4 *in, const int32_t *row_src, uint8_t *codes,
                          uint8_t *scales, int64_t rows, int32_t I, cudaStream_t stream) {
   auto kernel = swiglu_split_kernel<FORMAT>;
-  static int per_sm[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // resident CTAs per SM, by device
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  int &cap = per_sm[dev & 7];
-  if (cap == 0) {
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cap, kernel, kThreads, 0);
-    if (err != cudaSuccess) return err;
-    cap = std::max(cap, 1);
-  }
+  static OccupancyCache occupancy;
+  const int cap = resident_ctas(occupancy, reinterpret_cast<const void *>(kernel), kThreads, 0);
   const int32_t U = (I + kUnitCols - 1) / kUnitCols;
   const int64_t units = rows * U;
   const int64_t per_block = kThreads / kWarp;
@@ -567,16 +559,8 @@ cudaError_t launch(const uint4 *in, const int32_t *row_src, const float *gs, uin
     return launch_split<(FORMAT == 1 || FORMAT == 2) ? FORMAT : 3>(in, row_src, codes, scales,
                                                                   rows, I, stream);
   auto kernel = swiglu_quant_kernel<FORMAT, INTERLEAVED>;
-  static int per_sm[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // resident CTAs per SM, by device
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  int &cap = per_sm[dev & 7];
-  if (cap == 0) {
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cap, kernel, kThreads, 0);
-    if (err != cudaSuccess) return err;
-    cap = std::max(cap, 1);
-  }
+  static OccupancyCache occupancy;
+  const int cap = resident_ctas(occupancy, reinterpret_cast<const void *>(kernel), kThreads, 0);
   const int32_t G = I / kGroupCols;
   const int64_t groups = rows * G;
   const int64_t want = (groups + kThreads - 1) / kThreads;
