@@ -27,11 +27,14 @@
 // one outside the table (zero, tiny, huge, inf, NaN) evaluates the same
 // sequence directly, so the table changes no result, only the work.
 //
-// Persistent grid: the row-major list of (row, 32-column group) pairs is
-// dealt out lane by lane, consecutive lanes taking consecutive groups, so
-// no lane idles when I is not a multiple of 1024.  A lane owns 32
-// consecutive columns: eight 16-byte loads of gate/up, one MX block or two
-// NVFP4 blocks.
+// Two persistent kernels.  swiglu_quant_kernel (interleaved gate/up, and the
+// NVFP4 and MXFP6 outputs of the split layout) deals the row-major list of
+// (row, 32-column group) pairs out lane by lane, so no lane idles when I is
+// not a multiple of 1024; a lane owns 32 consecutive columns: eight 16-byte
+// loads of gate/up, one MX block or two NVFP4 blocks.  swiglu_split_kernel
+// (split layout; MXFP8, MXFP4, bf16) gives each warp 512 columns of a row
+// with 8-column runs per lane, so that its loads and stores are contiguous
+// per warp instruction.
 #include <algorithm>
 
 #include "common.cuh"
@@ -50,7 +53,6 @@ constexpr int kGroupCols = 32;  // columns of one lane
 constexpr uint32_t kTabFirst = 0x3300u;
 constexpr int kTabHalf = 4096;
 constexpr int kTabSize = 2 * kTabHalf;
-
 
 // max / min that return NaN when either operand is NaN
 __device__ __forceinline__ float max_nan(float a, float b) {
