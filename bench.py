@@ -44,17 +44,36 @@ FALLBACK_HBM_GBS = 6650.0
 # metric workload (summaries under profiles/), keyed by kernel; valid only
 # while the kernel's source file is unchanged (sha256 prefix at capture time)
 NCU_TRAFFIC: dict[str, dict] = {
-    "permute_bf16": {"bytes_per_launch": 117978624 + 881097984, "src_sha": "5be478fbcd4e6021"},
-    "permute_fp8": {"bytes_per_launch": 118063104 + 426921984, "src_sha": "5be478fbcd4e6021"},
-    "permute_nvfp4": {"bytes_per_launch": 118008832 + 207333888, "src_sha": "5be478fbcd4e6021"},
-    "combine": {"bytes_per_launch": 940064768 + 68223488, "src_sha": "3f9751dcacae9354"},
+    "permute_bf16": {"bytes_per_launch": 117978624 + 881097984, "src_sha": "stale"},
+    "permute_fp8": {"bytes_per_launch": 118063104 + 426921984, "src_sha": "stale"},
+    "permute_nvfp4": {"bytes_per_launch": 118008832 + 207333888, "src_sha": "stale"},
+    "combine": {"bytes_per_launch": 940064768 + 68223488, "src_sha": "72fe070818477ec9"},
 }
 
 
-def _kernel_src_sha(name: str) -> str:
-    path = os.path.join(ROOT, "combine_topk_ids_scan_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+# the kernel function each phase runs: (source file, function name)
+KERNEL_SRC = {"permute_bf16": ("permute.cu", "permute_bf16_kernel"),
+              "permute_fp8": ("permute.cu", "permute_fp8_kernel"),
+              "permute_nvfp4": ("permute.cu", "permute_fp4_kernel"),
+              "combine": ("combine.cu", "combine_kernel")}
+
+
+def _kernel_src_sha(phase: str) -> str:
+    """Hash of the device code a phase's ncu counters depend on: its kernel
+    function's text (from the __global__ line to the closing brace in column
+    0) plus the shared device helpers (common.cuh).  Host-side edits of the
+    same file leave it unchanged; any change to the kernel or the helpers
+    invalidates the stored traffic."""
+    fn, name = KERNEL_SRC[phase]
+    csrc = os.path.join(ROOT, "combine_topk_ids_scan_b200", "csrc")
+    text = open(os.path.join(csrc, fn)).read()
+    at = text.index(f"    {name}(")
+    start = text.rindex("__global__", 0, at)
+    start = text.rindex("\n", 0, start) + 1
+    end = text.index("\n}\n", at) + 3
+    h = hashlib.sha256(text[start:end].encode())
+    h.update(open(os.path.join(csrc, "common.cuh"), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def _peaks():
@@ -538,10 +557,8 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
         dom = max(("permute_bf16", "permute_fp8", "permute_nvfp4", "combine"),
                   key=lambda p: phase_ms[p])
         achieved = nbytes[dom] / (phase_ms[dom] * 1e-3) / 1e9
-        src = {"permute_bf16": "permute.cu", "permute_fp8": "permute.cu",
-               "permute_nvfp4": "permute.cu", "combine": "combine.cu"}[dom]
         tr = NCU_TRAFFIC.get(dom)
-        traffic = tr["bytes_per_launch"] if tr and tr.get("src_sha") == _kernel_src_sha(src) \
+        traffic = tr["bytes_per_launch"] if tr and tr.get("src_sha") == _kernel_src_sha(dom) \
             else None
         value = world * w.N / (ms * 1e-3)
         line = {
