@@ -44,9 +44,9 @@ FALLBACK_HBM_GBS = 6650.0
 # metric workload (summaries under profiles/), keyed by kernel; valid only
 # while the kernel's source file is unchanged (sha256 prefix at capture time)
 NCU_TRAFFIC: dict[str, dict] = {
-    "permute_bf16": {"bytes_per_launch": 117978624 + 881097984, "src_sha": "stale"},
-    "permute_fp8": {"bytes_per_launch": 118063104 + 426921984, "src_sha": "stale"},
-    "permute_nvfp4": {"bytes_per_launch": 118008832 + 207333888, "src_sha": "stale"},
+    "permute_bf16": {"bytes_per_launch": 117975296 + 881037312, "src_sha": "f744df6e82ed6952"},
+    "permute_fp8": {"bytes_per_launch": 118073600 + 427625472, "src_sha": "1f4ee0778a0f4a1d"},
+    "permute_nvfp4": {"bytes_per_launch": 118075904 + 216867584, "src_sha": "9ddc9db9f6c4a965"},
     "combine": {"bytes_per_launch": 940064768 + 68223488, "src_sha": "72fe070818477ec9"},
 }
 
