@@ -32,11 +32,14 @@
  *
  * Parity status: every function here is pinned by tests/test_oracle_*.py
  * to something other than itself (library sorts, torch casts, brute-force
- * nearest-value search over the format tables, closed forms, invariants
- * the pages state).  The block-scale conventions of the FP8 and NVFP4
- * quantisers (divide by the stored scale; scale = amax/448; NVFP4 block
- * scale = e4m3((amax/6)/global_scale)) are readings of the pages, which
- * print no worked example; the arithmetic under those readings is pinned.
+ * nearest-value search over the format tables, an arithmetic
+ * round-half-even for FP6, the OCP value tables, closed forms, adjoint
+ * identities, invariants the pages state).  The block-scale conventions of
+ * the FP8 and NVFP4 quantisers (divide by the stored scale; scale =
+ * amax/448; NVFP4 block scale = e4m3((amax/6)/global_scale)), the MX shared
+ * scale rule, the MXFP6 packing, the fixed e^x sequence of the SwiGLU and
+ * the scale-factor atom layout are readings of the pages, which print no
+ * worked example; the arithmetic under those readings is pinned.
  */
 #ifndef MOE_ORACLE_H
 #define MOE_ORACLE_H
