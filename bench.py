@@ -481,28 +481,29 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
     # Every step: H2D of the step's inputs (ids, hidden rows, gates, global
     # scale), the whole path with identity experts (the combine reads the bf16
     # dispatch output), D2H of the combined rows, the status word and the
-    # counts.  Two input/output sets and three streams let step i+1's H2D and
-    # step i-1's D2H overlap step i, as a serving loop would.
+    # counts.  Three input/output sets and three streams let the next steps'
+    # H2D and the previous steps' D2H overlap step i, as a serving loop would.
     e2e_steps = max(4, min(args.steps, 40))
-    h_y2 = [h_y, torch.empty_like(h_y).pin_memory()]
-    h_st2 = [h_status, torch.empty_like(h_status).pin_memory()]
+    NSETS = 3
+    h_y2 = [h_y] + [torch.empty_like(h_y).pin_memory() for _ in range(NSETS - 1)]
+    h_st2 = [h_status] + [torch.empty_like(h_status).pin_memory() for _ in range(NSETS - 1)]
     sets = [dict(ids=torch.empty_like(d_ids), hidden=torch.empty_like(d_hidden),
                  gates=torch.empty_like(d_gates), gs=torch.empty_like(d_gs),
                  y=torch.empty_like(d_y), st=torch.empty(1 + w.E, dtype=torch.int32, device=dev))
-            for _ in range(2)]
+            for _ in range(NSETS)]
     s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_comp = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(NSETS)]
+    ev_comp = [torch.cuda.Event() for _ in range(NSETS)]
+    ev_out = [torch.cuda.Event() for _ in range(NSETS)]
     h2d = h_ids.numel() * 4 + h_hidden.numel() * 2 + h_gates.numel() * 4 + h_gs.numel() * 4
     d2h = h_y.numel() * 2 + h_status.numel() * 4
 
     def e2e_step(i):
-        b = i % 2
+        b = i % NSETS
         S = sets[b]
         with torch.cuda.stream(s_in):
-            if i >= 2:
-                s_in.wait_event(ev_comp[b])      # step i-2 is done with set b's inputs
+            if i >= NSETS:
+                s_in.wait_event(ev_comp[b])      # step i-NSETS is done with set b's inputs
             S["ids"].copy_(h_ids, non_blocking=True)
             S["hidden"].view(torch.int16).copy_(h_hidden, non_blocking=True)
             S["gates"].copy_(h_gates, non_blocking=True)
@@ -510,7 +511,7 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
             ev_in[b].record(s_in)
         with torch.cuda.stream(s_comp):
             s_comp.wait_event(ev_in[b])
-            if i >= 2:
+            if i >= NSETS:
                 s_comp.wait_event(ev_out[b])     # set b's result has been read out
             B.layout(prob, S["ids"], buf)
             B.moe_permute(prob, S["hidden"], buf.row_src, buf.pair_slot, buf.out)
@@ -528,7 +529,7 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
             h_st2[b].copy_(S["st"], non_blocking=True)
             ev_out[b].record(s_out)
 
-    for i in range(4):                           # warm the streams and sets
+    for i in range(2 * NSETS):                   # warm the streams and sets
         e2e_step(i)
     torch.cuda.synchronize(dev)
     e_start = torch.cuda.Event(enable_timing=True)
