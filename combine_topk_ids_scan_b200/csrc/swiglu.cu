@@ -27,14 +27,14 @@
 // one outside the table (zero, tiny, huge, inf, NaN) evaluates the same
 // sequence directly, so the table changes no result, only the work.
 //
-// Two persistent kernels.  swiglu_quant_kernel (interleaved gate/up, and the
-// NVFP4 and MXFP6 outputs of the split layout) deals the row-major list of
-// (row, 32-column group) pairs out lane by lane, so no lane idles when I is
-// not a multiple of 1024; a lane owns 32 consecutive columns: eight 16-byte
-// loads of gate/up, one MX block or two NVFP4 blocks.  swiglu_split_kernel
-// (split layout; MXFP8, MXFP4, bf16) gives each warp 512 columns of a row
-// with 8-column runs per lane, so that its loads and stores are contiguous
-// per warp instruction.
+// Two persistent kernels.  swiglu_quant_kernel (the NVFP4 and MXFP6
+// outputs) deals the row-major list of (row, 32-column group) pairs out lane
+// by lane, so no lane idles when I is not a multiple of 1024; a lane owns 32
+// consecutive columns: eight 16-byte loads of gate/up, one MX block or two
+// NVFP4 blocks.  swiglu_split_kernel (MXFP8, MXFP4, bf16; split or
+// interleaved gate/up) gives each warp 512 columns of a row with short
+// column runs per lane, so that its loads and stores are contiguous per
+// warp instruction.
 #include <algorithm>
 
 #include "common.cuh"
@@ -462,12 +462,100 @@ __device__ __forceinline__ void swiglu_unit_split(const float *tab, const uint4 
   }
 }
 
+// Interleaved gate/up, same warp units: the unit's 512 columns are 1024
+// interleaved bf16; lane l holds the 4 columns [c0 + 4 l + 128 j, +4) of
+// the 16-byte vectors l + 32 j (j = 0..3), so loads and stores are again
+// contiguous per warp instruction.  A 32-column MX block spans 8 lanes.
+template <int FORMAT>
+__device__ __forceinline__ void swiglu_unit_interleaved(const float *tab,
+                                                        const uint4 *__restrict__ gate_up,
+                                                        bool live, uint8_t *__restrict__ codes,
+                                                        uint8_t *__restrict__ scales, int64_t r,
+                                                        int32_t c0, int32_t I, int lane) {
+  static_assert(FORMAT == 1 || FORMAT == 2 || FORMAT == 3, "MXFP8, MXFP4 or bf16");
+  constexpr uint32_t kFull = 0xFFFFFFFFu;
+  const uint4 *in = gate_up + r * ((int64_t)I / 4) + c0 / 4;  // 2I bf16 = I/4 vectors
+  int c[4];
+  bool act[4];
+  uint4 iv[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    c[j] = c0 + 4 * lane + (kUnitCols / 4) * j;
+    act[j] = c[j] < I;
+    iv[j] = live && act[j] ? ld_stream_v4(in + lane + 32 * j) : make_uint4(0, 0, 0, 0);
+  }
+  // each 32-bit word is one (gate, up) pair: gate in the low half
+  float2 y[8];  // y[2j + h] = columns c[j] + 2h, +1
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = make_float2(0.0f, 0.0f);
+  if (live) {
+    uint32_t check = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (act[j])
+        check |= table_check(iv[j].x) | table_check(iv[j].y) | table_check(iv[j].z) |
+                 table_check(iv[j].w);
+    const bool in_table = (check & kTableCheckBits & 0xFFFFu) == 0;  // gate halves only
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t wd[4] = {iv[j].x, iv[j].y, iv[j].z, iv[j].w};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t a = wd[2 * h], b = wd[2 * h + 1];
+        float2 sl;
+        if (in_table) {
+          uint32_t lo_a, hi_a, lo_b, hi_b;
+          table_offsets(a, lo_a, hi_a);
+          table_offsets(b, lo_b, hi_b);
+          sl = make_float2(table_at(tab, lo_a), table_at(tab, lo_b));
+        } else {
+          sl = silu2(make_float2(bf16lo(a), bf16lo(b)));
+        }
+        y[2 * j + h] = __fmul2_rn(sl, make_float2(bf16hi(a), bf16hi(b)));
+      }
+    }
+  }
+
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 p0 = y[2 * j], p1 = y[2 * j + 1];
+    if (FORMAT == 3) {
+      // ---- bf16, rounded to nearest even
+      if (act[j])
+        *reinterpret_cast<uint2 *>(codes + r * (2 * (int64_t)I) + 2 * (int64_t)c[j]) =
+            make_uint2(pack_bf16x2(p0.x, p0.y), pack_bf16x2(p1.x, p1.y));
+    } else {
+      // ---- MX: 32-column blocks over 8 lanes, E8M0 scale 2^X
+      constexpr int kEmax = FORMAT == 1 ? 8 : 2;
+      float amax = max_abs3(max_abs3(0.0f, p0.x, p0.y), p1.x, p1.y);
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
+      // an all-zero block is scale 0 and codes 0 (also for -0 elements)
+      const bool nz = amax > 0.0f;
+      const uint32_t sc = nz ? mx_scale_code(amax, kEmax) : 0u;
+      const float2 s2 = splat(pow2i(127 - (int)sc));
+      const float2 w0 = __fmul2_rn(p0, s2), w1 = __fmul2_rn(p1, s2);
+      if (FORMAT == 1) {
+        if (act[j])
+          *reinterpret_cast<uint32_t *>(codes + r * (int64_t)I + c[j]) =
+              nz ? cvt_e4m3x4(w0, w1) : 0u;
+      } else if (act[j]) {
+        const float2 z = make_float2(0.0f, 0.0f);
+        *reinterpret_cast<uint16_t *>(codes + r * ((int64_t)I / 2) + c[j] / 2) =
+            nz ? (uint16_t)(cvt_e2m1x8(w0, w1, z, z) & 0xFFFFu) : (uint16_t)0;
+      }
+      if (act[j] && (lane & 7) == 0) scales[r * ((int64_t)I / 32) + c[j] / 32] = (uint8_t)sc;
+    }
+  }
+}
+
 // Persistent over warp units: warp w takes units w, w + warps, ... of the
 // rows * U units (U = ceil(I / 512) per row); (row, unit) advance by
 // (step_rows, step_cols) = divmod(warps, U).  The row_src test is per warp.
 // MXFP8 is held to 4 resident CTAs per SM (64 registers), the others to 3
 // (measured on B200: MXFP8 230 -> 217 us; MXFP4 209 -> 215 us with 4).
-template <int FORMAT>
+template <int FORMAT, bool INTERLEAVED>
 __global__ void __launch_bounds__(kThreads, FORMAT == 1 ? 4 : 3)
     swiglu_split_kernel(const uint4 *__restrict__ gate_up, const int32_t *__restrict__ row_src,
                         uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int64_t units,
@@ -489,7 +577,11 @@ __global__ void __launch_bounds__(kThreads, FORMAT == 1 ? 4 : 3)
   int32_t cu = (int32_t)(w - row * U);
   for (; w < units; w += warps) {
     const bool live = __ldg(row_src + row) >= 0;  // no routed token: zero bytes
-    swiglu_unit_split<FORMAT>(tab, gate_up, live, codes, scales, row, cu * kUnitCols, I, lane);
+    if (INTERLEAVED)
+      swiglu_unit_interleaved<FORMAT>(tab, gate_up, live, codes, scales, row, cu * kUnitCols, I,
+                                      lane);
+    else
+      swiglu_unit_split<FORMAT>(tab, gate_up, live, codes, scales, row, cu * kUnitCols, I, lane);
     row += step_rows;
     cu += step_cols;
     if (cu >= U) {
@@ -537,10 +629,10 @@ __global__ void __launch_bounds__(kThreads, 3)
   }
 }
 
-template <int FORMAT>
+template <int FORMAT, bool INTERLEAVED>
 cudaError_t launch_split(const uint4 *in, const int32_t *row_src, uint8_t *codes,
                          uint8_t *scales, int64_t rows, int32_t I, cudaStream_t stream) {
-  auto kernel = swiglu_split_kernel<FORMAT>;
+  auto kernel = swiglu_split_kernel<FORMAT, INTERLEAVED>;
   static OccupancyCache occupancy;
   const int cap = resident_ctas(occupancy, reinterpret_cast<const void *>(kernel), kThreads, 0);
   const int32_t U = (I + kUnitCols - 1) / kUnitCols;
@@ -557,9 +649,9 @@ cudaError_t launch_split(const uint4 *in, const int32_t *row_src, uint8_t *codes
 template <int FORMAT, bool INTERLEAVED>
 cudaError_t launch(const uint4 *in, const int32_t *row_src, const float *gs, uint8_t *codes,
                    uint8_t *scales, int64_t rows, int32_t I, cudaStream_t stream) {
-  if (!INTERLEAVED && (FORMAT == 1 || FORMAT == 2 || FORMAT == 3))
-    return launch_split<(FORMAT == 1 || FORMAT == 2) ? FORMAT : 3>(in, row_src, codes, scales,
-                                                                  rows, I, stream);
+  if (FORMAT == 1 || FORMAT == 2 || FORMAT == 3)
+    return launch_split<(FORMAT == 1 || FORMAT == 2) ? FORMAT : 3, INTERLEAVED>(
+        in, row_src, codes, scales, rows, I, stream);
   auto kernel = swiglu_quant_kernel<FORMAT, INTERLEAVED>;
   static OccupancyCache occupancy;
   const int cap = resident_ctas(occupancy, reinterpret_cast<const void *>(kernel), kThreads, 0);
