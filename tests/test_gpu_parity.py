@@ -564,13 +564,15 @@ def test_swiglu_quant_wide_range(orc, gscale):
                   seed=0)
     run = GpuRun(ww, quant=False, combine=False)
     for fmt in (0, 1, 2, 3, 4, 5):
-        codes, scales = B.swiglu_buffers(rows, I, fmt)
-        gs = torch.tensor([gscale], dtype=torch.float32, device="cuda")
-        B.moe_swiglu_quant(run.prob, I, fmt, 0, to_dev_bf16(gu), run.buf.row_src, gs, codes,
-                           scales)
-        torch.cuda.synchronize()
-        want_c, want_s = orc.swiglu_quant(gu, np.arange(rows, dtype=np.int32), fmt,
-                                          global_scale=float(np.float32(gscale)))
-        if fmt != B.MOE_QUANT_BF16:
-            assert np.array_equal(scales.cpu().numpy(), want_s), fmt
-        assert np.array_equal(codes.cpu().numpy(), want_c), fmt
+        for layout in (0, 1):                      # split, interleaved
+            codes, scales = B.swiglu_buffers(rows, I, fmt)
+            gs = torch.tensor([gscale], dtype=torch.float32, device="cuda")
+            B.moe_swiglu_quant(run.prob, I, fmt, layout, to_dev_bf16(gu), run.buf.row_src, gs,
+                               codes, scales)
+            torch.cuda.synchronize()
+            want_c, want_s = orc.swiglu_quant(gu, np.arange(rows, dtype=np.int32), fmt,
+                                              interleaved=bool(layout),
+                                              global_scale=float(np.float32(gscale)))
+            if fmt != B.MOE_QUANT_BF16:
+                assert np.array_equal(scales.cpu().numpy(), want_s), (fmt, layout)
+            assert np.array_equal(codes.cpu().numpy(), want_c), (fmt, layout)
