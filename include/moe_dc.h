@@ -16,6 +16,12 @@
  *   moe_combine              expert outputs [rows,H] bf16 + gates [N,k] fp32
  *                            -> [N,H] bf16, fp32 weighted sum in fixed k order
  *
+ * Further calls: moe_permute_quant_mxfp4 (the MX token format: E2M1 codes +
+ * one E8M0 scale per 32 elements), moe_swiglu_quant (silu(gate) * up of the
+ * expert rows that hold a token, as bf16 or requantised), the gradients
+ * moe_permute_backward and moe_combine_backward, and
+ * moe_dispatch_layout_noalloc (the layout without a caller workspace).
+ *
  * Notation: N tokens, H hidden size, E experts, k = top_k choices per token,
  * S destination segments of L = E/S consecutive experts, P = N*k pairs; pair
  * p = t*k + j routes token t to expert topk_ids[p].  rows = recv_capacity in
