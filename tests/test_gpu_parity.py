@@ -411,6 +411,42 @@ def test_expert_padding_parity(orc, name, two_pass):
     assert_all_outputs(orc, w, run, ref)
 
 
+# ------------------------------------------------------------ random sweep
+def _random_spec(i):
+    """A seeded random problem: any mode (packed, padded, capacity), masked
+    and out-of-range ids, duplicates, ragged sizes."""
+    rng = np.random.default_rng(7000 + i)
+    E = int(rng.choice([1, 3, 8, 24, 64, 160, 256]))
+    divisors = [d for d in range(1, E + 1) if E % d == 0]
+    S = int(rng.choice(divisors))
+    k = int(rng.integers(1, min(16, E) + 1)) if rng.random() < 0.8 else int(rng.integers(1, 17))
+    N = int(rng.choice([0, 1, 2, 31, 257, 1000, 3333]))
+    H = int(32 * rng.choice([1, 3, 4, 7, 12, 16]))
+    spec = dict(N=N, H=H, E=E, k=k, S=S, p_mask=float(rng.choice([0, 0.05, 0.5])),
+                p_bad=float(rng.choice([0, 0, 0.02])), distinct=k <= E and rng.random() < 0.8)
+    mode = rng.choice(["packed", "padded", "capacity"])
+    pad = 0
+    if mode == "capacity":
+        spec["Ce"] = int(rng.integers(1, max(2, 2 * N * k // max(E, 1) + 2)))
+    elif mode == "padded":
+        pad = int(rng.choice([2, 4, 8, 128]))
+        spec["C"] = N * k + E * (pad - 1) - int(rng.integers(0, 3))
+    else:
+        spec["C"] = max(0, int(N * k * rng.uniform(0.8, 1.2)))
+    return spec, pad, bool(rng.random() < 0.5)
+
+
+@pytest.mark.parametrize("i", range(16))
+def test_random_problem_sweep(orc, i):
+    spec, pad, two_pass = _random_spec(i)
+    w = custom(seed=100 + i, **spec)
+    flags = B.MOE_FLAG_CHECK_DUPLICATES | (B.MOE_FLAG_LAYOUT_TWO_PASS if two_pass else 0)
+    run = GpuRun(w, flags=flags, pad=pad)
+    ref = oracle_layout(orc, w, flags=orc.FLAG_CHECK_DUPLICATES, pad=pad)
+    assert_layout(run, ref)
+    assert_all_outputs(orc, w, run, ref)
+
+
 # ------------------------------------------------------------ scale atom layout
 @pytest.mark.parametrize("spec", [
     dict(N=700, H=96, E=8, k=3, S=2, p_mask=0.2),          # 6 scale columns: column padding
