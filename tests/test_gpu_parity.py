@@ -445,6 +445,30 @@ def test_random_problem_sweep(orc, i):
     ref = oracle_layout(orc, w, flags=orc.FLAG_CHECK_DUPLICATES, pad=pad)
     assert_layout(run, ref)
     assert_all_outputs(orc, w, run, ref)
+    rows = run.buf.rows
+    if rows == 0:
+        return
+    rng = np.random.default_rng(9000 + i)
+    # SwiGLU of the dispatch rows: random width, format and gate/up layout
+    I = 32 * int(rng.integers(1, 24))
+    fmt, inter = int(rng.integers(0, 6)), bool(rng.random() < 0.5)
+    gu = _bits(rng.standard_normal((rows, 2 * I)) * 2)
+    codes, scales = B.swiglu_buffers(rows, I, fmt)
+    gs = torch.tensor([0.02], dtype=torch.float32, device="cuda")
+    B.moe_swiglu_quant(run.prob, I, fmt, int(inter), to_dev_bf16(gu), run.buf.row_src, gs,
+                       codes, scales)
+    # dispatch backward of a random row gradient
+    g_rows = _bits(rng.standard_normal((rows, w.H)))
+    gh = torch.empty((max(w.N, 1), w.H), dtype=torch.bfloat16, device="cuda")
+    if w.N > 0:
+        B.moe_permute_backward(run.prob, to_dev_bf16(g_rows), run.buf.pair_slot, gh)
+    torch.cuda.synchronize()
+    want_c, want_s = orc.swiglu_quant(gu, ref.row_src, fmt, interleaved=inter, global_scale=0.02)
+    assert np.array_equal(codes.cpu().numpy(), want_c), (fmt, inter)
+    if fmt != B.MOE_QUANT_BF16:
+        assert np.array_equal(scales.cpu().numpy(), want_s), (fmt, inter)
+    if w.N > 0:
+        assert np.array_equal(bf16_np(gh), orc.permute_backward(g_rows, ref.pair_slot))
 
 
 # ------------------------------------------------------------ scale atom layout
