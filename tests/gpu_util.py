@@ -31,6 +31,7 @@ class GpuRun:
                  expert_out: np.ndarray | None = None, pad: int = 0):
         prob = problem_of(w, flags, pad)
         self.prob = prob
+        self.swizzled = bool(flags & B.MOE_FLAG_NVFP4_SWIZZLED_SCALES)
         buf = B.Buffers(prob)
         self.buf = buf
         ids = torch.from_numpy(np.ascontiguousarray(w.ids)).cuda()

@@ -81,12 +81,21 @@ def assert_all_outputs(orc, w, run, ref, rows_sample=None, tokens_sample=None):
         assert np.array_equal(run.q8[idx], q), "fp8 codes"
         assert np.array_equal(run.s8[idx].view(np.uint32), s.view(np.uint32)), "fp8 scales"
     if run.has_fp4:
+        # atom-layout scales (MOE_FLAG_NVFP4_SWIZZLED_SCALES) are compared in full
+        swz = run.swizzled
+        assert not swz or rows_sample is None
+        def same_scales(got, want_linear):
+            if not swz:
+                return np.array_equal(got[idx], want_linear)
+            want = orc.swizzle_scales(want_linear).reshape(-1)   # empty when rows == 0
+            return got.size >= want.size and np.array_equal(got[:want.size], want)
+
         q, s = orc.permute_nvfp4(w.hidden, row_src[idx], w.global_scale)
         assert np.array_equal(run.q4[idx], q), "nvfp4 codes"
-        assert np.array_equal(run.s4[idx], s), "nvfp4 scales"
+        assert same_scales(run.s4, s), "nvfp4 scales"
         q, s = orc.permute_mxfp4(w.hidden, row_src[idx])
         assert np.array_equal(run.qmx[idx], q), "mxfp4 codes"
-        assert np.array_equal(run.smx[idx], s), "mxfp4 scales"
+        assert same_scales(run.smx, s), "mxfp4 scales"
     if run.y is not None:
         tok = np.arange(w.N) if tokens_sample is None else tokens_sample
         y = orc.combine(w.expert_out, w.gates[tok], ref.pair_slot[tok])
@@ -433,14 +442,15 @@ def _random_spec(i):
         spec["C"] = N * k + E * (pad - 1) - int(rng.integers(0, 3))
     else:
         spec["C"] = max(0, int(N * k * rng.uniform(0.8, 1.2)))
-    return spec, pad, bool(rng.random() < 0.5)
+    return spec, pad, bool(rng.random() < 0.5), bool(rng.random() < 0.4)
 
 
 @pytest.mark.parametrize("i", range(16))
 def test_random_problem_sweep(orc, i):
-    spec, pad, two_pass = _random_spec(i)
+    spec, pad, two_pass, swizzled = _random_spec(i)
     w = custom(seed=100 + i, **spec)
-    flags = B.MOE_FLAG_CHECK_DUPLICATES | (B.MOE_FLAG_LAYOUT_TWO_PASS if two_pass else 0)
+    flags = B.MOE_FLAG_CHECK_DUPLICATES | (B.MOE_FLAG_LAYOUT_TWO_PASS if two_pass else 0) | \
+        (B.MOE_FLAG_NVFP4_SWIZZLED_SCALES if swizzled else 0)
     run = GpuRun(w, flags=flags, pad=pad)
     ref = oracle_layout(orc, w, flags=orc.FLAG_CHECK_DUPLICATES, pad=pad)
     assert_layout(run, ref)
