@@ -3,8 +3,6 @@ world_size-2 gloo process groups on the CPU."""
 import os
 import socket
 
-import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
