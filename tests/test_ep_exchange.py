@@ -97,6 +97,20 @@ def _worker(rank, world, port, mode, q):
         back = ep.combine_exchange(recv, route)
         sent = route.send_total
         assert np.array_equal(back.numpy()[:sent], out[:sent])
+        # argument errors are raised before any collective (every rank raises)
+        bad = torch.zeros((4, world + 1), dtype=torch.int32)
+        try:
+            ep.exchange_counts(bad, p["H"], p["E"])
+            raise AssertionError("segments != ranks accepted")
+        except ValueError:
+            pass
+        one_each = ep.Route(send_rows=[1] * world, recv_rows=[1] * world)
+        for call, rows in ((ep.dispatch_exchange, world - 1), (ep.combine_exchange, world + 1)):
+            try:
+                call(torch.zeros((rows, 4)), one_each)
+                raise AssertionError(f"{call.__name__}: wrong row count accepted")
+            except ValueError:
+                pass
         q.put((rank, "ok"))
     except Exception as e:  # report to the parent instead of hanging it
         q.put((rank, repr(e)))
