@@ -282,9 +282,9 @@ __device__ __forceinline__ int64_t sf_atom_offset(int64_t m, int32_t c, int32_t 
 // MX == false: NVFP4 (two 16-element blocks per lane, E4M3 scales);
 // MX == true: MXFP4 (one 32-element block per lane, E8M0 scales).
 // SWIZZLED: scales in the block-scale atom layout.  The linear-scale kernels
-// are held to 5 resident CTAs per SM (48 registers; measured on B200 at the
-// metric shape: NVFP4 74 -> 70 us, MXFP4 61.4 -> 60.0 us), the atom-layout
-// kernels to 4 (with 5 they were slower).
+// are held to 5 resident CTAs per SM (at most 48 registers; measured on B200
+// at the metric shape: NVFP4 74 -> 70 us, MXFP4 61.4 -> 60.0 us), the
+// atom-layout kernels to 4 (with 5 they were slower).
 template <bool MX, bool SWIZZLED>
 __global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
     permute_fp4_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
@@ -354,19 +354,27 @@ __global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       x[i] = active ? ld_stream_v4(src + col / 8 + i) : make_uint4(0, 0, 0, 0);
-    float f[32];
+    // x[i] holds the lane's elements 8i..8i+7.  MXFP4 unpacks its one
+    // 32-element block; NVFP4 unpacks one 16-element block at a time, so
+    // that only 16 floats are live (under the 5-CTA bound the 32-float form
+    // spilled 40 bytes per thread, now 4 in the IEEE-division fallback;
+    // measured on B200 at the metric shape: 71.5 -> 69.0 us)
+    float f[MX ? 32 : 16];
+    const auto unpack = [&](int i0, int n) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t wd[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+      for (int i = 0; i < n; ++i) {
+        const uint32_t wd[4] = {x[i0 + i].x, x[i0 + i].y, x[i0 + i].z, x[i0 + i].w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        f[8 * i + 2 * e] = bf16lo(wd[e]);
-        f[8 * i + 2 * e + 1] = bf16hi(wd[e]);
+        for (int e = 0; e < 4; ++e) {
+          f[8 * i + 2 * e] = bf16lo(wd[e]);
+          f[8 * i + 2 * e + 1] = bf16hi(wd[e]);
+        }
       }
-    }
+    };
     uint4 codes;
     uint32_t sq, quad;
-    if (MX) {
+    if constexpr (MX) {
+      unpack(0, 4);
       sq = mxfp4_block(f, codes);
       // atom layout: lanes 4g..4g+3 hold scale columns 4g..4g+3 -- one
       // 4-byte store per four lanes (inactive lanes contribute zeros: the
@@ -375,8 +383,10 @@ __global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
       quad = a | (__shfl_down_sync(kFull, a, 1) << 8) | (__shfl_down_sync(kFull, a, 2) << 16) |
              (__shfl_down_sync(kFull, a, 3) << 24);
     } else {
+      unpack(0, 2);
       const uint32_t sq0 = nvfp4_block(f, gs, codes.x, codes.y);
-      const uint32_t sq1 = nvfp4_block(f + 16, gs, codes.z, codes.w);
+      unpack(2, 2);
+      const uint32_t sq1 = nvfp4_block(f, gs, codes.z, codes.w);
       sq = sq0 | (sq1 << 8);
       // atom layout: an even lane holds scale columns 4g, 4g+1 and its odd
       // neighbour 4g+2, 4g+3 -- one 4-byte store per pair of lanes (an
