@@ -46,7 +46,7 @@ FALLBACK_HBM_GBS = 6650.0
 NCU_TRAFFIC: dict[str, dict] = {
     "permute_bf16": {"bytes_per_launch": 117975296 + 881037312, "src_sha": "f744df6e82ed6952"},
     "permute_fp8": {"bytes_per_launch": 118073600 + 427625472, "src_sha": "1f4ee0778a0f4a1d"},
-    "permute_nvfp4": {"bytes_per_launch": 118075904 + 216867584, "src_sha": "9ddc9db9f6c4a965"},
+    "permute_nvfp4": {"bytes_per_launch": 118132480 + 209912832, "src_sha": "bd259e3412ffa849"},
     "combine": {"bytes_per_launch": 940064768 + 68223488, "src_sha": "72fe070818477ec9"},
 }
 

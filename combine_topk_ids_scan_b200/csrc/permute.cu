@@ -357,8 +357,9 @@ __global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
     // x[i] holds the lane's elements 8i..8i+7.  MXFP4 unpacks its one
     // 32-element block; NVFP4 unpacks one 16-element block at a time, so
     // that only 16 floats are live (under the 5-CTA bound the 32-float form
-    // spilled 40 bytes per thread, now 4 in the IEEE-division fallback;
-    // measured on B200 at the metric shape: 71.5 -> 69.0 us)
+    // spilled 40 bytes per thread: 7 local stores and 10 local loads per
+    // unit, now 1 and 4; measured on B200 at the metric shape:
+    // 71.5 -> 69.0 us)
     float f[MX ? 32 : 16];
     const auto unpack = [&](int i0, int n) {
 #pragma unroll
