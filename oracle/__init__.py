@@ -43,6 +43,34 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+# Every output buffer handed to the C code is filled with a poison byte and
+# followed by a guard of _GUARD poison bytes: an element the oracle fails to
+# write keeps the poison (and fails the value checks), and a write past the
+# end of the buffer is reported by _Outs.check.
+_GUARD = 64
+_POISON = 0xA5
+
+
+class _Outs:
+    """Allocator of poisoned, guarded output arrays for one oracle call."""
+
+    def __init__(self):
+        self._bufs = []
+
+    def __call__(self, shape, dtype) -> np.ndarray:
+        dt = np.dtype(dtype)
+        shape = tuple(int(d) for d in np.atleast_1d(shape)) if np.ndim(shape) else (int(shape),)
+        n = int(np.prod(shape, dtype=np.int64)) * dt.itemsize
+        raw = np.full(n + _GUARD, _POISON, np.uint8)
+        self._bufs.append((raw, n))
+        return raw[:n].view(dt).reshape(shape)
+
+    def check(self, fn: str) -> None:
+        for raw, n in self._bufs:
+            if not np.all(raw[n:] == _POISON):
+                raise RuntimeError(f"{fn} wrote past the end of an output buffer")
+
+
 def _p(a: np.ndarray | None):
     if a is None:
         return None
@@ -95,36 +123,46 @@ def lib():
 # ---------------------------------------------------------------- formats
 def bf16_from_f32(x: np.ndarray) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float32)
-    out = np.empty(x.shape, dtype=np.uint16)
+    o = _Outs()
+    out = o(x.shape, np.uint16)
     lib().orc_bf16_from_f32_n(_p(x), _p(out), x.size)
+    o.check("orc_bf16_from_f32_n")
     return out
 
 
 def e4m3_from_f32(x: np.ndarray) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float32)
-    out = np.empty(x.shape, dtype=np.uint8)
+    o = _Outs()
+    out = o(x.shape, np.uint8)
     lib().orc_e4m3_from_f32_n(_p(x), _p(out), x.size)
+    o.check("orc_e4m3_from_f32_n")
     return out
 
 
 def e2m1_from_f32(x: np.ndarray) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float32)
-    out = np.empty(x.shape, dtype=np.uint8)
+    o = _Outs()
+    out = o(x.shape, np.uint8)
     lib().orc_e2m1_from_f32_n(_p(x), _p(out), x.size)
+    o.check("orc_e2m1_from_f32_n")
     return out
 
 
 def e2m3_from_f32(x: np.ndarray) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float32)
-    out = np.empty(x.shape, np.uint8)
+    o = _Outs()
+    out = o(x.shape, np.uint8)
     lib().orc_e2m3_from_f32_n(_p(x), _p(out), x.size)
+    o.check("orc_e2m3_from_f32_n")
     return out
 
 
 def e3m2_from_f32(x: np.ndarray) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float32)
-    out = np.empty(x.shape, np.uint8)
+    o = _Outs()
+    out = o(x.shape, np.uint8)
     lib().orc_e3m2_from_f32_n(_p(x), _p(out), x.size)
+    o.check("orc_e3m2_from_f32_n")
     return out
 
 
@@ -138,8 +176,10 @@ def e3m2_to_f32(code: int) -> float:
 
 def pack_fp6(codes: np.ndarray) -> np.ndarray:
     codes = np.ascontiguousarray(codes, dtype=np.uint8).reshape(-1)
-    out = np.empty(codes.size * 3 // 4, np.uint8)
+    o = _Outs()
+    out = o(codes.size * 3 // 4, np.uint8)
     lib().orc_pack_fp6(_p(codes), codes.size, _p(out))
+    o.check("orc_pack_fp6")
     return out
 
 
@@ -173,16 +213,18 @@ def layout(ids: np.ndarray, num_experts: int, num_segments: int, hidden: int,
     N, k = ids.shape
     E, S = num_experts, num_segments
     rows = E * expert_capacity if expert_capacity > 0 else recv_capacity
-    counts = np.empty(E, np.int32)
-    offsets = np.empty(E + 1, np.int32)
-    meta = np.empty((4, S), np.uint32)
-    row_src = np.empty(rows, np.int32)
-    pair_slot = np.empty((N, k), np.int32)
-    drop = np.empty((N, k), np.uint8)
+    o = _Outs()
+    counts = o(E, np.int32)
+    offsets = o(E + 1, np.int32)
+    meta = o((4, S), np.uint32)
+    row_src = o(rows, np.int32)
+    pair_slot = o((N, k), np.int32)
+    drop = o((N, k), np.uint8)
     st = lib().orc_layout(N, k, E, S, recv_capacity, expert_capacity, expert_pad_multiple,
                           flags, hidden,
                           _p(ids), _p(counts), _p(offsets), _p(meta), _p(row_src),
                           _p(pair_slot), _p(drop))
+    o.check("orc_layout")
     return Layout(int(st), counts, offsets, meta, row_src, pair_slot, drop)
 
 
@@ -192,8 +234,10 @@ def permute_bf16(hidden_bits: np.ndarray, row_src: np.ndarray) -> np.ndarray:
     hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
     row_src = np.ascontiguousarray(row_src, dtype=np.int32)
     H = hidden_bits.shape[1]
-    out = np.empty((row_src.size, H), np.uint16)
+    o = _Outs()
+    out = o((row_src.size, H), np.uint16)
     lib().orc_permute_bf16(row_src.size, H, _p(hidden_bits), _p(row_src), _p(out))
+    o.check("orc_permute_bf16")
     return out
 
 
@@ -201,9 +245,11 @@ def permute_fp8(hidden_bits: np.ndarray, row_src: np.ndarray):
     hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
     row_src = np.ascontiguousarray(row_src, dtype=np.int32)
     H = hidden_bits.shape[1]
-    q = np.empty((row_src.size, H), np.uint8)
-    sc = np.empty((row_src.size, H // 128), np.float32)
+    o = _Outs()
+    q = o((row_src.size, H), np.uint8)
+    sc = o((row_src.size, H // 128), np.float32)
     lib().orc_permute_fp8(row_src.size, H, _p(hidden_bits), _p(row_src), _p(q), _p(sc))
+    o.check("orc_permute_fp8")
     return q, sc
 
 
@@ -211,10 +257,12 @@ def permute_nvfp4(hidden_bits: np.ndarray, row_src: np.ndarray, global_scale: fl
     hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
     row_src = np.ascontiguousarray(row_src, dtype=np.int32)
     H = hidden_bits.shape[1]
-    q = np.empty((row_src.size, H // 2), np.uint8)
-    sc = np.empty((row_src.size, H // 16), np.uint8)
+    o = _Outs()
+    q = o((row_src.size, H // 2), np.uint8)
+    sc = o((row_src.size, H // 16), np.uint8)
     lib().orc_permute_nvfp4(row_src.size, H, _p(hidden_bits), _p(row_src),
                             float(np.float32(global_scale)), _p(q), _p(sc))
+    o.check("orc_permute_nvfp4")
     return q, sc
 
 
@@ -222,9 +270,11 @@ def permute_mxfp4(hidden_bits: np.ndarray, row_src: np.ndarray):
     hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
     row_src = np.ascontiguousarray(row_src, dtype=np.int32)
     H = hidden_bits.shape[1]
-    q = np.empty((row_src.size, H // 2), np.uint8)
-    sc = np.empty((row_src.size, H // 32), np.uint8)
+    o = _Outs()
+    q = o((row_src.size, H // 2), np.uint8)
+    sc = o((row_src.size, H // 32), np.uint8)
     lib().orc_permute_mxfp4(row_src.size, H, _p(hidden_bits), _p(row_src), _p(q), _p(sc))
+    o.check("orc_permute_mxfp4")
     return q, sc
 
 
@@ -232,8 +282,10 @@ def swizzle_scales(linear: np.ndarray) -> np.ndarray:
     """[rows, nsf] uint8 scales -> the 128x4 atom layout (flat uint8)."""
     linear = np.ascontiguousarray(linear, dtype=np.uint8)
     rows, nsf = linear.shape
-    out = np.empty(((rows + 127) // 128 * 128) * ((nsf + 3) // 4 * 4), np.uint8)
+    o = _Outs()
+    out = o(((rows + 127) // 128 * 128) * ((nsf + 3) // 4 * 4), np.uint8)
     lib().orc_swizzle_scales(rows, nsf, _p(linear), _p(out))
+    o.check("orc_swizzle_scales")
     return out
 
 
@@ -246,8 +298,10 @@ def combine(expert_out_bits: np.ndarray, gates: np.ndarray,
     pair_slot = np.ascontiguousarray(pair_slot, dtype=np.int32)
     N, k = pair_slot.shape
     rows, H = expert_out_bits.shape
-    y = np.empty((N, H), np.uint16)
+    o = _Outs()
+    y = o((N, H), np.uint16)
     lib().orc_combine(N, k, H, rows, _p(expert_out_bits), _p(gates), _p(pair_slot), _p(y))
+    o.check("orc_combine")
     return y
 
 
@@ -258,8 +312,10 @@ def permute_backward(grad_out_bits: np.ndarray, pair_slot: np.ndarray) -> np.nda
     pair_slot = np.ascontiguousarray(pair_slot, dtype=np.int32)
     N, k = pair_slot.shape
     rows, H = grad_out_bits.shape
-    gh = np.empty((N, H), np.uint16)
+    o = _Outs()
+    gh = o((N, H), np.uint16)
     lib().orc_permute_backward(N, k, H, rows, _p(grad_out_bits), _p(pair_slot), _p(gh))
+    o.check("orc_permute_backward")
     return gh
 
 
@@ -272,10 +328,12 @@ def combine_backward(grad_y_bits: np.ndarray, expert_out_bits: np.ndarray, gates
     pair_slot = np.ascontiguousarray(pair_slot, dtype=np.int32)
     N, k = pair_slot.shape
     rows, H = expert_out_bits.shape
-    gx = np.empty((rows, H), np.uint16)
-    gw = np.empty((N, k), np.float32)
+    o = _Outs()
+    gx = o((rows, H), np.uint16)
+    gw = o((N, k), np.float32)
     lib().orc_combine_backward(N, k, H, rows, _p(grad_y_bits), _p(expert_out_bits), _p(gates),
                                _p(pair_slot), _p(gx), _p(gw))
+    o.check("orc_combine_backward")
     return gx, gw
 
 
@@ -296,8 +354,10 @@ def swiglu_scale_bytes(I: int, fmt: int) -> int:
 
 def exp_f32(x: np.ndarray) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float32)
-    out = np.empty_like(x)
+    o = _Outs()
+    out = o(x.shape, np.float32)
     lib().orc_exp_n(_p(x), _p(out), x.size)
+    o.check("orc_exp_n")
     return out
 
 
@@ -308,8 +368,10 @@ def swiglu_quant(gate_up_bits: np.ndarray, row_src: np.ndarray, fmt: int,
     row_src = np.ascontiguousarray(row_src, dtype=np.int32)
     rows, two_i = gate_up_bits.shape
     I = two_i // 2
-    codes = np.empty((rows, swiglu_code_bytes(I, fmt)), np.uint8)
-    scales = np.empty((rows, swiglu_scale_bytes(I, fmt)), np.uint8)
+    o = _Outs()
+    codes = o((rows, swiglu_code_bytes(I, fmt)), np.uint8)
+    scales = o((rows, swiglu_scale_bytes(I, fmt)), np.uint8)
     lib().orc_swiglu_quant(rows, I, _p(gate_up_bits), int(interleaved), _p(row_src), fmt,
                            float(np.float32(global_scale)), _p(codes), _p(scales))
+    o.check("orc_swiglu_quant")
     return codes, scales

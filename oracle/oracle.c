@@ -446,12 +446,12 @@ static uint8_t mx_scale_code(float amax, int32_t emax) {
   return (uint8_t)c;
 }
 
-/* y * 2^(127 - code): the MX scaling of an element (one rounding). */
+/* y * 2^(127 - code): the MX scaling of an element (one rounding).  The
+ * codes of mx_scale_code are at most 252 (floor(log2 amax) <= 127 for a
+ * float, emax >= 2), so 2^(127 - code) is a normal float: biased exponent
+ * 254 - code in [2, 254]. */
 static float mx_scale_down(float y, uint8_t code) {
-  const int32_t X = (int32_t)code - 127;
-  return -X >= -126 ? y * f32_from_bits((uint32_t)(-X + 127) << 23)
-                    : (y * f32_from_bits((uint32_t)(-X - 64 + 127) << 23)) *
-                          f32_from_bits((uint32_t)(64 + 127) << 23);
+  return y * f32_from_bits((uint32_t)(254 - code) << 23);
 }
 
 /* Mojo MAX ep_comm MXTokenFormat (MX FP4 token format): OCP MX v1.0 MXFP4,
@@ -725,9 +725,9 @@ void orc_swiglu_quant(int64_t rows, int32_t I, const uint16_t *gate_up,
         sd[b] = sc;
         const int32_t X = (int32_t)sc - 127;
         for (int32_t i = 0; i < 32; ++i) {
-          /* y * 2^-X: X in [-127, 127] */
-          float v = -X >= -126 ? y[32 * b + i] * pow2i(-X)
-                               : (y[32 * b + i] * pow2i(-X - 64)) * pow2i(64);
+          /* y * 2^-X: X in [-127, 125] (sc <= 252: floor(log2 amax) <= 127
+           * for a float and emax >= 2), so 2^-X is a normal float */
+          float v = y[32 * b + i] * pow2i(-X);
           if (format == 1) {
             cd[32 * b + i] = orc_e4m3_from_f32(v);
           } else if (i % 2 == 0) {

@@ -67,6 +67,52 @@ def test_combine_backward_adjoint_in_expert_outputs(orc):
     assert np.all(gx[lay.row_src < 0] == 0)
 
 
+def test_permute_backward_exact_on_integer_rows(orc):
+    """Integer gradients with |g| <= 16: every partial sum of k = 6 terms is
+    exact in fp32 and the total (|sum| <= 96) exact in bf16, so the dispatch
+    backward must equal numpy's gather-sum bit for bit; masked slots and a
+    slot equal to rows contribute nothing."""
+    w = make_workload("mid_zipf", n_tokens=256)
+    C = w.N * w.k + 37
+    lay = orc.layout(w.ids, w.E, w.S, w.H, recv_capacity=C)
+    H = 256                                   # any row width; keeps the test small
+    rng = np.random.default_rng(21)
+    g = rng.integers(-16, 17, size=(C, H)).astype(np.float32)
+    slots = lay.pair_slot.copy()
+    slots[0, 1] = C                           # == rows: outside the buffer
+    slots[1, 2] = -1
+    gh = orc.permute_backward(bf16_bits(g), slots)
+    valid = (slots >= 0) & (slots < C)
+    want = np.where(valid[:, :, None], g[np.clip(slots, 0, C - 1)], 0).sum(axis=1)
+    assert np.array_equal(f32(gh), want.astype(np.float32))
+
+
+def test_combine_backward_exact_on_integer_rows(orc):
+    """Power-of-two gates and small integer rows make every product and dot
+    exact: grad_expert_out[slot(t,j)] = w[t,j] * grad_y[t] and
+    grad_gates[t,j] = <grad_y[t], X[slot(t,j)]> (numpy einsum), zeros in the
+    rows no pair owns, gate gradient 0 for a masked slot or a slot equal to
+    rows."""
+    N, k, H, rows = 40, 4, 96, 200
+    rng = np.random.default_rng(22)
+    slots = (1 + rng.permutation(rows - 1)[:N * k]).astype(np.int32).reshape(N, k)
+    slots[3, 0] = -1
+    slots[7, 2] = rows
+    gates = (2.0 ** rng.integers(-3, 3, size=(N, k))).astype(np.float32)
+    gy = rng.integers(-8, 9, size=(N, H)).astype(np.float32)
+    X = rng.integers(-8, 9, size=(rows, H)).astype(np.float32)
+    gx, gw = orc.combine_backward(bf16_bits(gy), bf16_bits(X), gates, slots)
+    valid = (slots >= 0) & (slots < rows)
+    want_gx = np.zeros((rows, H), np.float32)
+    t_idx, j_idx = np.nonzero(valid)
+    want_gx[slots[t_idx, j_idx]] = gates[t_idx, j_idx, None] * gy[t_idx]
+    assert np.array_equal(f32(gx), want_gx)
+    want_gw = np.einsum("th,tjh->tj", gy.astype(np.float64),
+                        X[np.clip(slots, 0, rows - 1)].astype(np.float64))
+    want_gw = np.where(valid, want_gw, 0.0).astype(np.float32)
+    assert np.array_equal(gw, want_gw)
+
+
 def test_gate_gradient_closed_form(orc):
     """With constant expert rows X[s] = c_s and grad_y[t] = 1, the gate
     gradient is H * c_s exactly."""

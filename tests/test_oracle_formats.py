@@ -72,6 +72,21 @@ def test_bf16_matches_torch_cast(orc):
     assert np.array_equal(got, want)
 
 
+def test_bf16_infinities_and_nans(orc):
+    """IEEE 754: an infinity converts to the infinity of the same sign; a NaN
+    stays a NaN (all-ones exponent, non-zero fraction) with its sign, whatever
+    its payload (the payload itself is not pinned)."""
+    got = orc.bf16_from_f32(np.array([np.inf, -np.inf], np.float32))
+    assert got.tolist() == [0x7F80, 0xFF80]
+    nan_bits = np.array([0x7FC00000, 0x7F800001, 0xFF800001, 0x7FFFFFFF, 0x7F80FFFF,
+                         0xFFC12345, 0x7F810000], np.uint32)
+    got = orc.bf16_from_f32(nan_bits.view(np.float32)).astype(np.uint32)
+    assert np.all((got & 0x7F80) == 0x7F80) and np.all((got & 0x7F) != 0)
+    assert np.array_equal(got >> 15, nan_bits >> 31)
+    back = torch.from_numpy(got.astype(np.uint16).view(np.int16)).view(torch.bfloat16).float()
+    assert torch.isnan(back).all()
+
+
 # ------------------------------------------------------------------ e4m3
 def test_e4m3_decode_matches_torch_and_spec(orc):
     dec = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()

@@ -131,6 +131,47 @@ def test_id_range_and_duplicates_status(orc):
     assert not (lay.status & orc.STATUS_DUP_ID)
 
 
+def test_id_equal_to_num_experts_is_out_of_range(orc):
+    """Valid ids are [0, E): E itself is reported and treated as masked (no
+    row, not counted, not a drop), in both modes."""
+    ids = np.array([[4, 0], [3, 4], [2, 1]], np.int32)
+    for kw in (dict(recv_capacity=8), dict(expert_capacity=2)):
+        lay = orc.layout(ids, 4, 2, 8, **kw)
+        assert lay.status == orc.STATUS_ID_RANGE
+        assert lay.pair_slot[0, 0] == -1 and lay.pair_slot[1, 1] == -1
+        assert lay.drop_mask.sum() == 0
+        assert lay.expert_counts.tolist() == [1, 1, 1, 1]
+        ref = numpy_layout(ids, 4, 2, 8, C=kw.get("recv_capacity", 0),
+                           Ce=kw.get("expert_capacity", 0))
+        check_equal(lay, ref)
+
+
+@pytest.mark.parametrize("where", ["first", "middle", "last"])
+def test_duplicate_check_reaches_every_token(orc, where):
+    """A single token naming one expert twice is reported wherever it sits;
+    without it the same matrix is clean."""
+    N, k, E = 9, 3, 16
+    ids = (np.arange(N * k, dtype=np.int32) % E).reshape(N, k)   # distinct per token
+    lay = orc.layout(ids, E, 4, 8, recv_capacity=N * k, flags=orc.FLAG_CHECK_DUPLICATES)
+    assert lay.status == 0
+    t = {"first": 0, "middle": N // 2, "last": N - 1}[where]
+    ids[t, k - 1] = ids[t, 0]
+    lay = orc.layout(ids, E, 4, 8, recv_capacity=N * k, flags=orc.FLAG_CHECK_DUPLICATES)
+    assert lay.status == orc.STATUS_DUP_ID
+
+
+def test_duplicate_check_ignores_masked_and_out_of_range_ids(orc):
+    """Reading: the duplicate check concerns experts a token is routed to, so
+    repeated -1 (masked) entries are not duplicates, and repeated out-of-range
+    ids are reported as out of range only."""
+    ids = np.array([[-1, -1, 0], [2, 1, 3]], np.int32)
+    lay = orc.layout(ids, 4, 2, 8, recv_capacity=6, flags=orc.FLAG_CHECK_DUPLICATES)
+    assert lay.status == 0
+    ids = np.array([[4, 4, 0], [-2, -2, 1]], np.int32)
+    lay = orc.layout(ids, 4, 2, 8, recv_capacity=6, flags=orc.FLAG_CHECK_DUPLICATES)
+    assert lay.status == orc.STATUS_ID_RANGE
+
+
 @pytest.mark.parametrize("cfg", ["tiny", "mid_zipf", "nvfp4_hot", "balanced_static"])
 def test_packed_invariants_on_workloads(orc, cfg):
     w = make_workload(cfg, n_tokens=2048 if cfg != "tiny" else None,

@@ -121,6 +121,8 @@ def test_swiglu_mxfp6_block_rule(orc, fmt):
     rows, I = 16, 128
     gu = bf16_bits(rng.standard_normal((rows, 2 * I)) * 2)
     gu[2, I:I + 32] = 0                       # an all-zero block (u = 0)
+    gu[3, 32], gu[3, I + 32] = bf16_bits([8.0, 16.0])   # block max at its element 0
+    gu[5, I + 64:I + 96] = bf16_bits(np.full(32, 1e-39))  # tiny block: the scale clamps
     src = np.arange(rows, dtype=np.int32)
     src[7] = -1
     f = orc.FMT_MXFP6_E2M3 if fmt == "e2m3" else orc.FMT_MXFP6_E3M2
@@ -142,13 +144,18 @@ def test_swiglu_mxfp6_block_rule(orc, fmt):
             if amax == 0:
                 assert scales[r, k] == 0 and not c6[32 * k:32 * k + 32].any()
                 continue
-            X = math.frexp(amax)[1] - 1 - emax
+            # E8M0 holds 2^-127 .. 2^127: a smaller X takes the smallest scale
+            X = max(math.frexp(amax)[1] - 1 - emax, -127)
             assert scales[r, k] == X + 127
             v = rne_fp6(blk * 2.0 ** -X, fmt)
             got = np.where(c6[32 * k:32 * k + 32] >= 32, -1.0, 1.0) * tab[c6[32 * k:32 * k + 32] & 31]
             assert np.array_equal(got, v)
-            # the scaled block maximum lands in the top binade [2^emax, 2^(emax+1))
-            assert 2.0 ** emax <= amax * 2.0 ** -X < 2.0 ** (emax + 1)
+            if X > -127:
+                # the scaled block maximum lands in the top binade [2^emax, 2^(emax+1))
+                assert 2.0 ** emax <= amax * 2.0 ** -X < 2.0 ** (emax + 1)
+    blk = y[3, 32:64]
+    assert np.argmax(np.abs(blk)) == 0 and np.abs(blk[0]) >= 2 * np.abs(blk[1:]).max()
+    assert scales[5, 2] == 0 and 0 < np.abs(y[5, 64:96]).max() < 2.0 ** (-126 + emax)
 
 
 def test_permute_mxfp4_block_rule(orc):
@@ -163,6 +170,8 @@ def test_permute_mxfp4_block_rule(orc):
     x[5, :32] = bf16_bits(np.full(32, -0.0, np.float32))
     x[9, :64] = rng.integers(1, 0x7F, 64).astype(np.uint16)        # bf16 subnormals
     x[9, 64:96] = 0x7F7F                                            # bf16 maximum
+    x[7, 96:128] = bf16_bits(np.linspace(0.1, 0.2, 32))
+    x[7, 96] = bf16_bits([-3.0])[0]                                 # block max at element 0
     row_src = np.array([0, 3, -1, 5, 19, 7, 3, -1, 9], np.int32)
     q, s = orc.permute_mxfp4(x, row_src)
     assert q.shape == (9, H // 2) and s.shape == (9, H // 32)

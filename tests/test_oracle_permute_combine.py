@@ -77,6 +77,29 @@ def test_permute_fp8_against_brute_force(orc, tiny):
     assert np.all(q[7] == 0) and np.all(sc[7] == 0)
 
 
+@pytest.mark.parametrize("last", ["padding", "zero_block"])
+def test_permute_quantisers_fill_to_the_end_of_the_buffer(orc, last):
+    """The buffer's last row as a padding row, or as a row ending in an
+    all-zero block: its codes and scales are all zero up to the end of the
+    buffer and not a byte further (every oracle output is followed by a
+    guard that the call checks)."""
+    rng = np.random.default_rng(8)
+    H = 256
+    hidden = bf16_bits(rng.standard_normal((4, H)))
+    hidden[1, H - 128:] = 0                   # the last 128 elements are zero
+    row_src = np.array([0, 2, -1 if last == "padding" else 1], np.int32)
+    for name, (q, sc), block in (("fp8", orc.permute_fp8(hidden, row_src), 128),
+                                 ("nvfp4", orc.permute_nvfp4(hidden, row_src, 0.01), 16),
+                                 ("mxfp4", orc.permute_mxfp4(hidden, row_src), 32)):
+        code_bytes = q.shape[1] // (H // 128)        # code bytes of the last 128 elements
+        assert not q[2, -code_bytes:].any(), name
+        assert not sc[2, -(128 // block):].any(), name
+        if last == "padding":
+            assert not q[2].any() and not sc[2].any(), name
+        else:
+            assert q[2, :-code_bytes].any(), name
+
+
 def test_permute_nvfp4_hand_block(orc):
     # one row, H=32: block 0 = [6, 0.5, 0, ...], block 1 = [-3, 1.5, 0, ...]
     x = np.zeros((1, 32), np.float32)
@@ -153,9 +176,12 @@ def test_combine_k1_unit_gate_is_gather(orc):
 
 
 def test_combine_skips_masked_and_out_of_range(orc):
-    X = bf16_bits(np.arange(12, dtype=np.float32).reshape(3, 4))
-    gates = np.array([[0.5, 0.25, 2.0]], np.float32)
-    slots = np.array([[1, -1, 7]], np.int32)      # row 7 does not exist
+    # X is the first 3 rows of a 4-row array: a read of row 3 would see
+    # non-zero values
+    X4 = bf16_bits(np.arange(1, 17, dtype=np.float32).reshape(4, 4))
+    X = X4[:3]
+    gates = np.array([[0.5, 0.25, 2.0, 4.0]], np.float32)
+    slots = np.array([[1, -1, 7, 3]], np.int32)   # rows 7 and 3 (= rows) do not exist
     y = orc.combine(X, gates, slots)
     assert np.array_equal(f32(y[0]), np.float32(0.5) * f32(X[1]))
 

@@ -42,6 +42,28 @@ def test_exp_within_two_ulps(orc):
     assert orc.exp_f32(np.array([-200.0], np.float32))[0] == 0.0
 
 
+def test_exp_overflow_and_subnormal_tails(orc):
+    """Near the ends of the float range: x in [88.38, 88.72] (n = 128, the
+    result scaled in two steps) within 2 ulps of float64 exp, and inf once
+    e^x is clearly past the largest float; x in [-103.9, -87.4] (subnormal
+    results, scaled in two steps) within 2 ulps of the float64 value rounded
+    to float32."""
+    rng = np.random.default_rng(6)
+    hi = np.concatenate([rng.uniform(88.38, 88.7228, 20000), [88.4, 88.5, 88.7]]).astype(np.float32)
+    got = orc.exp_f32(hi)
+    want = np.exp(hi.astype(np.float64))
+    assert np.all(want < np.finfo(np.float32).max)
+    assert np.all(ulps(got, want.astype(np.float32)) <= 2)
+    over = np.array([88.7230, 88.73, 88.749], np.float32)
+    assert np.all(np.exp(over.astype(np.float64)) > 1.0001 * float(np.finfo(np.float32).max))
+    assert np.all(orc.exp_f32(over) == np.inf)
+    lo = np.concatenate([rng.uniform(-103.9, -87.4, 20000), [-88.0, -100.0]]).astype(np.float32)
+    got = orc.exp_f32(lo)
+    want = np.exp(lo.astype(np.float64)).astype(np.float32)
+    assert np.all(want < np.finfo(np.float32).tiny) and np.all(want > 0)
+    assert np.all(ulps(got, want) <= 2)
+
+
 def test_silu_closed_forms(orc):
     L = orc.lib()
     assert L.orc_silu(0.0) == 0.0
@@ -77,6 +99,10 @@ def test_mx_element_codes_brute_force(orc):
     rng = np.random.default_rng(3)
     rows, I = 40, 128
     gu = bf16_bits(rng.standard_normal((rows, 2 * I)) * 3)
+    gu[9, I + 32:I + 64] = 0                  # all-zero blocks: scale 0, codes 0
+    gu[11, I + 64:I + 96] = 0
+    gu[rows - 1, 2 * I - 32:] = 0             # ... the buffer's last block
+    gu[12, I:I + 32] = bf16_bits(np.full(32, 1e-39))   # tiny block: the scale clamps
     src = np.arange(rows, dtype=np.int32)
     src[5] = -1
     gf, uf = f32(gu[:, :I]), f32(gu[:, I:])
@@ -94,7 +120,12 @@ def test_mx_element_codes_brute_force(orc):
             for b in range(I // 32):
                 blk = y[r, 32 * b:32 * b + 32]
                 amax = np.abs(blk).max()
-                X = math.floor(math.log2(amax)) - emax
+                if amax == 0:
+                    w = 32 if fmt == 1 else 16
+                    assert scales[r, b] == 0 and not codes[r, w * b:w * b + w].any()
+                    continue
+                # E8M0 holds 2^-127 .. 2^127: a smaller X takes the smallest scale
+                X = max(math.floor(math.log2(amax)) - emax, -127)
                 assert scales[r, b] == X + 127
                 v = (blk.astype(np.float64) * 2.0 ** -X).astype(np.float32)
                 if fmt == 1:
@@ -105,6 +136,7 @@ def test_mx_element_codes_brute_force(orc):
                     mag = brute_nearest_even(v, c2, v2, 7)
                     c = mag | np.where(np.signbit(v), 8, 0)
                     assert np.array_equal(codes[r, 16 * b:16 * b + 16], c[0::2] | (c[1::2] << 4))
+        assert scales[12, 0] == 0 and 0 < np.abs(y[12, :32]).max() < 2.0 ** (-127 + emax)
 
 
 def test_nvfp4_matches_dispatch_rule_on_swiglu_output(orc):
@@ -114,12 +146,14 @@ def test_nvfp4_matches_dispatch_rule_on_swiglu_output(orc):
     rng = np.random.default_rng(4)
     I, rows = 64, 6
     y_bf = bf16_bits(rng.standard_normal((rows, I)))
+    y_bf[2, 16:32] = 0                        # an all-zero 16-element block
     g = np.full((rows, I), 64.0, np.float32)
     u = f32(y_bf) / np.float32(64.0)          # exact: power-of-two scaling
     gu = bf16_bits(np.concatenate([g, u], axis=1))
     codes, scales = orc.swiglu_quant(gu, np.arange(rows, dtype=np.int32), 0, global_scale=0.01)
     q, s = orc.permute_nvfp4(y_bf, np.arange(rows, dtype=np.int32), 0.01)
     assert np.array_equal(codes, q) and np.array_equal(scales, s)
+    assert scales[2, 1] == 0 and not codes[2, 8:16].any()
 
 
 def test_interleaved_equals_split(orc):
