@@ -74,8 +74,10 @@ typedef enum moe_status {
 /* Bits of the device status word written by moe_dispatch_layout. */
 enum {
   MOE_STATUS_ID_RANGE = 1u, /* an id outside [-1, E): treated as masked     */
-  MOE_STATUS_DUP_ID = 2u,   /* a token names one expert twice (checked only
-                               with MOE_FLAG_CHECK_DUPLICATES)             */
+  MOE_STATUS_DUP_ID = 2u,   /* a token names one expert (an id in [0, E))
+                               twice; repeated -1 or out-of-range ids are
+                               not duplicates (checked only with
+                               MOE_FLAG_CHECK_DUPLICATES)                  */
   MOE_STATUS_CAPACITY = 4u, /* packed mode: more routed pairs than
                                recv_capacity; the excess pairs get no row  */
   MOE_STATUS_TIMEOUT = 8u   /* a bounded wait of the scan gave up (about one
