@@ -117,6 +117,16 @@ def test_e4m3_encode_matches_torch_in_range(orc):
     assert np.array_equal(got, want)
 
 
+def test_e4m3_encode_nan(orc):
+    """E4M3 ("fn") keeps one NaN encoding, S.1111.111: a NaN of either sign
+    and any payload maps to it with its sign, as torch's cast does."""
+    nan_bits = np.array([0x7FC00000, 0xFFC00000, 0x7F800001, 0xFF812345, 0x7FFFFFFF], np.uint32)
+    x = nan_bits.view(np.float32)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = orc.e4m3_from_f32(x)
+    assert np.array_equal(got, want) and np.array_equal(got, [0x7F, 0xFF, 0x7F, 0xFF, 0x7F])
+
+
 def test_e4m3_encode_brute_force_and_saturation(orc):
     codes, vals = e4m3_table()
     rng = np.random.default_rng(3)
