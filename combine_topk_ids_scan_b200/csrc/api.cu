@@ -70,6 +70,25 @@ moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR
 
 }  // namespace
 
+namespace moe {
+
+moe_status check_layout_args(const moe_problem *problem, const int32_t *topk_ids,
+                             const int32_t *expert_counts, const int32_t *expert_offsets,
+                             const uint32_t *meta, const int32_t *row_src,
+                             const int32_t *pair_slot, const uint32_t *status, Shape *s) {
+  moe_status st = make_shape(problem, s);
+  if (st != MOE_OK) return st;
+  if (!expert_counts || !expert_offsets || !meta || !status) return MOE_ERR_INVALID_ARG;
+  if (s->P > 0 && (!topk_ids || !pair_slot)) return MOE_ERR_INVALID_ARG;
+  if (s->rows > 0 && !row_src) return MOE_ERR_INVALID_ARG;
+  if (!aligned(topk_ids, 4) || !aligned(expert_counts, 4) || !aligned(expert_offsets, 4) ||
+      !aligned(meta, 4) || !aligned(row_src, 4) || !aligned(pair_slot, 4) || !aligned(status, 4))
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+}  // namespace moe
+
 extern "C" {
 
 int64_t moe_output_rows(const moe_problem *problem) {
@@ -90,15 +109,10 @@ moe_status moe_dispatch_layout(const moe_problem *problem, const int32_t *topk_i
                                uint8_t *drop_mask, uint32_t *status, void *workspace,
                                moe_stream_t stream) {
   moe::Shape s;
-  moe_status st = make_shape(problem, &s);
+  moe_status st = moe::check_layout_args(problem, topk_ids, expert_counts, expert_offsets, meta,
+                                         row_src, pair_slot, status, &s);
   if (st != MOE_OK) return st;
-  if (!expert_counts || !expert_offsets || !meta || !status || !workspace)
-    return MOE_ERR_INVALID_ARG;
-  if (s.P > 0 && (!topk_ids || !pair_slot)) return MOE_ERR_INVALID_ARG;
-  if (s.rows > 0 && !row_src) return MOE_ERR_INVALID_ARG;
-  if (!aligned(workspace, 16) || !aligned(topk_ids, 4) || !aligned(pair_slot, 4) ||
-      !aligned(row_src, 4) || !aligned(status, 4))
-    return MOE_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 16)) return MOE_ERR_INVALID_ARG;
   moe::LayoutWorkspace ws = moe::layout_workspace_view(s, workspace);
   return from_cuda(moe::launch_layout(s, topk_ids, expert_counts, expert_offsets, meta, row_src,
                                       pair_slot, drop_mask, status, ws,
@@ -115,7 +129,9 @@ moe_status moe_permute(const moe_problem *problem, const void *hidden_states,
   if (s.rows == 0) return MOE_OK;
   if (!row_src || !out || (s.P > 0 && (!hidden_states || !pair_slot)))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned(hidden_states, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(hidden_states, 16) || !aligned(out, 16) || !aligned(row_src, 4) ||
+      !aligned(pair_slot, 4))
+    return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_permute_bf16(s, hidden_states, row_src, pair_slot, out,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -130,7 +146,8 @@ moe_status moe_permute_quant_fp8(const moe_problem *problem, const void *hidden_
   if (s.rows == 0) return MOE_OK;
   if (!row_src || !out_e4m3 || !scales || (s.P > 0 && (!hidden_states || !pair_slot)))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned(hidden_states, 16) || !aligned(out_e4m3, 16) || !aligned(scales, 4))
+  if (!aligned(hidden_states, 16) || !aligned(out_e4m3, 16) || !aligned(scales, 4) ||
+      !aligned(row_src, 4) || !aligned(pair_slot, 4))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_permute_fp8(s, hidden_states, row_src, pair_slot, out_e4m3,
                                            scales, reinterpret_cast<cudaStream_t>(stream)));
@@ -150,7 +167,8 @@ moe_status moe_permute_quant_nvfp4(const moe_problem *problem, const void *hidde
     return MOE_ERR_INVALID_ARG;
   const uintptr_t scale_align = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) ? 4 : 2;
   if (!aligned(hidden_states, 16) || !aligned(out_e2m1, 16) ||
-      !aligned(scales_e4m3, scale_align) || !aligned(global_scale, 4))
+      !aligned(scales_e4m3, scale_align) || !aligned(global_scale, 4) || !aligned(row_src, 4) ||
+      !aligned(pair_slot, 4))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_permute_nvfp4(s, hidden_states, row_src, pair_slot, global_scale,
                                              out_e2m1, scales_e4m3,
@@ -168,7 +186,8 @@ moe_status moe_permute_quant_mxfp4(const moe_problem *problem, const void *hidde
   if (!row_src || !out_e2m1 || !scales_e8m0 || (s.P > 0 && (!hidden_states || !pair_slot)))
     return MOE_ERR_INVALID_ARG;
   const uintptr_t scale_align = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) ? 4 : 1;
-  if (!aligned(hidden_states, 16) || !aligned(out_e2m1, 16) || !aligned(scales_e8m0, scale_align))
+  if (!aligned(hidden_states, 16) || !aligned(out_e2m1, 16) ||
+      !aligned(scales_e8m0, scale_align) || !aligned(row_src, 4) || !aligned(pair_slot, 4))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_permute_mxfp4(s, hidden_states, row_src, pair_slot, out_e2m1,
                                              scales_e8m0,
@@ -183,7 +202,8 @@ moe_status moe_combine(const moe_problem *problem, const void *expert_out, const
   if (s.H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (s.N == 0) return MOE_OK;
   if (!out || !gates || !pair_slot || (s.rows > 0 && !expert_out)) return MOE_ERR_INVALID_ARG;
-  if (!aligned(expert_out, 16) || !aligned(out, 16) || !aligned(gates, 4))
+  if (!aligned(expert_out, 16) || !aligned(out, 16) || !aligned(gates, 4) ||
+      !aligned(pair_slot, 4))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_combine(s, expert_out, gates, pair_slot, out,
                                        reinterpret_cast<cudaStream_t>(stream)));
@@ -198,7 +218,8 @@ moe_status moe_permute_backward(const moe_problem *problem, const void *grad_out
   if (s.H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (s.N == 0) return MOE_OK;
   if (!grad_hidden || !pair_slot || (s.rows > 0 && !grad_out)) return MOE_ERR_INVALID_ARG;
-  if (!aligned(grad_out, 16) || !aligned(grad_hidden, 16)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(grad_out, 16) || !aligned(grad_hidden, 16) || !aligned(pair_slot, 4))
+    return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_combine(s, grad_out, nullptr, pair_slot, grad_hidden,
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -216,7 +237,8 @@ moe_status moe_combine_backward(const moe_problem *problem, const void *grad_y,
       (s.rows > 0 && (!expert_out || !row_src || !grad_expert_out)))
     return MOE_ERR_INVALID_ARG;
   if (!aligned(grad_y, 16) || !aligned(expert_out, 16) || !aligned(grad_expert_out, 16) ||
-      !aligned(gates, 4) || !aligned(grad_gates, 4))
+      !aligned(gates, 4) || !aligned(grad_gates, 4) || !aligned(pair_slot, 4) ||
+      !aligned(row_src, 4))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_combine_backward(s, grad_y, expert_out, gates, pair_slot, row_src,
                                                 grad_expert_out, grad_gates,
@@ -244,7 +266,7 @@ moe_status moe_swiglu_quant(const moe_problem *problem, int32_t intermediate, ui
   const bool fp6 = format == MOE_QUANT_MXFP6_E2M3 || format == MOE_QUANT_MXFP6_E3M2;
   if (!aligned(gate_up, 16) || !aligned(codes, fp6 ? 8 : 16) ||
       (has_scales && !aligned(scales, format == MOE_QUANT_NVFP4 ? 2 : 1)) ||
-      (global_scale && !aligned(global_scale, 4)))
+      (global_scale && !aligned(global_scale, 4)) || !aligned(row_src, 4))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_swiglu_quant(s, intermediate, format,
                                             gate_up_layout == MOE_GATE_UP_INTERLEAVED, gate_up,

@@ -29,6 +29,13 @@ struct LayoutWorkspace {
   int32_t num_tiles; // T
 };
 
+// Host checks of moe_dispatch_layout's problem and pointers (everything but
+// the workspace); fills *s on success.  Launches nothing.
+moe_status check_layout_args(const moe_problem *problem, const int32_t *topk_ids,
+                             const int32_t *expert_counts, const int32_t *expert_offsets,
+                             const uint32_t *meta, const int32_t *row_src,
+                             const int32_t *pair_slot, const uint32_t *status, Shape *s);
+
 int32_t layout_num_tiles(int64_t P);
 size_t layout_workspace_bytes(const Shape &s);
 LayoutWorkspace layout_workspace_view(const Shape &s, void *workspace);

@@ -6,6 +6,7 @@
 
 #include <mutex>
 
+#include "internal.h"
 #include "moe_dc.h"
 
 namespace {
@@ -43,10 +44,12 @@ extern "C" moe_status moe_dispatch_layout_noalloc(
     const moe_problem *problem, const int32_t *topk_ids, int32_t *expert_counts,
     int32_t *expert_offsets, uint32_t *meta, int32_t *row_src, int32_t *pair_slot,
     uint8_t *drop_mask, uint32_t *status, moe_stream_t stream) {
-  const size_t need = moe_workspace_bytes(problem);
-  if (need == 0)  // an invalid problem: report it exactly as the layout does
-    return moe_dispatch_layout(problem, topk_ids, expert_counts, expert_offsets, meta, row_src,
-                               pair_slot, drop_mask, status, nullptr, stream);
+  // the layout's own host checks first: nothing is enqueued for bad arguments
+  moe::Shape s;
+  const moe_status st = moe::check_layout_args(problem, topk_ids, expert_counts, expert_offsets,
+                                               meta, row_src, pair_slot, status, &s);
+  if (st != MOE_OK) return st;
+  const size_t need = moe::layout_workspace_bytes(s);
   if (need > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED_SHAPE;
   void *scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;

@@ -34,6 +34,10 @@
  *     a HOST pointer, read during the call only.
  *   - bf16 data is passed as void* to 16-byte-aligned buffers of IEEE
  *     bfloat16 (the layout of __nv_bfloat16), row-major with no padding.
+ *   - int32, uint32 and fp32 arrays (ids, maps, counts, meta, status, gates,
+ *     fp32 scales) are 4-byte aligned; each call checks every pointer's
+ *     alignment on the host and returns MOE_ERR_INVALID_ARG, launching
+ *     nothing, for a misaligned one.
  *   - Every call only enqueues kernels on `stream` (a cudaStream_t) and
  *     returns; nothing synchronises with the host.
  *   - A moe_status return reports argument errors found on the host before

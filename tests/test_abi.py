@@ -132,6 +132,46 @@ def test_next_row_argument_rules(lib):
               None) == B.MOE_ERR_INVALID_ARG
 
 
+# entry point -> (fixed leading arguments after the problem, the pointer
+# arguments' required alignment in bytes (1: none); a trailing stream of None)
+ALIGNMENT_RULES = {
+    "moe_dispatch_layout": ((), (4, 4, 4, 4, 4, 4, 1, 4, 16)),
+    "moe_dispatch_layout_noalloc": ((), (4, 4, 4, 4, 4, 4, 1, 4)),
+    "moe_permute": ((), (16, 4, 4, 16)),
+    "moe_permute_quant_fp8": ((), (16, 4, 4, 16, 4)),
+    "moe_permute_quant_nvfp4": ((), (16, 4, 4, 4, 16, 2)),
+    "moe_permute_quant_mxfp4": ((), (16, 4, 4, 16, 1)),
+    "moe_combine": ((), (16, 4, 4, 16)),
+    "moe_permute_backward": ((), (16, 4, 16)),
+    "moe_combine_backward": ((), (16, 16, 4, 4, 4, 16, 4)),
+    "moe_swiglu_quant": ((128, 0, 0), (16, 4, 4, 16, 2)),   # I = 128, NVFP4, split
+}
+
+
+def test_every_pointer_alignment_is_checked_on_the_host(lib):
+    """Each call gets aligned, non-null (host) addresses except for one
+    misaligned pointer, and must reject it before launching anything.
+    Skipped where a GPU is present: the addresses are not device memory."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-side argument checks only; run on a machine without a GPU")
+    buf = ctypes.create_string_buffer(64 * 256 + 256)
+    base = (ctypes.addressof(buf) + 255) // 256 * 256
+    p = B.Problem(num_tokens=10, hidden=128, num_experts=8, top_k=2, num_segments=2,
+                  recv_capacity=20)
+    c = p.c()
+    checked = 0
+    for fn, (lead, aligns) in ALIGNMENT_RULES.items():
+        for i, a in enumerate(aligns):
+            for off in sorted({a // 2, 1} - {0}) if a > 1 else []:
+                ptrs = [base + 256 * n for n in range(len(aligns))]
+                ptrs[i] += off
+                rc = getattr(lib, fn)(ctypes.byref(c), *lead, *ptrs, None)
+                assert rc == B.MOE_ERR_INVALID_ARG, (fn, i, a, off, rc)
+                checked += 1
+    assert checked > 60
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(B, "_lib", None)
     with pytest.raises(RuntimeError, match="not found"):
