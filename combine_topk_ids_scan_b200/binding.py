@@ -37,7 +37,8 @@ MOE_MAX_TOPK = 16
 
 # every symbol include/moe_dc.h declares
 EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout",
-            "moe_dispatch_layout_noalloc", "moe_permute", "moe_permute_quant_fp8",
+            "moe_dispatch_layout_noalloc", "moe_permute", "moe_permute_premultiplied",
+            "moe_permute_quant_fp8",
             "moe_permute_quant_nvfp4", "moe_permute_quant_mxfp4", "moe_combine",
             "moe_permute_backward",
             "moe_combine_backward", "moe_swiglu_quant", "moe_status_string", "moe_version")
@@ -107,6 +108,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     L.moe_dispatch_layout_noalloc.argtypes = [P] + [vp] * 9
     L.moe_permute.restype = ctypes.c_int
     L.moe_permute.argtypes = [P] + [vp] * 5
+    L.moe_permute_premultiplied.restype = ctypes.c_int
+    L.moe_permute_premultiplied.argtypes = [P] + [vp] * 6
     L.moe_permute_quant_fp8.restype = ctypes.c_int
     L.moe_permute_quant_fp8.argtypes = [P] + [vp] * 6
     L.moe_permute_quant_nvfp4.restype = ctypes.c_int
@@ -192,6 +195,16 @@ def moe_permute(prob: Problem, hidden_states, row_src, pair_slot, out, stream=No
     c = prob.c()
     _check(load().moe_permute(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
                               _ptr(pair_slot), _ptr(out), _stream(stream)), "moe_permute")
+
+
+def moe_permute_premultiplied(prob: Problem, hidden_states, row_src, pair_slot, gates, out,
+                              stream=None) -> None:
+    """Dispatch with pre-multiplied gates: each pair's row is its token
+    scaled by its gate (see moe_permute_premultiplied in moe_dc.h)."""
+    c = prob.c()
+    _check(load().moe_permute_premultiplied(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
+                                            _ptr(pair_slot), _ptr(gates), _ptr(out),
+                                            _stream(stream)), "moe_permute_premultiplied")
 
 
 def moe_permute_quant_fp8(prob: Problem, hidden_states, row_src, pair_slot, out_e4m3, scales,

@@ -136,6 +136,23 @@ moe_status moe_permute(const moe_problem *problem, const void *hidden_states,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_permute_premultiplied(const moe_problem *problem, const void *hidden_states,
+                                     const int32_t *row_src, const int32_t *pair_slot,
+                                     const float *gates, void *out, moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.rows == 0) return MOE_OK;
+  if (!row_src || !out || (s.P > 0 && (!hidden_states || !pair_slot || !gates)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(hidden_states, 16) || !aligned(out, 16) || !aligned(row_src, 4) ||
+      !aligned(pair_slot, 4) || !aligned(gates, 4))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_permute_premultiplied(s, hidden_states, row_src, pair_slot, gates,
+                                                     out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_permute_quant_fp8(const moe_problem *problem, const void *hidden_states,
                                  const int32_t *row_src, const int32_t *pair_slot,
                                  uint8_t *out_e4m3, float *scales, moe_stream_t stream) {

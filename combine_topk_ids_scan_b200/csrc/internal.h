@@ -48,6 +48,10 @@ cudaError_t launch_layout(const Shape &s, const int32_t *ids, int32_t *expert_co
 cudaError_t launch_permute_bf16(const Shape &s, const void *hidden, const int32_t *row_src,
                                 const int32_t *pair_slot, void *out, cudaStream_t stream);
 
+cudaError_t launch_permute_premultiplied(const Shape &s, const void *hidden,
+                                         const int32_t *row_src, const int32_t *pair_slot,
+                                         const float *gates, void *out, cudaStream_t stream);
+
 cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t *row_src,
                                const int32_t *pair_slot, uint8_t *q, float *scales,
                                cudaStream_t stream);

@@ -119,6 +119,64 @@ __global__ void __launch_bounds__(kThreads)
 
 }
 
+// --------------------------------------------------- pre-multiplied gates
+// DeepSpeed's pre-multiplication of the token representations by their
+// router scores before expert compute: the bf16 permute's units, but pair
+// (t, j)'s row is bf16(w[t,j] * x[t]) -- one fp32 product and one rounding
+// (nearest even) per element.
+__device__ __forceinline__ uint4 scale_bf16x8(const uint4 &v, float g) {
+  return make_uint4(pack_bf16x2(g * bf16lo(v.x), g * bf16hi(v.x)),
+                    pack_bf16x2(g * bf16lo(v.y), g * bf16hi(v.y)),
+                    pack_bf16x2(g * bf16lo(v.z), g * bf16hi(v.z)),
+                    pack_bf16x2(g * bf16lo(v.w), g * bf16hi(v.w)));
+}
+
+__global__ void __launch_bounds__(kThreads)
+    permute_premultiplied_kernel(const uint4 *__restrict__ hidden,
+                                 const int32_t *__restrict__ row_src,
+                                 const int32_t *__restrict__ pair_slot,
+                                 const float *__restrict__ gates, uint4 *__restrict__ out,
+                                 int32_t N, int32_t k, int64_t rows, int32_t vecs,
+                                 int32_t chunks) {
+  allow_dependents();
+  grid_dependency_wait();
+  constexpr int U = kBf16Chunk / 8 / kWarp;  // 2
+  const int lane = threadIdx.x % kWarp;
+  const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
+  const int64_t units = (int64_t)N * chunks;
+  const int64_t pad_units = (rows + kWarp - 1) / kWarp;
+  if (w0 < pad_units) {
+    if (const uint32_t m = padding_mask(w0, lane, row_src, rows, rows))
+      zero_rows(m, w0, lane, out, vecs, 0, vecs, nullptr, 0, 0, 0);
+    return;
+  }
+  const int64_t w = w0 - pad_units;
+  if (w >= units) return;
+  const int64_t t = w / chunks;
+  const int v0 = (int)(w % chunks) * (kBf16Chunk / 8);
+  int32_t my_slot;
+  uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+  const float my_w = lane < k ? __ldg(gates + t * k + lane) : 0.0f;
+  const uint4 *src = hidden + t * vecs;
+  uint4 x[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int v = v0 + u * kWarp + lane;
+    if (v < vecs) x[u] = ld_stream_v4(src + v);
+  }
+  while (live) {
+    const int j = __ffs(live) - 1;
+    live &= live - 1;
+    const float g = __shfl_sync(kFull, my_w, j);
+    uint4 *dst = out + (int64_t)__shfl_sync(kFull, my_slot, j) * vecs;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + u * kWarp + lane;
+      if (v < vecs) st_v4(dst + v, scale_bf16x8(x[u], g));
+    }
+  }
+}
+
 // ------------------------------------------------------------------- FP8
 // Unit = (token, 1024 elements).  A lane takes 16 consecutive elements per
 // half (two 16-byte loads -> one 16-byte store of codes); 8 lanes form one
@@ -431,6 +489,17 @@ cudaError_t launch_permute_bf16(const Shape &s, const void *hidden, const int32_
   return launch_pdl(permute_bf16_kernel, dim3((unsigned)unit_blocks(s, chunks, s.rows)),
                     dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src,
                     pair_slot, static_cast<uint4 *>(out), s.N, s.k, s.rows, s.H / 8, chunks);
+}
+
+cudaError_t launch_permute_premultiplied(const Shape &s, const void *hidden,
+                                         const int32_t *row_src, const int32_t *pair_slot,
+                                         const float *gates, void *out, cudaStream_t stream) {
+  if (s.rows == 0) return cudaSuccess;
+  const int32_t chunks = chunks_of(s.H, kBf16Chunk);
+  return launch_pdl(permute_premultiplied_kernel,
+                    dim3((unsigned)unit_blocks(s, chunks, s.rows)), dim3(kThreads), 0, stream,
+                    static_cast<const uint4 *>(hidden), row_src, pair_slot, gates,
+                    static_cast<uint4 *>(out), s.N, s.k, s.rows, s.H / 8, chunks);
 }
 
 cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t *row_src,

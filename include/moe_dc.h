@@ -19,7 +19,8 @@
  * Further calls: moe_permute_quant_mxfp4 (the MX token format: E2M1 codes +
  * one E8M0 scale per 32 elements), moe_swiglu_quant (silu(gate) * up of the
  * expert rows that hold a token, as bf16 or requantised), the gradients
- * moe_permute_backward and moe_combine_backward, and
+ * moe_permute_backward and moe_combine_backward, moe_permute_premultiplied
+ * (the dispatch with each pair's row scaled by its gate), and
  * moe_dispatch_layout_noalloc (the layout without a caller workspace).
  *
  * Notation: N tokens, H hidden size, E experts, k = top_k choices per token,
@@ -235,6 +236,25 @@ MOE_API moe_status moe_dispatch_layout_noalloc(const moe_problem *problem,
 MOE_API moe_status moe_permute(const moe_problem *problem, const void *hidden_states,
                        const int32_t *row_src, const int32_t *pair_slot, void *out,
                        moe_stream_t stream);
+
+/* Permute with pre-multiplied gates: out[slot(t,j), :] = bf16(gates[t,j] *
+ * hidden_states[t, :]) -- one fp32 product and one rounding to nearest even
+ * per element -- and zeros in the rows no pair owns.  DeepSpeed v0.19.4
+ * function list: token representations pre-multiplied by their router
+ * scores before expert compute.  The combine of this variant is then the
+ * unweighted sum, moe_permute_backward's operation; its backward is
+ * moe_combine (gradient of hidden_states) and the gate gradient of
+ * moe_combine_backward with grad_y = hidden_states and expert_out = the
+ * rows' gradient.
+ *   hidden_states  bf16 [N, H], 16-byte aligned
+ *   row_src        int32 [rows] and pair_slot int32 [N, k] from the layout
+ *   gates          fp32 [N, k] (4-byte aligned)
+ *   out            bf16 [rows, H], 16-byte aligned, fully overwritten
+ * Requires H % 8 == 0; pair_slot entries outside [0, rows) are skipped. */
+MOE_API moe_status moe_permute_premultiplied(const moe_problem *problem,
+                                             const void *hidden_states, const int32_t *row_src,
+                                             const int32_t *pair_slot, const float *gates,
+                                             void *out, moe_stream_t stream);
 
 /* Permute with block FP8 quantisation (Mojo MAX ep_comm
  * BlockwiseFP8TokenFormat).  For each output row and each 1x128 block:

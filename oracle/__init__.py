@@ -95,6 +95,7 @@ def lib():
         L.orc_pack_fp6.argtypes = [vp, i64, vp]
         L.orc_combine.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp]
         L.orc_permute_backward.argtypes = [i32, i32, i32, i64, vp, vp, vp]
+        L.orc_permute_premultiplied.argtypes = [i32, i32, i32, i64, vp, vp, vp, vp]
         L.orc_exp.restype = f32
         L.orc_exp.argtypes = [f32]
         L.orc_silu.restype = f32
@@ -335,6 +336,24 @@ def combine_backward(grad_y_bits: np.ndarray, expert_out_bits: np.ndarray, gates
                                _p(pair_slot), _p(gx), _p(gw))
     o.check("orc_combine_backward")
     return gx, gw
+
+
+# ---------------------------------------------------------------- pre-multiplied gates
+def permute_premultiplied(hidden_bits: np.ndarray, gates: np.ndarray, pair_slot: np.ndarray,
+                          rows: int) -> np.ndarray:
+    """hidden: uint16 [N,H] bf16; gates f32 [N,k]; returns uint16 [rows,H]:
+    each pair's row is its token scaled by its gate (zeros elsewhere)."""
+    hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
+    gates = np.ascontiguousarray(gates, dtype=np.float32)
+    pair_slot = np.ascontiguousarray(pair_slot, dtype=np.int32)
+    N, k = pair_slot.shape
+    H = hidden_bits.shape[1]
+    o = _Outs()
+    out = o((rows, H), np.uint16)
+    lib().orc_permute_premultiplied(N, k, H, rows, _p(hidden_bits), _p(gates), _p(pair_slot),
+                                    _p(out))
+    o.check("orc_permute_premultiplied")
+    return out
 
 
 # ---------------------------------------------------------------- SwiGLU

@@ -582,6 +582,26 @@ void orc_combine_backward(int32_t N, int32_t k, int32_t H, int64_t rows,
     }
 }
 
+/* DeepSpeed "pre-multiply token representations by router scores before
+ * expert compute": every row starts as zeros; pair (t, j) with a row writes
+ * its token scaled by its gate, one fp32 product and one rounding to bf16
+ * per element. */
+void orc_permute_premultiplied(int32_t N, int32_t k, int32_t H, int64_t rows,
+                               const uint16_t *hidden, const float *gates,
+                               const int32_t *pair_slot, uint16_t *out) {
+  for (int64_t i = 0; i < rows * H; ++i) out[i] = 0;
+  for (int32_t t = 0; t < N; ++t)
+    for (int32_t j = 0; j < k; ++j) {
+      const int64_t p = (int64_t)t * k + j;
+      const int32_t s = pair_slot[p];
+      if (s < 0 || s >= rows) continue;
+      for (int32_t h = 0; h < H; ++h) {
+        const float x = orc_bf16_to_f32(hidden[(int64_t)t * H + h]);
+        out[(int64_t)s * H + h] = orc_bf16_from_f32(gates[p] * x);
+      }
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* SwiGLU + requantisation                                             */
 /* ------------------------------------------------------------------ */

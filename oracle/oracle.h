@@ -175,6 +175,18 @@ void orc_combine_backward(int32_t N, int32_t k, int32_t H, int64_t rows,
                           const float *gates, const int32_t *pair_slot,
                           uint16_t *grad_expert_out, float *grad_gates);
 
+/* ---- pre-multiplied gates ---------------------------------------------
+ * DeepSpeed v0.19.4 function list: token representations pre-multiplied by
+ * their router scores before expert compute.  The dispatch then writes each
+ * pair's row scaled by its gate,
+ *   out[slot(t,j)] = bf16(w[t,j] * hidden[t])  (fp32 product, one rounding),
+ * rows no pair owns are zero; the combine of this variant is the unweighted
+ * sum (orc_permute_backward's arithmetic) and its backward is the weighted
+ * combine (grad of hidden) and a dot product (grad of the gates).           */
+void orc_permute_premultiplied(int32_t N, int32_t k, int32_t H, int64_t rows,
+                               const uint16_t *hidden, const float *gates,
+                               const int32_t *pair_slot, uint16_t *out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -90,12 +90,14 @@ def test_payload_shape_rules(lib):
                   recv_capacity=20)
     assert _call(lib, "moe_permute", p, 5) == B.MOE_ERR_UNSUPPORTED_SHAPE       # H % 8
     assert _call(lib, "moe_combine", p, 5) == B.MOE_ERR_UNSUPPORTED_SHAPE
+    assert _call(lib, "moe_permute_premultiplied", p, 6) == B.MOE_ERR_UNSUPPORTED_SHAPE
     p.hidden = 96
     assert _call(lib, "moe_permute_quant_fp8", p, 6) == B.MOE_ERR_UNSUPPORTED_SHAPE  # H % 128
     p.hidden = 80
     assert _call(lib, "moe_permute_quant_nvfp4", p, 7) == B.MOE_ERR_UNSUPPORTED_SHAPE  # H % 32
     p.hidden = 128
-    for fn, n in (("moe_permute", 5), ("moe_permute_quant_fp8", 6),
+    for fn, n in (("moe_permute", 5), ("moe_permute_premultiplied", 6),
+                  ("moe_permute_quant_fp8", 6),
                   ("moe_permute_quant_nvfp4", 7), ("moe_combine", 5)):
         assert _call(lib, fn, p, n) == B.MOE_ERR_INVALID_ARG, fn      # null pointers
     assert lib.moe_permute(None, *([None] * 5)) == B.MOE_ERR_INVALID_ARG
@@ -138,6 +140,7 @@ ALIGNMENT_RULES = {
     "moe_dispatch_layout": ((), (4, 4, 4, 4, 4, 4, 1, 4, 16)),
     "moe_dispatch_layout_noalloc": ((), (4, 4, 4, 4, 4, 4, 1, 4)),
     "moe_permute": ((), (16, 4, 4, 16)),
+    "moe_permute_premultiplied": ((), (16, 4, 4, 4, 16)),
     "moe_permute_quant_fp8": ((), (16, 4, 4, 16, 4)),
     "moe_permute_quant_nvfp4": ((), (16, 4, 4, 4, 16, 2)),
     "moe_permute_quant_mxfp4": ((), (16, 4, 4, 16, 1)),

@@ -67,6 +67,10 @@ CASES = [
      "int64_t inner = (m % 32) * row_stride + ((m / 32) % 4) * 4 + c % atom_cols;",
      "int64_t inner = ((m / 32) % 4) * row_stride + (m % 32) * 4 + c % atom_cols;",
      "test_oracle_scale_layout.py"),
+    ("pre-multiplied dispatch: the next pair's gate",
+     "out[(int64_t)s * H + h] = orc_bf16_from_f32(gates[p] * x);",
+     "out[(int64_t)s * H + h] = orc_bf16_from_f32(gates[(p + 1) % ((int64_t)N * k)] * x);",
+     "test_oracle_premultiplied.py"),
     ("FP6 packing: codes in reverse bit order",
      "w |= (uint32_t)(codes[4 * g + i] & 0x3F) << (6 * i);",
      "w |= (uint32_t)(codes[4 * g + i] & 0x3F) << (18 - 6 * i);", "test_oracle_mx_fp6.py"),
