@@ -42,6 +42,22 @@ def test_matches_torch_product_and_cast(orc):
     assert not out[lay.row_src < 0].any()
 
 
+def test_hand_slots_unowned_rows_and_bounds(orc):
+    """Hand-made slots: rows 0, 4, 5 and 6 owned by no pair (zeros), a masked
+    pair, a slot equal to rows (skipped), and a valid-looking row of slots,
+    gates and tokens just past the end of each input, so that a read past
+    pair_slot, gates or hidden would change the output."""
+    H, rows = 16, 8
+    x_full = bf16_bits(np.arange(1, 4 * H + 1, dtype=np.float32).reshape(4, H))
+    g_full = np.array([[0.5, 2.0], [4.0, 0.25], [1.5, 3.0], [8.0, 8.0]], np.float32)
+    s_full = np.array([[1, 2], [-1, 7], [3, rows], [0, 0]], np.int32)
+    out = orc.permute_premultiplied(x_full[:3], g_full[:3], s_full[:3], rows)
+    want = np.zeros((rows, H), np.uint16)
+    for t, j in ((0, 0), (0, 1), (1, 1), (2, 0)):
+        want[s_full[t, j]] = bf16_bits(g_full[t, j] * f32(x_full[t]))
+    assert np.array_equal(out, want)
+
+
 def test_unit_gates_is_the_plain_dispatch(orc):
     w, lay, C = _layout(orc, "tiny", n_tokens=None, extra=5)
     out = orc.permute_premultiplied(w.hidden, np.ones_like(w.gates), lay.pair_slot, C)
