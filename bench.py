@@ -39,6 +39,7 @@ if ROOT not in sys.path:
 METRIC = "dispatch+combine tokens/s and HBM GB/s (% of peak) at N=8192 H=7168 E=256 k=8"
 WORKLOAD = "fp8_metric"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, nominal (DGX figure)
 
 # dram bytes (read + write) per launch from one ncu --set full capture on the
 # metric workload (summaries under profiles/), keyed by kernel; valid only
@@ -569,6 +570,7 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
             "dtype": "fp32", "data": "synthetic", "config": workload_config(w),
             "hbm_gbs": step_bytes / (ms * 1e-3) / 1e9,
             "hbm_frac_of_peak": step_bytes / (ms * 1e-3) / 1e9 / peak,
+            "hbm_frac_of_nominal": step_bytes / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
             "phases_us": {p: round(1e3 * v, 2) for p, v in phase_ms.items()},
             "phases_timing": (f"{n_phase} further steps with an event between kernels (an event "
                               f"ends the programmatic overlap of consecutive kernels); their "
