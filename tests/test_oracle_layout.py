@@ -160,6 +160,13 @@ def test_duplicate_check_reaches_every_token(orc, where):
     assert lay.status == orc.STATUS_DUP_ID
 
 
+def test_duplicate_check_with_fewer_tokens_than_choices(orc):
+    """One token, three choices, the duplicate in the last two."""
+    ids = np.array([[2, 1, 1]], np.int32)
+    lay = orc.layout(ids, 4, 2, 8, recv_capacity=3, flags=orc.FLAG_CHECK_DUPLICATES)
+    assert lay.status == orc.STATUS_DUP_ID
+
+
 def test_duplicate_check_ignores_masked_and_out_of_range_ids(orc):
     """Reading: the duplicate check concerns experts a token is routed to, so
     repeated -1 (masked) entries are not duplicates, and repeated out-of-range
