@@ -117,3 +117,22 @@ def test_pins_catch_planted_mistakes(tmp_path):
         if old is not None and rc == 0:
             bad.append(f"not caught by {f}: {what}")
     assert not bad, "\n".join(bad)
+
+
+def test_output_guard_reports_overruns_and_keeps_poison(orc):
+    """The poisoned, guarded output buffers themselves: a call that writes
+    past the end of an output (here 8 bf16 values into room for 4, i.e.
+    into the 64-byte guard that follows it) raises, and an element the call
+    does not write keeps the poison byte."""
+    import numpy as np
+    x = np.arange(8, dtype=np.float32)
+    o = orc._Outs()
+    out = o(4, np.uint16)
+    orc.lib().orc_bf16_from_f32_n(orc._p(x), orc._p(out), 8)
+    with pytest.raises(RuntimeError, match="past the end"):
+        o.check("overrun")
+    o = orc._Outs()
+    out = o(4, np.uint16)
+    orc.lib().orc_bf16_from_f32_n(orc._p(x), orc._p(out), 3)
+    o.check("short write")
+    assert int(out[3]) == orc._POISON * 0x101 and int(out[2]) == 0x4000
