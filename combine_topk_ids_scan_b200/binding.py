@@ -5,6 +5,12 @@ arguments: torch tensors become device pointers, the current torch CUDA
 stream becomes the launch stream.  Every step of the computation runs in the
 library's CUDA kernels; there is no fallback of any kind -- if the library
 cannot be loaded, the first call raises.
+
+The C ABI takes plain pointers and cannot see buffer sizes, so before a call
+each function checks that every tensor it passes holds at least the bytes
+the problem needs (moe_dc.h gives each array's shape) and raises
+MoeError(MOE_ERR_INVALID_ARG) otherwise: a short buffer becomes a Python
+error instead of an out-of-bounds device access.
 """
 from __future__ import annotations
 
@@ -50,9 +56,17 @@ MOE_GATE_UP_SPLIT, MOE_GATE_UP_INTERLEAVED = 0, 1
 MOE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
+_STATUS_TEXT = {MOE_OK: "ok", MOE_ERR_INVALID_ARG: "invalid argument",
+                MOE_ERR_UNSUPPORTED_SHAPE: "unsupported shape", MOE_ERR_CUDA: "CUDA error"}
+
+
 class MoeError(RuntimeError):
     def __init__(self, code: int, where: str):
-        super().__init__(f"{where}: {status_string(code)} (moe_status {code})")
+        try:
+            text = status_string(code)
+        except Exception:            # the library's own text when it can be loaded
+            text = _STATUS_TEXT.get(code, "unknown status")
+        super().__init__(f"{where}: {text} (moe_status {code})")
         self.code = code
 
 
@@ -151,6 +165,30 @@ def _ptr(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _sizes(prob: Problem):
+    """(N, H, E, k, S, P, rows) of a problem, negatives clamped to 0 (an
+    invalid problem is then rejected by the library itself)."""
+    N, H, E, k, S = (max(0, int(v)) for v in (prob.num_tokens, prob.hidden, prob.num_experts,
+                                                prob.top_k, prob.num_segments))
+    rows = E * max(0, prob.expert_capacity) if prob.expert_capacity > 0 \
+        else max(0, int(prob.recv_capacity))
+    return N, H, E, k, S, N * k, rows
+
+
+def _require(where: str, **need) -> None:
+    """need: argument name -> (tensor or None, bytes the problem needs).
+    Raises MoeError(MOE_ERR_INVALID_ARG) for a tensor holding fewer bytes;
+    None (the library checks which pointers may be null) and zero-byte needs
+    are skipped."""
+    for name, (t, nbytes) in need.items():
+        if t is None or nbytes <= 0:
+            continue
+        have = t.numel() * t.element_size()
+        if have < nbytes:
+            raise MoeError(MOE_ERR_INVALID_ARG,
+                           f"{where}: {name} holds {have} bytes, the problem needs {nbytes}")
+
+
 def _stream(stream: torch.cuda.Stream | None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
@@ -169,8 +207,21 @@ def moe_workspace_bytes(prob: Problem) -> int:
     return int(load().moe_workspace_bytes(ctypes.byref(prob.c())))
 
 
+def _layout_need(prob: Problem, topk_ids, expert_counts, expert_offsets, meta, row_src,
+                 pair_slot, drop_mask, status) -> dict:
+    N, H, E, k, S, P, rows = _sizes(prob)
+    return dict(topk_ids=(topk_ids, 4 * P), expert_counts=(expert_counts, 4 * E),
+                expert_offsets=(expert_offsets, 4 * (E + 1)), meta=(meta, 16 * S),
+                row_src=(row_src, 4 * rows), pair_slot=(pair_slot, 4 * P),
+                drop_mask=(drop_mask, P), status=(status, 4))
+
+
 def moe_dispatch_layout(prob: Problem, topk_ids, expert_counts, expert_offsets, meta, row_src,
                         pair_slot, drop_mask, status, workspace, stream=None) -> None:
+    _require("moe_dispatch_layout",
+             **_layout_need(prob, topk_ids, expert_counts, expert_offsets, meta, row_src,
+                            pair_slot, drop_mask, status),
+             workspace=(workspace, moe_workspace_bytes(prob)))
     c = prob.c()
     _check(load().moe_dispatch_layout(ctypes.byref(c), _ptr(topk_ids), _ptr(expert_counts),
                                       _ptr(expert_offsets), _ptr(meta), _ptr(row_src),
@@ -183,6 +234,9 @@ def moe_dispatch_layout_noalloc(prob: Problem, topk_ids, expert_counts, expert_o
                                 row_src, pair_slot, drop_mask, status, stream=None) -> None:
     """The layout without a caller workspace (for callers that cannot
     allocate); see moe_dispatch_layout_noalloc in moe_dc.h for its limits."""
+    _require("moe_dispatch_layout_noalloc",
+             **_layout_need(prob, topk_ids, expert_counts, expert_offsets, meta, row_src,
+                            pair_slot, drop_mask, status))
     c = prob.c()
     _check(load().moe_dispatch_layout_noalloc(ctypes.byref(c), _ptr(topk_ids),
                                               _ptr(expert_counts), _ptr(expert_offsets),
@@ -191,7 +245,16 @@ def moe_dispatch_layout_noalloc(prob: Problem, topk_ids, expert_counts, expert_o
            "moe_dispatch_layout_noalloc")
 
 
+def _permute_need(prob: Problem, hidden_states, row_src, pair_slot) -> dict:
+    N, H, E, k, S, P, rows = _sizes(prob)
+    return dict(hidden_states=(hidden_states, 2 * N * H), row_src=(row_src, 4 * rows),
+                pair_slot=(pair_slot, 4 * P))
+
+
 def moe_permute(prob: Problem, hidden_states, row_src, pair_slot, out, stream=None) -> None:
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_permute", **_permute_need(prob, hidden_states, row_src, pair_slot),
+             out=(out, 2 * rows * H))
     c = prob.c()
     _check(load().moe_permute(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
                               _ptr(pair_slot), _ptr(out), _stream(stream)), "moe_permute")
@@ -201,6 +264,10 @@ def moe_permute_premultiplied(prob: Problem, hidden_states, row_src, pair_slot, 
                               stream=None) -> None:
     """Dispatch with pre-multiplied gates: each pair's row is its token
     scaled by its gate (see moe_permute_premultiplied in moe_dc.h)."""
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_permute_premultiplied",
+             **_permute_need(prob, hidden_states, row_src, pair_slot), gates=(gates, 4 * P),
+             out=(out, 2 * rows * H))
     c = prob.c()
     _check(load().moe_permute_premultiplied(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
                                             _ptr(pair_slot), _ptr(gates), _ptr(out),
@@ -209,14 +276,27 @@ def moe_permute_premultiplied(prob: Problem, hidden_states, row_src, pair_slot, 
 
 def moe_permute_quant_fp8(prob: Problem, hidden_states, row_src, pair_slot, out_e4m3, scales,
                           stream=None) -> None:
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_permute_quant_fp8", **_permute_need(prob, hidden_states, row_src, pair_slot),
+             out_e4m3=(out_e4m3, rows * H), scales=(scales, 4 * rows * (H // 128)))
     c = prob.c()
     _check(load().moe_permute_quant_fp8(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
                                         _ptr(pair_slot), _ptr(out_e4m3), _ptr(scales),
                                         _stream(stream)), "moe_permute_quant_fp8")
 
 
+def _fp4_scale_bytes(prob: Problem, rows: int, H: int, block: int) -> int:
+    if prob.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES:
+        return nvfp4_swizzled_scale_bytes(rows, H, block) if rows > 0 else 0
+    return rows * (H // block)
+
+
 def moe_permute_quant_nvfp4(prob: Problem, hidden_states, row_src, pair_slot, global_scale,
                             out_e2m1, scales_e4m3, stream=None) -> None:
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_permute_quant_nvfp4", **_permute_need(prob, hidden_states, row_src, pair_slot),
+             global_scale=(global_scale, 4 if rows > 0 else 0), out_e2m1=(out_e2m1, rows * H // 2),
+             scales_e4m3=(scales_e4m3, _fp4_scale_bytes(prob, rows, H, 16)))
     c = prob.c()
     _check(load().moe_permute_quant_nvfp4(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
                                           _ptr(pair_slot), _ptr(global_scale), _ptr(out_e2m1),
@@ -226,6 +306,10 @@ def moe_permute_quant_nvfp4(prob: Problem, hidden_states, row_src, pair_slot, gl
 
 def moe_permute_quant_mxfp4(prob: Problem, hidden_states, row_src, pair_slot, out_e2m1,
                             scales_e8m0, stream=None) -> None:
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_permute_quant_mxfp4", **_permute_need(prob, hidden_states, row_src, pair_slot),
+             out_e2m1=(out_e2m1, rows * H // 2),
+             scales_e8m0=(scales_e8m0, _fp4_scale_bytes(prob, rows, H, 32)))
     c = prob.c()
     _check(load().moe_permute_quant_mxfp4(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
                                           _ptr(pair_slot), _ptr(out_e2m1), _ptr(scales_e8m0),
@@ -234,6 +318,9 @@ def moe_permute_quant_mxfp4(prob: Problem, hidden_states, row_src, pair_slot, ou
 
 
 def moe_combine(prob: Problem, expert_out, gates, pair_slot, out, stream=None) -> None:
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_combine", expert_out=(expert_out, 2 * rows * H if N > 0 else 0),
+             gates=(gates, 4 * P), pair_slot=(pair_slot, 4 * P), out=(out, 2 * N * H))
     c = prob.c()
     _check(load().moe_combine(ctypes.byref(c), _ptr(expert_out), _ptr(gates), _ptr(pair_slot),
                               _ptr(out), _stream(stream)), "moe_combine")
@@ -246,6 +333,9 @@ def nvfp4_swizzled_scale_bytes(rows: int, hidden: int, block: int = 16) -> int:
 
 
 def moe_permute_backward(prob: Problem, grad_out, pair_slot, grad_hidden, stream=None) -> None:
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_permute_backward", grad_out=(grad_out, 2 * rows * H if N > 0 else 0),
+             pair_slot=(pair_slot, 4 * P), grad_hidden=(grad_hidden, 2 * N * H))
     c = prob.c()
     _check(load().moe_permute_backward(ctypes.byref(c), _ptr(grad_out), _ptr(pair_slot),
                                        _ptr(grad_hidden), _stream(stream)),
@@ -254,6 +344,11 @@ def moe_permute_backward(prob: Problem, grad_out, pair_slot, grad_hidden, stream
 
 def moe_combine_backward(prob: Problem, grad_y, expert_out, gates, pair_slot, row_src,
                          grad_expert_out, grad_gates, stream=None) -> None:
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_combine_backward", grad_y=(grad_y, 2 * N * H),
+             expert_out=(expert_out, 2 * rows * H), gates=(gates, 4 * P),
+             pair_slot=(pair_slot, 4 * P), row_src=(row_src, 4 * rows),
+             grad_expert_out=(grad_expert_out, 2 * rows * H), grad_gates=(grad_gates, 4 * P))
     c = prob.c()
     _check(load().moe_combine_backward(ctypes.byref(c), _ptr(grad_y), _ptr(expert_out),
                                        _ptr(gates), _ptr(pair_slot), _ptr(row_src),
@@ -261,8 +356,22 @@ def moe_combine_backward(prob: Problem, grad_y, expert_out, gates, pair_slot, ro
                                        _stream(stream)), "moe_combine_backward")
 
 
+_SWIGLU_CODE_BYTES = {MOE_QUANT_NVFP4: (1, 2), MOE_QUANT_MXFP8: (1, 1),
+                      MOE_QUANT_MXFP4: (1, 2), MOE_QUANT_BF16: (2, 1),
+                      MOE_QUANT_MXFP6_E2M3: (3, 4), MOE_QUANT_MXFP6_E3M2: (3, 4)}
+
+
 def moe_swiglu_quant(prob: Problem, intermediate: int, fmt: int, gate_up_layout: int, gate_up,
                      row_src, global_scale, codes, scales, stream=None) -> None:
+    N, H, E, k, S, P, rows = _sizes(prob)
+    I = max(0, int(intermediate))
+    if fmt in _SWIGLU_CODE_BYTES:         # an unknown format is rejected by the library
+        num, den = _SWIGLU_CODE_BYTES[fmt]
+        scale_bytes = 0 if fmt == MOE_QUANT_BF16 else I // (16 if fmt == MOE_QUANT_NVFP4 else 32)
+        _require("moe_swiglu_quant", gate_up=(gate_up, 4 * rows * I),
+                 row_src=(row_src, 4 * rows), codes=(codes, rows * I * num // den),
+                 scales=(scales, rows * scale_bytes),
+                 global_scale=(global_scale, 4 if fmt == MOE_QUANT_NVFP4 and rows > 0 else 0))
     c = prob.c()
     _check(load().moe_swiglu_quant(ctypes.byref(c), intermediate, fmt, gate_up_layout,
                                    _ptr(gate_up), _ptr(row_src), _ptr(global_scale), _ptr(codes),

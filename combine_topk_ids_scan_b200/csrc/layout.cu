@@ -396,12 +396,19 @@ __device__ uint32_t duplicate_bits(const int32_t *__restrict__ ids, int64_t t0, 
 
 // The last block to arrive publishes the status word and returns the
 // workspace (tile states, totals, control words) to zero.  Called by all
-// threads of every block, last thing in the kernel.
+// threads of every block, last thing in the kernel.  Every block arrives
+// after all of its own workspace stores, so the last block runs after every
+// store of the launch.  n_states tile states are cleared here always, and
+// n_states_on_timeout when a bounded wait gave up: in the one-launch kernel
+// a tile whose look-back timed out may publish its state after the other
+// blocks, whose grid-wide wait also timed out, cleared the states.
 template <int THREADS>
 __device__ void finish_and_clean(uint32_t bits, uint32_t *s_status, uint32_t *ctrl,
-                                 int32_t *totals, uint64_t *tiles, int64_t n_states, int32_t E,
-                                 uint32_t *status_out, uint32_t n_blocks) {
+                                 int32_t *totals, uint64_t *tiles, int64_t n_states,
+                                 int64_t n_states_on_timeout, int32_t E, uint32_t *status_out,
+                                 uint32_t n_blocks) {
   __shared__ bool s_last;
+  __shared__ uint32_t s_final;
   if (bits) atomicOr(s_status, bits);
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -412,10 +419,14 @@ __device__ void finish_and_clean(uint32_t bits, uint32_t *s_status, uint32_t *ct
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int64_t i = threadIdx.x; i < n_states; i += THREADS) tiles[i] = 0;
+  if (threadIdx.x == 0) s_final = atomicExch(&ctrl[kCtrlStatus], 0u);
+  __syncthreads();
+  const int64_t n = (s_final & MOE_STATUS_TIMEOUT) ? max(n_states, n_states_on_timeout)
+                                                   : n_states;
+  for (int64_t i = threadIdx.x; i < n; i += THREADS) tiles[i] = 0;
   for (int e = threadIdx.x; e < E; e += THREADS) totals[e] = 0;
   if (threadIdx.x == 0) {
-    *status_out = atomicExch(&ctrl[kCtrlStatus], 0u);
+    *status_out = s_final;
     ctrl[kCtrlTicket] = 0;
     ctrl[kCtrlTilesDone] = 0;
     atomicExch(&ctrl[kCtrlDone], 0u);
@@ -468,10 +479,11 @@ __device__ void scan_step(const LayoutArgs &a, uint8_t *smem, uint32_t *s_status
 
 // Emit step: ranks -> rows for the pairs [gtid, P) in steps of gstride, the
 // padding rows, counts / offsets / meta (block 0), the duplicate check, then
-// the last block cleans up.  n_states: tile states the last block clears.
+// the last block cleans up.  n_states_on_timeout: tile states the last block
+// clears when a bounded wait gave up.
 template <int THREADS>
 __device__ void emit_step(const LayoutArgs &a, int64_t gtid, int64_t gstride,
-                          uint32_t *s_status, int64_t n_states) {
+                          uint32_t *s_status, int64_t n_states_on_timeout) {
   __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_kept[MOE_MAX_EXPERTS];
   expert_offsets_from_totals<THREADS>(a.totals, a.num_tiles > 0, a.E, a.Ce, a.pad, s_off,
@@ -492,8 +504,8 @@ __device__ void emit_step(const LayoutArgs &a, int64_t gtid, int64_t gstride,
                        a.row_src, blockIdx.x == 0, a.expert_counts, a.expert_offsets, a.meta);
   if (a.flags & MOE_FLAG_CHECK_DUPLICATES)
     bits |= duplicate_bits(a.ids, gtid, a.N, gstride, a.k, a.E);
-  finish_and_clean<THREADS>(bits, s_status, a.ctrl, a.totals, a.tiles, n_states, a.E,
-                            a.status_out, (uint32_t)gridDim.x);
+  finish_and_clean<THREADS>(bits, s_status, a.ctrl, a.totals, a.tiles, 0, n_states_on_timeout,
+                            a.E, a.status_out, (uint32_t)gridDim.x);
 }
 
 // One cooperative launch: scan (first T CTAs), grid-wide wait, emit (all).
@@ -518,9 +530,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) layout_fused_kernel(LayoutArg
   __syncthreads();
   const int64_t gtid = (int64_t)blockIdx.x * kScanThreads + threadIdx.x;
   const int64_t gstride = (int64_t)gridDim.x * kScanThreads;
-  // every look-back has finished: the tile states can be cleared by everyone
+  // every look-back has finished (unless a wait timed out, see
+  // finish_and_clean): the tile states can be cleared by everyone
   for (int64_t i = gtid; i < (int64_t)a.num_tiles * a.E; i += gstride) a.tiles[i] = 0;
-  emit_step<kScanThreads>(a, gtid, gstride, &s_status, 0);
+  emit_step<kScanThreads>(a, gtid, gstride, &s_status, (int64_t)a.num_tiles * a.E);
 }
 
 __global__ void __launch_bounds__(kScanThreads, 1) layout_count_scan_kernel(LayoutArgs a) {

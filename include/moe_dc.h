@@ -213,7 +213,10 @@ MOE_API moe_status moe_dispatch_layout(const moe_problem *problem, const int32_t
  *     moe_dispatch_layout with a workspace for such problems.
  *   - The first call on a device looks up the array's device address on that
  *     device (it must be the current device); make that first call before any
- *     stream capture.
+ *     stream capture.  The address is kept for the life of the process, so
+ *     do not call this entry point on a device after cudaDeviceReset() of
+ *     that device (the reset unloads the library's device code and the kept
+ *     address no longer names the array).
  *   - Every call shares the one array and finds what the previous call left
  *     in it; each call zero-fills the part it uses on its own stream before
  *     launching.  Calls that overlap on the GPU (other streams, other host

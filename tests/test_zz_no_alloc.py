@@ -44,20 +44,29 @@ def _outputs(buf, w):
     }
 
 
+def _poisoned(prob):
+    # poison the outputs so a skipped write cannot pass
+    buf = B.Buffers(prob, quant=False)
+    for t in (buf.expert_counts, buf.expert_offsets, buf.meta, buf.row_src, buf.pair_slot):
+        t.fill_(-7)
+    buf.drop_mask.fill_(9)
+    buf.status.fill_(-1)
+    return buf
+
+
+def _noalloc(prob, ids, buf):
+    B.moe_dispatch_layout_noalloc(prob, ids, buf.expert_counts, buf.expert_offsets, buf.meta,
+                                  buf.row_src, buf.pair_slot, buf.drop_mask, buf.status)
+
+
 def _run_both(w, flags=0):
     prob = _problem(w, flags)
     ids = torch.from_numpy(w.ids).cuda()
-    ref = B.Buffers(prob, quant=False)
+    ref = _poisoned(prob)
     B.moe_dispatch_layout(prob, ids, ref.expert_counts, ref.expert_offsets, ref.meta,
                           ref.row_src, ref.pair_slot, ref.drop_mask, ref.status, ref.workspace)
-    got = B.Buffers(prob, quant=False)
-    # poison the outputs so a skipped write cannot pass
-    for t in (got.expert_counts, got.expert_offsets, got.meta, got.row_src, got.pair_slot):
-        t.fill_(-7)
-    got.drop_mask.fill_(9)
-    got.status.fill_(-1)
-    B.moe_dispatch_layout_noalloc(prob, ids, got.expert_counts, got.expert_offsets, got.meta,
-                                  got.row_src, got.pair_slot, got.drop_mask, got.status)
+    got = _poisoned(prob)
+    _noalloc(prob, ids, got)
     torch.cuda.synchronize()
     return _outputs(ref, w), _outputs(got, w)
 
@@ -74,12 +83,36 @@ def test_noalloc_layout_matches_workspace_layout_twice_in_a_row():
         assert int(got["status"][0]) == 0
 
 
+def test_noalloc_after_a_call_that_timed_out():
+    """A call whose bounded waits run out (the test hook withholds the first
+    scan tile's counts) still leaves the shared scratch usable: the next
+    call matches the workspace path exactly."""
+    from combine_topk_ids_scan_b200.inputs import Workload
+    rng = np.random.default_rng(41)
+    N, k, E = 3000, 4, 16                     # 12000 pairs: 3 scan tiles
+    ids = np.argsort(rng.random((N, E)), axis=1)[:, :k].astype(np.int32)
+    w = Workload(name="stall", N=N, H=64, E=E, k=k, S=4, recv_capacity=N * k,
+                 expert_capacity=0, ids=ids, gates=np.ones((N, k), np.float32),
+                 hidden=np.zeros((N, 64), np.uint16), expert_out=None, global_scale=1.0, seed=0)
+    prob = _problem(w, flags=B.MOE_FLAG_TEST_STALL_SCAN)
+    buf = _poisoned(prob)
+    _noalloc(prob, torch.from_numpy(ids).cuda(), buf)
+    torch.cuda.synchronize()
+    assert int(buf.status.cpu().numpy().view(np.uint32)[0]) & B.MOE_STATUS_TIMEOUT
+    for _ in range(2):
+        ref, got = _run_both(w)
+        for key in ref:
+            assert np.array_equal(ref[key], got[key]), key
+        assert int(got["status"][0]) == 0
+
+
 def test_noalloc_rejects_problems_beyond_the_scratch():
     # 8M pairs at E = 256 need more than 1 MiB of scan state
     prob = B.Problem(num_tokens=1 << 20, hidden=64, num_experts=256, top_k=8,
                      num_segments=8, recv_capacity=8 << 20)
     assert B.moe_workspace_bytes(prob) > B.MOE_NOALLOC_SCRATCH_BYTES
-    d = torch.zeros(16, dtype=torch.int32, device="cuda")
+    buf = B.Buffers(prob, quant=False)
+    ids = torch.zeros((1 << 20, 8), dtype=torch.int32, device="cuda")
     with pytest.raises(B.MoeError) as e:
-        B.moe_dispatch_layout_noalloc(prob, d, d, d, d, d, d, None, d)
+        _noalloc(prob, ids, buf)
     assert e.value.code == B.MOE_ERR_UNSUPPORTED_SHAPE
