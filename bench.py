@@ -188,10 +188,16 @@ def max_over_ranks(values, device, world: int):
 
 
 # ------------------------------------------------------------------ oracle
-def oracle_tokens_per_s(w, n_tokens: int, start: int = 0) -> tuple[float, float]:
-    """Time the CPU oracle (as it stands, single thread) on the sub-batch of
-    tokens [start, start+n): layout, the three permutes and the combine.
-    Returns (tokens/s, seconds)."""
+def oracle_tokens_per_s(w, n_tokens: int, start: int = 0,
+                        threads: int = 1) -> tuple[float, float]:
+    """Time the CPU oracle (as it stands) on the sub-batch of tokens
+    [start, start+n): its own layout (packed with recv_capacity = n*k, or the
+    workload's expert capacity), the permutes the shape allows and the
+    combine.  threads > 1 splits the permutes' rows and the combine's tokens
+    over a thread pool (each oracle call is single-threaded C and releases
+    the GIL; the layout stays one call).  Returns (tokens/s, seconds)."""
+    import concurrent.futures as cf
+
     import oracle
     oracle.build()
     n = min(n_tokens, w.N)
@@ -199,15 +205,29 @@ def oracle_tokens_per_s(w, n_tokens: int, start: int = 0) -> tuple[float, float]
     ids = np.ascontiguousarray(w.ids[idx])
     hidden = np.ascontiguousarray(w.hidden[idx])
     gates = np.ascontiguousarray(w.gates[idx])
-    C = n * w.k
-    X = np.ascontiguousarray(w.expert_out[:C]) if w.expert_out is not None else None
+    if w.expert_capacity > 0:
+        lay_kw, rows = dict(expert_capacity=w.expert_capacity), w.E * w.expert_capacity
+    else:
+        lay_kw, rows = dict(recv_capacity=n * w.k), n * w.k
+    X = np.ascontiguousarray(w.expert_out[:rows]) if w.expert_out is not None else None
+
+    def split(fn, m, *arrays):
+        if threads <= 1:
+            return fn(*arrays)
+        step = max(1, -(-m // threads))
+        with cf.ThreadPoolExecutor(threads) as ex:
+            list(ex.map(lambda i: fn(*[a[i:i + step] for a in arrays]), range(0, m, step)))
+
     t0 = time.perf_counter()
-    lay = oracle.layout(ids, w.E, w.S, w.H, recv_capacity=C)
-    oracle.permute_bf16(hidden, lay.row_src)
-    oracle.permute_fp8(hidden, lay.row_src)
-    oracle.permute_nvfp4(hidden, lay.row_src, w.global_scale)
+    lay = oracle.layout(ids, w.E, w.S, w.H, **lay_kw)
+    rs = lay.row_src
+    split(lambda r: oracle.permute_bf16(hidden, r), rows, rs)
+    if w.H % 128 == 0:
+        split(lambda r: oracle.permute_fp8(hidden, r), rows, rs)
+    if w.H % 32 == 0:
+        split(lambda r: oracle.permute_nvfp4(hidden, r, w.global_scale), rows, rs)
     if X is not None:
-        oracle.combine(X, gates, lay.pair_slot)
+        split(lambda g, ps: oracle.combine(X, g, ps), n, gates, lay.pair_slot)
     dt = time.perf_counter() - t0
     return n / dt, dt
 
@@ -236,12 +256,108 @@ def run_reference(args, rank: int, world: int) -> int:
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
         "data": "synthetic", "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "box_cores": os.cpu_count()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# every workload of the benchmark set and the oracle sample timed beside it
+# (tokens; about a second or two of single-threaded oracle work each)
+CONFIG_SET = ("tiny", "mid_zipf", "fp8_metric", "nvfp4_hot", "decode_capacity",
+              "balanced_static")
+CPU_SAMPLE_TOKENS = {"tiny": 512, "mid_zipf": 512, "fp8_metric": 1024, "nvfp4_hot": 1024,
+                     "decode_capacity": 128, "balanced_static": 1024}
+
+
+def measure_workload(B, torch, w, dev, stream, flush_l2, n_steps: int, peak: float) -> dict:
+    """Times one workload of the benchmark set on this GPU (inputs resident,
+    L2 flushed before every step, outside the events): the whole step
+    (layout, the permutes the shape allows, combine) between two events,
+    the dispatch bf16 + combine trio between two events, and each kernel
+    with an event between kernels.  Returns a JSON-ready dict."""
+    prob = B.Problem(num_tokens=w.N, hidden=w.H, num_experts=w.E, top_k=w.k,
+                     num_segments=w.S, recv_capacity=w.recv_capacity,
+                     expert_capacity=w.expert_capacity)
+    buf = B.Buffers(prob, device=dev)
+    d_ids = torch.from_numpy(w.ids).to(dev)
+    d_hidden = torch.from_numpy(w.hidden.view(np.int16)).to(dev).view(torch.bfloat16)
+    d_gates = torch.from_numpy(w.gates).to(dev)
+    d_x = torch.from_numpy(w.expert_out.view(np.int16)).to(dev).view(torch.bfloat16)
+    d_gs = torch.tensor([w.global_scale], dtype=torch.float32, device=dev)
+    d_y = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
+    calls = {"layout": lambda: B.layout(prob, d_ids, buf),
+             "permute_bf16": lambda: B.moe_permute(prob, d_hidden, buf.row_src, buf.pair_slot,
+                                                   buf.out)}
+    if w.H % 128 == 0:
+        calls["permute_fp8"] = lambda: B.moe_permute_quant_fp8(
+            prob, d_hidden, buf.row_src, buf.pair_slot, buf.out_fp8, buf.scales_fp8)
+    if w.H % 32 == 0:
+        calls["permute_nvfp4"] = lambda: B.moe_permute_quant_nvfp4(
+            prob, d_hidden, buf.row_src, buf.pair_slot, d_gs, buf.out_fp4, buf.scales_fp4)
+    calls["combine"] = lambda: B.moe_combine(prob, d_x, d_gates, buf.pair_slot, d_y)
+    names = list(calls)
+    trio = ["layout", "permute_bf16", "combine"]
+
+    def timed(seq, per_kernel):
+        for _ in range(3):
+            flush_l2()
+            for nm in seq:
+                calls[nm]()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(seq) + 1)]
+              for _ in range(n_steps)]
+        torch.cuda.synchronize(dev)
+        for i in range(n_steps):
+            flush_l2()
+            ev[i][0].record(stream)
+            for j, nm in enumerate(seq):
+                calls[nm]()
+                if per_kernel or j == len(seq) - 1:
+                    ev[i][j + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        if per_kernel:
+            return [1e3 * sum(e[j].elapsed_time(e[j + 1]) for e in ev) / n_steps
+                    for j in range(len(seq))]
+        return 1e3 * sum(e[0].elapsed_time(e[-1]) for e in ev) / n_steps
+
+    step_us = timed(names, False)
+    trio_us = timed(trio, False)
+    per = dict(zip(names, timed(names, True)))
+    status = int(buf.status.cpu().numpy().view(np.uint32)[0])
+    total_rows = int(buf.expert_counts.sum().item())
+    nbytes = algorithmic_bytes(w, total_rows)
+    step_bytes = sum(nbytes[nm] for nm in names)
+    tiles = (w.P + 4095) // 4096
+    out = {
+        "workload": workload_config(w)["workload"],
+        "layout_mode": (f"capacity [E, {w.expert_capacity}, H], drops in (token, k) order"
+                        if w.expert_capacity > 0 else "packed, dropless"),
+        "routed_rows": total_rows, "steps": n_steps,
+        "step": " + ".join(names),
+        "step_us": round(step_us, 2), "step_tokens_per_s": w.N / (step_us * 1e-6),
+        "step_gbs": round(step_bytes / (step_us * 1e-6) / 1e9, 1),
+        "step_frac_of_peak": round(step_bytes / (step_us * 1e-6) / 1e9 / peak, 3),
+        "dispatch_bf16_plus_combine_us": round(trio_us, 2),
+        "dispatch_bf16_plus_combine_tokens_per_s": w.N / (trio_us * 1e-6),
+        "phases_us": {nm: round(v, 2) for nm, v in per.items()},
+        "phases_gbs": {nm: round(nbytes[nm] / (per[nm] * 1e-6) / 1e9, 1) for nm in names},
+        "phases_frac_of_peak": {nm: round(nbytes[nm] / (per[nm] * 1e-6) / 1e9 / peak, 3)
+                                for nm in names},
+        "algorithmic_bytes": {nm: nbytes[nm] for nm in names},
+        "launches_per_step": layout_launches(w.P) + len(names) - 1,
+        "layout_status": status,
+    }
+    del buf, d_ids, d_hidden, d_gates, d_x, d_gs, d_y
+    return out
+
+
+def layout_launches(P: int) -> int:
+    """Kernel launches of one moe_dispatch_layout call: one up to 128 scan
+    tiles of 4096 pairs (cooperative one-launch kernel), else a scan and an
+    emit launch."""
+    return 1 if (P + 4095) // 4096 <= 128 else 2
 
 
 def workload_config(w) -> dict:
@@ -329,10 +445,8 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
         B.moe_combine(prob, d_x, d_gates, buf.pair_slot, d_y)
         mark(5)
 
-    # the layout is one cooperative launch up to 128 scan tiles of 4096 pairs,
-    # else a scan and an emit launch; then three permutes and the combine
-    tiles = (w.P + 4095) // 4096
-    launches_per_step = (1 if tiles <= 128 else 2) + 4
+    # the layout's launches, then three permutes and the combine
+    launches_per_step = layout_launches(w.P) + 4
     for _ in range(args.warmup):
         flush_l2()
         step()
@@ -478,6 +592,29 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
             f3["swiglu"][name + "_gbs"] = round(nbytes / (us * 1e-6) / 1e9, 1)
             del codes, scales
 
+    # ---- every workload of the benchmark set, each timed alone beside the
+    # oracle on a bounded sample of it (one GPU only: a per-rank sweep would
+    # only repeat it)
+    configs = None
+    if args.configs and world == 1:
+        peak_c, _ = _peaks()
+        configs = {}
+        n_cfg = max(20, min(args.steps, 100))
+        for name in CONFIG_SET:
+            wc = w if name == WORKLOAD else make_workload(name)
+            r = measure_workload(B, torch, wc, dev, stream, flush_l2, n_cfg, peak_c)
+            if not args.no_cpu_baseline:
+                n_cpu = min(CPU_SAMPLE_TOKENS[name], wc.N)
+                tps, dt = oracle_tokens_per_s(wc, n_cpu)
+                r["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": 1,
+                                     "kind": "oracle",
+                                     "sample": f"first {n_cpu} tokens, own layout; "
+                                               f"{dt:.2f} s single-threaded"}
+                r["gpu_vs_cpu_step"] = r["step_tokens_per_s"] / tps
+            configs[name] = r
+            if wc is not w:
+                del wc
+
     # ---- end to end through the public API from pinned host memory
     # Every step: H2D of the step's inputs (ids, hidden rows, gates, global
     # scale), the whole path with identity experts (the combine reads the bf16
@@ -594,15 +731,23 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
             "gpu_launches": launches_per_step * args.steps,
             "next_rows": ({"f1_grouped_gemm_ready_nvfp4": f1, "f3_mx_and_swiglu_requant": f3,
                            "f4_backward": f4} if f1 or f3 or f4 else None),
+            "configs": configs,
             "clocks": clocks, "layout_status": st,
         }
         if world == 1 and not args.no_cpu_baseline:
             n_cpu = args.cpu_tokens
             tps, dt = oracle_tokens_per_s(w, n_cpu)
+            box = os.cpu_count() or 1
+            tps_all, dt_all = oracle_tokens_per_s(w, n_cpu, threads=box)
             line["cpu_baseline"] = {
                 "value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                 "sample": f"first {n_cpu} tokens of the batch, own layout with "
-                          f"recv_capacity = {n_cpu}*k; {dt:.1f} s single-threaded"}
+                          f"recv_capacity = {n_cpu}*k; {dt:.1f} s single-threaded",
+                "box_cores": box,
+                "all_cores": {"value": tps_all, "unit": "tokens/s", "threads": box,
+                              "seconds": round(dt_all, 2),
+                              "how": "the same oracle calls, the permutes' rows and the "
+                                     "combine's tokens split over a thread pool"}}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -619,6 +764,8 @@ def main() -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next-rows", dest="next_rows", action="store_false",
                     help="skip the extra measurement of the grouped-GEMM-ready dispatch")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the sweep over every workload of the benchmark set")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -36,6 +36,7 @@ MOE_STATUS_TIMEOUT = 8
 MOE_FLAG_CHECK_DUPLICATES = 1
 MOE_FLAG_LAYOUT_TWO_PASS = 2
 MOE_FLAG_NVFP4_SWIZZLED_SCALES = 4
+MOE_FLAG_LAYOUT_LOOKBACK = 8
 MOE_FLAG_TEST_STALL_SCAN = 0x80000000
 
 MOE_MAX_EXPERTS = 2048

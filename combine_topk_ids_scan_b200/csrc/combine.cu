@@ -12,7 +12,10 @@
 // and gate, shuffles broadcast them; per step each lane loads one 16-byte
 // vector (8 bf16) from every live row -- U steps at once, so up to k*U
 // independent 16-byte loads per lane are in flight -- and writes one 16-byte
-// vector of the result.
+// vector of the result.  With few tokens (fewer than the resident warps) a
+// token's row is split into `splits` column spans of `span` vectors, one
+// warp each, so that small batches still fill the GPU; every output element
+// is the same fma chain whatever the split.
 #include <algorithm>
 
 #include "common.cuh"
@@ -29,14 +32,17 @@ template <int KMAX, int U>
 __global__ void __launch_bounds__(kThreads)
     combine_kernel(const uint4 *__restrict__ x, const float *__restrict__ gates,
                    const int32_t *__restrict__ pair_slot, uint4 *__restrict__ out, int32_t N,
-                   int32_t k, int64_t rows, int32_t vecs) {
+                   int32_t k, int64_t rows, int32_t vecs, int32_t splits, int32_t span) {
   allow_dependents();
   grid_dependency_wait();
   const int lane = threadIdx.x % kWarp;
   const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t nw = ((int64_t)gridDim.x * kThreads) / kWarp;
 
-  for (int64_t t = gw; t < N; t += nw) {
+  for (int64_t item = gw; item < (int64_t)N * splits; item += nw) {
+    const int64_t t = item / splits;
+    const int32_t vb = (int32_t)(item % splits) * span;
+    const int32_t ve = min(vecs, vb + span);
     int32_t my_slot = -1;
     float my_w = 0.0f;
     if (lane < k) {
@@ -57,15 +63,15 @@ __global__ void __launch_bounds__(kThreads)
       w[j] = __shfl_sync(kFull, my_w, j);
     }
     uint4 *dst = out + t * vecs;
-    for (int v0 = 0; v0 < vecs; v0 += kWarp * U) {
+    for (int v0 = vb; v0 < ve; v0 += kWarp * U) {
       uint4 in[KMAX][U];
 #pragma unroll
       for (int j = 0; j < KMAX; ++j)
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int v = v0 + u * kWarp + lane;
-          in[j][u] = (row[j] >= 0 && v < vecs) ? ld_stream_v4(x + row[j] * vecs + v)
-                                                : make_uint4(0, 0, 0, 0);
+          in[j][u] = (row[j] >= 0 && v < ve) ? ld_stream_v4(x + row[j] * vecs + v)
+                                              : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -83,7 +89,7 @@ __global__ void __launch_bounds__(kThreads)
             acc[2 * i + 1] = fmaf(w[j], bf16hi(e[i]), acc[2 * i + 1]);
           }
         }
-        if (v < vecs)
+        if (v < ve)
           st_v4(dst + v, make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                                     pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7])));
       }
@@ -208,8 +214,21 @@ cudaError_t launch_forward(const Shape &s, const uint4 *x, const float *gates,
                            const int32_t *pair_slot, uint4 *o, cudaStream_t stream) {
   static OccupancyCache cache;
   auto kernel = combine_kernel<KMAX, U>;
-  return launch_pdl(kernel, dim3(grid_for(kernel, s.N, cache)), dim3(kThreads), 0, stream, x, gates,
-                    pair_slot, o, s.N, s.k, s.rows, s.H / 8);
+  // column spans per token: 1 when the tokens alone fill the resident warps
+  // (half of them at least), else enough spans of whole U-steps to do so
+  const int32_t vecs = s.H / 8;
+  const int32_t step = kWarp * U;
+  const int32_t steps = (vecs + step - 1) / step;
+  const int64_t resident = (int64_t)resident_ctas(cache, reinterpret_cast<const void *>(kernel),
+                                                  kThreads, 0) *
+                           device_sm_count() * (kThreads / kWarp);
+  int32_t splits = 1;
+  if ((int64_t)s.N * 2 < resident)
+    splits = (int32_t)std::min<int64_t>(steps, (resident + s.N - 1) / s.N);
+  const int32_t span = (steps + splits - 1) / splits * step;
+  splits = (vecs + span - 1) / span;
+  return launch_pdl(kernel, dim3(grid_for(kernel, (int64_t)s.N * splits, cache)), dim3(kThreads),
+                    0, stream, x, gates, pair_slot, o, s.N, s.k, s.rows, vecs, splits, span);
 }
 
 }  // namespace

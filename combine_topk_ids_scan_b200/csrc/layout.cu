@@ -33,6 +33,8 @@
 // packed_source_indices, send_counts, recv_capacity, [4, EP] metadata in
 // elements); DeepSpeed capacity dispatch ([e, c, m] buffer); NeMo AutoModel
 // token_dispatcher (-1 ids are masked; tokens per expert).
+#include <cooperative_groups.h>
+
 #include <algorithm>
 #include <atomic>
 
@@ -47,12 +49,12 @@ constexpr int kScanThreads = 512;
 constexpr int kScanWarps = kScanThreads / kWarp;        // 16
 constexpr int kScanRounds = 8;                          // pairs per lane
 constexpr int kTilePairs = kScanThreads * kScanRounds;  // 4096
-constexpr int kWarpPairs = kWarp * kScanRounds;         // 256
 constexpr uint64_t kFlagAggregate = 1ull;
 constexpr uint64_t kFlagInclusive = 2ull;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // every bounded wait: 1 s
 constexpr int kLookWindow = 8;                    // predecessor tiles per poll
 constexpr int kFusedMaxTiles = 128;               // last CTA clears <= 128*E words
+constexpr int64_t kClusterMaxRows = 1 << 18;      // cluster path: rows per launch
 
 constexpr int kEmitThreads = 256;
 
@@ -93,12 +95,14 @@ __device__ __forceinline__ bool keep_waiting(uint64_t &deadline) {
   return now <= deadline;
 }
 
-// Per-CTA state of one scan tile.  pk[r] packs the lane's r-th pair: expert
-// id in the low 16 bits (0xFFFF: no expert), rank inside the warp's 256 pairs
-// in the high 16 bits.
-struct TileScan {
+// Per-CTA state of one scan tile of ROUNDS * 512 pairs (each warp owns
+// ROUNDS * 32 consecutive pairs).  pk[r] packs the lane's r-th pair: expert
+// id in the low 16 bits (0xFFFF: no expert), rank inside the warp's pairs in
+// the high 16 bits.
+template <int ROUNDS>
+struct TileScanT {
   int tile;
-  uint32_t pk[kScanRounds];
+  uint32_t pk[ROUNDS];
   int64_t base;  // first pair of this warp
   __device__ __forceinline__ int32_t expert(int r) const {
     const uint32_t e = pk[r] & 0xFFFFu;
@@ -106,35 +110,30 @@ struct TileScan {
   }
   __device__ __forceinline__ uint32_t rank(int r) const { return pk[r] >> 16; }
 };
+using TileScan = TileScanT<kScanRounds>;
 
-// Phases 1-3 of a tile: in-warp ranks, warp bases (left in wcnt), tile
-// exclusive prefix per expert (left in tile_prefix); the last tile also
-// stores the per-expert totals.  Returns false when the ticket is past the
-// last tile (a workspace that was not zero-filled).
-__device__ bool scan_tile(TileScan &ts, const int32_t *__restrict__ ids, int64_t P, int32_t E,
-                          int32_t num_tiles, uint32_t flags, uint32_t *ctrl, uint64_t *tiles,
-                          int32_t *totals, const ScanSmem &sm, int *s_tile, uint32_t *s_status) {
+// Phases 1-2 of tile ts.tile (set by the caller): in-warp stable ranks and
+// per-warp histograms, then per expert the exclusive scan over the warps
+// (warp bases, left in wcnt; at most 16 * ROUNDS * 32 <= 65535) and the tile
+// aggregate (left in tile_prefix).  ORs MOE_STATUS_ID_RANGE into *s_status.
+// Called by all threads of the block; ends with a block barrier.
+template <int ROUNDS>
+__device__ void rank_tile(TileScanT<ROUNDS> &ts, const int32_t *__restrict__ ids, int64_t P,
+                          int32_t E, const ScanSmem &sm, uint32_t *s_status) {
   const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
   uint16_t *wcnt = sm.wcnt;
   uint32_t *tile_prefix = sm.tile_prefix;
-  if (tid == 0) {
-    *s_tile = (int)atomicAdd(&ctrl[kCtrlTicket], 1u);
-    *s_status = 0;
-  }
-  __syncthreads();
-  if (*s_tile >= num_tiles) return false;
   for (int i = tid; i < kScanWarps * E; i += kScanThreads) {
     wcnt[i] = 0;
     sm.wmask[i] = 0;
   }
   __syncthreads();
-  ts.tile = *s_tile;
 
   // ---- 1. per-warp stable ranks and histograms
-  ts.base = (int64_t)ts.tile * kTilePairs + (int64_t)warp * kWarpPairs;
-  int32_t ex[kScanRounds];
+  ts.base = (int64_t)ts.tile * (kScanThreads * ROUNDS) + (int64_t)warp * (kWarp * ROUNDS);
+  int32_t ex[ROUNDS];
 #pragma unroll
-  for (int r = 0; r < kScanRounds; ++r) {
+  for (int r = 0; r < ROUNDS; ++r) {
     const int64_t p = ts.base + r * kWarp + lane;
     ex[r] = p < P ? __ldg(ids + p) : -1;
   }
@@ -142,7 +141,7 @@ __device__ bool scan_tile(TileScan &ts, const int32_t *__restrict__ ids, int64_t
   uint16_t *my_cnt = wcnt + (size_t)warp * E;
   uint32_t *my_mask = sm.wmask + (size_t)warp * E;
 #pragma unroll
-  for (int r = 0; r < kScanRounds; ++r) {
+  for (int r = 0; r < ROUNDS; ++r) {
     const int32_t e = ex[r];
     const bool valid = (uint32_t)e < (uint32_t)E;
     bad_id |= (!valid && e != -1);
@@ -179,6 +178,26 @@ __device__ bool scan_tile(TileScan &ts, const int32_t *__restrict__ ids, int64_t
     }
     tile_prefix[e] = run;
   }
+  __syncthreads();
+}
+
+// Phases 1-3 of a tile: in-warp ranks, warp bases (left in wcnt), tile
+// exclusive prefix per expert (left in tile_prefix); the last tile also
+// stores the per-expert totals.  Returns false when the ticket is past the
+// last tile (a workspace that was not zero-filled).
+__device__ bool scan_tile(TileScan &ts, const int32_t *__restrict__ ids, int64_t P, int32_t E,
+                          int32_t num_tiles, uint32_t flags, uint32_t *ctrl, uint64_t *tiles,
+                          int32_t *totals, const ScanSmem &sm, int *s_tile, uint32_t *s_status) {
+  const int tid = threadIdx.x;
+  uint32_t *tile_prefix = sm.tile_prefix;
+  if (tid == 0) {
+    *s_tile = (int)atomicAdd(&ctrl[kCtrlTicket], 1u);
+    *s_status = 0;
+  }
+  __syncthreads();
+  if (*s_tile >= num_tiles) return false;
+  ts.tile = *s_tile;
+  rank_tile<kScanRounds>(ts, ids, P, E, sm, s_status);
 
   // ---- 3. decoupled look-back across tiles, one chain per expert
   const int tile = ts.tile;
@@ -306,13 +325,13 @@ __device__ int32_t block_exclusive_scan(int32_t *v, int n) {
 
 // Expert start rows s_off[E+1] and kept rows s_kept[E] from the totals
 // (packed mode: each expert's block is its count rounded up to `pad`).
-template <int THREADS>
+template <int THREADS, bool SMEM_TOTALS = false>
 __device__ void expert_offsets_from_totals(const int32_t *totals, bool have_totals, int32_t E,
                                            int32_t Ce, int32_t pad, int32_t *s_off,
                                            int32_t *s_kept) {
   const bool capacity = Ce > 0;
   for (int e = threadIdx.x; e < E; e += THREADS) {
-    const int32_t t = have_totals ? __ldcg(totals + e) : 0;
+    const int32_t t = !have_totals ? 0 : SMEM_TOTALS ? totals[e] : __ldcg(totals + e);
     s_kept[e] = capacity ? min(t, Ce) : t;
     s_off[e] = capacity ? e * Ce : (pad > 1 ? (t + pad - 1) / pad * pad : t);
   }
@@ -557,6 +576,87 @@ __global__ void __launch_bounds__(kEmitThreads) layout_emit_kernel(LayoutArgs a)
   emit_step<kEmitThreads>(a, gtid, gstride, &s_status, 0);
 }
 
+// One thread-block cluster for the whole layout (P <= cluster size * ROUNDS
+// * 512 pairs).  CTA c of the cluster ranks tile c (phases 1-2 above), then
+// the CTAs exchange their per-expert tile aggregates through distributed
+// shared memory: after a cluster barrier each CTA reads every tile's
+// aggregate, which gives its own exclusive prefix (tiles before it) and the
+// totals (all tiles) at once -- no look-back chain, no grid-wide wait, no
+// workspace.  Each CTA then turns its pairs' ranks (still in registers) into
+// rows, writes its share of the padding rows, and ORs its status bits into
+// CTA 0's shared word; a second cluster barrier keeps every CTA's shared
+// memory alive until the others have read it, and CTA 0 stores the status.
+// The barriers are hardware cluster barriers over co-scheduled CTAs: there
+// is no spin loop and nothing to time out.
+template <int ROUNDS>
+__global__ void __launch_bounds__(kScanThreads, 1) layout_cluster_kernel(LayoutArgs a) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  allow_dependents();  // the next kernel may be scheduled; it waits for this grid
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ uint32_t s_status;
+  const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
+  const int c = (int)cluster.block_rank();
+  const int nc = (int)cluster.num_blocks();
+  const int32_t E = a.E;
+  const ScanSmem sm = scan_smem(smem, E);
+  if (tid == 0) s_status = 0;
+  TileScanT<ROUNDS> ts;
+  ts.tile = c;
+  rank_tile<ROUNDS>(ts, a.ids, a.P, E, sm, &s_status);
+  cluster.sync();  // every tile's aggregate (tile_prefix) is visible
+
+  // the lane-mask words are free now: exclusive prefix, start rows, kept rows
+  int32_t *s_excl = reinterpret_cast<int32_t *>(sm.wmask);
+  int32_t *s_off = s_excl + E;       // [E + 1]
+  int32_t *s_kept = s_off + E + 1;   // [E]: the totals, then the kept rows
+  for (int e = tid; e < E; e += kScanThreads) {
+    uint32_t excl = 0, tot = 0;
+    for (int q = 0; q < nc; ++q) {
+      const uint32_t v = *cluster.map_shared_rank(sm.tile_prefix + e, q);
+      excl += q < c ? v : 0u;
+      tot += v;
+    }
+    s_excl[e] = (int32_t)excl;
+    s_kept[e] = (int32_t)tot;
+  }
+  __syncthreads();
+  expert_offsets_from_totals<kScanThreads, true>(s_kept, true, E, a.Ce, a.pad, s_off, s_kept);
+
+  // ranks -> rows for this tile's pairs
+  const bool capacity = a.Ce > 0;
+  uint32_t bits = 0;
+#pragma unroll
+  for (int r = 0; r < ROUNDS; ++r) {
+    const int64_t p = ts.base + r * kWarp + lane;
+    if (p < a.P) {
+      const int32_t e = ts.expert(r);
+      int32_t slot = -1;
+      uint8_t dropped = 0;
+      if (e >= 0) {
+        const int32_t rank =
+            s_excl[e] + (int32_t)sm.wcnt[(size_t)warp * E + e] + (int32_t)ts.rank(r);
+        slot = row_of(e, rank, s_off, a.C, a.Ce, capacity, dropped, bits);
+      }
+      a.pair_slot[p] = slot;
+      if (a.drop_mask) a.drop_mask[p] = dropped;
+      if (slot >= 0) a.row_src[slot] = (int32_t)(p / a.k);
+    }
+  }
+  const int64_t gtid = (int64_t)c * kScanThreads + tid;
+  const int64_t gstride = (int64_t)nc * kScanThreads;
+  emit_common<kScanThreads>(gtid, gstride, a.rows, E, a.S, a.Ce, a.pad, a.H, s_off, s_kept,
+                            a.row_src, c == 0, a.expert_counts, a.expert_offsets, a.meta);
+  if (a.flags & MOE_FLAG_CHECK_DUPLICATES)
+    bits |= duplicate_bits(a.ids, gtid, a.N, gstride, a.k, E);
+  if (bits) atomicOr(&s_status, bits);
+  __syncthreads();
+  if (tid == 0 && c != 0 && s_status != 0)
+    atomicOr(cluster.map_shared_rank(&s_status, 0), s_status);
+  cluster.sync();  // all remote reads and status bits are done
+  if (c == 0 && tid == 0) *a.status_out = s_status;
+}
+
 // Opt the scan kernels in to more than 48 KB of dynamic shared memory, once
 // per device.
 cudaError_t opt_in_smem() {
@@ -571,8 +671,81 @@ cudaError_t opt_in_smem() {
   if (err == cudaSuccess)
     err = cudaFuncSetAttribute(layout_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bytes);
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(layout_cluster_kernel<kScanRounds>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(layout_cluster_kernel<2 * kScanRounds>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (err == cudaSuccess && dev < kMaxDevices) done[dev].store(true);
   return err;
+}
+
+// Largest cluster of the cluster kernel this device can schedule (16 with
+// the non-portable size, else 8, else 0 = no cluster path), queried once per
+// device with the largest dynamic shared memory the kernel takes.
+int max_cluster_size() {
+  static std::atomic<int> cache[kMaxDevices];  // 0 = not queried, else size + 1
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < kMaxDevices) {
+    const int v = cache[dev].load();
+    if (v > 0) return v - 1;
+  }
+  if (opt_in_smem() != cudaSuccess) return 0;
+  int best = 0;
+  const int bytes = (int)scan_smem_bytes(MOE_MAX_EXPERTS);
+  const void *kernels[2] = {(const void *)layout_cluster_kernel<kScanRounds>,
+                            (const void *)layout_cluster_kernel<2 * kScanRounds>};
+  for (int size : {16, 8}) {
+    bool ok = true;
+    for (const void *kern : kernels) {
+      if (size > 8 &&
+          cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+              cudaSuccess) {
+        ok = false;
+        break;
+      }
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(size);
+      cfg.blockDim = dim3(kScanThreads);
+      cfg.dynamicSmemBytes = bytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = size;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
+        ok = false;
+    }
+    if (ok) {
+      best = size;
+      break;
+    }
+  }
+  (void)cudaGetLastError();  // a refused query leaves no sticky error
+  if (dev < kMaxDevices) cache[dev].store(best + 1);
+  return best;
+}
+
+template <int ROUNDS>
+cudaError_t launch_cluster(const LayoutArgs &a, int nc, size_t smem, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nc);
+  cfg.blockDim = dim3(kScanThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nc;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, layout_cluster_kernel<ROUNDS>, a);
 }
 
 // Largest grid of the fused kernel that is guaranteed co-resident.
@@ -636,6 +809,24 @@ cudaError_t launch_layout(const Shape &s, const int32_t *ids, int32_t *expert_co
   if (ws.num_tiles > 0 && smem > 32 * 1024) {
     cudaError_t err = opt_in_smem();
     if (err != cudaSuccess) return err;
+  }
+
+  // One cluster when the pairs fit in at most max_cluster_size() tiles of
+  // 4096 (or 8192) pairs and the rows in a few passes of its threads.
+  const uint32_t forced = MOE_FLAG_LAYOUT_TWO_PASS | MOE_FLAG_LAYOUT_LOOKBACK |
+                          MOE_FLAG_TEST_STALL_SCAN;
+  if (!(s.flags & forced) && s.rows <= kClusterMaxRows) {
+    const int maxc = max_cluster_size();
+    const int64_t t8 = std::max<int64_t>(1, (s.P + kTilePairs - 1) / kTilePairs);
+    const int64_t t16 = std::max<int64_t>(1, (s.P + 2 * kTilePairs - 1) / (2 * kTilePairs));
+    if (maxc > 0 && t8 <= maxc) {
+      if (opt_in_smem() != cudaSuccess) return cudaErrorUnknown;
+      return launch_cluster<kScanRounds>(a, (int)t8, smem, stream);
+    }
+    if (maxc > 0 && t16 <= maxc) {
+      if (opt_in_smem() != cudaSuccess) return cudaErrorUnknown;
+      return launch_cluster<2 * kScanRounds>(a, (int)t16, smem, stream);
+    }
   }
 
   if (ws.num_tiles > 0 && ws.num_tiles <= kFusedMaxTiles &&

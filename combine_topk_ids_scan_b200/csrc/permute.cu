@@ -54,6 +54,13 @@ __device__ __forceinline__ uint32_t padding_mask(int64_t g, int lane,
   return __ballot_sync(kFull, r < check_rows && (r >= rows || __ldg(row_src + r) < 0));
 }
 
+// Share c of `parts` near-equal shares of [0, n): [b, e).
+__device__ __forceinline__ void share_of(int c, int parts, int32_t n, int32_t &b, int32_t &e) {
+  const int32_t per = (n + parts - 1) / parts;
+  b = min(n, c * per);
+  e = min(n, b + per);
+}
+
 // Zero 16-byte vectors [v0, v1) of each row in `m` (rows 32g + bit) and,
 // when scales is not null, 2-byte words [s0, s1) of its scale row.
 __device__ __forceinline__ void zero_rows(uint32_t m, int64_t g, int lane, uint4 *out,
@@ -79,17 +86,22 @@ __device__ __forceinline__ void zero_rows(uint32_t m, int64_t g, int lane, uint4
 __global__ void __launch_bounds__(kThreads)
     permute_bf16_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                         const int32_t *__restrict__ pair_slot, uint4 *__restrict__ out,
-                        int32_t N, int32_t k, int64_t rows, int32_t vecs, int32_t chunks) {
+                        int32_t N, int32_t k, int64_t rows, int32_t vecs, int32_t chunks,
+                        int32_t psplit) {
   allow_dependents();
   grid_dependency_wait();
   constexpr int U = kBf16Chunk / 8 / kWarp;  // 2
   const int lane = threadIdx.x % kWarp;
   const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
-  const int64_t pad_units = (rows + kWarp - 1) / kWarp;
+  const int64_t pad_units = (rows + kWarp - 1) / kWarp * psplit;
   if (w0 < pad_units) {
-    if (const uint32_t m = padding_mask(w0, lane, row_src, rows, rows))
-      zero_rows(m, w0, lane, out, vecs, 0, vecs, nullptr, 0, 0, 0);
+    const int64_t g = w0 / psplit;
+    if (const uint32_t m = padding_mask(g, lane, row_src, rows, rows)) {
+      int32_t v0, v1;
+      share_of((int)(w0 % psplit), psplit, vecs, v0, v1);
+      zero_rows(m, g, lane, out, vecs, v0, v1, nullptr, 0, 0, 0);
+    }
     return;
   }
   const int64_t w = w0 - pad_units;
@@ -137,17 +149,21 @@ __global__ void __launch_bounds__(kThreads)
                                  const int32_t *__restrict__ pair_slot,
                                  const float *__restrict__ gates, uint4 *__restrict__ out,
                                  int32_t N, int32_t k, int64_t rows, int32_t vecs,
-                                 int32_t chunks) {
+                                 int32_t chunks, int32_t psplit) {
   allow_dependents();
   grid_dependency_wait();
   constexpr int U = kBf16Chunk / 8 / kWarp;  // 2
   const int lane = threadIdx.x % kWarp;
   const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
-  const int64_t pad_units = (rows + kWarp - 1) / kWarp;
+  const int64_t pad_units = (rows + kWarp - 1) / kWarp * psplit;
   if (w0 < pad_units) {
-    if (const uint32_t m = padding_mask(w0, lane, row_src, rows, rows))
-      zero_rows(m, w0, lane, out, vecs, 0, vecs, nullptr, 0, 0, 0);
+    const int64_t g = w0 / psplit;
+    if (const uint32_t m = padding_mask(g, lane, row_src, rows, rows)) {
+      int32_t v0, v1;
+      share_of((int)(w0 % psplit), psplit, vecs, v0, v1);
+      zero_rows(m, g, lane, out, vecs, v0, v1, nullptr, 0, 0, 0);
+    }
     return;
   }
   const int64_t w = w0 - pad_units;
@@ -186,20 +202,26 @@ __global__ void __launch_bounds__(kThreads)
     permute_fp8_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                        const int32_t *__restrict__ pair_slot, uint8_t *__restrict__ q,
                        float *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
-                       int32_t H, int32_t chunks) {
+                       int32_t H, int32_t chunks, int32_t psplit) {
   allow_dependents();
   grid_dependency_wait();
   constexpr int U = kChunk / 512;  // 2
   const int lane = threadIdx.x % kWarp;
   const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
-  const int64_t pad_units = (rows + kWarp - 1) / kWarp;
+  const int64_t pad_units = (rows + kWarp - 1) / kWarp * psplit;
   const int32_t vecs = H / 8;
   const int32_t nb = H / 128;
   if (w0 < pad_units) {
-    if (const uint32_t m = padding_mask(w0, lane, row_src, rows, rows))
-      zero_rows(m, w0, lane, reinterpret_cast<uint4 *>(q), H / 16, 0, H / 16,
-                reinterpret_cast<uint16_t *>(scales), 2 * nb, 0, 2 * nb);
+    const int64_t g = w0 / psplit;
+    if (const uint32_t m = padding_mask(g, lane, row_src, rows, rows)) {
+      const int c = (int)(w0 % psplit);
+      int32_t v0, v1, s0, s1;
+      share_of(c, psplit, H / 16, v0, v1);
+      share_of(c, psplit, 2 * nb, s0, s1);
+      zero_rows(m, g, lane, reinterpret_cast<uint4 *>(q), H / 16, v0, v1,
+                reinterpret_cast<uint16_t *>(scales), 2 * nb, s0, s1);
+    }
     return;
   }
   const int64_t w = w0 - pad_units;
@@ -349,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
                        const int32_t *__restrict__ pair_slot,
                        const float *__restrict__ global_scale, uint8_t *__restrict__ q,
                        uint8_t *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
-                       int32_t H, int32_t chunks) {
+                       int32_t H, int32_t chunks, int32_t psplit) {
   constexpr bool swizzled = SWIZZLED;
   allow_dependents();
   grid_dependency_wait();
@@ -359,40 +381,51 @@ __global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
   // swizzled scales: the rows that only complete the last 128-row tile are
   // padding for the scales too
   const int64_t check_rows = swizzled ? (rows + 127) / 128 * 128 : rows;
-  const int64_t pad_units = (check_rows + kWarp - 1) / kWarp;
+  const int64_t pad_units = (check_rows + kWarp - 1) / kWarp * psplit;
   const int32_t vecs = H / 8;
   const int32_t qrow = H / 2, srow = MX ? H / 32 : H / 16;
   const int32_t groups = (srow + 3) / 4;  // 4-scale groups per row (atom layout)
   if (w0 < pad_units) {
     // codes: H/2 bytes per row; scales: linear srow bytes per row, or the
-    // row's `groups` 4-byte groups in the atom layout
-    const uint32_t m = padding_mask(w0, lane, row_src, rows, check_rows);
+    // row's `groups` 4-byte groups in the atom layout; this warp zeroes its
+    // share c of each of them
+    const int64_t g = w0 / psplit;
+    const int c = (int)(w0 % psplit);
+    const uint32_t m = padding_mask(g, lane, row_src, rows, check_rows);
+    int32_t v0, v1;
+    share_of(c, psplit, qrow / 16, v0, v1);
     if (m && !swizzled && MX) {
+      int32_t s0, s1;
+      share_of(c, psplit, srow, s0, s1);
       uint32_t mm = m;
       const uint4 zero = make_uint4(0, 0, 0, 0);
       while (mm) {
         const int j = __ffs(mm) - 1;
         mm &= mm - 1;
-        const int64_t row = w0 * kWarp + j;
+        const int64_t row = g * kWarp + j;
         uint4 *dst = reinterpret_cast<uint4 *>(q) + row * (qrow / 16);
-        for (int v = lane; v < qrow / 16; v += kWarp) st_v4(dst + v, zero);
-        for (int v = lane; v < srow; v += kWarp) scales[row * srow + v] = 0;
+        for (int v = v0 + lane; v < v1; v += kWarp) st_v4(dst + v, zero);
+        for (int v = s0 + lane; v < s1; v += kWarp) scales[row * srow + v] = 0;
       }
     } else if (m && !swizzled) {
-      zero_rows(m, w0, lane, reinterpret_cast<uint4 *>(q), qrow / 16, 0, qrow / 16,
-                reinterpret_cast<uint16_t *>(scales), srow / 2, 0, srow / 2);
+      int32_t s0, s1;
+      share_of(c, psplit, srow / 2, s0, s1);
+      zero_rows(m, g, lane, reinterpret_cast<uint4 *>(q), qrow / 16, v0, v1,
+                reinterpret_cast<uint16_t *>(scales), srow / 2, s0, s1);
     } else if (m) {
+      int32_t g0, g1;
+      share_of(c, psplit, groups, g0, g1);
       uint32_t mm = m;
       const uint4 zero = make_uint4(0, 0, 0, 0);
       while (mm) {
         const int j = __ffs(mm) - 1;
         mm &= mm - 1;
-        const int64_t row = w0 * kWarp + j;
+        const int64_t row = g * kWarp + j;
         if (row < rows) {
           uint4 *dst = reinterpret_cast<uint4 *>(q) + row * (qrow / 16);
-          for (int v = lane; v < qrow / 16; v += kWarp) st_v4(dst + v, zero);
+          for (int v = v0 + lane; v < v1; v += kWarp) st_v4(dst + v, zero);
         }
-        for (int gg = lane; gg < groups; gg += kWarp)
+        for (int gg = g0 + lane; gg < g1; gg += kWarp)
           st_u32_evict_last(scales + sf_atom_offset(row, 4 * gg, groups), 0u);
       }
     }
@@ -471,10 +504,63 @@ __global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
   }
 }
 
-// One warp per unit: ceil(check_rows / 32) padding warps, then N * chunks
-// token units.
-inline int64_t unit_blocks(const Shape &s, int32_t chunks, int64_t check_rows) {
-  const int64_t warps = (check_rows + kWarp - 1) / kWarp + (int64_t)s.N * chunks;
+// Block-scale atom layout from linear scales, in place, one CTA per 128-row
+// tile.  When the scale columns per row (nsf) are a multiple of 4, a tile's
+// linear scales ([128, nsf] row-major, rows past `rows` unwritten) and its
+// atoms (nsf/4 atoms of 512 bytes) occupy the same bytes of the buffer, so
+// the permute writes linear scales there first (whole 64- or 32-byte runs
+// per warp instead of 4-byte pieces of 8 different rows per 32-byte sector)
+// and this kernel reads the whole tile into shared memory, then writes it
+// back in atom order; rows at or past `rows` become zeros.  Shared layout:
+// word (m, g) of 4-scale group g at g * 129 + (m % 32) * 4 + m / 32 -- the
+// atom order, so the write-back reads consecutive words, padded by one word
+// per group so that the scattered writes of a warp (consecutive g) fall in
+// distinct banks.
+constexpr int kAtomThreads = 256;
+constexpr int kAtomGroupWords = 129;
+
+inline size_t atom_tile_smem(int32_t nsf) {
+  return (size_t)(nsf / 4) * kAtomGroupWords * sizeof(uint32_t);
+}
+
+__global__ void __launch_bounds__(kAtomThreads)
+    scales_to_atoms_kernel(uint32_t *__restrict__ scales, int64_t rows, int32_t groups) {
+  allow_dependents();
+  extern __shared__ uint32_t tile_words[];
+  grid_dependency_wait();
+  const int64_t tile = blockIdx.x;
+  const int64_t left = rows - tile * 128;
+  const int32_t nrows = left < 128 ? (int32_t)left : 128;
+  uint32_t *base = scales + tile * 128 * groups;  // the tile's words (either layout)
+  const int32_t words = 128 * groups;
+  for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) {
+    const int32_t m = w / groups, g = w - m * groups;
+    const uint32_t v = m < nrows ? base[w] : 0u;
+    tile_words[g * kAtomGroupWords + (m & 31) * 4 + (m >> 5)] = v;
+  }
+  __syncthreads();
+  for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) {
+    const int32_t g = w >> 7, wi = w & 127;
+    base[w] = tile_words[g * kAtomGroupWords + wi];
+  }
+}
+
+// Padding warps per 32-row group: when the problem has more rows than pairs
+// (capacity layouts, padded experts, a recv_capacity above N*k) some rows
+// are certainly padding, and a group of 32 padding rows is shared by as many
+// warps as a token row has units (each zeroes the same column share of the
+// group's padding rows); otherwise one warp per group, which exits at once
+// when its rows all have a source.  Measured on B200 at N=128, H=7168,
+// E=256, k=8 with [256, 5] rows (340 padding rows): bf16 25.3 us with one
+// warp per group.
+inline int32_t padding_split(const Shape &s, int32_t chunks) {
+  return s.rows > s.P ? chunks : 1;
+}
+
+// One warp per unit: ceil(check_rows / 32) * psplit padding warps, then
+// N * chunks token units.
+inline int64_t unit_blocks(const Shape &s, int32_t chunks, int64_t check_rows, int32_t psplit) {
+  const int64_t warps = (check_rows + kWarp - 1) / kWarp * psplit + (int64_t)s.N * chunks;
   return std::max<int64_t>(1, (warps + kThreads / kWarp - 1) / (kThreads / kWarp));
 }
 
@@ -486,9 +572,10 @@ cudaError_t launch_permute_bf16(const Shape &s, const void *hidden, const int32_
                                 const int32_t *pair_slot, void *out, cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
   const int32_t chunks = chunks_of(s.H, kBf16Chunk);
-  return launch_pdl(permute_bf16_kernel, dim3((unsigned)unit_blocks(s, chunks, s.rows)),
+  const int32_t ps = padding_split(s, chunks);
+  return launch_pdl(permute_bf16_kernel, dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)),
                     dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src,
-                    pair_slot, static_cast<uint4 *>(out), s.N, s.k, s.rows, s.H / 8, chunks);
+                    pair_slot, static_cast<uint4 *>(out), s.N, s.k, s.rows, s.H / 8, chunks, ps);
 }
 
 cudaError_t launch_permute_premultiplied(const Shape &s, const void *hidden,
@@ -496,10 +583,11 @@ cudaError_t launch_permute_premultiplied(const Shape &s, const void *hidden,
                                          const float *gates, void *out, cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
   const int32_t chunks = chunks_of(s.H, kBf16Chunk);
+  const int32_t ps = padding_split(s, chunks);
   return launch_pdl(permute_premultiplied_kernel,
-                    dim3((unsigned)unit_blocks(s, chunks, s.rows)), dim3(kThreads), 0, stream,
+                    dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads), 0, stream,
                     static_cast<const uint4 *>(hidden), row_src, pair_slot, gates,
-                    static_cast<uint4 *>(out), s.N, s.k, s.rows, s.H / 8, chunks);
+                    static_cast<uint4 *>(out), s.N, s.k, s.rows, s.H / 8, chunks, ps);
 }
 
 cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t *row_src,
@@ -507,9 +595,30 @@ cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t
                                cudaStream_t stream) {
   if (s.rows == 0) return cudaSuccess;
   const int32_t chunks = chunks_of(s.H, kChunk);
-  return launch_pdl(permute_fp8_kernel, dim3((unsigned)unit_blocks(s, chunks, s.rows)),
+  const int32_t ps = padding_split(s, chunks);
+  return launch_pdl(permute_fp8_kernel, dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)),
                     dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src,
-                    pair_slot, q, scales, s.N, s.k, s.rows, s.H, chunks);
+                    pair_slot, q, scales, s.N, s.k, s.rows, s.H, chunks, ps);
+}
+
+// Atom-layout scales through linear scales and the in-place tile kernel:
+// possible when the scale columns per row are a multiple of 4 and a tile's
+// scales fit in shared memory.
+inline bool atoms_in_place(int32_t nsf) {
+  return nsf % 4 == 0 && atom_tile_smem(nsf) <= 200 * 1024;
+}
+
+cudaError_t launch_scales_to_atoms(const Shape &s, int32_t nsf, uint8_t *scales,
+                                   cudaStream_t stream) {
+  const size_t smem = atom_tile_smem(nsf);
+  if (smem > 48 * 1024) {
+    const cudaError_t err = cudaFuncSetAttribute(
+        scales_to_atoms_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+  }
+  return launch_pdl(scales_to_atoms_kernel, dim3((unsigned)((s.rows + 127) / 128)),
+                    dim3(kAtomThreads), smem, stream, reinterpret_cast<uint32_t *>(scales),
+                    s.rows, nsf / 4);
 }
 
 cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32_t *row_src,
@@ -518,11 +627,20 @@ cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32
   if (s.rows == 0) return cudaSuccess;
   const int32_t chunks = chunks_of(s.H, kChunk);
   const bool swizzled = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) != 0;
+  const int32_t ps = padding_split(s, chunks);
+  if (swizzled && atoms_in_place(s.H / 16)) {
+    const cudaError_t err = launch_pdl(
+        permute_fp4_kernel<false, false>, dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)),
+        dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src, pair_slot,
+        global_scale, q, scales, s.N, s.k, s.rows, s.H, chunks, ps);
+    if (err != cudaSuccess) return err;
+    return launch_scales_to_atoms(s, s.H / 16, scales, stream);
+  }
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
   return launch_pdl(swizzled ? permute_fp4_kernel<false, true> : permute_fp4_kernel<false, false>,
-                    dim3((unsigned)unit_blocks(s, chunks, check_rows)), dim3(kThreads), 0, stream,
-                    static_cast<const uint4 *>(hidden), row_src, pair_slot, global_scale, q,
-                    scales, s.N, s.k, s.rows, s.H, chunks);
+                    dim3((unsigned)unit_blocks(s, chunks, check_rows, ps)), dim3(kThreads), 0,
+                    stream, static_cast<const uint4 *>(hidden), row_src, pair_slot, global_scale,
+                    q, scales, s.N, s.k, s.rows, s.H, chunks, ps);
 }
 
 cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32_t *row_src,
@@ -531,12 +649,21 @@ cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32
   if (s.rows == 0) return cudaSuccess;
   const int32_t chunks = chunks_of(s.H, kChunk);
   const bool swizzled = (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES) != 0;
+  const int32_t ps = padding_split(s, chunks);
+  if (swizzled && atoms_in_place(s.H / 32)) {
+    const cudaError_t err = launch_pdl(
+        permute_fp4_kernel<true, false>, dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)),
+        dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src, pair_slot,
+        static_cast<const float *>(nullptr), q, scales, s.N, s.k, s.rows, s.H, chunks, ps);
+    if (err != cudaSuccess) return err;
+    return launch_scales_to_atoms(s, s.H / 32, scales, stream);
+  }
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
   return launch_pdl(swizzled ? permute_fp4_kernel<true, true> : permute_fp4_kernel<true, false>,
-                    dim3((unsigned)unit_blocks(s, chunks, check_rows)), dim3(kThreads), 0, stream,
-                    static_cast<const uint4 *>(hidden), row_src, pair_slot,
+                    dim3((unsigned)unit_blocks(s, chunks, check_rows, ps)), dim3(kThreads), 0,
+                    stream, static_cast<const uint4 *>(hidden), row_src, pair_slot,
                     static_cast<const float *>(nullptr), q, scales, s.N, s.k, s.rows, s.H,
-                    chunks);
+                    chunks, ps);
 }
 
 }  // namespace moe

@@ -20,12 +20,16 @@ every rank takes them:
   combine_exchange        the expert outputs back along the reverse route, to
                           the rows the dispatch output had, ready for moe_combine
 
-In packed mode a segment's rows are contiguous (meta row 1 is the exclusive
-cumsum), so the split of a send buffer is meta row 0 / H rows per rank; in
-capacity mode ([E, Ce, H], static positions) every segment is its full
-L * Ce rows, padding included.  The collectives are torch.distributed
-all_to_all_single calls (NCCL over NVLink / NVSwitch on GPUs, gloo on CPU);
-the split sizes are read to the host once per exchange_counts.
+In packed mode a segment's rows are contiguous and start at meta row 1 / H
+(the exclusive cumsum of the send counts); in capacity mode ([E, Ce, H],
+static positions) segment s is its full L * Ce rows from s * L * Ce, padding
+included.  The counts exchange is one all_to_all_single and the only step
+that reads sizes to the host.  The payload steps are grouped point-to-point
+transfers (torch.distributed batch_isend_irecv: on GPUs one NCCL group of
+sends and receives over NVLink / NVSwitch, on CPU gloo): for every peer, one
+send straight from the segment's first row (meta row 1) and one receive
+straight into its block of the receive buffer (meta row 3), so no staging
+copy of the send buffer is made; the segment a rank keeps is a local copy.
 """
 from __future__ import annotations
 
@@ -37,9 +41,26 @@ import torch.distributed as dist
 
 @dataclass
 class Route:
-    """Rows this rank sends to and receives from every rank of the group."""
+    """Rows this rank sends to and receives from every rank of the group,
+    and where each segment starts: send_offsets in the dispatch output
+    (meta row 1 / H), recv_offsets in the receive buffer (meta row 3 / H);
+    both default to the exclusive cumsum of the row counts."""
     send_rows: list[int]
     recv_rows: list[int]
+    send_offsets: list[int] | None = None
+    recv_offsets: list[int] | None = None
+
+    def __post_init__(self):
+        def cumsum(rows):
+            out, acc = [], 0
+            for r in rows:
+                out.append(acc)
+                acc += r
+            return out
+        if self.send_offsets is None:
+            self.send_offsets = cumsum(self.send_rows)
+        if self.recv_offsets is None:
+            self.recv_offsets = cumsum(self.recv_rows)
 
     @property
     def recv_total(self) -> int:
@@ -75,16 +96,20 @@ def exchange_counts(meta: torch.Tensor, hidden: int, num_experts: int,
     if expert_capacity > 0:
         seg = (num_experts // S) * expert_capacity
         send_rows = [seg] * S
+        send_offsets = [s * seg for s in range(S)]
         send_elems = torch.full((S,), seg * hidden, dtype=torch.int64, device=meta.device)
     else:
         send_elems = _u32(meta[0]).contiguous()
         send_rows = [int(v) // hidden for v in send_elems.tolist()]
+        send_offsets = [int(v) // hidden for v in _u32(meta[1]).tolist()]
     recv_elems = torch.empty_like(send_elems)
     dist.all_to_all_single(recv_elems, send_elems, group=group)
     displs = torch.cumsum(recv_elems, 0) - recv_elems
     meta[2].copy_(_to_u32_bits(recv_elems))
     meta[3].copy_(_to_u32_bits(displs))
-    return Route(send_rows=send_rows, recv_rows=[int(v) // hidden for v in recv_elems.tolist()])
+    return Route(send_rows=send_rows, recv_rows=[int(v) // hidden for v in recv_elems.tolist()],
+                 send_offsets=send_offsets,
+                 recv_offsets=[int(v) // hidden for v in displs.tolist()])
 
 
 def exchange_expert_counts(expert_counts: torch.Tensor, group=None) -> torch.Tensor:
@@ -103,15 +128,41 @@ def _row_bytes(t: torch.Tensor) -> torch.Tensor:
     return t.contiguous().view(torch.uint8).reshape(t.shape[0], -1)
 
 
+def _grouped_exchange(send: torch.Tensor, send_rows, send_offsets, recv: torch.Tensor,
+                      recv_rows, recv_offsets, group=None) -> None:
+    """Rows [send_offsets[p], +send_rows[p]) of `send` go to rank p, rows
+    [recv_offsets[p], +recv_rows[p]) of `recv` come from rank p: one grouped
+    batch of point-to-point transfers, this rank's own segment copied."""
+    me = dist.get_rank(group)
+    ops = []
+    for peer in range(_world(group)):
+        so, sn = send_offsets[peer], send_rows[peer]
+        ro, rn = recv_offsets[peer], recv_rows[peer]
+        if peer == me:
+            if sn != rn:
+                raise RuntimeError("own segment: send and receive counts differ")
+            recv[ro:ro + rn].copy_(send[so:so + sn])
+            continue
+        dst = peer if group is None else dist.get_global_rank(group, peer)
+        if sn > 0:
+            ops.append(dist.P2POp(dist.isend, send[so:so + sn], dst, group))
+        if rn > 0:
+            ops.append(dist.P2POp(dist.irecv, recv[ro:ro + rn], dst, group))
+    if ops:
+        for req in dist.batch_isend_irecv(ops):
+            req.wait()
+
+
 def dispatch_exchange(rows: torch.Tensor, route: Route, group=None) -> torch.Tensor:
     """Ship segment s of `rows` (the dispatch output, or its code or scale
     rows) to rank s; returns the received rows, source rank by source rank."""
-    if rows.shape[0] < route.send_total:
+    if rows.shape[0] < max((o + n for o, n in zip(route.send_offsets, route.send_rows)),
+                           default=0):
         raise ValueError("fewer rows than the route sends")
-    send = _row_bytes(rows[:route.send_total])
+    send = _row_bytes(rows)
     out = torch.empty((route.recv_total, send.shape[1]), dtype=torch.uint8, device=rows.device)
-    dist.all_to_all_single(out, send, output_split_sizes=route.recv_rows,
-                           input_split_sizes=route.send_rows, group=group)
+    _grouped_exchange(send, route.send_rows, route.send_offsets, out, route.recv_rows,
+                      route.recv_offsets, group)
     return out.view(rows.dtype).reshape((route.recv_total,) + tuple(rows.shape[1:]))
 
 
@@ -124,14 +175,13 @@ def combine_exchange(expert_rows: torch.Tensor, route: Route, out: torch.Tensor 
     (zero-filled when `out` is not given)."""
     if expert_rows.shape[0] != route.recv_total:
         raise ValueError("expert rows do not match the route")
+    end = max((o + n for o, n in zip(route.send_offsets, route.send_rows)), default=0)
     if out is None:
-        out = torch.zeros((route.send_total,) + tuple(expert_rows.shape[1:]),
+        out = torch.zeros((end,) + tuple(expert_rows.shape[1:]),
                           dtype=expert_rows.dtype, device=expert_rows.device)
-    send = _row_bytes(expert_rows)
-    back = torch.empty((route.send_total, send.shape[1]), dtype=torch.uint8,
-                       device=expert_rows.device)
-    dist.all_to_all_single(back, send, output_split_sizes=route.send_rows,
-                           input_split_sizes=route.recv_rows, group=group)
-    out[:route.send_total].copy_(
-        back.view(expert_rows.dtype).reshape((route.send_total,) + tuple(expert_rows.shape[1:])))
+    if out.shape[0] < end or not out.is_contiguous():
+        raise ValueError("out is not a contiguous buffer of the dispatch output's rows")
+    # the reverse route: receive straight into the rows the segments left
+    _grouped_exchange(_row_bytes(expert_rows), route.recv_rows, route.recv_offsets,
+                      _row_bytes(out), route.send_rows, route.send_offsets, group)
     return out

@@ -92,17 +92,25 @@ enum {
 /* Problem flags. */
 enum {
   MOE_FLAG_CHECK_DUPLICATES = 1u,
-  /* Run the layout as two kernels (scan, then emit) even where the one-launch
-   * cooperative kernel applies.  Results are identical; for testing and
-   * tuning. */
+  /* The layout picks one of three equivalent kernels by size: one
+   * thread-block cluster when the pairs fit in at most 16 tiles of 8192
+   * pairs (8 where the device cannot schedule 16-CTA clusters) and the rows
+   * number at most 2^18; else one cooperative launch with a decoupled
+   * look-back scan up to 128 tiles of 4096 pairs; else a scan kernel and an
+   * emit kernel.  These two flags force the latter kernels.  Results are
+   * identical; for testing and tuning. */
   MOE_FLAG_LAYOUT_TWO_PASS = 2u,
   /* moe_permute_quant_nvfp4 writes the E4M3 scales in the block-scale atom
    * layout of NVIDIA block-scaled tensor-core operands instead of row-major
    * (see moe_permute_quant_nvfp4). */
   MOE_FLAG_NVFP4_SWIZZLED_SCALES = 4u,
+  /* Run the layout as the one-launch look-back kernel even where the cluster
+   * kernel applies (see MOE_FLAG_LAYOUT_TWO_PASS). */
+  MOE_FLAG_LAYOUT_LOOKBACK = 8u,
   /* Test hook: the first scan tile never publishes its counts, so every
    * later tile's bounded wait runs out and MOE_STATUS_TIMEOUT is reported.
-   * Results are invalid; used only to test the timeout path. */
+   * Results are invalid; used only to test the timeout path.  Implies the
+   * look-back kernels (the cluster kernel has no bounded wait). */
   MOE_FLAG_TEST_STALL_SCAN = 0x80000000u
 };
 

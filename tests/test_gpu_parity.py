@@ -171,12 +171,18 @@ EDGE = {
 }
 
 
-@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
+# the three layout kernels: chosen by size (the cluster kernel for every
+# case here), the one-launch look-back kernel, the scan + emit kernels
+LAYOUT_PATHS = {"auto": 0, "lookback": B.MOE_FLAG_LAYOUT_LOOKBACK,
+                "two_pass": B.MOE_FLAG_LAYOUT_TWO_PASS}
+
+
+@pytest.mark.parametrize("path", sorted(LAYOUT_PATHS))
 @pytest.mark.parametrize("name", sorted(EDGE))
-def test_edge_case_parity(orc, name, two_pass):
+def test_edge_case_parity(orc, name, path):
     spec = dict(EDGE[name])
     w = custom(seed=zlib.crc32(name.encode()) % 1000, **spec)
-    flags = B.MOE_FLAG_CHECK_DUPLICATES | (B.MOE_FLAG_LAYOUT_TWO_PASS if two_pass else 0)
+    flags = B.MOE_FLAG_CHECK_DUPLICATES | LAYOUT_PATHS[path]
     run = GpuRun(w, flags=flags)
     ref = oracle_layout(orc, w, flags=orc.FLAG_CHECK_DUPLICATES)
     assert_layout(run, ref)
@@ -288,13 +294,30 @@ def test_host_argument_errors():
     assert e.value.code == B.MOE_ERR_UNSUPPORTED_SHAPE
 
 
+@pytest.mark.parametrize("path", ["lookback", "two_pass"])
 @pytest.mark.parametrize("cfg", ["tiny", "mid_zipf", "decode_capacity"])
-def test_two_pass_layout_matches_oracle(orc, cfg):
+def test_other_layout_paths_match_oracle(orc, cfg, path):
     w = make_workload(cfg)
-    run = GpuRun(w, flags=B.MOE_FLAG_LAYOUT_TWO_PASS, quant=False)
+    run = GpuRun(w, flags=LAYOUT_PATHS[path], quant=False)
     ref = oracle_layout(orc, w)
     assert_layout(run, ref)
     assert_all_outputs(orc, w, run, ref)
+
+
+@pytest.mark.parametrize("path", sorted(LAYOUT_PATHS))
+@pytest.mark.parametrize("N,k,E", [(12500, 8, 64), (16384, 8, 256), (8191, 8, 256),
+                                   (8193, 8, 256), (4097, 1, 3)])
+def test_layout_cluster_sizes(orc, N, k, E, path):
+    """Pair counts around the cluster kernel's limits: 8193 pairs (three
+    tiles of 4096), 65528 and 65544 pairs (one tile below and above sixteen
+    tiles of 4096), 100000 and 131072 pairs (tiles of 8192 pairs), with a
+    ragged last tile and masked, out-of-range and duplicate ids."""
+    w = custom(N=N, H=32, E=E, k=k, S=1, seed=N + E, p_mask=0.05, p_bad=0.01,
+               distinct=(N % 2 == 0), with_out=False)
+    flags = B.MOE_FLAG_CHECK_DUPLICATES | LAYOUT_PATHS[path]
+    run = GpuRun(w, flags=flags, quant=False, combine=False)
+    ref = oracle_layout(orc, w, flags=orc.FLAG_CHECK_DUPLICATES)
+    assert_layout(run, ref)
 
 
 def test_cuda_graph_capture_and_replay(orc):
@@ -425,12 +448,12 @@ PAD_EDGE = {
 }
 
 
-@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
+@pytest.mark.parametrize("path", sorted(LAYOUT_PATHS))
 @pytest.mark.parametrize("name", sorted(PAD_EDGE))
-def test_expert_padding_parity(orc, name, two_pass):
+def test_expert_padding_parity(orc, name, path):
     spec, pad = PAD_EDGE[name]
     w = custom(seed=zlib.crc32(name.encode()) % 1000, **spec)
-    flags = B.MOE_FLAG_CHECK_DUPLICATES | (B.MOE_FLAG_LAYOUT_TWO_PASS if two_pass else 0)
+    flags = B.MOE_FLAG_CHECK_DUPLICATES | LAYOUT_PATHS[path]
     run = GpuRun(w, flags=flags, pad=pad)
     ref = oracle_layout(orc, w, flags=orc.FLAG_CHECK_DUPLICATES, pad=pad)
     assert_layout(run, ref)
@@ -467,7 +490,8 @@ def _random_spec(i):
 def test_random_problem_sweep(orc, i):
     spec, pad, two_pass, swizzled = _random_spec(i)
     w = custom(seed=100 + i, **spec)
-    flags = B.MOE_FLAG_CHECK_DUPLICATES | (B.MOE_FLAG_LAYOUT_TWO_PASS if two_pass else 0) | \
+    path = "two_pass" if two_pass else ("lookback", "auto")[i % 2]
+    flags = B.MOE_FLAG_CHECK_DUPLICATES | LAYOUT_PATHS[path] | \
         (B.MOE_FLAG_NVFP4_SWIZZLED_SCALES if swizzled else 0)
     run = GpuRun(w, flags=flags, pad=pad)
     ref = oracle_layout(orc, w, flags=orc.FLAG_CHECK_DUPLICATES, pad=pad)
