@@ -21,7 +21,10 @@ from dataclasses import dataclass
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoedc.so")
+# MOE_LIB_PATH selects another build of the library, e.g. the build with
+# device index checks (libmoedc_debug.so, see moe_debug_violations)
+LIB_PATH = os.environ.get("MOE_LIB_PATH") or os.path.join(_PKG, "libmoedc.so")
+DEBUG_LIB_PATH = os.path.join(_PKG, "libmoedc_debug.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
@@ -48,7 +51,8 @@ EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout",
             "moe_permute_quant_fp8",
             "moe_permute_quant_nvfp4", "moe_permute_quant_mxfp4", "moe_combine",
             "moe_permute_backward",
-            "moe_combine_backward", "moe_swiglu_quant", "moe_status_string", "moe_version")
+            "moe_combine_backward", "moe_swiglu_quant", "moe_status_string", "moe_version",
+            "moe_debug_violations")
 
 (MOE_QUANT_NVFP4, MOE_QUANT_MXFP8, MOE_QUANT_MXFP4, MOE_QUANT_BF16, MOE_QUANT_MXFP6_E2M3,
  MOE_QUANT_MXFP6_E3M2) = 0, 1, 2, 3, 4, 5
@@ -144,6 +148,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     L.moe_status_string.argtypes = [ctypes.c_int]
     L.moe_version.restype = ctypes.c_char_p
     L.moe_version.argtypes = []
+    L.moe_debug_violations.restype = ctypes.c_int64
+    L.moe_debug_violations.argtypes = [ctypes.c_int]
     _lib = L
     return L
 
@@ -154,6 +160,12 @@ def status_string(code: int) -> str:
 
 def version() -> str:
     return load().moe_version().decode()
+
+
+def debug_violations(reset: bool = False) -> int:
+    """Bits of out-of-range indices the device checks recorded (0 = none),
+    or -1 when the loaded build has no checks (see moe_debug_violations)."""
+    return int(load().moe_debug_violations(int(reset)))
 
 
 def _ptr(t: torch.Tensor | None):

@@ -19,6 +19,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libmoedc.so")
+# the same sources with device index checks (-DMOE_DEBUG_CHECKS)
+DEBUG_LIB_PATH = os.path.join(PKG, "libmoedc_debug.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
@@ -42,30 +44,36 @@ def _inputs() -> list[str]:
             + sorted(glob.glob(os.path.join(INCLUDE, "*.h"))) + [os.path.abspath(__file__)])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
+def up_to_date(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return False
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB_PATH
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Build libmoedc.so, or with debug=True libmoedc_debug.so (device index
+    checks, see moe_debug_violations in moe_dc.h)."""
+    path = DEBUG_LIB_PATH if debug else LIB_PATH
+    if not force and up_to_date(path):
+        return path
+    tmp = path + f".tmp{os.getpid()}"
+    cmd = [_nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, *(["-DMOE_DEBUG_CHECKS"] if debug else []),
+           "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, path)
+    return path
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--debug", action="store_true",
+                    help="build libmoedc_debug.so with device index checks")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, debug=a.debug))
     sys.exit(0)

@@ -306,6 +306,24 @@ const char *moe_status_string(moe_status status) {
   }
 }
 
-const char *moe_version(void) { return "moedc 0.1.0 (sm_100a)"; }
+const char *moe_version(void) {
+#ifdef MOE_DEBUG_CHECKS
+  return "moedc 0.2.0 (sm_100a, device index checks)";
+#else
+  return "moedc 0.2.0 (sm_100a)";
+#endif
+}
+
+int64_t moe_debug_violations(int reset) {
+#ifdef MOE_DEBUG_CHECKS
+  return (int64_t)(moe::debug_violations_layout(reset != 0) |
+                   moe::debug_violations_permute(reset != 0) |
+                   moe::debug_violations_combine(reset != 0) |
+                   moe::debug_violations_swiglu(reset != 0));
+#else
+  (void)reset;
+  return -1;
+#endif
+}
 
 }  // extern "C"

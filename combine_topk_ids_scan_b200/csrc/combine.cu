@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
       const int32_t s = __shfl_sync(kFull, my_slot, j);
-      row[j] = s;
+      row[j] = s >= 0 && MOE_IN_RANGE(s, rows, kDbgCombineRow) ? s : -1;
       w[j] = __shfl_sync(kFull, my_w, j);
     }
     uint4 *dst = out + t * vecs;
@@ -133,7 +133,8 @@ __global__ void __launch_bounds__(kThreads)
     float w[KMAX], dot[KMAX];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
-      row[j] = __shfl_sync(kFull, my_slot, j);
+      const int32_t s = __shfl_sync(kFull, my_slot, j);
+      row[j] = s >= 0 && MOE_IN_RANGE(s, rows, kDbgCombineRow) ? s : -1;
       w[j] = __shfl_sync(kFull, my_w, j);
       dot[j] = 0.0f;
     }
@@ -232,6 +233,8 @@ cudaError_t launch_forward(const Shape &s, const uint4 *x, const float *gates,
 }
 
 }  // namespace
+
+uint32_t debug_violations_combine(bool reset) { return read_debug_violations(reset); }
 
 cudaError_t launch_combine_backward(const Shape &s, const void *grad_y, const void *expert_out,
                                     const float *gates, const int32_t *pair_slot,

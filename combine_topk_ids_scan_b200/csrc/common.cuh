@@ -10,6 +10,43 @@ namespace moe {
 
 constexpr int kWarp = 32;
 
+// ---------------------------------------------------------------- debug build
+// Built with -DMOE_DEBUG_CHECKS (libmoedc_debug.so), the kernels check every
+// computed row index and scale offset before they use it: an index outside
+// its buffer ORs the check's bit into this translation unit's debug word and
+// the access is skipped (no trap: the context stays usable), and
+// moe_debug_violations() reports the bits.  In normal builds the checks
+// compile to nothing.
+enum : uint32_t {
+  kDbgLayoutRow = 1u,    // a pair's row in the layout's row_src
+  kDbgPermuteRow = 2u,   // a permute's destination row
+  kDbgScaleOffset = 4u,  // a block-scale byte in the atom layout
+  kDbgCombineRow = 8u,   // a combine / backward source row
+  kDbgSwigluRow = 16u,   // a SwiGLU row
+};
+#ifdef MOE_DEBUG_CHECKS
+static __device__ uint32_t g_debug_violations;  // one per translation unit
+__device__ __forceinline__ bool debug_in_range(int64_t i, int64_t n, uint32_t bit) {
+  if (i >= 0 && i < n) return true;
+  atomicOr(&g_debug_violations, bit);
+  return false;
+}
+// This translation unit's debug word (and zero it when `reset`); host only.
+static inline uint32_t read_debug_violations(bool reset) {
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_debug_violations, sizeof(v)) != cudaSuccess) return ~0u;
+  if (reset) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_debug_violations, &zero, sizeof(zero)) != cudaSuccess) return ~0u;
+  }
+  return v;
+}
+#define MOE_IN_RANGE(i, n, bit) ::moe::debug_in_range((int64_t)(i), (int64_t)(n), (bit))
+#else
+static inline uint32_t read_debug_violations(bool) { return 0u; }
+#define MOE_IN_RANGE(i, n, bit) true
+#endif
+
 // Programmatic dependent launch (sm_90 and later).  The library's kernels
 // after the first of a step are launched with programmatic stream
 // serialisation allowed (launch_pdl in internal.h), so their CTAs may be

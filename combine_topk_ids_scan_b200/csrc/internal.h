@@ -78,6 +78,13 @@ cudaError_t launch_swiglu_quant(const Shape &s, int32_t I, uint32_t format, bool
                                 const float *global_scale, uint8_t *codes, uint8_t *scales,
                                 cudaStream_t stream);
 
+// Each kernel file's debug word (MOE_DEBUG_CHECKS builds; 0 otherwise),
+// zeroed when `reset`.
+uint32_t debug_violations_layout(bool reset);
+uint32_t debug_violations_permute(bool reset);
+uint32_t debug_violations_combine(bool reset);
+uint32_t debug_violations_swiglu(bool reset);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 

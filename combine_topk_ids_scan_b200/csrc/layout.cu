@@ -517,7 +517,7 @@ __device__ void emit_step(const LayoutArgs &a, int64_t gtid, int64_t gstride,
       slot = row_of(e, __ldcg(a.pair_slot + p), s_off, a.C, a.Ce, capacity, dropped, bits);
     a.pair_slot[p] = slot;
     if (a.drop_mask) a.drop_mask[p] = dropped;
-    if (slot >= 0) a.row_src[slot] = (int32_t)p / a.k;
+    if (slot >= 0 && MOE_IN_RANGE(slot, a.rows, kDbgLayoutRow)) a.row_src[slot] = (int32_t)p / a.k;
   }
   emit_common<THREADS>(gtid, gstride, a.rows, a.E, a.S, a.Ce, a.pad, a.H, s_off, s_kept,
                        a.row_src, blockIdx.x == 0, a.expert_counts, a.expert_offsets, a.meta);
@@ -640,7 +640,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) layout_cluster_kernel(LayoutA
       }
       a.pair_slot[p] = slot;
       if (a.drop_mask) a.drop_mask[p] = dropped;
-      if (slot >= 0) a.row_src[slot] = (int32_t)(p / a.k);
+      if (slot >= 0 && MOE_IN_RANGE(slot, a.rows, kDbgLayoutRow))
+        a.row_src[slot] = (int32_t)(p / a.k);
     }
   }
   const int64_t gtid = (int64_t)c * kScanThreads + tid;
@@ -758,6 +759,8 @@ int fused_capacity(size_t smem) {
 }
 
 }  // namespace
+
+uint32_t debug_violations_layout(bool reset) { return read_debug_violations(reset); }
 
 int32_t layout_num_tiles(int64_t P) { return (int32_t)((P + kTilePairs - 1) / kTilePairs); }
 

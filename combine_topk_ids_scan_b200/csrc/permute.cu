@@ -120,7 +120,9 @@ __global__ void __launch_bounds__(kThreads)
     while (live) {
       const int j = __ffs(live) - 1;
       live &= live - 1;
-      uint4 *dst = out + (int64_t)__shfl_sync(kFull, my_slot, j) * vecs;
+      const int64_t s = __shfl_sync(kFull, my_slot, j);
+      if (!MOE_IN_RANGE(s, rows, kDbgPermuteRow)) continue;
+      uint4 *dst = out + s * vecs;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int v = v0 + u * kWarp + lane;
@@ -184,7 +186,9 @@ __global__ void __launch_bounds__(kThreads)
     const int j = __ffs(live) - 1;
     live &= live - 1;
     const float g = __shfl_sync(kFull, my_w, j);
-    uint4 *dst = out + (int64_t)__shfl_sync(kFull, my_slot, j) * vecs;
+    const int64_t s = __shfl_sync(kFull, my_slot, j);
+    if (!MOE_IN_RANGE(s, rows, kDbgPermuteRow)) continue;
+    uint4 *dst = out + s * vecs;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int v = v0 + u * kWarp + lane;
@@ -283,6 +287,7 @@ __global__ void __launch_bounds__(kThreads)
       const int j = __ffs(live) - 1;
       live &= live - 1;
       const int64_t s = __shfl_sync(kFull, my_slot, j);
+      if (!MOE_IN_RANGE(s, rows, kDbgPermuteRow)) continue;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int col = c0 + u * 512 + lane * 16;
@@ -361,12 +366,14 @@ __device__ __forceinline__ int64_t sf_atom_offset(int64_t m, int32_t c, int32_t 
 
 // MX == false: NVFP4 (two 16-element blocks per lane, E4M3 scales);
 // MX == true: MXFP4 (one 32-element block per lane, E8M0 scales).
-// SWIZZLED: scales in the block-scale atom layout.  The linear-scale kernels
-// are held to 5 resident CTAs per SM (at most 48 registers; measured on B200
-// at the metric shape: NVFP4 74 -> 70 us, MXFP4 61.4 -> 60.0 us), the
-// atom-layout kernels to 4 (with 5 they were slower).
+// SWIZZLED: scales in the block-scale atom layout.  The token row's loads
+// are issued first, before the pair_slot load and its ballot.  The MXFP4
+// linear-scale kernel is held to 5 resident CTAs per SM (at most 48
+// registers; measured on B200 at the metric shape: 61.4 -> 60.0 us), the
+// NVFP4 and the atom-layout kernels to 4 (NVFP4 with its loads first: 65.5 us
+// at 5 CTAs with a 4-byte spill, 63.5 us at 4 without one).
 template <bool MX, bool SWIZZLED>
-__global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
+__global__ void __launch_bounds__(kThreads, (SWIZZLED || !MX) ? 4 : 5)
     permute_fp4_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                        const int32_t *__restrict__ pair_slot,
                        const float *__restrict__ global_scale, uint8_t *__restrict__ q,
@@ -425,8 +432,11 @@ __global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
           uint4 *dst = reinterpret_cast<uint4 *>(q) + row * (qrow / 16);
           for (int v = v0 + lane; v < v1; v += kWarp) st_v4(dst + v, zero);
         }
-        for (int gg = g0 + lane; gg < g1; gg += kWarp)
-          st_u32_evict_last(scales + sf_atom_offset(row, 4 * gg, groups), 0u);
+        for (int gg = g0 + lane; gg < g1; gg += kWarp) {
+          const int64_t off = sf_atom_offset(row, 4 * gg, groups);
+          if (MOE_IN_RANGE(off, check_rows * groups * 4, kDbgScaleOffset))
+            st_u32_evict_last(scales + off, 0u);
+        }
       }
     }
     return;
@@ -437,20 +447,20 @@ __global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
     const int64_t t = w / chunks;
     const int col = (int)(w % chunks) * kChunk + lane * 32;
     const bool active = col < H;
-    int32_t my_slot;
-    uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
-    const float gs = MX ? 0.0f : __ldg(global_scale);
     const uint4 *src = hidden + t * vecs;
     uint4 x[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       x[i] = active ? ld_stream_v4(src + col / 8 + i) : make_uint4(0, 0, 0, 0);
+    int32_t my_slot;
+    uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+    const float gs = MX ? 0.0f : __ldg(global_scale);
     // x[i] holds the lane's elements 8i..8i+7.  MXFP4 unpacks its one
     // 32-element block; NVFP4 unpacks one 16-element block at a time, so
     // that only 16 floats are live (under the 5-CTA bound the 32-float form
     // spilled 40 bytes per thread: 7 local stores and 10 local loads per
-    // unit, now 1 and 4; measured on B200 at the metric shape:
-    // 71.5 -> 69.0 us)
+    // unit, now 1 and 4, and none at 4 CTAs per SM; measured on B200 at the
+    // metric shape: 71.5 -> 69.0 us)
     float f[MX ? 32 : 16];
     const auto unpack = [&](int i0, int n) {
 #pragma unroll
@@ -491,13 +501,15 @@ __global__ void __launch_bounds__(kThreads, SWIZZLED ? 4 : 5)
       const int j = __ffs(live) - 1;
       live &= live - 1;
       const int64_t s = __shfl_sync(kFull, my_slot, j);
-      if (active) {
+      if (active && MOE_IN_RANGE(s, rows, kDbgPermuteRow)) {
         st_v4(reinterpret_cast<uint4 *>(q + s * qrow + col / 2), codes);
         if (!swizzled) {
           if (MX) scales[s * srow + sc_col] = (uint8_t)sq;
           else *reinterpret_cast<uint16_t *>(scales + s * srow + sc_col) = (uint16_t)sq;
         } else if ((lane & (MX ? 3 : 1)) == 0) {
-          st_u32_evict_last(scales + sf_atom_offset(s, sc_col, groups), quad);
+          const int64_t off = sf_atom_offset(s, sc_col, groups);
+          if (MOE_IN_RANGE(off, check_rows * groups * 4, kDbgScaleOffset))
+            st_u32_evict_last(scales + off, quad);
         }
       }
     }
@@ -567,6 +579,8 @@ inline int64_t unit_blocks(const Shape &s, int32_t chunks, int64_t check_rows, i
 inline int32_t chunks_of(int32_t H, int32_t chunk) { return (H + chunk - 1) / chunk; }
 
 }  // namespace
+
+uint32_t debug_violations_permute(bool reset) { return read_debug_violations(reset); }
 
 cudaError_t launch_permute_bf16(const Shape &s, const void *hidden, const int32_t *row_src,
                                 const int32_t *pair_slot, void *out, cudaStream_t stream) {

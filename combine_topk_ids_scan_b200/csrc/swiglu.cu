@@ -575,7 +575,9 @@ __global__ void __launch_bounds__(kThreads, FORMAT == 1 ? 4 : 3)
   int64_t w = (int64_t)blockIdx.x * (kThreads / kWarp) + threadIdx.x / kWarp;
   int64_t row = w / U;
   int32_t cu = (int32_t)(w - row * U);
+  const int64_t rows = units / U;
   for (; w < units; w += warps) {
+    if (!MOE_IN_RANGE(row, rows, kDbgSwigluRow)) break;
     const bool live = __ldg(row_src + row) >= 0;  // no routed token: zero bytes
     if (INTERLEAVED)
       swiglu_unit_interleaved<FORMAT>(tab, gate_up, live, codes, scales, row, cu * kUnitCols, I,
@@ -617,7 +619,9 @@ __global__ void __launch_bounds__(kThreads, 3)
   int64_t t = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   int64_t row = t / G;
   int32_t cg = (int32_t)(t - row * G);
+  const int64_t rows = groups / G;
   for (; t < groups; t += stride) {
+    if (!MOE_IN_RANGE(row, rows, kDbgSwigluRow)) break;
     swiglu_group<FORMAT, INTERLEAVED>(tab, gate_up, row_src, gs, codes, scales, row,
                                       cg * kGroupCols, I);
     row += step_rows;
@@ -666,6 +670,8 @@ cudaError_t launch(const uint4 *in, const int32_t *row_src, const float *gs, uin
 }
 
 }  // namespace
+
+uint32_t debug_violations_swiglu(bool reset) { return read_debug_violations(reset); }
 
 cudaError_t launch_swiglu_quant(const Shape &s, int32_t I, uint32_t format, bool interleaved,
                                 const void *gate_up, const int32_t *row_src,

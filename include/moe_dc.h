@@ -425,6 +425,17 @@ MOE_API moe_status moe_combine_backward(const moe_problem *problem, const void *
                                         void *grad_expert_out, float *grad_gates,
                                         moe_stream_t stream);
 
+/* Device index checks.  A build with -DMOE_DEBUG_CHECKS
+ * (`python -m combine_topk_ids_scan_b200.build --debug`, libmoedc_debug.so)
+ * checks every computed row index and block-scale offset in its kernels
+ * before use; an out-of-range one is skipped and recorded (no trap).  Returns
+ * the OR of the bits recorded on the current device since the last reset
+ * (1 layout row, 2 permute destination row, 4 atom-layout scale offset,
+ * 8 combine source row, 16 SwiGLU row; 0 = none), zeroing them when `reset`
+ * is non-zero; synchronises with the device.  Returns -1 from a build
+ * without the checks (no CUDA call is made then). */
+MOE_API int64_t moe_debug_violations(int reset);
+
 /* Static description of a moe_status value. */
 MOE_API const char *moe_status_string(moe_status status);
 

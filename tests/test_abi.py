@@ -50,6 +50,7 @@ def test_built_for_sm100a(lib):
 
 def test_host_only_entry_points(lib):
     assert B.version().startswith("moedc")
+    assert B.debug_violations() == -1          # the normal build has no device checks
     assert "invalid" in B.status_string(B.MOE_ERR_INVALID_ARG)
     p = B.Problem(num_tokens=8192, hidden=7168, num_experts=256, top_k=8, num_segments=8,
                   recv_capacity=65536)
