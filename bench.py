@@ -549,16 +549,21 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
         d_gx = torch.empty_like(d_x)
         d_gw = torch.empty_like(d_gates)
         f4_steps = max(10, args.steps // 10)
-        pb_us, cb_us = time_phases(
+        pb_us, cb_us, pm_us = time_phases(
             [lambda: B.moe_permute_backward(prob, d_grows, buf.pair_slot, d_gh),
              lambda: B.moe_combine_backward(prob, d_gtok, d_x, d_gates, buf.pair_slot,
-                                            buf.row_src, d_gx, d_gw)],
+                                            buf.row_src, d_gx, d_gw),
+             lambda: B.moe_permute_premultiplied(prob, d_hidden, buf.row_src, buf.pair_slot,
+                                                 d_gates, d_gx)],
             f4_steps)
         rows = buf.rows
         pb_bytes = 2 * total_rows * w.H + 4 * w.P + 2 * w.N * w.H
         cb_bytes = (2 * w.N * w.H + 2 * 2 * total_rows * w.H + 2 * (rows - total_rows) * w.H
                     + 4 * w.P * 3 + 4 * rows)
+        pm_bytes = 2 * w.N * w.H + 4 * w.P + 4 * rows + 4 * w.P + 2 * rows * w.H
         f4 = {"steps": f4_steps,
+              "permute_premultiplied_us": round(pm_us, 2),
+              "permute_premultiplied_gbs": round(pm_bytes / (pm_us * 1e-6) / 1e9, 1),
               "permute_backward_us": round(pb_us, 2),
               "permute_backward_gbs": round(pb_bytes / (pb_us * 1e-6) / 1e9, 1),
               "combine_backward_us": round(cb_us, 2),

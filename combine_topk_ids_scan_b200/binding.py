@@ -48,6 +48,7 @@ MOE_MAX_TOPK = 16
 # every symbol include/moe_dc.h declares
 EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout",
             "moe_dispatch_layout_noalloc", "moe_permute", "moe_permute_premultiplied",
+            "moe_permute_to_peers",
             "moe_permute_quant_fp8",
             "moe_permute_quant_nvfp4", "moe_permute_quant_mxfp4", "moe_combine",
             "moe_permute_backward",
@@ -127,6 +128,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     L.moe_dispatch_layout_noalloc.argtypes = [P] + [vp] * 9
     L.moe_permute.restype = ctypes.c_int
     L.moe_permute.argtypes = [P] + [vp] * 5
+    L.moe_permute_to_peers.restype = ctypes.c_int
+    L.moe_permute_to_peers.argtypes = [P] + [vp] * 7
     L.moe_permute_premultiplied.restype = ctypes.c_int
     L.moe_permute_premultiplied.argtypes = [P] + [vp] * 6
     L.moe_permute_quant_fp8.restype = ctypes.c_int
@@ -271,6 +274,22 @@ def moe_permute(prob: Problem, hidden_states, row_src, pair_slot, out, stream=No
     c = prob.c()
     _check(load().moe_permute(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
                               _ptr(pair_slot), _ptr(out), _stream(stream)), "moe_permute")
+
+
+def moe_permute_to_peers(prob: Problem, hidden_states, row_src, pair_slot, meta, peer_out,
+                         put_offsets, stream=None) -> None:
+    """Dispatch permute whose segment s lands in rank s's receive buffer:
+    peer_out is an int64 device tensor of S device addresses (e.g.
+    [t.data_ptr() for t in receive buffers]), put_offsets an int64 device
+    tensor of S first rows (see moe_permute_to_peers in moe_dc.h)."""
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_permute_to_peers", **_permute_need(prob, hidden_states, row_src, pair_slot),
+             meta=(meta, 16 * S), peer_out=(peer_out, 8 * S), put_offsets=(put_offsets, 8 * S))
+    c = prob.c()
+    _check(load().moe_permute_to_peers(ctypes.byref(c), _ptr(hidden_states), _ptr(row_src),
+                                       _ptr(pair_slot), _ptr(meta), _ptr(peer_out),
+                                       _ptr(put_offsets), _stream(stream)),
+           "moe_permute_to_peers")
 
 
 def moe_permute_premultiplied(prob: Problem, hidden_states, row_src, pair_slot, gates, out,

@@ -136,6 +136,26 @@ moe_status moe_permute(const moe_problem *problem, const void *hidden_states,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_permute_to_peers(const moe_problem *problem, const void *hidden_states,
+                                const int32_t *row_src, const int32_t *pair_slot,
+                                const uint32_t *meta, void *const *peer_out,
+                                const int64_t *put_offsets, moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.rows == 0) return MOE_OK;
+  if (!row_src || !peer_out || !put_offsets || (s.Ce == 0 && !meta) ||
+      (s.P > 0 && (!hidden_states || !pair_slot)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(hidden_states, 16) || !aligned(row_src, 4) || !aligned(pair_slot, 4) ||
+      !aligned(meta, 4) || !aligned(peer_out, 8) || !aligned(put_offsets, 8))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_permute_to_peers(s, hidden_states, row_src, pair_slot, meta,
+                                                peer_out, put_offsets,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_permute_premultiplied(const moe_problem *problem, const void *hidden_states,
                                      const int32_t *row_src, const int32_t *pair_slot,
                                      const float *gates, void *out, moe_stream_t stream) {

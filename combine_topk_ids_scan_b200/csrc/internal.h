@@ -48,6 +48,11 @@ cudaError_t launch_layout(const Shape &s, const int32_t *ids, int32_t *expert_co
 cudaError_t launch_permute_bf16(const Shape &s, const void *hidden, const int32_t *row_src,
                                 const int32_t *pair_slot, void *out, cudaStream_t stream);
 
+cudaError_t launch_permute_to_peers(const Shape &s, const void *hidden, const int32_t *row_src,
+                                    const int32_t *pair_slot, const uint32_t *meta,
+                                    void *const *peer_out, const int64_t *put_offsets,
+                                    cudaStream_t stream);
+
 cudaError_t launch_permute_premultiplied(const Shape &s, const void *hidden,
                                          const int32_t *row_src, const int32_t *pair_slot,
                                          const float *gates, void *out, cudaStream_t stream);

@@ -55,6 +55,7 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // every bounded wait: 1 s
 constexpr int kLookWindow = 8;                    // predecessor tiles per poll
 constexpr int kFusedMaxTiles = 128;               // last CTA clears <= 128*E words
 constexpr int64_t kClusterMaxRows = 1 << 18;      // cluster path: rows per launch
+constexpr int kClusterMax = 16;                   // largest cluster the path uses
 
 constexpr int kEmitThreads = 256;
 
@@ -358,7 +359,8 @@ __device__ void emit_common(int64_t r0, int64_t stride, int64_t rows, int32_t E,
   for (int64_t r = r0; r < rows; r += stride) {
     bool pad;
     if (capacity) {
-      pad = (int32_t)(r % Ce) >= s_kept[r / Ce];
+      const int32_t r32 = (int32_t)r;  // rows < 2^31 (host check)
+      pad = r32 % Ce >= s_kept[r32 / Ce];
     } else if (r >= (int64_t)s_off[E]) {
       pad = true;
     } else if (pad_multiple > 1) {
@@ -611,11 +613,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) layout_cluster_kernel(LayoutA
   int32_t *s_off = s_excl + E;       // [E + 1]
   int32_t *s_kept = s_off + E + 1;   // [E]: the totals, then the kept rows
   for (int e = tid; e < E; e += kScanThreads) {
+    // all of the cluster's remote loads in flight at once
+    uint32_t v[kClusterMax];
+#pragma unroll
+    for (int q = 0; q < kClusterMax; ++q)
+      v[q] = q < nc ? *cluster.map_shared_rank(sm.tile_prefix + e, q) : 0u;
     uint32_t excl = 0, tot = 0;
-    for (int q = 0; q < nc; ++q) {
-      const uint32_t v = *cluster.map_shared_rank(sm.tile_prefix + e, q);
-      excl += q < c ? v : 0u;
-      tot += v;
+#pragma unroll
+    for (int q = 0; q < kClusterMax; ++q) {
+      excl += q < c ? v[q] : 0u;
+      tot += v[q];
     }
     s_excl[e] = (int32_t)excl;
     s_kept[e] = (int32_t)tot;
@@ -658,6 +665,21 @@ __global__ void __launch_bounds__(kScanThreads, 1) layout_cluster_kernel(LayoutA
   if (c == 0 && tid == 0) *a.status_out = s_status;
 }
 
+// The cluster kernel's instantiations: pairs per lane 1, 2, 4, 8, 16.
+constexpr int kClusterRounds[5] = {1, 2, 4, 8, 16};
+inline const void *const *cluster_kernels() {
+  static const void *const k[5] = {
+      (const void *)layout_cluster_kernel<1>, (const void *)layout_cluster_kernel<2>,
+      (const void *)layout_cluster_kernel<4>, (const void *)layout_cluster_kernel<8>,
+      (const void *)layout_cluster_kernel<16>};
+  return k;
+}
+struct ClusterKernelList {
+  const void *const *begin() const { return cluster_kernels(); }
+  const void *const *end() const { return cluster_kernels() + 5; }
+};
+inline ClusterKernelList cluster_kernel_list() { return {}; }
+
 // Opt the scan kernels in to more than 48 KB of dynamic shared memory, once
 // per device.
 cudaError_t opt_in_smem() {
@@ -672,12 +694,9 @@ cudaError_t opt_in_smem() {
   if (err == cudaSuccess)
     err = cudaFuncSetAttribute(layout_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bytes);
-  if (err == cudaSuccess)
-    err = cudaFuncSetAttribute(layout_cluster_kernel<kScanRounds>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (err == cudaSuccess)
-    err = cudaFuncSetAttribute(layout_cluster_kernel<2 * kScanRounds>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  for (const void *kern : cluster_kernel_list())
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (err == cudaSuccess && dev < kMaxDevices) done[dev].store(true);
   return err;
 }
@@ -696,11 +715,9 @@ int max_cluster_size() {
   if (opt_in_smem() != cudaSuccess) return 0;
   int best = 0;
   const int bytes = (int)scan_smem_bytes(MOE_MAX_EXPERTS);
-  const void *kernels[2] = {(const void *)layout_cluster_kernel<kScanRounds>,
-                            (const void *)layout_cluster_kernel<2 * kScanRounds>};
   for (int size : {16, 8}) {
     bool ok = true;
-    for (const void *kern : kernels) {
+    for (const void *kern : cluster_kernel_list()) {
       if (size > 8 &&
           cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
               cudaSuccess) {
@@ -733,7 +750,7 @@ int max_cluster_size() {
 }
 
 template <int ROUNDS>
-cudaError_t launch_cluster(const LayoutArgs &a, int nc, size_t smem, cudaStream_t stream) {
+cudaError_t launch_cluster_t(const LayoutArgs &a, int nc, size_t smem, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nc);
   cfg.blockDim = dim3(kScanThreads);
@@ -747,6 +764,17 @@ cudaError_t launch_cluster(const LayoutArgs &a, int nc, size_t smem, cudaStream_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, layout_cluster_kernel<ROUNDS>, a);
+}
+
+cudaError_t launch_cluster(int rounds, const LayoutArgs &a, int nc, size_t smem,
+                           cudaStream_t stream) {
+  switch (rounds) {
+    case 1: return launch_cluster_t<1>(a, nc, smem, stream);
+    case 2: return launch_cluster_t<2>(a, nc, smem, stream);
+    case 4: return launch_cluster_t<4>(a, nc, smem, stream);
+    case 8: return launch_cluster_t<8>(a, nc, smem, stream);
+    default: return launch_cluster_t<16>(a, nc, smem, stream);
+  }
 }
 
 // Largest grid of the fused kernel that is guaranteed co-resident.
@@ -815,20 +843,20 @@ cudaError_t launch_layout(const Shape &s, const int32_t *ids, int32_t *expert_co
   }
 
   // One cluster when the pairs fit in at most max_cluster_size() tiles of
-  // 4096 (or 8192) pairs and the rows in a few passes of its threads.
+  // 512 * 16 pairs and the rows in a few passes of its threads; the fewest
+  // pairs per lane (1, 2, 4, 8 or 16) that fit, so that the ranking rounds,
+  // the serial part of a tile, stay short.
   const uint32_t forced = MOE_FLAG_LAYOUT_TWO_PASS | MOE_FLAG_LAYOUT_LOOKBACK |
                           MOE_FLAG_TEST_STALL_SCAN;
   if (!(s.flags & forced) && s.rows <= kClusterMaxRows) {
     const int maxc = max_cluster_size();
-    const int64_t t8 = std::max<int64_t>(1, (s.P + kTilePairs - 1) / kTilePairs);
-    const int64_t t16 = std::max<int64_t>(1, (s.P + 2 * kTilePairs - 1) / (2 * kTilePairs));
-    if (maxc > 0 && t8 <= maxc) {
-      if (opt_in_smem() != cudaSuccess) return cudaErrorUnknown;
-      return launch_cluster<kScanRounds>(a, (int)t8, smem, stream);
-    }
-    if (maxc > 0 && t16 <= maxc) {
-      if (opt_in_smem() != cudaSuccess) return cudaErrorUnknown;
-      return launch_cluster<2 * kScanRounds>(a, (int)t16, smem, stream);
+    for (int rounds : kClusterRounds) {
+      const int64_t per_tile = (int64_t)kScanThreads * rounds;
+      const int64_t tiles = std::max<int64_t>(1, (s.P + per_tile - 1) / per_tile);
+      if (maxc > 0 && tiles <= maxc) {
+        if (opt_in_smem() != cudaSuccess) return cudaErrorUnknown;
+        return launch_cluster(rounds, a, (int)tiles, smem, stream);
+      }
     }
   }
 

@@ -133,6 +133,111 @@ __global__ void __launch_bounds__(kThreads)
 
 }
 
+// ------------------------------------------------------- dispatch to peers
+// Expert-parallel dispatch with the send step fused into the permute: the
+// rows of segment s (experts [sL, (s+1)L): local rows [start_s, start_s +
+// rows_s)) are stored straight into rank s's receive buffer peer_out[s] at
+// rows put[s] + (r - start_s), instead of into a local send buffer that an
+// all-to-all then ships.  peer_out[s] is any device pointer this GPU can
+// store to (a peer mapping over NVLink / NVSwitch, or this rank's own buffer
+// for its own segment).  The bf16 permute's units; a lane holding pair j
+// finds its row's segment by binary search over the segment starts (staged
+// in shared memory) and the warp broadcasts the destination row.  Padding
+// rows inside a segment are zeroed at the destination; rows past the last
+// segment are not sent.
+__device__ __forceinline__ int segment_of(int64_t r, const int32_t *s_start,
+                                          const int32_t *s_rows, int32_t S) {
+  int lo = 0, hi = S - 1;
+  while (lo < hi) {  // last s with start[s] <= r
+    const int mid = (lo + hi + 1) / 2;
+    if (s_start[mid] <= r) lo = mid;
+    else hi = mid - 1;
+  }
+  return (r >= s_start[lo] && r - s_start[lo] < s_rows[lo]) ? lo : -1;
+}
+
+// Destination of local row r (nullptr when r belongs to no segment).
+__device__ __forceinline__ uint4 *peer_row(int64_t r, const int32_t *s_start,
+                                           const int32_t *s_rows, int32_t S,
+                                           uint4 *const *__restrict__ peer_out,
+                                           const int64_t *__restrict__ put, int32_t vecs) {
+  const int sg = segment_of(r, s_start, s_rows, S);
+  if (sg < 0) return nullptr;
+  return peer_out[sg] + (put[sg] + (r - s_start[sg])) * (int64_t)vecs;
+}
+
+__global__ void __launch_bounds__(kThreads)
+    permute_to_peers_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
+                            const int32_t *__restrict__ pair_slot,
+                            const uint32_t *__restrict__ meta, uint4 *const *__restrict__ peer_out,
+                            const int64_t *__restrict__ put, int32_t N, int32_t k, int64_t rows,
+                            int32_t vecs, int32_t chunks, int32_t psplit, int32_t S, int32_t H,
+                            int32_t static_seg_rows) {
+  allow_dependents();
+  extern __shared__ int32_t seg_smem[];  // [S] starts, [S] rows
+  int32_t *s_start = seg_smem, *s_rows = seg_smem + S;
+  grid_dependency_wait();
+  // segments: packed mode from meta rows 0-1 (elements), capacity mode the
+  // static blocks of L * Ce rows
+  for (int i = threadIdx.x; i < S; i += kThreads) {
+    if (static_seg_rows > 0) {
+      s_start[i] = i * static_seg_rows;
+      s_rows[i] = static_seg_rows;
+    } else {
+      s_start[i] = (int32_t)(__ldg(meta + S + i) / (uint32_t)H);
+      s_rows[i] = (int32_t)(__ldg(meta + i) / (uint32_t)H);
+    }
+  }
+  __syncthreads();
+  constexpr int U = kBf16Chunk / 8 / kWarp;  // 2
+  const int lane = threadIdx.x % kWarp;
+  const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
+  const int64_t units = (int64_t)N * chunks;
+  const int64_t pad_units = (rows + kWarp - 1) / kWarp * psplit;
+  if (w0 < pad_units) {
+    const int64_t g = w0 / psplit;
+    uint32_t m = padding_mask(g, lane, row_src, rows, rows);
+    int32_t v0, v1;
+    share_of((int)(w0 % psplit), psplit, vecs, v0, v1);
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    while (m) {
+      const int j = __ffs(m) - 1;
+      m &= m - 1;
+      uint4 *dst = peer_row(g * kWarp + j, s_start, s_rows, S, peer_out, put, vecs);
+      if (dst)
+        for (int v = v0 + lane; v < v1; v += kWarp) st_v4(dst + v, zero);
+    }
+    return;
+  }
+  const int64_t w = w0 - pad_units;
+  if (w >= units) return;
+  const int64_t t = w / chunks;
+  const int v0 = (int)(w % chunks) * (kBf16Chunk / 8);
+  const uint4 *src = hidden + t * vecs;
+  uint4 x[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int v = v0 + u * kWarp + lane;
+    if (v < vecs) x[u] = ld_stream_v4(src + v);
+  }
+  int32_t my_slot;
+  const uint32_t live_rows = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+  uint4 *my_dst = my_slot >= 0 ? peer_row(my_slot, s_start, s_rows, S, peer_out, put, vecs)
+                               : nullptr;
+  uint32_t live = live_rows & __ballot_sync(kFull, my_dst != nullptr);
+  while (live) {
+    const int j = __ffs(live) - 1;
+    live &= live - 1;
+    uint4 *dst = reinterpret_cast<uint4 *>(
+        __shfl_sync(kFull, reinterpret_cast<unsigned long long>(my_dst), j));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + u * kWarp + lane;
+      if (v < vecs) st_v4(dst + v, x[u]);
+    }
+  }
+}
+
 // --------------------------------------------------- pre-multiplied gates
 // DeepSpeed's pre-multiplication of the token representations by their
 // router scores before expert compute: the bf16 permute's units, but pair
@@ -535,6 +640,12 @@ inline size_t atom_tile_smem(int32_t nsf) {
   return (size_t)(nsf / 4) * kAtomGroupWords * sizeof(uint32_t);
 }
 
+// VEC: the buffer is 16-byte aligned, and the tile moves as 16-byte vectors
+// (4 words of one row / of one atom row), kAtomBatch loads in flight per
+// thread before their shared-memory stores; else as 4-byte words.
+constexpr int kAtomBatch = 8;
+
+template <bool VEC>
 __global__ void __launch_bounds__(kAtomThreads)
     scales_to_atoms_kernel(uint32_t *__restrict__ scales, int64_t rows, int32_t groups) {
   allow_dependents();
@@ -545,15 +656,50 @@ __global__ void __launch_bounds__(kAtomThreads)
   const int32_t nrows = left < 128 ? (int32_t)left : 128;
   uint32_t *base = scales + tile * 128 * groups;  // the tile's words (either layout)
   const int32_t words = 128 * groups;
-  for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) {
+  const auto put = [&](int32_t w, uint32_t v) {  // linear word w -> shared, atom order
     const int32_t m = w / groups, g = w - m * groups;
-    const uint32_t v = m < nrows ? base[w] : 0u;
-    tile_words[g * kAtomGroupWords + (m & 31) * 4 + (m >> 5)] = v;
-  }
-  __syncthreads();
-  for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) {
-    const int32_t g = w >> 7, wi = w & 127;
-    base[w] = tile_words[g * kAtomGroupWords + wi];
+    tile_words[g * kAtomGroupWords + (m & 31) * 4 + (m >> 5)] = m < nrows ? v : 0u;
+  };
+  if constexpr (VEC) {
+    // groups % 4 == 0 (the scale columns are a multiple of 16), so a vector
+    // never straddles two rows
+    const uint4 *vb = reinterpret_cast<const uint4 *>(base);
+    const int32_t vecs = words / 4;
+    const int32_t valid = nrows * groups / 4;  // vectors of rows < nrows
+    for (int32_t v0 = threadIdx.x; v0 < vecs; v0 += kAtomThreads * kAtomBatch) {
+      uint4 x[kAtomBatch];
+#pragma unroll
+      for (int b = 0; b < kAtomBatch; ++b) {
+        const int32_t v = v0 + b * kAtomThreads;
+        x[b] = v < valid ? vb[v] : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int b = 0; b < kAtomBatch; ++b) {
+        const int32_t v = v0 + b * kAtomThreads;
+        if (v < vecs) {  // words (m, g0 .. g0 + 3); rows past nrows were loaded as 0
+          const int32_t m = 4 * v / groups, g0 = 4 * v - m * groups;
+          uint32_t *t = tile_words + g0 * kAtomGroupWords + (m & 31) * 4 + (m >> 5);
+          t[0] = x[b].x;
+          t[kAtomGroupWords] = x[b].y;
+          t[2 * kAtomGroupWords] = x[b].z;
+          t[3 * kAtomGroupWords] = x[b].w;
+        }
+      }
+    }
+    __syncthreads();
+    uint4 *ob = reinterpret_cast<uint4 *>(base);
+    for (int32_t v = threadIdx.x; v < vecs; v += kAtomThreads) {
+      const int32_t w = 4 * v, g = w >> 7, wi = w & 127;
+      const uint32_t *t = tile_words + g * kAtomGroupWords + wi;
+      ob[v] = make_uint4(t[0], t[1], t[2], t[3]);
+    }
+  } else {
+    for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) put(w, w < nrows * groups ? base[w] : 0u);
+    __syncthreads();
+    for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) {
+      const int32_t g = w >> 7, wi = w & 127;
+      base[w] = tile_words[g * kAtomGroupWords + wi];
+    }
   }
 }
 
@@ -604,6 +750,21 @@ cudaError_t launch_permute_premultiplied(const Shape &s, const void *hidden,
                     static_cast<uint4 *>(out), s.N, s.k, s.rows, s.H / 8, chunks, ps);
 }
 
+cudaError_t launch_permute_to_peers(const Shape &s, const void *hidden, const int32_t *row_src,
+                                    const int32_t *pair_slot, const uint32_t *meta,
+                                    void *const *peer_out, const int64_t *put_offsets,
+                                    cudaStream_t stream) {
+  if (s.rows == 0) return cudaSuccess;
+  const int32_t chunks = chunks_of(s.H, kBf16Chunk);
+  const int32_t ps = padding_split(s, chunks);
+  const int32_t static_seg = s.Ce > 0 ? (s.E / s.S) * s.Ce : 0;
+  return launch_pdl(permute_to_peers_kernel, dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)),
+                    dim3(kThreads), (size_t)2 * s.S * sizeof(int32_t), stream,
+                    static_cast<const uint4 *>(hidden), row_src, pair_slot, meta,
+                    reinterpret_cast<uint4 *const *>(peer_out), put_offsets, s.N, s.k, s.rows,
+                    s.H / 8, chunks, ps, s.S, s.H, static_seg);
+}
+
 cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t *row_src,
                                const int32_t *pair_slot, uint8_t *q, float *scales,
                                cudaStream_t stream) {
@@ -625,14 +786,15 @@ inline bool atoms_in_place(int32_t nsf) {
 cudaError_t launch_scales_to_atoms(const Shape &s, int32_t nsf, uint8_t *scales,
                                    cudaStream_t stream) {
   const size_t smem = atom_tile_smem(nsf);
+  const bool vec = reinterpret_cast<uintptr_t>(scales) % 16 == 0 && (nsf / 4) % 4 == 0;
+  auto kernel = vec ? scales_to_atoms_kernel<true> : scales_to_atoms_kernel<false>;
   if (smem > 48 * 1024) {
-    const cudaError_t err = cudaFuncSetAttribute(
-        scales_to_atoms_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const cudaError_t err =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
   }
-  return launch_pdl(scales_to_atoms_kernel, dim3((unsigned)((s.rows + 127) / 128)),
-                    dim3(kAtomThreads), smem, stream, reinterpret_cast<uint32_t *>(scales),
-                    s.rows, nsf / 4);
+  return launch_pdl(kernel, dim3((unsigned)((s.rows + 127) / 128)), dim3(kAtomThreads), smem,
+                    stream, reinterpret_cast<uint32_t *>(scales), s.rows, nsf / 4);
 }
 
 cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32_t *row_src,

@@ -20,6 +20,12 @@ every rank takes them:
   combine_exchange        the expert outputs back along the reverse route, to
                           the rows the dispatch output had, ready for moe_combine
 
+or, with the send fused into the permute (moe_permute_to_peers: each
+segment's rows stored straight into the owning rank's receive buffer over
+NVLink / NVSwitch), exchange_counts, then put_offsets (where this rank's
+block starts in every receiver's buffer), the kernel, and a barrier before
+the receivers read.
+
 In packed mode a segment's rows are contiguous and start at meta row 1 / H
 (the exclusive cumsum of the send counts); in capacity mode ([E, Ce, H],
 static positions) segment s is its full L * Ce rows from s * L * Ce, padding
@@ -110,6 +116,20 @@ def exchange_counts(meta: torch.Tensor, hidden: int, num_experts: int,
     return Route(send_rows=send_rows, recv_rows=[int(v) // hidden for v in recv_elems.tolist()],
                  send_offsets=send_offsets,
                  recv_offsets=[int(v) // hidden for v in displs.tolist()])
+
+
+def put_offsets(route: Route, group=None) -> list[int]:
+    """First row of this rank's block in every rank's receive buffer, for
+    moe_permute_to_peers: rank d tells each source s where s's rows start in
+    d's buffer (its receive displacement of s, meta row 3 / H), through one
+    all-to-all."""
+    S = _world(group)
+    if len(route.recv_offsets) != S:
+        raise ValueError("route does not match the group")
+    mine = torch.tensor(route.recv_offsets, dtype=torch.int64)
+    got = torch.empty_like(mine)
+    dist.all_to_all_single(got, mine, group=group)
+    return [int(v) for v in got.tolist()]
 
 
 def exchange_expert_counts(expert_counts: torch.Tensor, group=None) -> torch.Tensor:

@@ -20,8 +20,10 @@
  * one E8M0 scale per 32 elements), moe_swiglu_quant (silu(gate) * up of the
  * expert rows that hold a token, as bf16 or requantised), the gradients
  * moe_permute_backward and moe_combine_backward, moe_permute_premultiplied
- * (the dispatch with each pair's row scaled by its gate), and
- * moe_dispatch_layout_noalloc (the layout without a caller workspace).
+ * (the dispatch with each pair's row scaled by its gate), moe_permute_to_peers
+ * (the dispatch written straight into the receive buffers of the ranks that
+ * own the experts), and moe_dispatch_layout_noalloc (the layout without a
+ * caller workspace).
  *
  * Notation: N tokens, H hidden size, E experts, k = top_k choices per token,
  * S destination segments of L = E/S consecutive experts, P = N*k pairs; pair
@@ -247,6 +249,34 @@ MOE_API moe_status moe_dispatch_layout_noalloc(const moe_problem *problem,
 MOE_API moe_status moe_permute(const moe_problem *problem, const void *hidden_states,
                        const int32_t *row_src, const int32_t *pair_slot, void *out,
                        moe_stream_t stream);
+
+/* Dispatch permute fused with the expert-parallel send: each segment's rows
+ * are stored straight into the receive buffer of the rank that owns its
+ * experts (peer stores over NVLink / NVSwitch) instead of into a local send
+ * buffer that an all-to-all then ships.  NKI "Permute A2AV Kernel API
+ * Reference" (the [4, EP] table: segment s of the packed buffer is the block
+ * for rank s, at its send displacement); Mojo MAX ep_comm (dispatch kernels
+ * that write tokens into the remote ranks' receive buffers).
+ * Segment s = experts [sL, (s+1)L): packed mode, local rows [meta[1][s]/H,
+ * + meta[0][s]/H) (expert blocks with their padding); capacity mode, rows
+ * [s*L*Ce, (s+1)*L*Ce).  Row r of segment s is written, as moe_permute would
+ * write it (padding rows as zeros), to row put_offsets[s] + r of the bf16
+ * [*, H] buffer peer_out[s]; rows past the last segment are not written.
+ *   hidden_states  bf16 [N, H], 16-byte aligned
+ *   row_src, pair_slot, meta   from moe_dispatch_layout (meta may be NULL in
+ *                  capacity mode)
+ *   peer_out       DEVICE array of S device pointers (8-byte aligned array;
+ *                  every pointer 16-byte aligned and writable from this GPU:
+ *                  a peer mapping, or this rank's own receive buffer)
+ *   put_offsets    DEVICE int64 [S]: first row of this rank's block in rank
+ *                  s's receive buffer (rank s's receive displacement of this
+ *                  source, in rows)
+ * Requires H % 8 == 0.  The call only enqueues the stores: the receivers may
+ * read after a barrier that follows the kernel's completion. */
+MOE_API moe_status moe_permute_to_peers(const moe_problem *problem, const void *hidden_states,
+                                        const int32_t *row_src, const int32_t *pair_slot,
+                                        const uint32_t *meta, void *const *peer_out,
+                                        const int64_t *put_offsets, moe_stream_t stream);
 
 /* Permute with pre-multiplied gates: out[slot(t,j), :] = bf16(gates[t,j] *
  * hidden_states[t, :]) -- one fp32 product and one rounding to nearest even

@@ -81,6 +81,12 @@ def _worker(rank, world, port, mode, q):
         assert list(got2) == [r * p["H"] for r in recv_rows], (got2, recv_rows)
         assert list(got3) == list(np.cumsum([0] + recv_rows[:-1]) * p["H"])
         assert route.recv_rows == recv_rows
+        # put offsets for the fused send: where this rank's block starts in
+        # every receiver's buffer (the receiver's displacement of this source)
+        po = ep.put_offsets(route)
+        want_po = [sum(len(_segment_rows(refs[s][0], probs[s], d)) for s in range(rank))
+                   for d in range(world)]
+        assert po == want_po, (po, want_po)
         # per-expert counts of every source for this rank's experts
         L = p["E"] // world
         ec = ep.exchange_expert_counts(torch.from_numpy(lay.expert_counts.copy()))

@@ -688,3 +688,61 @@ def test_swiglu_quant_wide_range(orc, gscale):
             if fmt != B.MOE_QUANT_BF16:
                 assert np.array_equal(scales.cpu().numpy(), want_s), (fmt, layout)
             assert np.array_equal(codes.cpu().numpy(), want_c), (fmt, layout)
+
+
+# ------------------------------------------------------------ dispatch to peers
+@pytest.mark.parametrize("mode", ["packed", "padded", "capacity"])
+def test_permute_to_peers(orc, mode):
+    """moe_permute_to_peers with S local buffers standing in for the S
+    ranks' receive buffers: segment s of the oracle's dispatch output lands
+    at rows [put[s], put[s] + rows_s) of buffer s, bit for bit (padding rows
+    inside a segment as zeros), and every other row of every buffer keeps
+    its poison (no stray store)."""
+    spec = dict(N=1500, H=264, E=24, k=3, S=4, p_mask=0.05, p_bad=0.01)
+    pad = 0
+    if mode == "padded":
+        pad = 8
+        spec["C"] = 1500 * 3 + 24 * 7
+    elif mode == "capacity":
+        spec["Ce"] = 150
+    w = custom(seed=31, with_out=False, **spec)
+    run = GpuRun(w, quant=False, combine=False, pad=pad)
+    ref = oracle_layout(orc, w, pad=pad)
+    assert_layout(run, ref)
+    want = orc.permute_bf16(w.hidden, ref.row_src)
+    L = w.E // w.S
+    if mode == "capacity":
+        starts = [s * L * w.expert_capacity for s in range(w.S)]
+        seg_rows = [L * w.expert_capacity] * w.S
+    else:
+        starts = [int(v) // w.H for v in ref.meta[1]]
+        seg_rows = [int(v) // w.H for v in ref.meta[0]]
+    rng = np.random.default_rng(9)
+    put = [int(rng.integers(0, 300)) for _ in range(w.S)]
+    bufs = [poisoned_empty((put[s] + seg_rows[s] + 17, w.H), torch.bfloat16)
+            for s in range(w.S)]
+    peer = torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device="cuda")
+    put_d = torch.tensor(put, dtype=torch.int64, device="cuda")
+    B.moe_permute_to_peers(run.prob, to_dev_bf16(w.hidden), run.buf.row_src, run.buf.pair_slot,
+                           run.buf.meta, peer, put_d)
+    torch.cuda.synchronize()
+    from gpu_util import BF16_POISON
+    for s in range(w.S):
+        got = bf16_np(bufs[s])
+        seg = want[starts[s]:starts[s] + seg_rows[s]]
+        assert np.array_equal(got[put[s]:put[s] + seg_rows[s]], seg), s
+        untouched = np.concatenate([got[:put[s]], got[put[s] + seg_rows[s]:]])
+        assert np.all(untouched == BF16_POISON), s
+
+
+def test_grouped_gemm_ready_dispatch_full_size(orc):
+    """The f1 configuration the benchmark times: the metric workload with
+    experts padded to 128 rows (recv_capacity = N*k + 127*E) and FP4 scales
+    in the atom layout; every row, code and scale byte against the oracle."""
+    w = make_workload("fp8_metric", with_expert_out=False)
+    pad = 128
+    w = Workload(**{**w.__dict__, "recv_capacity": w.N * w.k + w.E * (pad - 1)})
+    run = GpuRun(w, flags=B.MOE_FLAG_NVFP4_SWIZZLED_SCALES, combine=False, pad=pad)
+    ref = oracle_layout(orc, w, pad=pad)
+    assert_layout(run, ref)
+    assert_all_outputs(orc, w, run, ref)
