@@ -539,6 +539,28 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
               "tokens_per_s": w.N / ((lay_us + nv_us) * 1e-6)}
         del buf_p
 
+    # ---- expert-parallel send fused into the permute (NEXT row f2): segment
+    # s of the dispatch goes straight into "rank" s's receive buffer; on one
+    # GPU the S receive buffers are local stand-ins for the peers' buffers
+    f2 = None
+    if args.next_rows:
+        meta_h = buf.meta.cpu().numpy().view(np.uint32)
+        seg_rows = [int(v) // w.H for v in meta_h[0]]
+        recv = [torch.empty((max(r, 1), w.H), dtype=torch.bfloat16, device=dev)
+                for r in seg_rows]
+        peer = torch.tensor([t.data_ptr() for t in recv], dtype=torch.int64, device=dev)
+        put = torch.zeros(w.S, dtype=torch.int64, device=dev)
+        f2_steps = max(10, args.steps // 10)
+        (pp_us,) = time_phases([lambda: B.moe_permute_to_peers(
+            prob, d_hidden, buf.row_src, buf.pair_slot, buf.meta, peer, put)], f2_steps)
+        pp_bytes = 2 * w.N * w.H + 4 * w.P + 4 * buf.rows + 2 * sum(seg_rows) * w.H + 16 * w.S
+        f2 = {"steps": f2_steps, "segments": w.S,
+              "permute_to_peers_us": round(pp_us, 2),
+              "permute_to_peers_gbs": round(pp_bytes / (pp_us * 1e-6) / 1e9, 1),
+              "receivers": "S local buffers standing in for the peers' receive buffers "
+                           "(one GPU); across GPUs the same stores go over NVLink"}
+        del recv, peer, put
+
     # ---- backward (NEXT row f4): dispatch backward (gather-sum of the rows'
     # gradients) and combine backward (scaled scatter + gate gradients)
     f4 = None
@@ -734,8 +756,9 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
                             "combined rows, status and counts; copies of neighbouring steps "
                             "overlap on separate streams"},
             "gpu_launches": launches_per_step * args.steps,
-            "next_rows": ({"f1_grouped_gemm_ready_nvfp4": f1, "f3_mx_and_swiglu_requant": f3,
-                           "f4_backward": f4} if f1 or f3 or f4 else None),
+            "next_rows": ({"f1_grouped_gemm_ready_nvfp4": f1,
+                           "f2_permute_to_peers": f2, "f3_mx_and_swiglu_requant": f3,
+                           "f4_backward": f4} if f1 or f2 or f3 or f4 else None),
             "configs": configs,
             "clocks": clocks, "layout_status": st,
         }

@@ -382,20 +382,29 @@ __device__ void emit_common(int64_t r0, int64_t stride, int64_t rows, int32_t E,
     for (int e = tid; e < E; e += THREADS) expert_counts[e] = s_kept[e];
     for (int e = tid; e <= E; e += THREADS) expert_offsets[e] = s_off[e];
     const int32_t L = E / S;
-    for (int s = tid; s < S; s += THREADS) {
+    // one warp per segment: capacity mode sums the segment's kept rows over
+    // its L experts with the lanes and a shuffle reduction (packed mode reads
+    // the difference of two start rows)
+    const int lane = tid % kWarp;
+    for (int s = tid / kWarp; s < S; s += THREADS / kWarp) {
       int64_t seg_rows = 0;
       if (capacity) {
-        for (int e = s * L; e < (s + 1) * L; ++e) seg_rows += s_kept[e];
+        for (int e = s * L + lane; e < (s + 1) * L; e += kWarp) seg_rows += s_kept[e];
+#pragma unroll
+        for (int o = kWarp / 2; o > 0; o >>= 1)
+          seg_rows += __shfl_xor_sync(0xFFFFFFFFu, seg_rows, o);
       } else {
         seg_rows = (int64_t)s_off[(s + 1) * L] - s_off[s * L];  // blocks incl. padding
       }
-      const uint32_t count_el = (uint32_t)(seg_rows * H);
-      const uint32_t displ_el = capacity ? (uint32_t)((int64_t)s * L * Ce * H)
-                                         : (uint32_t)((int64_t)s_off[s * L] * H);
-      meta[0 * S + s] = count_el;
-      meta[1 * S + s] = displ_el;
-      meta[2 * S + s] = count_el;
-      meta[3 * S + s] = displ_el;
+      if (lane == 0) {
+        const uint32_t count_el = (uint32_t)(seg_rows * H);
+        const uint32_t displ_el = capacity ? (uint32_t)((int64_t)s * L * Ce * H)
+                                           : (uint32_t)((int64_t)s_off[s * L] * H);
+        meta[0 * S + s] = count_el;
+        meta[1 * S + s] = displ_el;
+        meta[2 * S + s] = count_el;
+        meta[3 * S + s] = displ_el;
+      }
     }
   }
 }

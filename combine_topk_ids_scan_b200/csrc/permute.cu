@@ -5,7 +5,8 @@
 // Movement is token-major ("push"): each token's row is read from HBM once
 // with 16-byte streaming loads and stored (or its quantised form) to each of
 // its k destination rows with 16-byte stores, so the quantisation is computed
-// once per token, not once per copy.  The unit of work is one chunk of one
+// once per token, not once per copy.  A warp issues its row loads before the
+// load of the token's pair_slot entries, so the two latencies overlap.  The unit of work is one chunk of one
 // token (512 elements for bf16, 1024 for the quantisers): one warp takes one
 // unit and exits.  Short warps over a grid of many blocks keep the write
 // stream denser than long-lived persistent warps do (measured on B200 for the
@@ -108,8 +109,6 @@ __global__ void __launch_bounds__(kThreads)
   if (w < units) {
     const int64_t t = w / chunks;
     const int v0 = (int)(w % chunks) * (kBf16Chunk / 8);
-    int32_t my_slot;
-    uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
     const uint4 *src = hidden + t * vecs;
     uint4 x[U];
 #pragma unroll
@@ -117,6 +116,8 @@ __global__ void __launch_bounds__(kThreads)
       const int v = v0 + u * kWarp + lane;
       if (v < vecs) x[u] = ld_stream_v4(src + v);
     }
+    int32_t my_slot;
+    uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
     while (live) {
       const int j = __ffs(live) - 1;
       live &= live - 1;
@@ -277,9 +278,6 @@ __global__ void __launch_bounds__(kThreads)
   if (w >= units) return;
   const int64_t t = w / chunks;
   const int v0 = (int)(w % chunks) * (kBf16Chunk / 8);
-  int32_t my_slot;
-  uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
-  const float my_w = lane < k ? __ldg(gates + t * k + lane) : 0.0f;
   const uint4 *src = hidden + t * vecs;
   uint4 x[U];
 #pragma unroll
@@ -287,6 +285,9 @@ __global__ void __launch_bounds__(kThreads)
     const int v = v0 + u * kWarp + lane;
     if (v < vecs) x[u] = ld_stream_v4(src + v);
   }
+  int32_t my_slot;
+  uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+  const float my_w = lane < k ? __ldg(gates + t * k + lane) : 0.0f;
   while (live) {
     const int j = __ffs(live) - 1;
     live &= live - 1;
@@ -636,14 +637,26 @@ __global__ void __launch_bounds__(kThreads, (SWIZZLED || !MX) ? 4 : 5)
 constexpr int kAtomThreads = 256;
 constexpr int kAtomGroupWords = 129;
 
-inline size_t atom_tile_smem(int32_t nsf) {
+inline size_t atom_tile_smem(int32_t nsf) {  // the larger of the two layouts
   return (size_t)(nsf / 4) * kAtomGroupWords * sizeof(uint32_t);
 }
 
-// VEC: the buffer is 16-byte aligned, and the tile moves as 16-byte vectors
-// (4 words of one row / of one atom row), kAtomBatch loads in flight per
-// thread before their shared-memory stores; else as 4-byte words.
+// VEC: the buffer is 16-byte aligned and the groups per row a multiple of
+// 4, and the tile moves as 16-byte vectors, kAtomBatch loads in flight per
+// thread before their shared-memory stores; else as 4-byte words through the
+// padded layout above.  VEC shared layout: group g's 128 words in atom order
+// as 32 chunks of 4 (chunk c = m % 32 holds m / 32 = 0..3), with the chunk
+// index XORed by (g / 4) % 8 and the words of a chunk rotated by
+// (g / 32) % 4.  A warp's scatter of one word per thread (32 consecutive
+// values of g / 4, one m) then falls in 32 distinct banks, and the
+// write-back reads each chunk as one 16-byte shared load (a warp reads one
+// group's 512 bytes, no conflict) and undoes the rotation in registers.
 constexpr int kAtomBatch = 8;
+
+__device__ __forceinline__ uint32_t atom_vec_slot(int32_t m, int32_t g) {
+  const int32_t q = g >> 2;
+  return (uint32_t)g * 128u + (uint32_t)(((m & 31) ^ (q & 7)) * 4 + (((m >> 5) + (q >> 3)) & 3));
+}
 
 template <bool VEC>
 __global__ void __launch_bounds__(kAtomThreads)
@@ -678,20 +691,28 @@ __global__ void __launch_bounds__(kAtomThreads)
         const int32_t v = v0 + b * kAtomThreads;
         if (v < vecs) {  // words (m, g0 .. g0 + 3); rows past nrows were loaded as 0
           const int32_t m = 4 * v / groups, g0 = 4 * v - m * groups;
-          uint32_t *t = tile_words + g0 * kAtomGroupWords + (m & 31) * 4 + (m >> 5);
+          uint32_t *t = tile_words + atom_vec_slot(m, g0);  // g0 .. g0+3 share g / 4
           t[0] = x[b].x;
-          t[kAtomGroupWords] = x[b].y;
-          t[2 * kAtomGroupWords] = x[b].z;
-          t[3 * kAtomGroupWords] = x[b].w;
+          t[128] = x[b].y;
+          t[256] = x[b].z;
+          t[384] = x[b].w;
         }
       }
     }
     __syncthreads();
     uint4 *ob = reinterpret_cast<uint4 *>(base);
     for (int32_t v = threadIdx.x; v < vecs; v += kAtomThreads) {
-      const int32_t w = 4 * v, g = w >> 7, wi = w & 127;
-      const uint32_t *t = tile_words + g * kAtomGroupWords + wi;
-      ob[v] = make_uint4(t[0], t[1], t[2], t[3]);
+      // output vector v: group g = v / 32, atom chunk c = v % 32
+      const int32_t g = v >> 5, c = v & 31, q = g >> 2;
+      const uint4 p = *reinterpret_cast<const uint4 *>(tile_words + g * 128 + (c ^ (q & 7)) * 4);
+      uint4 o;
+      switch ((q >> 3) & 3) {  // word o of the chunk sits at (o + r) % 4
+        case 0: o = p; break;
+        case 1: o = make_uint4(p.y, p.z, p.w, p.x); break;
+        case 2: o = make_uint4(p.z, p.w, p.x, p.y); break;
+        default: o = make_uint4(p.w, p.x, p.y, p.z); break;
+      }
+      ob[v] = o;
     }
   } else {
     for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) put(w, w < nrows * groups ? base[w] : 0u);
