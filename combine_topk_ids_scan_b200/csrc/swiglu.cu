@@ -575,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, FORMAT == 1 ? 4 : 3)
   int64_t w = (int64_t)blockIdx.x * (kThreads / kWarp) + threadIdx.x / kWarp;
   int64_t row = w / U;
   int32_t cu = (int32_t)(w - row * U);
-  const int64_t rows = units / U;
+  [[maybe_unused]] const int64_t rows = units / U;  // for the debug checks
   for (; w < units; w += warps) {
     if (!MOE_IN_RANGE(row, rows, kDbgSwigluRow)) break;
     const bool live = __ldg(row_src + row) >= 0;  // no routed token: zero bytes
@@ -619,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 3)
   int64_t t = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   int64_t row = t / G;
   int32_t cg = (int32_t)(t - row * G);
-  const int64_t rows = groups / G;
+  [[maybe_unused]] const int64_t rows = groups / G;  // for the debug checks
   for (; t < groups; t += stride) {
     if (!MOE_IN_RANGE(row, rows, kDbgSwigluRow)) break;
     swiglu_group<FORMAT, INTERLEAVED>(tab, gate_up, row_src, gs, codes, scales, row,
