@@ -492,6 +492,30 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
     phase_ms = {p: sum(v) / len(v) for p, v in per.items()}
     phase_step_ms = sum(e[0].elapsed_time(e[5]) for e in pevs) / n_phase
 
+    # ---- each kernel alone: the L2 flushed before every kernel (the dirty
+    # lines the previous kernel left are written back inside the flush, not
+    # inside the next kernel's events), as an ncu capture runs it
+    calls = [lambda: B.layout(prob, d_ids, buf),
+             lambda: B.moe_permute(prob, d_hidden, buf.row_src, buf.pair_slot, buf.out),
+             lambda: B.moe_permute_quant_fp8(prob, d_hidden, buf.row_src, buf.pair_slot,
+                                             buf.out_fp8, buf.scales_fp8),
+             lambda: B.moe_permute_quant_nvfp4(prob, d_hidden, buf.row_src, buf.pair_slot, d_gs,
+                                               buf.out_fp4, buf.scales_fp4),
+             lambda: B.moe_combine(prob, d_x, d_gates, buf.pair_slot, d_y)]
+    n_alone = max(10, min(args.steps, 100))
+    aev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in calls] for _ in range(n_alone)]
+    torch.cuda.synchronize(dev)
+    for i in range(n_alone):
+        for j, c in enumerate(calls):
+            flush_l2()
+            aev[i][j][0].record(stream)
+            c()
+            aev[i][j][1].record(stream)
+    torch.cuda.synchronize(dev)
+    alone_ms = {p: sum(aev[i][j][0].elapsed_time(aev[i][j][1]) for i in range(n_alone)) / n_alone
+                for j, p in enumerate(phases)}
+
     def time_phases(calls, n_steps):
         """Average device time (us) of each call in `calls`, run in order as
         one step; L2 flushed before every step, 3 untimed warm-up steps."""
@@ -741,6 +765,12 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
                               f"mean step {phase_step_ms:.4f} ms"),
             "phases_gbs": {p: round(nbytes[p] / (phase_ms[p] * 1e-3) / 1e9, 1)
                            for p in phases},
+            "phases_alone_us": {p: round(1e3 * v, 2) for p, v in alone_ms.items()},
+            "phases_alone_gbs": {p: round(nbytes[p] / (alone_ms[p] * 1e-3) / 1e9, 1)
+                                 for p in phases},
+            "phases_alone_timing": (f"{n_alone} more passes, each kernel alone: the L2 flushed "
+                                    "before every kernel, one event pair around it (context; the "
+                                    "roofline uses the in-step phases above)"),
             "dispatch_bf16_plus_combine_tokens_per_s":
                 world * w.N / ((phase_ms["layout"] + phase_ms["permute_bf16"]
                                 + phase_ms["combine"]) * 1e-3),

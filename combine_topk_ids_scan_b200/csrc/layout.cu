@@ -56,6 +56,7 @@ constexpr int kLookWindow = 8;                    // predecessor tiles per poll
 constexpr int kFusedMaxTiles = 128;               // last CTA clears <= 128*E words
 constexpr int64_t kClusterMaxRows = 1 << 18;      // cluster path: rows per launch
 constexpr int kClusterMax = 16;                   // largest cluster the path uses
+constexpr int64_t kSingleMaxRows = 1 << 14;       // single-CTA path: rows per launch
 
 constexpr int kEmitThreads = 256;
 
@@ -598,43 +599,51 @@ __global__ void __launch_bounds__(kEmitThreads) layout_emit_kernel(LayoutArgs a)
 // CTA 0's shared word; a second cluster barrier keeps every CTA's shared
 // memory alive until the others have read it, and CTA 0 stores the status.
 // The barriers are hardware cluster barriers over co-scheduled CTAs: there
-// is no spin loop and nothing to time out.
-template <int ROUNDS>
+// is no spin loop and nothing to time out.  SINGLE: the problem fits one
+// tile, the kernel is one ordinary CTA, and block barriers with local reads
+// replace the cluster barriers (with their release / acquire fences) and the
+// remote reads.
+template <int ROUNDS, bool SINGLE>
 __global__ void __launch_bounds__(kScanThreads, 1) layout_cluster_kernel(LayoutArgs a) {
   namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
   allow_dependents();  // the next kernel may be scheduled; it waits for this grid
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ uint32_t s_status;
   const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
-  const int c = (int)cluster.block_rank();
-  const int nc = (int)cluster.num_blocks();
+  const int c = SINGLE ? 0 : (int)cg::this_cluster().block_rank();
+  const int nc = SINGLE ? 1 : (int)cg::this_cluster().num_blocks();
   const int32_t E = a.E;
   const ScanSmem sm = scan_smem(smem, E);
   if (tid == 0) s_status = 0;
   TileScanT<ROUNDS> ts;
   ts.tile = c;
-  rank_tile<ROUNDS>(ts, a.ids, a.P, E, sm, &s_status);
-  cluster.sync();  // every tile's aggregate (tile_prefix) is visible
+  rank_tile<ROUNDS>(ts, a.ids, a.P, E, sm, &s_status);  // ends with a block barrier
+  if constexpr (!SINGLE) cg::this_cluster().sync();  // every tile's aggregate is visible
 
   // the lane-mask words are free now: exclusive prefix, start rows, kept rows
   int32_t *s_excl = reinterpret_cast<int32_t *>(sm.wmask);
   int32_t *s_off = s_excl + E;       // [E + 1]
   int32_t *s_kept = s_off + E + 1;   // [E]: the totals, then the kept rows
   for (int e = tid; e < E; e += kScanThreads) {
-    // all of the cluster's remote loads in flight at once
-    uint32_t v[kClusterMax];
+    if constexpr (SINGLE) {
+      s_excl[e] = 0;
+      s_kept[e] = (int32_t)sm.tile_prefix[e];
+    } else {
+      // all of the cluster's remote loads in flight at once
+      cg::cluster_group cluster = cg::this_cluster();
+      uint32_t v[kClusterMax];
 #pragma unroll
-    for (int q = 0; q < kClusterMax; ++q)
-      v[q] = q < nc ? *cluster.map_shared_rank(sm.tile_prefix + e, q) : 0u;
-    uint32_t excl = 0, tot = 0;
+      for (int q = 0; q < kClusterMax; ++q)
+        v[q] = q < nc ? *cluster.map_shared_rank(sm.tile_prefix + e, q) : 0u;
+      uint32_t excl = 0, tot = 0;
 #pragma unroll
-    for (int q = 0; q < kClusterMax; ++q) {
-      excl += q < c ? v[q] : 0u;
-      tot += v[q];
+      for (int q = 0; q < kClusterMax; ++q) {
+        excl += q < c ? v[q] : 0u;
+        tot += v[q];
+      }
+      s_excl[e] = (int32_t)excl;
+      s_kept[e] = (int32_t)tot;
     }
-    s_excl[e] = (int32_t)excl;
-    s_kept[e] = (int32_t)tot;
   }
   __syncthreads();
   expert_offsets_from_totals<kScanThreads, true>(s_kept, true, E, a.Ce, a.pad, s_off, s_kept);
@@ -668,9 +677,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) layout_cluster_kernel(LayoutA
     bits |= duplicate_bits(a.ids, gtid, a.N, gstride, a.k, E);
   if (bits) atomicOr(&s_status, bits);
   __syncthreads();
-  if (tid == 0 && c != 0 && s_status != 0)
-    atomicOr(cluster.map_shared_rank(&s_status, 0), s_status);
-  cluster.sync();  // all remote reads and status bits are done
+  if constexpr (!SINGLE) {
+    cg::cluster_group cluster = cg::this_cluster();
+    if (tid == 0 && c != 0 && s_status != 0)
+      atomicOr(cluster.map_shared_rank(&s_status, 0), s_status);
+    cluster.sync();  // all remote reads and status bits are done
+  }
   if (c == 0 && tid == 0) *a.status_out = s_status;
 }
 
@@ -678,9 +690,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) layout_cluster_kernel(LayoutA
 constexpr int kClusterRounds[5] = {1, 2, 4, 8, 16};
 inline const void *const *cluster_kernels() {
   static const void *const k[5] = {
-      (const void *)layout_cluster_kernel<1>, (const void *)layout_cluster_kernel<2>,
-      (const void *)layout_cluster_kernel<4>, (const void *)layout_cluster_kernel<8>,
-      (const void *)layout_cluster_kernel<16>};
+      (const void *)layout_cluster_kernel<1, false>, (const void *)layout_cluster_kernel<2, false>,
+      (const void *)layout_cluster_kernel<4, false>, (const void *)layout_cluster_kernel<8, false>,
+      (const void *)layout_cluster_kernel<16, false>};
+  return k;
+}
+// The single-CTA instantiations (one tile of 512, 1024 or 2048 pairs).
+constexpr int kSingleRounds[3] = {1, 2, 4};
+inline const void *const *single_kernels() {
+  static const void *const k[3] = {(const void *)layout_cluster_kernel<1, true>,
+                                   (const void *)layout_cluster_kernel<2, true>,
+                                   (const void *)layout_cluster_kernel<4, true>};
   return k;
 }
 struct ClusterKernelList {
@@ -706,6 +726,10 @@ cudaError_t opt_in_smem() {
   for (const void *kern : cluster_kernel_list())
     if (err == cudaSuccess)
       err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  for (int i = 0; i < 3; ++i)
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(single_kernels()[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 bytes);
   if (err == cudaSuccess && dev < kMaxDevices) done[dev].store(true);
   return err;
 }
@@ -772,7 +796,17 @@ cudaError_t launch_cluster_t(const LayoutArgs &a, int nc, size_t smem, cudaStrea
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, layout_cluster_kernel<ROUNDS>, a);
+  return cudaLaunchKernelEx(&cfg, layout_cluster_kernel<ROUNDS, false>, a);
+}
+
+// One CTA, no cluster (a problem of one tile).
+cudaError_t launch_single(int rounds, const LayoutArgs &a, size_t smem, cudaStream_t stream) {
+  switch (rounds) {
+    case 1: layout_cluster_kernel<1, true><<<1, kScanThreads, smem, stream>>>(a); break;
+    case 2: layout_cluster_kernel<2, true><<<1, kScanThreads, smem, stream>>>(a); break;
+    default: layout_cluster_kernel<4, true><<<1, kScanThreads, smem, stream>>>(a); break;
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_cluster(int rounds, const LayoutArgs &a, int nc, size_t smem,
@@ -857,6 +891,15 @@ cudaError_t launch_layout(const Shape &s, const int32_t *ids, int32_t *expert_co
   // the serial part of a tile, stay short.
   const uint32_t forced = MOE_FLAG_LAYOUT_TWO_PASS | MOE_FLAG_LAYOUT_LOOKBACK |
                           MOE_FLAG_TEST_STALL_SCAN;
+  if (!(s.flags & forced) && s.P <= (int64_t)kScanThreads * 4 && s.rows <= kSingleMaxRows) {
+    // one tile: one ordinary CTA, the fewest pairs per lane that fit
+    for (int rounds : kSingleRounds) {
+      if (s.P <= (int64_t)kScanThreads * rounds) {
+        if (opt_in_smem() != cudaSuccess) return cudaErrorUnknown;
+        return launch_single(rounds, a, smem, stream);
+      }
+    }
+  }
   if (!(s.flags & forced) && s.rows <= kClusterMaxRows) {
     const int maxc = max_cluster_size();
     for (int rounds : kClusterRounds) {

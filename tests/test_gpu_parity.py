@@ -306,12 +306,14 @@ def test_other_layout_paths_match_oracle(orc, cfg, path):
 
 @pytest.mark.parametrize("path", sorted(LAYOUT_PATHS))
 @pytest.mark.parametrize("N,k,E", [(12500, 8, 64), (16384, 8, 256), (8191, 8, 256),
-                                   (8193, 8, 256), (4097, 1, 3)])
+                                   (8193, 8, 256), (4097, 1, 3), (1025, 1, 7), (256, 8, 40),
+                                   (2049, 1, 9)])
 def test_layout_cluster_sizes(orc, N, k, E, path):
-    """Pair counts around the cluster kernel's limits: 8193 pairs (three
-    tiles of 4096), 65528 and 65544 pairs (one tile below and above sixteen
-    tiles of 4096), 100000 and 131072 pairs (tiles of 8192 pairs), with a
-    ragged last tile and masked, out-of-range and duplicate ids."""
+    """Pair counts around the size limits of the layout kernels: 1025 and
+    2048 pairs (one CTA, 4 pairs per lane), 2049 and 4097 pairs (a cluster
+    of 1-pair lanes), 65528 and 65544 pairs (one tile below and above
+    sixteen tiles of 4096), 100000 and 131072 pairs (tiles of 8192 pairs),
+    with a ragged last tile and masked, out-of-range and duplicate ids."""
     w = custom(N=N, H=32, E=E, k=k, S=1, seed=N + E, p_mask=0.05, p_bad=0.01,
                distinct=(N % 2 == 0), with_out=False)
     flags = B.MOE_FLAG_CHECK_DUPLICATES | LAYOUT_PATHS[path]
