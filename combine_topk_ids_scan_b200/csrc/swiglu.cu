@@ -28,13 +28,13 @@
 // sequence directly, so the table changes no result, only the work.
 //
 // Two persistent kernels.  swiglu_quant_kernel (the NVFP4 and MXFP6
-// outputs) deals the row-major list of (row, 32-column group) pairs out lane
-// by lane, so no lane idles when I is not a multiple of 1024; a lane owns 32
-// consecutive columns: eight 16-byte loads of gate/up, one MX block or two
-// NVFP4 blocks.  swiglu_split_kernel (MXFP8, MXFP4, bf16; split or
-// interleaved gate/up) gives each warp 512 columns of a row with short
-// column runs per lane, so that its loads and stores are contiguous per
-// warp instruction.
+// outputs) deals the row-major list of (row, column group) pairs out lane by
+// lane, so no lane idles when I is not a multiple of 1024; a lane owns one
+// block: 32 consecutive columns for MXFP6 (eight 16-byte loads of gate/up),
+// 16 for NVFP4 (four loads), so that each block's scale work stays in one
+// lane.  swiglu_split_kernel (MXFP8, MXFP4, bf16; split or interleaved
+// gate/up) gives each warp 512 columns of a row with short column runs per
+// lane, so that its loads and stores are contiguous per warp instruction.
 #include <algorithm>
 
 #include "common.cuh"
@@ -351,6 +351,97 @@ __device__ __forceinline__ void swiglu_group(const float *tab, const uint4 *__re
   }
 }
 
+// One lane's NVFP4 block: the 16 columns [c, c + 16) of row r, the rule of
+// the 32-column group above on one block.  Lanes 32 bytes apart (split
+// gate/up) or 64 bytes apart (interleaved) instead of 64 / 128, so each
+// warp-wide 16-byte load touches a quarter / half as many cache lines, while
+// each block's scale work stays in one lane.
+template <bool INTERLEAVED>
+__device__ __forceinline__ void swiglu_nvfp4_block(const float *tab,
+                                                   const uint4 *__restrict__ gate_up,
+                                                   const int32_t *__restrict__ row_src, float gs,
+                                                   uint8_t *__restrict__ codes,
+                                                   uint8_t *__restrict__ scales, int64_t r,
+                                                   int32_t c, int32_t I) {
+  uint8_t *cd = codes + r * ((int64_t)I / 2) + c / 2;  // 8 bytes of codes
+  uint8_t *sd = scales + r * ((int64_t)I / 16) + c / 16;
+  if (__ldg(row_src + r) < 0) {  // no routed token: zero bytes, input not read
+    *reinterpret_cast<uint2 *>(cd) = make_uint2(0, 0);
+    *sd = 0;
+    return;
+  }
+  const uint4 *in = gate_up + r * ((int64_t)I / 4);  // 2I bf16 = I/4 vectors of 8
+  uint4 gv[2], uv[2];
+  if (INTERLEAVED) {
+    uint4 iv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) iv[i] = ld_stream_v4(in + c / 4 + i);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint4 a = iv[2 * i], b = iv[2 * i + 1];
+      gv[i] = make_uint4(__byte_perm(a.x, a.y, 0x5410), __byte_perm(a.z, a.w, 0x5410),
+                         __byte_perm(b.x, b.y, 0x5410), __byte_perm(b.z, b.w, 0x5410));
+      uv[i] = make_uint4(__byte_perm(a.x, a.y, 0x7632), __byte_perm(a.z, a.w, 0x7632),
+                         __byte_perm(b.x, b.y, 0x7632), __byte_perm(b.z, b.w, 0x7632));
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      gv[i] = ld_stream_v4(in + c / 8 + i);
+      uv[i] = ld_stream_v4(in + I / 8 + c / 8 + i);
+    }
+  }
+  uint32_t check = 0;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    check |= table_check(gv[i].x) | table_check(gv[i].y) | table_check(gv[i].z) |
+             table_check(gv[i].w);
+  float2 y[8];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t g4[4] = {gv[i].x, gv[i].y, gv[i].z, gv[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if ((check & kTableCheckBits) == 0) {
+        uint32_t lo, hi;
+        table_offsets(g4[e], lo, hi);
+        y[4 * i + e] = make_float2(table_at(tab, lo), table_at(tab, hi));
+      } else {
+        y[4 * i + e] = silu2(make_float2(bf16lo(g4[e]), bf16hi(g4[e])));
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t u4[4] = {uv[i].x, uv[i].y, uv[i].z, uv[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      y[4 * i + e] = __fmul2_rn(y[4 * i + e], make_float2(bf16lo(u4[e]), bf16hi(u4[e])));
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) amax = max_abs3(amax, y[j].x, y[j].y);
+  const uint32_t sq = cvt_e4m3x2(__fdiv_rn(__fdiv_rn(amax, 6.0f), gs), 0.0f) & 0xFFu;
+  const float d = __fmul_rn(e4m3_to_float(sq), gs);
+  uint32_t cw[2] = {0, 0};
+  if (d > 0.0f) {
+    float2 q[8];
+    // |y / d| <= 12.01 unless the block scale saturated at 448 (0x7E)
+    if (sq < 0x7Eu && d >= kQuotientMinDivisor && d <= kQuotientMaxDivisor) {
+      const float rd = __frcp_rn(d);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) q[j] = rn_quotient2(y[j], d, rd);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) q[j] = make_float2(__fdiv_rn(y[j].x, d), __fdiv_rn(y[j].y, d));
+    }
+    cw[0] = cvt_e2m1x8(q[0], q[1], q[2], q[3]);
+    cw[1] = cvt_e2m1x8(q[4], q[5], q[6], q[7]);
+  }
+  *reinterpret_cast<uint2 *>(cd) = make_uint2(cw[0], cw[1]);
+  *sd = (uint8_t)sq;
+}
+
 // ---- split layout: coalesced warp units
 // A warp takes a unit of 512 columns of one row; lane l holds the 8 columns
 // [c0 + 256 s + 8 l, +8) for s = 0, 1, so every 16-byte load and every code
@@ -596,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, FORMAT == 1 ? 4 : 3)
 // Persistent: thread t of the grid takes groups t, t + stride, ... of the
 // rows * G groups (G = I / 32 per row); (row, group) advance by
 // (step_rows, step_cols) = divmod(stride, G).
-template <int FORMAT, bool INTERLEAVED>
+template <int FORMAT, bool INTERLEAVED, int COLS>
 __global__ void __launch_bounds__(kThreads, 3)
     swiglu_quant_kernel(const uint4 *__restrict__ gate_up, const int32_t *__restrict__ row_src,
                         const float *__restrict__ global_scale, uint8_t *__restrict__ codes,
@@ -622,8 +713,11 @@ __global__ void __launch_bounds__(kThreads, 3)
   [[maybe_unused]] const int64_t rows = groups / G;  // for the debug checks
   for (; t < groups; t += stride) {
     if (!MOE_IN_RANGE(row, rows, kDbgSwigluRow)) break;
-    swiglu_group<FORMAT, INTERLEAVED>(tab, gate_up, row_src, gs, codes, scales, row,
-                                      cg * kGroupCols, I);
+    if constexpr (COLS == 16)
+      swiglu_nvfp4_block<INTERLEAVED>(tab, gate_up, row_src, gs, codes, scales, row, cg * 16, I);
+    else
+      swiglu_group<FORMAT, INTERLEAVED>(tab, gate_up, row_src, gs, codes, scales, row,
+                                        cg * kGroupCols, I);
     row += step_rows;
     cg += step_cols;
     if (cg >= G) {
@@ -656,10 +750,12 @@ cudaError_t launch(const uint4 *in, const int32_t *row_src, const float *gs, uin
   if (FORMAT == 1 || FORMAT == 2 || FORMAT == 3)
     return launch_split<(FORMAT == 1 || FORMAT == 2) ? FORMAT : 3, INTERLEAVED>(
         in, row_src, codes, scales, rows, I, stream);
-  auto kernel = swiglu_quant_kernel<FORMAT, INTERLEAVED>;
+  // NVFP4: one 16-column block per lane; MXFP6: one 32-column MX block
+  constexpr int kCols = FORMAT == 0 ? 16 : kGroupCols;
+  auto kernel = swiglu_quant_kernel<FORMAT, INTERLEAVED, kCols>;
   static OccupancyCache occupancy;
   const int cap = resident_ctas(occupancy, reinterpret_cast<const void *>(kernel), kThreads, 0);
-  const int32_t G = I / kGroupCols;
+  const int32_t G = I / kCols;
   const int64_t groups = rows * G;
   const int64_t want = (groups + kThreads - 1) / kThreads;
   const int64_t blocks = std::max<int64_t>(
