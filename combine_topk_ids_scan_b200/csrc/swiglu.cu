@@ -28,13 +28,15 @@
 // sequence directly, so the table changes no result, only the work.
 //
 // Two persistent kernels.  swiglu_quant_kernel (the NVFP4 and MXFP6
-// outputs) deals the row-major list of (row, column group) pairs out lane by
-// lane, so no lane idles when I is not a multiple of 1024; a lane owns one
-// block: 32 consecutive columns for MXFP6 (eight 16-byte loads of gate/up),
-// 16 for NVFP4 (four loads), so that each block's scale work stays in one
-// lane.  swiglu_split_kernel (MXFP8, MXFP4, bf16; split or interleaved
-// gate/up) gives each warp 512 columns of a row with short column runs per
-// lane, so that its loads and stores are contiguous per warp instruction.
+// outputs) deals the row-major list of (row, 16-column group) pairs out lane
+// by lane, so no lane idles when I is not a multiple of 1024: an NVFP4 lane
+// owns one whole block, so its scale work stays in one lane; an MXFP6 lane
+// owns half of a 32-column block and shares the block maximum with its
+// neighbour by one shuffle.  (32-column groups per lane, the first form,
+// put lanes 64 bytes apart, and the L1 data path saturated.)
+// swiglu_split_kernel (MXFP8, MXFP4, bf16; split or interleaved gate/up)
+// gives each warp 512 columns of a row with short column runs per lane, so
+// that its loads and stores are contiguous per warp instruction.
 #include <algorithm>
 
 #include "common.cuh"
@@ -442,6 +444,98 @@ __device__ __forceinline__ void swiglu_nvfp4_block(const float *tab,
   *sd = (uint8_t)sq;
 }
 
+// One lane's half of an MXFP6 block: the 16 columns [c, c + 16) of row r;
+// the block's other half is the partner lane (lane ^ 1, columns c ^ 16),
+// which the dealing of column groups keeps in the same warp and row (G is
+// even).  The block maximum is one xor-shuffle over the two lanes, both
+// derive the same E8M0 scale; each packs its 16 six-bit codes into 12 bytes
+// (bits [96 h, 96 h + 96) of the block's 24), the even lane stores the scale.
+template <int FORMAT, bool INTERLEAVED>
+__device__ __forceinline__ void swiglu_mxfp6_half(const float *tab,
+                                                  const uint4 *__restrict__ gate_up,
+                                                  const int32_t *__restrict__ row_src,
+                                                  uint8_t *__restrict__ codes,
+                                                  uint8_t *__restrict__ scales, int64_t r,
+                                                  int32_t c, int32_t I, int lane) {
+  constexpr int kEmax = FORMAT == 4 ? 2 : 4;
+  const bool upper = (c & 16) != 0;
+  uint32_t *cd = reinterpret_cast<uint32_t *>(codes + r * ((int64_t)I / 32 * 24) +
+                                              (int64_t)(c / 32) * 24 + (upper ? 12 : 0));
+  uint8_t *sd = scales + r * ((int64_t)I / 32) + c / 32;
+  if (__ldg(row_src + r) < 0) {  // no routed token (the partner lane is in the same row)
+    cd[0] = cd[1] = cd[2] = 0;
+    if (!upper) *sd = 0;
+    return;
+  }
+  const uint4 *in = gate_up + r * ((int64_t)I / 4);
+  uint4 gv[2], uv[2];
+  if (INTERLEAVED) {
+    uint4 iv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) iv[i] = ld_stream_v4(in + c / 4 + i);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint4 a = iv[2 * i], b = iv[2 * i + 1];
+      gv[i] = make_uint4(__byte_perm(a.x, a.y, 0x5410), __byte_perm(a.z, a.w, 0x5410),
+                         __byte_perm(b.x, b.y, 0x5410), __byte_perm(b.z, b.w, 0x5410));
+      uv[i] = make_uint4(__byte_perm(a.x, a.y, 0x7632), __byte_perm(a.z, a.w, 0x7632),
+                         __byte_perm(b.x, b.y, 0x7632), __byte_perm(b.z, b.w, 0x7632));
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      gv[i] = ld_stream_v4(in + c / 8 + i);
+      uv[i] = ld_stream_v4(in + I / 8 + c / 8 + i);
+    }
+  }
+  uint32_t check = 0;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    check |= table_check(gv[i].x) | table_check(gv[i].y) | table_check(gv[i].z) |
+             table_check(gv[i].w);
+  float2 y[8];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t g4[4] = {gv[i].x, gv[i].y, gv[i].z, gv[i].w};
+    const uint32_t u4[4] = {uv[i].x, uv[i].y, uv[i].z, uv[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float2 sg;
+      if ((check & kTableCheckBits) == 0) {
+        uint32_t lo, hi;
+        table_offsets(g4[e], lo, hi);
+        sg = make_float2(table_at(tab, lo), table_at(tab, hi));
+      } else {
+        sg = silu2(make_float2(bf16lo(g4[e]), bf16hi(g4[e])));
+      }
+      y[4 * i + e] = __fmul2_rn(sg, make_float2(bf16lo(u4[e]), bf16hi(u4[e])));
+    }
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) amax = max_abs3(amax, y[j].x, y[j].y);
+  // the two lanes of the block (same branch, same row): exactly those two
+  amax = fmaxf(amax, __shfl_xor_sync(3u << (lane & 30), amax, 1));
+  uint32_t sc = 0, w[3] = {0, 0, 0};
+  if (amax > 0.0f) {
+    sc = mx_scale_code(amax, kEmax);
+    const float2 s2 = splat(pow2i(127 - (int)sc));
+    float2 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = __fmul2_rn(y[j], s2);
+    uint32_t lo[2], hi[2];
+#pragma unroll
+    for (int g = 0; g < 2; ++g) cvt_fp6x8<FORMAT == 4>(v + 4 * g, lo[g], hi[g]);
+    w[0] = lo[0];
+    w[1] = hi[0] | (lo[1] << 16);
+    w[2] = (lo[1] >> 16) | (hi[1] << 16);
+  }
+  cd[0] = w[0];
+  cd[1] = w[1];
+  cd[2] = w[2];
+  if (!upper) *sd = (uint8_t)sc;
+}
+
 // ---- split layout: coalesced warp units
 // A warp takes a unit of 512 columns of one row; lane l holds the 8 columns
 // [c0 + 256 s + 8 l, +8) for s = 0, 1, so every 16-byte load and every code
@@ -713,8 +807,11 @@ __global__ void __launch_bounds__(kThreads, 3)
   [[maybe_unused]] const int64_t rows = groups / G;  // for the debug checks
   for (; t < groups; t += stride) {
     if (!MOE_IN_RANGE(row, rows, kDbgSwigluRow)) break;
-    if constexpr (COLS == 16)
+    if constexpr (COLS == 16 && FORMAT == 0)
       swiglu_nvfp4_block<INTERLEAVED>(tab, gate_up, row_src, gs, codes, scales, row, cg * 16, I);
+    else if constexpr (COLS == 16)
+      swiglu_mxfp6_half<FORMAT, INTERLEAVED>(tab, gate_up, row_src, codes, scales, row, cg * 16,
+                                             I, threadIdx.x % kWarp);
     else
       swiglu_group<FORMAT, INTERLEAVED>(tab, gate_up, row_src, gs, codes, scales, row,
                                         cg * kGroupCols, I);
@@ -750,8 +847,9 @@ cudaError_t launch(const uint4 *in, const int32_t *row_src, const float *gs, uin
   if (FORMAT == 1 || FORMAT == 2 || FORMAT == 3)
     return launch_split<(FORMAT == 1 || FORMAT == 2) ? FORMAT : 3, INTERLEAVED>(
         in, row_src, codes, scales, rows, I, stream);
-  // NVFP4: one 16-column block per lane; MXFP6: one 32-column MX block
-  constexpr int kCols = FORMAT == 0 ? 16 : kGroupCols;
+  // NVFP4: one 16-column block per lane; MXFP6: half of a 32-column MX
+  // block per lane (the other half in the neighbouring lane)
+  constexpr int kCols = (FORMAT == 0 || FORMAT >= 4) ? 16 : kGroupCols;
   auto kernel = swiglu_quant_kernel<FORMAT, INTERLEAVED, kCols>;
   static OccupancyCache occupancy;
   const int cap = resident_ctas(occupancy, reinterpret_cast<const void *>(kernel), kThreads, 0);
