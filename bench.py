@@ -475,6 +475,7 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
     clocks = sampler.stop() if sampler else None
     step_ms = [e[0].elapsed_time(e[5]) for e in evs]
     ms = sum(step_ms) / len(step_ms)
+    ms_median, ms_min = statistics.median(step_ms), min(step_ms)
 
     # ---- per-kernel breakdown: further steps with an event between kernels
     phases = ["layout", "permute_bf16", "permute_fp8", "permute_nvfp4", "combine"]
@@ -754,6 +755,7 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "ms_per_step_median": ms_median, "ms_per_step_min": ms_min,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp32", "data": "synthetic", "config": workload_config(w),
             "hbm_gbs": step_bytes / (ms * 1e-3) / 1e9,
