@@ -45,10 +45,10 @@ NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, nominal (DGX figure)
 # metric workload (summaries under profiles/), keyed by kernel; valid only
 # while the kernel's source file is unchanged (sha256 prefix at capture time)
 NCU_TRAFFIC: dict[str, dict] = {
-    "permute_bf16": {"bytes_per_launch": 117979136 + 882330624, "src_sha": "1eb3661d6de44200"},
-    "permute_fp8": {"bytes_per_launch": 118069760 + 426646528, "src_sha": "a0efff8b48c5274f"},
+    "permute_bf16": {"bytes_per_launch": 117985536 + 880217344, "src_sha": "a0218bc31711bbc1"},
+    "permute_fp8": {"bytes_per_launch": 118066944 + 422894336, "src_sha": "c6c0d1cc4d647560"},
     "permute_nvfp4": {"bytes_per_launch": 118020096 + 207139584, "src_sha": "669914b64a79a75e"},
-    "combine": {"bytes_per_launch": 940067072 + 69790720, "src_sha": "6c7f98a5b6533638"},
+    "combine": {"bytes_per_launch": 940131840 + 64447232, "src_sha": "709371a62977d2c7"},
 }
 
 

@@ -22,14 +22,18 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 # MOE_LIB_PATH selects another build of the library, e.g. the build with
-# device index checks (libmoedc_debug.so, see moe_debug_violations)
+# device index checks (libmoedc_debug.so, see moe_debug_violations) or the
+# build with trace records
 LIB_PATH = os.environ.get("MOE_LIB_PATH") or os.path.join(_PKG, "libmoedc.so")
 DEBUG_LIB_PATH = os.path.join(_PKG, "libmoedc_debug.so")
+# per-CTA trace records (libmoedc_trace.so, see moe_trace_attach)
+TRACE_LIB_PATH = os.path.join(_PKG, "libmoedc_trace.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
 MOE_ERR_UNSUPPORTED_SHAPE = 2
 MOE_ERR_CUDA = 3
+MOE_ERR_NOT_BUILT = 4
 
 MOE_STATUS_ID_RANGE = 1
 MOE_STATUS_DUP_ID = 2
@@ -53,7 +57,7 @@ EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout",
             "moe_permute_quant_nvfp4", "moe_permute_quant_mxfp4", "moe_combine",
             "moe_permute_backward",
             "moe_combine_backward", "moe_swiglu_quant", "moe_status_string", "moe_version",
-            "moe_debug_violations")
+            "moe_debug_violations", "moe_trace_attach")
 
 (MOE_QUANT_NVFP4, MOE_QUANT_MXFP8, MOE_QUANT_MXFP4, MOE_QUANT_BF16, MOE_QUANT_MXFP6_E2M3,
  MOE_QUANT_MXFP6_E3M2) = 0, 1, 2, 3, 4, 5
@@ -63,7 +67,8 @@ MOE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
 _STATUS_TEXT = {MOE_OK: "ok", MOE_ERR_INVALID_ARG: "invalid argument",
-                MOE_ERR_UNSUPPORTED_SHAPE: "unsupported shape", MOE_ERR_CUDA: "CUDA error"}
+                MOE_ERR_UNSUPPORTED_SHAPE: "unsupported shape", MOE_ERR_CUDA: "CUDA error",
+                MOE_ERR_NOT_BUILT: "not in this build"}
 
 
 class MoeError(RuntimeError):
@@ -153,6 +158,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     L.moe_version.argtypes = []
     L.moe_debug_violations.restype = ctypes.c_int64
     L.moe_debug_violations.argtypes = [ctypes.c_int]
+    L.moe_trace_attach.restype = ctypes.c_int
+    L.moe_trace_attach.argtypes = [vp, ctypes.c_uint32, vp, vp]
     _lib = L
     return L
 
@@ -169,6 +176,23 @@ def debug_violations(reset: bool = False) -> int:
     """Bits of out-of-range indices the device checks recorded (0 = none),
     or -1 when the loaded build has no checks (see moe_debug_violations)."""
     return int(load().moe_debug_violations(int(reset)))
+
+
+TRACE_RECORD_BYTES = 32   # sizeof(moe_trace_record)
+
+
+def moe_trace_attach(records, count, stream=None) -> None:
+    """Attach a trace record buffer (the build with -DMOE_TRACE): `records`
+    is a device tensor of capacity * 32 bytes, `count` a device int32 tensor
+    of at least one element that the caller has zeroed; records=None
+    detaches.  Raises MoeError(MOE_ERR_NOT_BUILT) on other builds."""
+    if records is None:
+        _check(load().moe_trace_attach(None, 0, None, _stream(stream)), "moe_trace_attach")
+        return
+    capacity = records.numel() * records.element_size() // TRACE_RECORD_BYTES
+    _require("moe_trace_attach", count=(count, 4))
+    _check(load().moe_trace_attach(_ptr(records), capacity, _ptr(count), _stream(stream)),
+           "moe_trace_attach")
 
 
 def _ptr(t: torch.Tensor | None):

@@ -1,6 +1,6 @@
 """Build libmoedc.so (the C-ABI CUDA library) in-tree with nvcc for sm_100a.
 
-    python -m combine_topk_ids_scan_b200.build [--verbose] [--force]
+    python -m combine_topk_ids_scan_b200.build [--verbose] [--force] [--debug | --trace]
 
 No fast-math: the FP8 / NVFP4 scales use IEEE round-to-nearest division and
 the combine relies on exact fused multiply-adds.
@@ -21,6 +21,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libmoedc.so")
 # the same sources with device index checks (-DMOE_DEBUG_CHECKS)
 DEBUG_LIB_PATH = os.path.join(PKG, "libmoedc_debug.so")
+# the same sources with per-CTA trace records (-DMOE_TRACE)
+TRACE_LIB_PATH = os.path.join(PKG, "libmoedc_trace.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
@@ -51,14 +53,19 @@ def up_to_date(path: str = LIB_PATH) -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
-    """Build libmoedc.so, or with debug=True libmoedc_debug.so (device index
-    checks, see moe_debug_violations in moe_dc.h)."""
-    path = DEBUG_LIB_PATH if debug else LIB_PATH
+def build(force: bool = False, verbose: bool = False, debug: bool = False,
+          trace: bool = False) -> str:
+    """Build libmoedc.so; with debug=True libmoedc_debug.so (device index
+    checks, see moe_debug_violations in moe_dc.h); with trace=True
+    libmoedc_trace.so (per-CTA trace records, see moe_trace_attach)."""
+    if debug and trace:
+        raise ValueError("one build option at a time")
+    path = DEBUG_LIB_PATH if debug else TRACE_LIB_PATH if trace else LIB_PATH
     if not force and up_to_date(path):
         return path
     tmp = path + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, *(["-DMOE_DEBUG_CHECKS"] if debug else []),
+    defines = ["-DMOE_DEBUG_CHECKS"] if debug else ["-DMOE_TRACE"] if trace else []
+    cmd = [_nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, *defines,
            "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -74,6 +81,8 @@ if __name__ == "__main__":
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--debug", action="store_true",
                     help="build libmoedc_debug.so with device index checks")
+    ap.add_argument("--trace", action="store_true",
+                    help="build libmoedc_trace.so with per-CTA trace records")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose, debug=a.debug))
+    print(build(force=a.force, verbose=a.verbose, debug=a.debug, trace=a.trace))
     sys.exit(0)

@@ -34,6 +34,8 @@ namespace {
 
 constexpr int64_t kU32Max = 4294967295ll;
 
+static_assert(sizeof(moe_trace_record) == 32, "moe_trace_record is 32 bytes");
+
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Validates the problem and fills the derived sizes.
@@ -321,16 +323,46 @@ const char *moe_status_string(moe_status status) {
       return "unsupported shape (size outside the library's limits)";
     case MOE_ERR_CUDA:
       return "CUDA error while launching";
+    case MOE_ERR_NOT_BUILT:
+      return "not in this build (see the build options in moe_dc.h)";
     default:
       return "unknown status";
   }
 }
 
 const char *moe_version(void) {
-#ifdef MOE_DEBUG_CHECKS
+#if defined(MOE_DEBUG_CHECKS) && defined(MOE_TRACE)
+  return "moedc 0.2.0 (sm_100a, device index checks, trace records)";
+#elif defined(MOE_DEBUG_CHECKS)
   return "moedc 0.2.0 (sm_100a, device index checks)";
+#elif defined(MOE_TRACE)
+  return "moedc 0.2.0 (sm_100a, trace records)";
 #else
   return "moedc 0.2.0 (sm_100a)";
+#endif
+}
+
+moe_status moe_trace_attach(moe_trace_record *records, uint32_t capacity, uint32_t *count,
+                            moe_stream_t stream) {
+#ifdef MOE_TRACE
+  if (records != nullptr && (count == nullptr || capacity == 0)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(records, 8) || !aligned(count, 4)) return MOE_ERR_INVALID_ARG;
+  if (records == nullptr) {
+    count = nullptr;
+    capacity = 0;
+  }
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t err = moe::trace_attach_layout(records, count, capacity, st);
+  if (err == cudaSuccess) err = moe::trace_attach_permute(records, count, capacity, st);
+  if (err == cudaSuccess) err = moe::trace_attach_combine(records, count, capacity, st);
+  if (err == cudaSuccess) err = moe::trace_attach_swiglu(records, count, capacity, st);
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+#else
+  (void)records;
+  (void)capacity;
+  (void)count;
+  (void)stream;
+  return MOE_ERR_NOT_BUILT;
 #endif
 }
 

@@ -20,6 +20,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "trace.cuh"
 
 namespace moe {
 
@@ -33,6 +34,7 @@ __global__ void __launch_bounds__(kThreads)
     combine_kernel(const uint4 *__restrict__ x, const float *__restrict__ gates,
                    const int32_t *__restrict__ pair_slot, uint4 *__restrict__ out, int32_t N,
                    int32_t k, int64_t rows, int32_t vecs, int32_t splits, int32_t span) {
+  MOE_TRACE_CTA(gates ? MOE_TRACE_COMBINE : MOE_TRACE_PERMUTE_BACKWARD, KMAX);
   allow_dependents();
   grid_dependency_wait();
   const int lane = threadIdx.x % kWarp;
@@ -118,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int32_t *__restrict__ row_src, uint4 *__restrict__ grad_x,
                             float *__restrict__ grad_gates, int32_t N, int32_t k, int64_t rows,
                             int32_t vecs) {
+  MOE_TRACE_CTA(MOE_TRACE_COMBINE_BACKWARD, KMAX);
   allow_dependents();
   grid_dependency_wait();
   const int lane = threadIdx.x % kWarp;
@@ -252,6 +255,13 @@ cudaError_t launch_forward(const Shape &s, const uint4 *x, const float *gates,
 }  // namespace
 
 uint32_t debug_violations_combine(bool reset) { return read_debug_violations(reset); }
+
+#ifdef MOE_TRACE
+cudaError_t trace_attach_combine(moe_trace_record *records, uint32_t *count, uint32_t capacity,
+                              cudaStream_t stream) {
+  return trace_attach_tu(records, count, capacity, stream);
+}
+#endif
 
 cudaError_t launch_combine_backward(const Shape &s, const void *grad_y, const void *expert_out,
                                     const float *gates, const int32_t *pair_slot,

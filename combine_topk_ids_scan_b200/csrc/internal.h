@@ -90,6 +90,19 @@ uint32_t debug_violations_permute(bool reset);
 uint32_t debug_violations_combine(bool reset);
 uint32_t debug_violations_swiglu(bool reset);
 
+// Each kernel translation unit's trace attachment (the build with
+// -DMOE_TRACE; trace.cuh).
+#ifdef MOE_TRACE
+cudaError_t trace_attach_layout(moe_trace_record *records, uint32_t *count, uint32_t capacity,
+                                cudaStream_t stream);
+cudaError_t trace_attach_permute(moe_trace_record *records, uint32_t *count, uint32_t capacity,
+                                 cudaStream_t stream);
+cudaError_t trace_attach_combine(moe_trace_record *records, uint32_t *count, uint32_t capacity,
+                                 cudaStream_t stream);
+cudaError_t trace_attach_swiglu(moe_trace_record *records, uint32_t *count, uint32_t capacity,
+                                cudaStream_t stream);
+#endif
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 

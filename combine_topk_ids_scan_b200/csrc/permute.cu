@@ -23,6 +23,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "trace.cuh"
 
 namespace moe {
 
@@ -89,6 +90,7 @@ __global__ void __launch_bounds__(kThreads)
                         const int32_t *__restrict__ pair_slot, uint4 *__restrict__ out,
                         int32_t N, int32_t k, int64_t rows, int32_t vecs, int32_t chunks,
                         int32_t psplit) {
+  MOE_TRACE_CTA(MOE_TRACE_PERMUTE_BF16, 0);
   allow_dependents();
   grid_dependency_wait();
   constexpr int U = kBf16Chunk / 8 / kWarp;  // 2
@@ -174,6 +176,7 @@ __global__ void __launch_bounds__(kThreads)
                             const int64_t *__restrict__ put, int32_t N, int32_t k, int64_t rows,
                             int32_t vecs, int32_t chunks, int32_t psplit, int32_t S, int32_t H,
                             int32_t static_seg_rows) {
+  MOE_TRACE_CTA(MOE_TRACE_PERMUTE_TO_PEERS, 0);
   allow_dependents();
   extern __shared__ int32_t seg_smem[];  // [S] starts, [S] rows
   int32_t *s_start = seg_smem, *s_rows = seg_smem + S;
@@ -258,6 +261,7 @@ __global__ void __launch_bounds__(kThreads)
                                  const float *__restrict__ gates, uint4 *__restrict__ out,
                                  int32_t N, int32_t k, int64_t rows, int32_t vecs,
                                  int32_t chunks, int32_t psplit) {
+  MOE_TRACE_CTA(MOE_TRACE_PERMUTE_PREMULTIPLIED, 0);
   allow_dependents();
   grid_dependency_wait();
   constexpr int U = kBf16Chunk / 8 / kWarp;  // 2
@@ -313,6 +317,7 @@ __global__ void __launch_bounds__(kThreads)
                        const int32_t *__restrict__ pair_slot, uint8_t *__restrict__ q,
                        float *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
                        int32_t H, int32_t chunks, int32_t psplit) {
+  MOE_TRACE_CTA(MOE_TRACE_PERMUTE_FP8, 0);
   allow_dependents();
   grid_dependency_wait();
   constexpr int U = kChunk / 512;  // 2
@@ -472,19 +477,22 @@ __device__ __forceinline__ int64_t sf_atom_offset(int64_t m, int32_t c, int32_t 
 
 // MX == false: NVFP4 (two 16-element blocks per lane, E4M3 scales);
 // MX == true: MXFP4 (one 32-element block per lane, E8M0 scales).
-// SWIZZLED: scales in the block-scale atom layout.  The token row's loads
+// SWIZZLED: scales in the block-scale atom layout.  PAD_SCALES == false
+// (linear scales that scales_to_atoms_kernel converts next): padding rows'
+// scales are left unwritten, the atom kernel zeroes them.  The token row's loads
 // are issued first, before the pair_slot load and its ballot.  The MXFP4
 // linear-scale kernel is held to 5 resident CTAs per SM (at most 48
 // registers; measured on B200 at the metric shape: 61.4 -> 60.0 us), the
 // NVFP4 and the atom-layout kernels to 4 (NVFP4 with its loads first: 65.5 us
 // at 5 CTAs with a 4-byte spill, 63.5 us at 4 without one).
-template <bool MX, bool SWIZZLED>
+template <bool MX, bool SWIZZLED, bool PAD_SCALES = true>
 __global__ void __launch_bounds__(kThreads, (SWIZZLED || !MX) ? 4 : 5)
     permute_fp4_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                        const int32_t *__restrict__ pair_slot,
                        const float *__restrict__ global_scale, uint8_t *__restrict__ q,
                        uint8_t *__restrict__ scales, int32_t N, int32_t k, int64_t rows,
                        int32_t H, int32_t chunks, int32_t psplit) {
+  MOE_TRACE_CTA(MX ? MOE_TRACE_PERMUTE_MXFP4 : MOE_TRACE_PERMUTE_NVFP4, SWIZZLED ? 1 : 0);
   constexpr bool swizzled = SWIZZLED;
   allow_dependents();
   grid_dependency_wait();
@@ -518,13 +526,14 @@ __global__ void __launch_bounds__(kThreads, (SWIZZLED || !MX) ? 4 : 5)
         const int64_t row = g * kWarp + j;
         uint4 *dst = reinterpret_cast<uint4 *>(q) + row * (qrow / 16);
         for (int v = v0 + lane; v < v1; v += kWarp) st_v4(dst + v, zero);
-        for (int v = s0 + lane; v < s1; v += kWarp) scales[row * srow + v] = 0;
+        if (PAD_SCALES)
+          for (int v = s0 + lane; v < s1; v += kWarp) scales[row * srow + v] = 0;
       }
     } else if (m && !swizzled) {
       int32_t s0, s1;
       share_of(c, psplit, srow / 2, s0, s1);
       zero_rows(m, g, lane, reinterpret_cast<uint4 *>(q), qrow / 16, v0, v1,
-                reinterpret_cast<uint16_t *>(scales), srow / 2, s0, s1);
+                PAD_SCALES ? reinterpret_cast<uint16_t *>(scales) : nullptr, srow / 2, s0, s1);
     } else if (m) {
       int32_t g0, g1;
       share_of(c, psplit, groups, g0, g1);
@@ -629,7 +638,9 @@ __global__ void __launch_bounds__(kThreads, (SWIZZLED || !MX) ? 4 : 5)
 // the permute writes linear scales there first (whole 64- or 32-byte runs
 // per warp instead of 4-byte pieces of 8 different rows per 32-byte sector)
 // and this kernel reads the whole tile into shared memory, then writes it
-// back in atom order; rows at or past `rows` become zeros.  Shared layout:
+// back in atom order.  The permute leaves the padding rows' scales unwritten
+// (row_src -1): this kernel reads only the rows that hold a token and writes
+// zeros for the others and for rows at or past `rows`.  Shared layout:
 // word (m, g) of 4-scale group g at g * 129 + (m % 32) * 4 + m / 32 -- the
 // atom order, so the write-back reads consecutive words, padded by one word
 // per group so that the scattered writes of a warp (consecutive g) fall in
@@ -660,7 +671,9 @@ __device__ __forceinline__ uint32_t atom_vec_slot(int32_t m, int32_t g) {
 
 template <bool VEC>
 __global__ void __launch_bounds__(kAtomThreads)
-    scales_to_atoms_kernel(uint32_t *__restrict__ scales, int64_t rows, int32_t groups) {
+    scales_to_atoms_kernel(uint32_t *__restrict__ scales, const int32_t *__restrict__ row_src,
+                           int64_t rows, int32_t groups) {
+  MOE_TRACE_CTA(MOE_TRACE_SCALES_TO_ATOMS, VEC ? 1 : 0);
   allow_dependents();
   extern __shared__ uint32_t tile_words[];
   grid_dependency_wait();
@@ -669,27 +682,36 @@ __global__ void __launch_bounds__(kAtomThreads)
   const int32_t nrows = left < 128 ? (int32_t)left : 128;
   uint32_t *base = scales + tile * 128 * groups;  // the tile's words (either layout)
   const int32_t words = 128 * groups;
+  // bit m of s_live: row m of the tile holds a token (its scales were written)
+  __shared__ uint32_t s_live[4];
+  if (threadIdx.x < 128) {
+    const int32_t m = threadIdx.x;
+    const bool live = m < nrows && row_src[tile * 128 + m] >= 0;
+    const uint32_t bits = __ballot_sync(0xFFFFFFFFu, live);
+    if (m % kWarp == 0) s_live[m / kWarp] = bits;
+  }
+  __syncthreads();
+  const auto live = [&](int32_t m) { return ((s_live[m >> 5] >> (m & 31)) & 1u) != 0u; };
   const auto put = [&](int32_t w, uint32_t v) {  // linear word w -> shared, atom order
     const int32_t m = w / groups, g = w - m * groups;
-    tile_words[g * kAtomGroupWords + (m & 31) * 4 + (m >> 5)] = m < nrows ? v : 0u;
+    tile_words[g * kAtomGroupWords + (m & 31) * 4 + (m >> 5)] = v;
   };
   if constexpr (VEC) {
     // groups % 4 == 0 (the scale columns are a multiple of 16), so a vector
     // never straddles two rows
     const uint4 *vb = reinterpret_cast<const uint4 *>(base);
     const int32_t vecs = words / 4;
-    const int32_t valid = nrows * groups / 4;  // vectors of rows < nrows
     for (int32_t v0 = threadIdx.x; v0 < vecs; v0 += kAtomThreads * kAtomBatch) {
       uint4 x[kAtomBatch];
 #pragma unroll
       for (int b = 0; b < kAtomBatch; ++b) {
         const int32_t v = v0 + b * kAtomThreads;
-        x[b] = v < valid ? vb[v] : make_uint4(0, 0, 0, 0);
+        x[b] = v < vecs && live(4 * v / groups) ? vb[v] : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int b = 0; b < kAtomBatch; ++b) {
         const int32_t v = v0 + b * kAtomThreads;
-        if (v < vecs) {  // words (m, g0 .. g0 + 3); rows past nrows were loaded as 0
+        if (v < vecs) {  // words (m, g0 .. g0 + 3); rows without a token were loaded as 0
           const int32_t m = 4 * v / groups, g0 = 4 * v - m * groups;
           uint32_t *t = tile_words + atom_vec_slot(m, g0);  // g0 .. g0+3 share g / 4
           t[0] = x[b].x;
@@ -715,7 +737,8 @@ __global__ void __launch_bounds__(kAtomThreads)
       ob[v] = o;
     }
   } else {
-    for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) put(w, w < nrows * groups ? base[w] : 0u);
+    for (int32_t w = threadIdx.x; w < words; w += kAtomThreads)
+      put(w, live(w / groups) ? base[w] : 0u);
     __syncthreads();
     for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) {
       const int32_t g = w >> 7, wi = w & 127;
@@ -748,6 +771,13 @@ inline int32_t chunks_of(int32_t H, int32_t chunk) { return (H + chunk - 1) / ch
 }  // namespace
 
 uint32_t debug_violations_permute(bool reset) { return read_debug_violations(reset); }
+
+#ifdef MOE_TRACE
+cudaError_t trace_attach_permute(moe_trace_record *records, uint32_t *count, uint32_t capacity,
+                                 cudaStream_t stream) {
+  return trace_attach_tu(records, count, capacity, stream);
+}
+#endif
 
 cudaError_t launch_permute_bf16(const Shape &s, const void *hidden, const int32_t *row_src,
                                 const int32_t *pair_slot, void *out, cudaStream_t stream) {
@@ -805,7 +835,7 @@ inline bool atoms_in_place(int32_t nsf) {
 }
 
 cudaError_t launch_scales_to_atoms(const Shape &s, int32_t nsf, uint8_t *scales,
-                                   cudaStream_t stream) {
+                                   const int32_t *row_src, cudaStream_t stream) {
   const bool vec = reinterpret_cast<uintptr_t>(scales) % 16 == 0 && (nsf / 4) % 4 == 0;
   // both layouts get the padded size: 3 tiles per SM at H = 7168 (the
   // vector layout's exact 56 KB would fit 4; measured slower on B200, 19.1
@@ -818,7 +848,7 @@ cudaError_t launch_scales_to_atoms(const Shape &s, int32_t nsf, uint8_t *scales,
     if (err != cudaSuccess) return err;
   }
   return launch_pdl(kernel, dim3((unsigned)((s.rows + 127) / 128)), dim3(kAtomThreads), smem,
-                    stream, reinterpret_cast<uint32_t *>(scales), s.rows, nsf / 4);
+                    stream, reinterpret_cast<uint32_t *>(scales), row_src, s.rows, nsf / 4);
 }
 
 cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32_t *row_src,
@@ -830,11 +860,12 @@ cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32
   const int32_t ps = padding_split(s, chunks);
   if (swizzled && atoms_in_place(s.H / 16)) {
     const cudaError_t err = launch_pdl(
-        permute_fp4_kernel<false, false>, dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)),
-        dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src, pair_slot,
-        global_scale, q, scales, s.N, s.k, s.rows, s.H, chunks, ps);
+        permute_fp4_kernel<false, false, false>,
+        dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads), 0, stream,
+        static_cast<const uint4 *>(hidden), row_src, pair_slot, global_scale, q, scales, s.N,
+        s.k, s.rows, s.H, chunks, ps);
     if (err != cudaSuccess) return err;
-    return launch_scales_to_atoms(s, s.H / 16, scales, stream);
+    return launch_scales_to_atoms(s, s.H / 16, scales, row_src, stream);
   }
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
   return launch_pdl(swizzled ? permute_fp4_kernel<false, true> : permute_fp4_kernel<false, false>,
@@ -852,11 +883,12 @@ cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32
   const int32_t ps = padding_split(s, chunks);
   if (swizzled && atoms_in_place(s.H / 32)) {
     const cudaError_t err = launch_pdl(
-        permute_fp4_kernel<true, false>, dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)),
-        dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src, pair_slot,
+        permute_fp4_kernel<true, false, false>,
+        dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads), 0, stream,
+        static_cast<const uint4 *>(hidden), row_src, pair_slot,
         static_cast<const float *>(nullptr), q, scales, s.N, s.k, s.rows, s.H, chunks, ps);
     if (err != cudaSuccess) return err;
-    return launch_scales_to_atoms(s, s.H / 32, scales, stream);
+    return launch_scales_to_atoms(s, s.H / 32, scales, row_src, stream);
   }
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
   return launch_pdl(swizzled ? permute_fp4_kernel<true, true> : permute_fp4_kernel<true, false>,

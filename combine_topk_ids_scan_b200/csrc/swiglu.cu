@@ -41,6 +41,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "trace.cuh"
 
 namespace moe {
 
@@ -745,6 +746,7 @@ __global__ void __launch_bounds__(kThreads, FORMAT == 1 ? 4 : 3)
     swiglu_split_kernel(const uint4 *__restrict__ gate_up, const int32_t *__restrict__ row_src,
                         uint8_t *__restrict__ codes, uint8_t *__restrict__ scales, int64_t units,
                         int32_t I, int32_t U, int64_t step_rows, int32_t step_cols) {
+  MOE_TRACE_CTA(MOE_TRACE_SWIGLU_SPLIT, FORMAT);
   allow_dependents();
   __shared__ float tab[kTabSize];
   for (int i = 2 * threadIdx.x; i < kTabSize; i += 2 * kThreads) {
@@ -787,6 +789,7 @@ __global__ void __launch_bounds__(kThreads, 3)
                         const float *__restrict__ global_scale, uint8_t *__restrict__ codes,
                         uint8_t *__restrict__ scales, int64_t groups, int32_t I, int32_t G,
                         int64_t step_rows, int32_t step_cols) {
+  MOE_TRACE_CTA(MOE_TRACE_SWIGLU_QUANT, FORMAT);
   allow_dependents();
   __shared__ float tab[kTabSize];
   // the table needs no global memory: it is built while the previous kernel
@@ -866,6 +869,13 @@ cudaError_t launch(const uint4 *in, const int32_t *row_src, const float *gs, uin
 }  // namespace
 
 uint32_t debug_violations_swiglu(bool reset) { return read_debug_violations(reset); }
+
+#ifdef MOE_TRACE
+cudaError_t trace_attach_swiglu(moe_trace_record *records, uint32_t *count, uint32_t capacity,
+                              cudaStream_t stream) {
+  return trace_attach_tu(records, count, capacity, stream);
+}
+#endif
 
 cudaError_t launch_swiglu_quant(const Shape &s, int32_t I, uint32_t format, bool interleaved,
                                 const void *gate_up, const int32_t *row_src,

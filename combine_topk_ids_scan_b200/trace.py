@@ -1,0 +1,123 @@
+"""Per-CTA trace records of the build with -DMOE_TRACE (libmoedc_trace.so).
+
+The library's kernels append one 32-byte record per CTA (moe_trace_record in
+include/moe_dc.h: start and end on the GPU's nanosecond timer, launch id,
+block index, SM, kernel id and variant) to a buffer attached with
+moe_trace_attach.  This module decodes the records on the host and groups
+them into launches; Tracer attaches a buffer around a block of calls:
+
+    from combine_topk_ids_scan_b200 import binding as B, trace
+    with trace.Tracer(capacity=1 << 16) as tr:     # MOE_LIB_PATH = the trace build
+        B.layout(prob, ids, buf)
+        B.moe_permute(prob, hidden, buf.row_src, buf.pair_slot, buf.out)
+    for launch in tr.launches():
+        print(launch.kernel, launch.ctas, launch.duration_us)
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+RECORD_DTYPE = np.dtype([("start_ns", "<u8"), ("end_ns", "<u8"), ("grid", "<u8"),
+                         ("block", "<u4"), ("smid", "<u2"), ("kernel", "u1"),
+                         ("variant", "u1")])
+assert RECORD_DTYPE.itemsize == 32
+
+# moe_trace_kernel
+KERNELS = {
+    1: "layout_single", 2: "layout_cluster", 3: "layout_lookback", 4: "layout_scan",
+    5: "layout_emit", 6: "permute_bf16", 7: "permute_fp8", 8: "permute_nvfp4",
+    9: "permute_mxfp4", 10: "scales_to_atoms", 11: "permute_premultiplied",
+    12: "permute_to_peers", 13: "combine", 14: "permute_backward", 15: "combine_backward",
+    16: "swiglu_split", 17: "swiglu_quant",
+}
+LAYOUT_KERNELS = frozenset(range(1, 6))
+
+
+@dataclass(frozen=True)
+class Launch:
+    """The CTAs of one kernel launch (one %gridid)."""
+    kernel: str
+    kernel_id: int
+    variant: int
+    grid: int
+    ctas: int
+    sms: int          # distinct SMs its CTAs ran on
+    start_ns: int     # earliest CTA start
+    end_ns: int       # latest CTA end
+
+    @property
+    def duration_us(self) -> float:
+        return (self.end_ns - self.start_ns) / 1e3
+
+
+def decode(raw: np.ndarray, count: int) -> np.ndarray:
+    """The records a traced run wrote: `raw` is the record buffer's bytes
+    (uint8, capacity * 32), `count` the device counter's final value.
+    Records past the capacity were dropped by the kernels."""
+    raw = np.ascontiguousarray(raw).view(np.uint8).reshape(-1)
+    capacity = raw.size // RECORD_DTYPE.itemsize
+    recs = raw[:capacity * RECORD_DTYPE.itemsize].view(RECORD_DTYPE)
+    return recs[:min(int(count), capacity)].copy()
+
+
+def dropped(count: int, capacity: int) -> int:
+    """Records the kernels could not write (count ran past the capacity)."""
+    return max(0, int(count) - int(capacity))
+
+
+def launches(records: np.ndarray) -> list[Launch]:
+    """Group records by launch, in the order the launches started."""
+    out = []
+    for g in np.unique(records["grid"]):
+        r = records[records["grid"] == g]
+        kid = int(r["kernel"][0])
+        if np.any(r["kernel"] != kid) or np.any(r["variant"] != r["variant"][0]):
+            raise ValueError(f"launch {int(g)} mixes kernel ids or variants")
+        out.append(Launch(kernel=KERNELS.get(kid, f"kernel{kid}"), kernel_id=kid,
+                          variant=int(r["variant"][0]), grid=int(g), ctas=int(r.size),
+                          sms=int(np.unique(r["smid"]).size),
+                          start_ns=int(r["start_ns"].min()), end_ns=int(r["end_ns"].max())))
+    out.sort(key=lambda launch: (launch.start_ns, launch.grid))
+    return out
+
+
+class Tracer:
+    """Attach a record buffer of `capacity` records on entry (on the current
+    stream), detach and read the records back on exit."""
+
+    def __init__(self, capacity: int = 1 << 16, stream=None):
+        self.capacity = int(capacity)
+        self.stream = stream
+        self.count = 0
+        self._records = None
+
+    def __enter__(self) -> "Tracer":
+        import torch
+
+        from combine_topk_ids_scan_b200 import binding as B
+        self._raw = torch.zeros(self.capacity * RECORD_DTYPE.itemsize, dtype=torch.uint8,
+                                device="cuda")
+        self._count = torch.zeros(1, dtype=torch.int32, device="cuda")
+        B.moe_trace_attach(self._raw, self._count, self.stream)
+        return self
+
+    def __exit__(self, *exc) -> None:
+        import torch
+
+        from combine_topk_ids_scan_b200 import binding as B
+        B.moe_trace_attach(None, None, self.stream)
+        torch.cuda.synchronize()
+        self.count = int(self._count.cpu().numpy().view(np.uint32)[0])
+        self._records = decode(self._raw.cpu().numpy(), self.count)
+
+    @property
+    def dropped(self) -> int:
+        return dropped(self.count, self.capacity)
+
+    def records(self) -> np.ndarray:
+        return self._records
+
+    def launches(self) -> list[Launch]:
+        return launches(self._records)

@@ -23,7 +23,9 @@
  * (the dispatch with each pair's row scaled by its gate), moe_permute_to_peers
  * (the dispatch written straight into the receive buffers of the ranks that
  * own the experts), and moe_dispatch_layout_noalloc (the layout without a
- * caller workspace).
+ * caller workspace).  Two builds of the same sources add checks and records:
+ * device index checks (moe_debug_violations) and per-CTA trace records
+ * (moe_trace_attach).
  *
  * Notation: N tokens, H hidden size, E experts, k = top_k choices per token,
  * S destination segments of L = E/S consecutive experts, P = N*k pairs; pair
@@ -75,7 +77,9 @@ typedef enum moe_status {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,       /* null pointer, negative size, misaligned */
   MOE_ERR_UNSUPPORTED_SHAPE = 2, /* a size outside the supported limits     */
-  MOE_ERR_CUDA = 3               /* a CUDA launch or runtime error          */
+  MOE_ERR_CUDA = 3,              /* a CUDA launch or runtime error          */
+  MOE_ERR_NOT_BUILT = 4          /* the call needs a build option that this
+                                    library was built without               */
 } moe_status;
 
 /* Bits of the device status word written by moe_dispatch_layout. */
@@ -465,6 +469,65 @@ MOE_API moe_status moe_combine_backward(const moe_problem *problem, const void *
  * is non-zero; synchronises with the device.  Returns -1 from a build
  * without the checks (no CUDA call is made then). */
 MOE_API int64_t moe_debug_violations(int reset);
+
+/* Per-CTA trace records.  A build with -DMOE_TRACE
+ * (`python -m combine_topk_ids_scan_b200.build --trace`, libmoedc_trace.so)
+ * has every CTA of every library kernel append one record to the buffer
+ * attached with moe_trace_attach: the CTA's start and end on the GPU's
+ * global nanosecond timer, the launch it belongs to, its block index and the
+ * SM it ran on -- the per-CTA timeline of a step, kernel by kernel (the
+ * pages' Mojo ep_comm DispatchTraceSink; NullDispatchTrace, the sink that
+ * discards events, is the normal build, whose kernels hold no trace code).
+ * Tracing costs one atomic add, one barrier and a 32-byte record per CTA
+ * and one atomic max per warp. */
+typedef struct moe_trace_record {
+  uint64_t start_ns; /* %globaltimer when the CTA started (for a kernel that
+                        overlaps its predecessor, before it waits for it)   */
+  uint64_t end_ns;   /* %globaltimer when the CTA's last warp finished      */
+  uint64_t grid;     /* %gridid: one value per launch, shared by its CTAs   */
+  uint32_t block;    /* blockIdx.x                                          */
+  uint16_t smid;     /* the SM the CTA ran on                               */
+  uint8_t kernel;    /* moe_trace_kernel                                    */
+  uint8_t variant;   /* the kernel's compile-time variant (below), else 0   */
+} moe_trace_record;  /* 32 bytes */
+
+/* moe_trace_record.kernel, with the variant each one records. */
+typedef enum moe_trace_kernel {
+  MOE_TRACE_LAYOUT_SINGLE = 1,         /* one-CTA layout; variant: pair rounds     */
+  MOE_TRACE_LAYOUT_CLUSTER = 2,        /* cluster layout; variant: pair rounds     */
+  MOE_TRACE_LAYOUT_LOOKBACK = 3,       /* cooperative look-back layout             */
+  MOE_TRACE_LAYOUT_SCAN = 4,           /* two-pass layout, scan kernel             */
+  MOE_TRACE_LAYOUT_EMIT = 5,           /* two-pass layout, emit kernel             */
+  MOE_TRACE_PERMUTE_BF16 = 6,          /* moe_permute                              */
+  MOE_TRACE_PERMUTE_FP8 = 7,           /* moe_permute_quant_fp8                    */
+  MOE_TRACE_PERMUTE_NVFP4 = 8,         /* variant: 1 scales stored in the atom
+                                          layout, 0 linear (final, or converted
+                                          by MOE_TRACE_SCALES_TO_ATOMS)            */
+  MOE_TRACE_PERMUTE_MXFP4 = 9,         /* variant as MOE_TRACE_PERMUTE_NVFP4       */
+  MOE_TRACE_SCALES_TO_ATOMS = 10,      /* variant: 1 with 16-byte vectors          */
+  MOE_TRACE_PERMUTE_PREMULTIPLIED = 11,
+  MOE_TRACE_PERMUTE_TO_PEERS = 12,
+  MOE_TRACE_COMBINE = 13,              /* variant: the largest top_k it handles    */
+  MOE_TRACE_PERMUTE_BACKWARD = 14,     /* variant as MOE_TRACE_COMBINE             */
+  MOE_TRACE_COMBINE_BACKWARD = 15,     /* variant as MOE_TRACE_COMBINE             */
+  MOE_TRACE_SWIGLU_SPLIT = 16,         /* variant: the MOE_QUANT_* format          */
+  MOE_TRACE_SWIGLU_QUANT = 17          /* variant: the MOE_QUANT_* format          */
+} moe_trace_kernel;
+
+/* Attach the trace record buffer (the build with -DMOE_TRACE): the kernels
+ * of every later call on `stream` append one record per CTA.
+ *   records   device array of `capacity` records, or NULL to stop tracing
+ *   count     device uint32, zeroed by the caller; each CTA adds 1 and
+ *             writes records[old value] if that is below `capacity`, so a
+ *             count above capacity tells how many records were dropped
+ * The attachment is a copy enqueued on `stream` (kernels enqueued on other
+ * streams see it in no defined order) and lasts until the next call.  The
+ * caller owns both buffers and keeps them alive while traced kernels run.
+ * Returns MOE_ERR_NOT_BUILT, making no CUDA call, from a build without
+ * -DMOE_TRACE; MOE_ERR_INVALID_ARG for records without count, misaligned
+ * pointers (records 8 bytes, count 4) or capacity 0 with records. */
+MOE_API moe_status moe_trace_attach(moe_trace_record *records, uint32_t capacity,
+                                    uint32_t *count, moe_stream_t stream);
 
 /* Static description of a moe_status value. */
 MOE_API const char *moe_status_string(moe_status status);

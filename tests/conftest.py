@@ -33,3 +33,29 @@ def _device_index_checks():
         return
     v = B.debug_violations(reset=True)
     assert v == 0, f"device index checks recorded violations {v:#x} (-1: not a debug build)"
+
+
+def _trace_build_loaded() -> bool:
+    return os.path.basename(os.environ.get("MOE_LIB_PATH", "")) == "libmoedc_trace.so"
+
+
+@pytest.fixture(autouse=True)
+def _trace_every_test():
+    """When MOE_TRACE_EVERY_TEST=1 and the session runs on the build with
+    trace records (MOE_LIB_PATH names libmoedc_trace.so), every test runs
+    with a record buffer attached, and afterwards its launches must be
+    consistent: each CTA of a launch recorded exactly once, start <= end,
+    and stream order kept (no CTA of a launch starts before every CTA of the
+    previous one has started, none ends before the previous one ended)."""
+    if os.environ.get("MOE_TRACE_EVERY_TEST") != "1" or not _trace_build_loaded():
+        yield
+        return
+    import torch
+    if not torch.cuda.is_available():
+        yield
+        return
+    from trace_checks import check_launches
+    from combine_topk_ids_scan_b200 import trace as T
+    with T.Tracer(capacity=1 << 20) as tr:
+        yield
+    check_launches(tr)
