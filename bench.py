@@ -576,15 +576,41 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
         peer = torch.tensor([t.data_ptr() for t in recv], dtype=torch.int64, device=dev)
         put = torch.zeros(w.S, dtype=torch.int64, device=dev)
         f2_steps = max(10, args.steps // 10)
-        (pp_us,) = time_phases([lambda: B.moe_permute_to_peers(
-            prob, d_hidden, buf.row_src, buf.pair_slot, buf.meta, peer, put)], f2_steps)
-        pp_bytes = 2 * w.N * w.H + 4 * w.P + 4 * buf.rows + 2 * sum(seg_rows) * w.H + 16 * w.S
+        # the quantised forms: codes and scales per receiver
+        r8 = [(torch.empty((max(r, 1), w.H), dtype=torch.uint8, device=dev),
+               torch.empty((max(r, 1), w.H // 128), dtype=torch.float32, device=dev))
+              for r in seg_rows]
+        r4 = [(torch.empty((max(r, 1), w.H // 2), dtype=torch.uint8, device=dev),
+               torch.empty((max(r, 1), w.H // 16), dtype=torch.uint8, device=dev))
+              for r in seg_rows]
+
+        def ptrs(bufs, i):
+            return torch.tensor([b[i].data_ptr() for b in bufs], dtype=torch.int64, device=dev)
+
+        c8, s8, c4, s4 = ptrs(r8, 0), ptrs(r8, 1), ptrs(r4, 0), ptrs(r4, 1)
+        pp_us, p8_us, p4_us = time_phases(
+            [lambda: B.moe_permute_to_peers(prob, d_hidden, buf.row_src, buf.pair_slot,
+                                            buf.meta, peer, put),
+             lambda: B.moe_permute_quant_fp8_to_peers(prob, d_hidden, buf.row_src,
+                                                      buf.pair_slot, buf.meta, c8, s8, put),
+             lambda: B.moe_permute_quant_nvfp4_to_peers(prob, d_hidden, buf.row_src,
+                                                        buf.pair_slot, buf.meta, d_gs, c4, s4,
+                                                        put)], f2_steps)
+        maps = 2 * w.N * w.H + 4 * w.P + 4 * buf.rows + 16 * w.S
+        routed = sum(seg_rows)
+        pp_bytes = maps + 2 * routed * w.H
+        p8_bytes = maps + routed * (w.H + 4 * (w.H // 128))
+        p4_bytes = maps + routed * (w.H // 2 + w.H // 16) + 4
         f2 = {"steps": f2_steps, "segments": w.S,
               "permute_to_peers_us": round(pp_us, 2),
               "permute_to_peers_gbs": round(pp_bytes / (pp_us * 1e-6) / 1e9, 1),
+              "permute_fp8_to_peers_us": round(p8_us, 2),
+              "permute_fp8_to_peers_gbs": round(p8_bytes / (p8_us * 1e-6) / 1e9, 1),
+              "permute_nvfp4_to_peers_us": round(p4_us, 2),
+              "permute_nvfp4_to_peers_gbs": round(p4_bytes / (p4_us * 1e-6) / 1e9, 1),
               "receivers": "S local buffers standing in for the peers' receive buffers "
                            "(one GPU); across GPUs the same stores go over NVLink"}
-        del recv, peer, put
+        del recv, peer, put, r8, r4, c8, s8, c4, s4
 
     # ---- backward (NEXT row f4): dispatch backward (gather-sum of the rows'
     # gradients) and combine backward (scaled scatter + gate gradients)

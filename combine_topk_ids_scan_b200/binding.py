@@ -52,7 +52,8 @@ MOE_MAX_TOPK = 16
 # every symbol include/moe_dc.h declares
 EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout",
             "moe_dispatch_layout_noalloc", "moe_permute", "moe_permute_premultiplied",
-            "moe_permute_to_peers",
+            "moe_permute_to_peers", "moe_permute_quant_fp8_to_peers",
+            "moe_permute_quant_nvfp4_to_peers",
             "moe_permute_quant_fp8",
             "moe_permute_quant_nvfp4", "moe_permute_quant_mxfp4", "moe_combine",
             "moe_permute_backward",
@@ -135,6 +136,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
     L.moe_permute.argtypes = [P] + [vp] * 5
     L.moe_permute_to_peers.restype = ctypes.c_int
     L.moe_permute_to_peers.argtypes = [P] + [vp] * 7
+    L.moe_permute_quant_fp8_to_peers.restype = ctypes.c_int
+    L.moe_permute_quant_fp8_to_peers.argtypes = [P] + [vp] * 8
+    L.moe_permute_quant_nvfp4_to_peers.restype = ctypes.c_int
+    L.moe_permute_quant_nvfp4_to_peers.argtypes = [P] + [vp] * 9
     L.moe_permute_premultiplied.restype = ctypes.c_int
     L.moe_permute_premultiplied.argtypes = [P] + [vp] * 6
     L.moe_permute_quant_fp8.restype = ctypes.c_int
@@ -314,6 +319,43 @@ def moe_permute_to_peers(prob: Problem, hidden_states, row_src, pair_slot, meta,
                                        _ptr(pair_slot), _ptr(meta), _ptr(peer_out),
                                        _ptr(put_offsets), _stream(stream)),
            "moe_permute_to_peers")
+
+
+def moe_permute_quant_fp8_to_peers(prob: Problem, hidden_states, row_src, pair_slot, meta,
+                                   peer_codes, peer_scales, put_offsets, stream=None) -> None:
+    """FP8 dispatch whose segment s lands in rank s's receive buffers:
+    peer_codes / peer_scales are int64 device tensors of S device addresses
+    (E4M3 [rows, H] and fp32 [rows, H/128] buffers), put_offsets as in
+    moe_permute_to_peers (see moe_permute_quant_fp8_to_peers in moe_dc.h)."""
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_permute_quant_fp8_to_peers",
+             **_permute_need(prob, hidden_states, row_src, pair_slot), meta=(meta, 16 * S),
+             peer_codes=(peer_codes, 8 * S), peer_scales=(peer_scales, 8 * S),
+             put_offsets=(put_offsets, 8 * S))
+    c = prob.c()
+    _check(load().moe_permute_quant_fp8_to_peers(
+        ctypes.byref(c), _ptr(hidden_states), _ptr(row_src), _ptr(pair_slot), _ptr(meta),
+        _ptr(peer_codes), _ptr(peer_scales), _ptr(put_offsets), _stream(stream)),
+        "moe_permute_quant_fp8_to_peers")
+
+
+def moe_permute_quant_nvfp4_to_peers(prob: Problem, hidden_states, row_src, pair_slot, meta,
+                                     global_scale, peer_codes, peer_scales, put_offsets,
+                                     stream=None) -> None:
+    """NVFP4 dispatch whose segment s lands in rank s's receive buffers
+    (E2M1 [rows, H/2] codes, E4M3 [rows, H/16] row-major scales); see
+    moe_permute_quant_nvfp4_to_peers in moe_dc.h."""
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_permute_quant_nvfp4_to_peers",
+             **_permute_need(prob, hidden_states, row_src, pair_slot), meta=(meta, 16 * S),
+             global_scale=(global_scale, 4 if rows > 0 else 0),
+             peer_codes=(peer_codes, 8 * S), peer_scales=(peer_scales, 8 * S),
+             put_offsets=(put_offsets, 8 * S))
+    c = prob.c()
+    _check(load().moe_permute_quant_nvfp4_to_peers(
+        ctypes.byref(c), _ptr(hidden_states), _ptr(row_src), _ptr(pair_slot), _ptr(meta),
+        _ptr(global_scale), _ptr(peer_codes), _ptr(peer_scales), _ptr(put_offsets),
+        _stream(stream)), "moe_permute_quant_nvfp4_to_peers")
 
 
 def moe_permute_premultiplied(prob: Problem, hidden_states, row_src, pair_slot, gates, out,

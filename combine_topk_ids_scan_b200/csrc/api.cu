@@ -158,6 +158,52 @@ moe_status moe_permute_to_peers(const moe_problem *problem, const void *hidden_s
                                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_permute_quant_fp8_to_peers(const moe_problem *problem, const void *hidden_states,
+                                          const int32_t *row_src, const int32_t *pair_slot,
+                                          const uint32_t *meta, void *const *peer_codes,
+                                          void *const *peer_scales, const int64_t *put_offsets,
+                                          moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.rows == 0) return MOE_OK;
+  if (!row_src || !peer_codes || !peer_scales || !put_offsets || (s.Ce == 0 && !meta) ||
+      (s.P > 0 && (!hidden_states || !pair_slot)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(hidden_states, 16) || !aligned(row_src, 4) || !aligned(pair_slot, 4) ||
+      !aligned(meta, 4) || !aligned(peer_codes, 8) || !aligned(peer_scales, 8) ||
+      !aligned(put_offsets, 8))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_permute_fp8_to_peers(s, hidden_states, row_src, pair_slot, meta,
+                                                    peer_codes, peer_scales, put_offsets,
+                                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute_quant_nvfp4_to_peers(const moe_problem *problem,
+                                            const void *hidden_states, const int32_t *row_src,
+                                            const int32_t *pair_slot, const uint32_t *meta,
+                                            const float *global_scale, void *const *peer_codes,
+                                            void *const *peer_scales, const int64_t *put_offsets,
+                                            moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 32 != 0 || (s.flags & MOE_FLAG_NVFP4_SWIZZLED_SCALES))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.rows == 0) return MOE_OK;
+  if (!row_src || !peer_codes || !peer_scales || !put_offsets || !global_scale ||
+      (s.Ce == 0 && !meta) || (s.P > 0 && (!hidden_states || !pair_slot)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(hidden_states, 16) || !aligned(row_src, 4) || !aligned(pair_slot, 4) ||
+      !aligned(meta, 4) || !aligned(global_scale, 4) || !aligned(peer_codes, 8) ||
+      !aligned(peer_scales, 8) || !aligned(put_offsets, 8))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_permute_nvfp4_to_peers(
+      s, hidden_states, row_src, pair_slot, meta, global_scale, peer_codes, peer_scales,
+      put_offsets, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_permute_premultiplied(const moe_problem *problem, const void *hidden_states,
                                      const int32_t *row_src, const int32_t *pair_slot,
                                      const float *gates, void *out, moe_stream_t stream) {

@@ -57,6 +57,16 @@ cudaError_t launch_permute_premultiplied(const Shape &s, const void *hidden,
                                          const int32_t *row_src, const int32_t *pair_slot,
                                          const float *gates, void *out, cudaStream_t stream);
 
+cudaError_t launch_permute_fp8_to_peers(const Shape &s, const void *hidden,
+                                       const int32_t *row_src, const int32_t *pair_slot,
+                                       const uint32_t *meta, void *const *peer_codes,
+                                       void *const *peer_scales, const int64_t *put_offsets,
+                                       cudaStream_t stream);
+cudaError_t launch_permute_nvfp4_to_peers(const Shape &s, const void *hidden,
+                                         const int32_t *row_src, const int32_t *pair_slot,
+                                         const uint32_t *meta, const float *global_scale,
+                                         void *const *peer_codes, void *const *peer_scales,
+                                         const int64_t *put_offsets, cudaStream_t stream);
 cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t *row_src,
                                const int32_t *pair_slot, uint8_t *q, float *scales,
                                cudaStream_t stream);

@@ -159,6 +159,33 @@ __device__ __forceinline__ int segment_of(int64_t r, const int32_t *s_start,
   return (r >= s_start[lo] && r - s_start[lo] < s_rows[lo]) ? lo : -1;
 }
 
+// Segment starts and rows into shared memory: packed mode from meta rows 0-1
+// (elements), capacity mode the static blocks of L * Ce rows.  Called by
+// every thread; the caller synchronises the block afterwards.
+__device__ __forceinline__ void stage_segments(const uint32_t *__restrict__ meta, int32_t S,
+                                               int32_t H, int32_t static_seg_rows,
+                                               int32_t *s_start, int32_t *s_rows) {
+  for (int i = threadIdx.x; i < S; i += kThreads) {
+    if (static_seg_rows > 0) {
+      s_start[i] = i * static_seg_rows;
+      s_rows[i] = static_seg_rows;
+    } else {
+      s_start[i] = (int32_t)(__ldg(meta + S + i) / (uint32_t)H);
+      s_rows[i] = (int32_t)(__ldg(meta + i) / (uint32_t)H);
+    }
+  }
+}
+
+// Segment of local row r (-1: none) and, for a segment, r's row in that
+// rank's receive buffer.
+__device__ __forceinline__ int peer_dest(int64_t r, const int32_t *s_start, const int32_t *s_rows,
+                                         int32_t S, const int64_t *__restrict__ put,
+                                         int64_t &prow) {
+  const int sg = segment_of(r, s_start, s_rows, S);
+  prow = sg >= 0 ? __ldg(put + sg) + (r - s_start[sg]) : 0;
+  return sg;
+}
+
 // Destination of local row r (nullptr when r belongs to no segment).
 __device__ __forceinline__ uint4 *peer_row(int64_t r, const int32_t *s_start,
                                            const int32_t *s_rows, int32_t S,
@@ -181,17 +208,7 @@ __global__ void __launch_bounds__(kThreads)
   extern __shared__ int32_t seg_smem[];  // [S] starts, [S] rows
   int32_t *s_start = seg_smem, *s_rows = seg_smem + S;
   grid_dependency_wait();
-  // segments: packed mode from meta rows 0-1 (elements), capacity mode the
-  // static blocks of L * Ce rows
-  for (int i = threadIdx.x; i < S; i += kThreads) {
-    if (static_seg_rows > 0) {
-      s_start[i] = i * static_seg_rows;
-      s_rows[i] = static_seg_rows;
-    } else {
-      s_start[i] = (int32_t)(__ldg(meta + S + i) / (uint32_t)H);
-      s_rows[i] = (int32_t)(__ldg(meta + i) / (uint32_t)H);
-    }
-  }
+  stage_segments(meta, S, H, static_seg_rows, s_start, s_rows);
   __syncthreads();
   constexpr int U = kBf16Chunk / 8 / kWarp;  // 2
   const int lane = threadIdx.x % kWarp;
@@ -308,10 +325,47 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ------------------------------------------------------------------- FP8
+// One lane's 16 consecutive elements (a: the first 8, b: the next 8) of a
+// 1x128 block that 8 consecutive lanes share -> 16 E4M3 codes; returns the
+// block's scale amax / 448 (0 and zero codes for an all-zero block).  The
+// block amax is three xor-shuffles, so all 32 lanes call it together.
+__device__ __forceinline__ float fp8_quant16(const uint4 &a, const uint4 &b, uint4 &codes) {
+  const uint32_t wd[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  float f[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = bf16lo(wd[i]);
+    f[2 * i + 1] = bf16hi(wd[i]);
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = max_abs3(amax, f[2 * i], f[2 * i + 1]);
+  amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+  amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
+  uint32_t cw[4] = {0, 0, 0, 0};
+  float sc = 0.0f;
+  if (amax > 0.0f) {
+    sc = amax / 448.0f;  // IEEE round-to-nearest division
+    float2 qt[8];        // x / sc, |x / sc| <= 448
+    if (sc >= kQuotientMinDivisor && sc <= kQuotientMaxDivisor) {
+      const float rs = __frcp_rn(sc);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qt[i] = rn_quotient2(make_float2(f[2 * i], f[2 * i + 1]), sc, rs);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qt[i] = make_float2(f[2 * i] / sc, f[2 * i + 1] / sc);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) cw[i] = cvt_e4m3x4(qt[2 * i], qt[2 * i + 1]);
+  }
+  codes = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+  return sc;
+}
+
 // Unit = (token, 1024 elements).  A lane takes 16 consecutive elements per
 // half (two 16-byte loads -> one 16-byte store of codes); 8 lanes form one
-// 1x128 block, so the block amax is three xor-shuffles; a half-unit covers
-// 512 elements.
+// 1x128 block; a half-unit covers 512 elements.
 __global__ void __launch_bounds__(kThreads)
     permute_fp8_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                        const int32_t *__restrict__ pair_slot, uint8_t *__restrict__ q,
@@ -361,39 +415,7 @@ __global__ void __launch_bounds__(kThreads)
     uint4 codes[U];
     float scale[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const uint32_t wd[8] = {a[u].x, a[u].y, a[u].z, a[u].w, b[u].x, b[u].y, b[u].z, b[u].w};
-      float f[16];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        f[2 * i] = bf16lo(wd[i]);
-        f[2 * i + 1] = bf16hi(wd[i]);
-      }
-      float amax = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = max_abs3(amax, f[2 * i], f[2 * i + 1]);
-      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
-      uint32_t cw[4] = {0, 0, 0, 0};
-      float sc = 0.0f;
-      if (amax > 0.0f) {
-        sc = amax / 448.0f;  // IEEE round-to-nearest division
-        float2 qt[8];        // x / sc, |x / sc| <= 448
-        if (sc >= kQuotientMinDivisor && sc <= kQuotientMaxDivisor) {
-          const float rs = __frcp_rn(sc);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) qt[i] = rn_quotient2(make_float2(f[2 * i], f[2 * i + 1]), sc, rs);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) qt[i] = make_float2(f[2 * i] / sc, f[2 * i + 1] / sc);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) cw[i] = cvt_e4m3x4(qt[2 * i], qt[2 * i + 1]);
-      }
-      codes[u] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      scale[u] = sc;
-    }
+    for (int u = 0; u < U; ++u) scale[u] = fp8_quant16(a[u], b[u], codes[u]);
     while (live) {
       const int j = __ffs(live) - 1;
       live &= live - 1;
@@ -477,15 +499,13 @@ __device__ __forceinline__ int64_t sf_atom_offset(int64_t m, int32_t c, int32_t 
 
 // MX == false: NVFP4 (two 16-element blocks per lane, E4M3 scales);
 // MX == true: MXFP4 (one 32-element block per lane, E8M0 scales).
-// SWIZZLED: scales in the block-scale atom layout.  PAD_SCALES == false
-// (linear scales that scales_to_atoms_kernel converts next): padding rows'
-// scales are left unwritten, the atom kernel zeroes them.  The token row's loads
+// SWIZZLED: scales in the block-scale atom layout.  The token row's loads
 // are issued first, before the pair_slot load and its ballot.  The MXFP4
 // linear-scale kernel is held to 5 resident CTAs per SM (at most 48
 // registers; measured on B200 at the metric shape: 61.4 -> 60.0 us), the
 // NVFP4 and the atom-layout kernels to 4 (NVFP4 with its loads first: 65.5 us
 // at 5 CTAs with a 4-byte spill, 63.5 us at 4 without one).
-template <bool MX, bool SWIZZLED, bool PAD_SCALES = true>
+template <bool MX, bool SWIZZLED>
 __global__ void __launch_bounds__(kThreads, (SWIZZLED || !MX) ? 4 : 5)
     permute_fp4_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ row_src,
                        const int32_t *__restrict__ pair_slot,
@@ -526,14 +546,13 @@ __global__ void __launch_bounds__(kThreads, (SWIZZLED || !MX) ? 4 : 5)
         const int64_t row = g * kWarp + j;
         uint4 *dst = reinterpret_cast<uint4 *>(q) + row * (qrow / 16);
         for (int v = v0 + lane; v < v1; v += kWarp) st_v4(dst + v, zero);
-        if (PAD_SCALES)
-          for (int v = s0 + lane; v < s1; v += kWarp) scales[row * srow + v] = 0;
+        for (int v = s0 + lane; v < s1; v += kWarp) scales[row * srow + v] = 0;
       }
     } else if (m && !swizzled) {
       int32_t s0, s1;
       share_of(c, psplit, srow / 2, s0, s1);
       zero_rows(m, g, lane, reinterpret_cast<uint4 *>(q), qrow / 16, v0, v1,
-                PAD_SCALES ? reinterpret_cast<uint16_t *>(scales) : nullptr, srow / 2, s0, s1);
+                reinterpret_cast<uint16_t *>(scales), srow / 2, s0, s1);
     } else if (m) {
       int32_t g0, g1;
       share_of(c, psplit, groups, g0, g1);
@@ -631,6 +650,204 @@ __global__ void __launch_bounds__(kThreads, (SWIZZLED || !MX) ? 4 : 5)
   }
 }
 
+// ------------------------------------------- quantised dispatch to peers
+// The FP8 and NVFP4 dispatches with the send fused in, as
+// permute_to_peers_kernel does for bf16 rows: the codes and the linear
+// scales of local row r of segment s are stored into rank s's receive
+// buffers peer_codes[s] / peer_scales[s] at row put[s] + (r - start_s), in
+// the layouts of moe_permute_quant_fp8 / moe_permute_quant_nvfp4 (row-major
+// scales).  The units and arithmetic of permute_fp8_kernel and of
+// permute_fp4_kernel's NVFP4 path; a lane holding pair j finds its row's
+// segment and receive row, and the warp broadcasts both.  Padding rows
+// inside a segment are zeroed at the destination; rows past the last
+// segment are not sent.
+__global__ void __launch_bounds__(kThreads)
+    permute_fp8_to_peers_kernel(const uint4 *__restrict__ hidden,
+                                const int32_t *__restrict__ row_src,
+                                const int32_t *__restrict__ pair_slot,
+                                const uint32_t *__restrict__ meta,
+                                uint8_t *const *__restrict__ peer_codes,
+                                float *const *__restrict__ peer_scales,
+                                const int64_t *__restrict__ put, int32_t N, int32_t k,
+                                int64_t rows, int32_t H, int32_t chunks, int32_t psplit, int32_t S,
+                                int32_t static_seg_rows) {
+  MOE_TRACE_CTA(MOE_TRACE_PERMUTE_FP8_TO_PEERS, 0);
+  allow_dependents();
+  extern __shared__ int32_t seg_smem[];  // [S] starts, [S] rows
+  int32_t *s_start = seg_smem, *s_rows = seg_smem + S;
+  grid_dependency_wait();
+  stage_segments(meta, S, H, static_seg_rows, s_start, s_rows);
+  __syncthreads();
+  constexpr int U = kChunk / 512;  // 2
+  const int lane = threadIdx.x % kWarp;
+  const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
+  const int64_t units = (int64_t)N * chunks;
+  const int64_t pad_units = (rows + kWarp - 1) / kWarp * psplit;
+  const int32_t vecs = H / 8;
+  const int32_t nb = H / 128;
+  if (w0 < pad_units) {
+    const int64_t g = w0 / psplit;
+    uint32_t m = padding_mask(g, lane, row_src, rows, rows);
+    const int c = (int)(w0 % psplit);
+    int32_t v0, v1, s0, s1;
+    share_of(c, psplit, H / 16, v0, v1);
+    share_of(c, psplit, nb, s0, s1);
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    while (m) {
+      const int j = __ffs(m) - 1;
+      m &= m - 1;
+      int64_t pr;
+      const int sg = peer_dest(g * kWarp + j, s_start, s_rows, S, put, pr);
+      if (sg < 0) continue;
+      uint4 *qd = reinterpret_cast<uint4 *>(peer_codes[sg] + pr * H);
+      float *sd = peer_scales[sg] + pr * nb;
+      for (int v = v0 + lane; v < v1; v += kWarp) st_v4(qd + v, zero);
+      for (int v = s0 + lane; v < s1; v += kWarp) sd[v] = 0.0f;
+    }
+    return;
+  }
+  const int64_t w = w0 - pad_units;
+  if (w >= units) return;
+  const int64_t t = w / chunks;
+  const int c0 = (int)(w % chunks) * kChunk;
+  const uint4 *src = hidden + t * vecs;
+  uint4 a[U], b[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int col = c0 + u * 512 + lane * 16;
+    if (col < H) {
+      a[u] = ld_stream_v4(src + col / 8);
+      b[u] = ld_stream_v4(src + col / 8 + 1);
+    } else {
+      a[u] = b[u] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  int32_t my_slot;
+  uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+  int64_t my_prow = 0;
+  const int my_sg = my_slot >= 0 ? peer_dest(my_slot, s_start, s_rows, S, put, my_prow) : -1;
+  live &= __ballot_sync(kFull, my_sg >= 0);
+  uint4 codes[U];
+  float scale[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) scale[u] = fp8_quant16(a[u], b[u], codes[u]);
+  while (live) {
+    const int j = __ffs(live) - 1;
+    live &= live - 1;
+    const int sg = __shfl_sync(kFull, my_sg, j);
+    const int64_t pr = __shfl_sync(kFull, my_prow, j);
+    uint8_t *qd = peer_codes[sg] + pr * H;
+    float *sd = peer_scales[sg] + pr * nb;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int col = c0 + u * 512 + lane * 16;
+      if (col < H) {
+        st_v4(reinterpret_cast<uint4 *>(qd + col), codes[u]);
+        if ((lane & 7) == 0) sd[col / 128] = scale[u];
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 4)
+    permute_nvfp4_to_peers_kernel(const uint4 *__restrict__ hidden,
+                                  const int32_t *__restrict__ row_src,
+                                  const int32_t *__restrict__ pair_slot,
+                                  const uint32_t *__restrict__ meta,
+                                  const float *__restrict__ global_scale,
+                                  uint8_t *const *__restrict__ peer_codes,
+                                  uint8_t *const *__restrict__ peer_scales,
+                                  const int64_t *__restrict__ put, int32_t N, int32_t k,
+                                  int64_t rows, int32_t H, int32_t chunks, int32_t psplit,
+                                  int32_t S, int32_t static_seg_rows) {
+  MOE_TRACE_CTA(MOE_TRACE_PERMUTE_NVFP4_TO_PEERS, 0);
+  allow_dependents();
+  extern __shared__ int32_t seg_smem[];  // [S] starts, [S] rows
+  int32_t *s_start = seg_smem, *s_rows = seg_smem + S;
+  grid_dependency_wait();
+  stage_segments(meta, S, H, static_seg_rows, s_start, s_rows);
+  __syncthreads();
+  const int lane = threadIdx.x % kWarp;
+  const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
+  const int64_t units = (int64_t)N * chunks;
+  const int64_t pad_units = (rows + kWarp - 1) / kWarp * psplit;
+  const int32_t vecs = H / 8;
+  const int32_t qrow = H / 2, srow = H / 16;
+  if (w0 < pad_units) {
+    const int64_t g = w0 / psplit;
+    uint32_t m = padding_mask(g, lane, row_src, rows, rows);
+    const int c = (int)(w0 % psplit);
+    int32_t v0, v1, s0, s1;
+    share_of(c, psplit, qrow / 16, v0, v1);  // 16-byte code vectors
+    share_of(c, psplit, srow / 2, s0, s1);   // 2-byte scale pairs
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    while (m) {
+      const int j = __ffs(m) - 1;
+      m &= m - 1;
+      int64_t pr;
+      const int sg = peer_dest(g * kWarp + j, s_start, s_rows, S, put, pr);
+      if (sg < 0) continue;
+      uint4 *qd = reinterpret_cast<uint4 *>(peer_codes[sg] + pr * qrow);
+      uint16_t *sd = reinterpret_cast<uint16_t *>(peer_scales[sg] + pr * srow);
+      for (int v = v0 + lane; v < v1; v += kWarp) st_v4(qd + v, zero);
+      for (int v = s0 + lane; v < s1; v += kWarp) sd[v] = 0;
+    }
+    return;
+  }
+  const int64_t w = w0 - pad_units;
+  if (w >= units) return;
+  const int64_t t = w / chunks;
+  const int col = (int)(w % chunks) * kChunk + lane * 32;
+  const bool active = col < H;
+  const uint4 *src = hidden + t * vecs;
+  uint4 x[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    x[i] = active ? ld_stream_v4(src + col / 8 + i) : make_uint4(0, 0, 0, 0);
+  int32_t my_slot;
+  uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+  int64_t my_prow = 0;
+  const int my_sg = my_slot >= 0 ? peer_dest(my_slot, s_start, s_rows, S, put, my_prow) : -1;
+  live &= __ballot_sync(kFull, my_sg >= 0);
+  const float gs = __ldg(global_scale);
+  // two 16-element blocks, one at a time (16 floats live)
+  float f[16];
+  uint4 codes;
+  uint32_t sq = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint4 v = x[2 * h + i];
+      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        f[8 * i + 2 * e] = bf16lo(wd[e]);
+        f[8 * i + 2 * e + 1] = bf16hi(wd[e]);
+      }
+    }
+    uint32_t lo, hi;
+    sq |= nvfp4_block(f, gs, lo, hi) << (8 * h);
+    if (h == 0) {
+      codes.x = lo;
+      codes.y = hi;
+    } else {
+      codes.z = lo;
+      codes.w = hi;
+    }
+  }
+  while (live) {
+    const int j = __ffs(live) - 1;
+    live &= live - 1;
+    const int sg = __shfl_sync(kFull, my_sg, j);
+    const int64_t pr = __shfl_sync(kFull, my_prow, j);
+    if (active) {
+      st_v4(reinterpret_cast<uint4 *>(peer_codes[sg] + pr * qrow + col / 2), codes);
+      *reinterpret_cast<uint16_t *>(peer_scales[sg] + pr * srow + col / 16) = (uint16_t)sq;
+    }
+  }
+}
+
 // Block-scale atom layout from linear scales, in place, one CTA per 128-row
 // tile.  When the scale columns per row (nsf) are a multiple of 4, a tile's
 // linear scales ([128, nsf] row-major, rows past `rows` unwritten) and its
@@ -638,9 +855,11 @@ __global__ void __launch_bounds__(kThreads, (SWIZZLED || !MX) ? 4 : 5)
 // the permute writes linear scales there first (whole 64- or 32-byte runs
 // per warp instead of 4-byte pieces of 8 different rows per 32-byte sector)
 // and this kernel reads the whole tile into shared memory, then writes it
-// back in atom order.  The permute leaves the padding rows' scales unwritten
-// (row_src -1): this kernel reads only the rows that hold a token and writes
-// zeros for the others and for rows at or past `rows`.  Shared layout:
+// back in atom order; rows at or past `rows` become zeros.  (Leaving the
+// padding rows' scales to this kernel -- the permute skips them, this kernel
+// reads row_src first and loads only rows that hold a token -- measured the
+// same on B200 at the metric shape with 128-padded experts: the permute
+// 4 us faster, this kernel 3.5 us slower.)  Shared layout:
 // word (m, g) of 4-scale group g at g * 129 + (m % 32) * 4 + m / 32 -- the
 // atom order, so the write-back reads consecutive words, padded by one word
 // per group so that the scattered writes of a warp (consecutive g) fall in
@@ -671,8 +890,7 @@ __device__ __forceinline__ uint32_t atom_vec_slot(int32_t m, int32_t g) {
 
 template <bool VEC>
 __global__ void __launch_bounds__(kAtomThreads)
-    scales_to_atoms_kernel(uint32_t *__restrict__ scales, const int32_t *__restrict__ row_src,
-                           int64_t rows, int32_t groups) {
+    scales_to_atoms_kernel(uint32_t *__restrict__ scales, int64_t rows, int32_t groups) {
   MOE_TRACE_CTA(MOE_TRACE_SCALES_TO_ATOMS, VEC ? 1 : 0);
   allow_dependents();
   extern __shared__ uint32_t tile_words[];
@@ -682,36 +900,27 @@ __global__ void __launch_bounds__(kAtomThreads)
   const int32_t nrows = left < 128 ? (int32_t)left : 128;
   uint32_t *base = scales + tile * 128 * groups;  // the tile's words (either layout)
   const int32_t words = 128 * groups;
-  // bit m of s_live: row m of the tile holds a token (its scales were written)
-  __shared__ uint32_t s_live[4];
-  if (threadIdx.x < 128) {
-    const int32_t m = threadIdx.x;
-    const bool live = m < nrows && row_src[tile * 128 + m] >= 0;
-    const uint32_t bits = __ballot_sync(0xFFFFFFFFu, live);
-    if (m % kWarp == 0) s_live[m / kWarp] = bits;
-  }
-  __syncthreads();
-  const auto live = [&](int32_t m) { return ((s_live[m >> 5] >> (m & 31)) & 1u) != 0u; };
   const auto put = [&](int32_t w, uint32_t v) {  // linear word w -> shared, atom order
     const int32_t m = w / groups, g = w - m * groups;
-    tile_words[g * kAtomGroupWords + (m & 31) * 4 + (m >> 5)] = v;
+    tile_words[g * kAtomGroupWords + (m & 31) * 4 + (m >> 5)] = m < nrows ? v : 0u;
   };
   if constexpr (VEC) {
     // groups % 4 == 0 (the scale columns are a multiple of 16), so a vector
     // never straddles two rows
     const uint4 *vb = reinterpret_cast<const uint4 *>(base);
     const int32_t vecs = words / 4;
+    const int32_t valid = nrows * groups / 4;  // vectors of rows < nrows
     for (int32_t v0 = threadIdx.x; v0 < vecs; v0 += kAtomThreads * kAtomBatch) {
       uint4 x[kAtomBatch];
 #pragma unroll
       for (int b = 0; b < kAtomBatch; ++b) {
         const int32_t v = v0 + b * kAtomThreads;
-        x[b] = v < vecs && live(4 * v / groups) ? vb[v] : make_uint4(0, 0, 0, 0);
+        x[b] = v < valid ? vb[v] : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int b = 0; b < kAtomBatch; ++b) {
         const int32_t v = v0 + b * kAtomThreads;
-        if (v < vecs) {  // words (m, g0 .. g0 + 3); rows without a token were loaded as 0
+        if (v < vecs) {  // words (m, g0 .. g0 + 3); rows past nrows were loaded as 0
           const int32_t m = 4 * v / groups, g0 = 4 * v - m * groups;
           uint32_t *t = tile_words + atom_vec_slot(m, g0);  // g0 .. g0+3 share g / 4
           t[0] = x[b].x;
@@ -737,8 +946,7 @@ __global__ void __launch_bounds__(kAtomThreads)
       ob[v] = o;
     }
   } else {
-    for (int32_t w = threadIdx.x; w < words; w += kAtomThreads)
-      put(w, live(w / groups) ? base[w] : 0u);
+    for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) put(w, w < nrows * groups ? base[w] : 0u);
     __syncthreads();
     for (int32_t w = threadIdx.x; w < words; w += kAtomThreads) {
       const int32_t g = w >> 7, wi = w & 127;
@@ -816,6 +1024,41 @@ cudaError_t launch_permute_to_peers(const Shape &s, const void *hidden, const in
                     s.H / 8, chunks, ps, s.S, s.H, static_seg);
 }
 
+cudaError_t launch_permute_fp8_to_peers(const Shape &s, const void *hidden,
+                                       const int32_t *row_src, const int32_t *pair_slot,
+                                       const uint32_t *meta, void *const *peer_codes,
+                                       void *const *peer_scales, const int64_t *put_offsets,
+                                       cudaStream_t stream) {
+  if (s.rows == 0) return cudaSuccess;
+  const int32_t chunks = chunks_of(s.H, kChunk);
+  const int32_t ps = padding_split(s, chunks);
+  const int32_t static_seg = s.Ce > 0 ? (s.E / s.S) * s.Ce : 0;
+  return launch_pdl(permute_fp8_to_peers_kernel,
+                    dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads),
+                    (size_t)2 * s.S * sizeof(int32_t), stream, static_cast<const uint4 *>(hidden),
+                    row_src, pair_slot, meta, reinterpret_cast<uint8_t *const *>(peer_codes),
+                    reinterpret_cast<float *const *>(peer_scales), put_offsets, s.N, s.k, s.rows,
+                    s.H, chunks, ps, s.S, static_seg);
+}
+
+cudaError_t launch_permute_nvfp4_to_peers(const Shape &s, const void *hidden,
+                                         const int32_t *row_src, const int32_t *pair_slot,
+                                         const uint32_t *meta, const float *global_scale,
+                                         void *const *peer_codes, void *const *peer_scales,
+                                         const int64_t *put_offsets, cudaStream_t stream) {
+  if (s.rows == 0) return cudaSuccess;
+  const int32_t chunks = chunks_of(s.H, kChunk);
+  const int32_t ps = padding_split(s, chunks);
+  const int32_t static_seg = s.Ce > 0 ? (s.E / s.S) * s.Ce : 0;
+  return launch_pdl(permute_nvfp4_to_peers_kernel,
+                    dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads),
+                    (size_t)2 * s.S * sizeof(int32_t), stream, static_cast<const uint4 *>(hidden),
+                    row_src, pair_slot, meta, global_scale,
+                    reinterpret_cast<uint8_t *const *>(peer_codes),
+                    reinterpret_cast<uint8_t *const *>(peer_scales), put_offsets, s.N, s.k,
+                    s.rows, s.H, chunks, ps, s.S, static_seg);
+}
+
 cudaError_t launch_permute_fp8(const Shape &s, const void *hidden, const int32_t *row_src,
                                const int32_t *pair_slot, uint8_t *q, float *scales,
                                cudaStream_t stream) {
@@ -835,7 +1078,7 @@ inline bool atoms_in_place(int32_t nsf) {
 }
 
 cudaError_t launch_scales_to_atoms(const Shape &s, int32_t nsf, uint8_t *scales,
-                                   const int32_t *row_src, cudaStream_t stream) {
+                                   cudaStream_t stream) {
   const bool vec = reinterpret_cast<uintptr_t>(scales) % 16 == 0 && (nsf / 4) % 4 == 0;
   // both layouts get the padded size: 3 tiles per SM at H = 7168 (the
   // vector layout's exact 56 KB would fit 4; measured slower on B200, 19.1
@@ -848,7 +1091,7 @@ cudaError_t launch_scales_to_atoms(const Shape &s, int32_t nsf, uint8_t *scales,
     if (err != cudaSuccess) return err;
   }
   return launch_pdl(kernel, dim3((unsigned)((s.rows + 127) / 128)), dim3(kAtomThreads), smem,
-                    stream, reinterpret_cast<uint32_t *>(scales), row_src, s.rows, nsf / 4);
+                    stream, reinterpret_cast<uint32_t *>(scales), s.rows, nsf / 4);
 }
 
 cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32_t *row_src,
@@ -860,12 +1103,11 @@ cudaError_t launch_permute_nvfp4(const Shape &s, const void *hidden, const int32
   const int32_t ps = padding_split(s, chunks);
   if (swizzled && atoms_in_place(s.H / 16)) {
     const cudaError_t err = launch_pdl(
-        permute_fp4_kernel<false, false, false>,
-        dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads), 0, stream,
-        static_cast<const uint4 *>(hidden), row_src, pair_slot, global_scale, q, scales, s.N,
-        s.k, s.rows, s.H, chunks, ps);
+        permute_fp4_kernel<false, false>, dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)),
+        dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src, pair_slot,
+        global_scale, q, scales, s.N, s.k, s.rows, s.H, chunks, ps);
     if (err != cudaSuccess) return err;
-    return launch_scales_to_atoms(s, s.H / 16, scales, row_src, stream);
+    return launch_scales_to_atoms(s, s.H / 16, scales, stream);
   }
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
   return launch_pdl(swizzled ? permute_fp4_kernel<false, true> : permute_fp4_kernel<false, false>,
@@ -883,12 +1125,11 @@ cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32
   const int32_t ps = padding_split(s, chunks);
   if (swizzled && atoms_in_place(s.H / 32)) {
     const cudaError_t err = launch_pdl(
-        permute_fp4_kernel<true, false, false>,
-        dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads), 0, stream,
-        static_cast<const uint4 *>(hidden), row_src, pair_slot,
+        permute_fp4_kernel<true, false>, dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)),
+        dim3(kThreads), 0, stream, static_cast<const uint4 *>(hidden), row_src, pair_slot,
         static_cast<const float *>(nullptr), q, scales, s.N, s.k, s.rows, s.H, chunks, ps);
     if (err != cudaSuccess) return err;
-    return launch_scales_to_atoms(s, s.H / 32, scales, row_src, stream);
+    return launch_scales_to_atoms(s, s.H / 32, scales, stream);
   }
   const int64_t check_rows = swizzled ? (s.rows + 127) / 128 * 128 : s.rows;
   return launch_pdl(swizzled ? permute_fp4_kernel<true, true> : permute_fp4_kernel<true, false>,

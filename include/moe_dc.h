@@ -21,8 +21,8 @@
  * expert rows that hold a token, as bf16 or requantised), the gradients
  * moe_permute_backward and moe_combine_backward, moe_permute_premultiplied
  * (the dispatch with each pair's row scaled by its gate), moe_permute_to_peers
- * (the dispatch written straight into the receive buffers of the ranks that
- * own the experts), and moe_dispatch_layout_noalloc (the layout without a
+ * and its FP8 / NVFP4 forms (the dispatch written straight into the receive
+ * buffers of the ranks that own the experts), and moe_dispatch_layout_noalloc (the layout without a
  * caller workspace).  Two builds of the same sources add checks and records:
  * device index checks (moe_debug_violations) and per-CTA trace records
  * (moe_trace_attach).
@@ -282,6 +282,48 @@ MOE_API moe_status moe_permute_to_peers(const moe_problem *problem, const void *
                                         const uint32_t *meta, void *const *peer_out,
                                         const int64_t *put_offsets, moe_stream_t stream);
 
+/* The FP8 and NVFP4 dispatches fused with the expert-parallel send, as
+ * moe_permute_to_peers is for bf16 rows: the codes and scales that
+ * moe_permute_quant_fp8 / moe_permute_quant_nvfp4 would write to local row r
+ * of segment s are stored to row put_offsets[s] + (r - start of segment s)
+ * of rank s's receive buffers peer_codes[s] and peer_scales[s] (padding
+ * rows inside a segment as zeros; rows past the last segment are not
+ * written).  Mojo MAX ep.dispatch_async.block.scaled.nv (the EP dispatch
+ * with an NVFP4 payload and a per-tensor global input scale) and ep_comm
+ * (BlockwiseFP8TokenFormat, NVBlockScaledTokenFormat); segments as in
+ * moe_permute_to_peers.  Receive layouts, per rank s (rows = that rank's
+ * receive rows):
+ *   FP8    peer_codes[s]  E4M3 [rows, H], 16-byte aligned
+ *          peer_scales[s] fp32 [rows, H/128] (row-major), 4-byte aligned
+ *   NVFP4  peer_codes[s]  E2M1 [rows, H/2] (element 2m in the low nibble of
+ *                         byte m), 16-byte aligned
+ *          peer_scales[s] E4M3 [rows, H/16] row-major, 2-byte aligned
+ *   peer_codes, peer_scales  DEVICE arrays of S device pointers (8-byte
+ *                  aligned arrays; every pointer writable from this GPU)
+ *   put_offsets    DEVICE int64 [S], rows, as in moe_permute_to_peers
+ *   global_scale   NVFP4: DEVICE fp32 scalar, as in moe_permute_quant_nvfp4
+ * Requires H % 128 == 0 (FP8) or H % 32 == 0 (NVFP4);
+ * MOE_FLAG_NVFP4_SWIZZLED_SCALES is not supported here (rejected with
+ * MOE_ERR_UNSUPPORTED_SHAPE): the atom layout tiles a receive buffer by 128
+ * rows, which the receiver arranges over all of its sources. */
+MOE_API moe_status moe_permute_quant_fp8_to_peers(const moe_problem *problem,
+                                                  const void *hidden_states,
+                                                  const int32_t *row_src,
+                                                  const int32_t *pair_slot, const uint32_t *meta,
+                                                  void *const *peer_codes,
+                                                  void *const *peer_scales,
+                                                  const int64_t *put_offsets, moe_stream_t stream);
+MOE_API moe_status moe_permute_quant_nvfp4_to_peers(const moe_problem *problem,
+                                                    const void *hidden_states,
+                                                    const int32_t *row_src,
+                                                    const int32_t *pair_slot,
+                                                    const uint32_t *meta,
+                                                    const float *global_scale,
+                                                    void *const *peer_codes,
+                                                    void *const *peer_scales,
+                                                    const int64_t *put_offsets,
+                                                    moe_stream_t stream);
+
 /* Permute with pre-multiplied gates: out[slot(t,j), :] = bf16(gates[t,j] *
  * hidden_states[t, :]) -- one fp32 product and one rounding to nearest even
  * per element -- and zeros in the rows no pair owns.  DeepSpeed v0.19.4
@@ -511,7 +553,9 @@ typedef enum moe_trace_kernel {
   MOE_TRACE_PERMUTE_BACKWARD = 14,     /* variant as MOE_TRACE_COMBINE             */
   MOE_TRACE_COMBINE_BACKWARD = 15,     /* variant as MOE_TRACE_COMBINE             */
   MOE_TRACE_SWIGLU_SPLIT = 16,         /* variant: the MOE_QUANT_* format          */
-  MOE_TRACE_SWIGLU_QUANT = 17          /* variant: the MOE_QUANT_* format          */
+  MOE_TRACE_SWIGLU_QUANT = 17,         /* variant: the MOE_QUANT_* format          */
+  MOE_TRACE_PERMUTE_FP8_TO_PEERS = 18,
+  MOE_TRACE_PERMUTE_NVFP4_TO_PEERS = 19
 } moe_trace_kernel;
 
 /* Attach the trace record buffer (the build with -DMOE_TRACE): the kernels

@@ -143,6 +143,8 @@ ALIGNMENT_RULES = {
     "moe_permute": ((), (16, 4, 4, 16)),
     "moe_permute_premultiplied": ((), (16, 4, 4, 4, 16)),
     "moe_permute_to_peers": ((), (16, 4, 4, 4, 8, 8)),
+    "moe_permute_quant_fp8_to_peers": ((), (16, 4, 4, 4, 8, 8, 8)),
+    "moe_permute_quant_nvfp4_to_peers": ((), (16, 4, 4, 4, 4, 8, 8, 8)),
     "moe_permute_quant_fp8": ((), (16, 4, 4, 16, 4)),
     "moe_permute_quant_nvfp4": ((), (16, 4, 4, 4, 16, 2)),
     "moe_permute_quant_mxfp4": ((), (16, 4, 4, 16, 1)),

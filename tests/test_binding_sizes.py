@@ -69,6 +69,13 @@ def cases():
         "moe_permute_premultiplied": (p, [bf16(N, H), m(R), m(N, K), f32(N, K), bf16(R, H)], ()),
         "moe_permute_to_peers": (p, [bf16(N, H), m(R), m(N, K), m(4, S),
                                      m(S, dtype=torch.int64), m(S, dtype=torch.int64)], ()),
+        "moe_permute_quant_fp8_to_peers": (p, [bf16(N, H), m(R), m(N, K), m(4, S),
+                                               m(S, dtype=torch.int64), m(S, dtype=torch.int64),
+                                               m(S, dtype=torch.int64)], ()),
+        "moe_permute_quant_nvfp4_to_peers": (p, [bf16(N, H), m(R), m(N, K), m(4, S), f32(1),
+                                                 m(S, dtype=torch.int64),
+                                                 m(S, dtype=torch.int64),
+                                                 m(S, dtype=torch.int64)], ()),
         "moe_permute_quant_fp8": (p, [bf16(N, H), m(R), m(N, K), u8(R, H), f32(R, H // 128)], ()),
         "moe_permute_quant_nvfp4": (p, [bf16(N, H), m(R), m(N, K), f32(1), u8(R, H // 2),
                                         u8(R, H // 16)], ()),

@@ -737,6 +737,87 @@ def test_permute_to_peers(orc, mode):
         assert np.all(untouched == BF16_POISON), s
 
 
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+@pytest.mark.parametrize("mode", ["packed", "padded", "capacity"])
+def test_quantised_permute_to_peers(orc, mode, fmt):
+    """moe_permute_quant_fp8_to_peers / moe_permute_quant_nvfp4_to_peers with
+    S local code and scale buffers standing in for the S ranks' receive
+    buffers: segment s of the oracle's FP8 / NVFP4 dispatch (codes and
+    row-major scales) lands at rows [put[s], put[s] + rows_s) of rank s's
+    buffers, bit for bit (padding rows inside a segment as zeros), and every
+    other row of every buffer keeps its poison."""
+    spec = dict(N=1500, H=384, E=24, k=3, S=4, p_mask=0.05, p_bad=0.01)
+    pad = 0
+    if mode == "padded":
+        pad = 8
+        spec["C"] = 1500 * 3 + 24 * 7
+    elif mode == "capacity":
+        spec["Ce"] = 150
+    w = custom(seed=41, with_out=False, **spec)
+    run = GpuRun(w, quant=False, combine=False, pad=pad)
+    ref = oracle_layout(orc, w, pad=pad)
+    assert_layout(run, ref)
+    H = w.H
+    if fmt == "fp8":
+        q_want, s_want = orc.permute_fp8(w.hidden, ref.row_src)
+        s_want = s_want.view(np.uint32)
+        code_w, scale_w, scale_dt = H, H // 128, torch.float32
+    else:
+        q_want, s_want = orc.permute_nvfp4(w.hidden, ref.row_src, w.global_scale)
+        code_w, scale_w, scale_dt = H // 2, H // 16, torch.uint8
+    L = w.E // w.S
+    if mode == "capacity":
+        starts = [s * L * w.expert_capacity for s in range(w.S)]
+        seg_rows = [L * w.expert_capacity] * w.S
+    else:
+        starts = [int(v) // H for v in ref.meta[1]]
+        seg_rows = [int(v) // H for v in ref.meta[0]]
+    rng = np.random.default_rng(13)
+    put = [int(rng.integers(0, 300)) for _ in range(w.S)]
+    codes = [poisoned_empty((put[s] + seg_rows[s] + 17, code_w), torch.uint8)
+             for s in range(w.S)]
+    scales = [poisoned_empty((put[s] + seg_rows[s] + 17, scale_w), scale_dt)
+              for s in range(w.S)]
+    pc = torch.tensor([t.data_ptr() for t in codes], dtype=torch.int64, device="cuda")
+    psc = torch.tensor([t.data_ptr() for t in scales], dtype=torch.int64, device="cuda")
+    put_d = torch.tensor(put, dtype=torch.int64, device="cuda")
+    hid = to_dev_bf16(w.hidden)
+    if fmt == "fp8":
+        B.moe_permute_quant_fp8_to_peers(run.prob, hid, run.buf.row_src, run.buf.pair_slot,
+                                         run.buf.meta, pc, psc, put_d)
+    else:
+        gs = torch.tensor([w.global_scale], dtype=torch.float32, device="cuda")
+        B.moe_permute_quant_nvfp4_to_peers(run.prob, hid, run.buf.row_src, run.buf.pair_slot,
+                                           run.buf.meta, gs, pc, psc, put_d)
+    torch.cuda.synchronize()
+    from gpu_util import BYTE_POISON, F32_POISON
+    for s in range(w.S):
+        lo, hi = put[s], put[s] + seg_rows[s]
+        got_q = codes[s].cpu().numpy()
+        got_s = scales[s].cpu().numpy()
+        if fmt == "fp8":
+            got_s = got_s.view(np.uint32)
+            s_poison = np.uint32(F32_POISON)
+        else:
+            s_poison = BYTE_POISON
+        assert np.array_equal(got_q[lo:hi], q_want[starts[s]:starts[s] + seg_rows[s]]), s
+        assert np.array_equal(got_s[lo:hi], s_want[starts[s]:starts[s] + seg_rows[s]]), s
+        assert np.all(np.concatenate([got_q[:lo], got_q[hi:]]) == BYTE_POISON), s
+        assert np.all(np.concatenate([got_s[:lo], got_s[hi:]]) == s_poison), s
+
+
+def test_quantised_permute_to_peers_rejects_the_atom_layout():
+    w = custom(N=64, H=256, E=8, k=2, S=2, seed=3, with_out=False)
+    prob = problem_of(w, flags=B.MOE_FLAG_NVFP4_SWIZZLED_SCALES)
+    z = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    i32 = torch.zeros(1 << 12, dtype=torch.int32, device="cuda")
+    p64 = torch.zeros(w.S, dtype=torch.int64, device="cuda")
+    with pytest.raises(B.MoeError) as e:
+        B.moe_permute_quant_nvfp4_to_peers(prob, z, i32, i32, i32, i32.view(torch.float32),
+                                           p64, p64, p64)
+    assert e.value.code == B.MOE_ERR_UNSUPPORTED_SHAPE
+
+
 def test_grouped_gemm_ready_dispatch_full_size(orc):
     """The f1 configuration the benchmark times: the metric workload with
     experts padded to 128 rows (recv_capacity = N*k + 127*E) and FP4 scales

@@ -135,6 +135,12 @@ def test_next_row_kernels_record_with_their_variants():
     seg = torch.empty((rows, H), dtype=torch.bfloat16, device="cuda")
     peer = torch.tensor([seg.data_ptr()] * w.S, dtype=torch.int64, device="cuda")
     put = torch.zeros(w.S, dtype=torch.int64, device="cuda")
+    bufs8 = (torch.empty((rows, H), dtype=torch.uint8, device="cuda"),
+             torch.empty((rows, H // 128), dtype=torch.float32, device="cuda"))
+    bufs4 = (torch.empty((rows, H // 2), dtype=torch.uint8, device="cuda"),
+             torch.empty((rows, H // 16), dtype=torch.uint8, device="cuda"))
+    q8 = [torch.tensor([t.data_ptr()] * w.S, dtype=torch.int64, device="cuda") for t in bufs8]
+    q4 = [torch.tensor([t.data_ptr()] * w.S, dtype=torch.int64, device="cuda") for t in bufs4]
     with T.Tracer() as tr:
         B.moe_permute_premultiplied(prob, hidden, buf.row_src, buf.pair_slot, gates, buf.out)
         B.moe_permute_backward(prob, X, buf.pair_slot, poisoned_empty((w.N, H), torch.bfloat16))
@@ -150,10 +156,15 @@ def test_next_row_kernels_record_with_their_variants():
         # every segment into the same buffer at offset 0 (each segment fits;
         # only the records matter here)
         B.moe_permute_to_peers(prob, hidden, buf.row_src, buf.pair_slot, buf.meta, peer, put)
+        B.moe_permute_quant_fp8_to_peers(prob, hidden, buf.row_src, buf.pair_slot, buf.meta,
+                                         *q8, put)
+        B.moe_permute_quant_nvfp4_to_peers(prob, hidden, buf.row_src, buf.pair_slot, buf.meta,
+                                           gs, *q4, put)
     got = [(launch.kernel, launch.variant) for launch in check_launches(tr)]
     nvfp4 = [g for g in got if g[0] in ("permute_nvfp4", "scales_to_atoms")]
     assert got[:3] == [("permute_premultiplied", 0), ("permute_backward", 8),
                        ("combine_backward", 8)]
     assert nvfp4 in ([("permute_nvfp4", 0), ("scales_to_atoms", 1)], [("permute_nvfp4", 1)])
-    assert got[-3:] == [("swiglu_split", B.MOE_QUANT_MXFP8),
-                        ("swiglu_quant", B.MOE_QUANT_MXFP6_E2M3), ("permute_to_peers", 0)]
+    assert got[-5:] == [("swiglu_split", B.MOE_QUANT_MXFP8),
+                        ("swiglu_quant", B.MOE_QUANT_MXFP6_E2M3), ("permute_to_peers", 0),
+                        ("permute_fp8_to_peers", 0), ("permute_nvfp4_to_peers", 0)]
