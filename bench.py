@@ -41,14 +41,15 @@ WORKLOAD = "fp8_metric"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, nominal (DGX figure)
 
-# dram bytes (read + write) per launch from one ncu --set full capture on the
-# metric workload (summaries under profiles/), keyed by kernel; valid only
-# while the kernel's source file is unchanged (sha256 prefix at capture time)
+# dram bytes (read + write) per launch from one ncu capture of the DRAM
+# counters on the metric workload (profiles/traffic_fp8_metric.md), keyed by
+# kernel; valid only while the kernel's device code is unchanged (sha256
+# prefix of its text and the shared helpers at capture time)
 NCU_TRAFFIC: dict[str, dict] = {
-    "permute_bf16": {"bytes_per_launch": 117985536 + 880217344, "src_sha": "a0218bc31711bbc1"},
-    "permute_fp8": {"bytes_per_launch": 118066944 + 422894336, "src_sha": "c6c0d1cc4d647560"},
-    "permute_nvfp4": {"bytes_per_launch": 118020096 + 207139584, "src_sha": "669914b64a79a75e"},
-    "combine": {"bytes_per_launch": 940131840 + 64447232, "src_sha": "709371a62977d2c7"},
+    "permute_bf16": {"bytes_per_launch": 118010880 + 881758976, "src_sha": "a0218bc31711bbc1"},
+    "permute_fp8": {"bytes_per_launch": 118075392 + 422765568, "src_sha": "28d14b0055d493d3"},
+    "permute_nvfp4": {"bytes_per_launch": 118034432 + 203461888, "src_sha": "84fc6bc2afa495d1"},
+    "combine": {"bytes_per_launch": 940088320 + 64898048, "src_sha": "709371a62977d2c7"},
 }
 
 

@@ -176,14 +176,48 @@ __device__ __forceinline__ void stage_segments(const uint32_t *__restrict__ meta
   }
 }
 
-// Segment of local row r (-1: none) and, for a segment, r's row in that
-// rank's receive buffer.
-__device__ __forceinline__ int peer_dest(int64_t r, const int32_t *s_start, const int32_t *s_rows,
-                                         int32_t S, const int64_t *__restrict__ put,
-                                         int64_t &prow) {
-  const int sg = segment_of(r, s_start, s_rows, S);
-  prow = sg >= 0 ? __ldg(put + sg) + (r - s_start[sg]) : 0;
-  return sg;
+// Per-rank table of the quantised peer kernels in shared memory: code and
+// scale buffer addresses and put offsets (8 bytes each), then the segment
+// starts and rows; 32 * S bytes.
+struct PeerTable {
+  uint8_t **codes;
+  uint8_t **scales;
+  int64_t *put;
+  int32_t *start;
+  int32_t *rows;
+};
+__device__ __forceinline__ PeerTable stage_peer_table(uint64_t *smem, const uint32_t *meta,
+                                                      int32_t S, int32_t H,
+                                                      int32_t static_seg_rows,
+                                                      uint8_t *const *peer_codes,
+                                                      uint8_t *const *peer_scales,
+                                                      const int64_t *__restrict__ put) {
+  PeerTable t;
+  t.codes = reinterpret_cast<uint8_t **>(smem);
+  t.scales = reinterpret_cast<uint8_t **>(smem + S);
+  t.put = reinterpret_cast<int64_t *>(smem + 2 * S);
+  t.start = reinterpret_cast<int32_t *>(smem + 3 * S);
+  t.rows = t.start + S;
+  stage_segments(meta, S, H, static_seg_rows, t.start, t.rows);
+  for (int i = threadIdx.x; i < S; i += kThreads) {
+    t.codes[i] = peer_codes[i];
+    t.scales[i] = peer_scales[i];
+    t.put[i] = __ldg(put + i);
+  }
+  return t;
+}
+
+// Code and scale row addresses of local row r in its rank's receive buffers
+// (false when r belongs to no segment).
+__device__ __forceinline__ bool peer_rows(int64_t r, const PeerTable &t, int32_t S,
+                                          int64_t code_bytes, int64_t scale_bytes,
+                                          uint8_t *&q, uint8_t *&sc) {
+  const int sg = segment_of(r, t.start, t.rows, S);
+  if (sg < 0) return false;
+  const int64_t pr = t.put[sg] + (r - t.start[sg]);
+  q = t.codes[sg] + pr * code_bytes;
+  sc = t.scales[sg] + pr * scale_bytes;
+  return true;
 }
 
 // Destination of local row r (nullptr when r belongs to no segment).
@@ -673,10 +707,11 @@ __global__ void __launch_bounds__(kThreads)
                                 int32_t static_seg_rows) {
   MOE_TRACE_CTA(MOE_TRACE_PERMUTE_FP8_TO_PEERS, 0);
   allow_dependents();
-  extern __shared__ int32_t seg_smem[];  // [S] starts, [S] rows
-  int32_t *s_start = seg_smem, *s_rows = seg_smem + S;
+  extern __shared__ uint64_t table_smem[];
   grid_dependency_wait();
-  stage_segments(meta, S, H, static_seg_rows, s_start, s_rows);
+  const PeerTable tab =
+      stage_peer_table(table_smem, meta, S, H, static_seg_rows,
+                       peer_codes, reinterpret_cast<uint8_t *const *>(peer_scales), put);
   __syncthreads();
   constexpr int U = kChunk / 512;  // 2
   const int lane = threadIdx.x % kWarp;
@@ -696,11 +731,10 @@ __global__ void __launch_bounds__(kThreads)
     while (m) {
       const int j = __ffs(m) - 1;
       m &= m - 1;
-      int64_t pr;
-      const int sg = peer_dest(g * kWarp + j, s_start, s_rows, S, put, pr);
-      if (sg < 0) continue;
-      uint4 *qd = reinterpret_cast<uint4 *>(peer_codes[sg] + pr * H);
-      float *sd = peer_scales[sg] + pr * nb;
+      uint8_t *q, *sc;
+      if (!peer_rows(g * kWarp + j, tab, S, H, 4 * nb, q, sc)) continue;
+      uint4 *qd = reinterpret_cast<uint4 *>(q);
+      float *sd = reinterpret_cast<float *>(sc);
       for (int v = v0 + lane; v < v1; v += kWarp) st_v4(qd + v, zero);
       for (int v = s0 + lane; v < s1; v += kWarp) sd[v] = 0.0f;
     }
@@ -724,9 +758,11 @@ __global__ void __launch_bounds__(kThreads)
   }
   int32_t my_slot;
   uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
-  int64_t my_prow = 0;
-  const int my_sg = my_slot >= 0 ? peer_dest(my_slot, s_start, s_rows, S, put, my_prow) : -1;
-  live &= __ballot_sync(kFull, my_sg >= 0);
+  // this lane's pair: its receive rows (resolved before the quantisation, so
+  // the pointer loads overlap it)
+  uint8_t *my_q = nullptr, *my_s = nullptr;
+  const bool mine = my_slot >= 0 && peer_rows(my_slot, tab, S, H, 4 * nb, my_q, my_s);
+  live &= __ballot_sync(kFull, mine);
   uint4 codes[U];
   float scale[U];
 #pragma unroll
@@ -734,10 +770,10 @@ __global__ void __launch_bounds__(kThreads)
   while (live) {
     const int j = __ffs(live) - 1;
     live &= live - 1;
-    const int sg = __shfl_sync(kFull, my_sg, j);
-    const int64_t pr = __shfl_sync(kFull, my_prow, j);
-    uint8_t *qd = peer_codes[sg] + pr * H;
-    float *sd = peer_scales[sg] + pr * nb;
+    uint8_t *qd = reinterpret_cast<uint8_t *>(
+        __shfl_sync(kFull, reinterpret_cast<unsigned long long>(my_q), j));
+    float *sd = reinterpret_cast<float *>(
+        __shfl_sync(kFull, reinterpret_cast<unsigned long long>(my_s), j));
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int col = c0 + u * 512 + lane * 16;
@@ -762,10 +798,10 @@ __global__ void __launch_bounds__(kThreads, 4)
                                   int32_t S, int32_t static_seg_rows) {
   MOE_TRACE_CTA(MOE_TRACE_PERMUTE_NVFP4_TO_PEERS, 0);
   allow_dependents();
-  extern __shared__ int32_t seg_smem[];  // [S] starts, [S] rows
-  int32_t *s_start = seg_smem, *s_rows = seg_smem + S;
+  extern __shared__ uint64_t table_smem[];
   grid_dependency_wait();
-  stage_segments(meta, S, H, static_seg_rows, s_start, s_rows);
+  const PeerTable tab =
+      stage_peer_table(table_smem, meta, S, H, static_seg_rows, peer_codes, peer_scales, put);
   __syncthreads();
   const int lane = threadIdx.x % kWarp;
   const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
@@ -784,11 +820,10 @@ __global__ void __launch_bounds__(kThreads, 4)
     while (m) {
       const int j = __ffs(m) - 1;
       m &= m - 1;
-      int64_t pr;
-      const int sg = peer_dest(g * kWarp + j, s_start, s_rows, S, put, pr);
-      if (sg < 0) continue;
-      uint4 *qd = reinterpret_cast<uint4 *>(peer_codes[sg] + pr * qrow);
-      uint16_t *sd = reinterpret_cast<uint16_t *>(peer_scales[sg] + pr * srow);
+      uint8_t *q, *sc;
+      if (!peer_rows(g * kWarp + j, tab, S, qrow, srow, q, sc)) continue;
+      uint4 *qd = reinterpret_cast<uint4 *>(q);
+      uint16_t *sd = reinterpret_cast<uint16_t *>(sc);
       for (int v = v0 + lane; v < v1; v += kWarp) st_v4(qd + v, zero);
       for (int v = s0 + lane; v < s1; v += kWarp) sd[v] = 0;
     }
@@ -806,9 +841,11 @@ __global__ void __launch_bounds__(kThreads, 4)
     x[i] = active ? ld_stream_v4(src + col / 8 + i) : make_uint4(0, 0, 0, 0);
   int32_t my_slot;
   uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
-  int64_t my_prow = 0;
-  const int my_sg = my_slot >= 0 ? peer_dest(my_slot, s_start, s_rows, S, put, my_prow) : -1;
-  live &= __ballot_sync(kFull, my_sg >= 0);
+  // this lane's pair: its receive rows (resolved before the quantisation, so
+  // the pointer loads overlap it)
+  uint8_t *my_q = nullptr, *my_s = nullptr;
+  const bool mine = my_slot >= 0 && peer_rows(my_slot, tab, S, qrow, srow, my_q, my_s);
+  live &= __ballot_sync(kFull, mine);
   const float gs = __ldg(global_scale);
   // two 16-element blocks, one at a time (16 floats live)
   float f[16];
@@ -839,11 +876,13 @@ __global__ void __launch_bounds__(kThreads, 4)
   while (live) {
     const int j = __ffs(live) - 1;
     live &= live - 1;
-    const int sg = __shfl_sync(kFull, my_sg, j);
-    const int64_t pr = __shfl_sync(kFull, my_prow, j);
+    uint8_t *qd = reinterpret_cast<uint8_t *>(
+        __shfl_sync(kFull, reinterpret_cast<unsigned long long>(my_q), j));
+    uint8_t *sd = reinterpret_cast<uint8_t *>(
+        __shfl_sync(kFull, reinterpret_cast<unsigned long long>(my_s), j));
     if (active) {
-      st_v4(reinterpret_cast<uint4 *>(peer_codes[sg] + pr * qrow + col / 2), codes);
-      *reinterpret_cast<uint16_t *>(peer_scales[sg] + pr * srow + col / 16) = (uint16_t)sq;
+      st_v4(reinterpret_cast<uint4 *>(qd + col / 2), codes);
+      *reinterpret_cast<uint16_t *>(sd + col / 16) = (uint16_t)sq;
     }
   }
 }
@@ -1024,6 +1063,15 @@ cudaError_t launch_permute_to_peers(const Shape &s, const void *hidden, const in
                     s.H / 8, chunks, ps, s.S, s.H, static_seg);
 }
 
+// Shared memory of the quantised peer kernels' table (PeerTable), and the
+// opt-in a kernel needs above the default 48 KB (S up to 2048: 64 KB).
+inline size_t peer_table_smem(int32_t S) { return (size_t)32 * S; }
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t smem) {
+  if (smem <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
 cudaError_t launch_permute_fp8_to_peers(const Shape &s, const void *hidden,
                                        const int32_t *row_src, const int32_t *pair_slot,
                                        const uint32_t *meta, void *const *peer_codes,
@@ -1033,9 +1081,12 @@ cudaError_t launch_permute_fp8_to_peers(const Shape &s, const void *hidden,
   const int32_t chunks = chunks_of(s.H, kChunk);
   const int32_t ps = padding_split(s, chunks);
   const int32_t static_seg = s.Ce > 0 ? (s.E / s.S) * s.Ce : 0;
+  const size_t smem = peer_table_smem(s.S);
+  const cudaError_t err = allow_smem(permute_fp8_to_peers_kernel, smem);
+  if (err != cudaSuccess) return err;
   return launch_pdl(permute_fp8_to_peers_kernel,
-                    dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads),
-                    (size_t)2 * s.S * sizeof(int32_t), stream, static_cast<const uint4 *>(hidden),
+                    dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads), smem,
+                    stream, static_cast<const uint4 *>(hidden),
                     row_src, pair_slot, meta, reinterpret_cast<uint8_t *const *>(peer_codes),
                     reinterpret_cast<float *const *>(peer_scales), put_offsets, s.N, s.k, s.rows,
                     s.H, chunks, ps, s.S, static_seg);
@@ -1050,9 +1101,12 @@ cudaError_t launch_permute_nvfp4_to_peers(const Shape &s, const void *hidden,
   const int32_t chunks = chunks_of(s.H, kChunk);
   const int32_t ps = padding_split(s, chunks);
   const int32_t static_seg = s.Ce > 0 ? (s.E / s.S) * s.Ce : 0;
+  const size_t smem = peer_table_smem(s.S);
+  const cudaError_t err = allow_smem(permute_nvfp4_to_peers_kernel, smem);
+  if (err != cudaSuccess) return err;
   return launch_pdl(permute_nvfp4_to_peers_kernel,
-                    dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads),
-                    (size_t)2 * s.S * sizeof(int32_t), stream, static_cast<const uint4 *>(hidden),
+                    dim3((unsigned)unit_blocks(s, chunks, s.rows, ps)), dim3(kThreads), smem,
+                    stream, static_cast<const uint4 *>(hidden),
                     row_src, pair_slot, meta, global_scale,
                     reinterpret_cast<uint8_t *const *>(peer_codes),
                     reinterpret_cast<uint8_t *const *>(peer_scales), put_offsets, s.N, s.k,
