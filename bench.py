@@ -326,6 +326,31 @@ def measure_workload(B, torch, w, dev, stream, flush_l2, n_steps: int, peak: flo
     step_us = timed(names, False)
     trio_us = timed(trio, False)
     per = dict(zip(names, timed(names, True)))
+
+    # launch-bound sizes (decode): the same step captured once into a CUDA
+    # graph and replayed, as a serving loop would run it
+    graph_us = None
+    if w.P <= 4096:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for nm in names:
+                calls[nm]()
+        for _ in range(3):
+            flush_l2()
+            graph.replay()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_steps)]
+        torch.cuda.synchronize(dev)
+        for a, b in ev:
+            flush_l2()
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        graph_us = 1e3 * sum(a.elapsed_time(b) for a, b in ev) / n_steps
+        del graph
     status = int(buf.status.cpu().numpy().view(np.uint32)[0])
     total_rows = int(buf.expert_counts.sum().item())
     nbytes = algorithmic_bytes(w, total_rows)
@@ -350,6 +375,9 @@ def measure_workload(B, torch, w, dev, stream, flush_l2, n_steps: int, peak: flo
         "launches_per_step": layout_launches(w.P) + len(names) - 1,
         "layout_status": status,
     }
+    if graph_us is not None:
+        out["graph_step_us"] = round(graph_us, 2)
+        out["graph_step_tokens_per_s"] = w.N / (graph_us * 1e-6)
     del buf, d_ids, d_hidden, d_gates, d_x, d_gs, d_y
     return out
 
