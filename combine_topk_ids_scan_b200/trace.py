@@ -12,9 +12,16 @@ them into launches; Tracer attaches a buffer around a block of calls:
         B.moe_permute(prob, hidden, buf.row_src, buf.pair_slot, buf.out)
     for launch in tr.launches():
         print(launch.kernel, launch.ctas, launch.duration_us)
+
+`python -m combine_topk_ids_scan_b200.trace [--workload NAME] [--steps K]`
+builds and loads the trace build and prints the per-kernel timeline of one
+benchmark step (layout, bf16 / FP8 / NVFP4 permutes, combine) on a seeded
+workload, the L2 flushed before every step.
 """
 from __future__ import annotations
 
+import argparse
+import statistics
 from dataclasses import dataclass
 
 import numpy as np
@@ -122,3 +129,88 @@ class Tracer:
 
     def launches(self) -> list[Launch]:
         return launches(self._records)
+
+
+def _step_calls(B, torch, w):
+    """The benchmark step's calls on device copies of workload w."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(
+            torch.bfloat16)
+
+    prob = B.Problem(num_tokens=w.N, hidden=w.H, num_experts=w.E, top_k=w.k,
+                     num_segments=w.S, recv_capacity=w.recv_capacity,
+                     expert_capacity=w.expert_capacity)
+    buf = B.Buffers(prob, device=dev)
+    ids = torch.from_numpy(w.ids).to(dev)
+    hidden, x = bf16(w.hidden), bf16(w.expert_out)
+    gates = torch.from_numpy(w.gates).to(dev)
+    gs = torch.tensor([w.global_scale], dtype=torch.float32, device=dev)
+    y = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
+    calls = [lambda: B.layout(prob, ids, buf),
+             lambda: B.moe_permute(prob, hidden, buf.row_src, buf.pair_slot, buf.out)]
+    if w.H % 128 == 0:
+        calls.append(lambda: B.moe_permute_quant_fp8(prob, hidden, buf.row_src, buf.pair_slot,
+                                                     buf.out_fp8, buf.scales_fp8))
+    if w.H % 32 == 0:
+        calls.append(lambda: B.moe_permute_quant_nvfp4(prob, hidden, buf.row_src,
+                                                       buf.pair_slot, gs, buf.out_fp4,
+                                                       buf.scales_fp4))
+    calls.append(lambda: B.moe_combine(prob, x, gates, buf.pair_slot, y))
+    return calls, (buf, ids, hidden, x, gates, gs, y)
+
+
+def main(argv=None) -> None:
+    from combine_topk_ids_scan_b200.inputs import CONFIG_NAMES, make_workload
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--workload", default="fp8_metric", choices=CONFIG_NAMES)
+    ap.add_argument("--steps", type=int, default=10)
+    a = ap.parse_args(argv)
+
+    import torch
+
+    from combine_topk_ids_scan_b200 import binding as B
+    from combine_topk_ids_scan_b200 import build
+    B.load(build.build(trace=True))
+    if "trace records" not in B.version():
+        raise SystemExit(f"not the trace build: {B.version()}")
+    w = make_workload(a.workload)
+    calls, _keep = _step_calls(B, torch, w)
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    scratch = torch.empty(2 * l2, dtype=torch.uint8, device="cuda")
+    for i in range(3):
+        for c in calls:
+            c()
+    per: dict[tuple, list] = {}
+    for i in range(a.steps):
+        scratch.fill_(i & 0xFF)
+        torch.cuda.synchronize()
+        with Tracer(capacity=1 << 18) as tr:
+            for c in calls:
+                c()
+        if tr.dropped:
+            raise SystemExit(f"{tr.dropped} records dropped")
+        prev_end = None
+        for j, launch in enumerate(tr.launches()):
+            # the kernel's own span: from the later of its first CTA's start
+            # and the previous kernel's end (a dependent launch starts its
+            # CTAs early, and they wait) to its last CTA's end
+            own = launch.end_ns - (launch.start_ns if prev_end is None
+                                   else max(launch.start_ns, prev_end))
+            per.setdefault((j, launch.kernel, launch.variant), []).append(
+                (own / 1e3, launch.duration_us, launch.ctas, launch.sms))
+            prev_end = launch.end_ns
+    print(f"workload {a.workload}: N={w.N} H={w.H} E={w.E} k={w.k}; {a.steps} steps, "
+          f"L2 flushed before each; medians")
+    print("| kernel | variant | CTAs | SMs | us after the previous kernel ended | "
+          "us first CTA start to last CTA end |")
+    print("|---|---|---|---|---|---|")
+    for (j, name, var), v in sorted(per.items()):
+        print(f"| {name} | {var} | {v[0][2]} | {v[0][3]} | "
+              f"{statistics.median(x[0] for x in v):.1f} | "
+              f"{statistics.median(x[1] for x in v):.1f} |")
+
+
+if __name__ == "__main__":
+    main()
