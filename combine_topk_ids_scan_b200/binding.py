@@ -310,7 +310,9 @@ def moe_permute_to_peers(prob: Problem, hidden_states, row_src, pair_slot, meta,
     """Dispatch permute whose segment s lands in rank s's receive buffer:
     peer_out is an int64 device tensor of S device addresses (e.g.
     [t.data_ptr() for t in receive buffers]), put_offsets an int64 device
-    tensor of S first rows (see moe_permute_to_peers in moe_dc.h)."""
+    tensor of S first rows (see moe_permute_to_peers in moe_dc.h).  The
+    library sees only the addresses: that every receive buffer holds its
+    rows is the caller's to guarantee."""
     N, H, E, k, S, P, rows = _sizes(prob)
     _require("moe_permute_to_peers", **_permute_need(prob, hidden_states, row_src, pair_slot),
              meta=(meta, 16 * S), peer_out=(peer_out, 8 * S), put_offsets=(put_offsets, 8 * S))
@@ -326,7 +328,8 @@ def moe_permute_quant_fp8_to_peers(prob: Problem, hidden_states, row_src, pair_s
     """FP8 dispatch whose segment s lands in rank s's receive buffers:
     peer_codes / peer_scales are int64 device tensors of S device addresses
     (E4M3 [rows, H] and fp32 [rows, H/128] buffers), put_offsets as in
-    moe_permute_to_peers (see moe_permute_quant_fp8_to_peers in moe_dc.h)."""
+    moe_permute_to_peers (see moe_permute_quant_fp8_to_peers in moe_dc.h);
+    the receive buffers' sizes are the caller's to guarantee."""
     N, H, E, k, S, P, rows = _sizes(prob)
     _require("moe_permute_quant_fp8_to_peers",
              **_permute_need(prob, hidden_states, row_src, pair_slot), meta=(meta, 16 * S),
@@ -344,7 +347,8 @@ def moe_permute_quant_nvfp4_to_peers(prob: Problem, hidden_states, row_src, pair
                                      stream=None) -> None:
     """NVFP4 dispatch whose segment s lands in rank s's receive buffers
     (E2M1 [rows, H/2] codes, E4M3 [rows, H/16] row-major scales); see
-    moe_permute_quant_nvfp4_to_peers in moe_dc.h."""
+    moe_permute_quant_nvfp4_to_peers in moe_dc.h; the receive buffers' sizes
+    are the caller's to guarantee."""
     N, H, E, k, S, P, rows = _sizes(prob)
     _require("moe_permute_quant_nvfp4_to_peers",
              **_permute_need(prob, hidden_states, row_src, pair_slot), meta=(meta, 16 * S),

@@ -564,8 +564,10 @@ typedef enum moe_trace_kernel {
  *   count     device uint32, zeroed by the caller; each CTA adds 1 and
  *             writes records[old value] if that is below `capacity`, so a
  *             count above capacity tells how many records were dropped
- * The attachment is a copy enqueued on `stream` (kernels enqueued on other
- * streams see it in no defined order) and lasts until the next call.  The
+ * The attachment is a host-to-device copy from pageable memory enqueued on
+ * `stream` (so not a call to make inside a CUDA graph capture; kernels
+ * enqueued on other streams see it in no defined order) and lasts until the
+ * next call; captured graphs of library calls record when replayed.  The
  * caller owns both buffers and keeps them alive while traced kernels run.
  * Returns MOE_ERR_NOT_BUILT, making no CUDA call, from a build without
  * -DMOE_TRACE; MOE_ERR_INVALID_ARG for records without count, misaligned
