@@ -709,6 +709,10 @@ __global__ void __launch_bounds__(kThreads)
   allow_dependents();
   extern __shared__ uint64_t table_smem[];
   grid_dependency_wait();
+  const PeerTable tab =
+      stage_peer_table(table_smem, meta, S, H, static_seg_rows,
+                       peer_codes, reinterpret_cast<uint8_t *const *>(peer_scales), put);
+  __syncthreads();
   constexpr int U = kChunk / 512;  // 2
   const int lane = threadIdx.x % kWarp;
   const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
@@ -716,29 +720,6 @@ __global__ void __launch_bounds__(kThreads)
   const int64_t pad_units = (rows + kWarp - 1) / kWarp * psplit;
   const int32_t vecs = H / 8;
   const int32_t nb = H / 128;
-  // a token unit issues its row loads and its pair loads first; the block
-  // then stages the per-rank table while they are in flight
-  const int64_t w = w0 - pad_units;
-  const bool token_unit = w0 >= pad_units && w < units;
-  const int64_t t = token_unit ? w / chunks : 0;
-  const int c0 = token_unit ? (int)(w % chunks) * kChunk : H;
-  uint4 a[U], b[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int col = c0 + u * 512 + lane * 16;
-    if (col < H) {
-      a[u] = ld_stream_v4(hidden + t * vecs + col / 8);
-      b[u] = ld_stream_v4(hidden + t * vecs + col / 8 + 1);
-    } else {
-      a[u] = b[u] = make_uint4(0, 0, 0, 0);
-    }
-  }
-  int32_t my_slot = -1;
-  uint32_t live = token_unit ? load_token_slots(pair_slot, t, k, rows, lane, my_slot) : 0u;
-  const PeerTable tab =
-      stage_peer_table(table_smem, meta, S, H, static_seg_rows,
-                       peer_codes, reinterpret_cast<uint8_t *const *>(peer_scales), put);
-  __syncthreads();
   if (w0 < pad_units) {
     const int64_t g = w0 / psplit;
     uint32_t m = padding_mask(g, lane, row_src, rows, rows);
@@ -759,8 +740,26 @@ __global__ void __launch_bounds__(kThreads)
     }
     return;
   }
-  if (!token_unit) return;
-  // this lane's pair: its receive rows (resolved before the quantisation)
+  const int64_t w = w0 - pad_units;
+  if (w >= units) return;
+  const int64_t t = w / chunks;
+  const int c0 = (int)(w % chunks) * kChunk;
+  const uint4 *src = hidden + t * vecs;
+  uint4 a[U], b[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int col = c0 + u * 512 + lane * 16;
+    if (col < H) {
+      a[u] = ld_stream_v4(src + col / 8);
+      b[u] = ld_stream_v4(src + col / 8 + 1);
+    } else {
+      a[u] = b[u] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  int32_t my_slot;
+  uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+  // this lane's pair: its receive rows (resolved before the quantisation, so
+  // the pointer loads overlap it)
   uint8_t *my_q = nullptr, *my_s = nullptr;
   const bool mine = my_slot >= 0 && peer_rows(my_slot, tab, S, H, 4 * nb, my_q, my_s);
   live &= __ballot_sync(kFull, mine);
@@ -801,28 +800,15 @@ __global__ void __launch_bounds__(kThreads, 4)
   allow_dependents();
   extern __shared__ uint64_t table_smem[];
   grid_dependency_wait();
+  const PeerTable tab =
+      stage_peer_table(table_smem, meta, S, H, static_seg_rows, peer_codes, peer_scales, put);
+  __syncthreads();
   const int lane = threadIdx.x % kWarp;
   const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
   const int64_t units = (int64_t)N * chunks;
   const int64_t pad_units = (rows + kWarp - 1) / kWarp * psplit;
   const int32_t vecs = H / 8;
   const int32_t qrow = H / 2, srow = H / 16;
-  // a token unit issues its row loads and its pair loads first; the block
-  // then stages the per-rank table while they are in flight
-  const int64_t w = w0 - pad_units;
-  const bool token_unit = w0 >= pad_units && w < units;
-  const int64_t t = token_unit ? w / chunks : 0;
-  const int col = token_unit ? (int)(w % chunks) * kChunk + lane * 32 : H;
-  const bool active = col < H;
-  uint4 x[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    x[i] = active ? ld_stream_v4(hidden + t * vecs + col / 8 + i) : make_uint4(0, 0, 0, 0);
-  int32_t my_slot = -1;
-  uint32_t live = token_unit ? load_token_slots(pair_slot, t, k, rows, lane, my_slot) : 0u;
-  const PeerTable tab =
-      stage_peer_table(table_smem, meta, S, H, static_seg_rows, peer_codes, peer_scales, put);
-  __syncthreads();
   if (w0 < pad_units) {
     const int64_t g = w0 / psplit;
     uint32_t m = padding_mask(g, lane, row_src, rows, rows);
@@ -843,8 +829,20 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
     return;
   }
-  if (!token_unit) return;
-  // this lane's pair: its receive rows (resolved before the quantisation)
+  const int64_t w = w0 - pad_units;
+  if (w >= units) return;
+  const int64_t t = w / chunks;
+  const int col = (int)(w % chunks) * kChunk + lane * 32;
+  const bool active = col < H;
+  const uint4 *src = hidden + t * vecs;
+  uint4 x[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    x[i] = active ? ld_stream_v4(src + col / 8 + i) : make_uint4(0, 0, 0, 0);
+  int32_t my_slot;
+  uint32_t live = load_token_slots(pair_slot, t, k, rows, lane, my_slot);
+  // this lane's pair: its receive rows (resolved before the quantisation, so
+  // the pointer loads overlap it)
   uint8_t *my_q = nullptr, *my_s = nullptr;
   const bool mine = my_slot >= 0 && peer_rows(my_slot, tab, S, qrow, srow, my_q, my_s);
   live &= __ballot_sync(kFull, mine);
