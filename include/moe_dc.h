@@ -265,7 +265,9 @@ MOE_API moe_status moe_permute(const moe_problem *problem, const void *hidden_st
  * + meta[0][s]/H) (expert blocks with their padding); capacity mode, rows
  * [s*L*Ce, (s+1)*L*Ce).  Row r of segment s is written, as moe_permute would
  * write it (padding rows as zeros), to row put_offsets[s] + r of the bf16
- * [*, H] buffer peer_out[s]; rows past the last segment are not written.
+ * [*, H] buffer peer_out[s]; rows past the last segment are not written, nor
+ * are segment rows at or past `rows` (a padded layout whose recv_capacity
+ * cuts the last expert block short: meta still counts the whole block).
  *   hidden_states  bf16 [N, H], 16-byte aligned
  *   row_src, pair_slot, meta   from moe_dispatch_layout (meta may be NULL in
  *                  capacity mode)

@@ -488,7 +488,74 @@ def _random_spec(i):
     return spec, pad, bool(rng.random() < 0.5), bool(rng.random() < 0.4)
 
 
-@pytest.mark.parametrize("i", range(16))
+def _check_peer_sends(orc, w, run, ref, rng):
+    """The bf16, FP8 (H % 128 == 0) and NVFP4 dispatches sent to S stand-in
+    receive buffers at random put offsets: each segment of the oracle's
+    dispatch output lands at its offset bit for bit, every other row of every
+    buffer keeps its poison."""
+    from gpu_util import BF16_POISON, BYTE_POISON, F32_POISON
+    H, S = w.H, w.S
+    L = w.E // S
+    if w.expert_capacity > 0:
+        starts = [s * L * w.expert_capacity for s in range(S)]
+        seg_rows = [L * w.expert_capacity] * S
+    else:
+        starts = [int(v) // H for v in ref.meta[1]]
+        seg_rows = [int(v) // H for v in ref.meta[0]]
+    put = [int(v) for v in rng.integers(0, 40, S)]
+    hid = to_dev_bf16(w.hidden) if w.N > 0 else torch.empty((1, H), dtype=torch.bfloat16,
+                                                             device="cuda")
+    put_d = torch.tensor(put, dtype=torch.int64, device="cuda")
+    gs = torch.tensor([w.global_scale], dtype=torch.float32, device="cuda")
+
+    def bufs(width, dtype):
+        return [poisoned_empty((put[s] + seg_rows[s] + 3, width), dtype) for s in range(S)]
+
+    def ptrs(ts):
+        return torch.tensor([t.data_ptr() for t in ts], dtype=torch.int64, device="cuda")
+
+    cases = [("bf16", (H, torch.bfloat16), None)]
+    if H % 128 == 0:
+        cases.append(("fp8", (H, torch.uint8), (H // 128, torch.float32)))
+    cases.append(("nvfp4", (H // 2, torch.uint8), (H // 16, torch.uint8)))
+    for fmt, code_spec, scale_spec in cases:
+        codes = bufs(*code_spec)
+        scales = bufs(*scale_spec) if scale_spec else None
+        if fmt == "bf16":
+            B.moe_permute_to_peers(run.prob, hid, run.buf.row_src, run.buf.pair_slot,
+                                   run.buf.meta, ptrs(codes), put_d)
+            want = [orc.permute_bf16(w.hidden, ref.row_src)]
+        elif fmt == "fp8":
+            B.moe_permute_quant_fp8_to_peers(run.prob, hid, run.buf.row_src, run.buf.pair_slot,
+                                             run.buf.meta, ptrs(codes), ptrs(scales), put_d)
+            q, sc = orc.permute_fp8(w.hidden, ref.row_src)
+            want = [q, sc.view(np.uint32)]
+        else:
+            B.moe_permute_quant_nvfp4_to_peers(run.prob, hid, run.buf.row_src,
+                                               run.buf.pair_slot, run.buf.meta, gs,
+                                               ptrs(codes), ptrs(scales), put_d)
+            want = list(orc.permute_nvfp4(w.hidden, ref.row_src, w.global_scale))
+        torch.cuda.synchronize()
+        R = ref.row_src.size
+        for s in range(S):
+            # a padded layout whose recv_capacity cuts the last expert block
+            # short has segment rows past the last local row: those are not
+            # written (moe_dc.h), and keep their poison
+            n = max(0, min(starts[s] + seg_rows[s], R) - starts[s])
+            lo, hi = put[s], put[s] + n
+            got = [codes[s].view(torch.int16).cpu().numpy().view(np.uint16) if fmt == "bf16"
+                   else codes[s].cpu().numpy()]
+            poison_of = [BF16_POISON if fmt == "bf16" else BYTE_POISON]
+            if scales is not None:
+                sv = scales[s].cpu().numpy()
+                got.append(sv.view(np.uint32) if fmt == "fp8" else sv)
+                poison_of.append(np.uint32(F32_POISON) if fmt == "fp8" else BYTE_POISON)
+            for g, wnt, p in zip(got, want, poison_of):
+                assert np.array_equal(g[lo:hi], wnt[starts[s]:starts[s] + n]), (fmt, s)
+                assert np.all(g[:lo] == p) and np.all(g[hi:] == p), (fmt, s)
+
+
+@pytest.mark.parametrize("i", range(40))
 def test_random_problem_sweep(orc, i):
     spec, pad, two_pass, swizzled = _random_spec(i)
     w = custom(seed=100 + i, **spec)
@@ -523,6 +590,9 @@ def test_random_problem_sweep(orc, i):
         assert np.array_equal(scales.cpu().numpy(), want_s), (fmt, inter)
     if w.N > 0:
         assert np.array_equal(bf16_np(gh), orc.permute_backward(g_rows, ref.pair_slot))
+    # the sends to peers (not in overflow: a segment would then run past rows)
+    if not (ref.status & orc.STATUS_CAPACITY) and not swizzled:
+        _check_peer_sends(orc, w, run, ref, rng)
 
 
 # ------------------------------------------------------------ scale atom layout
