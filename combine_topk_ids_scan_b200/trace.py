@@ -45,11 +45,14 @@ LAYOUT_KERNELS = frozenset(range(1, 6))
 
 @dataclass(frozen=True)
 class Launch:
-    """The CTAs of one kernel launch (one %gridid)."""
+    """The CTAs of one kernel launch: one %gridid, and the instance-th launch
+    with that id (replays of a captured CUDA graph reuse their kernel node's
+    id)."""
     kernel: str
     kernel_id: int
     variant: int
     grid: int
+    instance: int
     ctas: int
     sms: int          # distinct SMs its CTAs ran on
     start_ns: int     # earliest CTA start
@@ -75,19 +78,44 @@ def dropped(count: int, capacity: int) -> int:
     return max(0, int(count) - int(capacity))
 
 
+def instances(records: np.ndarray) -> np.ndarray:
+    """Launch instance of each record: how many earlier records (in slot
+    order, which is the order the CTAs started) have its %gridid and block.
+    A grid id recurs when a captured CUDA graph is replayed; the n-th replay's
+    CTAs all start after the (n-1)-th replay's have finished."""
+    n = records.size
+    slot = np.arange(n)
+    order = np.lexsort((slot, records["block"], records["grid"]))
+    g, b = records["grid"][order], records["block"][order]
+    new = np.ones(n, bool)
+    new[1:] = (g[1:] != g[:-1]) | (b[1:] != b[:-1])
+    first = np.maximum.accumulate(np.where(new, slot, 0))
+    inst = np.empty(n, np.int64)
+    inst[order] = slot - first
+    return inst
+
+
+def records_of(records: np.ndarray, launch: Launch) -> np.ndarray:
+    """The records of one launch."""
+    return records[(records["grid"] == launch.grid) & (instances(records) == launch.instance)]
+
+
 def launches(records: np.ndarray) -> list[Launch]:
     """Group records by launch, in the order the launches started."""
+    inst = instances(records)
     out = []
     for g in np.unique(records["grid"]):
-        r = records[records["grid"] == g]
-        kid = int(r["kernel"][0])
-        if np.any(r["kernel"] != kid) or np.any(r["variant"] != r["variant"][0]):
-            raise ValueError(f"launch {int(g)} mixes kernel ids or variants")
-        out.append(Launch(kernel=KERNELS.get(kid, f"kernel{kid}"), kernel_id=kid,
-                          variant=int(r["variant"][0]), grid=int(g), ctas=int(r.size),
-                          sms=int(np.unique(r["smid"]).size),
-                          start_ns=int(r["start_ns"].min()), end_ns=int(r["end_ns"].max())))
-    out.sort(key=lambda launch: (launch.start_ns, launch.grid))
+        for i in np.unique(inst[records["grid"] == g]):
+            r = records[(records["grid"] == g) & (inst == i)]
+            kid = int(r["kernel"][0])
+            if np.any(r["kernel"] != kid) or np.any(r["variant"] != r["variant"][0]):
+                raise ValueError(f"launch {int(g)}.{int(i)} mixes kernel ids or variants")
+            out.append(Launch(kernel=KERNELS.get(kid, f"kernel{kid}"), kernel_id=kid,
+                              variant=int(r["variant"][0]), grid=int(g), instance=int(i),
+                              ctas=int(r.size), sms=int(np.unique(r["smid"]).size),
+                              start_ns=int(r["start_ns"].min()),
+                              end_ns=int(r["end_ns"].max())))
+    out.sort(key=lambda launch: (launch.start_ns, launch.grid, launch.instance))
     return out
 
 

@@ -528,7 +528,10 @@ typedef struct moe_trace_record {
   uint64_t start_ns; /* %globaltimer when the CTA started (for a kernel that
                         overlaps its predecessor, before it waits for it)   */
   uint64_t end_ns;   /* %globaltimer when the CTA's last warp finished      */
-  uint64_t grid;     /* %gridid: one value per launch, shared by its CTAs   */
+  uint64_t grid;     /* %gridid, shared by the CTAs of a launch (replays of
+                        a captured CUDA graph reuse their kernel node's
+                        value; a later replay's CTAs start after the
+                        earlier one's have finished)                        */
   uint32_t block;    /* blockIdx.x                                          */
   uint16_t smid;     /* the SM the CTA ran on                               */
   uint8_t kernel;    /* moe_trace_kernel                                    */

@@ -51,6 +51,18 @@ def test_launches_group_by_grid_in_start_order():
     assert b.duration_us == pytest.approx(0.47)
 
 
+def test_a_recurring_grid_id_splits_into_launch_instances():
+    # two replays of one captured graph node: the same grid id, blocks 0-1
+    # twice, the second replay's CTAs in later slots
+    recs = np.concatenate([_rec(10, 20, 5, 0, 0, 6), _rec(11, 21, 5, 1, 1, 6),
+                           _rec(30, 40, 5, 1, 2, 6), _rec(31, 42, 5, 0, 3, 6)])
+    assert T.instances(recs).tolist() == [0, 0, 1, 1]
+    a, b = T.launches(recs)
+    assert (a.instance, a.ctas, a.start_ns, a.end_ns) == (0, 2, 10, 21)
+    assert (b.instance, b.ctas, b.start_ns, b.end_ns) == (1, 2, 30, 42)
+    assert sorted(T.records_of(recs, b)["block"].tolist()) == [0, 1]
+
+
 def test_a_launch_mixing_kernel_ids_is_rejected():
     recs = np.concatenate([_rec(1, 2, 9, 0, 0, 6), _rec(1, 2, 9, 1, 0, 7)])
     with pytest.raises(ValueError):

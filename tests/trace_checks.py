@@ -22,12 +22,12 @@ def check_launches(tr: T.Tracer) -> list[T.Launch]:
     assert set(np.unique(recs["kernel"]).tolist()) <= set(T.KERNELS)
     ls = T.launches(recs)
     for launch in ls:
-        blocks = np.sort(recs["block"][recs["grid"] == launch.grid])
+        blocks = np.sort(T.records_of(recs, launch)["block"])
         assert np.array_equal(blocks, np.arange(launch.ctas)), launch
     ordered = sorted(ls, key=lambda x: (x.start_ns, x.end_ns))
     for a, b in zip(ordered, ordered[1:]):
-        ra = recs[recs["grid"] == a.grid]
-        rb = recs[recs["grid"] == b.grid]
+        ra = T.records_of(recs, a)
+        rb = T.records_of(recs, b)
         assert int(rb["start_ns"].min()) >= int(ra["start_ns"].max()), (a, b)
         assert int(rb["end_ns"].min()) >= int(ra["end_ns"].max()), (a, b)
     return ordered

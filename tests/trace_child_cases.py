@@ -102,6 +102,28 @@ def test_detach_stops_recording():
     assert int(count.item()) == once
 
 
+def test_graph_replays_record():
+    """Kernels captured into a CUDA graph record on every replay (the
+    attachment is read by the kernels when they run)."""
+    w = make_workload("tiny", with_expert_out=False)
+    run = GpuRun(w, quant=False, combine=False)
+    hidden = to_dev_bf16(w.hidden)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        B.moe_permute(run.prob, hidden, run.buf.row_src, run.buf.pair_slot, run.buf.out)
+    with T.Tracer() as tr:
+        _permute_once(run, w)
+    (one,) = check_launches(tr)
+    with T.Tracer() as tr:
+        graph.replay()
+        graph.replay()
+    ls = check_launches(tr)
+    assert [launch.kernel for launch in ls] == ["permute_bf16", "permute_bf16"]
+    assert all(launch.ctas == one.ctas for launch in ls)
+
+
 def test_attach_argument_errors():
     raw = torch.zeros(4096, dtype=torch.uint8, device="cuda")
     count = torch.zeros(1, dtype=torch.int32, device="cuda")
