@@ -165,6 +165,7 @@ EDGE = {
     "k16": dict(N=1300, H=256, E=64, k=16, S=16),
     "E1": dict(N=999, H=64, E=1, k=1, S=1),
     "E2048_S2048": dict(N=2048, H=32, E=2048, k=8, S=2048),
+    "H65536": dict(N=40, H=65536, E=8, k=2, S=2, p_mask=0.1),
     "duplicates": dict(N=1000, H=128, E=6, k=4, S=3, distinct=False),
     "capacity_drops": dict(N=900, H=256, E=32, k=4, S=8, Ce=3),
     "capacity_masked": dict(N=333, H=160, E=12, k=3, S=4, Ce=40, p_mask=0.2, p_bad=0.01),
