@@ -13,6 +13,9 @@ against the concatenation over source ranks of the oracle's dispatch
 segments for it, and that no row past them was touched.  The kernels never
 wait on another process (completion is the host barrier), so the two ranks
 sharing one GPU cannot deadlock; across GPUs the same stores go over NVLink.
+
+A last case runs the ep module's host-level route on the NCCL backend with
+CUDA tensors, with one rank (NCCL takes one rank per GPU).
 """
 import datetime
 import os
@@ -169,3 +172,61 @@ def test_fused_send_between_two_processes(orc, mode):
     for p in procs:
         p.join(timeout=120)
     assert all(v == "ok" for v in res.values()), res
+
+
+def _nccl_single(port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    try:
+        torch.cuda.set_device(0)
+        dist.init_process_group("nccl", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120))
+        import oracle as orc
+        from combine_topk_ids_scan_b200 import binding as B
+        from combine_topk_ids_scan_b200 import ep
+        B.load()
+        p = _rank_problem(0, "packed")
+        N, H, E, k = p["N"], p["H"], p["E"], p["k"]
+        prob = B.Problem(num_tokens=N, hidden=H, num_experts=E, top_k=k, num_segments=1,
+                         recv_capacity=p["C"])
+        buf = B.Buffers(prob, quant=False)
+        hid = torch.from_numpy(p["hidden"].view(np.int16)).cuda().view(torch.bfloat16)
+        B.layout(prob, torch.from_numpy(p["ids"]).cuda(), buf)
+        B.moe_permute(prob, hid, buf.row_src, buf.pair_slot, buf.out)
+        # the counts all-to-all and the payload route on NCCL, CUDA tensors
+        route = ep.exchange_counts(buf.meta, H, E)
+        recv = ep.dispatch_exchange(buf.out, route)
+        gates = torch.from_numpy(
+            np.full((N, k), 1.0 / k, np.float32)).cuda()
+        back = ep.combine_exchange(recv, route, out=torch.zeros_like(buf.out))
+        y = torch.empty((N, H), dtype=torch.bfloat16, device="cuda")
+        B.moe_combine(prob, back, gates, buf.pair_slot, y)
+        torch.cuda.synchronize()
+        lay = orc.layout(p["ids"], E, 1, H, recv_capacity=p["C"])
+        out = orc.permute_bf16(p["hidden"], lay.row_src)
+        assert np.array_equal(recv.view(torch.int16).cpu().numpy().view(np.uint16),
+                              out[:route.recv_total])
+        assert np.array_equal(buf.meta.cpu().numpy()[2:], buf.meta.cpu().numpy()[:2])
+        want = orc.combine(out, np.full((N, k), 1.0 / k, np.float32), lay.pair_slot)
+        assert np.array_equal(y.view(torch.int16).cpu().numpy().view(np.uint16), want)
+        q.put("ok")
+    except Exception as e:  # report to the parent instead of hanging it
+        q.put(repr(e))
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def test_ep_module_on_nccl_with_one_rank(orc):
+    """The ep module's collectives on the NCCL backend with CUDA tensors (one
+    rank: the counts all-to-all is a self exchange, the payload route a
+    local copy): a dispatch, its exchange there and back, and the combine
+    of the returned rows match the oracle."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    proc = ctx.Process(target=_nccl_single, args=(_free_port(), q))
+    proc.start()
+    res = q.get(timeout=300)
+    proc.join(timeout=120)
+    assert res == "ok", res
