@@ -383,9 +383,9 @@ def measure_workload(B, torch, w, dev, stream, flush_l2, n_steps: int, peak: flo
 
 
 def layout_launches(P: int) -> int:
-    """Kernel launches of one moe_dispatch_layout call: one up to 128 scan
-    tiles of 4096 pairs (cooperative one-launch kernel), else a scan and an
-    emit launch."""
+    """Kernel launches of one moe_dispatch_layout call: one up to 128 tiles
+    of 4096 pairs (the one-CTA, cluster or cooperative look-back kernel),
+    else a scan and an emit launch."""
     return 1 if (P + 4095) // 4096 <= 128 else 2
 
 
