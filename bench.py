@@ -625,6 +625,13 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
              lambda: B.moe_permute_quant_nvfp4_to_peers(prob, d_hidden, buf.row_src,
                                                         buf.pair_slot, buf.meta, d_gs, c4, s4,
                                                         put)], f2_steps)
+        # the return: every rank's combine reads the expert outputs straight
+        # from the owners' buffers (here the bf16 receive buffers the send
+        # just filled: identity experts)
+        (cp_us,) = time_phases([lambda: B.moe_combine_from_peers(
+            prob, peer, put, buf.meta, d_gates, buf.pair_slot, d_y)], f2_steps)
+        cp_bytes = (2 * int(buf.expert_counts.sum().item()) * w.H + 8 * w.P
+                    + 2 * w.N * w.H)       # the combine's algorithmic bytes
         maps = 2 * w.N * w.H + 4 * w.P + 4 * buf.rows + 16 * w.S
         routed = sum(seg_rows)
         pp_bytes = maps + 2 * routed * w.H
@@ -637,6 +644,8 @@ def run_ours(args, rank: int, world: int, local: int) -> int:
               "permute_fp8_to_peers_gbs": round(p8_bytes / (p8_us * 1e-6) / 1e9, 1),
               "permute_nvfp4_to_peers_us": round(p4_us, 2),
               "permute_nvfp4_to_peers_gbs": round(p4_bytes / (p4_us * 1e-6) / 1e9, 1),
+              "combine_from_peers_us": round(cp_us, 2),
+              "combine_from_peers_gbs": round(cp_bytes / (cp_us * 1e-6) / 1e9, 1),
               "receivers": "S local buffers standing in for the peers' receive buffers "
                            "(one GPU); across GPUs the same stores go over NVLink"}
         del recv, peer, put, r8, r4, c8, s8, c4, s4

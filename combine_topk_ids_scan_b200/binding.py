@@ -53,7 +53,7 @@ MOE_MAX_TOPK = 16
 EXPORTED = ("moe_output_rows", "moe_workspace_bytes", "moe_dispatch_layout",
             "moe_dispatch_layout_noalloc", "moe_permute", "moe_permute_premultiplied",
             "moe_permute_to_peers", "moe_permute_quant_fp8_to_peers",
-            "moe_permute_quant_nvfp4_to_peers",
+            "moe_permute_quant_nvfp4_to_peers", "moe_combine_from_peers",
             "moe_permute_quant_fp8",
             "moe_permute_quant_nvfp4", "moe_permute_quant_mxfp4", "moe_combine",
             "moe_permute_backward",
@@ -140,6 +140,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     L.moe_permute_quant_fp8_to_peers.argtypes = [P] + [vp] * 8
     L.moe_permute_quant_nvfp4_to_peers.restype = ctypes.c_int
     L.moe_permute_quant_nvfp4_to_peers.argtypes = [P] + [vp] * 9
+    L.moe_combine_from_peers.restype = ctypes.c_int
+    L.moe_combine_from_peers.argtypes = [P] + [vp] * 7
     L.moe_permute_premultiplied.restype = ctypes.c_int
     L.moe_permute_premultiplied.argtypes = [P] + [vp] * 6
     L.moe_permute_quant_fp8.restype = ctypes.c_int
@@ -432,6 +434,24 @@ def nvfp4_swizzled_scale_bytes(rows: int, hidden: int, block: int = 16) -> int:
     """Bytes of FP4 block scales (block 16: NVFP4, 32: MXFP4) in the 128x4
     atom layout (see moe_dc.h)."""
     return max(1, -(-rows // 128) * 128 * (-(-(hidden // block) // 4) * 4))
+
+
+def moe_combine_from_peers(prob: Problem, peer_expert_out, get_offsets, meta, gates, pair_slot,
+                           out, stream=None) -> None:
+    """Combine reading each expert output from the rank that computed it:
+    peer_expert_out is an int64 device tensor of S device addresses (bf16
+    [*, H] expert-output buffers), get_offsets an int64 device tensor of S
+    first rows (see moe_combine_from_peers in moe_dc.h); the buffers' sizes
+    are the caller's to guarantee."""
+    N, H, E, k, S, P, rows = _sizes(prob)
+    _require("moe_combine_from_peers", peer_expert_out=(peer_expert_out, 8 * S),
+             get_offsets=(get_offsets, 8 * S), meta=(meta, 16 * S), gates=(gates, 4 * P),
+             pair_slot=(pair_slot, 4 * P), out=(out, 2 * N * H))
+    c = prob.c()
+    _check(load().moe_combine_from_peers(ctypes.byref(c), _ptr(peer_expert_out),
+                                         _ptr(get_offsets), _ptr(meta), _ptr(gates),
+                                         _ptr(pair_slot), _ptr(out), _stream(stream)),
+           "moe_combine_from_peers")
 
 
 def moe_permute_backward(prob: Problem, grad_out, pair_slot, grad_hidden, stream=None) -> None:

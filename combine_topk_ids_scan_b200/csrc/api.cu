@@ -294,6 +294,25 @@ moe_status moe_combine(const moe_problem *problem, const void *expert_out, const
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_combine_from_peers(const moe_problem *problem, const void *const *peer_expert_out,
+                                  const int64_t *get_offsets, const uint32_t *meta,
+                                  const float *gates, const int32_t *pair_slot, void *out,
+                                  moe_stream_t stream) {
+  moe::Shape s;
+  moe_status st = make_shape(problem, &s);
+  if (st != MOE_OK) return st;
+  if (s.H % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s.N == 0) return MOE_OK;
+  if (!out || !gates || !pair_slot || !peer_expert_out || !get_offsets || (s.Ce == 0 && !meta))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(peer_expert_out, 8) || !aligned(get_offsets, 8) || !aligned(meta, 4) ||
+      !aligned(gates, 4) || !aligned(pair_slot, 4) || !aligned(out, 16))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_combine_from_peers(s, peer_expert_out, get_offsets, meta, gates,
+                                                  pair_slot, out,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_permute_backward(const moe_problem *problem, const void *grad_out,
                                 const int32_t *pair_slot, void *grad_hidden,
                                 moe_stream_t stream) {

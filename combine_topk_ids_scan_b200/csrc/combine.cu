@@ -99,6 +99,111 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// Combine fused with the expert-parallel return (the reverse of the fused
+// send): the expert output of local row r of segment s is read straight from
+// rank s's expert-output buffer peer_x[s] at row get[s] + (r - start_s) --
+// where that rank received the row -- instead of being shipped back first.
+// combine_kernel's units, loads and fp32 fma order, so the result is the
+// one moe_combine gives on the returned rows.  Each CTA stages the S segment
+// starts and sizes, get offsets and buffer addresses in shared memory (24
+// bytes per rank); a lane holding pair j resolves its row's source address
+// and the warp broadcasts the k addresses.
+template <int KMAX, int U>
+__global__ void __launch_bounds__(kThreads)
+    combine_from_peers_kernel(const uint4 *const *__restrict__ peer_x,
+                              const int64_t *__restrict__ get, const uint32_t *__restrict__ meta,
+                              const float *__restrict__ gates,
+                              const int32_t *__restrict__ pair_slot, uint4 *__restrict__ out,
+                              int32_t N, int32_t k, int64_t rows, int32_t vecs, int32_t splits,
+                              int32_t span, int32_t S, int32_t H, int32_t static_seg_rows) {
+  MOE_TRACE_CTA(MOE_TRACE_COMBINE_FROM_PEERS, KMAX);
+  allow_dependents();
+  extern __shared__ uint64_t peer_smem[];
+  const uint4 **s_ptr = reinterpret_cast<const uint4 **>(peer_smem);
+  int64_t *s_get = reinterpret_cast<int64_t *>(peer_smem + S);
+  int32_t *s_start = reinterpret_cast<int32_t *>(peer_smem + 2 * S);
+  int32_t *s_rows = s_start + S;
+  grid_dependency_wait();
+  for (int i = threadIdx.x; i < S; i += kThreads) {
+    s_ptr[i] = peer_x[i];
+    s_get[i] = __ldg(get + i);
+    if (static_seg_rows > 0) {
+      s_start[i] = i * static_seg_rows;
+      s_rows[i] = static_seg_rows;
+    } else {
+      s_start[i] = (int32_t)(__ldg(meta + S + i) / (uint32_t)H);
+      s_rows[i] = (int32_t)(__ldg(meta + i) / (uint32_t)H);
+    }
+  }
+  __syncthreads();
+  const int lane = threadIdx.x % kWarp;
+  const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / kWarp;
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) / kWarp;
+
+  for (int64_t item = gw; item < (int64_t)N * splits; item += nw) {
+    const int64_t t = item / splits;
+    const int32_t vb = (int32_t)(item % splits) * span;
+    const int32_t ve = min(vecs, vb + span);
+    const uint4 *my_src = nullptr;
+    float my_w = 0.0f;
+    if (lane < k) {
+      const int32_t r = __ldg(pair_slot + t * k + lane);
+      if (r >= 0 && r < rows && MOE_IN_RANGE(r, rows, kDbgCombineRow)) {
+        int lo = 0, hi = S - 1;  // last segment starting at or before r
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) / 2;
+          if (s_start[mid] <= r) lo = mid;
+          else hi = mid - 1;
+        }
+        if (r >= s_start[lo] && r - s_start[lo] < s_rows[lo]) {
+          my_src = s_ptr[lo] + (s_get[lo] + (r - s_start[lo])) * (int64_t)vecs;
+          my_w = __ldg(gates + t * k + lane);
+        }
+      }
+    }
+    const uint4 *src[KMAX];
+    float w[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      src[j] = reinterpret_cast<const uint4 *>(
+          __shfl_sync(kFull, reinterpret_cast<unsigned long long>(my_src), j));
+      w[j] = __shfl_sync(kFull, my_w, j);
+    }
+    uint4 *dst = out + t * vecs;
+    for (int v0 = vb; v0 < ve; v0 += kWarp * U) {
+      uint4 in[KMAX][U];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * kWarp + lane;
+          in[j][u] = (src[j] != nullptr && v < ve) ? ld_stream_v4(src[j] + v)
+                                                   : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int v = v0 + u * kWarp + lane;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          if (src[j] == nullptr) continue;
+          const uint32_t e[4] = {in[j][u].x, in[j][u].y, in[j][u].z, in[j][u].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] = fmaf(w[j], bf16lo(e[i]), acc[2 * i]);
+            acc[2 * i + 1] = fmaf(w[j], bf16hi(e[i]), acc[2 * i + 1]);
+          }
+        }
+        if (v < ve)
+          st_v4(dst + v, make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                    pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7])));
+      }
+    }
+  }
+}
+
 // Combine backward.  y[t] = sum_j w[t,j] x[slot(t,j)], so the expert rows get
 // grad_x[slot(t,j)] = bf16(w[t,j] * grad_y[t]) and the gates get
 // grad_w[t,j] = <grad_y[t], x[slot(t,j)]>.  One warp per token: per step a
@@ -214,8 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Grid of a persistent kernel: resident CTAs per SM x SMs, or fewer when
 // there is less work.
 template <typename Kernel>
-int grid_for(Kernel kernel, int64_t N, OccupancyCache &cache) {
-  const int per_sm = resident_ctas(cache, reinterpret_cast<const void *>(kernel), kThreads, 0);
+int grid_for(Kernel kernel, int64_t N, OccupancyCache &cache, size_t smem = 0) {
+  const int per_sm = resident_ctas(cache, reinterpret_cast<const void *>(kernel), kThreads, smem);
   const int64_t need = std::max<int64_t>(1, (N + kThreads / kWarp - 1) / (kThreads / kWarp));
   return (int)std::min<int64_t>(need, (int64_t)per_sm * device_sm_count());
 }
@@ -228,6 +333,36 @@ cudaError_t launch_backward(const Shape &s, const uint4 *gy, const uint4 *x, con
   auto kernel = combine_backward_kernel<KMAX>;
   return launch_pdl(kernel, dim3(grid_for(kernel, work, cache)), dim3(kThreads), 0, stream, gy, x,
                     gates, pair_slot, row_src, gx, grad_gates, s.N, s.k, s.rows, s.H / 8);
+}
+
+template <int KMAX, int U>
+cudaError_t launch_from_peers(const Shape &s, const uint4 *const *peer_x, const int64_t *get,
+                              const uint32_t *meta, const float *gates,
+                              const int32_t *pair_slot, uint4 *o, cudaStream_t stream) {
+  static OccupancyCache cache;
+  auto kernel = combine_from_peers_kernel<KMAX, U>;
+  const size_t smem = (size_t)24 * s.S;
+  if (smem > 48 * 1024) {
+    const cudaError_t err =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+  }
+  // column spans per token as in launch_forward
+  const int32_t vecs = s.H / 8;
+  const int32_t step = kWarp * U;
+  const int32_t steps = (vecs + step - 1) / step;
+  const int64_t resident = (int64_t)resident_ctas(cache, reinterpret_cast<const void *>(kernel),
+                                                  kThreads, smem) *
+                           device_sm_count() * (kThreads / kWarp);
+  int32_t splits = 1;
+  if ((int64_t)s.N * 2 < resident)
+    splits = (int32_t)std::min<int64_t>(steps, (resident + s.N - 1) / s.N);
+  const int32_t span = (steps + splits - 1) / splits * step;
+  splits = (vecs + span - 1) / span;
+  const int32_t static_seg = s.Ce > 0 ? (s.E / s.S) * s.Ce : 0;
+  return launch_pdl(kernel, dim3(grid_for(kernel, (int64_t)s.N * splits, cache, smem)),
+                    dim3(kThreads), smem, stream, peer_x, get, meta, gates, pair_slot, o, s.N,
+                    s.k, s.rows, vecs, splits, span, s.S, s.H, static_seg);
 }
 
 template <int KMAX, int U>
@@ -277,6 +412,19 @@ cudaError_t launch_combine_backward(const Shape &s, const void *grad_y, const vo
   if (s.k <= 8)
     return launch_backward<8>(s, gy, x, gates, pair_slot, row_src, gx, grad_gates, work, stream);
   return launch_backward<16>(s, gy, x, gates, pair_slot, row_src, gx, grad_gates, work, stream);
+}
+
+cudaError_t launch_combine_from_peers(const Shape &s, const void *const *peer_expert_out,
+                                      const int64_t *get_offsets, const uint32_t *meta,
+                                      const float *gates, const int32_t *pair_slot, void *out,
+                                      cudaStream_t stream) {
+  if (s.N == 0) return cudaSuccess;
+  const uint4 *const *px = reinterpret_cast<const uint4 *const *>(peer_expert_out);
+  uint4 *o = static_cast<uint4 *>(out);
+  if (s.k <= 2) return launch_from_peers<2, 4>(s, px, get_offsets, meta, gates, pair_slot, o, stream);
+  if (s.k <= 4) return launch_from_peers<4, 2>(s, px, get_offsets, meta, gates, pair_slot, o, stream);
+  if (s.k <= 8) return launch_from_peers<8, 2>(s, px, get_offsets, meta, gates, pair_slot, o, stream);
+  return launch_from_peers<16, 1>(s, px, get_offsets, meta, gates, pair_slot, o, stream);
 }
 
 cudaError_t launch_combine(const Shape &s, const void *expert_out, const float *gates,

@@ -80,6 +80,10 @@ cudaError_t launch_permute_mxfp4(const Shape &s, const void *hidden, const int32
                                  cudaStream_t stream);
 
 // gates == nullptr: unit weights (the dispatch backward)
+cudaError_t launch_combine_from_peers(const Shape &s, const void *const *peer_expert_out,
+                                      const int64_t *get_offsets, const uint32_t *meta,
+                                      const float *gates, const int32_t *pair_slot, void *out,
+                                      cudaStream_t stream);
 cudaError_t launch_combine(const Shape &s, const void *expert_out, const float *gates,
                            const int32_t *pair_slot, void *out, cudaStream_t stream);
 

@@ -38,7 +38,7 @@ KERNELS = {
     9: "permute_mxfp4", 10: "scales_to_atoms", 11: "permute_premultiplied",
     12: "permute_to_peers", 13: "combine", 14: "permute_backward", 15: "combine_backward",
     16: "swiglu_split", 17: "swiglu_quant", 18: "permute_fp8_to_peers",
-    19: "permute_nvfp4_to_peers",
+    19: "permute_nvfp4_to_peers", 20: "combine_from_peers",
 }
 LAYOUT_KERNELS = frozenset(range(1, 6))
 

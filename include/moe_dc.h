@@ -413,6 +413,31 @@ MOE_API moe_status moe_combine(const moe_problem *problem, const void *expert_ou
                        const float *gates, const int32_t *pair_slot, void *out,
                        moe_stream_t stream);
 
+/* The combine fused with the expert-parallel return: instead of shipping
+ * the expert outputs back to this rank first, the expert output of local row
+ * r of segment s is read straight from rank s's expert-output buffer
+ * peer_expert_out[s], at row get_offsets[s] + (r - start of segment s) --
+ * where rank s received row r through a fused send (moe_permute_to_peers
+ * with put_offsets = get_offsets) and wrote its expert's output.  Segments
+ * as in moe_permute_to_peers.  The result is the one moe_combine gives on the
+ * returned rows, bit for bit.  DeepSpeed combine docstring; Mojo MAX ep_comm
+ * (combine kernels reading the remote ranks' expert outputs).
+ *   peer_expert_out  DEVICE array of S device pointers (8-byte aligned
+ *                    array) to bf16 [*, H] buffers, each 16-byte aligned
+ *                    and readable from this GPU (a peer mapping, or this
+ *                    rank's own buffer for its own segment)
+ *   get_offsets      DEVICE int64 [S]: first row of this rank's block in
+ *                    rank s's buffer (ep.put_offsets)
+ *   meta             from moe_dispatch_layout (may be NULL in capacity mode)
+ *   gates, pair_slot, out   as in moe_combine
+ * Requires H % 8 == 0.  The caller orders the read after the experts'
+ * writes (a barrier); the kernel does not wait on other GPUs. */
+MOE_API moe_status moe_combine_from_peers(const moe_problem *problem,
+                                          const void *const *peer_expert_out,
+                                          const int64_t *get_offsets, const uint32_t *meta,
+                                          const float *gates, const int32_t *pair_slot,
+                                          void *out, moe_stream_t stream);
+
 /* ---- fused SwiGLU + requantisation -----------------------------------------
  * The step after the experts' gate/up projection (Mojo MAX ep_comm:
  * fused_silu_kernel, fused_silu_mx_kernel, fused_silu_nvfp4_kernel,
@@ -560,7 +585,8 @@ typedef enum moe_trace_kernel {
   MOE_TRACE_SWIGLU_SPLIT = 16,         /* variant: the MOE_QUANT_* format          */
   MOE_TRACE_SWIGLU_QUANT = 17,         /* variant: the MOE_QUANT_* format          */
   MOE_TRACE_PERMUTE_FP8_TO_PEERS = 18,
-  MOE_TRACE_PERMUTE_NVFP4_TO_PEERS = 19
+  MOE_TRACE_PERMUTE_NVFP4_TO_PEERS = 19,
+  MOE_TRACE_COMBINE_FROM_PEERS = 20    /* variant as MOE_TRACE_COMBINE             */
 } moe_trace_kernel;
 
 /* Attach the trace record buffer (the build with -DMOE_TRACE): the kernels

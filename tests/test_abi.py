@@ -149,6 +149,7 @@ ALIGNMENT_RULES = {
     "moe_permute_quant_nvfp4": ((), (16, 4, 4, 4, 16, 2)),
     "moe_permute_quant_mxfp4": ((), (16, 4, 4, 16, 1)),
     "moe_combine": ((), (16, 4, 4, 16)),
+    "moe_combine_from_peers": ((), (8, 8, 4, 4, 4, 16)),
     "moe_permute_backward": ((), (16, 4, 16)),
     "moe_combine_backward": ((), (16, 16, 4, 4, 4, 16, 4)),
     "moe_swiglu_quant": ((128, 0, 0), (16, 4, 4, 16, 2)),   # I = 128, NVFP4, split

@@ -86,6 +86,8 @@ def cases():
         "moe_permute_quant_mxfp4[atoms]": (sw, [bf16(N, H), m(R), m(N, K), u8(R, H // 2),
                                                u8(B.nvfp4_swizzled_scale_bytes(R, H, 32))], ()),
         "moe_combine": (p, [bf16(R, H), f32(N, K), m(N, K), bf16(N, H)], ()),
+        "moe_combine_from_peers": (p, [m(S, dtype=torch.int64), m(S, dtype=torch.int64),
+                                       m(4, S), f32(N, K), m(N, K), bf16(N, H)], ()),
         "moe_permute_backward": (p, [bf16(R, H), m(N, K), bf16(N, H)], ()),
         "moe_combine_backward": (p, [bf16(N, H), bf16(R, H), f32(N, K), m(N, K), m(R),
                                      bf16(R, H), f32(N, K)], ()),

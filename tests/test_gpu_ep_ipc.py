@@ -8,9 +8,13 @@ exchanges counts (ep.exchange_counts) and put offsets (ep.put_offsets),
 then stores its segments straight into the owners' receive buffers with
 moe_permute_to_peers, moe_permute_quant_fp8_to_peers and
 moe_permute_quant_nvfp4_to_peers.  After a device synchronisation and a
-barrier each rank checks its own receive buffers, every row, code and scale,
-against the concatenation over source ranks of the oracle's dispatch
-segments for it, and that no row past them was touched.  The kernels never
+barrier, with identity experts (the received bf16 rows are the expert
+outputs), every rank combines with moe_combine_from_peers, reading its rows
+back from the owners' buffers, and checks the result against the oracle's
+combine of its own dispatch; each rank then checks its own receive buffers,
+every row, code and scale, against the concatenation over source ranks of
+the oracle's dispatch segments for it, and that no row past them was
+touched.  The kernels never
 wait on another process (completion is the host barrier), so the two ranks
 sharing one GPU cannot deadlock; across GPUs the same stores go over NVLink.
 
@@ -130,6 +134,16 @@ def _worker(rank, port, mode, q):
         B.moe_permute_quant_nvfp4_to_peers(prob, hid, buf.row_src, buf.pair_slot, buf.meta, gs,
                                            ptrs(3), ptrs(4), put)
         torch.cuda.synchronize()
+        dist.barrier()
+        # identity experts: each rank's received bf16 rows are its expert
+        # outputs; every rank combines reading its rows back from the owners
+        gates = np.random.default_rng(1300 + rank).random((p["N"], p["k"])).astype(np.float32)
+        y = torch.empty((p["N"], H), dtype=torch.bfloat16, device="cuda")
+        B.moe_combine_from_peers(prob, ptrs(0), put, buf.meta, torch.from_numpy(gates).cuda(),
+                                 buf.pair_slot, y)
+        torch.cuda.synchronize()
+        want_y = orc.combine(refs[rank][1], gates, refs[rank][0].pair_slot)
+        assert np.array_equal(y.view(torch.int16).cpu().numpy().view(np.uint16), want_y), mode
         dist.barrier()
         # every row this rank received, from every source, in source order
         total = route.recv_total

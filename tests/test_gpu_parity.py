@@ -911,6 +911,47 @@ def test_quantised_permute_to_peers(orc, mode, fmt):
         assert np.all(np.concatenate([got_s[:lo], got_s[hi:]]) == s_poison), s
 
 
+@pytest.mark.parametrize("mode", ["packed", "padded", "capacity"])
+def test_combine_from_peers(orc, mode):
+    """moe_combine_from_peers with S local buffers standing in for the S
+    ranks' expert-output buffers: segment s of the expert outputs sits at
+    rows [get[s], get[s] + rows_s) of buffer s (poison elsewhere); the result
+    equals the oracle's combine of the local expert outputs, bit for bit."""
+    spec = dict(N=1500, H=264, E=24, k=3, S=4, p_mask=0.05, p_bad=0.01)
+    pad = 0
+    if mode == "padded":
+        pad = 8
+        spec["C"] = 1500 * 3 + 24 * 7
+    elif mode == "capacity":
+        spec["Ce"] = 150
+    w = custom(seed=47, **spec)
+    run = GpuRun(w, quant=False, combine=False, pad=pad)
+    ref = oracle_layout(orc, w, pad=pad)
+    assert_layout(run, ref)
+    L = w.E // w.S
+    if mode == "capacity":
+        starts = [s * L * w.expert_capacity for s in range(w.S)]
+        seg_rows = [L * w.expert_capacity] * w.S
+    else:
+        starts = [int(v) // w.H for v in ref.meta[1]]
+        seg_rows = [int(v) // w.H for v in ref.meta[0]]
+    rng = np.random.default_rng(21)
+    get = [int(rng.integers(0, 300)) for _ in range(w.S)]
+    X = w.expert_out
+    bufs = []
+    for s in range(w.S):
+        b = np.full((get[s] + seg_rows[s] + 9, w.H), 0x7FC1, np.uint16)
+        b[get[s]:get[s] + seg_rows[s]] = X[starts[s]:starts[s] + seg_rows[s]]
+        bufs.append(to_dev_bf16(b))
+    peer = torch.tensor([t.data_ptr() for t in bufs], dtype=torch.int64, device="cuda")
+    get_d = torch.tensor(get, dtype=torch.int64, device="cuda")
+    y = poisoned_empty((w.N, w.H), torch.bfloat16)
+    B.moe_combine_from_peers(run.prob, peer, get_d, run.buf.meta,
+                             torch.from_numpy(w.gates).cuda(), run.buf.pair_slot, y)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_np(y), orc.combine(X, w.gates, ref.pair_slot))
+
+
 def test_quantised_permute_to_peers_rejects_the_atom_layout():
     w = custom(N=64, H=256, E=8, k=2, S=2, seed=3, with_out=False)
     prob = problem_of(w, flags=B.MOE_FLAG_NVFP4_SWIZZLED_SCALES)
