@@ -182,11 +182,14 @@ def test_next_row_kernels_record_with_their_variants():
                                          *q8, put)
         B.moe_permute_quant_nvfp4_to_peers(prob, hidden, buf.row_src, buf.pair_slot, buf.meta,
                                            gs, *q4, put)
+        B.moe_combine_from_peers(prob, peer, put, buf.meta, gates, buf.pair_slot,
+                                 poisoned_empty((w.N, H), torch.bfloat16))
     got = [(launch.kernel, launch.variant) for launch in check_launches(tr)]
     nvfp4 = [g for g in got if g[0] in ("permute_nvfp4", "scales_to_atoms")]
     assert got[:3] == [("permute_premultiplied", 0), ("permute_backward", 8),
                        ("combine_backward", 8)]
     assert nvfp4 in ([("permute_nvfp4", 0), ("scales_to_atoms", 1)], [("permute_nvfp4", 1)])
-    assert got[-5:] == [("swiglu_split", B.MOE_QUANT_MXFP8),
+    assert got[-6:] == [("swiglu_split", B.MOE_QUANT_MXFP8),
                         ("swiglu_quant", B.MOE_QUANT_MXFP6_E2M3), ("permute_to_peers", 0),
-                        ("permute_fp8_to_peers", 0), ("permute_nvfp4_to_peers", 0)]
+                        ("permute_fp8_to_peers", 0), ("permute_nvfp4_to_peers", 0),
+                        ("combine_from_peers", 8)]
