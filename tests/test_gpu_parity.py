@@ -493,7 +493,8 @@ def _check_peer_sends(orc, w, run, ref, rng):
     """The bf16, FP8 (H % 128 == 0) and NVFP4 dispatches sent to S stand-in
     receive buffers at random put offsets: each segment of the oracle's
     dispatch output lands at its offset bit for bit, every other row of every
-    buffer keeps its poison."""
+    buffer keeps its poison; the combine reading the bf16 rows back from the
+    buffers equals the oracle's combine of the dispatch output."""
     from gpu_util import BF16_POISON, BYTE_POISON, F32_POISON
     H, S = w.H, w.S
     L = w.E // S
@@ -526,6 +527,13 @@ def _check_peer_sends(orc, w, run, ref, rng):
             B.moe_permute_to_peers(run.prob, hid, run.buf.row_src, run.buf.pair_slot,
                                    run.buf.meta, ptrs(codes), put_d)
             want = [orc.permute_bf16(w.hidden, ref.row_src)]
+            if w.N > 0:
+                # and back: the combine reading the rows where they landed
+                y = poisoned_empty((w.N, H), torch.bfloat16)
+                B.moe_combine_from_peers(run.prob, ptrs(codes), put_d, run.buf.meta,
+                                         torch.from_numpy(w.gates).cuda(), run.buf.pair_slot, y)
+                torch.cuda.synchronize()
+                assert np.array_equal(bf16_np(y), orc.combine(want[0], w.gates, ref.pair_slot))
         elif fmt == "fp8":
             B.moe_permute_quant_fp8_to_peers(run.prob, hid, run.buf.row_src, run.buf.pair_slot,
                                              run.buf.meta, ptrs(codes), ptrs(scales), put_d)
