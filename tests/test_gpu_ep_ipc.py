@@ -1,5 +1,5 @@
-"""The dispatch fused with the expert-parallel send, run by two ranks: two
-processes on one GPU, a gloo group for the counts, offsets and barriers,
+"""The dispatch fused with the expert-parallel send, run by two and three
+ranks: as many processes on one GPU, a gloo group for the counts, offsets and barriers,
 each rank's receive buffers mapped into the other process with CUDA IPC
 (torch's CUDA tensor sharing).
 
@@ -33,9 +33,6 @@ import torch.multiprocessing as mp
 
 pytestmark = pytest.mark.gpu
 
-WORLD = 2
-
-
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
@@ -44,10 +41,10 @@ def _free_port():
     return port
 
 
-def _rank_problem(r, mode):
+def _rank_problem(r, mode, world=1):
     rng = np.random.default_rng(900 + r)
     N, H, L, k = 300 + 37 * r, 384, 4, 3
-    E = L * WORLD
+    E = L * world
     ids = np.argsort(rng.random((N, E)), axis=1)[:, :k].astype(np.int32)
     ids[rng.random((N, k)) < 0.05] = -1
     hidden = (rng.standard_normal((N, H)).astype(np.float32).view(np.uint32) >> 16).astype(
@@ -60,17 +57,17 @@ def _rank_problem(r, mode):
                 gs=float(np.float32(amax) / np.float32(2688.0)))
 
 
-def _segment_rows(lay, p, s):
-    L = p["E"] // WORLD
+def _segment_rows(lay, p, s, world):
+    L = p["E"] // world
     if p["Ce"]:
         return np.arange(s * L * p["Ce"], (s + 1) * L * p["Ce"])
     return np.arange(lay.expert_offsets[s * L], lay.expert_offsets[(s + 1) * L])
 
 
-def _worker(rank, port, mode, q):
+def _worker(rank, world, port, mode, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     # a short timeout: a rank that fails makes the other's next barrier fail
-    dist.init_process_group("gloo", rank=rank, world_size=WORLD,
+    dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=120))
     keep = []
     try:
@@ -81,10 +78,10 @@ def _worker(rank, port, mode, q):
         from combine_topk_ids_scan_b200 import ep
         torch.cuda.set_device(0)
         B.load()
-        probs = [_rank_problem(r, mode) for r in range(WORLD)]
+        probs = [_rank_problem(r, mode, world) for r in range(world)]
         refs = []
         for p in probs:
-            lay = orc.layout(p["ids"], p["E"], WORLD, p["H"], recv_capacity=p["C"],
+            lay = orc.layout(p["ids"], p["E"], world, p["H"], recv_capacity=p["C"],
                              expert_capacity=p["Ce"], expert_pad_multiple=p["pad"])
             q8, s8 = orc.permute_fp8(p["hidden"], lay.row_src)
             q4, s4 = orc.permute_nvfp4(p["hidden"], lay.row_src, p["gs"])
@@ -93,7 +90,7 @@ def _worker(rank, port, mode, q):
         p = probs[rank]
         H = p["H"]
         prob = B.Problem(num_tokens=p["N"], hidden=H, num_experts=p["E"], top_k=p["k"],
-                         num_segments=WORLD, recv_capacity=p["C"], expert_capacity=p["Ce"],
+                         num_segments=world, recv_capacity=p["C"], expert_capacity=p["Ce"],
                          expert_pad_multiple=p["pad"])
         buf = B.Buffers(prob, quant=False)
         hid = torch.from_numpy(p["hidden"].view(np.int16)).cuda().view(torch.bfloat16)
@@ -112,10 +109,10 @@ def _worker(rank, port, mode, q):
                 torch.full((n, H // 16), 0xA5, dtype=torch.uint8, device="cuda")]
         torch.cuda.synchronize()
         # share them: every rank maps every other rank's buffers
-        handles = [None] * WORLD
+        handles = [None] * world
         dist.all_gather_object(handles, [reduce_tensor(t) for t in mine])
         bufs = []
-        for r in range(WORLD):
+        for r in range(world):
             if r == rank:
                 bufs.append(mine)
             else:
@@ -124,7 +121,7 @@ def _worker(rank, port, mode, q):
                 bufs.append(mapped)
 
         def ptrs(i):
-            return torch.tensor([bufs[r][i].data_ptr() for r in range(WORLD)],
+            return torch.tensor([bufs[r][i].data_ptr() for r in range(world)],
                                 dtype=torch.int64, device="cuda")
 
         gs = torch.tensor([p["gs"]], dtype=torch.float32, device="cuda")
@@ -151,8 +148,8 @@ def _worker(rank, port, mode, q):
         got[0] = got[0].view(np.uint16)
         got[2] = got[2].view(np.uint32)
         for i, j in ((0, 1), (1, 2), (2, 3), (3, 4), (4, 5)):
-            want = np.concatenate([refs[s][j][_segment_rows(refs[s][0], probs[s], rank)]
-                                   for s in range(WORLD)])
+            want = np.concatenate([refs[s][j][_segment_rows(refs[s][0], probs[s], rank, world)]
+                                   for s in range(world)])
             assert want.shape[0] == total
             assert np.array_equal(got[i][:total], want), (mode, i)
         assert np.all(got[0][total:] == 0x7FC1) and np.all(got[1][total:] == 0xA5)
@@ -170,8 +167,9 @@ def _worker(rank, port, mode, q):
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("world", [2, 3])
 @pytest.mark.parametrize("mode", ["packed", "padded", "capacity"])
-def test_fused_send_between_two_processes(orc, mode):
+def test_fused_send_between_processes(orc, mode, world):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from combine_topk_ids_scan_b200 import build
@@ -179,7 +177,7 @@ def test_fused_send_between_two_processes(orc, mode):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, port, mode, q)) for r in range(WORLD)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, mode, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = dict(q.get(timeout=300) for _ in procs)
@@ -198,7 +196,7 @@ def _nccl_single(port, q):
         from combine_topk_ids_scan_b200 import binding as B
         from combine_topk_ids_scan_b200 import ep
         B.load()
-        p = _rank_problem(0, "packed")
+        p = _rank_problem(0, "packed", 1)
         N, H, E, k = p["N"], p["H"], p["E"], p["k"]
         prob = B.Problem(num_tokens=N, hidden=H, num_experts=E, top_k=k, num_segments=1,
                          recv_capacity=p["C"])
