@@ -127,6 +127,15 @@ __device__ void rank_tile(TileScanT<ROUNDS> &ts, const int32_t *__restrict__ ids
   const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
   uint16_t *wcnt = sm.wcnt;
   uint32_t *tile_prefix = sm.tile_prefix;
+  // the tile's ids first: their loads are in flight while shared memory is
+  // cleared
+  ts.base = (int64_t)ts.tile * (kScanThreads * ROUNDS) + (int64_t)warp * (kWarp * ROUNDS);
+  int32_t ex[ROUNDS];
+#pragma unroll
+  for (int r = 0; r < ROUNDS; ++r) {
+    const int64_t p = ts.base + r * kWarp + lane;
+    ex[r] = p < P ? __ldg(ids + p) : -1;
+  }
   {
     // the per-warp counts and lane masks start at zero: 16 * E * (2 + 4)
     // bytes, contiguous from the (16-byte aligned) start of shared memory,
@@ -139,13 +148,6 @@ __device__ void rank_tile(TileScanT<ROUNDS> &ts, const int32_t *__restrict__ ids
   __syncthreads();
 
   // ---- 1. per-warp stable ranks and histograms
-  ts.base = (int64_t)ts.tile * (kScanThreads * ROUNDS) + (int64_t)warp * (kWarp * ROUNDS);
-  int32_t ex[ROUNDS];
-#pragma unroll
-  for (int r = 0; r < ROUNDS; ++r) {
-    const int64_t p = ts.base + r * kWarp + lane;
-    ex[r] = p < P ? __ldg(ids + p) : -1;
-  }
   bool bad_id = false;
   uint16_t *my_cnt = wcnt + (size_t)warp * E;
   uint32_t *my_mask = sm.wmask + (size_t)warp * E;
