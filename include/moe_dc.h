@@ -22,7 +22,8 @@
  * moe_permute_backward and moe_combine_backward, moe_permute_premultiplied
  * (the dispatch with each pair's row scaled by its gate), moe_permute_to_peers
  * and its FP8 / NVFP4 forms (the dispatch written straight into the receive
- * buffers of the ranks that own the experts), and moe_dispatch_layout_noalloc (the layout without a
+ * buffers of the ranks that own the experts), moe_combine_from_peers (the
+ * combine reading the expert outputs where those ranks computed them), and moe_dispatch_layout_noalloc (the layout without a
  * caller workspace).  Two builds of the same sources add checks and records:
  * device index checks (moe_debug_violations) and per-CTA trace records
  * (moe_trace_attach).
