@@ -182,14 +182,18 @@ __device__ void rank_tile(TileScanT<ROUNDS> &ts, const int32_t *__restrict__ ids
   if (__any_sync(0xFFFFFFFFu, bad_id) && lane == 0) atomicOr(s_status, MOE_STATUS_ID_RANGE);
   __syncthreads();
 
-  // ---- 2. per expert: exclusive scan over the warps, tile aggregate
+  // ---- 2. per expert: exclusive scan over the warps, tile aggregate (the
+  // 16 counts are loaded before any base is stored, so the loads are in
+  // flight together instead of each waiting behind the previous store)
   for (int e = tid; e < E; e += kScanThreads) {
+    uint32_t c[kScanWarps];
+#pragma unroll
+    for (int w = 0; w < kScanWarps; ++w) c[w] = wcnt[w * E + e];
     uint32_t run = 0;
-#pragma unroll 4
+#pragma unroll
     for (int w = 0; w < kScanWarps; ++w) {
-      const uint32_t c = wcnt[w * E + e];
       wcnt[w * E + e] = (uint16_t)run;
-      run += c;
+      run += c[w];
     }
     tile_prefix[e] = run;
   }
