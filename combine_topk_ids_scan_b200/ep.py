@@ -201,6 +201,8 @@ def combine_exchange(expert_rows: torch.Tensor, route: Route, out: torch.Tensor 
                           dtype=expert_rows.dtype, device=expert_rows.device)
     if out.shape[0] < end or not out.is_contiguous():
         raise ValueError("out is not a contiguous buffer of the dispatch output's rows")
+    if out.dtype != expert_rows.dtype or out.shape[1:] != expert_rows.shape[1:]:
+        raise ValueError("out's rows differ from the expert rows in dtype or shape")
     # the reverse route: receive straight into the rows the segments left
     _grouped_exchange(_row_bytes(expert_rows), route.recv_rows, route.recv_offsets,
                       _row_bytes(out), route.send_rows, route.send_offsets, group)

@@ -117,6 +117,12 @@ def _worker(rank, world, port, mode, q):
                 raise AssertionError(f"{call.__name__}: wrong row count accepted")
             except ValueError:
                 pass
+        try:
+            ep.combine_exchange(torch.zeros((world, 4)), one_each,
+                                out=torch.zeros((world, 4), dtype=torch.float64))
+            raise AssertionError("combine_exchange: out of another dtype accepted")
+        except ValueError:
+            pass
         q.put((rank, "ok"))
     except Exception as e:  # report to the parent instead of hanging it
         q.put((rank, repr(e)))
