@@ -351,6 +351,18 @@ def measure_workload(B, torch, w, dev, stream, flush_l2, n_steps: int, peak: flo
         torch.cuda.synchronize(dev)
         graph_us = 1e3 * sum(a.elapsed_time(b) for a, b in ev) / n_steps
         del graph
+        # one trivial kernel (a 4-byte fill) between two events after the same
+        # flush: the launch and event cost that each of the phases above
+        # carries when it is timed alone between events
+        one = torch.zeros(1, dtype=torch.int32, device=dev)
+        torch.cuda.synchronize(dev)
+        for a, b in ev:
+            flush_l2()
+            a.record(stream)
+            one.fill_(1)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        floor_us = 1e3 * sum(a.elapsed_time(b) for a, b in ev) / n_steps
     status = int(buf.status.cpu().numpy().view(np.uint32)[0])
     total_rows = int(buf.expert_counts.sum().item())
     nbytes = algorithmic_bytes(w, total_rows)
@@ -378,6 +390,7 @@ def measure_workload(B, torch, w, dev, stream, flush_l2, n_steps: int, peak: flo
     if graph_us is not None:
         out["graph_step_us"] = round(graph_us, 2)
         out["graph_step_tokens_per_s"] = w.N / (graph_us * 1e-6)
+        out["trivial_kernel_between_events_us"] = round(floor_us, 2)
     del buf, d_ids, d_hidden, d_gates, d_x, d_gs, d_y
     return out
 
